@@ -1,0 +1,364 @@
+"""Pins for the CPU oracle: each routine checked against something other than itself.
+
+Routing  -- brute force over all k-subsets; all-equal logits; k = E; +0/-0 and NaN order;
+            softmax weights against torch's float64 softmax (library special case).
+Map      -- the block diagram of the MegaBlocks walkthrough (section 3, golden fixture);
+            invariants of sections 2 and 5 (padding <= 127, one expert per 128-row block,
+            sum of counts = T*k); numpy's stable argsort (library) for the sorted order; the
+            padded-row index math of section 4.2 restated element by element.
+Forward  -- closed form with permutation/selection weights (catches transposed operands and
+            wrong indices); zero inputs; exact scaling; E = 1, k = 1 against torch float64
+            (textbook gated MLP); invariance under relabelling experts.
+Backward -- central finite differences of the oracle's own forward (in double) for x, W1,
+            W3, W2 and the routing weights; dw = <dy, y_ts>; linearity in dy; the sampled
+            routines against the full backward.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------------------------------
+# routing
+# ----------------------------------------------------------------------------------------
+
+def _beats(a, ia, b, ib):
+    """Total order used for selection: larger value first, NaN lowest, then lower index."""
+    if math.isnan(a) and math.isnan(b):
+        return ia < ib
+    if math.isnan(a):
+        return False
+    if math.isnan(b):
+        return True
+    if a != b:
+        return a > b
+    return ia < ib
+
+
+def test_route_brute_force_subsets(oracle_mod):
+    rng = np.random.default_rng(7)
+    vals = np.array([-1.5, -0.0, 0.0, 0.25, 0.25, 1.0, 2.0, -np.inf], dtype=np.float32)
+    for E in (1, 2, 3, 5, 8):
+        for k in range(1, E + 1):
+            logits = rng.choice(vals, size=(64, E)).astype(np.float32)
+            top, _ = oracle_mod.route(logits, k)
+            for t in range(64):
+                l = [float(v) for v in logits[t]]
+                dominant = []
+                for S in itertools.combinations(range(E), k):
+                    rest = [e for e in range(E) if e not in S]
+                    if all(_beats(l[a], a, l[b], b) for a in S for b in rest):
+                        dominant.append(set(S))
+                assert len(dominant) == 1
+                assert set(top[t].tolist()) == dominant[0]
+                for s in range(k - 1):  # slot order follows the same total order
+                    a, b = top[t, s], top[t, s + 1]
+                    assert _beats(l[a], a, l[b], b)
+
+
+def test_route_all_equal_logits(oracle_mod):
+    for E, k in ((8, 2), (64, 8), (256, 8), (4, 4)):
+        logits = np.full((5, E), 0.375, np.float32)
+        top, w = oracle_mod.route(logits, k)
+        assert (top == np.arange(k)[None, :]).all()
+        assert (w.astype(np.float32) == np.float32(1.0 / E)).all()
+
+
+def test_route_k_equals_E_descending(oracle_mod):
+    rng = np.random.default_rng(3)
+    logits = rng.standard_normal((32, 6)).astype(np.float32)
+    top, _ = oracle_mod.route(logits, 6)
+    # library special case: a stable descending argsort (no ties in continuous draws)
+    ref = np.argsort(-logits, axis=1, kind="stable")
+    assert (top == ref).all()
+
+
+def test_route_signed_zero_and_nan(oracle_mod):
+    top, _ = oracle_mod.route(np.array([[-0.0, 0.0, -1.0]], np.float32), 1)
+    assert top[0, 0] == 0  # -0 == +0: the lower index wins
+    top, _ = oracle_mod.route(np.array([[0.0, -0.0, -1.0]], np.float32), 2)
+    assert top[0].tolist() == [0, 1]
+    top, _ = oracle_mod.route(np.array([[np.nan, -np.inf, -3.0]], np.float32), 3)
+    assert top[0].tolist() == [2, 1, 0]  # NaN ranks below -inf
+
+
+def test_route_weights_match_library_softmax(oracle_mod):
+    rng = np.random.default_rng(11)
+    for E, k in ((8, 2), (64, 8), (256, 8)):
+        logits = torch.randn(128, E, generator=torch.Generator().manual_seed(E)).to(torch.bfloat16).float()
+        top, w = oracle_mod.route(logits.numpy(), k)
+        sm = torch.softmax(logits.double(), dim=1).numpy()
+        ref = np.take_along_axis(sm, top.astype(np.int64), axis=1)
+        np.testing.assert_allclose(w, ref, rtol=1e-13, atol=0)
+        assert (w.sum(1) <= 1 + 1e-12).all()  # no renormalisation over the chosen k
+
+
+# ----------------------------------------------------------------------------------------
+# sparse map
+# ----------------------------------------------------------------------------------------
+
+def test_map_block_diagram_golden(oracle_mod):
+    g = json.load(open(os.path.join(GOLDEN, "block_diagram.json")))
+    E = g["E"]
+    top = np.concatenate([np.full(c, e, np.int32) for e, c in enumerate(g["counts"])])
+    np.random.default_rng(0).shuffle(top)
+    m = oracle_mod.sparse_map(top[:, None], E)
+    assert m["tokens_per_expert"].tolist() == g["counts"]
+    assert m["bins"].tolist() == g["expected_bins"]
+    assert m["padded_bins"].tolist() == g["expected_padded_bins"]
+    assert np.diff([0] + m["padded_bins"].tolist()).tolist() == g["expected_padded_tokens_per_expert"]
+    assert m["num_blocks"] == g["expected_num_blocks"]
+    nb = m["num_blocks"]
+    assert m["block_expert"][:nb].tolist() == g["expected_block_expert"]
+    assert (m["block_expert"][nb:] == -1).all()
+    cb = g["ffn"] // 128
+    cols = [[int(e) * cb + c for c in range(cb)] for e in m["block_expert"][:nb]]
+    assert cols == g["expected_column_blocks"]
+
+
+def _check_map_invariants(top, E, m):
+    T, k = top.shape
+    N = T * k
+    c = m["tokens_per_expert"].astype(np.int64)
+    assert c.sum() == N
+    assert (c == np.bincount(top.ravel(), minlength=E)).all()
+    padded = np.diff(np.concatenate([[0], m["padded_bins"].astype(np.int64)]))
+    assert (padded % 128 == 0).all()
+    assert ((padded - c >= 0) & (padded - c <= 127)).all()
+    assert (m["bins"] == np.cumsum(c)).all()
+    # stable sort: numpy's stable argsort is the library special case
+    assert (m["indices"] == np.argsort(top.ravel(), kind="stable")).all()
+    assert (m["bin_ids"] == top.ravel()[m["indices"]]).all()
+    assert (np.diff(m["bin_ids"]) >= 0).all()
+    # the index math of section 4.2, element by element
+    bins_ex = np.concatenate([[0], m["bins"][:-1]])
+    pb_ex = np.concatenate([[0], m["padded_bins"][:-1]])
+    i = np.arange(N)
+    e = m["bin_ids"]
+    dest = np.empty(N, np.int64)
+    dest[m["indices"]] = (i - bins_ex[e]) + pb_ex[e]
+    assert (m["dest_row"] == dest).all()
+    P = int(m["padded_bins"][-1])
+    assert len(set(m["dest_row"].tolist())) == N and m["dest_row"].min() >= 0 and m["dest_row"].max() < P
+    # every 128-row block belongs to exactly one expert (section 2)
+    nb = m["num_blocks"]
+    assert nb * 128 == P
+    owner = np.full(P, -1)
+    owner[m["dest_row"]] = top.ravel()
+    for b in range(nb):
+        rows = owner[b * 128:(b + 1) * 128]
+        real = rows[rows >= 0]
+        assert len(real) > 0 and (real == m["block_expert"][b]).all()
+    assert (m["block_expert"][nb:] == -1).all()
+
+
+@pytest.mark.parametrize("T,E,k,seed", [(256, 8, 2, 0), (1000, 64, 8, 1), (37, 300, 3, 2),
+                                         (300, 1, 1, 3), (129, 5, 5, 4), (5000, 256, 8, 5)])
+def test_map_invariants_random(oracle_mod, T, E, k, seed):
+    rng = np.random.default_rng(seed)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    top, _ = oracle_mod.route(logits, k)
+    m = oracle_mod.sparse_map(top, E)
+    _check_map_invariants(top, E, m)
+
+
+def test_map_skewed_and_empty_experts(oracle_mod):
+    T, E, k = 700, 16, 2
+    top = np.zeros((T, k), np.int32)
+    top[:, 1] = 1 + (np.arange(T) % 3)  # experts 4..15 are empty, expert 0 holds every token
+    m = oracle_mod.sparse_map(top, E)
+    _check_map_invariants(top, E, m)
+    assert (m["tokens_per_expert"][4:] == 0).all()
+
+
+def test_map_rejects_bad_expert(oracle_mod):
+    with pytest.raises(ValueError):
+        oracle_mod.sparse_map(np.array([[0], [3]], np.int32), 3)
+
+
+# ----------------------------------------------------------------------------------------
+# forward
+# ----------------------------------------------------------------------------------------
+
+def _silu(z):
+    return z / (1.0 + np.exp(-z))
+
+
+def test_forward_closed_form_selection_weights(oracle_mod):
+    """Weights that select one input element per output: the FFN is then an elementwise
+    closed form, and any transposed operand or wrong index changes it."""
+    rng = np.random.default_rng(5)
+    T, h, f, E, k = 16, 128, 256, 3, 2
+    x = rng.standard_normal((T, h)).astype(np.float32)
+    W1 = np.zeros((E, f, h), np.float32)
+    W3 = np.zeros((E, f, h), np.float32)
+    W2 = np.zeros((E, h, f), np.float32)
+    p1 = rng.integers(0, h, (E, f))
+    p3 = rng.integers(0, h, (E, f))
+    p2 = rng.integers(0, f, (E, h))
+    al, be, ga = [np.float32(v) for v in (0.75, -1.25, 0.5)]
+    for e in range(E):
+        W1[e, np.arange(f), p1[e]] = al * (e + 1)
+        W3[e, np.arange(f), p3[e]] = be
+        W2[e, np.arange(h), p2[e]] = ga * (e + 2)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    top, w = oracle_mod.route(logits, k)
+    y = oracle_mod.forward(x, W1, W3, W2, top, w)
+    ref = np.zeros((T, h))
+    for t in range(T):
+        for s in range(k):
+            e = top[t, s]
+            xt = x[t].astype(np.float64)
+            hh = _silu(float(al) * (e + 1) * xt[p1[e]]) * (float(be) * xt[p3[e]])
+            ref[t] += w[t, s] * float(ga) * (e + 2) * hh[p2[e]]
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-14)
+
+
+def _rand_layer(rng, T, h, f, E, k, scale=0.05):
+    x = rng.standard_normal((T, h)).astype(np.float32)
+    W1 = (scale * rng.standard_normal((E, f, h))).astype(np.float32)
+    W3 = (scale * rng.standard_normal((E, f, h))).astype(np.float32)
+    W2 = (scale * rng.standard_normal((E, h, f))).astype(np.float32)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    return x, W1, W3, W2, logits
+
+
+def test_forward_zero_and_scaling(oracle_mod):
+    rng = np.random.default_rng(9)
+    x, W1, W3, W2, logits = _rand_layer(rng, 12, 128, 128, 4, 2)
+    top, w = oracle_mod.route(logits, 2)
+    assert (oracle_mod.forward(np.zeros_like(x), W1, W3, W2, top, w) == 0).all()
+    assert (oracle_mod.forward(x, W1, W3, np.zeros_like(W2), top, w) == 0).all()
+    assert (oracle_mod.forward(x, W1, np.zeros_like(W3), W2, top, w) == 0).all()
+    y = oracle_mod.forward(x, W1, W3, W2, top, w)
+    y2 = oracle_mod.forward(x, W1, W3, 2 * W2, top, w)
+    assert (y2 == 2 * y).all()  # scaling W2 by 2 is exact in binary floating point
+
+
+def test_forward_single_expert_is_textbook_gated_mlp(oracle_mod):
+    rng = np.random.default_rng(13)
+    x, W1, W3, W2, logits = _rand_layer(rng, 20, 128, 256, 1, 1)
+    top, w = oracle_mod.route(logits, 1)
+    assert (top == 0).all() and (w == 1.0).all()
+    y = oracle_mod.forward(x, W1, W3, W2, top, w)
+    X = torch.from_numpy(x).double()
+    ref = (torch.nn.functional.silu(X @ torch.from_numpy(W1[0]).double().T)
+           * (X @ torch.from_numpy(W3[0]).double().T)) @ torch.from_numpy(W2[0]).double().T
+    np.testing.assert_allclose(y, ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_forward_expert_relabelling_invariance(oracle_mod):
+    rng = np.random.default_rng(17)
+    x, W1, W3, W2, logits = _rand_layer(rng, 24, 128, 128, 6, 3)
+    top, w = oracle_mod.route(logits, 3)
+    y = oracle_mod.forward(x, W1, W3, W2, top, w)
+    perm = rng.permutation(6)  # new expert id of old expert e is perm[e]
+    inv = np.argsort(perm)
+    top2, w2 = oracle_mod.route(logits[:, inv], 3)
+    assert (top2 == perm[top]).all()
+    y2 = oracle_mod.forward(x, W1[inv], W3[inv], W2[inv], top2, w2)
+    np.testing.assert_allclose(y2, y, rtol=1e-12, atol=1e-13)
+
+
+def test_forward_token_subset_matches_full(oracle_mod):
+    rng = np.random.default_rng(19)
+    x, W1, W3, W2, logits = _rand_layer(rng, 30, 128, 128, 4, 2)
+    top, w = oracle_mod.route(logits, 2)
+    y, yts = oracle_mod.forward(x, W1, W3, W2, top, w, want_yts=True, threads=2)
+    toks = np.array([29, 0, 7], np.int32)
+    ys = oracle_mod.forward(x, W1, W3, W2, top, w, tokens=toks)
+    assert (ys == y[toks]).all()
+    np.testing.assert_allclose((w[:, :, None] * yts).sum(1), y, rtol=1e-12, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------------------
+# backward
+# ----------------------------------------------------------------------------------------
+
+def _loss(oracle_mod, x, W1, W3, W2, top, w, dy):
+    return float((oracle_mod.forward(x, W1, W3, W2, top, w) * dy).sum())
+
+
+def _fd_check(oracle_mod, name, args, grad, idxs, top, w, dy, step):
+    x, W1, W3, W2 = args
+    for ix in idxs:
+        plus = [a.copy() for a in args]
+        minus = [a.copy() for a in args]
+        i = ["x", "W1", "W3", "W2"].index(name)
+        plus[i][ix] += np.float32(step)
+        minus[i][ix] -= np.float32(step)
+        delta = float(plus[i][ix]) - float(minus[i][ix])
+        fd = (_loss(oracle_mod, *plus, top, w, dy) - _loss(oracle_mod, *minus, top, w, dy)) / delta
+        assert abs(fd - grad[ix]) <= 2e-6 + 2e-5 * abs(grad[ix]), (name, ix, fd, grad[ix])
+
+
+def test_backward_finite_differences(oracle_mod):
+    rng = np.random.default_rng(23)
+    T, h, f, E, k = 8, 128, 128, 4, 2
+    x, W1, W3, W2, logits = _rand_layer(rng, T, h, f, E, k, scale=0.1)
+    dy = rng.standard_normal((T, h)).astype(np.float32)
+    top, w = oracle_mod.route(logits, k)
+    g = oracle_mod.backward(x, dy, W1, W3, W2, top, w)
+    args = (x, W1, W3, W2)
+    pick = lambda shape, n: [tuple(rng.integers(0, s) for s in shape) for _ in range(n)]
+    used = sorted(set(top.ravel().tolist()))
+    for name, grad, shape in (("x", g["dx"], x.shape), ("W1", g["dW1"], W1.shape),
+                              ("W3", g["dW3"], W3.shape), ("W2", g["dW2"], W2.shape)):
+        idxs = pick(shape, 12)
+        if name != "x":  # make sure most probes land on experts that receive tokens
+            idxs = [(used[i % len(used)],) + ix[1:] for i, ix in enumerate(idxs)]
+        _fd_check(oracle_mod, name, args, grad, idxs, top, w, dy, step=2.0 ** -7)
+    # routing-weight gradient: perturb w directly
+    for (t, s) in [(0, 0), (3, 1), (7, 0)]:
+        wp, wm = w.copy(), w.copy()
+        wp[t, s] += 1e-3
+        wm[t, s] -= 1e-3
+        fd = (_loss(oracle_mod, *args, top, wp, dy) - _loss(oracle_mod, *args, top, wm, dy)) / 2e-3
+        assert abs(fd - g["dw"][t, s]) <= 1e-8 + 1e-8 * abs(fd)
+    # unrouted experts get exactly zero gradient
+    for e in range(E):
+        if e not in used:
+            assert (g["dW1"][e] == 0).all() and (g["dW2"][e] == 0).all()
+
+
+def test_backward_dw_identity_and_linearity(oracle_mod):
+    rng = np.random.default_rng(29)
+    T, h, f, E, k = 10, 128, 128, 4, 2
+    x, W1, W3, W2, logits = _rand_layer(rng, T, h, f, E, k)
+    top, w = oracle_mod.route(logits, k)
+    dy = rng.standard_normal((T, h)).astype(np.float32)
+    g = oracle_mod.backward(x, dy, W1, W3, W2, top, w)
+    _, yts = oracle_mod.forward(x, W1, W3, W2, top, w, want_yts=True)
+    np.testing.assert_allclose(g["dw"], np.einsum("th,tsh->ts", dy.astype(np.float64), yts),
+                               rtol=1e-12, atol=1e-13)
+    g2 = oracle_mod.backward(x, 2 * dy, W1, W3, W2, top, w)
+    assert (g2["dx"] == 2 * g["dx"]).all() and (g2["dW1"] == 2 * g["dW1"]).all()
+
+
+def test_backward_sampled_routines_match_full(oracle_mod):
+    rng = np.random.default_rng(31)
+    T, h, f, E, k = 12, 128, 256, 4, 2
+    x, W1, W3, W2, logits = _rand_layer(rng, T, h, f, E, k)
+    top, w = oracle_mod.route(logits, k)
+    dy = rng.standard_normal((T, h)).astype(np.float32)
+    g = oracle_mod.backward(x, dy, W1, W3, W2, top, w)
+    toks = np.array([11, 2, 5], np.int32)
+    dx, dw = oracle_mod.backward_tokens(x, dy, W1, W3, W2, top, w, toks, threads=2)
+    np.testing.assert_allclose(dx, g["dx"][toks], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(dw, g["dw"][toks], rtol=1e-12, atol=1e-14)
+    q = []
+    for e in range(E):
+        q += [(1, e, rng.integers(f), rng.integers(h)), (3, e, rng.integers(f), rng.integers(h)),
+              (2, e, rng.integers(h), rng.integers(f))]
+    q = np.array(q, np.int32)
+    vals = oracle_mod.wgrad_elements(x, dy, W1, W3, W2, top, w, q, threads=2)
+    full = {1: g["dW1"], 3: g["dW3"], 2: g["dW2"]}
+    ref = np.array([full[a][b, c, d] for a, b, c, d in q])
+    np.testing.assert_allclose(vals, ref, rtol=1e-11, atol=1e-14)
