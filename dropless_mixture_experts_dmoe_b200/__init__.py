@@ -1,0 +1,10 @@
+"""dMoE expert layer for NVIDIA B200 (sm_100a): routing, sparse map, padded gather, grouped
+tcgen05 gated-SiLU expert GEMMs, weighted combine and backward, behind the C ABI of
+``libdmoe.so`` (include/dmoe.h).  ``binding`` is the thin ctypes layer over it."""
+from . import binding  # noqa: F401
+from .binding import (Buffers, DMoEError, SparseMap, dmoe_backward, dmoe_expert_down,  # noqa: F401
+                      dmoe_expert_glu, dmoe_forward, dmoe_padded_gather, dmoe_padded_rows_max,
+                      dmoe_padded_scatter, dmoe_saved_bytes, dmoe_sparse_map, dmoe_workspace_bytes,
+                      make_dims)
+
+__version__ = "0.1"

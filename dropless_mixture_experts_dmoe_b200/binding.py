@@ -1,0 +1,271 @@
+"""Thin ctypes binding of libdmoe.so (declared in include/dmoe.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA kernels.
+PyTorch is used for device memory and streams.  There is no fallback: if the library is
+missing or the device is not a B200 the calls raise.
+
+The functions carry the C names (``dmoe_sparse_map``, ``dmoe_forward``, ``dmoe_backward`` and
+the step entry points) and take torch tensors where the C call takes device pointers.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from .build import LIB
+
+BLOCKING = 128
+MAX_EXPERTS = 1024
+MAX_TOP_K = 32
+
+WS_MAP, WS_FORWARD, WS_BACKWARD = 0, 1, 2
+
+STATUS_NONFINITE_LOGITS = 0x1
+STATUS_EXPERT_OUT_OF_RANGE = 0x2
+STATUS_DUPLICATE_EXPERT = 0x4
+STATUS_TIMEOUT = 0x8
+
+_P = ctypes.c_void_p
+_SZ = ctypes.c_size_t
+_I = ctypes.c_int
+
+
+class dmoe_dims(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("hidden", ctypes.c_int32), ("ffn", ctypes.c_int32),
+                ("num_experts", ctypes.c_int32), ("top_k", ctypes.c_int32)]
+
+    def __repr__(self):
+        return (f"dmoe_dims(T={self.T}, hidden={self.hidden}, ffn={self.ffn}, "
+                f"num_experts={self.num_experts}, top_k={self.top_k})")
+
+
+MAP_FIELDS = ("top_experts", "weights", "tokens_per_expert", "bins", "padded_bins", "indices",
+              "bin_ids", "dest_row", "block_expert", "num_blocks", "status")
+
+
+class dmoe_map(ctypes.Structure):
+    _fields_ = [(n, _P) for n in MAP_FIELDS]
+
+
+class DMoEError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {error_string(code)} ({code})")
+        self.code = code
+
+
+_lib = None
+
+
+def load():
+    """Load the in-tree libdmoe.so (build it first with ``build.build()``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB):
+        raise ImportError(f"libdmoe.so not built: {LIB} is missing "
+                          "(run python -m dropless_mixture_experts_dmoe_b200.build)")
+    lib = ctypes.CDLL(LIB)
+    D = ctypes.POINTER(dmoe_dims)
+    M = ctypes.POINTER(dmoe_map)
+    lib.dmoe_padded_rows_max.argtypes = [D]
+    lib.dmoe_padded_rows_max.restype = _SZ
+    lib.dmoe_workspace_bytes.argtypes = [D, _I]
+    lib.dmoe_workspace_bytes.restype = _SZ
+    lib.dmoe_saved_bytes.argtypes = [D, ctypes.POINTER(_SZ)]
+    lib.dmoe_saved_bytes.restype = _SZ
+    lib.dmoe_sparse_map.argtypes = [D, _P, M, _P, _SZ, _P]
+    lib.dmoe_forward.argtypes = [D, _P, _P, _P, _P, M, _P, _P, _P, _SZ, _P]
+    lib.dmoe_backward.argtypes = [D, _P, _P, _P, _P, M, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+    lib.dmoe_padded_gather.argtypes = [D, _P, M, _P, _P]
+    lib.dmoe_expert_glu.argtypes = [D, _P, _P, _P, M, _P, _P, _P, _P]
+    lib.dmoe_expert_down.argtypes = [D, _P, _P, M, _P, _P]
+    lib.dmoe_padded_scatter.argtypes = [D, _P, M, _P, _P, _P]
+    for fn in ("dmoe_sparse_map", "dmoe_forward", "dmoe_backward", "dmoe_padded_gather",
+               "dmoe_expert_glu", "dmoe_expert_down", "dmoe_padded_scatter"):
+        getattr(lib, fn).restype = _I
+    lib.dmoe_error_string.argtypes = [_I]
+    lib.dmoe_error_string.restype = ctypes.c_char_p
+    lib.dmoe_status_string.argtypes = [ctypes.c_int32]
+    lib.dmoe_status_string.restype = ctypes.c_char_p
+    lib.dmoe_version.argtypes = []
+    lib.dmoe_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def error_string(code: int) -> str:
+    return load().dmoe_error_string(code).decode()
+
+
+def status_string(status: int) -> str:
+    return load().dmoe_status_string(int(status)).decode()
+
+
+def version() -> str:
+    return load().dmoe_version().decode()
+
+
+def make_dims(T: int, hidden: int, ffn: int, num_experts: int, top_k: int) -> dmoe_dims:
+    return dmoe_dims(T, hidden, ffn, num_experts, top_k)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise DMoEError(rc, what)
+
+
+# ---- sizes ------------------------------------------------------------------------------------
+
+def dmoe_padded_rows_max(dims: dmoe_dims) -> int:
+    return int(load().dmoe_padded_rows_max(ctypes.byref(dims)))
+
+
+def dmoe_workspace_bytes(dims: dmoe_dims, kind: int) -> int:
+    return int(load().dmoe_workspace_bytes(ctypes.byref(dims), kind))
+
+
+def dmoe_saved_bytes(dims: dmoe_dims):
+    offs = (_SZ * 5)()
+    total = int(load().dmoe_saved_bytes(ctypes.byref(dims), offs))
+    return total, [int(o) for o in offs]
+
+
+# ---- the sparse map -----------------------------------------------------------------------------
+
+class SparseMap:
+    """Device tensors of the sparse map (torch allocations) and their C view."""
+
+    def __init__(self, dims: dmoe_dims, device="cuda"):
+        T, E, k = dims.T, dims.num_experts, dims.top_k
+        P = dmoe_padded_rows_max(dims)
+        if P == 0:
+            raise DMoEError(-2, "SparseMap")
+        i32 = dict(dtype=torch.int32, device=device)
+        self.dims = dims
+        self.top_experts = torch.empty((T, k), **i32)
+        self.weights = torch.empty((T, k), dtype=torch.float32, device=device)
+        self.tokens_per_expert = torch.empty(E, **i32)
+        self.bins = torch.empty(E, **i32)
+        self.padded_bins = torch.empty(E, **i32)
+        self.indices = torch.empty(T * k, **i32)
+        self.bin_ids = torch.empty(T * k, **i32)
+        self.dest_row = torch.empty(T * k, **i32)
+        self.block_expert = torch.empty(max(P // BLOCKING, 1), **i32)
+        self.num_blocks = torch.empty(1, **i32)
+        self.status = torch.zeros(1, **i32)
+        self._c = dmoe_map(*[getattr(self, n).data_ptr() for n in MAP_FIELDS])
+
+    @property
+    def c(self) -> dmoe_map:
+        return self._c
+
+    def as_dict(self) -> dict:
+        return {n: getattr(self, n) for n in MAP_FIELDS}
+
+
+def dmoe_sparse_map(dims: dmoe_dims, logits, smap: SparseMap, ws, stream=None):
+    """Routing + sparse map.  logits: [T,E] bf16 CUDA tensor or None (top_experts given)."""
+    ws_bytes = ws.numel() * ws.element_size()
+    rc = load().dmoe_sparse_map(ctypes.byref(dims), _ptr(logits), ctypes.byref(smap.c), _ptr(ws),
+                                ws_bytes, _stream(stream))
+    _check(rc, "dmoe_sparse_map")
+
+
+def dmoe_forward(dims: dmoe_dims, x, w1, w3, w2, smap: SparseMap, y, saved=None, ws=None,
+                 stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    rc = load().dmoe_forward(ctypes.byref(dims), _ptr(x), _ptr(w1), _ptr(w3), _ptr(w2),
+                             ctypes.byref(smap.c), _ptr(y), _ptr(saved), _ptr(ws), ws_bytes,
+                             _stream(stream))
+    _check(rc, "dmoe_forward")
+
+
+def dmoe_backward(dims: dmoe_dims, dy, w1, w3, w2, smap: SparseMap, saved, dx, dw1, dw3, dw2,
+                  dweights, ws, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    rc = load().dmoe_backward(ctypes.byref(dims), _ptr(dy), _ptr(w1), _ptr(w3), _ptr(w2),
+                              ctypes.byref(smap.c), _ptr(saved), _ptr(dx), _ptr(dw1), _ptr(dw3),
+                              _ptr(dw2), _ptr(dweights), _ptr(ws), ws_bytes, _stream(stream))
+    _check(rc, "dmoe_backward")
+
+
+def dmoe_padded_gather(dims, x, smap: SparseMap, x_pad, stream=None):
+    _check(load().dmoe_padded_gather(ctypes.byref(dims), _ptr(x), ctypes.byref(smap.c), _ptr(x_pad),
+                                     _stream(stream)), "dmoe_padded_gather")
+
+
+def dmoe_expert_glu(dims, x_pad, w1, w3, smap: SparseMap, h_out, a_out=None, b_out=None,
+                    stream=None):
+    _check(load().dmoe_expert_glu(ctypes.byref(dims), _ptr(x_pad), _ptr(w1), _ptr(w3),
+                                  ctypes.byref(smap.c), _ptr(h_out), _ptr(a_out), _ptr(b_out),
+                                  _stream(stream)), "dmoe_expert_glu")
+
+
+def dmoe_expert_down(dims, h_in, w2, smap: SparseMap, y_pad, stream=None):
+    _check(load().dmoe_expert_down(ctypes.byref(dims), _ptr(h_in), _ptr(w2), ctypes.byref(smap.c),
+                                   _ptr(y_pad), _stream(stream)), "dmoe_expert_down")
+
+
+def dmoe_padded_scatter(dims, y_pad, smap: SparseMap, weights, y, stream=None):
+    _check(load().dmoe_padded_scatter(ctypes.byref(dims), _ptr(y_pad), ctypes.byref(smap.c),
+                                      _ptr(weights), _ptr(y), _stream(stream)),
+           "dmoe_padded_scatter")
+
+
+# ---- buffers (allocation only) ----------------------------------------------------------------
+
+class Buffers:
+    """Caller-side device allocations for one layer shape: map, workspaces, saved activations.
+
+    train=True: ``saved`` (X_pad, A, Bm, H, Y_pad for the backward) and the backward
+    workspace; ``view(name)`` gives bf16 views of the saved activations.
+    train=False: the inference workspace of ``dmoe_forward`` plus separate X_pad / H / Y_pad
+    tensors (``step``) for driving the step entry points one by one."""
+
+    def __init__(self, dims: dmoe_dims, train: bool = False, device="cuda"):
+        self.dims = dims
+        self.P = dmoe_padded_rows_max(dims)
+        self.map = SparseMap(dims, device)
+        u8 = dict(dtype=torch.uint8, device=device)
+        self.ws_map = torch.empty(max(dmoe_workspace_bytes(dims, WS_MAP), 16), **u8)
+        self.train = train
+        P, h, f = self.P, dims.hidden, dims.ffn
+        self.saved = self.ws_fwd = self.ws_bwd = None
+        self.step = {}
+        if train:
+            total, offs = dmoe_saved_bytes(dims)
+            self.saved = torch.empty(total, **u8)
+            self.offsets = dict(x_pad=offs[0], a=offs[1], bm=offs[2], h=offs[3], y_pad=offs[4])
+            self.ws_bwd = torch.empty(max(dmoe_workspace_bytes(dims, WS_BACKWARD), 16), **u8)
+        else:
+            self.ws_fwd = torch.empty(dmoe_workspace_bytes(dims, WS_FORWARD), **u8)
+            bf = dict(dtype=torch.bfloat16, device=device)
+            self.step = dict(x_pad=torch.empty((P, h), **bf), h=torch.empty((P, f), **bf),
+                             y_pad=torch.empty((P, h), **bf))
+
+    def view(self, name: str) -> torch.Tensor:
+        """bf16 [P, cols] view of a saved activation (train=True only)."""
+        if not self.train:
+            return self.step[name]
+        off = self.offsets[name]
+        cols = self.dims.hidden if name in ("x_pad", "y_pad") else self.dims.ffn
+        n = self.P * cols * 2
+        return self.saved[off:off + n].view(torch.bfloat16).view(self.P, cols)

@@ -1,0 +1,299 @@
+// api.cu -- the C ABI of libdmoe.so (declared in include/dmoe.h): argument checks, workspace
+// layout and the launch sequence of each entry point.  Every check runs on the host before
+// the first launch of a call; nothing here reads device memory or synchronises.
+#include <stdio.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace dmoe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape validation shared by all entry points.
+int check_dims(const dmoe_dims *d) {
+  if (!d) return DMOE_ERR_NULL;
+  if (d->num_experts < 1 || d->num_experts > DMOE_MAX_EXPERTS) return DMOE_ERR_TOO_MANY_EXPERTS;
+  if (d->T < 1 || d->top_k < 1 || d->top_k > d->num_experts || d->top_k > DMOE_MAX_TOP_K)
+    return DMOE_ERR_SHAPE;
+  if (d->ffn < DMOE_BLOCKING || d->ffn % DMOE_BLOCKING != 0) return DMOE_ERR_SHAPE;
+  if (d->hidden < DMOE_BLOCKING || d->hidden % DMOE_BLOCKING != 0) return DMOE_ERR_SHAPE;
+  const long long n = (long long)d->T * d->top_k;
+  const long long pmax =
+      (n + (long long)(DMOE_BLOCKING - 1) * d->num_experts) / DMOE_BLOCKING * DMOE_BLOCKING;
+  if (n > 0x7FFFFFFFLL || pmax > 0x7FFFFFFFLL) return DMOE_ERR_TOO_LARGE;
+  return DMOE_OK;
+}
+
+long long pmax_of(const dmoe_dims *d) {
+  const long long n = (long long)d->T * d->top_k;
+  return (n + (long long)(DMOE_BLOCKING - 1) * d->num_experts) / DMOE_BLOCKING * DMOE_BLOCKING;
+}
+
+int check_device() {
+  static int cached = -1;
+  if (cached < 0) {
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+      return DMOE_ERR_DEVICE;
+    cached = (major == 10) ? 1 : 0;
+  }
+  return cached == 1 ? DMOE_OK : DMOE_ERR_DEVICE;
+}
+
+int check_map(const dmoe_map *m, bool need_weights) {
+  if (!m || !m->top_experts || !m->tokens_per_expert || !m->bins || !m->padded_bins ||
+      !m->indices || !m->bin_ids || !m->dest_row || !m->block_expert || !m->num_blocks ||
+      !m->status)
+    return DMOE_ERR_NULL;
+  if (need_weights && !m->weights) return DMOE_ERR_NULL;
+  return DMOE_OK;
+}
+
+inline int launch_rc(cudaError_t e) { return e == cudaSuccess ? DMOE_OK : DMOE_ERR_LAUNCH; }
+
+// Forward workspace layout (inference): X_pad [P,h] | H [P,f] | Y_pad [P,h]
+struct FwdLayout {
+  size_t xpad, h, ypad, total;
+};
+FwdLayout fwd_layout(const dmoe_dims *d) {
+  const size_t P = (size_t)pmax_of(d);
+  FwdLayout l;
+  l.xpad = 0;
+  l.h = align_up(l.xpad + P * d->hidden * 2);
+  l.ypad = align_up(l.h + P * d->ffn * 2);
+  l.total = align_up(l.ypad + P * d->hidden * 2);
+  return l;
+}
+
+// Saved activations: X_pad [P,h] | A [P,f] | Bm [P,f] | H [P,f] | Y_pad [P,h]
+void saved_layout(const dmoe_dims *d, size_t off[5], size_t *total) {
+  const size_t P = (size_t)pmax_of(d);
+  off[0] = 0;
+  off[1] = align_up(off[0] + P * d->hidden * 2);
+  off[2] = align_up(off[1] + P * d->ffn * 2);
+  off[3] = align_up(off[2] + P * d->ffn * 2);
+  off[4] = align_up(off[3] + P * d->ffn * 2);
+  *total = align_up(off[4] + P * d->hidden * 2);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dmoe_padded_rows_max(const dmoe_dims *dims) {
+  if (check_dims(dims) != DMOE_OK) return 0;
+  return (size_t)pmax_of(dims);
+}
+
+size_t dmoe_workspace_bytes(const dmoe_dims *dims, int kind) {
+  if (check_dims(dims) != DMOE_OK) return 0;
+  switch (kind) {
+    case DMOE_WS_MAP:
+      return align_up(sizeof(int32_t) * (size_t)map_tiles(dims->T) * dims->num_experts);
+    case DMOE_WS_FORWARD:
+      return fwd_layout(dims).total;
+    case DMOE_WS_BACKWARD:
+      return 0;
+    default:
+      return 0;
+  }
+}
+
+size_t dmoe_saved_bytes(const dmoe_dims *dims, size_t offsets[5]) {
+  if (check_dims(dims) != DMOE_OK) return 0;
+  size_t off[5], total;
+  saved_layout(dims, off, &total);
+  if (offsets)
+    for (int i = 0; i < 5; ++i) offsets[i] = off[i];
+  return total;
+}
+
+int dmoe_sparse_map(const dmoe_dims *dims, const void *logits, const dmoe_map *map, void *ws,
+                    size_t ws_bytes, void *stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_map(map, logits != nullptr))) return rc;
+  if (!ws) return DMOE_ERR_NULL;
+  if (ws_bytes < dmoe_workspace_bytes(dims, DMOE_WS_MAP)) return DMOE_ERR_WORKSPACE;
+  if ((logits && !aligned16(logits)) || !aligned16(ws) || !aligned16(map->top_experts) ||
+      (logits && !aligned16(map->weights)))
+    return DMOE_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int T = dims->T, E = dims->num_experts, k = dims->top_k;
+  const int nblk_cap = (int)(pmax_of(dims) / DMOE_BLOCKING);
+  int32_t *tile_hist = static_cast<int32_t *>(ws);
+  if (cudaMemsetAsync(map->status, 0, sizeof(int32_t), st) != cudaSuccess) return DMOE_ERR_LAUNCH;
+  if ((rc = launch_rc(launch_route_hist(static_cast<const uint16_t *>(logits), T, E, k,
+                                        map->top_experts, map->weights, tile_hist, map->status,
+                                        st))))
+    return rc;
+  if ((rc = launch_rc(launch_map_scan(T, E, nblk_cap, tile_hist, map->tokens_per_expert,
+                                      map->bins, map->padded_bins, map->block_expert,
+                                      map->num_blocks, st))))
+    return rc;
+  return launch_rc(launch_map_scatter(T, E, k, map->top_experts, tile_hist, map->bins,
+                                      map->padded_bins, map->indices, map->bin_ids,
+                                      map->dest_row, st));
+}
+
+int dmoe_padded_gather(const dmoe_dims *dims, const void *x, const dmoe_map *map, void *x_pad,
+                       void *stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_map(map, false))) return rc;
+  if (!x || !x_pad) return DMOE_ERR_NULL;
+  if (!aligned16(x) || !aligned16(x_pad)) return DMOE_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return launch_rc(launch_gather(dims->T, dims->hidden, dims->top_k, dims->num_experts, x,
+                                 map->dest_row, map->tokens_per_expert, map->padded_bins, x_pad,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+int dmoe_expert_glu(const dmoe_dims *dims, const void *x_pad, const void *w1, const void *w3,
+                    const dmoe_map *map, void *h_out, void *a_out, void *b_out, void *stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_map(map, false))) return rc;
+  if (!x_pad || !w1 || !w3 || !h_out) return DMOE_ERR_NULL;
+  if (!aligned16(x_pad) || !aligned16(w1) || !aligned16(w3) || !aligned16(h_out) ||
+      (a_out && !aligned16(a_out)) || (b_out && !aligned16(b_out)))
+    return DMOE_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  const int nblk_cap = (int)(pmax_of(dims) / DMOE_BLOCKING);
+  return launch_rc(launch_glu_gemm(dims->hidden, dims->ffn, dims->num_experts, nblk_cap, x_pad, w1,
+                                   w3, map->num_blocks, map->block_expert, h_out, a_out, b_out,
+                                   map->status, static_cast<cudaStream_t>(stream)));
+}
+
+int dmoe_expert_down(const dmoe_dims *dims, const void *h_in, const void *w2,
+                     const dmoe_map *map, void *y_pad, void *stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_map(map, false))) return rc;
+  if (!h_in || !w2 || !y_pad) return DMOE_ERR_NULL;
+  if (!aligned16(h_in) || !aligned16(w2) || !aligned16(y_pad)) return DMOE_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  const int nblk_cap = (int)(pmax_of(dims) / DMOE_BLOCKING);
+  return launch_rc(launch_down_gemm(dims->hidden, dims->ffn, dims->num_experts, nblk_cap, h_in, w2,
+                                    map->num_blocks, map->block_expert, y_pad, map->status,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+int dmoe_padded_scatter(const dmoe_dims *dims, const void *y_pad, const dmoe_map *map,
+                        const float *weights, void *y, void *stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_map(map, false))) return rc;
+  if (!y_pad || !y) return DMOE_ERR_NULL;
+  if (!aligned16(y_pad) || !aligned16(y)) return DMOE_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return launch_rc(launch_combine(dims->T, dims->hidden, dims->top_k, y_pad, map->dest_row,
+                                  weights, y, static_cast<cudaStream_t>(stream)));
+}
+
+int dmoe_forward(const dmoe_dims *dims, const void *x, const void *w1, const void *w3,
+                 const void *w2, const dmoe_map *map, void *y, void *saved, void *ws,
+                 size_t ws_bytes, void *stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_map(map, true))) return rc;
+  if (!x || !w1 || !w3 || !w2 || !y) return DMOE_ERR_NULL;
+  uint8_t *xpad, *hbuf, *ypad, *abuf = nullptr, *bbuf = nullptr;
+  if (saved) {
+    size_t off[5], total;
+    saved_layout(dims, off, &total);
+    uint8_t *s = static_cast<uint8_t *>(saved);
+    xpad = s + off[0];
+    abuf = s + off[1];
+    bbuf = s + off[2];
+    hbuf = s + off[3];
+    ypad = s + off[4];
+  } else {
+    if (!ws) return DMOE_ERR_NULL;
+    FwdLayout l = fwd_layout(dims);
+    if (ws_bytes < l.total) return DMOE_ERR_WORKSPACE;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    xpad = w + l.xpad;
+    hbuf = w + l.h;
+    ypad = w + l.ypad;
+  }
+  if (!aligned16(x) || !aligned16(w1) || !aligned16(w3) || !aligned16(w2) || !aligned16(y) ||
+      !aligned16(xpad) || !aligned16(map->weights))
+    return DMOE_ERR_ALIGN;
+  if ((rc = dmoe_padded_gather(dims, x, map, xpad, stream))) return rc;
+  if ((rc = dmoe_expert_glu(dims, xpad, w1, w3, map, hbuf, abuf, bbuf, stream))) return rc;
+  if ((rc = dmoe_expert_down(dims, hbuf, w2, map, ypad, stream))) return rc;
+  return dmoe_padded_scatter(dims, ypad, map, map->weights, y, stream);
+}
+
+int dmoe_backward(const dmoe_dims *dims, const void *dy, const void *w1, const void *w3,
+                  const void *w2, const dmoe_map *map, const void *saved, void *dx, void *dw1,
+                  void *dw3, void *dw2, float *dweights, void *ws, size_t ws_bytes,
+                  void *stream) {
+  (void)dims;
+  (void)dy;
+  (void)w1;
+  (void)w3;
+  (void)w2;
+  (void)map;
+  (void)saved;
+  (void)dx;
+  (void)dw1;
+  (void)dw3;
+  (void)dw2;
+  (void)dweights;
+  (void)ws;
+  (void)ws_bytes;
+  (void)stream;
+  return DMOE_ERR_SHAPE;
+}
+
+const char *dmoe_error_string(int code) {
+  switch (code) {
+    case DMOE_OK:
+      return "ok";
+    case DMOE_ERR_NULL:
+      return "a required pointer is NULL";
+    case DMOE_ERR_SHAPE:
+      return "invalid shape (ffn and hidden must be multiples of 128; 1 <= top_k <= min(E, 32); T >= 1)";
+    case DMOE_ERR_TOO_MANY_EXPERTS:
+      return "number of experts outside [1, 1024]";
+    case DMOE_ERR_WORKSPACE:
+      return "workspace too small";
+    case DMOE_ERR_ALIGN:
+      return "a pointer is not 16-byte aligned";
+    case DMOE_ERR_LAUNCH:
+      return "a CUDA launch failed";
+    case DMOE_ERR_DEVICE:
+      return "current device is not sm_100 (B200)";
+    case DMOE_ERR_TOO_LARGE:
+      return "T*top_k or the padded row bound exceeds 2^31-1";
+    default:
+      return "unknown error";
+  }
+}
+
+const char *dmoe_status_string(int32_t status) {
+  static thread_local char buf[160];
+  buf[0] = 0;
+  if (status == 0) return "ok";
+  if (status & DMOE_STATUS_NONFINITE_LOGITS) strcat(buf, "nonfinite_logits ");
+  if (status & DMOE_STATUS_EXPERT_OUT_OF_RANGE) strcat(buf, "expert_out_of_range ");
+  if (status & DMOE_STATUS_DUPLICATE_EXPERT) strcat(buf, "duplicate_expert ");
+  if (status & DMOE_STATUS_TIMEOUT) strcat(buf, "timeout ");
+  return buf;
+}
+
+const char *dmoe_version(void) { return "dmoe-b200 0.1"; }
+
+}  // extern "C"

@@ -1,0 +1,48 @@
+// kernels.h -- host-side launchers of the dMoE kernels (internal to libdmoe.so).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dmoe {
+
+// Tokens per map tile: one CTA of the routing/histogram kernel and of the stable-scatter
+// kernel handles this many tokens (kMapTokTile * top_k entries).
+constexpr int kMapTokTile = 64;
+
+inline int map_tiles(int T) { return (T + kMapTokTile - 1) / kMapTokTile; }
+
+// Map: routing + per-tile histogram (logits given) or histogram of given top_experts.
+cudaError_t launch_route_hist(const uint16_t *logits, int T, int E, int k, int32_t *top,
+                              float *weights, int32_t *tile_hist, int32_t *status,
+                              cudaStream_t st);
+// Map: scan over tiles and experts, bins / padded_bins / block table.
+cudaError_t launch_map_scan(int T, int E, int nblk_cap, int32_t *tile_hist,
+                            int32_t *tokens_per_expert, int32_t *bins, int32_t *padded_bins,
+                            int32_t *block_expert, int32_t *num_blocks, cudaStream_t st);
+// Map: stable scatter of entries to sorted order; indices, bin_ids, dest_row.
+cudaError_t launch_map_scatter(int T, int E, int k, const int32_t *top, const int32_t *tile_off,
+                               const int32_t *bins, const int32_t *padded_bins, int32_t *indices,
+                               int32_t *bin_ids, int32_t *dest_row, cudaStream_t st);
+
+// Token-major padded gather with zero-filled padding rows.
+cudaError_t launch_gather(int T, int h, int k, int E, const void *x, const int32_t *dest_row,
+                          const int32_t *counts, const int32_t *padded_bins, void *x_pad,
+                          cudaStream_t st);
+// Token-major weighted combine (weights may be NULL: w = 1).
+cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const int32_t *dest_row,
+                           const float *weights, void *y, cudaStream_t st);
+
+// Grouped tcgen05 GEMMs over the non-empty row blocks.
+cudaError_t launch_glu_gemm(int h, int f, int E, int nblk_cap, const void *x_pad,
+                            const void *w1, const void *w3, const int32_t *num_blocks,
+                            const int32_t *block_expert, void *h_out, void *a_out, void *b_out,
+                            int32_t *status, cudaStream_t st);
+cudaError_t launch_down_gemm(int h, int f, int E, int nblk_cap, const void *h_in,
+                             const void *w2, const int32_t *num_blocks,
+                             const int32_t *block_expert, void *y_pad, int32_t *status,
+                             cudaStream_t st);
+
+int device_sm_count();
+
+}  // namespace dmoe

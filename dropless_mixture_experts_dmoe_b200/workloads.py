@@ -3,9 +3,9 @@
 This module holds only the shapes and the seeded random inputs; it contains none of the
 layer's arithmetic, so both the CUDA path and the CPU oracle can take their inputs from it.
 
-Recipe (one torch CPU generator per workload, seed = 1000 + workload number, draws in the
-order x, W1, W3, W2, logits, dy; every tensor drawn in fp32 and rounded to bf16 with
-round-to-nearest-even):
+Recipe: workload seed s = 1000 + workload number; every tensor has its own torch CPU
+generator seeded with 100*s + i (i = 0 x, 1 W1, 2 W3, 3 W2, 4 logits, 5 dy), so any tensor
+can be regenerated alone; each is drawn in fp32 and rounded to bf16 (round-to-nearest-even):
   x ~ N(0, 1)                         [T, hidden]
   W1, W3 ~ 0.02 * N(0, 1)             [E, ffn, hidden]   (out, in) layout; W1 = gate
   W2 ~ 0.02 * N(0, 1)                 [E, hidden, ffn]
@@ -71,27 +71,32 @@ def zipf_bias(E: int) -> torch.Tensor:
     return torch.tensor([-1.5 * math.log(e + 1) for e in range(E)], dtype=torch.float32)
 
 
+TENSORS = ("x", "w1", "w3", "w2", "logits", "dy")
+
+
+def make_tensor(w: Workload, name: str, seed: int | None = None) -> torch.Tensor:
+    """One CPU bf16 input tensor of workload ``w`` (see the module recipe)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(100 * (w.seed if seed is None else seed) + TENSORS.index(name))
+    shape, scale = {
+        "x": ((w.T, w.hidden), 1.0),
+        "w1": ((w.E, w.ffn, w.hidden), 0.02),
+        "w3": ((w.E, w.ffn, w.hidden), 0.02),
+        "w2": ((w.E, w.hidden, w.ffn), 0.02),
+        "logits": ((w.T, w.E), 1.0),
+        "dy": ((w.T, w.hidden), 1.0),
+    }[name]
+    t = torch.randn(shape, generator=g, dtype=torch.float32)
+    if scale != 1.0:
+        t.mul_(scale)
+    if name == "logits" and w.zipf_bias:
+        t += zipf_bias(w.E)[None, :]
+    return t.to(torch.bfloat16)
+
+
 def make_inputs(w: Workload, seed: int | None = None, with_dy: bool | None = None) -> dict:
     """CPU bf16 tensors x, w1, w3, w2, logits (and dy) for workload ``w``."""
-    g = torch.Generator(device="cpu")
-    g.manual_seed(w.seed if seed is None else seed)
-
-    def draw(shape, scale=1.0):
-        t = torch.randn(shape, generator=g, dtype=torch.float32)
-        if scale != 1.0:
-            t.mul_(scale)
-        return t.to(torch.bfloat16)
-
-    out = {
-        "x": draw((w.T, w.hidden)),
-        "w1": draw((w.E, w.ffn, w.hidden), 0.02),
-        "w3": draw((w.E, w.ffn, w.hidden), 0.02),
-        "w2": draw((w.E, w.hidden, w.ffn), 0.02),
-    }
-    lg = torch.randn((w.T, w.E), generator=g, dtype=torch.float32)
-    if w.zipf_bias:
-        lg += zipf_bias(w.E)[None, :]
-    out["logits"] = lg.to(torch.bfloat16)
+    names = list(TENSORS[:5])
     if w.backward if with_dy is None else with_dy:
-        out["dy"] = draw((w.T, w.hidden))
-    return out
+        names.append("dy")
+    return {n: make_tensor(w, n, seed) for n in names}

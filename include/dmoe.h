@@ -1,0 +1,216 @@
+/*
+ * dmoe.h -- C ABI of libdmoe.so, the dropless mixture-of-experts (dMoE) expert layer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (MegaBlocks walkthrough "02 · dropless MoE 与 block-sparse 重构", sections 2-4;
+ * Fast-LLM issue #56 "[feat] Support sparse copy for a large number of experts", error log):
+ *   1. route each token to its top-k experts (top-k of the softmax over E logits);
+ *   2. build the sparse map: per-expert histogram, stable sort of (token, slot) entries by
+ *      expert, bins, padded_bins rounded up to 128 rows so that every 128-row block belongs
+ *      to exactly one expert (walkthrough section 2, section 4.1);
+ *   3. padded_gather: copy each token row to its padded row (section 4.2);
+ *   4. gated-SiLU expert FFN on the non-empty 128-row blocks only:
+ *        H = silu(X_pad W1_e^T) * (X_pad W3_e^T),  Y_pad = H W2_e^T
+ *      (block-sparse view of sections 2-3; gated SiLU of the issue's config);
+ *   5. padded_scatter: y_t = sum_s w_ts * Y_pad[dest_row[t*k+s]] (section 4.2);
+ *   6. backward: gather and scatter swap roles, plus the routing-weight gradient
+ *      (section 4.2); the activation is recomputed from the saved pre-activations
+ *      (section 4.4).
+ *
+ * Conventions (all entry points)
+ *   - The caller owns and allocates ALL device memory, including workspaces; the library
+ *     never allocates, frees or synchronises.  Query sizes with dmoe_workspace_bytes and
+ *     dmoe_saved_bytes.
+ *   - Every launch is asynchronous on `stream` (a cudaStream_t, passed as void*; NULL is
+ *     the legacy default stream).  No call reads device memory on the host, so the whole
+ *     layer can run without a host synchronisation.
+ *   - Every call returns an int: DMOE_OK (0) or a negative DMOE_ERR_* detected on the host
+ *     BEFORE any launch (nothing is launched then), or DMOE_ERR_LAUNCH if a launch failed.
+ *   - Conditions only the device can see set bits in the caller's int32 status word
+ *     (dmoe_map.status); read it after synchronising and decode with dmoe_status_string.
+ *     No kernel traps; every wait in a kernel is bounded and sets DMOE_STATUS_TIMEOUT when
+ *     it gives up.
+ *   - All device pointers must be 16-byte aligned.
+ *   - bf16 = IEEE bfloat16 stored as uint16; all matrices row-major, C-contiguous.
+ *   - Weights use the (out, in) layout: W1, W3 are [E, ffn, hidden] (W1 = gate, W3 = up),
+ *     W2 is [E, hidden, ffn].
+ *   - Entries are flattened j = t*k + s (token t, slot s); this is the flattening implied by
+ *     the gather rule "source row = index_a // TOP_K" (walkthrough section 4.2).
+ *   - Blocking is fixed at 128 rows ("self.blocking = 128", walkthrough section 2).
+ *   - Requires an sm_100 device (B200); other devices get DMOE_ERR_DEVICE.
+ */
+#ifndef DMOE_H
+#define DMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Symbols exported from libdmoe.so (the library is built with hidden default visibility). */
+#if defined(__GNUC__)
+#define DMOE_API __attribute__((visibility("default")))
+#else
+#define DMOE_API
+#endif
+
+#define DMOE_BLOCKING 128
+#define DMOE_MAX_EXPERTS 1024
+#define DMOE_MAX_TOP_K 32
+
+/* Error codes (returned). */
+#define DMOE_OK 0
+#define DMOE_ERR_NULL (-1)             /* a required pointer is NULL */
+#define DMOE_ERR_SHAPE (-2)            /* ffn % 128 != 0 (walkthrough section 5: the topology
+                                          rejects it), hidden % 128 != 0, T < 1, top_k < 1,
+                                          top_k > E, top_k > DMOE_MAX_TOP_K */
+#define DMOE_ERR_TOO_MANY_EXPERTS (-3) /* E < 1 or E > DMOE_MAX_EXPERTS: a documented limit,
+                                          never an opaque resource failure (the issue's
+                                          OutOfResources at E = 64) */
+#define DMOE_ERR_WORKSPACE (-4)        /* workspace smaller than dmoe_workspace_bytes */
+#define DMOE_ERR_ALIGN (-5)            /* a pointer is not 16-byte aligned */
+#define DMOE_ERR_LAUNCH (-6)           /* a CUDA launch or runtime call failed */
+#define DMOE_ERR_DEVICE (-7)           /* current device is not sm_100 */
+#define DMOE_ERR_TOO_LARGE (-8)        /* T*top_k or the padded row bound exceeds 2^31-1 */
+
+/* Device status bits (OR-ed into dmoe_map.status by the kernels). */
+#define DMOE_STATUS_NONFINITE_LOGITS 0x1   /* a NaN or +-inf logit was routed on */
+#define DMOE_STATUS_EXPERT_OUT_OF_RANGE 0x2 /* caller-given top_experts outside [0, E) */
+#define DMOE_STATUS_DUPLICATE_EXPERT 0x4   /* caller-given top_experts repeat within a token */
+#define DMOE_STATUS_TIMEOUT 0x8            /* a bounded in-kernel wait gave up */
+
+/* Problem shape.  T tokens, hidden size h, ffn size f (per expert), E experts, top_k. */
+typedef struct {
+  int32_t T, hidden, ffn, num_experts, top_k;
+} dmoe_dims;
+
+/* The sparse map.  All device pointers, caller-owned; N = T*top_k entries,
+ * P_max = dmoe_padded_rows_max(dims).  Meaning (walkthrough sections 4.1-4.3):
+ *   top_experts [T, k] int32   expert of entry t*k+s, slot s = s-th pick in descending
+ *                              logit order, ties to the lower expert index.  Output of
+ *                              dmoe_sparse_map when logits are given, else its INPUT.
+ *   weights     [T, k] fp32    softmax over all E logits at the chosen expert (no
+ *                              renormalisation over the k picks).  Output when logits are
+ *                              given; otherwise caller-provided and only read by forward.
+ *   tokens_per_expert [E]      histogram of top_experts
+ *   bins [E]                   inclusive cumsum of tokens_per_expert
+ *   padded_bins [E]            inclusive cumsum of round_up(tokens_per_expert, 128)
+ *   indices [N]                entries stably sorted by expert: flattened entry index
+ *   bin_ids [N]                expert of the i-th sorted entry
+ *   dest_row [N]               padded row of entry j: (i - bins[e-1]) + padded_bins[e-1],
+ *                              i its sorted position, e its expert, bins[-1] = 0
+ *   block_expert [P_max/128]   expert owning 128-row block b; -1 for b >= num_blocks
+ *   num_blocks [1]             padded_bins[E-1] / 128
+ *   status [1]                 device status bits; dmoe_sparse_map clears it first          */
+typedef struct {
+  int32_t *top_experts;
+  float *weights;
+  int32_t *tokens_per_expert;
+  int32_t *bins;
+  int32_t *padded_bins;
+  int32_t *indices;
+  int32_t *bin_ids;
+  int32_t *dest_row;
+  int32_t *block_expert;
+  int32_t *num_blocks;
+  int32_t *status;
+} dmoe_map;
+
+/* Workspace kinds for dmoe_workspace_bytes. */
+#define DMOE_WS_MAP 0      /* dmoe_sparse_map */
+#define DMOE_WS_FORWARD 1  /* dmoe_forward with saved == NULL (inference) */
+#define DMOE_WS_BACKWARD 2 /* dmoe_backward */
+
+/* Static bound on the padded row count: floor((T*k + 127*E)/128)*128.  Every padded
+ * buffer is sized from it, so no call needs the data-dependent size on the host (the
+ * walkthrough's padded_gather reads padded_bins[-1] on the host, section 4.2; this library
+ * does not). Returns 0 for invalid dims. */
+DMOE_API size_t dmoe_padded_rows_max(const dmoe_dims *dims);
+
+/* Bytes of workspace the call `kind` needs (0 for invalid dims). */
+DMOE_API size_t dmoe_workspace_bytes(const dmoe_dims *dims, int kind);
+
+/* Bytes of the activations dmoe_forward saves for dmoe_backward, and their byte offsets
+ * inside that buffer: offsets[0] X_pad [P_max,h], [1] A = X_pad W1^T [P_max,f],
+ * [2] Bm = X_pad W3^T [P_max,f], [3] H = silu(A)*Bm [P_max,f], [4] Y_pad [P_max,h], all bf16.
+ * offsets may be NULL.  Returns 0 for invalid dims. */
+DMOE_API size_t dmoe_saved_bytes(const dmoe_dims *dims, size_t offsets[5]);
+
+/* Routing + sparse map (walkthrough section 4.1; the Fast-LLM get_sparse_map step).
+ *   logits: [T, E] bf16 device pointer, or NULL to take map->top_experts as given (then
+ *           map->weights is not written; out-of-range or duplicate experts set status bits
+ *           and such entries are dropped from the map).
+ *   map:    caller-owned outputs (see dmoe_map); map->status is cleared, then OR-ed.
+ *   ws:     workspace of dmoe_workspace_bytes(dims, DMOE_WS_MAP) bytes.
+ * Shared memory per CTA is O(E) and independent of T (the issue's kernel needed 262144 B
+ * at E = 64, top-8, 2 x 2048 tokens).  Three kernels, no atomics on global memory, no
+ * host sync; results are deterministic. */
+DMOE_API int dmoe_sparse_map(const dmoe_dims *dims, const void *logits, const dmoe_map *map, void *ws,
+                    size_t ws_bytes, void *stream);
+
+/* Forward of the expert layer (walkthrough section 4.5 schematic, gated SiLU).
+ *   x [T,h], w1 [E,f,h], w3 [E,f,h], w2 [E,h,f]: bf16 inputs.  map: from dmoe_sparse_map.
+ *   y [T,h] bf16 output.
+ *   saved: NULL for inference, else a buffer of dmoe_saved_bytes(dims) bytes that receives
+ *          X_pad, A, Bm, H, Y_pad for dmoe_backward (then ws may be NULL / 0 bytes).
+ *   ws: dmoe_workspace_bytes(dims, DMOE_WS_FORWARD) bytes when saved == NULL.
+ * Runs padded_gather, the GLU GEMM, the down GEMM and the weighted padded_scatter. */
+DMOE_API int dmoe_forward(const dmoe_dims *dims, const void *x, const void *w1, const void *w3,
+                 const void *w2, const dmoe_map *map, void *y, void *saved, void *ws,
+                 size_t ws_bytes, void *stream);
+
+/* Backward (walkthrough section 4.2: the gradient of padded_scatter is padded_gather plus a
+ * routing-weight gradient, the gradient of padded_gather is padded_scatter; section 4.4:
+ * the activation is recomputed from the saved pre-activations).
+ *   dy [T,h] bf16; w1, w3, w2 as in dmoe_forward; map from dmoe_sparse_map; saved from
+ *   dmoe_forward(saved != NULL).
+ *   Outputs: dx [T,h] bf16; dw1, dw3 [E,f,h] bf16; dw2 [E,h,f] bf16 (experts that receive
+ *   no token get exact zeros); dweights [T,k] fp32 = <dy_t, Y_ts>.
+ *   ws: dmoe_workspace_bytes(dims, DMOE_WS_BACKWARD) bytes. */
+DMOE_API int dmoe_backward(const dmoe_dims *dims, const void *dy, const void *w1, const void *w3,
+                  const void *w2, const dmoe_map *map, const void *saved, void *dx, void *dw1,
+                  void *dw3, void *dw2, float *dweights, void *ws, size_t ws_bytes,
+                  void *stream);
+
+/* ---- Step entry points (each one kernel; dmoe_forward is exactly this sequence). ---- */
+
+/* padded_gather (walkthrough section 4.2, A_TO_B direction): x_pad[dest_row[t*k+s]] = x[t]
+ * for every slot s; the padding rows of every expert's last block are written as zeros
+ * (section 5: padding rows hold zeros).  x [T,h] bf16 -> x_pad [P_max,h] bf16; rows at or
+ * beyond num_blocks*128 are not touched. */
+DMOE_API int dmoe_padded_gather(const dmoe_dims *dims, const void *x, const dmoe_map *map, void *x_pad,
+                       void *stream);
+
+/* GLU GEMM over the non-empty row blocks: for every block b < num_blocks with expert
+ * e = block_expert[b], A = X_pad[b] W1_e^T, Bm = X_pad[b] W3_e^T (fp32 accumulation in
+ * tensor memory) and H[b] = bf16(silu(A) * Bm).  a_out / b_out (may be NULL) receive
+ * bf16(A), bf16(Bm).  x_pad [P_max,h] -> h_out, a_out, b_out [P_max,f], all bf16. */
+DMOE_API int dmoe_expert_glu(const dmoe_dims *dims, const void *x_pad, const void *w1, const void *w3,
+                    const dmoe_map *map, void *h_out, void *a_out, void *b_out, void *stream);
+
+/* Down GEMM: Y_pad[b] = bf16(H[b] W2_e^T) for every block b < num_blocks.
+ * h_in [P_max,f] -> y_pad [P_max,h], bf16. */
+DMOE_API int dmoe_expert_down(const dmoe_dims *dims, const void *h_in, const void *w2,
+                     const dmoe_map *map, void *y_pad, void *stream);
+
+/* Weighted padded_scatter (walkthrough section 4.2, B_TO_A direction, times the routing
+ * weight): y_t = bf16(sum_{s=0..k-1} w_ts * Y_pad[dest_row[t*k+s]]), summed in fp32 in
+ * slot order, no atomics.  weights == NULL means w = 1 (the backward's gather gradient,
+ * dx_t = sum_s dX_pad[dest_row[t*k+s]]).  y_pad [P_max,h] -> y [T,h], bf16. */
+DMOE_API int dmoe_padded_scatter(const dmoe_dims *dims, const void *y_pad, const dmoe_map *map,
+                        const float *weights, void *y, void *stream);
+
+/* ---- Diagnostics. ---- */
+DMOE_API const char *dmoe_error_string(int code);
+/* Human-readable list of the bits set in a host copy of the status word. */
+DMOE_API const char *dmoe_status_string(int32_t status);
+/* Library version, e.g. "dmoe-b200 0.1". */
+DMOE_API const char *dmoe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DMOE_H */

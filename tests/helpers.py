@@ -1,0 +1,107 @@
+"""Shared test helpers: run the CUDA path through the C ABI, run the oracle, compare.
+
+The CUDA side goes through ``dropless_mixture_experts_dmoe_b200.binding`` only; the oracle
+side through ``oracle`` only.  Inputs for both come from ``workloads`` (seeded, bf16)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from dropless_mixture_experts_dmoe_b200 import binding as B
+from dropless_mixture_experts_dmoe_b200.workloads import Workload
+
+# Float tolerance of the layer's outputs and gradients against the fp32-input oracle
+# (relative L2 error and max-abs error relative to the reference RMS).
+REL_L2 = 1e-2
+MAX_ABS_RMS = 5e-2
+# fp32 routing weights (fp32 expf/sum on the GPU, double in the oracle).
+WEIGHT_RTOL = 2e-6
+
+
+def metrics(got, ref):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    diff = got - ref
+    rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
+    rel = float(np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-300))
+    mx = float(np.max(np.abs(diff))) if ref.size else 0.0
+    return rel, mx, rms
+
+
+def assert_close(got, ref, what=""):
+    rel, mx, rms = metrics(got, ref)
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    assert rel <= REL_L2, f"{what}: relative L2 {rel:.3e} > {REL_L2}"
+    assert mx <= MAX_ABS_RMS * rms, f"{what}: max abs {mx:.3e} > {MAX_ABS_RMS} * RMS {rms:.3e}"
+    return rel, mx, rms
+
+
+def dims_of(w: Workload):
+    return B.make_dims(w.T, w.hidden, w.ffn, w.E, w.top_k)
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    if t.dtype == torch.bfloat16:
+        t = t.float()
+    return t.detach().cpu().numpy()
+
+
+def gpu_map(dims, logits=None, top_experts=None, bufs=None):
+    """Run dmoe_sparse_map; returns (Buffers, dict of numpy arrays)."""
+    if bufs is None:
+        bufs = B.Buffers(dims, train=True)
+    if top_experts is not None:
+        bufs.map.top_experts.copy_(torch.as_tensor(top_experts, dtype=torch.int32))
+    lg = None if logits is None else logits.cuda()
+    B.dmoe_sparse_map(dims, lg, bufs.map, bufs.ws_map)
+    torch.cuda.synchronize()
+    out = {k: to_np(v) for k, v in bufs.map.as_dict().items()}
+    out["num_blocks"] = int(out["num_blocks"][0])
+    out["status"] = int(out["status"][0])
+    return bufs, out
+
+
+def compare_map(g: dict, o: dict, top_expected=None):
+    """Bit-exact comparison of every integer map array."""
+    if top_expected is not None:
+        np.testing.assert_array_equal(g["top_experts"], top_expected)
+    for k in ("tokens_per_expert", "bins", "padded_bins", "indices", "bin_ids", "dest_row"):
+        np.testing.assert_array_equal(g[k], o[k], err_msg=k)
+    assert g["num_blocks"] == o["num_blocks"]
+    np.testing.assert_array_equal(g["block_expert"], o["block_expert"], err_msg="block_expert")
+
+
+def oracle_inputs(inp: dict) -> dict:
+    """fp32 numpy copies (exact widening of the bf16 inputs) for the oracle."""
+    return {k: v.float().numpy() for k, v in inp.items()}
+
+
+def gpu_forward(dims, inp: dict, train=True):
+    """Full layer forward through the C ABI: map (from logits) + dmoe_forward."""
+    bufs = B.Buffers(dims, train=train)
+    dev = {k: v.cuda() for k, v in inp.items()}
+    B.dmoe_sparse_map(dims, dev["logits"], bufs.map, bufs.ws_map)
+    y = torch.empty((dims.T, dims.hidden), dtype=torch.bfloat16, device="cuda")
+    B.dmoe_forward(dims, dev["x"], dev["w1"], dev["w3"], dev["w2"], bufs.map, y,
+                   saved=bufs.saved, ws=bufs.ws_fwd)
+    torch.cuda.synchronize()
+    return bufs, dev, y
+
+
+def sample_tokens(top: np.ndarray, E: int, n: int, seed: int = 0) -> np.ndarray:
+    """A token sample that touches as many experts as possible plus random tokens,
+    including the last token (ragged tail)."""
+    rng = np.random.default_rng(seed)
+    T = top.shape[0]
+    picks = {T - 1, 0}
+    seen = set()
+    for t in rng.permutation(T):
+        if len(picks) >= n:
+            break
+        if not set(top[t].tolist()) <= seen:
+            picks.add(int(t))
+            seen |= set(top[t].tolist())
+    while len(picks) < min(n, T):
+        picks.add(int(rng.integers(T)))
+    return np.array(sorted(picks), np.int32)

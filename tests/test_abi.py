@@ -1,0 +1,84 @@
+"""C-ABI checks that need no GPU: the library builds/loads, exports every symbol the header
+declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from dropless_mixture_experts_dmoe_b200 import binding as B
+from dropless_mixture_experts_dmoe_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.load()
+
+
+def _declared_symbols():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"DMOE_API\s+[\w\s\*]+?\b(dmoe_\w+)\s*\(", txt)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_symbols()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(lib, n), n
+    assert B.version().startswith("dmoe-b200")
+
+
+def test_sizes():
+    d = B.make_dims(4096, 4096, 14336, 8, 2)
+    P = B.dmoe_padded_rows_max(d)
+    assert P == ((4096 * 2 + 127 * 8) // 128) * 128
+    assert B.dmoe_workspace_bytes(d, B.WS_MAP) >= 4 * 64 * 8
+    assert B.dmoe_workspace_bytes(d, B.WS_FORWARD) >= P * (2 * 4096 + 14336) * 2
+    total, offs = B.dmoe_saved_bytes(d)
+    assert offs == sorted(offs) and offs[0] == 0 and all(o % 256 == 0 for o in offs)
+    assert total >= offs[4] + P * 4096 * 2
+
+
+@pytest.mark.parametrize("dims,code", [
+    ((256, 128, 100, 8, 2), -2),    # ffn % 128 != 0 (the walkthrough's topology guard)
+    ((256, 96, 128, 8, 2), -2),     # hidden % 128 != 0
+    ((256, 128, 128, 8, 9), -2),    # top_k > E
+    ((256, 128, 128, 64, 33), -2),  # top_k > 32
+    ((0, 128, 128, 8, 2), -2),      # T < 1
+    ((256, 128, 128, 1025, 2), -3),  # E > 1024
+    ((256, 128, 128, 0, 1), -3),
+    ((2 ** 28, 128, 128, 32, 16), -8),  # T*k overflows int32
+])
+def test_bad_dims_rejected_before_launch(lib, dims, code):
+    d = B.make_dims(*dims)
+    assert B.dmoe_padded_rows_max(d) == 0
+    m = B.dmoe_map()
+    rc = lib.dmoe_sparse_map(ctypes.byref(d), None, ctypes.byref(m), None, 0, None)
+    assert rc == code
+    rc = lib.dmoe_forward(ctypes.byref(d), None, None, None, None, ctypes.byref(m), None, None, None,
+                          0, None)
+    assert rc == code
+    assert B.error_string(code) != "unknown error"
+
+
+def test_null_and_workspace_checks(lib):
+    d = B.make_dims(256, 128, 128, 8, 2)
+    m = B.dmoe_map()
+    assert lib.dmoe_sparse_map(ctypes.byref(d), None, ctypes.byref(m), None, 0, None) == -1
+    fake = 1 << 20  # host-side checks only: nothing is launched when a check fails
+    m = B.dmoe_map(*([fake] * len(B.MAP_FIELDS)))
+    assert lib.dmoe_sparse_map(ctypes.byref(d), fake, ctypes.byref(m), fake, 16, None) == -4
+    assert lib.dmoe_sparse_map(ctypes.byref(d), fake + 2, ctypes.byref(m), fake, 1 << 20, None) == -5
+
+
+def test_status_strings(lib):
+    assert B.status_string(0) == "ok"
+    s = B.status_string(B.STATUS_TIMEOUT | B.STATUS_NONFINITE_LOGITS)
+    assert "timeout" in s and "nonfinite" in s

@@ -1,0 +1,77 @@
+"""padded_gather / padded_scatter data-movement parity (bit-exact where the maths is exact)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dropless_mixture_experts_dmoe_b200 import binding as B
+from dropless_mixture_experts_dmoe_b200.workloads import WORKLOADS, custom, make_tensor
+
+from helpers import compare_map, gpu_map, to_np
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [
+    WORKLOADS[1],
+    WORKLOADS[3],
+    custom(1000, 384, 128, 5, 3),    # h/8 = 48 vectors per row: a ragged vector chunk
+    custom(777, 4096, 128, 16, 2),   # wide rows (two 256-vector chunks)
+    custom(64, 128, 128, 300, 8),    # most experts empty
+]
+
+
+def _setup(w):
+    dims = B.make_dims(w.T, w.hidden, w.ffn, w.E, w.top_k)
+    logits = make_tensor(w, "logits")
+    bufs, g = gpu_map(dims, logits)
+    top, _ = oracle.route(logits.float().numpy(), w.top_k)
+    compare_map(g, oracle.sparse_map(top, w.E), top_expected=top)
+    x = make_tensor(w, "x").cuda()
+    return dims, bufs, g, x
+
+
+@pytest.mark.parametrize("w", SHAPES, ids=lambda w: w.describe())
+def test_gather_bit_exact_and_zero_padding(w):
+    dims, bufs, g, x = _setup(w)
+    xp = bufs.view("x_pad")
+    xp.view(torch.int16).fill_(0x7F81)  # sentinel (a NaN pattern) to see untouched rows
+    B.dmoe_padded_gather(dims, x, bufs.map, xp)
+    torch.cuda.synchronize()
+    P = g["num_blocks"] * 128
+    xp16 = xp.view(torch.int16).cpu().numpy()
+    x16 = x.view(torch.int16).cpu().numpy()
+    t_of_j = np.arange(w.T * w.top_k) // w.top_k
+    np.testing.assert_array_equal(xp16[g["dest_row"]], x16[t_of_j])
+    real = np.zeros(P, bool)
+    real[g["dest_row"]] = True
+    assert (xp16[:P][~real] == 0).all(), "padding rows must be zero"
+    assert (xp16[P:] == 0x7F81).all(), "rows past the padded size must be untouched"
+
+
+@pytest.mark.parametrize("w", SHAPES, ids=lambda w: w.describe())
+def test_scatter_of_gather_is_k_times_x(w):
+    dims, bufs, g, x = _setup(w)
+    xp = bufs.view("x_pad")
+    B.dmoe_padded_gather(dims, x, bufs.map, xp)
+    y = torch.empty_like(x)
+    B.dmoe_padded_scatter(dims, xp, bufs.map, None, y)  # w = 1: the gather's gradient
+    torch.cuda.synchronize()
+    ref = (x.float() * w.top_k).to(torch.bfloat16)  # k*x is exact in fp32
+    assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
+
+
+@pytest.mark.parametrize("w", SHAPES[:3], ids=lambda w: w.describe())
+def test_weighted_scatter(w):
+    dims, bufs, g, x = _setup(w)
+    yp = bufs.view("y_pad")
+    yp.copy_(torch.randn(yp.shape, device="cuda").to(torch.bfloat16))
+    y = torch.empty_like(x)
+    B.dmoe_padded_scatter(dims, yp, bufs.map, bufs.map.weights, y)
+    torch.cuda.synchronize()
+    ypn = to_np(yp).astype(np.float64)
+    wts = g["weights"].astype(np.float64)
+    rows = g["dest_row"].reshape(w.T, w.top_k)
+    ref = np.einsum("ts,tsh->th", wts, ypn[rows])
+    got = to_np(y).astype(np.float64)
+    # one bf16 rounding of an fp32 sum: within 2^-8 relative, plus fp32 summation slack
+    assert (np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5).all()

@@ -1,0 +1,108 @@
+"""Sparse-map parity: routing and every map array bit-exact against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dropless_mixture_experts_dmoe_b200 import binding as B
+from dropless_mixture_experts_dmoe_b200.workloads import WORKLOADS, make_inputs, make_tensor
+
+from helpers import WEIGHT_RTOL, compare_map, gpu_map
+
+pytestmark = pytest.mark.gpu
+
+
+def _logits_only(w):
+    return make_tensor(w, "logits")
+
+
+@pytest.mark.parametrize("num", [1, 2, 3, 4, 5])
+def test_map_parity_workloads(num):
+    w = WORKLOADS[num]
+    logits = _logits_only(w)
+    dims = B.make_dims(w.T, w.hidden, w.ffn, w.E, w.top_k)
+    _, g = gpu_map(dims, logits)
+    top, wts = oracle.route(logits.float().numpy(), w.top_k)
+    o = oracle.sparse_map(top, w.E)
+    compare_map(g, o, top_expected=top)
+    np.testing.assert_allclose(g["weights"], wts, rtol=WEIGHT_RTOL, atol=0)
+    assert g["status"] == 0
+
+
+def test_map_parity_real_inputs_tiny():
+    w = WORKLOADS[1]
+    inp = make_inputs(w)
+    dims = B.make_dims(w.T, w.hidden, w.ffn, w.E, w.top_k)
+    _, g = gpu_map(dims, inp["logits"])
+    top, wts = oracle.route(inp["logits"].float().numpy(), w.top_k)
+    compare_map(g, oracle.sparse_map(top, w.E), top_expected=top)
+
+
+@pytest.mark.parametrize("T,E,k,kind", [
+    (300, 8, 2, "all_equal"),      # every row ties: experts 0..k-1
+    (257, 16, 4, "few_values"),    # many ties, +0 / -0 mixed
+    (130, 8, 8, "continuous"),     # k = E
+    (1000, 1, 1, "continuous"),    # E = 1
+    (999, 64, 1, "continuous"),    # k = 1
+    (2000, 1024, 8, "continuous"),  # maximum E
+    (4097, 32, 32, "few_values"),  # maximum k
+    (1, 8, 2, "continuous"),       # single token
+    (8192, 64, 8, "continuous"),   # the issue's failing shape with 4096-long sequences
+])
+def test_map_parity_edge_cases(T, E, k, kind):
+    g = torch.Generator().manual_seed(T * 7 + E)
+    if kind == "all_equal":
+        logits = torch.full((T, E), 0.5)
+    elif kind == "few_values":
+        vals = torch.tensor([-1.0, -0.0, 0.0, 0.5, 0.5, 2.0])
+        logits = vals[torch.randint(0, len(vals), (T, E), generator=g)]
+    else:
+        logits = torch.randn((T, E), generator=g)
+    logits = logits.to(torch.bfloat16)
+    dims = B.make_dims(T, 128, 128, E, k)
+    _, gm = gpu_map(dims, logits)
+    top, wts = oracle.route(logits.float().numpy(), k)
+    compare_map(gm, oracle.sparse_map(top, E), top_expected=top)
+    np.testing.assert_allclose(gm["weights"], wts, rtol=WEIGHT_RTOL, atol=0)
+
+
+def test_map_skew_and_empty_experts_given_top():
+    """Caller-given top_experts: one expert takes every token, most experts are empty."""
+    T, E, k = 5000, 256, 8
+    top = np.zeros((T, k), np.int32)
+    top[:, 1:] = (np.arange(T)[:, None] * 7 + np.arange(1, k)[None, :]) % 5 + 1
+    dims = B.make_dims(T, 128, 128, E, k)
+    _, g = gpu_map(dims, top_experts=top)
+    compare_map(g, oracle.sparse_map(top, E), top_expected=top)
+    assert g["status"] & B.STATUS_DUPLICATE_EXPERT  # slots 1..7 repeat experts within a token
+
+
+def test_map_given_top_out_of_range_is_dropped():
+    T, E, k = 100, 8, 2
+    top = np.tile(np.array([[1, 2]], np.int32), (T, 1))
+    top[5, 1] = 8
+    top[17, 0] = -3
+    dims = B.make_dims(T, 128, 128, E, k)
+    _, g = gpu_map(dims, top_experts=top)
+    assert g["status"] & B.STATUS_EXPERT_OUT_OF_RANGE
+    assert g["dest_row"][5 * k + 1] == -1 and g["dest_row"][17 * k] == -1
+    valid = top.ravel()[(top.ravel() >= 0) & (top.ravel() < E)]
+    assert g["tokens_per_expert"].sum() == valid.size
+
+
+def test_map_nonfinite_logits_flagged():
+    logits = torch.randn(64, 8)
+    logits[3, 2] = float("nan")
+    dims = B.make_dims(64, 128, 128, 8, 2)
+    _, g = gpu_map(dims, logits.to(torch.bfloat16))
+    assert g["status"] & B.STATUS_NONFINITE_LOGITS
+
+
+def test_map_deterministic_repeat():
+    w = WORKLOADS[5]
+    logits = _logits_only(w)
+    dims = B.make_dims(w.T, w.hidden, w.ffn, w.E, w.top_k)
+    bufs, g1 = gpu_map(dims, logits)
+    _, g2 = gpu_map(dims, logits, bufs=bufs)
+    for key in ("top_experts", "weights", "indices", "dest_row", "block_expert"):
+        assert (g1[key] == g2[key]).all()
