@@ -37,8 +37,8 @@ L2_BYTES = 126 * 2 ** 20
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=20)
-    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", type=int, default=2)
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -79,9 +79,9 @@ def ncu_traffic(kernel: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """nvidia-smi clock / throttle sampling; keeps the samples taken inside [t0, t1]."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -90,12 +90,12 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def stop(self, t0: float, t1: float):
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -104,22 +104,28 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
             out, _ = self.proc.communicate()
+        import datetime
+
         sm, mx, reasons = [], [], set()
         for line in out.strip().splitlines():
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 8:
+            if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                f_sm, f_mx = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
+            if not (t0 - 0.05 <= ts <= t1 + 0.05):
+                continue
+            sm.append(f_sm)
+            mx.append(f_mx)
             names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-            for n, v in zip(names, parts[4:8]):
+            for n, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
         if not sm:
-            return None
+            return {"sm_mhz": None, "sm_max_mhz": None, "samples": 0, "reasons": []}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
                 "reasons": sorted(reasons)}
 
@@ -168,10 +174,9 @@ def run_reference(args, w):
     oracle.build()
     threads = oracle.max_threads()
     inp32 = oracle_inputs32(w)
-    n_tok = cpu_sample_tokens(w, args.cpu_sample)
-    n_tok = max(1, n_tok // 4)  # each reference step is a quarter-size sample
-    for _ in range(max(args.warmup, 0) and 1):
-        oracle_sample_run(w, inp32, 1, threads)
+    # calibrate on a 4-token sample, then size each step so the K steps take about a minute
+    dt4, _ = oracle_sample_run(w, inp32, 4, threads)
+    n_tok = int(max(1, min(w.T, 60.0 / max(args.steps, 1) / (dt4 / 4))))
     times = []
     for _ in range(args.steps):
         dt, _ = oracle_sample_run(w, inp32, n_tok, threads)
@@ -259,17 +264,22 @@ def run_ours(args, w):
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    time.sleep(0.3 if sampler else 0.0)  # let the sampler start before the timed region
+    for _ in range(args.warmup):
+        step()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    wall0 = time.time()
     start.record(st)
     for i in range(args.steps):
         step(evs[i])
     stop.record(st)
     torch.cuda.synchronize()
+    wall1 = time.time()
     if world > 1:
         dist.barrier()
-    clocks = sampler.stop() if sampler else None
+    clocks = sampler.stop(wall0, wall1) if sampler else None
     ms = start.elapsed_time(stop)
     per_kernel = {n: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)]
                   for j, n in enumerate(names)}
