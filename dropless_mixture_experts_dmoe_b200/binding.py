@@ -230,6 +230,16 @@ def dmoe_padded_scatter(dims, y_pad, smap: SparseMap, weights, y, stream=None):
            "dmoe_padded_scatter")
 
 
+def dmoe_sparse_map_noalloc(dims: dmoe_dims, logits, smap: SparseMap, stream=None):
+    """Allocation-free routing + sparse map (static scratch inside the library; see
+    include/dmoe.h).  For callers that cannot allocate a workspace."""
+    fn = load().dmoe_sparse_map_noalloc
+    fn.argtypes = [ctypes.POINTER(dmoe_dims), _P, ctypes.POINTER(dmoe_map), _P]
+    fn.restype = _I
+    _check(fn(ctypes.byref(dims), _ptr(logits), ctypes.byref(smap.c), _stream(stream)),
+           "dmoe_sparse_map_noalloc")
+
+
 # ---- buffers (allocation only) ----------------------------------------------------------------
 
 class Buffers:

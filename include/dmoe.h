@@ -174,6 +174,28 @@ DMOE_API int dmoe_backward(const dmoe_dims *dims, const void *dy, const void *w1
                   void *dw3, void *dw2, float *dweights, void *ws, size_t ws_bytes,
                   void *stream);
 
+/* Allocation-free variant of dmoe_sparse_map.  The pages have no counterpart: this entry
+ * point exists for callers that cannot allocate device memory when they build the map, e.g.
+ * a plugin whose host application owns every device allocation, or a loop that must not
+ * call cudaMalloc (it can synchronise the device and its cost is unbounded), and therefore
+ * cannot provide the DMOE_WS_MAP workspace.
+ *   Same arguments, results and status bits as dmoe_sparse_map, without ws / ws_bytes.
+ *   Scratch: a static array of DMOE_NOALLOC_SCRATCH_BYTES in device global memory inside
+ *     libdmoe.so; every GPU that loads the library holds it until the process exits.  The
+ *     call needs ceil(T/64) * num_experts * 4 bytes of it and returns DMOE_ERR_WORKSPACE,
+ *     before any launch, when that exceeds the limit (e.g. T > 65536 at E = 256).
+ *   The call performs no allocation (no cudaMalloc, no cudaFree, no allocating library
+ *     routine).  Its first call on a device looks up the array's device address with
+ *     cudaGetSymbolAddress (once per device, with that device current); make that first call
+ *     before any stream capture.
+ *   Every call on a device shares the one array and leaves its contents behind; each call
+ *     rewrites all of the scratch it reads before reading it, so stale contents never leak
+ *     into a result.  Calls whose executions overlap on the GPU (different streams, or
+ *     different host threads without ordering) race on the array: serialise them. */
+#define DMOE_NOALLOC_SCRATCH_BYTES (1u << 20)
+DMOE_API int dmoe_sparse_map_noalloc(const dmoe_dims *dims, const void *logits,
+                                     const dmoe_map *map, void *stream);
+
 /* ---- Step entry points (each one kernel; dmoe_forward is exactly this sequence). ---- */
 
 /* padded_gather (walkthrough section 4.2, A_TO_B direction): x_pad[dest_row[t*k+s]] = x[t]
