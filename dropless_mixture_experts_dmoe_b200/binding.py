@@ -82,8 +82,13 @@ def load():
     lib.dmoe_expert_glu.argtypes = [D, _P, _P, _P, M, _P, _P, _P, _P]
     lib.dmoe_expert_down.argtypes = [D, _P, _P, M, _P, _P]
     lib.dmoe_padded_scatter.argtypes = [D, _P, M, _P, _P, _P]
+    lib.dmoe_bwd_dy_gather.argtypes = [D, _P, M, _P, _P, _P, _P]
+    lib.dmoe_bwd_dglu.argtypes = [D, _P, _P, _P, _P, M, _P, _P, _P]
+    lib.dmoe_bwd_dx.argtypes = [D, _P, _P, _P, _P, M, _P, _P]
+    lib.dmoe_bwd_wgrad.argtypes = [D, _P, _P, _P, _P, _P, M, _P, _P, _P, _P]
     for fn in ("dmoe_sparse_map", "dmoe_forward", "dmoe_backward", "dmoe_padded_gather",
-               "dmoe_expert_glu", "dmoe_expert_down", "dmoe_padded_scatter"):
+               "dmoe_expert_glu", "dmoe_expert_down", "dmoe_padded_scatter", "dmoe_bwd_dy_gather",
+               "dmoe_bwd_dglu", "dmoe_bwd_dx", "dmoe_bwd_wgrad"):
         getattr(lib, fn).restype = _I
     lib.dmoe_error_string.argtypes = [_I]
     lib.dmoe_error_string.restype = ctypes.c_char_p
@@ -230,6 +235,30 @@ def dmoe_padded_scatter(dims, y_pad, smap: SparseMap, weights, y, stream=None):
            "dmoe_padded_scatter")
 
 
+def dmoe_bwd_dy_gather(dims, dy, smap: SparseMap, y_pad, dy_pad, dweights, stream=None):
+    _check(load().dmoe_bwd_dy_gather(ctypes.byref(dims), _ptr(dy), ctypes.byref(smap.c), _ptr(y_pad),
+                                     _ptr(dy_pad), _ptr(dweights), _stream(stream)),
+           "dmoe_bwd_dy_gather")
+
+
+def dmoe_bwd_dglu(dims, dy_pad, w2, a_saved, bm_saved, smap: SparseMap, da, dbm, stream=None):
+    _check(load().dmoe_bwd_dglu(ctypes.byref(dims), _ptr(dy_pad), _ptr(w2), _ptr(a_saved),
+                                _ptr(bm_saved), ctypes.byref(smap.c), _ptr(da), _ptr(dbm),
+                                _stream(stream)), "dmoe_bwd_dglu")
+
+
+def dmoe_bwd_dx(dims, da, dbm, w1, w3, smap: SparseMap, dx_pad, stream=None):
+    _check(load().dmoe_bwd_dx(ctypes.byref(dims), _ptr(da), _ptr(dbm), _ptr(w1), _ptr(w3),
+                              ctypes.byref(smap.c), _ptr(dx_pad), _stream(stream)), "dmoe_bwd_dx")
+
+
+def dmoe_bwd_wgrad(dims, x_pad, h_saved, dy_pad, da, dbm, smap: SparseMap, dw1, dw3, dw2,
+                   stream=None):
+    _check(load().dmoe_bwd_wgrad(ctypes.byref(dims), _ptr(x_pad), _ptr(h_saved), _ptr(dy_pad),
+                                 _ptr(da), _ptr(dbm), ctypes.byref(smap.c), _ptr(dw1), _ptr(dw3),
+                                 _ptr(dw2), _stream(stream)), "dmoe_bwd_wgrad")
+
+
 def dmoe_sparse_map_noalloc(dims: dmoe_dims, logits, smap: SparseMap, stream=None):
     """Allocation-free routing + sparse map (static scratch inside the library; see
     include/dmoe.h).  For callers that cannot allocate a workspace."""
@@ -265,6 +294,10 @@ class Buffers:
             self.saved = torch.empty(total, **u8)
             self.offsets = dict(x_pad=offs[0], a=offs[1], bm=offs[2], h=offs[3], y_pad=offs[4])
             self.ws_bwd = torch.empty(max(dmoe_workspace_bytes(dims, WS_BACKWARD), 16), **u8)
+            bf = dict(dtype=torch.bfloat16, device=device)
+            # separate step buffers for driving the backward step entry points one by one
+            self.bstep = dict(dy_pad=torch.empty((P, h), **bf), da=torch.empty((P, f), **bf),
+                              dbm=torch.empty((P, f), **bf), dx_pad=torch.empty((P, h), **bf))
         else:
             self.ws_fwd = torch.empty(dmoe_workspace_bytes(dims, WS_FORWARD), **u8)
             bf = dict(dtype=torch.bfloat16, device=device)

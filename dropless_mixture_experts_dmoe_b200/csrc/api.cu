@@ -60,6 +60,34 @@ int check_map(const dmoe_map *m, bool need_weights) {
 
 inline int launch_rc(cudaError_t e) { return e == cudaSuccess ? DMOE_OK : DMOE_ERR_LAUNCH; }
 
+GemmProblem problem_of(const dmoe_dims *d, const dmoe_map *m) {
+  GemmProblem g;
+  g.h = d->hidden;
+  g.f = d->ffn;
+  g.E = d->num_experts;
+  g.nblk_cap = (int)(pmax_of(d) / DMOE_BLOCKING);
+  g.num_blocks = m->num_blocks;
+  g.block_expert = m->block_expert;
+  g.padded_bins = m->padded_bins;
+  g.status = m->status;
+  return g;
+}
+
+// Backward workspace layout: dY_pad [P,h] | dA [P,f] | dBm [P,f] | dX_pad [P,h]
+struct BwdLayout {
+  size_t dy, da, db, dx, total;
+};
+BwdLayout bwd_layout(const dmoe_dims *d) {
+  const size_t P = (size_t)pmax_of(d);
+  BwdLayout l;
+  l.dy = 0;
+  l.da = align_up(l.dy + P * d->hidden * 2);
+  l.db = align_up(l.da + P * d->ffn * 2);
+  l.dx = align_up(l.db + P * d->ffn * 2);
+  l.total = align_up(l.dx + P * d->hidden * 2);
+  return l;
+}
+
 // Forward workspace layout (inference): X_pad [P,h] | H [P,f] | Y_pad [P,h]
 struct FwdLayout {
   size_t xpad, h, ypad, total;
@@ -102,7 +130,7 @@ size_t dmoe_workspace_bytes(const dmoe_dims *dims, int kind) {
     case DMOE_WS_FORWARD:
       return fwd_layout(dims).total;
     case DMOE_WS_BACKWARD:
-      return 0;
+      return bwd_layout(dims).total;
     default:
       return 0;
   }
@@ -169,10 +197,8 @@ int dmoe_expert_glu(const dmoe_dims *dims, const void *x_pad, const void *w1, co
       (a_out && !aligned16(a_out)) || (b_out && !aligned16(b_out)))
     return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
-  const int nblk_cap = (int)(pmax_of(dims) / DMOE_BLOCKING);
-  return launch_rc(launch_glu_gemm(dims->hidden, dims->ffn, dims->num_experts, nblk_cap, x_pad, w1,
-                                   w3, map->num_blocks, map->block_expert, h_out, a_out, b_out,
-                                   map->status, static_cast<cudaStream_t>(stream)));
+  return launch_rc(launch_glu_gemm(problem_of(dims, map), x_pad, w1, w3, h_out, a_out, b_out,
+                                   static_cast<cudaStream_t>(stream)));
 }
 
 int dmoe_expert_down(const dmoe_dims *dims, const void *h_in, const void *w2,
@@ -183,10 +209,8 @@ int dmoe_expert_down(const dmoe_dims *dims, const void *h_in, const void *w2,
   if (!h_in || !w2 || !y_pad) return DMOE_ERR_NULL;
   if (!aligned16(h_in) || !aligned16(w2) || !aligned16(y_pad)) return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
-  const int nblk_cap = (int)(pmax_of(dims) / DMOE_BLOCKING);
-  return launch_rc(launch_down_gemm(dims->hidden, dims->ffn, dims->num_experts, nblk_cap, h_in, w2,
-                                    map->num_blocks, map->block_expert, y_pad, map->status,
-                                    static_cast<cudaStream_t>(stream)));
+  return launch_rc(
+      launch_down_gemm(problem_of(dims, map), h_in, w2, y_pad, static_cast<cudaStream_t>(stream)));
 }
 
 int dmoe_padded_scatter(const dmoe_dims *dims, const void *y_pad, const dmoe_map *map,
@@ -236,26 +260,86 @@ int dmoe_forward(const dmoe_dims *dims, const void *x, const void *w1, const voi
   return dmoe_padded_scatter(dims, ypad, map, map->weights, y, stream);
 }
 
+int dmoe_bwd_dy_gather(const dmoe_dims *dims, const void *dy, const dmoe_map *map,
+                       const void *y_pad, void *dy_pad, float *dweights, void *stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_map(map, true))) return rc;
+  if (!dy || !y_pad || !dy_pad || !dweights) return DMOE_ERR_NULL;
+  if (!aligned16(dy) || !aligned16(y_pad) || !aligned16(dy_pad)) return DMOE_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return launch_rc(launch_dy_gather(dims->T, dims->hidden, dims->top_k, dims->num_experts, dy,
+                                    map->dest_row, map->weights, map->tokens_per_expert,
+                                    map->padded_bins, y_pad, dy_pad, dweights,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+int dmoe_bwd_dglu(const dmoe_dims *dims, const void *dy_pad, const void *w2, const void *a_saved,
+                  const void *bm_saved, const dmoe_map *map, void *da, void *dbm, void *stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_map(map, false))) return rc;
+  if (!dy_pad || !w2 || !a_saved || !bm_saved || !da || !dbm) return DMOE_ERR_NULL;
+  if (!aligned16(dy_pad) || !aligned16(w2) || !aligned16(a_saved) || !aligned16(bm_saved) ||
+      !aligned16(da) || !aligned16(dbm))
+    return DMOE_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return launch_rc(launch_dglu_gemm(problem_of(dims, map), dy_pad, w2, a_saved, bm_saved, da, dbm,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+int dmoe_bwd_dx(const dmoe_dims *dims, const void *da, const void *dbm, const void *w1,
+                const void *w3, const dmoe_map *map, void *dx_pad, void *stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_map(map, false))) return rc;
+  if (!da || !dbm || !w1 || !w3 || !dx_pad) return DMOE_ERR_NULL;
+  if (!aligned16(da) || !aligned16(dbm) || !aligned16(w1) || !aligned16(w3) || !aligned16(dx_pad))
+    return DMOE_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return launch_rc(
+      launch_dx_gemm(problem_of(dims, map), da, dbm, w1, w3, dx_pad, static_cast<cudaStream_t>(stream)));
+}
+
+int dmoe_bwd_wgrad(const dmoe_dims *dims, const void *x_pad, const void *h_saved,
+                   const void *dy_pad, const void *da, const void *dbm, const dmoe_map *map,
+                   float *dw1, float *dw3, float *dw2, void *stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_map(map, false))) return rc;
+  if (!x_pad || !h_saved || !dy_pad || !da || !dbm || !dw1 || !dw3 || !dw2) return DMOE_ERR_NULL;
+  if (!aligned16(x_pad) || !aligned16(h_saved) || !aligned16(dy_pad) || !aligned16(da) ||
+      !aligned16(dbm) || !aligned16(dw1) || !aligned16(dw3) || !aligned16(dw2))
+    return DMOE_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return launch_rc(launch_wgrad_gemm(problem_of(dims, map), x_pad, h_saved, dy_pad, da, dbm, dw1,
+                                     dw3, dw2, static_cast<cudaStream_t>(stream)));
+}
+
 int dmoe_backward(const dmoe_dims *dims, const void *dy, const void *w1, const void *w3,
-                  const void *w2, const dmoe_map *map, const void *saved, void *dx, void *dw1,
-                  void *dw3, void *dw2, float *dweights, void *ws, size_t ws_bytes,
+                  const void *w2, const dmoe_map *map, const void *saved, void *dx, float *dw1,
+                  float *dw3, float *dw2, float *dweights, void *ws, size_t ws_bytes,
                   void *stream) {
-  (void)dims;
-  (void)dy;
-  (void)w1;
-  (void)w3;
-  (void)w2;
-  (void)map;
-  (void)saved;
-  (void)dx;
-  (void)dw1;
-  (void)dw3;
-  (void)dw2;
-  (void)dweights;
-  (void)ws;
-  (void)ws_bytes;
-  (void)stream;
-  return DMOE_ERR_SHAPE;
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_map(map, true))) return rc;
+  if (!dy || !w1 || !w3 || !w2 || !saved || !dx || !dw1 || !dw3 || !dw2 || !dweights || !ws)
+    return DMOE_ERR_NULL;
+  const BwdLayout l = bwd_layout(dims);
+  if (ws_bytes < l.total) return DMOE_ERR_WORKSPACE;
+  if (!aligned16(saved) || !aligned16(ws) || !aligned16(dx)) return DMOE_ERR_ALIGN;
+  size_t off[5], total;
+  saved_layout(dims, off, &total);
+  const uint8_t *sv = static_cast<const uint8_t *>(saved);
+  const void *xpad = sv + off[0], *abuf = sv + off[1], *bbuf = sv + off[2], *hbuf = sv + off[3],
+             *ypad = sv + off[4];
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  void *dypad = w + l.dy, *da = w + l.da, *db = w + l.db, *dxpad = w + l.dx;
+  if ((rc = dmoe_bwd_dy_gather(dims, dy, map, ypad, dypad, dweights, stream))) return rc;
+  if ((rc = dmoe_bwd_dglu(dims, dypad, w2, abuf, bbuf, map, da, db, stream))) return rc;
+  if ((rc = dmoe_bwd_wgrad(dims, xpad, hbuf, dypad, da, db, map, dw1, dw3, dw2, stream))) return rc;
+  if ((rc = dmoe_bwd_dx(dims, da, db, w1, w3, map, dxpad, stream))) return rc;
+  return dmoe_padded_scatter(dims, dxpad, map, nullptr, dx, stream);
 }
 
 const char *dmoe_error_string(int code) {

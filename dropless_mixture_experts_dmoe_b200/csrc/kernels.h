@@ -33,15 +33,37 @@ cudaError_t launch_gather(int T, int h, int k, int E, const void *x, const int32
 cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const int32_t *dest_row,
                            const float *weights, void *y, cudaStream_t st);
 
-// Grouped tcgen05 GEMMs over the non-empty row blocks.
-cudaError_t launch_glu_gemm(int h, int f, int E, int nblk_cap, const void *x_pad,
-                            const void *w1, const void *w3, const int32_t *num_blocks,
-                            const int32_t *block_expert, void *h_out, void *a_out, void *b_out,
-                            int32_t *status, cudaStream_t st);
-cudaError_t launch_down_gemm(int h, int f, int E, int nblk_cap, const void *h_in,
-                             const void *w2, const int32_t *num_blocks,
-                             const int32_t *block_expert, void *y_pad, int32_t *status,
+// dY gather for the backward: dY_pad[dest_row[t*k+s]] = bf16(w_ts * dy_t), padding rows zero,
+// and the routing-weight gradient dweights[t*k+s] = <dy_t, Y_pad[dest_row[t*k+s]]>.
+cudaError_t launch_dy_gather(int T, int h, int k, int E, const void *dy, const int32_t *dest_row,
+                             const float *weights, const int32_t *counts,
+                             const int32_t *padded_bins, const void *y_pad, void *dy_pad,
+                             float *dweights, cudaStream_t st);
+
+// Shape and map pointers shared by the grouped GEMM launchers.
+struct GemmProblem {
+  int h, f, E, nblk_cap;
+  const int32_t *num_blocks;
+  const int32_t *block_expert;
+  const int32_t *padded_bins;
+  int32_t *status;
+};
+
+// Grouped tcgen05 GEMMs over the non-empty row blocks (forward) ...
+cudaError_t launch_glu_gemm(const GemmProblem &g, const void *x_pad, const void *w1,
+                            const void *w3, void *h_out, void *a_out, void *b_out,
+                            cudaStream_t st);
+cudaError_t launch_down_gemm(const GemmProblem &g, const void *h_in, const void *w2, void *y_pad,
                              cudaStream_t st);
+// ... and the backward: dH with the fused dGLU epilogue, dX, and the weight gradients.
+cudaError_t launch_dglu_gemm(const GemmProblem &g, const void *dy_pad, const void *w2,
+                             const void *a_in, const void *b_in, void *da_out, void *db_out,
+                             cudaStream_t st);
+cudaError_t launch_dx_gemm(const GemmProblem &g, const void *da, const void *db, const void *w1,
+                           const void *w3, void *dx_pad, cudaStream_t st);
+cudaError_t launch_wgrad_gemm(const GemmProblem &g, const void *x_pad, const void *h_in,
+                              const void *dy_pad, const void *da, const void *db, float *dw1,
+                              float *dw3, float *dw2, cudaStream_t st);
 
 int device_sm_count();
 

@@ -166,12 +166,13 @@ DMOE_API int dmoe_forward(const dmoe_dims *dims, const void *x, const void *w1, 
  * the activation is recomputed from the saved pre-activations).
  *   dy [T,h] bf16; w1, w3, w2 as in dmoe_forward; map from dmoe_sparse_map; saved from
  *   dmoe_forward(saved != NULL).
- *   Outputs: dx [T,h] bf16; dw1, dw3 [E,f,h] bf16; dw2 [E,h,f] bf16 (experts that receive
- *   no token get exact zeros); dweights [T,k] fp32 = <dy_t, Y_ts>.
+ *   Outputs: dx [T,h] bf16; dw1, dw3 [E,f,h] fp32; dw2 [E,h,f] fp32 (the weight gradients
+ *   of a mixed-precision step are kept in fp32; experts that receive no token get exact
+ *   zeros); dweights [T,k] fp32 = <dy_t, Y_ts>.
  *   ws: dmoe_workspace_bytes(dims, DMOE_WS_BACKWARD) bytes. */
 DMOE_API int dmoe_backward(const dmoe_dims *dims, const void *dy, const void *w1, const void *w3,
-                  const void *w2, const dmoe_map *map, const void *saved, void *dx, void *dw1,
-                  void *dw3, void *dw2, float *dweights, void *ws, size_t ws_bytes,
+                  const void *w2, const dmoe_map *map, const void *saved, void *dx, float *dw1,
+                  float *dw3, float *dw2, float *dweights, void *ws, size_t ws_bytes,
                   void *stream);
 
 /* Allocation-free variant of dmoe_sparse_map.  The pages have no counterpart: this entry
@@ -223,6 +224,42 @@ DMOE_API int dmoe_expert_down(const dmoe_dims *dims, const void *h_in, const voi
  * dx_t = sum_s dX_pad[dest_row[t*k+s]]).  y_pad [P_max,h] -> y [T,h], bf16. */
 DMOE_API int dmoe_padded_scatter(const dmoe_dims *dims, const void *y_pad, const dmoe_map *map,
                         const float *weights, void *y, void *stream);
+
+/* ---- Backward step entry points (each one kernel); dmoe_backward runs dy_gather, dglu,
+ * wgrad, dx and dmoe_padded_scatter(weights = NULL) in that order. ---- */
+
+/* Gradient of the weighted padded_scatter (walkthrough section 4.2: a padded_gather of dy
+ * plus the routing-weight gradient of _padded_copy_wgrad):
+ *   dy_pad[dest_row[t*k+s]] = bf16(w_ts * dy_t); padding rows of every expert's last block = 0;
+ *   dweights[t*k+s] = <dy_t, Y_pad[dest_row[t*k+s]]> (fp32; 0 for dropped entries).
+ * dy [T,h], y_pad [P_max,h] (forward output rows) -> dy_pad [P_max,h] bf16, dweights [T,k] fp32. */
+DMOE_API int dmoe_bwd_dy_gather(const dmoe_dims *dims, const void *dy, const dmoe_map *map,
+                                const void *y_pad, void *dy_pad, float *dweights, void *stream);
+
+/* dH GEMM with the gated-SiLU gradient fused into its epilogue (walkthrough section 4.4:
+ * the activation is recomputed from the saved pre-activations instead of being stored):
+ *   dH = dY_pad[b] W2_e (fp32), s = sigmoid(A), dA = bf16(dH * Bm * s * (1 + A (1 - s))),
+ *   dBm = bf16(dH * A * s), for every row block b < num_blocks of expert e.
+ * a_saved, bm_saved: bf16 A, Bm of dmoe_forward; all [P_max,f] except dy_pad [P_max,h]. */
+DMOE_API int dmoe_bwd_dglu(const dmoe_dims *dims, const void *dy_pad, const void *w2,
+                           const void *a_saved, const void *bm_saved, const dmoe_map *map,
+                           void *da, void *dbm, void *stream);
+
+/* dX GEMM: dX_pad[b] = bf16(dA[b] W1_e + dBm[b] W3_e), one fp32 accumulator over both K
+ * passes.  da, dbm [P_max,f] -> dx_pad [P_max,h]. */
+DMOE_API int dmoe_bwd_dx(const dmoe_dims *dims, const void *da, const void *dbm, const void *w1,
+                         const void *w3, const dmoe_map *map, void *dx_pad, void *stream);
+
+/* Weight gradients, per expert e over its padded rows r in [padded_bins[e-1], padded_bins[e])
+ * (padding rows are zero, so they add nothing; the walkthrough's stk path needs a transposed
+ * topology for this, section 4.3; here each output tile walks its expert's rows directly):
+ *   dW1_e = sum_r dA_r^T X_pad_r,  dW3_e = sum_r dBm_r^T X_pad_r  ([f,h] each),
+ *   dW2_e = sum_r dY_pad_r^T H_r  ([h,f]); fp32 accumulation and fp32 output (dw1, dw3,
+ * dw2 are float*), no split-K, so the result is deterministic; experts without rows get
+ * exact zeros. */
+DMOE_API int dmoe_bwd_wgrad(const dmoe_dims *dims, const void *x_pad, const void *h_saved,
+                            const void *dy_pad, const void *da, const void *dbm,
+                            const dmoe_map *map, float *dw1, float *dw3, float *dw2, void *stream);
 
 /* ---- Diagnostics. ---- */
 DMOE_API const char *dmoe_error_string(int code);

@@ -29,11 +29,18 @@ def metrics(got, ref):
     return rel, mx, rms
 
 
-def assert_close(got, ref, what=""):
+# Stress shapes outside the five named workloads (few tokens per expert): a bf16 pipeline's
+# element error is up to ~3 roundings (2^-8 each) of the element's largest product, and with
+# few products per element those are up to ~20x the tensor RMS, so the max-abs bound is
+# 2.5e-1 * RMS there; a wrong element errs by about one RMS and still fails it.
+MAX_ABS_RMS_STRESS = 2.5e-1
+
+
+def assert_close(got, ref, what="", max_abs_rms=MAX_ABS_RMS):
     rel, mx, rms = metrics(got, ref)
     assert np.isfinite(got).all(), f"{what}: non-finite values"
     assert rel <= REL_L2, f"{what}: relative L2 {rel:.3e} > {REL_L2}"
-    assert mx <= MAX_ABS_RMS * rms, f"{what}: max abs {mx:.3e} > {MAX_ABS_RMS} * RMS {rms:.3e}"
+    assert mx <= max_abs_rms * rms, f"{what}: max abs {mx:.3e} > {max_abs_rms} * RMS {rms:.3e}"
     return rel, mx, rms
 
 
@@ -105,3 +112,23 @@ def sample_tokens(top: np.ndarray, E: int, n: int, seed: int = 0) -> np.ndarray:
     while len(picks) < min(n, T):
         picks.add(int(rng.integers(T)))
     return np.array(sorted(picks), np.int32)
+
+
+def gpu_backward(dims, inp: dict):
+    """Map + training forward + dmoe_backward through the C ABI.
+
+    Returns (bufs, dev, y, grads) with grads = dict(dx, dw1, dw3, dw2, dw) on the device."""
+    bufs, dev, y = gpu_forward(dims, inp, train=True)
+    dev["dy"] = inp["dy"].cuda()
+    E, f, h, T, k = dims.num_experts, dims.ffn, dims.hidden, dims.T, dims.top_k
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    f32 = dict(dtype=torch.float32, device="cuda")
+    g = dict(dx=torch.empty((T, h), **bf), dw1=torch.empty((E, f, h), **f32),
+             dw3=torch.empty((E, f, h), **f32), dw2=torch.empty((E, h, f), **f32),
+             dw=torch.empty((T, k), **f32))
+    for v in g.values():  # poison: every output element must be written
+        v.fill_(float("nan"))
+    B.dmoe_backward(dims, dev["dy"], dev["w1"], dev["w3"], dev["w2"], bufs.map, bufs.saved,
+                    g["dx"], g["dw1"], g["dw3"], g["dw2"], g["dw"], bufs.ws_bwd)
+    torch.cuda.synchronize()
+    return bufs, dev, y, g

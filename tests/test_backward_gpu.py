@@ -1,0 +1,146 @@
+"""Backward parity (dY gather + routing-weight gradient, dH with the fused dGLU epilogue,
+dX, scatter-sum, weight gradients) against the oracle, and each backward GEMM against
+float64 PyTorch on the same bf16 operands."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dropless_mixture_experts_dmoe_b200 import binding as B
+from dropless_mixture_experts_dmoe_b200.workloads import WORKLOADS, custom, make_inputs
+
+from helpers import (MAX_ABS_RMS, MAX_ABS_RMS_STRESS, assert_close, dims_of, gpu_backward,
+                     oracle_inputs, sample_tokens, to_np)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    WORKLOADS[1],                     # tiny
+    custom(512, 384, 384, 8, 2),      # ragged column tiles in every GEMM
+    custom(300, 256, 256, 16, 4),     # top-4
+    custom(1000, 128, 512, 5, 3),     # h = 128 < 256: half-empty dX / dW1 column tiles
+    custom(600, 640, 128, 64, 8),     # many experts with few rows each
+    custom(40, 128, 256, 64, 2),      # most experts without any row: exact-zero gradients
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.describe())
+def test_backward_full_parity_small(w):
+    inp = make_inputs(w, with_dy=True)
+    dims = dims_of(w)
+    bufs, dev, y, g = gpu_backward(dims, inp)
+    assert int(bufs.map.status.item()) == 0
+    o = oracle_inputs(inp)
+    top, wts = oracle.route(o["logits"], w.top_k)
+    ref = oracle.backward(o["x"], o["dy"], o["w1"], o["w3"], o["w2"], top, wts)
+    tol = MAX_ABS_RMS if w.number else MAX_ABS_RMS_STRESS  # named workload vs stress shape
+    for gk, rk in (("dx", "dx"), ("dw1", "dW1"), ("dw3", "dW3"), ("dw2", "dW2"), ("dw", "dw")):
+        assert_close(to_np(g[gk]), ref[rk], f"{rk} {w.describe()}", max_abs_rms=tol)
+    counts = np.bincount(top.ravel(), minlength=w.E)
+    for e in np.nonzero(counts == 0)[0]:  # experts without tokens: exact zeros
+        assert (g["dw1"][e] == 0).all() and (g["dw3"][e] == 0).all() and (g["dw2"][e] == 0).all()
+
+
+@pytest.mark.parametrize("w", SMALL[1:4], ids=lambda w: w.describe())
+def test_backward_gemms_against_float64(w):
+    """Every backward GEMM mode on its own bf16 inputs (MN-major operands included)."""
+    inp = make_inputs(w, with_dy=True)
+    dims = dims_of(w)
+    bufs, dev, y, g = gpu_backward(dims, inp)
+    st = bufs.bstep
+    B.dmoe_bwd_dy_gather(dims, dev["dy"], bufs.map, bufs.view("y_pad"), st["dy_pad"],
+                         torch.empty((w.T, w.top_k), dtype=torch.float32, device="cuda"))
+    B.dmoe_bwd_dglu(dims, st["dy_pad"], dev["w2"], bufs.view("a"), bufs.view("bm"), bufs.map,
+                    st["da"], st["dbm"])
+    B.dmoe_bwd_dx(dims, st["da"], st["dbm"], dev["w1"], dev["w3"], bufs.map, st["dx_pad"])
+    torch.cuda.synchronize()
+    nb = int(bufs.map.num_blocks.item())
+    P = nb * 128
+    be = bufs.map.block_expert.cpu().numpy()
+    D = lambda t: t[:P].double().cpu()
+    dy_pad, da, dbm, dx_pad = D(st["dy_pad"]), D(st["da"]), D(st["dbm"]), D(st["dx_pad"])
+    A, Bm, H, Xp = D(bufs.view("a")), D(bufs.view("bm")), D(bufs.view("h")), D(bufs.view("x_pad"))
+    W1, W3, W2 = inp["w1"].double(), inp["w3"].double(), inp["w2"].double()
+    # dY_pad rows hold w * dy of their token (bf16), padding rows are zero
+    dest = bufs.map.dest_row.cpu().numpy()
+    wts = bufs.map.weights.cpu().double()
+    ref_dy = torch.zeros(P, w.hidden, dtype=torch.float64)
+    tok = torch.arange(w.T * w.top_k) // w.top_k
+    ref_dy[dest] = (wts.reshape(-1, 1) * inp["dy"].double()[tok]).to(torch.bfloat16).double()
+    assert torch.equal(dy_pad, ref_dy)
+    for b in range(nb):
+        e = int(be[b])
+        rows = slice(b * 128, (b + 1) * 128)
+        dh = dy_pad[rows] @ W2[e]
+        s = torch.sigmoid(A[rows])
+        da_ref = dh * Bm[rows] * s * (1 + A[rows] * (1 - s))
+        db_ref = dh * A[rows] * s
+        assert torch.allclose(da[rows], da_ref, rtol=2e-2, atol=2e-3), ("dA", b)
+        assert torch.allclose(dbm[rows], db_ref, rtol=2e-2, atol=2e-3), ("dBm", b)
+        dx_ref = da[rows] @ W1[e] + dbm[rows] @ W3[e]
+        assert torch.allclose(dx_pad[rows], dx_ref, rtol=2e-2, atol=2e-3), ("dX", b)
+    pb = bufs.map.padded_bins.cpu().numpy()
+    for e in range(w.E):
+        r0 = 0 if e == 0 else int(pb[e - 1])
+        r1 = int(pb[e])
+        dw1 = da[r0:r1].T @ Xp[r0:r1]
+        dw3 = dbm[r0:r1].T @ Xp[r0:r1]
+        dw2 = dy_pad[r0:r1].T @ H[r0:r1]
+        for got, ref, n in ((g["dw1"][e], dw1, "dW1"), (g["dw3"][e], dw3, "dW3"), (g["dw2"][e], dw2, "dW2")):
+            got = got.double().cpu()
+            assert torch.allclose(got, ref, rtol=1e-4, atol=1e-5 * (ref.abs().max().item() + 1e-30)), (n, e)
+
+
+def test_backward_skewed_full_size_sampled():
+    """The skewed fwd+bwd workload at full size: sampled dx / dw tokens and sampled weight-
+    gradient elements (heavy, light and empty experts) against the oracle."""
+    w = WORKLOADS[5]
+    inp = make_inputs(w, with_dy=True)
+    dims = dims_of(w)
+    bufs, dev, y, g = gpu_backward(dims, inp)
+    assert int(bufs.map.status.item()) == 0
+    for k in ("dx", "dw1", "dw3", "dw2", "dw"):
+        assert torch.isfinite(g[k].float()).all(), k
+    o = {k: inp[k].float().numpy() for k in ("x", "dy", "w1", "w3", "w2")}
+    top, wts = oracle.route(inp["logits"].float().numpy(), w.top_k)
+    assert (bufs.map.top_experts.cpu().numpy() == top).all()
+    toks = sample_tokens(top, w.E, 48, seed=5)
+    dx_ref, dw_ref = oracle.backward_tokens(o["x"], o["dy"], o["w1"], o["w3"], o["w2"], top, wts,
+                                            toks, threads=oracle.max_threads())
+    assert_close(to_np(g["dx"])[toks], dx_ref, "dx sampled")
+    assert_close(to_np(g["dw"])[toks], dw_ref, "dw sampled")
+    counts = np.bincount(top.ravel(), minlength=w.E)
+    empty = np.nonzero(counts == 0)[0]
+    for e in empty:
+        assert (g["dw1"][e] == 0).all() and (g["dw2"][e] == 0).all()
+    rng = np.random.default_rng(55)
+    heavy = int(np.argmax(counts))
+    light = [int(e) for e in np.nonzero((counts > 0) & (counts < 200))[0][:3]]
+    experts = [heavy] + light + [int(e) for e in rng.choice(np.nonzero(counts > 0)[0], 4)]
+    q = []
+    for e in experts:
+        for _ in range(3):
+            q.append((1, e, rng.integers(w.ffn), rng.integers(w.hidden)))
+            q.append((3, e, rng.integers(w.ffn), rng.integers(w.hidden)))
+            q.append((2, e, rng.integers(w.hidden), rng.integers(w.ffn)))
+    q = np.array(q, np.int32)
+    ref = oracle.wgrad_elements(o["x"], o["dy"], o["w1"], o["w3"], o["w2"], top, wts, q,
+                                threads=oracle.max_threads())
+    gm = {1: g["dw1"], 3: g["dw3"], 2: g["dw2"]}
+    got = np.array([float(gm[a][b, c, d]) for a, b, c, d in q])
+    assert_close(got, ref, "sampled weight-gradient elements")
+
+
+def test_backward_deterministic():
+    w = SMALL[2]
+    inp = make_inputs(w, with_dy=True)
+    dims = dims_of(w)
+    _, _, _, g1 = gpu_backward(dims, inp)
+    _, _, _, g2 = gpu_backward(dims, inp)
+    for k in g1:
+        a, b = g1[k], g2[k]
+        if a.dtype == torch.bfloat16:
+            a, b = a.view(torch.int16), b.view(torch.int16)
+        else:
+            a, b = a.view(torch.int32), b.view(torch.int32)
+        assert torch.equal(a, b), k

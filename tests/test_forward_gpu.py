@@ -9,7 +9,8 @@ import oracle
 from dropless_mixture_experts_dmoe_b200 import binding as B
 from dropless_mixture_experts_dmoe_b200.workloads import WORKLOADS, custom, make_inputs
 
-from helpers import assert_close, compare_map, dims_of, gpu_forward, oracle_inputs, sample_tokens, to_np
+from helpers import (MAX_ABS_RMS, MAX_ABS_RMS_STRESS, assert_close, compare_map, dims_of,
+                     gpu_forward, oracle_inputs, sample_tokens, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -35,7 +36,8 @@ def test_forward_full_parity_small(w):
     compare_map(g, m, top_expected=top)
     assert int(g["status"][0]) == 0
     ref = oracle.forward(o["x"], o["w1"], o["w3"], o["w2"], top, wts, threads=8)
-    assert_close(to_np(y), ref, f"y {w.describe()}")
+    tol = MAX_ABS_RMS if w.number else MAX_ABS_RMS_STRESS  # named workload vs stress shape
+    assert_close(to_np(y), ref, f"y {w.describe()}", max_abs_rms=tol)
 
 
 @pytest.mark.parametrize("w", SMALL[:3], ids=lambda w: w.describe())
