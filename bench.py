@@ -147,21 +147,26 @@ def oracle_sample_run(w, inp32, n_tok, threads):
     toks = np.arange(n_tok, dtype=np.int32)
     oracle.forward(inp32["x"], inp32["w1"], inp32["w3"], inp32["w2"], top, wts, tokens=toks,
                    threads=threads)
+    if w.backward:  # the sample's own backward: dx, dw and its weight-gradient contributions
+        oracle.backward(inp32["x"][:n_tok], inp32["dy"][:n_tok], inp32["w1"], inp32["w3"],
+                        inp32["w2"], top[:n_tok], wts[:n_tok])
     return time.perf_counter() - t0, n_tok
 
 
 def oracle_inputs32(w):
     from dropless_mixture_experts_dmoe_b200.workloads import make_inputs
 
-    inp = make_inputs(w, with_dy=False)
+    inp = make_inputs(w)
     return {k: v.float().numpy() for k, v in inp.items()}
 
 
 def cpu_sample_tokens(w, requested):
     if requested:
         return requested
-    # about 10-30 s of oracle work on a few dozen cores
+    # about 10-30 s of oracle work on a few dozen cores (the backward sample runs on one)
     per_tok = 6 * w.top_k * w.hidden * w.ffn
+    if w.backward:
+        return max(8, min(w.T, int(2e10 / (3 * per_tok))))
     return max(8, min(w.T, int(4e11 / per_tok)))
 
 
@@ -227,32 +232,55 @@ def run_ours(args, w):
     B.load()
 
     dims = B.make_dims(w.T, w.hidden, w.ffn, w.E, w.top_k)
-    inp = make_inputs(w, with_dy=False)
+    train = w.backward
+    inp = make_inputs(w, with_dy=train)
     dev = {k: v.cuda() for k, v in inp.items()}
-    bufs = B.Buffers(dims, train=False)
+    bufs = B.Buffers(dims, train=train)
     y = torch.empty((w.T, w.hidden), dtype=torch.bfloat16, device="cuda")
     st = torch.cuda.current_stream()
-    xp, hb, yp = bufs.step["x_pad"], bufs.step["h"], bufs.step["y_pad"]
+    if train:
+        xp, hb, yp = bufs.view("x_pad"), bufs.view("h"), bufs.view("y_pad")
+        ab, bb = bufs.view("a"), bufs.view("bm")
+        bs = bufs.bstep
+        f32 = dict(dtype=torch.float32, device="cuda")
+        grads = dict(dx=torch.empty_like(y), dw1=torch.empty((w.E, w.ffn, w.hidden), **f32),
+                     dw3=torch.empty((w.E, w.ffn, w.hidden), **f32),
+                     dw2=torch.empty((w.E, w.hidden, w.ffn), **f32), dw=torch.empty((w.T, w.top_k), **f32))
+    else:
+        xp, hb, yp = bufs.step["x_pad"], bufs.step["h"], bufs.step["y_pad"]
+        ab = bb = None
     names = ["map", "gather", "glu_gemm", "down_gemm", "scatter"]
+    if train:
+        names += ["dy_gather", "dglu_gemm", "wgrad_gemm", "dx_gemm", "dx_scatter"]
+    n_ev = len(names) + 1
 
     def step(ev=None):
-        if ev is not None:
-            ev[0].record(st)
+        def mark(i):
+            if ev is not None:
+                ev[i].record(st)
+        mark(0)
         B.dmoe_sparse_map(dims, dev["logits"], bufs.map, bufs.ws_map, st)
-        if ev is not None:
-            ev[1].record(st)
+        mark(1)
         B.dmoe_padded_gather(dims, dev["x"], bufs.map, xp, st)
-        if ev is not None:
-            ev[2].record(st)
-        B.dmoe_expert_glu(dims, xp, dev["w1"], dev["w3"], bufs.map, hb, None, None, st)
-        if ev is not None:
-            ev[3].record(st)
+        mark(2)
+        B.dmoe_expert_glu(dims, xp, dev["w1"], dev["w3"], bufs.map, hb, ab, bb, st)
+        mark(3)
         B.dmoe_expert_down(dims, hb, dev["w2"], bufs.map, yp, st)
-        if ev is not None:
-            ev[4].record(st)
+        mark(4)
         B.dmoe_padded_scatter(dims, yp, bufs.map, bufs.map.weights, y, st)
-        if ev is not None:
-            ev[5].record(st)
+        mark(5)
+        if train:
+            B.dmoe_bwd_dy_gather(dims, dev["dy"], bufs.map, yp, bs["dy_pad"], grads["dw"], st)
+            mark(6)
+            B.dmoe_bwd_dglu(dims, bs["dy_pad"], dev["w2"], ab, bb, bufs.map, bs["da"], bs["dbm"], st)
+            mark(7)
+            B.dmoe_bwd_wgrad(dims, xp, hb, bs["dy_pad"], bs["da"], bs["dbm"], bufs.map,
+                             grads["dw1"], grads["dw3"], grads["dw2"], st)
+            mark(8)
+            B.dmoe_bwd_dx(dims, bs["da"], bs["dbm"], dev["w1"], dev["w3"], bufs.map, bs["dx_pad"], st)
+            mark(9)
+            B.dmoe_padded_scatter(dims, bs["dx_pad"], bufs.map, None, grads["dx"], st)
+            mark(10)
 
     for _ in range(args.warmup):
         step()
@@ -261,7 +289,7 @@ def run_ours(args, w):
     if status:
         raise RuntimeError(f"device status after warm-up: {B.status_string(status)}")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     time.sleep(0.3 if sampler else 0.0)  # let the sampler start before the timed region
@@ -295,12 +323,24 @@ def run_ours(args, w):
     lg_h = inp["logits"].pin_memory()
     y_h = torch.empty((w.T, w.hidden), dtype=torch.bfloat16).pin_memory()
     x_d, lg_d = torch.empty_like(dev["x"]), torch.empty_like(dev["logits"])
+    if train:
+        dy_h = inp["dy"].pin_memory()
+        dx_h = torch.empty_like(y_h).pin_memory()
+        dy_d = torch.empty_like(dev["dy"])
 
     def e2e_step():
         x_d.copy_(x_h, non_blocking=True)
         lg_d.copy_(lg_h, non_blocking=True)
         B.dmoe_sparse_map(dims, lg_d, bufs.map, bufs.ws_map, st)
-        B.dmoe_forward(dims, x_d, dev["w1"], dev["w3"], dev["w2"], bufs.map, y, None, bufs.ws_fwd, st)
+        if train:
+            dy_d.copy_(dy_h, non_blocking=True)
+            B.dmoe_forward(dims, x_d, dev["w1"], dev["w3"], dev["w2"], bufs.map, y, bufs.saved, None, st)
+            B.dmoe_backward(dims, dy_d, dev["w1"], dev["w3"], dev["w2"], bufs.map, bufs.saved,
+                            grads["dx"], grads["dw1"], grads["dw3"], grads["dw2"], grads["dw"],
+                            bufs.ws_bwd, st)
+            dx_h.copy_(grads["dx"], non_blocking=True)
+        else:
+            B.dmoe_forward(dims, x_d, dev["w1"], dev["w3"], dev["w2"], bufs.map, y, None, bufs.ws_fwd, st)
         y_h.copy_(y, non_blocking=True)
 
     for _ in range(max(3, args.warmup)):
@@ -318,8 +358,8 @@ def run_ours(args, w):
     if world > 1:
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
     e2e_value = world * w.T * args.steps / (float(te.item()) / 1e3)
-    h2d = x_h.numel() * 2 + lg_h.numel() * 2
-    d2h = y_h.numel() * 2
+    h2d = x_h.numel() * 2 + lg_h.numel() * 2 + (dy_h.numel() * 2 if train else 0)
+    d2h = y_h.numel() * 2 + (dx_h.numel() * 2 if train else 0)
 
     # parity spot check of the timed output against the oracle is done by the tests; here we
     # only confirm the device status stayed clean.
@@ -338,28 +378,31 @@ def run_ours(args, w):
     P = nb * 128
     N = w.entries
     pad_frac = (P - N) / P
-    useful = w.useful_flops(backward=False)
-    glu_flops = 4 * N * w.hidden * w.ffn
-    down_flops = 2 * N * w.hidden * w.ffn
+    useful = w.useful_flops()
+    nhf = N * w.hidden * w.ffn
+    flops = dict(glu_gemm=4 * nhf, down_gemm=2 * nhf, dglu_gemm=2 * nhf, dx_gemm=4 * nhf,
+                 wgrad_gemm=6 * nhf)
+    byts = dict(
+        map=2 * w.T * w.E + 8 * w.T * w.top_k + 12 * N,
+        gather=2 * w.T * w.hidden + 2 * N * w.hidden,
+        scatter=2 * N * w.hidden + 8 * N + 4 * N + 2 * w.T * w.hidden,
+        dy_gather=2 * w.T * w.hidden + 4 * N * w.hidden + 12 * N,
+        dx_scatter=2 * N * w.hidden + 4 * N + 2 * w.T * w.hidden)
     km = {n: statistics.mean(v) for n, v in per_kernel.items()}
-    gather_bytes = 2 * w.T * w.hidden + 2 * N * w.hidden
-    scatter_bytes = 2 * N * w.hidden + 8 * N + 4 * N + 2 * w.T * w.hidden
-    map_bytes = 2 * w.T * w.E + 8 * w.T * w.top_k + 12 * N
-    kernels = {
-        "map": {"ms": km["map"], "GB/s": map_bytes / km["map"] / 1e6},
-        "gather": {"ms": km["gather"], "GB/s": gather_bytes / km["gather"] / 1e6,
-                   "frac_hbm": gather_bytes / km["gather"] / 1e6 / pk["hbm"]},
-        "glu_gemm": {"ms": km["glu_gemm"], "TFLOP/s": glu_flops / km["glu_gemm"] / 1e9,
-                     "frac_bf16": glu_flops / km["glu_gemm"] / 1e9 / pk["bf16_sus"]},
-        "down_gemm": {"ms": km["down_gemm"], "TFLOP/s": down_flops / km["down_gemm"] / 1e9,
-                      "frac_bf16": down_flops / km["down_gemm"] / 1e9 / pk["bf16_sus"]},
-        "scatter": {"ms": km["scatter"], "GB/s": scatter_bytes / km["scatter"] / 1e6,
-                    "frac_hbm": scatter_bytes / km["scatter"] / 1e6 / pk["hbm"]},
-    }
-    dom = "glu_gemm"
-    achieved = glu_flops / km[dom] / 1e9
+    kernels = {}
+    for n in names:
+        ent = {"ms": km[n]}
+        if n in flops:
+            ent["TFLOP/s"] = flops[n] / km[n] / 1e9
+            ent["frac_bf16"] = ent["TFLOP/s"] / pk["bf16_sus"]
+        else:
+            ent["GB/s"] = byts[n] / km[n] / 1e6
+            ent["frac_hbm"] = ent["GB/s"] / pk["hbm"]
+        kernels[n] = ent
+    dom = max(flops.keys() & set(names), key=lambda n: km[n])
+    achieved = flops[dom] / km[dom] / 1e9
     wl_name = f"{w.name} {w.describe()}"
-    traffic = ncu_traffic("glu_gemm", w.name)
+    traffic = ncu_traffic(dom, w.name)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -373,15 +416,15 @@ def run_ours(args, w):
         "useful_tflops": useful / (ms_per_step / 1e3) / 1e12,
         "useful_tflops_frac_bf16": useful / (ms_per_step / 1e3) / 1e12 / pk["bf16_sus"],
         "padded_frac": pad_frac,
-        "roofline": {"bound": "tensor", "kernel": "k_grouped_gemm<GLU>", "achieved": achieved,
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved,
                      "peak": pk["bf16_sus"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_sus"],
-                     "peak_kind": f"{pk['source']} sustained bf16",
+                     "peak_kind": f"{pk['source']} sustained bf16 (burst {pk['bf16']})",
                      "traffic": traffic,
-                     "algorithmic_flops_per_launch": glu_flops},
+                     "algorithmic_flops_per_launch": flops[dom]},
         "kernels": kernels,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 7 * args.steps,
+        "gpu_launches": (7 + (5 if train else 0)) * args.steps,
         "status": status,
     }
     if clocks:
@@ -397,7 +440,8 @@ def run_ours(args, w):
             dt, nt = oracle_sample_run(w, inp32, n_tok, threads)
             line["cpu_baseline"] = {
                 "value": nt / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                "sample": f"routing+map over all {w.T} tokens + forward of {nt} tokens "
+                "sample": f"routing+map over all {w.T} tokens + forward"
+                          f"{' and backward' if w.backward else ''} of {nt} tokens "
                           f"({dt:.1f} s, fp64 accumulation, OpenMP over tokens)"}
         except Exception as ex:  # the baseline is reported, never required
             line["cpu_baseline"] = {"value": None, "unit": "tokens/s", "cores": 0,

@@ -1,35 +1,46 @@
-// gemm.cu -- grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+// gemm.cu -- grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM + TMA),
+// one SM pair per tile (tcgen05.mma.cta_group::2, M = 256, N = 256).
 //
 // The walkthrough ("02 · dropless MoE 与 block-sparse 重构", sections 2-3) views the expert
 // FFN as a block-sparse product in which 128-row block i of the padded activations only
 // meets the ffn/128 column blocks of its own expert.  Here that non-zero set is enumerated
-// directly: a tile is (row block b, output column tile n) and its B operand is the weight
-// slab of expert block_expert[b].  The tile list is read on the device from num_blocks, so no
-// host synchronisation is needed and no tile past the real padded size is ever issued.  The
-// backward's weight gradients (section 4.2's role swap, section 4.3's transposed topology)
-// are a tile per (expert, output tile) whose K loop walks that expert's row blocks.
+// directly: the unit of work is a pair of consecutive row blocks of one expert (they share the
+// expert's weight slab as the B operand) times an output column tile.  The unit list is built
+// on the device from padded_bins, so no host synchronisation is needed and no tile past the
+// real padded size is ever issued.  The backward's weight gradients (section 4.2's role swap;
+// section 4.3's transposed topology) are a tile per (expert, pair of output row tiles, column
+// tile) whose K loop walks that expert's padded rows.
 //
-// Kernel structure (one persistent CTA per SM, 192 threads):
-//   warp 0      TMA producer: A tile (128 x 64 bf16) and B tile (256 x 64 bf16) per stage,
-//               4-stage ring, 128-byte swizzle, completion on an mbarrier (expect-tx).
-//   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma (M=128, N=256,
-//               K=16; bf16 in, fp32 accumulate) and tcgen05.commit to release smem stages and
-//               to hand a finished accumulator to the epilogue.
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator (each warp its 32-lane TMEM
-//               sub-partition), fused element-wise work, bf16 stores.
+// Kernel structure (clusters of 2 CTAs on an SM pair, 192 threads each, persistent):
+//   warp 0      TMA producer (both CTAs): this CTA's 128 rows of A and its half (128 rows)
+//               of B per stage, 5-stage ring of 32 KB, 128-byte swizzle; every load completes
+//               on the pair leader's mbarrier (expect-tx of both halves).
+//   warp 1      allocates 512 TMEM columns in both CTAs; one thread of the leader issues
+//               tcgen05.mma.cta_group::2 (bf16 in, fp32 accumulate), which reads both CTAs'
+//               shared memory and writes each CTA's 128 accumulator rows into its own TMEM,
+//               and tcgen05.commit (multicast to both CTAs) to free stages and hand over
+//               accumulators.
+//   warps 2-5   epilogue (both CTAs): tcgen05.ld of the accumulator (each warp its 32-lane
+//               TMEM sub-partition), fused element-wise work, results staged in 128-byte-
+//               swizzled shared memory (32 rows x 128 B per box) and written with TMA
+//               bulk-tensor stores, double-buffered per warp.
 // Two accumulators (2 x 256 columns) let the epilogue of tile i overlap the MMAs of i+1.
+// An expert with an odd number of row blocks ends with a unit whose second CTA reads zero
+// rows (TMA fill past the last padded row) and stores nothing.
 //
 // Modes (operand majors: K = K-major, MN = M/N-major; weights are (out, in) = [E, f, h] for
 // W1/W3 and [E, h, f] for W2):
-//   GLU   A = X_pad (K)      B = [W1_e ; W3_e] rows of 128 f-columns each (K)
+//   GLU   A = X_pad (K)      B = W1_e rows (leader) / W3_e rows (peer), 128 f-columns each (K)
 //         out H = bf16(silu(gate) * up); optionally bf16(gate), bf16(up) for the backward
 //   DOWN  A = H (K)          B = W2_e (K)                 out Y_pad
 //   DGLU  A = dY_pad (K)     B = W2_e^T (MN)              dH; epilogue recomputes the
 //         activation from the saved A, Bm: dA = dH*Bm*s*(1+A(1-s)), dBm = dH*A*s, s = sigmoid(A)
 //   DX    A = dA then dBm (K), B = W1_e then W3_e (MN), one accumulator over both K passes
-//   WGRAD per expert e and output tile: dW1_e = dA^T X_pad, dW3_e = dBm^T X_pad,
-//         dW2_e = dY^T H, K = the expert's padded rows (both operands MN-major); fp32
-//         outputs; experts without rows get exact zeros.
+//   WGRAD dW1_e = dA^T X_pad, dW3_e = dBm^T X_pad, dW2_e = dY^T H over the expert's padded
+//         rows (both operands MN-major); fp32 outputs; experts without rows get exact zeros.
+//
+// Every mbarrier wait is bounded; on expiry the kernel sets DMOE_STATUS_TIMEOUT, raises an
+// abort flag for the other roles of its CTA, drains what it issued and returns.
 #include <string.h>
 
 #include <mutex>
@@ -39,20 +50,23 @@
 
 namespace dmoe {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int BK = 64;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;  // 16 KB
-constexpr int B_BYTES = BN * BK * 2;  // 32 KB
+constexpr int BM = 128;  // rows of A per CTA (= one padded row block)
+constexpr int BN = 256;  // output columns per tile
+constexpr int BK = 64;   // K per pipeline stage (one 128-byte swizzle row of bf16)
+constexpr int STAGES = 5;
+constexpr int A_BYTES = BM * BK * 2;        // 16 KB: this CTA's 128 rows of A
+constexpr int B_BYTES = (BN / 2) * BK * 2;  // 16 KB: this CTA's half of B
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int CHUNK_BYTES = 64 * BK * 2;  // one 64 x 64 MN-major box: 8 KB
+constexpr int CHUNK_BYTES = 64 * BK * 2;    // one 64 x 64 MN-major box: 8 KB
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = 256;
 constexpr int GEMM_THREADS = 192;
-constexpr int EPI_THREADS = 128;
-constexpr int RASTER_GROUP = 16;  // row blocks per raster group
-constexpr size_t GEMM_SMEM = (size_t)STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int EPI_WARPS = 4;
+constexpr int EPI_THREADS = 32 * EPI_WARPS;
+constexpr int BOX_BYTES = 32 * 128;  // one result box: 32 rows x 128 B
+constexpr int OUT_BYTES = EPI_WARPS * 2 * BOX_BYTES;
+constexpr size_t SMEM_BYTES = 1024 /*align*/ + (size_t)STAGES * STAGE_BYTES + OUT_BYTES +
+                              256 /*barriers*/ + sizeof(int) * (DMOE_MAX_EXPERTS + 1);
 
 enum GemmMode { MODE_GLU = 0, MODE_DOWN = 1, MODE_DGLU = 2, MODE_DX = 3, MODE_WGRAD = 4 };
 
@@ -63,248 +77,282 @@ struct ModeTraits {
 };
 
 struct GemmParams {
-  CUtensorMap tm[5];
-  const int32_t *num_blocks;
-  const int32_t *block_expert;
+  CUtensorMap tm[5];   // operand tensor maps (loads)
+  CUtensorMap tmo[3];  // result tensor maps (stores)
   const int32_t *padded_bins;
   int E, h, f;
-  int n_tiles;  // row-block modes: column tiles per row block
-  int k_iters;  // row-block modes: 64-wide K steps per tile
-  __nv_bfloat16 *out0, *out1, *out2;
-  float *fout0, *fout1, *fout2;  // WGRAD: fp32 dW1, dW3, dW2
-  const __nv_bfloat16 *in0, *in1;
+  int n_tiles;   // row-block modes: column tiles per unit
+  int k_iters;   // row-block modes: 64-wide K steps per tile
+  int nblk_cap;  // P_max / 128: rows at or past nblk_cap * 128 read as zeros
+  int group;     // row-block modes: units per raster chunk
+  int outs;      // GLU: 1 (H) or 3 (H, A, Bm)
+  const __nv_bfloat16 *in0, *in1;  // DGLU: saved A, Bm
   int32_t *status;
 };
 
 struct Tile {
-  int b, n, e, m, which, row0, kit;
+  int e, n, m, which, row0, kit;
+  bool dummy;  // this CTA's half of the unit has no rows: load zeros, store nothing
 };
 
-// Row-block modes: tile t -> (row block b, column tile n).  Groups of RASTER_GROUP row blocks;
-// inside a group the row block varies fastest, so CTAs running together share B tiles.
-__device__ __forceinline__ void rowblock_coords(int t, int nb, int n_tiles, int &b, int &n) {
-  const int per_group = RASTER_GROUP * n_tiles;
-  const int g = t / per_group;
-  const int local = t - g * per_group;
-  const int gb0 = g * RASTER_GROUP;
-  const int gsz = min(RASTER_GROUP, nb - gb0);
-  n = local / gsz;
-  b = gb0 + (local - n * gsz);
-}
-
-// Weight-gradient tiles per expert: dW1 and dW3 are [f, h] (f/128 x ceil(h/256) tiles), dW2 is
-// [h, f] (h/128 x ceil(f/256) tiles).
-__device__ __forceinline__ int wg_tiles13(const GemmParams &p) {
-  return (p.f / BM) * ((p.h + BN - 1) / BN);
-}
-__device__ __forceinline__ int wg_tiles2(const GemmParams &p) {
-  return (p.h / BM) * ((p.f + BN - 1) / BN);
-}
-
+// Pair tile t -> expert, column tile, this CTA's rows.
 template <int MODE>
-__device__ __forceinline__ int total_tiles(const GemmParams &p, int nb) {
-  if (MODE == MODE_WGRAD) return p.E * (2 * wg_tiles13(p) + wg_tiles2(p));
-  return nb * p.n_tiles;
-}
-
-template <int MODE>
-__device__ __forceinline__ Tile decode(const GemmParams &p, int t, int nb) {
+__device__ __forceinline__ Tile decode(const GemmParams &p, int t, const int *ustart,
+                                       uint32_t rank) {
   Tile tl;
+  tl.which = 0;
+  tl.m = 0;
   if (MODE == MODE_WGRAD) {
-    const int t13 = wg_tiles13(p), t2 = wg_tiles2(p);
-    const int tpe = 2 * t13 + t2;
+    const int mt13 = p.f / BM, mt2 = p.h / BM;
+    const int mp13 = (mt13 + 1) / 2, mp2 = (mt2 + 1) / 2;
+    const int nt13 = (p.h + BN - 1) / BN, nt2 = (p.f + BN - 1) / BN;
+    const int tpe = 2 * mp13 * nt13 + mp2 * nt2;
     tl.e = t / tpe;
     int r = t - tl.e * tpe;
-    int ncols;
-    if (r < 2 * t13) {
-      tl.which = r / t13;
-      r -= tl.which * t13;
-      ncols = (p.h + BN - 1) / BN;
+    int ncols, mtiles;
+    if (r < 2 * mp13 * nt13) {
+      tl.which = r / (mp13 * nt13);
+      r -= tl.which * mp13 * nt13;
+      ncols = nt13;
+      mtiles = mt13;
     } else {
       tl.which = 2;
-      r -= 2 * t13;
-      ncols = (p.f + BN - 1) / BN;
+      r -= 2 * mp13 * nt13;
+      ncols = nt2;
+      mtiles = mt2;
     }
-    tl.m = r / ncols;
-    tl.n = r - tl.m * ncols;
+    const int mp = r / ncols;
+    tl.n = r - mp * ncols;
+    tl.m = 2 * mp + (int)rank;
+    tl.dummy = tl.m >= mtiles;  // its A boxes start past the matrix: zeros
     const int start = (tl.e > 0) ? p.padded_bins[tl.e - 1] : 0;
-    const int end = p.padded_bins[tl.e];
     tl.row0 = start;
-    tl.kit = (end - start) / BK;
-    tl.b = 0;
-  } else {
-    rowblock_coords(t, nb, p.n_tiles, tl.b, tl.n);
-    tl.e = p.block_expert[tl.b];
-    tl.m = 0;
-    tl.which = 0;
-    tl.row0 = tl.b * BM;
-    tl.kit = p.k_iters;
+    tl.kit = (p.padded_bins[tl.e] - start) / BK;
+    return tl;
   }
+  const int vu = t / p.n_tiles;  // units partition the tile list in order
+  int lo = 0, hi = p.E - 1;      // the expert whose unit range holds vu
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (ustart[mid] <= vu)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  const int e = lo;
+  const int units = ustart[e + 1] - ustart[e];
+  const int c0 = ((vu - ustart[e]) / p.group) * p.group;  // raster chunk inside the expert
+  const int cs = min(p.group, units - c0);
+  const int lt = t - (ustart[e] + c0) * p.n_tiles;
+  tl.n = lt / cs;  // the unit varies fastest: concurrent pairs share B
+  const int unit = c0 + (lt - tl.n * cs);
+  const int first = ((e > 0) ? p.padded_bins[e - 1] : 0) / BM;
+  const int end = p.padded_bins[e] / BM;
+  const int b = first + 2 * unit + (int)rank;
+  tl.e = e;
+  tl.dummy = b >= end;
+  tl.row0 = tl.dummy ? p.nblk_cap * BM : b * BM;  // a dummy half reads rows past P_max: zeros
+  tl.kit = p.k_iters;
   return tl;
 }
 
-// Issue the TMA loads of K step kb of tile tl into stage buffers sa (A) and sb (B).
 template <int MODE>
-__device__ __forceinline__ void load_stage(const GemmParams &p, const Tile &tl, int kb, uint8_t *sa,
-                                           uint8_t *sb, uint64_t *bar) {
+__device__ __forceinline__ void load_stage(const GemmParams &p, const Tile &tl, int kb,
+                                           uint32_t rank, uint8_t *sa, uint8_t *sb,
+                                           uint32_t bar) {
   if (MODE == MODE_GLU) {
-    const int brow = tl.e * p.f + tl.n * (BN / 2);
-    tma_load_2d(sa, &p.tm[0], bar, kb * BK, tl.row0);
-    tma_load_2d(sb, &p.tm[1], bar, kb * BK, brow);
-    tma_load_2d(sb + B_BYTES / 2, &p.tm[2], bar, kb * BK, brow);
+    tma_load_2d_pair(sa, &p.tm[0], bar, kb * BK, tl.row0);
+    tma_load_2d_pair(sb, &p.tm[rank == 0 ? 1 : 2], bar, kb * BK, tl.e * p.f + tl.n * (BN / 2));
   } else if (MODE == MODE_DOWN) {
-    tma_load_2d(sa, &p.tm[0], bar, kb * BK, tl.row0);
-    tma_load_2d(sb, &p.tm[1], bar, kb * BK, tl.e * p.h + tl.n * BN);
+    tma_load_2d_pair(sa, &p.tm[0], bar, kb * BK, tl.row0);
+    tma_load_2d_pair(sb, &p.tm[1], bar, kb * BK, tl.e * p.h + tl.n * BN + (int)rank * (BN / 2));
   } else if (MODE == MODE_DGLU) {
-    tma_load_2d(sa, &p.tm[0], bar, kb * BK, tl.row0);
+    tma_load_2d_pair(sa, &p.tm[0], bar, kb * BK, tl.row0);
 #pragma unroll
-    for (int c = 0; c < BN / 64; ++c)
-      tma_load_2d(sb + c * CHUNK_BYTES, &p.tm[1], bar, tl.n * BN + c * 64, tl.e * p.h + kb * BK);
+    for (int c = 0; c < 2; ++c)
+      tma_load_2d_pair(sb + c * CHUNK_BYTES, &p.tm[1], bar, tl.n * BN + (2 * (int)rank + c) * 64,
+                       tl.e * p.h + kb * BK);
   } else if (MODE == MODE_DX) {
     const int kf = p.f / BK;
     const int pass = (kb < kf) ? 0 : 1;
     const int kk = kb - pass * kf;
-    tma_load_2d(sa, &p.tm[pass], bar, kk * BK, tl.row0);
+    tma_load_2d_pair(sa, &p.tm[pass], bar, kk * BK, tl.row0);
 #pragma unroll
-    for (int c = 0; c < BN / 64; ++c)
-      tma_load_2d(sb + c * CHUNK_BYTES, &p.tm[2 + pass], bar, tl.n * BN + c * 64,
-                  tl.e * p.f + kk * BK);
+    for (int c = 0; c < 2; ++c)
+      tma_load_2d_pair(sb + c * CHUNK_BYTES, &p.tm[2 + pass], bar,
+                       tl.n * BN + (2 * (int)rank + c) * 64, tl.e * p.f + kk * BK);
   } else {  // MODE_WGRAD
-    const int ya = tl.row0 + kb * BK;
-    const CUtensorMap *ta = &p.tm[tl.which];             // dA, dBm, dY_pad
+    const int y = tl.row0 + kb * BK;
+    const CUtensorMap *ta = &p.tm[tl.which];               // dA, dBm, dY_pad
     const CUtensorMap *tb = &p.tm[tl.which == 2 ? 4 : 3];  // X_pad, X_pad, H
 #pragma unroll
-    for (int c = 0; c < BM / 64; ++c) tma_load_2d(sa + c * CHUNK_BYTES, ta, bar, tl.m * BM + c * 64, ya);
+    for (int c = 0; c < 2; ++c) tma_load_2d_pair(sa + c * CHUNK_BYTES, ta, bar, tl.m * BM + c * 64, y);
 #pragma unroll
-    for (int c = 0; c < BN / 64; ++c) tma_load_2d(sb + c * CHUNK_BYTES, tb, bar, tl.n * BN + c * 64, ya);
+    for (int c = 0; c < 2; ++c)
+      tma_load_2d_pair(sb + c * CHUNK_BYTES, tb, bar, tl.n * BN + (2 * (int)rank + c) * 64, y);
   }
 }
 
-__device__ __forceinline__ void store16_bf16(__nv_bfloat16 *dst, const float *v) {
-  uint32_t p[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) p[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-  st_global_v4(dst, p[0], p[1], p[2], p[3]);
-  st_global_v4(dst + 8, p[4], p[5], p[6], p[7]);
-}
+// ---- epilogue ---------------------------------------------------------------------------------
 
-__device__ __forceinline__ void store16_f32(float *dst, const float *v) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    st_global_v4(dst + 4 * i, __float_as_uint(v[4 * i]), __float_as_uint(v[4 * i + 1]),
-                 __float_as_uint(v[4 * i + 2]), __float_as_uint(v[4 * i + 3]));
-}
+// Per-warp result staging: two 4 KB buffers, each one box of 32 rows x 128 B in the 128-byte
+// swizzled layout that a SWIZZLE_128B tensor map expects (16-byte chunk c of row r sits at
+// chunk position c ^ (r & 7)).  Lane l writes row l; lane 0 issues the TMA store.
+struct Stager {
+  uint32_t bufs;  // shared address of buffer 0 (buffer 1 follows)
+  int cur;
+  int lane;
 
-__device__ __forceinline__ void load16_bf16(const __nv_bfloat16 *src, float *v) {
-  const uint4 *s = reinterpret_cast<const uint4 *>(src);
-  const uint4 q0 = s[0], q1 = s[1];
-  const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+  __device__ __forceinline__ void emit(const CUtensorMap *map, const uint32_t (&w)[32], int x,
+                                       int y) {
+    const uint32_t buf = bufs + (uint32_t)(cur * BOX_BYTES);
+    if (lane == 0) bulk_wait_read<1>();  // the store that last used this buffer has read it
+    __syncwarp();
+    const uint32_t row = buf + (uint32_t)(lane * 128);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    v[2 * i] = bf16_lo(w[i]);
-    v[2 * i + 1] = bf16_hi(w[i]);
+    for (int c = 0; c < 8; ++c)
+      st_shared_v4(row + (uint32_t)((c ^ (lane & 7)) << 4), w[4 * c], w[4 * c + 1], w[4 * c + 2],
+                   w[4 * c + 3]);
+    fence_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d_u32(map, buf, x, y);
+      bulk_commit();
+    }
+    cur ^= 1;
+  }
+};
+
+__device__ __forceinline__ void pack_bf16_row(const uint32_t (&lo)[32], const uint32_t (&hi)[32],
+                                              uint32_t (&w)[32]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    w[i] = pack_bf16x2(__uint_as_float(lo[2 * i]), __uint_as_float(lo[2 * i + 1]));
+    w[16 + i] = pack_bf16x2(__uint_as_float(hi[2 * i]), __uint_as_float(hi[2 * i + 1]));
   }
 }
 
-// Epilogue of one tile for the thread that owns accumulator row `r` (TMEM lane).
+// Epilogue of one tile for the warp owning TMEM sub-partition `sub` (rows sub*32 .. +31 of
+// this CTA's 128 rows); tb = TMEM address of the warp's lanes at accumulator column 0.
 template <int MODE>
 __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &tl, uint32_t tb,
-                                              int r) {
+                                              int sub, int lane, Stager &st) {
+  const int y0 = tl.row0 + sub * 32;  // first row of this warp's boxes
   if (MODE == MODE_GLU) {
-    const size_t grow = (size_t)tl.row0 + r;
     const int n0 = tl.n * (BN / 2);
-    const size_t off = grow * p.f + n0;
-    for (int c = 0; c < BN / 2; c += 16) {
-      uint32_t g[16], u[16];
-      tmem_ld16(tb + c, g);
-      tmem_ld16(tb + BN / 2 + c, u);
+#pragma unroll 1
+    for (int c = 0; c < BN / 2; c += 64) {  // one 64-column box of H (and of A, Bm)
+      uint32_t g0[32], g1[32], u0[32], u1[32], w[32];
+      tmem_ld32(tb + c, g0);
+      tmem_ld32(tb + c + 32, g1);
+      tmem_ld32(tb + BN / 2 + c, u0);
+      tmem_ld32(tb + BN / 2 + c + 32, u1);
       tmem_ld_wait();
-      float hv[16], gv[16], uv[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        gv[i] = __uint_as_float(g[i]);
-        uv[i] = __uint_as_float(u[i]);
-        hv[i] = silu_f(gv[i]) * uv[i];
+        w[i] = pack_bf16x2(silu_f(__uint_as_float(g0[2 * i])) * __uint_as_float(u0[2 * i]),
+                           silu_f(__uint_as_float(g0[2 * i + 1])) * __uint_as_float(u0[2 * i + 1]));
+        w[16 + i] = pack_bf16x2(silu_f(__uint_as_float(g1[2 * i])) * __uint_as_float(u1[2 * i]),
+                                silu_f(__uint_as_float(g1[2 * i + 1])) * __uint_as_float(u1[2 * i + 1]));
       }
-      store16_bf16(p.out0 + off + c, hv);
-      if (p.out1) store16_bf16(p.out1 + off + c, gv);
-      if (p.out2) store16_bf16(p.out2 + off + c, uv);
+      st.emit(&p.tmo[0], w, n0 + c, y0);
+      if (p.outs > 1) {
+        pack_bf16_row(g0, g1, w);
+        st.emit(&p.tmo[1], w, n0 + c, y0);
+        pack_bf16_row(u0, u1, w);
+        st.emit(&p.tmo[2], w, n0 + c, y0);
+      }
     }
   } else if (MODE == MODE_DOWN || MODE == MODE_DX) {
-    const size_t grow = (size_t)tl.row0 + r;
     const int n0 = tl.n * BN;
-    for (int c = 0; c < BN; c += 16) {
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 64) {
       if (n0 + c >= p.h) break;  // uniform across the warp
-      uint32_t v[16];
-      tmem_ld16(tb + c, v);
+      uint32_t v0[32], v1[32], w[32];
+      tmem_ld32(tb + c, v0);
+      tmem_ld32(tb + c + 32, v1);
       tmem_ld_wait();
-      float fv[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) fv[i] = __uint_as_float(v[i]);
-      store16_bf16(p.out0 + grow * p.h + n0 + c, fv);
+      pack_bf16_row(v0, v1, w);
+      st.emit(&p.tmo[0], w, n0 + c, y0);
     }
   } else if (MODE == MODE_DGLU) {
-    const size_t grow = (size_t)tl.row0 + r;
     const int n0 = tl.n * BN;
-    for (int c = 0; c < BN; c += 16) {
+    const size_t grow = (size_t)y0 + lane;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 64) {
       if (n0 + c >= p.f) break;
-      uint32_t v[16];
-      tmem_ld16(tb + c, v);
-      const size_t off = grow * p.f + n0 + c;
-      float a[16], bm[16], da[16], db[16];
-      load16_bf16(p.in0 + off, a);
-      load16_bf16(p.in1 + off, bm);
+      uint32_t v0[32], v1[32], wa[32], wb[32];
+      uint4 qa[8], qb[8];
+      tmem_ld32(tb + c, v0);
+      tmem_ld32(tb + c + 32, v1);
+      const uint4 *sa = reinterpret_cast<const uint4 *>(p.in0 + grow * p.f + n0 + c);
+      const uint4 *sb = reinterpret_cast<const uint4 *>(p.in1 + grow * p.f + n0 + c);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        qa[i] = __ldg(sa + i);
+        qb[i] = __ldg(sb + i);
+      }
       tmem_ld_wait();
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float dh = __uint_as_float(v[i]);
-        const float s = 1.0f / (1.0f + __expf(-a[i]));
-        da[i] = dh * bm[i] * s * (1.0f + a[i] * (1.0f - s));
-        db[i] = dh * a[i] * s;
+      for (int i = 0; i < 32; ++i) {  // bf16 pairs 2i, 2i+1 of this 64-column chunk
+        const uint32_t aw = reinterpret_cast<const uint32_t *>(qa)[i];
+        const uint32_t bw = reinterpret_cast<const uint32_t *>(qb)[i];
+        const float dh0 = __uint_as_float(i < 16 ? v0[2 * i] : v1[2 * i - 32]);
+        const float dh1 = __uint_as_float(i < 16 ? v0[2 * i + 1] : v1[2 * i - 31]);
+        const float a0 = bf16_lo(aw), a1 = bf16_hi(aw), b0 = bf16_lo(bw), b1 = bf16_hi(bw);
+        const float s0 = 1.0f / (1.0f + __expf(-a0)), s1 = 1.0f / (1.0f + __expf(-a1));
+        wa[i] = pack_bf16x2(dh0 * b0 * s0 * (1.0f + a0 * (1.0f - s0)),
+                            dh1 * b1 * s1 * (1.0f + a1 * (1.0f - s1)));
+        wb[i] = pack_bf16x2(dh0 * a0 * s0, dh1 * a1 * s1);
       }
-      store16_bf16(p.out0 + off, da);
-      store16_bf16(p.out1 + off, db);
+      st.emit(&p.tmo[0], wa, n0 + c, y0);
+      st.emit(&p.tmo[1], wb, n0 + c, y0);
     }
-  } else {  // MODE_WGRAD
+  } else {  // MODE_WGRAD: fp32 results, boxes of 32 columns
     const int rows = (tl.which == 2) ? p.h : p.f;
     const int cols = (tl.which == 2) ? p.f : p.h;
-    float *base = (tl.which == 0) ? p.fout0 : (tl.which == 1) ? p.fout1 : p.fout2;
-    float *dst = base + (size_t)tl.e * rows * cols + (size_t)(tl.m * BM + r) * cols;
+    const int yw = tl.e * rows + tl.m * BM + sub * 32;
     const int n0 = tl.n * BN;
-    for (int c = 0; c < BN; c += 16) {
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
       if (n0 + c >= cols) break;
-      float fv[16];
+      uint32_t v[32];
       if (tl.kit > 0) {
-        uint32_t v[16];
-        tmem_ld16(tb + c, v);
+        tmem_ld32(tb + c, v);
         tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) fv[i] = __uint_as_float(v[i]);
       } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) fv[i] = 0.0f;  // expert without rows: exact zeros
+        for (int i = 0; i < 32; ++i) v[i] = 0u;  // expert without rows: exact zeros
       }
-      store16_f32(dst + n0 + c, fv);
+      st.emit(&p.tmo[tl.which], v, n0 + c, yw);
     }
   }
 }
 
+// ---- the kernel -------------------------------------------------------------------------------
+
 template <int MODE>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     k_grouped_gemm(const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base_u32 = smem_u32(smem_raw);
   uint8_t *tiles = smem_raw + ((1024u - (base_u32 & 1023u)) & 1023u);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(tiles + STAGES * STAGE_BYTES);
-  uint64_t *full = bars;                     // [STAGES] TMA landed
-  uint64_t *empty = bars + STAGES;           // [STAGES] MMAs done reading
-  uint64_t *tfull = bars + 2 * STAGES;       // [2] accumulator ready
-  uint64_t *tempty = bars + 2 * STAGES + 2;  // [2] accumulator drained
-  uint64_t *drain = bars + 2 * STAGES + 4;   // teardown: all MMAs finished
+  uint8_t *outbuf = tiles + STAGES * STAGE_BYTES;  // 1024-aligned
+  uint64_t *bars = reinterpret_cast<uint64_t *>(outbuf + OUT_BYTES);
+  uint64_t *full = bars;                       // [STAGES] leader: both halves landed
+  uint64_t *empty = bars + STAGES;             // [STAGES] MMAs done reading the stage
+  uint64_t *tfull = bars + 2 * STAGES;         // [2] accumulator ready
+  uint64_t *tempty = bars + 2 * STAGES + 2;    // [2] leader: accumulator drained (256 arrivals)
+  uint64_t *drain = bars + 2 * STAGES + 4;     // leader: all MMAs finished
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  int *ustart = reinterpret_cast<int *>(outbuf + OUT_BYTES + 256);  // [E + 1]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -312,7 +360,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], EPI_THREADS);
+      mbar_init(&tempty[a], 2 * EPI_THREADS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -320,36 +368,63 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
     for (int i = 0; i < 5; ++i) prefetch_tmap(&p.tm[i]);
   }
-  if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
+  if (MODE != MODE_WGRAD) {
+    // units (pairs of row blocks) per expert -> exclusive prefix ustart[0..E]
+    for (int e = threadIdx.x; e < p.E; e += GEMM_THREADS) {
+      const int blocks = (p.padded_bins[e] - ((e > 0) ? p.padded_bins[e - 1] : 0)) / BM;
+      ustart[e + 1] = (blocks + 1) / 2;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      int carry = 0;
+      for (int base = 0; base < p.E; base += 32) {
+        const int e = base + lane;
+        int v = (e < p.E) ? ustart[e + 1] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int nv = __shfl_up_sync(0xFFFFFFFFu, v, off);
+          if (lane >= off) v += nv;
+        }
+        if (e < p.E) ustart[e + 1] = carry + v;
+        carry += __shfl_sync(0xFFFFFFFFu, v, 31);
+      }
+      if (lane == 0) ustart[0] = 0;
+    }
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, TMEM_COLS);
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // the peer's barriers are initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int nb = (MODE == MODE_WGRAD) ? 0 : *p.num_blocks;
-  const int total = total_tiles<MODE>(p, nb);
+  int total;
+  if (MODE == MODE_WGRAD) {
+    const int mp13 = (p.f / BM + 1) / 2, mp2 = (p.h / BM + 1) / 2;
+    total = p.E * (2 * mp13 * ((p.h + BN - 1) / BN) + mp2 * ((p.f + BN - 1) / BN));
+  } else {
+    total = ustart[p.E] * p.n_tiles;
+  }
+  const uint32_t leader_full0 = mapa_shared(smem_u32(&full[0]), 0);
+  const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
 
   if (warp == 0 && lane == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (both CTAs) ----------------
     int stage = 0;
     uint32_t phase = 0;
     long long issued = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      const Tile tl = decode<MODE>(p, t, nb);
-      if (MODE != MODE_WGRAD && tl.e < 0) {  // cannot happen with a map from dmoe_sparse_map
-        set_status(p.status, DMOE_STATUS_TIMEOUT);
-        *abort_flag = 1;
-        break;
-      }
+    for (int t = cluster; t < total; t += nclusters) {
+      const Tile tl = decode<MODE>(p, t, ustart, rank);
       bool ok = true;
       for (int kb = 0; kb < tl.kit; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, p.status, abort_flag)) {
           ok = false;
           break;
         }
+        if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
         uint8_t *sa = tiles + stage * STAGE_BYTES;
-        mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-        load_stage<MODE>(p, tl, kb, sa, sa + A_BYTES, &full[stage]);
+        load_stage<MODE>(p, tl, kb, rank, sa, sa + A_BYTES,
+                         leader_full0 + (uint32_t)(stage * sizeof(uint64_t)));
         ++issued;
         if (++stage == STAGES) {
           stage = 0;
@@ -358,19 +433,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       }
       if (!ok) break;
     }
-    // Teardown: every issued copy must have landed before the CTA may exit.
-    for (long long i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
-      mbar_wait_plain(&full[i % STAGES], (uint32_t)((i / STAGES) & 1));
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer ----------------
+    if (leader)  // every issued copy (of both CTAs) has landed before the pair may exit
+      for (long long i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+        mbar_wait_plain(&full[i % STAGES], (uint32_t)((i / STAGES) & 1));
+  } else if (warp == 1 && lane == 0 && leader) {
+    // ---------------- MMA issuer (leader only) ----------------
     constexpr uint32_t idesc =
-        idesc_bf16_f32(BM, BN, ModeTraits<MODE>::a_mn, ModeTraits<MODE>::b_mn);
+        idesc_bf16_f32(2 * BM, BN, ModeTraits<MODE>::a_mn, ModeTraits<MODE>::b_mn);
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      const Tile tl = decode<MODE>(p, t, nb);
+    for (int t = cluster; t < total; t += nclusters) {
+      const Tile tl = decode<MODE>(p, t, ustart, rank);
       if (tl.kit == 0) continue;  // weight gradient of an expert without rows: no MMA
       if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.status, abort_flag)) break;
       tc_fence_after();
@@ -392,49 +467,54 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const uint64_t bd = ModeTraits<MODE>::b_mn
                                   ? sdesc_mnmajor_sw128(b_addr + kk * 2048, CHUNK_BYTES)
                                   : sdesc_kmajor_sw128(b_addr + kk * 32);
-          tc_mma(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          tc_mma_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
         }
-        tc_commit(&empty[stage]);
+        tc_commit_pair_mc(&empty[stage]);
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
         }
       }
       if (!ok) break;
-      tc_commit(&tfull[acc]);
+      tc_commit_pair_mc(&tfull[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
-    // Teardown: wait until every MMA issued by this thread has completed.
-    tc_commit(drain);
+    tc_commit_pair(drain);
     mbar_wait_plain(drain, 0);
   } else if (warp >= 2) {
-    // ---------------- epilogue ----------------
+    // ---------------- epilogue (both CTAs) ----------------
     const int sub = warp & 3;  // TMEM sub-partition this warp may read
-    const int r = sub * 32 + lane;
+    Stager st;
+    st.bufs = smem_u32(outbuf) + (uint32_t)((warp - 2) * 2 * BOX_BYTES);
+    st.cur = 0;
+    st.lane = lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      const Tile tl = decode<MODE>(p, t, nb);
+    for (int t = cluster; t < total; t += nclusters) {
+      const Tile tl = decode<MODE>(p, t, ustart, rank);
       if (tl.kit == 0) {  // no accumulator involved
-        epilogue_tile<MODE>(p, tl, 0u, r);
+        if (!tl.dummy) epilogue_tile<MODE>(p, tl, 0u, sub, lane, st);
         continue;
       }
       if (!mbar_wait(&tfull[acc], acc_phase, p.status, abort_flag)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * ACC_COLS);
-      epilogue_tile<MODE>(p, tl, tb, r);
+      if (!tl.dummy) epilogue_tile<MODE>(p, tl, tb, sub, lane, st);
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      mbar_arrive_cluster(leader_tempty0 + (uint32_t)(acc * sizeof(uint64_t)));
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    if (lane == 0) bulk_wait_all();  // results written before the CTA exits
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // the leader's MMAs into this CTA's TMEM are done; no more remote traffic
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
@@ -459,18 +539,19 @@ static EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// Row-major bf16 matrix [rows, cols] as a 2D tensor; box = box_rows x 64 columns, 128-byte
-// swizzle (64 bf16 per box row = exactly one swizzle row).
+// Row-major matrix [rows, cols] of bf16 (esize 2) or fp32 (esize 4) as a 2D tensor; box =
+// box_rows x (128 / esize) columns, 128-byte swizzle (one box row = one swizzle row).
 static bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols,
-                      uint32_t box_rows) {
+                      uint32_t box_rows, int esize = 2) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {64u, box_rows};
+  cuuint64_t strides[1] = {cols * (uint64_t)esize};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / esize), box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = enc(m, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                   2, const_cast<void *>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -485,119 +566,141 @@ int device_sm_count() {
   return cached;
 }
 
+// Raster chunk: as many units (2 row blocks) as keep their A tiles (2 x 128 x K bf16 per
+// unit) within about 40 MB of L2, 1..64.
+static int raster_units(int K) {
+  const long long per_unit = 2LL * BM * K * 2;
+  long long g = (40LL << 20) / per_unit;
+  if (g < 1) g = 1;
+  if (g > 64) g = 64;
+  return (int)g;
+}
+
 template <int MODE>
 static cudaError_t launch_gemm(const GemmParams &p, long long max_tiles, cudaStream_t st) {
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
+  static int max_clusters = 0;
   std::call_once(once, [] {
     attr_err = cudaFuncSetAttribute(k_grouped_gemm<MODE>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GEMM_SMEM);
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (attr_err != cudaSuccess) return;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (device_sm_count() / 2), 1, 1);
+    cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k_grouped_gemm<MODE>, &cfg) != cudaSuccess || n < 1)
+      n = device_sm_count() / 2;
+    max_clusters = n;
   });
   if (attr_err != cudaSuccess) return attr_err;
-  long long grid = device_sm_count();
-  if (max_tiles < grid) grid = max_tiles;
-  if (grid < 1) grid = 1;
-  k_grouped_gemm<MODE><<<(int)grid, GEMM_THREADS, GEMM_SMEM, st>>>(p);
+  long long clusters = max_clusters;
+  if (max_tiles < clusters) clusters = max_tiles;
+  if (clusters < 1) clusters = 1;
+  k_grouped_gemm<MODE><<<(int)(2 * clusters), GEMM_THREADS, SMEM_BYTES, st>>>(p);
   return cudaGetLastError();
 }
 
-static GemmParams base_params(int h, int f, int E, const int32_t *num_blocks,
-                              const int32_t *block_expert, const int32_t *padded_bins,
-                              int32_t *status) {
+static GemmParams base_params(const GemmProblem &g) {
   GemmParams p;
   memset(&p, 0, sizeof(p));
-  p.num_blocks = num_blocks;
-  p.block_expert = block_expert;
-  p.padded_bins = padded_bins;
-  p.E = E;
-  p.h = h;
-  p.f = f;
-  p.status = status;
+  p.padded_bins = g.padded_bins;
+  p.E = g.E;
+  p.h = g.h;
+  p.f = g.f;
+  p.nblk_cap = g.nblk_cap;
+  p.group = 1;
+  p.outs = 1;
+  p.status = g.status;
   return p;
 }
 
-static inline __nv_bfloat16 *bf(void *q) { return static_cast<__nv_bfloat16 *>(q); }
-static inline const __nv_bfloat16 *cbf(const void *q) {
-  return static_cast<const __nv_bfloat16 *>(q);
-}
+static inline long long max_units(const GemmProblem &g) { return (long long)g.nblk_cap / 2 + g.E; }
 
 cudaError_t launch_glu_gemm(const GemmProblem &g, const void *x_pad, const void *w1,
                             const void *w3, void *h_out, void *a_out, void *b_out,
                             cudaStream_t st) {
-  GemmParams p = base_params(g.h, g.f, g.E, g.num_blocks, g.block_expert, g.padded_bins, g.status);
+  GemmParams p = base_params(g);
   const uint64_t P = (uint64_t)g.nblk_cap * BM;
-  if (!make_tmap(&p.tm[0], x_pad, P, g.h, BM) || !make_tmap(&p.tm[1], w1, (uint64_t)g.E * g.f, g.h, BN / 2) ||
-      !make_tmap(&p.tm[2], w3, (uint64_t)g.E * g.f, g.h, BN / 2))
+  const uint64_t EF = (uint64_t)g.E * g.f;
+  if (!make_tmap(&p.tm[0], x_pad, P, g.h, BM) || !make_tmap(&p.tm[1], w1, EF, g.h, BN / 2) ||
+      !make_tmap(&p.tm[2], w3, EF, g.h, BN / 2) || !make_tmap(&p.tmo[0], h_out, P, g.f, 32))
     return cudaErrorInvalidValue;
-  p.tm[3] = p.tm[0];
-  p.tm[4] = p.tm[0];
+  if (a_out && b_out) {
+    if (!make_tmap(&p.tmo[1], a_out, P, g.f, 32) || !make_tmap(&p.tmo[2], b_out, P, g.f, 32))
+      return cudaErrorInvalidValue;
+    p.outs = 3;
+  }
+  p.tm[3] = p.tm[4] = p.tm[0];
   p.n_tiles = g.f / (BN / 2);
   p.k_iters = g.h / BK;
-  p.out0 = bf(h_out);
-  p.out1 = bf(a_out);
-  p.out2 = bf(b_out);
-  return launch_gemm<MODE_GLU>(p, (long long)g.nblk_cap * p.n_tiles, st);
+  p.group = raster_units(g.h);
+  return launch_gemm<MODE_GLU>(p, max_units(g) * p.n_tiles, st);
 }
 
 cudaError_t launch_down_gemm(const GemmProblem &g, const void *h_in, const void *w2, void *y_pad,
                              cudaStream_t st) {
-  GemmParams p = base_params(g.h, g.f, g.E, g.num_blocks, g.block_expert, g.padded_bins, g.status);
+  GemmParams p = base_params(g);
   const uint64_t P = (uint64_t)g.nblk_cap * BM;
-  if (!make_tmap(&p.tm[0], h_in, P, g.f, BM) || !make_tmap(&p.tm[1], w2, (uint64_t)g.E * g.h, g.f, BN))
+  if (!make_tmap(&p.tm[0], h_in, P, g.f, BM) ||
+      !make_tmap(&p.tm[1], w2, (uint64_t)g.E * g.h, g.f, BN / 2) ||
+      !make_tmap(&p.tmo[0], y_pad, P, g.h, 32))
     return cudaErrorInvalidValue;
   p.tm[2] = p.tm[3] = p.tm[4] = p.tm[0];
   p.n_tiles = (g.h + BN - 1) / BN;
   p.k_iters = g.f / BK;
-  p.out0 = bf(y_pad);
-  return launch_gemm<MODE_DOWN>(p, (long long)g.nblk_cap * p.n_tiles, st);
+  p.group = raster_units(g.f);
+  return launch_gemm<MODE_DOWN>(p, max_units(g) * p.n_tiles, st);
 }
 
 cudaError_t launch_dglu_gemm(const GemmProblem &g, const void *dy_pad, const void *w2,
                              const void *a_in, const void *b_in, void *da_out, void *db_out,
                              cudaStream_t st) {
-  GemmParams p = base_params(g.h, g.f, g.E, g.num_blocks, g.block_expert, g.padded_bins, g.status);
+  GemmParams p = base_params(g);
   const uint64_t P = (uint64_t)g.nblk_cap * BM;
-  if (!make_tmap(&p.tm[0], dy_pad, P, g.h, BM) || !make_tmap(&p.tm[1], w2, (uint64_t)g.E * g.h, g.f, 64))
+  if (!make_tmap(&p.tm[0], dy_pad, P, g.h, BM) ||
+      !make_tmap(&p.tm[1], w2, (uint64_t)g.E * g.h, g.f, 64) ||
+      !make_tmap(&p.tmo[0], da_out, P, g.f, 32) || !make_tmap(&p.tmo[1], db_out, P, g.f, 32))
     return cudaErrorInvalidValue;
   p.tm[2] = p.tm[3] = p.tm[4] = p.tm[0];
   p.n_tiles = (g.f + BN - 1) / BN;
   p.k_iters = g.h / BK;
-  p.out0 = bf(da_out);
-  p.out1 = bf(db_out);
-  p.in0 = cbf(a_in);
-  p.in1 = cbf(b_in);
-  return launch_gemm<MODE_DGLU>(p, (long long)g.nblk_cap * p.n_tiles, st);
+  p.group = raster_units(g.h);
+  p.in0 = static_cast<const __nv_bfloat16 *>(a_in);
+  p.in1 = static_cast<const __nv_bfloat16 *>(b_in);
+  return launch_gemm<MODE_DGLU>(p, max_units(g) * p.n_tiles, st);
 }
 
 cudaError_t launch_dx_gemm(const GemmProblem &g, const void *da, const void *db, const void *w1,
                            const void *w3, void *dx_pad, cudaStream_t st) {
-  GemmParams p = base_params(g.h, g.f, g.E, g.num_blocks, g.block_expert, g.padded_bins, g.status);
+  GemmParams p = base_params(g);
   const uint64_t P = (uint64_t)g.nblk_cap * BM;
+  const uint64_t EF = (uint64_t)g.E * g.f;
   if (!make_tmap(&p.tm[0], da, P, g.f, BM) || !make_tmap(&p.tm[1], db, P, g.f, BM) ||
-      !make_tmap(&p.tm[2], w1, (uint64_t)g.E * g.f, g.h, 64) ||
-      !make_tmap(&p.tm[3], w3, (uint64_t)g.E * g.f, g.h, 64))
+      !make_tmap(&p.tm[2], w1, EF, g.h, 64) || !make_tmap(&p.tm[3], w3, EF, g.h, 64) ||
+      !make_tmap(&p.tmo[0], dx_pad, P, g.h, 32))
     return cudaErrorInvalidValue;
   p.tm[4] = p.tm[0];
   p.n_tiles = (g.h + BN - 1) / BN;
   p.k_iters = 2 * (g.f / BK);
-  p.out0 = bf(dx_pad);
-  return launch_gemm<MODE_DX>(p, (long long)g.nblk_cap * p.n_tiles, st);
+  p.group = raster_units(2 * g.f);
+  return launch_gemm<MODE_DX>(p, max_units(g) * p.n_tiles, st);
 }
 
 cudaError_t launch_wgrad_gemm(const GemmProblem &g, const void *x_pad, const void *h_in,
                               const void *dy_pad, const void *da, const void *db, float *dw1,
                               float *dw3, float *dw2, cudaStream_t st) {
-  GemmParams p = base_params(g.h, g.f, g.E, g.num_blocks, g.block_expert, g.padded_bins, g.status);
+  GemmParams p = base_params(g);
   const uint64_t P = (uint64_t)g.nblk_cap * BM;
+  const uint64_t EF = (uint64_t)g.E * g.f, EH = (uint64_t)g.E * g.h;
   if (!make_tmap(&p.tm[0], da, P, g.f, 64) || !make_tmap(&p.tm[1], db, P, g.f, 64) ||
       !make_tmap(&p.tm[2], dy_pad, P, g.h, 64) || !make_tmap(&p.tm[3], x_pad, P, g.h, 64) ||
-      !make_tmap(&p.tm[4], h_in, P, g.f, 64))
+      !make_tmap(&p.tm[4], h_in, P, g.f, 64) || !make_tmap(&p.tmo[0], dw1, EF, g.h, 32, 4) ||
+      !make_tmap(&p.tmo[1], dw3, EF, g.h, 32, 4) || !make_tmap(&p.tmo[2], dw2, EH, g.f, 32, 4))
     return cudaErrorInvalidValue;
-  p.fout0 = dw1;
-  p.fout1 = dw3;
-  p.fout2 = dw2;
-  const long long t13 = (long long)(g.f / BM) * ((g.h + BN - 1) / BN);
-  const long long t2 = (long long)(g.h / BM) * ((g.f + BN - 1) / BN);
+  const long long t13 = (long long)((g.f / BM + 1) / 2) * ((g.h + BN - 1) / BN);
+  const long long t2 = (long long)((g.h / BM + 1) / 2) * ((g.f + BN - 1) / BN);
   return launch_gemm<MODE_WGRAD>(p, (long long)g.E * (2 * t13 + t2), st);
 }
 
