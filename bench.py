@@ -41,6 +41,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", type=int, default=2)
+    p.add_argument("--shape", default="",
+                   help="T,hidden,ffn,E,top_k[,bwd]: a custom workload (forward, or fwd+bwd)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample", type=int, default=0, help="tokens in the oracle sample")
     return p.parse_args()
@@ -456,6 +458,12 @@ def main():
     from dropless_mixture_experts_dmoe_b200.workloads import WORKLOADS
 
     w = WORKLOADS[args.workload]
+    if args.shape:
+        from dropless_mixture_experts_dmoe_b200.workloads import custom
+
+        parts = args.shape.split(",")
+        T, h, f, E, k = (int(v) for v in parts[:5])
+        w = custom(T, h, f, E, k, number=100, name="custom", backward="bwd" in parts[5:])
     if args.impl == "reference":
         run_reference(args, w)
     else:

@@ -126,7 +126,7 @@ size_t dmoe_workspace_bytes(const dmoe_dims *dims, int kind) {
   if (check_dims(dims) != DMOE_OK) return 0;
   switch (kind) {
     case DMOE_WS_MAP:
-      return align_up(sizeof(int32_t) * (size_t)map_tiles(dims->T) * dims->num_experts);
+      return align_up(sizeof(int32_t) * map_workspace_ints(dims->T, dims->num_experts));
     case DMOE_WS_FORWARD:
       return fwd_layout(dims).total;
     case DMOE_WS_BACKWARD:

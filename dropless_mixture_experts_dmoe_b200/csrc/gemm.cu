@@ -53,7 +53,14 @@ namespace dmoe {
 constexpr int BM = 128;  // rows of A per CTA (= one padded row block)
 constexpr int BN = 256;  // output columns per tile
 constexpr int BK = 64;   // K per pipeline stage (one 128-byte swizzle row of bf16)
-constexpr int STAGES = 5;
+#ifndef DMOE_GEMM_STAGES
+#define DMOE_GEMM_STAGES 5
+#endif
+#ifndef DMOE_GEMM_OUT_BUFS
+#define DMOE_GEMM_OUT_BUFS 2
+#endif
+constexpr int STAGES = DMOE_GEMM_STAGES;     // pipeline depth (32 KB per stage per CTA)
+constexpr int OUT_BUFS = DMOE_GEMM_OUT_BUFS;  // epilogue staging buffers per warp (1 or 2)
 constexpr int A_BYTES = BM * BK * 2;        // 16 KB: this CTA's 128 rows of A
 constexpr int B_BYTES = (BN / 2) * BK * 2;  // 16 KB: this CTA's half of B
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -64,7 +71,7 @@ constexpr int GEMM_THREADS = 192;
 constexpr int EPI_WARPS = 4;
 constexpr int EPI_THREADS = 32 * EPI_WARPS;
 constexpr int BOX_BYTES = 32 * 128;  // one result box: 32 rows x 128 B
-constexpr int OUT_BYTES = EPI_WARPS * 2 * BOX_BYTES;
+constexpr int OUT_BYTES = EPI_WARPS * OUT_BUFS * BOX_BYTES;
 constexpr size_t SMEM_BYTES = 1024 /*align*/ + (size_t)STAGES * STAGE_BYTES + OUT_BYTES +
                               256 /*barriers*/ + sizeof(int) * (DMOE_MAX_EXPERTS + 1);
 
@@ -206,7 +213,7 @@ struct Stager {
   __device__ __forceinline__ void emit(const CUtensorMap *map, const uint32_t (&w)[32], int x,
                                        int y) {
     const uint32_t buf = bufs + (uint32_t)(cur * BOX_BYTES);
-    if (lane == 0) bulk_wait_read<1>();  // the store that last used this buffer has read it
+    if (lane == 0) bulk_wait_read<OUT_BUFS - 1>();  // the store that last used it has read it
     __syncwarp();
     const uint32_t row = buf + (uint32_t)(lane * 128);
 #pragma unroll
@@ -219,7 +226,7 @@ struct Stager {
       tma_store_2d_u32(map, buf, x, y);
       bulk_commit();
     }
-    cur ^= 1;
+    cur = (cur + 1) % OUT_BUFS;
   }
 };
 
@@ -300,7 +307,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
         const float dh0 = __uint_as_float(i < 16 ? v0[2 * i] : v1[2 * i - 32]);
         const float dh1 = __uint_as_float(i < 16 ? v0[2 * i + 1] : v1[2 * i - 31]);
         const float a0 = bf16_lo(aw), a1 = bf16_hi(aw), b0 = bf16_lo(bw), b1 = bf16_hi(bw);
-        const float s0 = 1.0f / (1.0f + __expf(-a0)), s1 = 1.0f / (1.0f + __expf(-a1));
+        const float s0 = sigmoid_f(a0), s1 = sigmoid_f(a1);
         wa[i] = pack_bf16x2(dh0 * b0 * s0 * (1.0f + a0 * (1.0f - s0)),
                             dh1 * b1 * s1 * (1.0f + a1 * (1.0f - s1)));
         wb[i] = pack_bf16x2(dh0 * a0 * s0, dh1 * a1 * s1);
@@ -486,7 +493,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     // ---------------- epilogue (both CTAs) ----------------
     const int sub = warp & 3;  // TMEM sub-partition this warp may read
     Stager st;
-    st.bufs = smem_u32(outbuf) + (uint32_t)((warp - 2) * 2 * BOX_BYTES);
+    st.bufs = smem_u32(outbuf) + (uint32_t)((warp - 2) * OUT_BUFS * BOX_BYTES);
     st.cur = 0;
     st.lane = lane;
     int acc = 0;

@@ -12,6 +12,12 @@ constexpr int kMapTokTile = 64;
 
 inline int map_tiles(int T) { return (T + kMapTokTile - 1) / kMapTokTile; }
 
+// Map workspace: per-tile histograms [map_tiles(T), E] int32, then one ticket counter.
+inline size_t map_workspace_ints(int T, int E) { return (size_t)map_tiles(T) * E + 1; }
+inline unsigned int *map_ticket(int32_t *tile_hist, int T, int E) {
+  return reinterpret_cast<unsigned int *>(tile_hist + (size_t)map_tiles(T) * E);
+}
+
 // Map: routing + per-tile histogram (logits given) or histogram of given top_experts.
 cudaError_t launch_route_hist(const uint16_t *logits, int T, int E, int k, int32_t *top,
                               float *weights, int32_t *tile_hist, int32_t *status,

@@ -1,12 +1,14 @@
 // map.cu -- routing and sparse-map construction (MegaBlocks walkthrough "02 · dropless MoE 与
 // block-sparse 重构", sections 4.1-4.3; Fast-LLM issue #56 get_sparse_map).
 //
-// Three kernels, no global atomics, no spin-waits, deterministic results:
+// Three kernels, no spin-waits, deterministic results (the only global atomic is the scan's
+// completion ticket):
 //   k_route_hist   one warp per token: top-k by integer max over order-preserving keys
 //                  (ties -> lower expert index), fp32 softmax weights, per-tile histogram in
 //                  shared memory (O(E) bytes, independent of T).
-//   k_map_scan     one CTA: per-expert exclusive offsets of every tile, bins, padded_bins
-//                  (round_up to 128), num_blocks and the block -> expert table.
+//   k_map_scan     one CTA per 32 experts: per-expert exclusive offsets of every tile; the
+//                  last CTA to finish (a ticket counter, no waiting) computes bins,
+//                  padded_bins (round_up to 128), num_blocks and the block -> expert table.
 //   k_map_scatter  one CTA per tile: stable rank of every entry inside its expert (warp
 //                  histograms + __match_any_sync ranks in entry order), then indices,
 //                  bin_ids and dest_row from the index math of section 4.2.
@@ -29,8 +31,10 @@ __global__ void __launch_bounds__(kMapThreads) k_route_hist(const uint16_t *__re
                                                             int32_t *__restrict__ top,
                                                             float *__restrict__ weights,
                                                             int32_t *__restrict__ tile_hist,
-                                                            int32_t *status) {
+                                                            int32_t *status,
+                                                            unsigned int *__restrict__ done) {
   extern __shared__ int hist[];  // [E]
+  if (blockIdx.x == 0 && threadIdx.x == 0) *done = 0u;  // ticket counter of k_map_scan
   for (int e = threadIdx.x; e < E; e += kMapThreads) hist[e] = 0;
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -101,8 +105,10 @@ __global__ void __launch_bounds__(kMapThreads) k_route_hist(const uint16_t *__re
 __global__ void __launch_bounds__(kMapThreads) k_given_hist(const int32_t *__restrict__ top,
                                                             int T, int E, int k,
                                                             int32_t *__restrict__ tile_hist,
-                                                            int32_t *status) {
+                                                            int32_t *status,
+                                                            unsigned int *__restrict__ done) {
   extern __shared__ int hist[];
+  if (blockIdx.x == 0 && threadIdx.x == 0) *done = 0u;  // ticket counter of k_map_scan
   for (int e = threadIdx.x; e < E; e += kMapThreads) hist[e] = 0;
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -161,60 +167,80 @@ __device__ __forceinline__ int block_incl_scan(int v, int *warp_tot) {
   return v;
 }
 
+// Per-tile exclusive offsets inside each expert, then (in the last CTA to finish) bins,
+// padded_bins, num_blocks and the block -> expert table.  Grid: one CTA per 32 experts; warp c
+// of a CTA owns tile chunk c (32 chunks), lane l owns expert 32*blockIdx.x + l, so every load
+// of a tile's histogram row is one coalesced 128-byte access.  No CTA waits for another: the
+// CTA that takes the last ticket of `done` (zeroed by the routing kernel) does the final part.
 __global__ void __launch_bounds__(kScanThreads) k_map_scan(int n_tiles, int E, int nblk_cap,
                                                            int32_t *__restrict__ tile_hist,
                                                            int32_t *__restrict__ tokens_per_expert,
                                                            int32_t *__restrict__ bins,
                                                            int32_t *__restrict__ padded_bins,
                                                            int32_t *__restrict__ block_expert,
-                                                           int32_t *__restrict__ num_blocks) {
-  __shared__ int chunk[kScanThreads];  // [C][E] partial sums, then exclusive chunk offsets
+                                                           int32_t *__restrict__ num_blocks,
+                                                           unsigned int *__restrict__ done) {
+  __shared__ int chunk[32][33];
   __shared__ int s_pb[DMOE_MAX_EXPERTS];
   __shared__ int warp_tot[32];
-  const int tid = threadIdx.x;
-  const int C = max(1, kScanThreads / E);  // tile chunks per expert
-  const int e = tid % E, c = tid / E;
-  const bool active = c < C;
-  const int tpc = (n_tiles + C - 1) / C;
+  __shared__ bool is_last;
+  const int c = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * 32 + lane;
+  const int tpc = (n_tiles + 31) / 32;
   const int tb = c * tpc, te = min(n_tiles, tb + tpc);
   int sum = 0;
-  if (active)
-    for (int t = tb; t < te; ++t) sum += tile_hist[(size_t)t * E + e];
-  chunk[tid] = active ? sum : 0;
+  if (e < E) {
+    int t = tb;
+    for (; t + 4 <= te; t += 4) {  // independent loads in flight
+      const int v0 = tile_hist[(size_t)t * E + e], v1 = tile_hist[(size_t)(t + 1) * E + e];
+      const int v2 = tile_hist[(size_t)(t + 2) * E + e], v3 = tile_hist[(size_t)(t + 3) * E + e];
+      sum += v0 + v1 + v2 + v3;
+    }
+    for (; t < te; ++t) sum += tile_hist[(size_t)t * E + e];
+  }
+  chunk[c][lane] = sum;
   __syncthreads();
-  int total = 0;
-  if (tid < E) {
+  if (c == 0) {  // exclusive scan over the 32 chunks of this lane's expert
     int run = 0;
-    for (int cc = 0; cc < C; ++cc) {
-      const int v = chunk[cc * E + tid];
-      chunk[cc * E + tid] = run;
+    for (int cc = 0; cc < 32; ++cc) {
+      const int v = chunk[cc][lane];
+      chunk[cc][lane] = run;
       run += v;
     }
-    total = run;
+    if (e < E) tokens_per_expert[e] = run;
   }
   __syncthreads();
-  if (active) {  // per-tile exclusive offsets inside the expert
-    int run = chunk[tid];
+  if (e < E) {  // counts -> exclusive offsets inside the expert
+    int run = chunk[c][lane];
     for (int t = tb; t < te; ++t) {
       const int v = tile_hist[(size_t)t * E + e];
       tile_hist[(size_t)t * E + e] = run;
       run += v;
     }
   }
-  // bins = inclusive cumsum(counts); padded_bins = inclusive cumsum(round_up(counts, 128)).
-  const int cnt = (tid < E) ? total : 0;
-  const int pad = (tid < E) ? ((cnt + kBlock - 1) / kBlock) * kBlock : 0;
+  // ---- last CTA: bins, padded_bins, block table ----
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = (atomicAdd(done, 1u) == gridDim.x - 1);
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  const int tid = threadIdx.x;
+  const int cnt = (tid < E) ? *((volatile int32_t *)tokens_per_expert + tid) : 0;
+  const int pad = ((cnt + kBlock - 1) / kBlock) * kBlock;
   const int incl = block_incl_scan(cnt, warp_tot);
   const int pincl = block_incl_scan(pad, warp_tot);
   if (tid < E) {
-    tokens_per_expert[tid] = cnt;
     bins[tid] = incl;
     padded_bins[tid] = pincl;
     s_pb[tid] = pincl;
   }
   __syncthreads();
   const int nb = s_pb[E - 1] / kBlock;
-  if (tid == 0) *num_blocks = nb;
+  if (tid == 0) {
+    *num_blocks = nb;
+    *done = 0u;  // ready for the next call
+  }
   for (int b = tid; b < nblk_cap; b += kScanThreads) {
     int owner = -1;
     if (b < nb) {  // smallest e with padded_bins[e] > b*128
@@ -311,13 +337,14 @@ cudaError_t launch_route_hist(const uint16_t *logits, int T, int E, int k, int32
                               cudaStream_t st) {
   const int tiles = map_tiles(T);
   const size_t smem = sizeof(int) * (size_t)E;
+  unsigned int *done = map_ticket(tile_hist, T, E);
   if (!logits) {
-    k_given_hist<<<tiles, kMapThreads, smem, st>>>(top, T, E, k, tile_hist, status);
+    k_given_hist<<<tiles, kMapThreads, smem, st>>>(top, T, E, k, tile_hist, status, done);
     return cudaGetLastError();
   }
 #define DMOE_ROUTE(KPL)                                                                      \
   k_route_hist<KPL><<<tiles, kMapThreads, smem, st>>>(logits, T, E, k, top, weights, tile_hist, \
-                                                      status)
+                                                      status, done)
   if (E <= 32)
     DMOE_ROUTE(1);
   else if (E <= 64)
@@ -337,8 +364,10 @@ cudaError_t launch_route_hist(const uint16_t *logits, int T, int E, int k, int32
 cudaError_t launch_map_scan(int T, int E, int nblk_cap, int32_t *tile_hist,
                             int32_t *tokens_per_expert, int32_t *bins, int32_t *padded_bins,
                             int32_t *block_expert, int32_t *num_blocks, cudaStream_t st) {
-  k_map_scan<<<1, kScanThreads, 0, st>>>(map_tiles(T), E, nblk_cap, tile_hist, tokens_per_expert,
-                                         bins, padded_bins, block_expert, num_blocks);
+  k_map_scan<<<(E + 31) / 32, kScanThreads, 0, st>>>(map_tiles(T), E, nblk_cap, tile_hist,
+                                                      tokens_per_expert, bins, padded_bins,
+                                                      block_expert, num_blocks,
+                                                      map_ticket(tile_hist, T, E));
   return cudaGetLastError();
 }
 

@@ -20,8 +20,8 @@
 
 namespace {
 
-// Capacity of the static scratch, in int32 per-tile histogram entries: ceil(T/64) * E must
-// not exceed it (1 MiB; e.g. T <= 65536 tokens at E = 256, T <= 16384 at E = 1024).
+// Capacity of the static scratch in int32 words: the per-tile histograms (ceil(T/64) * E) plus
+// one counter must fit (1 MiB; e.g. T <= 65472 tokens at E = 256, T <= 16320 at E = 1024).
 constexpr size_t kNoAllocScratchInts = DMOE_NOALLOC_SCRATCH_BYTES / sizeof(int32_t);
 
 static __device__ __align__(256) int32_t g_map_scratch[kNoAllocScratchInts];
@@ -63,7 +63,7 @@ extern "C" int dmoe_sparse_map_noalloc(const dmoe_dims *dims, const void *logits
       !map->num_blocks || !map->status || (logits && !map->weights))
     return DMOE_ERR_NULL;
   const int T = dims->T, E = dims->num_experts, k = dims->top_k;
-  if ((size_t)dmoe::map_tiles(T) * (size_t)E > kNoAllocScratchInts) return DMOE_ERR_WORKSPACE;
+  if (dmoe::map_workspace_ints(T, E) > kNoAllocScratchInts) return DMOE_ERR_WORKSPACE;
   const uintptr_t a = reinterpret_cast<uintptr_t>(logits) |
                       reinterpret_cast<uintptr_t>(map->top_experts) |
                       (logits ? reinterpret_cast<uintptr_t>(map->weights) : 0);
@@ -81,8 +81,9 @@ extern "C" int dmoe_sparse_map_noalloc(const dmoe_dims *dims, const void *logits
   const long long n = (long long)T * k;
   const int nblk_cap =
       (int)((n + (long long)(DMOE_BLOCKING - 1) * E) / DMOE_BLOCKING);
-  // The histogram kernel writes every (tile, expert) entry of the scratch it later reads,
-  // so nothing left over from an earlier call is ever read; only the status word is cleared.
+  // The histogram kernel writes every (tile, expert) entry of the scratch it later reads and
+  // zeroes the counter after them, so nothing left over from an earlier call is ever read;
+  // the status word is cleared here.
   if (cudaMemsetAsync(map->status, 0, sizeof(int32_t), st) != cudaSuccess) return DMOE_ERR_LAUNCH;
   if ((rc = rc_of(dmoe::launch_route_hist(static_cast<const uint16_t *>(logits), T, E, k,
                                           map->top_experts, map->weights, scratch, map->status,
