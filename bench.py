@@ -321,47 +321,83 @@ def run_ours(args, w):
     value = world * w.T * args.steps / (ms_max / 1e3)
 
     # ---- e2e through the public API with host buffers ----
-    x_h = inp["x"].pin_memory()
-    lg_h = inp["logits"].pin_memory()
-    y_h = torch.empty((w.T, w.hidden), dtype=torch.bfloat16).pin_memory()
-    x_d, lg_d = torch.empty_like(dev["x"]), torch.empty_like(dev["logits"])
+    # Every step copies its inputs from pinned host memory and its results back.  Three
+    # streams (host->device copies, compute, device->host copies) and double-buffered device
+    # inputs/outputs let step i's copies overlap the compute of steps i-1 / i+1, as a serving
+    # loop would; the timed region spans the first copy in to the last copy out.
+    nbuf = 2
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    x_h = [inp["x"].pin_memory() for _ in range(nbuf)]
+    lg_h = [inp["logits"].pin_memory() for _ in range(nbuf)]
+    y_h = [torch.empty((w.T, w.hidden), dtype=torch.bfloat16).pin_memory() for _ in range(nbuf)]
+    x_d = [torch.empty_like(dev["x"]) for _ in range(nbuf)]
+    lg_d = [torch.empty_like(dev["logits"]) for _ in range(nbuf)]
+    y_d = [torch.empty_like(y) for _ in range(nbuf)]
     if train:
-        dy_h = inp["dy"].pin_memory()
-        dx_h = torch.empty_like(y_h).pin_memory()
-        dy_d = torch.empty_like(dev["dy"])
+        dy_h = [inp["dy"].pin_memory() for _ in range(nbuf)]
+        dx_h = [torch.empty_like(y_h[0]).pin_memory() for _ in range(nbuf)]
+        dy_d = [torch.empty_like(dev["dy"]) for _ in range(nbuf)]
+        dx_d = [torch.empty_like(y) for _ in range(nbuf)]
+    ev_in = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_comp = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_out = [torch.cuda.Event() for _ in range(nbuf)]
+    used = [False] * nbuf
 
-    def e2e_step():
-        x_d.copy_(x_h, non_blocking=True)
-        lg_d.copy_(lg_h, non_blocking=True)
-        B.dmoe_sparse_map(dims, lg_d, bufs.map, bufs.ws_map, st)
+    def e2e_step(i):
+        j = i % nbuf
+        with torch.cuda.stream(s_in):
+            if used[j]:
+                s_in.wait_event(ev_comp[j])  # the compute that read this buffer is done
+            x_d[j].copy_(x_h[j], non_blocking=True)
+            lg_d[j].copy_(lg_h[j], non_blocking=True)
+            if train:
+                dy_d[j].copy_(dy_h[j], non_blocking=True)
+            ev_in[j].record(s_in)
+        st.wait_event(ev_in[j])
+        if used[j]:
+            st.wait_event(ev_out[j])  # the results of this buffer have been copied out
+        B.dmoe_sparse_map(dims, lg_d[j], bufs.map, bufs.ws_map, st)
         if train:
-            dy_d.copy_(dy_h, non_blocking=True)
-            B.dmoe_forward(dims, x_d, dev["w1"], dev["w3"], dev["w2"], bufs.map, y, bufs.saved, None, st)
-            B.dmoe_backward(dims, dy_d, dev["w1"], dev["w3"], dev["w2"], bufs.map, bufs.saved,
-                            grads["dx"], grads["dw1"], grads["dw3"], grads["dw2"], grads["dw"],
+            B.dmoe_forward(dims, x_d[j], dev["w1"], dev["w3"], dev["w2"], bufs.map, y_d[j], bufs.saved,
+                           None, st)
+            B.dmoe_backward(dims, dy_d[j], dev["w1"], dev["w3"], dev["w2"], bufs.map, bufs.saved,
+                            dx_d[j], grads["dw1"], grads["dw3"], grads["dw2"], grads["dw"],
                             bufs.ws_bwd, st)
-            dx_h.copy_(grads["dx"], non_blocking=True)
         else:
-            B.dmoe_forward(dims, x_d, dev["w1"], dev["w3"], dev["w2"], bufs.map, y, None, bufs.ws_fwd, st)
-        y_h.copy_(y, non_blocking=True)
+            B.dmoe_forward(dims, x_d[j], dev["w1"], dev["w3"], dev["w2"], bufs.map, y_d[j], None,
+                           bufs.ws_fwd, st)
+        ev_comp[j].record(st)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[j])
+            y_h[j].copy_(y_d[j], non_blocking=True)
+            if train:
+                dx_h[j].copy_(dx_d[j], non_blocking=True)
+            ev_out[j].record(s_out)
+        used[j] = True
 
-    for _ in range(max(3, args.warmup)):
-        e2e_step()
+    for i in range(max(3, args.warmup)):
+        e2e_step(i)
+    torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(st)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(st)
+    e0.record(s_in)
+    for i in range(args.steps):
+        e2e_step(i)
+    s_out.wait_stream(st)
+    s_out.wait_stream(s_in)
+    e1.record(s_out)
     torch.cuda.synchronize()
     te = torch.tensor([e0.elapsed_time(e1)], device="cuda", dtype=torch.float64)
     if world > 1:
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
     e2e_value = world * w.T * args.steps / (float(te.item()) / 1e3)
-    h2d = x_h.numel() * 2 + lg_h.numel() * 2 + (dy_h.numel() * 2 if train else 0)
-    d2h = y_h.numel() * 2 + (dx_h.numel() * 2 if train else 0)
+    h2d = x_h[0].numel() * 2 + lg_h[0].numel() * 2 + (dy_h[0].numel() * 2 if train else 0)
+    d2h = y_h[0].numel() * 2 + (dx_h[0].numel() * 2 if train else 0)
+    # the pipelined e2e output is checked against the device-resident one
+    torch.cuda.synchronize()
+    e2e_matches = bool(torch.equal(y_h[(args.steps - 1) % nbuf].view(torch.int16),
+                                   y.cpu().view(torch.int16)))
 
     # parity spot check of the timed output against the oracle is done by the tests; here we
     # only confirm the device status stayed clean.
@@ -425,8 +461,10 @@ def run_ours(args, w):
                      "algorithmic_flops_per_launch": flops[dom]},
         "kernels": kernels,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h, "pipelined": "copies overlap compute (3 streams)",
+                "output_matches_device_run": e2e_matches},
         "gpu_launches": (7 + (5 if train else 0)) * args.steps,
+        "gpu_launches_note": "kernels of this library in the device-resident timed region",
         "status": status,
     }
     if clocks:

@@ -26,7 +26,12 @@ __device__ __forceinline__ uint4 ld_nc_v4(const uint4 *p) {
   return v;
 }
 
-// Work items: [0, T) tokens; [T, T + 128*E) padding rows (expert e, row r of its last block).
+// A row slice is 32 * kGatherVPL 16-byte vectors (4 KB); a token's row is split into
+// ceil(vpr / slice) slices so that short-T workloads still keep many warps busy.
+constexpr int kSliceVecs = 32 * kGatherVPL;
+
+// Work items: [0, T*S) token slices (S slices per row); then 128*E padding rows (expert e,
+// row r of its last block).
 __global__ void __launch_bounds__(kCopyThreads) k_gather(int T, int h, int k, int E,
                                                          const uint4 *__restrict__ x,
                                                          const int32_t *__restrict__ dest_row,
@@ -35,34 +40,35 @@ __global__ void __launch_bounds__(kCopyThreads) k_gather(int T, int h, int k, in
                                                          uint4 *__restrict__ x_pad) {
   const int lane = threadIdx.x & 31;
   const int vpr = h >> 3;  // 16-byte vectors per row
-  const long long items = (long long)T + (long long)kBlock * E;
+  const int S = (vpr + kSliceVecs - 1) / kSliceVecs;
+  const long long ntok = (long long)T * S;
+  const long long items = ntok + (long long)kBlock * E;
   const long long nw = (long long)gridDim.x * kCopyWarps;
   for (long long it = (long long)blockIdx.x * kCopyWarps + (threadIdx.x >> 5); it < items;
        it += nw) {
-    if (it < T) {
-      const int t = (int)it;
+    if (it < ntok) {
+      const int t = (int)(it / S);
+      const int v0 = (int)(it - (long long)t * S) * kSliceVecs;
       const int d = (lane < k) ? dest_row[(size_t)t * k + lane] : -1;
       const uint4 *src = x + (size_t)t * vpr;
-      for (int v0 = 0; v0 < vpr; v0 += 32 * kGatherVPL) {
-        uint4 buf[kGatherVPL];
+      uint4 buf[kGatherVPL];
+#pragma unroll
+      for (int u = 0; u < kGatherVPL; ++u) {
+        const int v = v0 + u * 32 + lane;
+        if (v < vpr) buf[u] = ld_nc_v4(src + v);
+      }
+      for (int s = 0; s < k; ++s) {
+        const int r = __shfl_sync(0xFFFFFFFFu, d, s);
+        if (r < 0) continue;
+        uint4 *dst = x_pad + (size_t)r * vpr;
 #pragma unroll
         for (int u = 0; u < kGatherVPL; ++u) {
           const int v = v0 + u * 32 + lane;
-          if (v < vpr) buf[u] = ld_nc_v4(src + v);
-        }
-        for (int s = 0; s < k; ++s) {
-          const int r = __shfl_sync(0xFFFFFFFFu, d, s);
-          if (r < 0) continue;
-          uint4 *dst = x_pad + (size_t)r * vpr;
-#pragma unroll
-          for (int u = 0; u < kGatherVPL; ++u) {
-            const int v = v0 + u * 32 + lane;
-            if (v < vpr) dst[v] = buf[u];
-          }
+          if (v < vpr) dst[v] = buf[u];
         }
       }
     } else {
-      const long long p = it - T;
+      const long long p = it - ntok;
       const int e = (int)(p / kBlock), r = (int)(p % kBlock);
       const int c = counts[e];
       const int pend = padded_bins[e];
@@ -86,12 +92,17 @@ __global__ void __launch_bounds__(kCopyThreads) k_combine(int T, int h, int k,
                                                           uint4 *__restrict__ y) {
   const int lane = threadIdx.x & 31;
   const int vpr = h >> 3;
+  const int S = (vpr + kSliceVecs - 1) / kSliceVecs;
+  const long long items = (long long)T * S;
   const long long nw = (long long)gridDim.x * kCopyWarps;
-  for (long long it = (long long)blockIdx.x * kCopyWarps + (threadIdx.x >> 5); it < T; it += nw) {
-    const int t = (int)it;
+  for (long long it = (long long)blockIdx.x * kCopyWarps + (threadIdx.x >> 5); it < items;
+       it += nw) {
+    const int t = (int)(it / S);
+    const int vs = (int)(it - (long long)t * S) * kSliceVecs;
+    const int ve = min(vpr, vs + kSliceVecs);
     const int d = (lane < k) ? dest_row[(size_t)t * k + lane] : -1;
     const float wl = (lane < k) ? (weights ? weights[(size_t)t * k + lane] : 1.0f) : 0.0f;
-    for (int v0 = 0; v0 < vpr; v0 += 32 * kCombineVPL) {
+    for (int v0 = vs; v0 < ve; v0 += 32 * kCombineVPL) {
       float acc[kCombineVPL][8];
 #pragma unroll
       for (int u = 0; u < kCombineVPL; ++u)
@@ -107,7 +118,7 @@ __global__ void __launch_bounds__(kCopyThreads) k_combine(int T, int h, int k,
 #pragma unroll
             for (int u = 0; u < kCombineVPL; ++u) {
               const int v = v0 + u * 32 + lane;
-              if (v < vpr) buf[ss][u] = ld_nc_v4(y_pad + (size_t)r * vpr + v);
+              if (v < ve) buf[ss][u] = ld_nc_v4(y_pad + (size_t)r * vpr + v);
             }
           }
         }
@@ -132,7 +143,7 @@ __global__ void __launch_bounds__(kCopyThreads) k_combine(int T, int h, int k,
 #pragma unroll
       for (int u = 0; u < kCombineVPL; ++u) {
         const int v = v0 + u * 32 + lane;
-        if (v < vpr) {
+        if (v < ve) {
           uint4 o;
           o.x = pack_bf16x2(acc[u][0], acc[u][1]);
           o.y = pack_bf16x2(acc[u][2], acc[u][3]);
@@ -231,10 +242,12 @@ static int copy_grid(long long items) {
   return (int)(want < 1 ? 1 : want);
 }
 
+static long long slices(int h) { return ((h >> 3) + kSliceVecs - 1) / kSliceVecs; }
+
 cudaError_t launch_gather(int T, int h, int k, int E, const void *x, const int32_t *dest_row,
                           const int32_t *counts, const int32_t *padded_bins, void *x_pad,
                           cudaStream_t st) {
-  const long long items = (long long)T + (long long)kBlock * E;
+  const long long items = (long long)T * slices(h) + (long long)kBlock * E;
   k_gather<<<copy_grid(items), kCopyThreads, 0, st>>>(
       T, h, k, E, static_cast<const uint4 *>(x), dest_row, counts, padded_bins,
       static_cast<uint4 *>(x_pad));
@@ -243,7 +256,8 @@ cudaError_t launch_gather(int T, int h, int k, int E, const void *x, const int32
 
 cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const int32_t *dest_row,
                            const float *weights, void *y, cudaStream_t st) {
-  k_combine<<<copy_grid(T), kCopyThreads, 0, st>>>(T, h, k, static_cast<const uint4 *>(y_pad),
+  k_combine<<<copy_grid((long long)T * slices(h)), kCopyThreads, 0, st>>>(
+      T, h, k, static_cast<const uint4 *>(y_pad),
                                                    dest_row, weights, static_cast<uint4 *>(y));
   return cudaGetLastError();
 }

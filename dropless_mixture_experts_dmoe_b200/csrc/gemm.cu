@@ -20,8 +20,9 @@
 //               shared memory and writes each CTA's 128 accumulator rows into its own TMEM,
 //               and tcgen05.commit (multicast to both CTAs) to free stages and hand over
 //               accumulators.
-//   warps 2-5   epilogue (both CTAs): tcgen05.ld of the accumulator (each warp its 32-lane
-//               TMEM sub-partition), fused element-wise work, results staged in 128-byte-
+//   warps 2..   epilogue (both CTAs; 4 warps, or 8 for a DOWN GEMM with ffn <= 256): tcgen05.ld of
+//               the accumulator (each warp its 32-lane TMEM sub-partition and, with 8 warps,
+//               half of the columns), fused element-wise work, results staged in 128-byte-
 //               swizzled shared memory (32 rows x 128 B per box) and written with TMA
 //               bulk-tensor stores, double-buffered per warp.
 // Two accumulators (2 x 256 columns) let the epilogue of tile i overlap the MMAs of i+1.
@@ -53,34 +54,32 @@ namespace dmoe {
 constexpr int BM = 128;  // rows of A per CTA (= one padded row block)
 constexpr int BN = 256;  // output columns per tile
 constexpr int BK = 64;   // K per pipeline stage (one 128-byte swizzle row of bf16)
-#ifndef DMOE_GEMM_STAGES
-#define DMOE_GEMM_STAGES 5
-#endif
-#ifndef DMOE_GEMM_OUT_BUFS
-#define DMOE_GEMM_OUT_BUFS 2
-#endif
-constexpr int STAGES = DMOE_GEMM_STAGES;     // pipeline depth (32 KB per stage per CTA)
-constexpr int OUT_BUFS = DMOE_GEMM_OUT_BUFS;  // epilogue staging buffers per warp (1 or 2)
 constexpr int A_BYTES = BM * BK * 2;        // 16 KB: this CTA's 128 rows of A
 constexpr int B_BYTES = (BN / 2) * BK * 2;  // 16 KB: this CTA's half of B
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int CHUNK_BYTES = 64 * BK * 2;    // one 64 x 64 MN-major box: 8 KB
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = 256;
-constexpr int GEMM_THREADS = 192;
-constexpr int EPI_WARPS = 4;
-constexpr int EPI_THREADS = 32 * EPI_WARPS;
 constexpr int BOX_BYTES = 32 * 128;  // one result box: 32 rows x 128 B
-constexpr int OUT_BYTES = EPI_WARPS * OUT_BUFS * BOX_BYTES;
-constexpr size_t SMEM_BYTES = 1024 /*align*/ + (size_t)STAGES * STAGE_BYTES + OUT_BYTES +
-                              256 /*barriers*/ + sizeof(int) * (DMOE_MAX_EXPERTS + 1);
 
 enum GemmMode { MODE_GLU = 0, MODE_DOWN = 1, MODE_DGLU = 2, MODE_DX = 3, MODE_WGRAD = 4 };
 
-template <int MODE>
-struct ModeTraits {
+// Per-launch configuration.  A 5-stage ring of 32 KB per CTA; 4 epilogue warps (one per TMEM
+// sub-partition, double-buffered result staging) by default, or 8 (two per sub-partition,
+// each taking half of the tile's columns, one staging buffer each) for GEMMs whose K is so
+// short (4 stages per tile) that the epilogue, not the MMA, bounds a tile.
+template <int MODE, int EPI>
+struct Cfg {
   static constexpr int a_mn = (MODE == MODE_WGRAD) ? 1 : 0;
   static constexpr int b_mn = (MODE == MODE_DGLU || MODE == MODE_DX || MODE == MODE_WGRAD) ? 1 : 0;
+  static constexpr int epi_warps = EPI;
+  static constexpr int col_split = epi_warps / 4;  // warps per TMEM sub-partition
+  static constexpr int threads = 64 + 32 * epi_warps;
+  static constexpr int stages = 5;
+  static constexpr int out_bufs = (EPI == 8) ? 1 : 2;
+  static constexpr int out_bytes = epi_warps * out_bufs * BOX_BYTES;
+  static constexpr size_t smem = 1024 /*align*/ + (size_t)stages * STAGE_BYTES + out_bytes +
+                                 256 /*barriers*/ + sizeof(int) * (DMOE_MAX_EXPERTS + 1);
 };
 
 struct GemmParams {
@@ -205,8 +204,9 @@ __device__ __forceinline__ void load_stage(const GemmParams &p, const Tile &tl, 
 // Per-warp result staging: two 4 KB buffers, each one box of 32 rows x 128 B in the 128-byte
 // swizzled layout that a SWIZZLE_128B tensor map expects (16-byte chunk c of row r sits at
 // chunk position c ^ (r & 7)).  Lane l writes row l; lane 0 issues the TMA store.
+template <int OUT_BUFS>
 struct Stager {
-  uint32_t bufs;  // shared address of buffer 0 (buffer 1 follows)
+  uint32_t bufs;  // shared address of buffer 0 (the others follow)
   int cur;
   int lane;
 
@@ -241,10 +241,12 @@ __device__ __forceinline__ void pack_bf16_row(const uint32_t (&lo)[32], const ui
 
 // Epilogue of one tile for the warp owning TMEM sub-partition `sub` (rows sub*32 .. +31 of
 // this CTA's 128 rows); tb = TMEM address of the warp's lanes at accumulator column 0.
-template <int MODE>
+template <int MODE, int EPI>
 __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &tl, uint32_t tb,
-                                              int sub, int lane, Stager &st) {
+                                              int sub, int half, int lane,
+                                              Stager<Cfg<MODE, EPI>::out_bufs> &st) {
   const int y0 = tl.row0 + sub * 32;  // first row of this warp's boxes
+  constexpr int kw = BN / Cfg<MODE, EPI>::col_split;  // accumulator columns per warp (non-GLU)
   if (MODE == MODE_GLU) {
     const int n0 = tl.n * (BN / 2);
 #pragma unroll 1
@@ -271,22 +273,30 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
       }
     }
   } else if (MODE == MODE_DOWN || MODE == MODE_DX) {
-    const int n0 = tl.n * BN;
+    const int n0 = tl.n * BN + half * kw;  // this warp's first column
+    const int ncols = min(kw, p.h - n0);   // multiple of 64 (may be <= 0)
+    if (ncols <= 0) return;
+    tb += (uint32_t)(half * kw);
+    uint32_t v0[32], v1[32], w[32];
+    tmem_ld32(tb, v0);
+    tmem_ld32(tb + 32, v1);
+    tmem_ld_wait();
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 64) {
-      if (n0 + c >= p.h) break;  // uniform across the warp
-      uint32_t v0[32], v1[32], w[32];
-      tmem_ld32(tb + c, v0);
-      tmem_ld32(tb + c + 32, v1);
-      tmem_ld_wait();
+    for (int c = 0; c < ncols; c += 64) {
       pack_bf16_row(v0, v1, w);
+      if (c + 64 < ncols) {  // the next box's accumulator loads overlap this box's store
+        tmem_ld32(tb + c + 64, v0);
+        tmem_ld32(tb + c + 96, v1);
+      }
       st.emit(&p.tmo[0], w, n0 + c, y0);
+      tmem_ld_wait();
     }
   } else if (MODE == MODE_DGLU) {
-    const int n0 = tl.n * BN;
+    const int n0 = tl.n * BN + half * kw;
+    tb += (uint32_t)(half * kw);
     const size_t grow = (size_t)y0 + lane;
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 64) {
+    for (int c = 0; c < kw; c += 64) {
       if (n0 + c >= p.f) break;
       uint32_t v0[32], v1[32], wa[32], wb[32];
       uint4 qa[8], qb[8];
@@ -319,33 +329,42 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
     const int rows = (tl.which == 2) ? p.h : p.f;
     const int cols = (tl.which == 2) ? p.f : p.h;
     const int yw = tl.e * rows + tl.m * BM + sub * 32;
-    const int n0 = tl.n * BN;
-#pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
-      if (n0 + c >= cols) break;
-      uint32_t v[32];
-      if (tl.kit > 0) {
-        tmem_ld32(tb + c, v);
-        tmem_ld_wait();
-      } else {
+    const int n0 = tl.n * BN + half * kw;
+    const int ncols = min(kw, cols - n0);  // multiple of 32 (may be <= 0)
+    if (ncols <= 0) return;
+    tb += (uint32_t)(half * kw);
+    uint32_t v[32], w[32];
+    if (tl.kit > 0) {
+      tmem_ld32(tb, v);
+      tmem_ld_wait();
+    } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = 0u;  // expert without rows: exact zeros
-      }
-      st.emit(&p.tmo[tl.which], v, n0 + c, yw);
+      for (int i = 0; i < 32; ++i) v[i] = 0u;  // expert without rows: exact zeros
+    }
+#pragma unroll 1
+    for (int c = 0; c < ncols; c += 32) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) w[i] = v[i];
+      if (tl.kit > 0 && c + 32 < ncols) tmem_ld32(tb + c + 32, v);  // overlaps the store
+      st.emit(&p.tmo[tl.which], w, n0 + c, yw);
+      if (tl.kit > 0) tmem_ld_wait();
     }
   }
 }
 
 // ---- the kernel -------------------------------------------------------------------------------
 
-template <int MODE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
+template <int MODE, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::threads, 1)
     k_grouped_gemm(const __grid_constant__ GemmParams p) {
+  using C = Cfg<MODE, EPI>;
+  constexpr int STAGES = C::stages;
+  constexpr int EPI_THREADS = 32 * C::epi_warps;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base_u32 = smem_u32(smem_raw);
   uint8_t *tiles = smem_raw + ((1024u - (base_u32 & 1023u)) & 1023u);
   uint8_t *outbuf = tiles + STAGES * STAGE_BYTES;  // 1024-aligned
-  uint64_t *bars = reinterpret_cast<uint64_t *>(outbuf + OUT_BYTES);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(outbuf + C::out_bytes);
   uint64_t *full = bars;                       // [STAGES] leader: both halves landed
   uint64_t *empty = bars + STAGES;             // [STAGES] MMAs done reading the stage
   uint64_t *tfull = bars + 2 * STAGES;         // [2] accumulator ready
@@ -353,7 +372,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   uint64_t *drain = bars + 2 * STAGES + 4;     // leader: all MMAs finished
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  int *ustart = reinterpret_cast<int *>(outbuf + OUT_BYTES + 256);  // [E + 1]
+  int *ustart = reinterpret_cast<int *>(outbuf + C::out_bytes + 256);  // [E + 1]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -377,7 +396,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   }
   if (MODE != MODE_WGRAD) {
     // units (pairs of row blocks) per expert -> exclusive prefix ustart[0..E]
-    for (int e = threadIdx.x; e < p.E; e += GEMM_THREADS) {
+    for (int e = threadIdx.x; e < p.E; e += C::threads) {
       const int blocks = (p.padded_bins[e] - ((e > 0) ? p.padded_bins[e - 1] : 0)) / BM;
       ustart[e + 1] = (blocks + 1) / 2;
     }
@@ -446,7 +465,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   } else if (warp == 1 && lane == 0 && leader) {
     // ---------------- MMA issuer (leader only) ----------------
     constexpr uint32_t idesc =
-        idesc_bf16_f32(2 * BM, BN, ModeTraits<MODE>::a_mn, ModeTraits<MODE>::b_mn);
+        idesc_bf16_f32(2 * BM, BN, C::a_mn, C::b_mn);
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
@@ -468,10 +487,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t ad = ModeTraits<MODE>::a_mn
+          const uint64_t ad = C::a_mn
                                   ? sdesc_mnmajor_sw128(a_addr + kk * 2048, CHUNK_BYTES)
                                   : sdesc_kmajor_sw128(a_addr + kk * 32);
-          const uint64_t bd = ModeTraits<MODE>::b_mn
+          const uint64_t bd = C::b_mn
                                   ? sdesc_mnmajor_sw128(b_addr + kk * 2048, CHUNK_BYTES)
                                   : sdesc_kmajor_sw128(b_addr + kk * 32);
           tc_mma_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
@@ -491,9 +510,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     mbar_wait_plain(drain, 0);
   } else if (warp >= 2) {
     // ---------------- epilogue (both CTAs) ----------------
-    const int sub = warp & 3;  // TMEM sub-partition this warp may read
-    Stager st;
-    st.bufs = smem_u32(outbuf) + (uint32_t)((warp - 2) * OUT_BUFS * BOX_BYTES);
+    const int sub = warp & 3;           // TMEM sub-partition this warp may read
+    const int half = (warp - 2) >> 2;   // which part of the tile's columns (8-warp modes)
+    Stager<C::out_bufs> st;
+    st.bufs = smem_u32(outbuf) + (uint32_t)((warp - 2) * C::out_bufs * BOX_BYTES);
     st.cur = 0;
     st.lane = lane;
     int acc = 0;
@@ -501,13 +521,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     for (int t = cluster; t < total; t += nclusters) {
       const Tile tl = decode<MODE>(p, t, ustart, rank);
       if (tl.kit == 0) {  // no accumulator involved
-        if (!tl.dummy) epilogue_tile<MODE>(p, tl, 0u, sub, lane, st);
+        if (!tl.dummy) epilogue_tile<MODE, EPI>(p, tl, 0u, sub, half, lane, st);
         continue;
       }
       if (!mbar_wait(&tfull[acc], acc_phase, p.status, abort_flag)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * ACC_COLS);
-      if (!tl.dummy) epilogue_tile<MODE>(p, tl, tb, sub, lane, st);
+      if (!tl.dummy) epilogue_tile<MODE, EPI>(p, tl, tb, sub, half, lane, st);
       tc_fence_before();
       mbar_arrive_cluster(leader_tempty0 + (uint32_t)(acc * sizeof(uint64_t)));
       acc ^= 1;
@@ -583,21 +603,23 @@ static int raster_units(int K) {
   return (int)g;
 }
 
-template <int MODE>
+template <int MODE, int EPI>
 static cudaError_t launch_gemm(const GemmParams &p, long long max_tiles, cudaStream_t st) {
+  using C = Cfg<MODE, EPI>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   static int max_clusters = 0;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(k_grouped_gemm<MODE>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    attr_err = cudaFuncSetAttribute(k_grouped_gemm<MODE, EPI>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::smem);
     if (attr_err != cudaSuccess) return;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (device_sm_count() / 2), 1, 1);
-    cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.blockDim = dim3(C::threads, 1, 1);
+    cfg.dynamicSmemBytes = C::smem;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, k_grouped_gemm<MODE>, &cfg) != cudaSuccess || n < 1)
+    if (cudaOccupancyMaxActiveClusters(&n, k_grouped_gemm<MODE, EPI>, &cfg) != cudaSuccess ||
+        n < 1)
       n = device_sm_count() / 2;
     max_clusters = n;
   });
@@ -605,7 +627,7 @@ static cudaError_t launch_gemm(const GemmParams &p, long long max_tiles, cudaStr
   long long clusters = max_clusters;
   if (max_tiles < clusters) clusters = max_tiles;
   if (clusters < 1) clusters = 1;
-  k_grouped_gemm<MODE><<<(int)(2 * clusters), GEMM_THREADS, SMEM_BYTES, st>>>(p);
+  k_grouped_gemm<MODE, EPI><<<(int)(2 * clusters), C::threads, C::smem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -643,7 +665,7 @@ cudaError_t launch_glu_gemm(const GemmProblem &g, const void *x_pad, const void 
   p.n_tiles = g.f / (BN / 2);
   p.k_iters = g.h / BK;
   p.group = raster_units(g.h);
-  return launch_gemm<MODE_GLU>(p, max_units(g) * p.n_tiles, st);
+  return launch_gemm<MODE_GLU, 4>(p, max_units(g) * p.n_tiles, st);
 }
 
 cudaError_t launch_down_gemm(const GemmProblem &g, const void *h_in, const void *w2, void *y_pad,
@@ -658,7 +680,9 @@ cudaError_t launch_down_gemm(const GemmProblem &g, const void *h_in, const void 
   p.n_tiles = (g.h + BN - 1) / BN;
   p.k_iters = g.f / BK;
   p.group = raster_units(g.f);
-  return launch_gemm<MODE_DOWN>(p, max_units(g) * p.n_tiles, st);
+  if (p.k_iters <= 4)  // ffn <= 256: the epilogue bounds a tile; give it 8 warps
+    return launch_gemm<MODE_DOWN, 8>(p, max_units(g) * p.n_tiles, st);
+  return launch_gemm<MODE_DOWN, 4>(p, max_units(g) * p.n_tiles, st);
 }
 
 cudaError_t launch_dglu_gemm(const GemmProblem &g, const void *dy_pad, const void *w2,
@@ -676,7 +700,7 @@ cudaError_t launch_dglu_gemm(const GemmProblem &g, const void *dy_pad, const voi
   p.group = raster_units(g.h);
   p.in0 = static_cast<const __nv_bfloat16 *>(a_in);
   p.in1 = static_cast<const __nv_bfloat16 *>(b_in);
-  return launch_gemm<MODE_DGLU>(p, max_units(g) * p.n_tiles, st);
+  return launch_gemm<MODE_DGLU, 4>(p, max_units(g) * p.n_tiles, st);
 }
 
 cudaError_t launch_dx_gemm(const GemmProblem &g, const void *da, const void *db, const void *w1,
@@ -692,7 +716,7 @@ cudaError_t launch_dx_gemm(const GemmProblem &g, const void *da, const void *db,
   p.n_tiles = (g.h + BN - 1) / BN;
   p.k_iters = 2 * (g.f / BK);
   p.group = raster_units(2 * g.f);
-  return launch_gemm<MODE_DX>(p, max_units(g) * p.n_tiles, st);
+  return launch_gemm<MODE_DX, 4>(p, max_units(g) * p.n_tiles, st);
 }
 
 cudaError_t launch_wgrad_gemm(const GemmProblem &g, const void *x_pad, const void *h_in,
@@ -708,7 +732,7 @@ cudaError_t launch_wgrad_gemm(const GemmProblem &g, const void *x_pad, const voi
     return cudaErrorInvalidValue;
   const long long t13 = (long long)((g.f / BM + 1) / 2) * ((g.h + BN - 1) / BN);
   const long long t2 = (long long)((g.h / BM + 1) / 2) * ((g.f + BN - 1) / BN);
-  return launch_gemm<MODE_WGRAD>(p, (long long)g.E * (2 * t13 + t2), st);
+  return launch_gemm<MODE_WGRAD, 4>(p, (long long)g.E * (2 * t13 + t2), st);
 }
 
 }  // namespace dmoe

@@ -40,10 +40,24 @@ __global__ void __launch_bounds__(kMapThreads) k_route_hist(const uint16_t *__re
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * kMapTokTile;
   bool bad = false;
+  // this warp's tokens are t0 + warp, t0 + warp + 8, ...; the next token's logits are loaded
+  // while the current token is ranked
+  uint16_t nxt[KPL];
+  auto load_row = [&](int t) {
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) {
+      const int e = lane + 32 * i;
+      nxt[i] = (t < T && e < E) ? __ldg(logits + (size_t)t * E + e) : (uint16_t)0;
+    }
+  };
+  load_row(t0 + warp);
   for (int tt = warp; tt < kMapTokTile; tt += kMapWarps) {
     const int t = t0 + tt;
     if (t >= T) break;
-    const uint16_t *row = logits + (size_t)t * E;
+    uint16_t cur[KPL];
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) cur[i] = nxt[i];
+    if (tt + kMapWarps < kMapTokTile) load_row(t + kMapWarps);
     uint32_t key[KPL];
     float val[KPL];
 #pragma unroll
@@ -52,7 +66,7 @@ __global__ void __launch_bounds__(kMapThreads) k_route_hist(const uint16_t *__re
       key[i] = 0u;
       val[i] = 0.0f;
       if (e < E) {
-        const uint16_t b = __ldg(row + e);
+        const uint16_t b = cur[i];
         bad |= bf16_nonfinite(b);
         key[i] = (bf16_order(b) << 16) | (0xFFFFu - (uint32_t)e);
         val[i] = __uint_as_float((uint32_t)b << 16);
