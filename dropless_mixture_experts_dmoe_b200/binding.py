@@ -80,6 +80,7 @@ def load():
     lib.dmoe_backward.argtypes = [D, _P, _P, _P, _P, M, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
     lib.dmoe_padded_gather.argtypes = [D, _P, M, _P, _P]
     lib.dmoe_expert_glu.argtypes = [D, _P, _P, _P, M, _P, _P, _P, _P]
+    lib.dmoe_expert_glu_gather.argtypes = [D, _P, _P, _P, M, _P, _P, _P, _P]
     lib.dmoe_expert_down.argtypes = [D, _P, _P, M, _P, _P]
     lib.dmoe_padded_scatter.argtypes = [D, _P, M, _P, _P, _P]
     lib.dmoe_bwd_dy_gather.argtypes = [D, _P, M, _P, _P, _P, _P]
@@ -87,7 +88,7 @@ def load():
     lib.dmoe_bwd_dx.argtypes = [D, _P, _P, _P, _P, M, _P, _P]
     lib.dmoe_bwd_wgrad.argtypes = [D, _P, _P, _P, _P, _P, M, _P, _P, _P, _P]
     for fn in ("dmoe_sparse_map", "dmoe_forward", "dmoe_backward", "dmoe_padded_gather",
-               "dmoe_expert_glu", "dmoe_expert_down", "dmoe_padded_scatter", "dmoe_bwd_dy_gather",
+               "dmoe_expert_glu", "dmoe_expert_glu_gather", "dmoe_expert_down", "dmoe_padded_scatter", "dmoe_bwd_dy_gather",
                "dmoe_bwd_dglu", "dmoe_bwd_dx", "dmoe_bwd_wgrad"):
         getattr(lib, fn).restype = _I
     lib.dmoe_error_string.argtypes = [_I]
@@ -222,6 +223,13 @@ def dmoe_expert_glu(dims, x_pad, w1, w3, smap: SparseMap, h_out, a_out=None, b_o
     _check(load().dmoe_expert_glu(ctypes.byref(dims), _ptr(x_pad), _ptr(w1), _ptr(w3),
                                   ctypes.byref(smap.c), _ptr(h_out), _ptr(a_out), _ptr(b_out),
                                   _stream(stream)), "dmoe_expert_glu")
+
+
+def dmoe_expert_glu_gather(dims, x, w1, w3, smap: SparseMap, h_out, a_out=None, b_out=None,
+                           stream=None):
+    _check(load().dmoe_expert_glu_gather(ctypes.byref(dims), _ptr(x), _ptr(w1), _ptr(w3),
+                                         ctypes.byref(smap.c), _ptr(h_out), _ptr(a_out),
+                                         _ptr(b_out), _stream(stream)), "dmoe_expert_glu_gather")
 
 
 def dmoe_expert_down(dims, h_in, w2, smap: SparseMap, y_pad, stream=None):

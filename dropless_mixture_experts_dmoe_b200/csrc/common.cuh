@@ -275,6 +275,20 @@ __device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const CUtensorM
       : "memory");
 }
 
+// TMA gather of 4 rows (row indices y0..y3, 64 bf16 columns from x) by either CTA of a pair,
+// completing on the pair leader's mbarrier.  The tensor map's box is one row high; the rows
+// land at 4 consecutive 128-byte smem rows (128-byte swizzle).  Out-of-range rows read zeros.
+__device__ __forceinline__ void tma_gather4_pair(void *smem_dst, const CUtensorMap *map,
+                                                 uint32_t bar_cluster, int32_t x, int32_t y0,
+                                                 int32_t y1, int32_t y2, int32_t y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::"
+      "complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3),
+      "r"(bar_cluster)
+      : "memory");
+}
+
 // Whole-warp TMEM allocation shared by a CTA pair (one warp with the same id in each CTA).
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(

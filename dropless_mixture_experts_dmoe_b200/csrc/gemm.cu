@@ -33,6 +33,12 @@
 // W1/W3 and [E, h, f] for W2):
 //   GLU   A = X_pad (K)      B = W1_e rows (leader) / W3_e rows (peer), 128 f-columns each (K)
 //         out H = bf16(silu(gate) * up); optionally bf16(gate), bf16(up) for the backward
+//   GLU_GATHER  the same, with A's 128 rows gathered straight from x by the map (TMA
+//         tile::gather4, four rows per lane per stage; padding rows read zeros), so the
+//         padded copy X_pad is never written or read (the gather of walkthrough section 4.2
+//         fused into the GEMM's operand load).  32 gather instructions per 16 KB stage are
+//         more than the TMA unit issues in one stage's MMA time: about 3x slower than
+//         gather kernel + GLU on B200, so it is not the default path.
 //   DOWN  A = H (K)          B = W2_e (K)                 out Y_pad
 //   DGLU  A = dY_pad (K)     B = W2_e^T (MN)              dH; epilogue recomputes the
 //         activation from the saved A, Bm: dA = dH*Bm*s*(1+A(1-s)), dBm = dH*A*s, s = sigmoid(A)
@@ -62,7 +68,18 @@ constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = 256;
 constexpr int BOX_BYTES = 32 * 128;  // one result box: 32 rows x 128 B
 
-enum GemmMode { MODE_GLU = 0, MODE_DOWN = 1, MODE_DGLU = 2, MODE_DX = 3, MODE_WGRAD = 4 };
+enum GemmMode {
+  MODE_GLU = 0,
+  MODE_DOWN = 1,
+  MODE_DGLU = 2,
+  MODE_DX = 3,
+  MODE_WGRAD = 4,
+  MODE_GLU_GATHER = 5  // GLU whose A rows are gathered from the token rows of x
+};
+
+__host__ __device__ constexpr bool is_glu(int mode) {
+  return mode == MODE_GLU || mode == MODE_GLU_GATHER;
+}
 
 // Per-launch configuration.  A 5-stage ring of 32 KB per CTA; 4 epilogue warps (one per TMEM
 // sub-partition, double-buffered result staging) by default, or 8 (two per sub-partition,
@@ -86,6 +103,9 @@ struct GemmParams {
   CUtensorMap tm[5];   // operand tensor maps (loads)
   CUtensorMap tmo[3];  // result tensor maps (stores)
   const int32_t *padded_bins;
+  const int32_t *bins;     // GLU_GATHER: real expert boundaries
+  const int32_t *indices;  // GLU_GATHER: sorted entry -> flattened (token, slot)
+  int T, k;                // GLU_GATHER: tokens, top_k
   int E, h, f;
   int n_tiles;   // row-block modes: column tiles per unit
   int k_iters;   // row-block modes: 64-wide K steps per tile
@@ -160,6 +180,21 @@ __device__ __forceinline__ Tile decode(const GemmParams &p, int t, const int *us
   tl.row0 = tl.dummy ? p.nblk_cap * BM : b * BM;  // a dummy half reads rows past P_max: zeros
   tl.kit = p.k_iters;
   return tl;
+}
+
+// GLU_GATHER: the token rows (rows of x) behind padded rows row0 + 4*lane .. +3 of this
+// CTA's block; padding rows and a dummy half get T, past the last row of x: TMA reads zeros.
+__device__ __forceinline__ void gather_rows(const GemmParams &p, const Tile &tl, int lane,
+                                            int (&rows)[4]) {
+  const int e = tl.e;
+  const int pstart = (e > 0) ? p.padded_bins[e - 1] : 0;
+  const int bstart = (e > 0) ? p.bins[e - 1] : 0;
+  const int count = p.bins[e] - bstart;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int local = tl.row0 + 4 * lane + i - pstart;  // position inside the expert's rows
+    rows[i] = (!tl.dummy && local < count) ? p.indices[bstart + local] / p.k : p.T;
+  }
 }
 
 template <int MODE>
@@ -247,7 +282,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
                                               Stager<Cfg<MODE, EPI>::out_bufs> &st) {
   const int y0 = tl.row0 + sub * 32;  // first row of this warp's boxes
   constexpr int kw = BN / Cfg<MODE, EPI>::col_split;  // accumulator columns per warp (non-GLU)
-  if (MODE == MODE_GLU) {
+  if (is_glu(MODE)) {
     const int n0 = tl.n * (BN / 2);
 #pragma unroll 1
     for (int c = 0; c < BN / 2; c += 64) {  // one 64-column box of H (and of A, Bm)
@@ -434,23 +469,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
   const uint32_t leader_full0 = mapa_shared(smem_u32(&full[0]), 0);
   const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0) {
     // ---------------- TMA producer (both CTAs) ----------------
+    // Lane 0 waits for free stages and issues the tile loads; in GLU_GATHER mode every lane
+    // also issues one 4-row gather of the A tile (32 x 4 = 128 rows).
     int stage = 0;
     uint32_t phase = 0;
     long long issued = 0;
+    int rows[4] = {0, 0, 0, 0};
     for (int t = cluster; t < total; t += nclusters) {
       const Tile tl = decode<MODE>(p, t, ustart, rank);
+      if (MODE == MODE_GLU_GATHER) gather_rows(p, tl, lane, rows);
       bool ok = true;
       for (int kb = 0; kb < tl.kit; ++kb) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, p.status, abort_flag)) {
+        int good = 1;
+        if (lane == 0) good = mbar_wait(&empty[stage], phase ^ 1u, p.status, abort_flag) ? 1 : 0;
+        if (!__shfl_sync(0xFFFFFFFFu, good, 0)) {
           ok = false;
           break;
         }
-        if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
         uint8_t *sa = tiles + stage * STAGE_BYTES;
-        load_stage<MODE>(p, tl, kb, rank, sa, sa + A_BYTES,
-                         leader_full0 + (uint32_t)(stage * sizeof(uint64_t)));
+        const uint32_t bar = leader_full0 + (uint32_t)(stage * sizeof(uint64_t));
+        if (lane == 0 && leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+        if (MODE == MODE_GLU_GATHER) {
+          tma_gather4_pair(sa + lane * 4 * 128, &p.tm[3], bar, kb * BK, rows[0], rows[1], rows[2],
+                           rows[3]);
+          if (lane == 0)
+            tma_load_2d_pair(sa + A_BYTES, &p.tm[rank == 0 ? 1 : 2], bar, kb * BK,
+                             tl.e * p.f + tl.n * (BN / 2));
+        } else if (lane == 0) {
+          load_stage<MODE>(p, tl, kb, rank, sa, sa + A_BYTES, bar);
+        }
         ++issued;
         if (++stage == STAGES) {
           stage = 0;
@@ -459,7 +508,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
       }
       if (!ok) break;
     }
-    if (leader)  // every issued copy (of both CTAs) has landed before the pair may exit
+    if (lane == 0 && leader)  // every issued copy (of both CTAs) has landed before exit
       for (long long i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
         mbar_wait_plain(&full[i % STAGES], (uint32_t)((i / STAGES) & 1));
   } else if (warp == 1 && lane == 0 && leader) {
@@ -635,6 +684,10 @@ static GemmParams base_params(const GemmProblem &g) {
   GemmParams p;
   memset(&p, 0, sizeof(p));
   p.padded_bins = g.padded_bins;
+  p.bins = g.bins;
+  p.indices = g.indices;
+  p.T = g.T;
+  p.k = g.k;
   p.E = g.E;
   p.h = g.h;
   p.f = g.f;
@@ -666,6 +719,28 @@ cudaError_t launch_glu_gemm(const GemmProblem &g, const void *x_pad, const void 
   p.k_iters = g.h / BK;
   p.group = raster_units(g.h);
   return launch_gemm<MODE_GLU, 4>(p, max_units(g) * p.n_tiles, st);
+}
+
+cudaError_t launch_glu_gather_gemm(const GemmProblem &g, const void *x, const void *w1,
+                                   const void *w3, void *h_out, void *a_out, void *b_out,
+                                   cudaStream_t st) {
+  GemmParams p = base_params(g);
+  const uint64_t P = (uint64_t)g.nblk_cap * BM;
+  const uint64_t EF = (uint64_t)g.E * g.f;
+  if (!make_tmap(&p.tm[3], x, (uint64_t)g.T, g.h, 1) ||
+      !make_tmap(&p.tm[1], w1, EF, g.h, BN / 2) || !make_tmap(&p.tm[2], w3, EF, g.h, BN / 2) ||
+      !make_tmap(&p.tmo[0], h_out, P, g.f, 32))
+    return cudaErrorInvalidValue;
+  if (a_out && b_out) {
+    if (!make_tmap(&p.tmo[1], a_out, P, g.f, 32) || !make_tmap(&p.tmo[2], b_out, P, g.f, 32))
+      return cudaErrorInvalidValue;
+    p.outs = 3;
+  }
+  p.tm[0] = p.tm[4] = p.tm[3];
+  p.n_tiles = g.f / (BN / 2);
+  p.k_iters = g.h / BK;
+  p.group = raster_units(g.h);
+  return launch_gemm<MODE_GLU_GATHER, 4>(p, max_units(g) * p.n_tiles, st);
 }
 
 cudaError_t launch_down_gemm(const GemmProblem &g, const void *h_in, const void *w2, void *y_pad,

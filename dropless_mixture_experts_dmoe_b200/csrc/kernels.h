@@ -49,9 +49,12 @@ cudaError_t launch_dy_gather(int T, int h, int k, int E, const void *dy, const i
 // Shape and map pointers shared by the grouped GEMM launchers.
 struct GemmProblem {
   int h, f, E, nblk_cap;
+  int T, k;
   const int32_t *num_blocks;
   const int32_t *block_expert;
   const int32_t *padded_bins;
+  const int32_t *bins;
+  const int32_t *indices;
   int32_t *status;
 };
 
@@ -59,6 +62,9 @@ struct GemmProblem {
 cudaError_t launch_glu_gemm(const GemmProblem &g, const void *x_pad, const void *w1,
                             const void *w3, void *h_out, void *a_out, void *b_out,
                             cudaStream_t st);
+cudaError_t launch_glu_gather_gemm(const GemmProblem &g, const void *x, const void *w1,
+                                   const void *w3, void *h_out, void *a_out, void *b_out,
+                                   cudaStream_t st);
 cudaError_t launch_down_gemm(const GemmProblem &g, const void *h_in, const void *w2, void *y_pad,
                              cudaStream_t st);
 // ... and the backward: dH with the fused dGLU epilogue, dX, and the weight gradients.

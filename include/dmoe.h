@@ -214,6 +214,17 @@ DMOE_API int dmoe_padded_gather(const dmoe_dims *dims, const void *x, const dmoe
 DMOE_API int dmoe_expert_glu(const dmoe_dims *dims, const void *x_pad, const void *w1, const void *w3,
                     const dmoe_map *map, void *h_out, void *a_out, void *b_out, void *stream);
 
+/* GLU GEMM with the padded gather fused into its operand load (walkthrough section 4.2's
+ * gather, out[index_b] = x[index_a // TOP_K], done by the GEMM's TMA row gathers, four rows
+ * per instruction): the same results as dmoe_padded_gather followed by dmoe_expert_glu, bit
+ * for bit, and X_pad is never written or read.  x [T,h] bf16 -> h_out (a_out, b_out: both or
+ * neither) [P_max,f] bf16.  Measured on B200 it is about 3x slower than the gather kernel +
+ * dmoe_expert_glu (the row-gather instruction rate cannot feed the MMAs), so dmoe_forward
+ * does not use it; it serves callers that cannot hold the X_pad buffer. */
+DMOE_API int dmoe_expert_glu_gather(const dmoe_dims *dims, const void *x, const void *w1,
+                                    const void *w3, const dmoe_map *map, void *h_out, void *a_out,
+                                    void *b_out, void *stream);
+
 /* Down GEMM: Y_pad[b] = bf16(H[b] W2_e^T) for every block b < num_blocks.
  * h_in [P_max,f] -> y_pad [P_max,h], bf16. */
 DMOE_API int dmoe_expert_down(const dmoe_dims *dims, const void *h_in, const void *w2,

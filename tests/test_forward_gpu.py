@@ -92,6 +92,25 @@ def test_forward_sampled_parity_full_size(num):
     assert torch.isfinite(y.float()).all()
 
 
+@pytest.mark.parametrize("w", SMALL + [WORKLOADS[3]], ids=lambda w: w.describe())
+def test_gathered_glu_matches_padded_glu(w):
+    """The GLU GEMM that gathers its rows from x must equal, bit for bit, gather + GLU on the
+    materialised X_pad (padding rows, odd last blocks and all)."""
+    inp = make_inputs(w)
+    dims = dims_of(w)
+    bufs, dev, y = gpu_forward(dims, inp, train=True)
+    P = bufs.P
+    h2 = torch.full((P, w.ffn), float("nan"), dtype=torch.bfloat16, device="cuda")
+    a2 = torch.full_like(h2, float("nan"))
+    b2 = torch.full_like(h2, float("nan"))
+    B.dmoe_expert_glu_gather(dims, dev["x"], dev["w1"], dev["w3"], bufs.map, h2, a2, b2)
+    torch.cuda.synchronize()
+    rows = int(bufs.map.num_blocks.item()) * 128
+    for name, got in (("h", h2), ("a", a2), ("bm", b2)):
+        ref = bufs.view(name)[:rows]
+        assert torch.equal(got[:rows].view(torch.int16), ref.view(torch.int16)), name
+
+
 def test_forward_deterministic():
     w = SMALL[1]
     inp = make_inputs(w)
