@@ -97,6 +97,8 @@ def load():
     lib.dmoe_status_string.restype = ctypes.c_char_p
     lib.dmoe_version.argtypes = []
     lib.dmoe_version.restype = ctypes.c_char_p
+    lib.dmoe_debug_inject_stall.argtypes = [_I]
+    lib.dmoe_debug_inject_stall.restype = _I
     _lib = lib
     return lib
 
@@ -111,6 +113,12 @@ def status_string(status: int) -> str:
 
 def version() -> str:
     return load().dmoe_version().decode()
+
+
+def dmoe_debug_inject_stall(enable: bool = True) -> None:
+    """Test-only: the next grouped-GEMM launch stalls on purpose and reports
+    STATUS_TIMEOUT (see include/dmoe.h)."""
+    _check(load().dmoe_debug_inject_stall(1 if enable else 0), "dmoe_debug_inject_stall")
 
 
 def make_dims(T: int, hidden: int, ffn: int, num_experts: int, top_k: int) -> dmoe_dims:

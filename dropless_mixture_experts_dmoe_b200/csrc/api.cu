@@ -402,4 +402,9 @@ const char *dmoe_status_string(int32_t status) {
 
 const char *dmoe_version(void) { return "dmoe-b200 0.1"; }
 
+int dmoe_debug_inject_stall(int enable) {
+  set_inject_stall(enable);
+  return DMOE_OK;
+}
+
 }  // extern "C"

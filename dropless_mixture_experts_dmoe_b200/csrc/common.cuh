@@ -23,6 +23,8 @@ constexpr int kBlock = DMOE_BLOCKING;  // rows per padded block
 
 // Cycle budget of one bounded wait (about a second at B200 clocks).
 constexpr long long kWaitCycles = 2000000000LL;
+// Budget used by a launch with a stall injected on purpose (a few milliseconds).
+constexpr long long kInjectedWaitCycles = 10000000LL;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -94,16 +96,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Returns false (and sets
-// DMOE_STATUS_TIMEOUT and *abort) if it did not within kWaitCycles or if *abort was raised by
-// another role of the same CTA.
+// DMOE_STATUS_TIMEOUT and *abort) if it did not within `limit` cycles or if *abort was raised
+// by another role of the same CTA.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status,
-                                          volatile int *abort) {
+                                          volatile int *abort, long long limit = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       set_status(status, DMOE_STATUS_TIMEOUT);
       *abort = 1;
       return false;
@@ -112,10 +114,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_
 }
 
 // Bounded wait used during teardown (no abort flag check).
-__device__ __forceinline__ bool mbar_wait_plain(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_plain(uint64_t *bar, uint32_t parity,
+                                                long long limit = kWaitCycles) {
   long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   }
   return true;
 }

@@ -50,6 +50,7 @@
 // abort flag for the other roles of its CTA, drains what it issued and returns.
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -112,6 +113,8 @@ struct GemmParams {
   int nblk_cap;  // P_max / 128: rows at or past nblk_cap * 128 read as zeros
   int group;     // row-block modes: units per raster chunk
   int outs;      // GLU: 1 (H) or 3 (H, A, Bm)
+  int inject;    // test-only: pair leaders withhold their first stage (waits then expire)
+  long long wait_cycles;  // budget of every bounded wait of this launch
   const __nv_bfloat16 *in0, *in1;  // DGLU: saved A, Bm
   int32_t *status;
 };
@@ -483,13 +486,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
       bool ok = true;
       for (int kb = 0; kb < tl.kit; ++kb) {
         int good = 1;
-        if (lane == 0) good = mbar_wait(&empty[stage], phase ^ 1u, p.status, abort_flag) ? 1 : 0;
+        if (lane == 0)
+          good = mbar_wait(&empty[stage], phase ^ 1u, p.status, abort_flag, p.wait_cycles) ? 1 : 0;
         if (!__shfl_sync(0xFFFFFFFFu, good, 0)) {
           ok = false;
           break;
         }
         uint8_t *sa = tiles + stage * STAGE_BYTES;
         const uint32_t bar = leader_full0 + (uint32_t)(stage * sizeof(uint64_t));
+        if (p.inject && leader && issued == 0 && kb == 0) {
+          // test-only stall: this stage is never armed, so the MMA's wait on it expires
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          ++issued;
+          continue;
+        }
         if (lane == 0 && leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
         if (MODE == MODE_GLU_GATHER) {
           tma_gather4_pair(sa + lane * 4 * 128, &p.tm[3], bar, kb * BK, rows[0], rows[1], rows[2],
@@ -510,7 +523,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
     }
     if (lane == 0 && leader)  // every issued copy (of both CTAs) has landed before exit
       for (long long i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
-        mbar_wait_plain(&full[i % STAGES], (uint32_t)((i / STAGES) & 1));
+        mbar_wait_plain(&full[i % STAGES], (uint32_t)((i / STAGES) & 1), p.wait_cycles);
   } else if (warp == 1 && lane == 0 && leader) {
     // ---------------- MMA issuer (leader only) ----------------
     constexpr uint32_t idesc =
@@ -522,12 +535,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
     for (int t = cluster; t < total; t += nclusters) {
       const Tile tl = decode<MODE>(p, t, ustart, rank);
       if (tl.kit == 0) continue;  // weight gradient of an expert without rows: no MMA
-      if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.status, abort_flag)) break;
+      if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.status, abort_flag, p.wait_cycles)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
       bool ok = true;
       for (int kb = 0; kb < tl.kit; ++kb) {
-        if (!mbar_wait(&full[stage], phase, p.status, abort_flag)) {
+        if (!mbar_wait(&full[stage], phase, p.status, abort_flag, p.wait_cycles)) {
           ok = false;
           break;
         }
@@ -556,7 +569,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
       if (acc == 0) acc_phase ^= 1u;
     }
     tc_commit_pair(drain);
-    mbar_wait_plain(drain, 0);
+    mbar_wait_plain(drain, 0, p.wait_cycles);
   } else if (warp >= 2) {
     // ---------------- epilogue (both CTAs) ----------------
     const int sub = warp & 3;           // TMEM sub-partition this warp may read
@@ -573,7 +586,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
         if (!tl.dummy) epilogue_tile<MODE, EPI>(p, tl, 0u, sub, half, lane, st);
         continue;
       }
-      if (!mbar_wait(&tfull[acc], acc_phase, p.status, abort_flag)) break;
+      if (!mbar_wait(&tfull[acc], acc_phase, p.status, abort_flag, p.wait_cycles)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * ACC_COLS);
       if (!tl.dummy) epilogue_tile<MODE, EPI>(p, tl, tb, sub, half, lane, st);
@@ -652,9 +665,17 @@ static int raster_units(int K) {
   return (int)g;
 }
 
+// Test-only stall injection (dmoe_debug_inject_stall): consumed by the next GEMM launch.
+static std::atomic<int> g_inject_stall{0};
+
+void set_inject_stall(int on) { g_inject_stall.store(on ? 1 : 0); }
+
 template <int MODE, int EPI>
-static cudaError_t launch_gemm(const GemmParams &p, long long max_tiles, cudaStream_t st) {
+static cudaError_t launch_gemm(const GemmParams &p_in, long long max_tiles, cudaStream_t st) {
   using C = Cfg<MODE, EPI>;
+  GemmParams p = p_in;
+  p.inject = g_inject_stall.exchange(0);
+  p.wait_cycles = p.inject ? kInjectedWaitCycles : kWaitCycles;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   static int max_clusters = 0;

@@ -79,4 +79,7 @@ cudaError_t launch_wgrad_gemm(const GemmProblem &g, const void *x_pad, const voi
 
 int device_sm_count();
 
+// Test-only: make the next grouped-GEMM launch stall on purpose (see dmoe_debug_inject_stall).
+void set_inject_stall(int on);
+
 }  // namespace dmoe

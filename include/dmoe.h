@@ -280,6 +280,15 @@ DMOE_API const char *dmoe_status_string(int32_t status);
 /* Library version, e.g. "dmoe-b200 0.1". */
 DMOE_API const char *dmoe_version(void);
 
+/* Test-only fault injection (no counterpart on the pages; it exercises the library's own
+ * failure path).  With enable != 0, the NEXT grouped-GEMM launch of this process (any GEMM
+ * step) runs with a wait budget of ~10^7 cycles and its pair leaders withhold their first
+ * operand stage: the MMA's bounded wait on that stage expires, the kernel sets
+ * DMOE_STATUS_TIMEOUT in map->status, every role of every CTA leaves through its own
+ * bounded waits, and the launch returns normally with that launch's results invalid.  No
+ * trap, no fault; the context stays usable.  The switch clears itself on that launch. */
+DMOE_API int dmoe_debug_inject_stall(int enable);
+
 #ifdef __cplusplus
 }
 #endif
