@@ -278,16 +278,18 @@ def run_ours(args, w):
         i += 1
         mark(i)
         if train:
-            B.dmoe_bwd_dy_gather(dims, dev["dy"], bufs.map, yp, bs["dy_pad"], grads["dw"], st)
+            # the sequence of dmoe_backward, dX_pad reusing dY_pad's buffer as it does
+            B.dmoe_padded_gather(dims, dev["dy"], bufs.map, bs["dy_pad"], st)
             mark(i + 1)
-            B.dmoe_bwd_dglu(dims, bs["dy_pad"], dev["w2"], ab, bb, bufs.map, bs["da"], bs["dbm"], st)
+            B.dmoe_bwd_dglu(dims, bs["dy_pad"], dev["w2"], ab, bb, bufs.map, bs["da"], bs["dbm"],
+                            bs["hw"], bs["dw_part"], st)
             mark(i + 2)
-            B.dmoe_bwd_wgrad(dims, xp, hb, bs["dy_pad"], bs["da"], bs["dbm"], bufs.map,
+            B.dmoe_bwd_wgrad(dims, xp, bs["hw"], bs["dy_pad"], bs["da"], bs["dbm"], bufs.map,
                              grads["dw1"], grads["dw3"], grads["dw2"], st)
             mark(i + 3)
-            B.dmoe_bwd_dx(dims, bs["da"], bs["dbm"], dev["w1"], dev["w3"], bufs.map, bs["dx_pad"], st)
+            B.dmoe_bwd_dx(dims, bs["da"], bs["dbm"], dev["w1"], dev["w3"], bufs.map, bs["dy_pad"], st)
             mark(i + 4)
-            B.dmoe_padded_scatter(dims, bs["dx_pad"], bufs.map, None, grads["dx"], st)
+            B.dmoe_bwd_scatter(dims, bs["dy_pad"], bs["dw_part"], bufs.map, grads["dx"], grads["dw"], st)
             mark(i + 5)
 
     for _ in range(args.warmup):
@@ -365,7 +367,7 @@ def run_ours(args, w):
         B.dmoe_sparse_map(dims, lg_d[j], bufs.map, bufs.ws_map, st)
         if train:
             B.dmoe_forward(dims, x_d[j], dev["w1"], dev["w3"], dev["w2"], bufs.map, y_d[j], bufs.saved,
-                           None, st)
+                           bufs.ws_fwd, st)
             B.dmoe_backward(dims, dy_d[j], dev["w1"], dev["w3"], dev["w2"], bufs.map, bufs.saved,
                             dx_d[j], grads["dw1"], grads["dw3"], grads["dw2"], grads["dw"],
                             bufs.ws_bwd, st)
@@ -430,8 +432,9 @@ def run_ours(args, w):
         map=2 * w.T * w.E + 8 * w.T * w.top_k + 12 * N,
         gather=2 * w.T * w.hidden + 2 * N * w.hidden,
         scatter=2 * N * w.hidden + 8 * N + 4 * N + 2 * w.T * w.hidden,
-        dy_gather=2 * w.T * w.hidden + 4 * N * w.hidden + 12 * N,
-        dx_scatter=2 * N * w.hidden + 4 * N + 2 * w.T * w.hidden)
+        dy_gather=2 * w.T * w.hidden + 2 * N * w.hidden,
+        dx_scatter=2 * N * w.hidden + 4 * N + 2 * w.T * w.hidden
+        + 4 * N * ((w.ffn + 255) // 256) + 4 * N)
     km = {n: statistics.mean(v) for n, v in per_kernel.items()}
     kernels = {}
     for n in names:

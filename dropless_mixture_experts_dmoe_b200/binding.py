@@ -20,7 +20,8 @@ BLOCKING = 128
 MAX_EXPERTS = 1024
 MAX_TOP_K = 32
 
-WS_MAP, WS_FORWARD, WS_BACKWARD = 0, 1, 2
+WS_MAP, WS_FORWARD, WS_BACKWARD, WS_FORWARD_TRAIN = 0, 1, 2, 3
+DGLU_TILE_COLS = 256
 
 STATUS_NONFINITE_LOGITS = 0x1
 STATUS_EXPERT_OUT_OF_RANGE = 0x2
@@ -83,13 +84,13 @@ def load():
     lib.dmoe_expert_glu_gather.argtypes = [D, _P, _P, _P, M, _P, _P, _P, _P]
     lib.dmoe_expert_down.argtypes = [D, _P, _P, M, _P, _P]
     lib.dmoe_padded_scatter.argtypes = [D, _P, M, _P, _P, _P]
-    lib.dmoe_bwd_dy_gather.argtypes = [D, _P, M, _P, _P, _P, _P]
-    lib.dmoe_bwd_dglu.argtypes = [D, _P, _P, _P, _P, M, _P, _P, _P]
+    lib.dmoe_bwd_dglu.argtypes = [D, _P, _P, _P, _P, M, _P, _P, _P, _P, _P]
+    lib.dmoe_bwd_scatter.argtypes = [D, _P, _P, M, _P, _P, _P]
     lib.dmoe_bwd_dx.argtypes = [D, _P, _P, _P, _P, M, _P, _P]
     lib.dmoe_bwd_wgrad.argtypes = [D, _P, _P, _P, _P, _P, M, _P, _P, _P, _P]
     for fn in ("dmoe_sparse_map", "dmoe_forward", "dmoe_backward", "dmoe_padded_gather",
-               "dmoe_expert_glu", "dmoe_expert_glu_gather", "dmoe_expert_down", "dmoe_padded_scatter", "dmoe_bwd_dy_gather",
-               "dmoe_bwd_dglu", "dmoe_bwd_dx", "dmoe_bwd_wgrad"):
+               "dmoe_expert_glu", "dmoe_expert_glu_gather", "dmoe_expert_down", "dmoe_padded_scatter",
+               "dmoe_bwd_dglu", "dmoe_bwd_dx", "dmoe_bwd_wgrad", "dmoe_bwd_scatter"):
         getattr(lib, fn).restype = _I
     lib.dmoe_error_string.argtypes = [_I]
     lib.dmoe_error_string.restype = ctypes.c_char_p
@@ -157,7 +158,7 @@ def dmoe_workspace_bytes(dims: dmoe_dims, kind: int) -> int:
 
 
 def dmoe_saved_bytes(dims: dmoe_dims):
-    offs = (_SZ * 5)()
+    offs = (_SZ * 3)()
     total = int(load().dmoe_saved_bytes(ctypes.byref(dims), offs))
     return total, [int(o) for o in offs]
 
@@ -251,16 +252,17 @@ def dmoe_padded_scatter(dims, y_pad, smap: SparseMap, weights, y, stream=None):
            "dmoe_padded_scatter")
 
 
-def dmoe_bwd_dy_gather(dims, dy, smap: SparseMap, y_pad, dy_pad, dweights, stream=None):
-    _check(load().dmoe_bwd_dy_gather(ctypes.byref(dims), _ptr(dy), ctypes.byref(smap.c), _ptr(y_pad),
-                                     _ptr(dy_pad), _ptr(dweights), _stream(stream)),
-           "dmoe_bwd_dy_gather")
-
-
-def dmoe_bwd_dglu(dims, dy_pad, w2, a_saved, bm_saved, smap: SparseMap, da, dbm, stream=None):
+def dmoe_bwd_dglu(dims, dy_pad, w2, a_saved, bm_saved, smap: SparseMap, da, dbm, hw, dw_part,
+                  stream=None):
     _check(load().dmoe_bwd_dglu(ctypes.byref(dims), _ptr(dy_pad), _ptr(w2), _ptr(a_saved),
                                 _ptr(bm_saved), ctypes.byref(smap.c), _ptr(da), _ptr(dbm),
-                                _stream(stream)), "dmoe_bwd_dglu")
+                                _ptr(hw), _ptr(dw_part), _stream(stream)), "dmoe_bwd_dglu")
+
+
+def dmoe_bwd_scatter(dims, dx_pad, dw_part, smap: SparseMap, dx, dweights, stream=None):
+    _check(load().dmoe_bwd_scatter(ctypes.byref(dims), _ptr(dx_pad), _ptr(dw_part),
+                                   ctypes.byref(smap.c), _ptr(dx), _ptr(dweights),
+                                   _stream(stream)), "dmoe_bwd_scatter")
 
 
 def dmoe_bwd_dx(dims, da, dbm, w1, w3, smap: SparseMap, dx_pad, stream=None):
@@ -268,9 +270,9 @@ def dmoe_bwd_dx(dims, da, dbm, w1, w3, smap: SparseMap, dx_pad, stream=None):
                               ctypes.byref(smap.c), _ptr(dx_pad), _stream(stream)), "dmoe_bwd_dx")
 
 
-def dmoe_bwd_wgrad(dims, x_pad, h_saved, dy_pad, da, dbm, smap: SparseMap, dw1, dw3, dw2,
+def dmoe_bwd_wgrad(dims, x_pad, hw, dy_pad, da, dbm, smap: SparseMap, dw1, dw3, dw2,
                    stream=None):
-    _check(load().dmoe_bwd_wgrad(ctypes.byref(dims), _ptr(x_pad), _ptr(h_saved), _ptr(dy_pad),
+    _check(load().dmoe_bwd_wgrad(ctypes.byref(dims), _ptr(x_pad), _ptr(hw), _ptr(dy_pad),
                                  _ptr(da), _ptr(dbm), ctypes.byref(smap.c), _ptr(dw1), _ptr(dw3),
                                  _ptr(dw2), _stream(stream)), "dmoe_bwd_wgrad")
 
@@ -290,10 +292,13 @@ def dmoe_sparse_map_noalloc(dims: dmoe_dims, logits, smap: SparseMap, stream=Non
 class Buffers:
     """Caller-side device allocations for one layer shape: map, workspaces, saved activations.
 
-    train=True: ``saved`` (X_pad, A, Bm, H, Y_pad for the backward) and the backward
-    workspace; ``view(name)`` gives bf16 views of the saved activations.
-    train=False: the inference workspace of ``dmoe_forward`` plus separate X_pad / H / Y_pad
-    tensors (``step``) for driving the step entry points one by one."""
+    train=True: ``saved`` (X_pad, A, Bm for the backward), the training forward workspace
+    ``ws_fwd`` (H, Y_pad), the backward workspace, and separate step buffers ``bstep``
+    (dy_pad, da, dbm, hw, dw_part, dx_pad) for driving the backward step entry points one by
+    one.  train=False: the inference workspace of ``dmoe_forward`` plus separate X_pad / H /
+    Y_pad tensors (``step``) for the forward step entry points.  ``view(name)`` gives bf16
+    [P_max, cols] views: x_pad, a, bm of the saved buffer, and h, y_pad of the forward
+    workspace (valid until the workspace is reused)."""
 
     def __init__(self, dims: dmoe_dims, train: bool = False, device="cuda"):
         self.dims = dims
@@ -303,28 +308,35 @@ class Buffers:
         self.ws_map = torch.empty(max(dmoe_workspace_bytes(dims, WS_MAP), 16), **u8)
         self.train = train
         P, h, f = self.P, dims.hidden, dims.ffn
-        self.saved = self.ws_fwd = self.ws_bwd = None
+        bf = dict(dtype=torch.bfloat16, device=device)
+        self.saved = self.ws_bwd = None
         self.step = {}
         if train:
             total, offs = dmoe_saved_bytes(dims)
             self.saved = torch.empty(total, **u8)
-            self.offsets = dict(x_pad=offs[0], a=offs[1], bm=offs[2], h=offs[3], y_pad=offs[4])
+            self.offsets = dict(x_pad=offs[0], a=offs[1], bm=offs[2])
+            self.ws_fwd = torch.empty(dmoe_workspace_bytes(dims, WS_FORWARD_TRAIN), **u8)
             self.ws_bwd = torch.empty(max(dmoe_workspace_bytes(dims, WS_BACKWARD), 16), **u8)
-            bf = dict(dtype=torch.bfloat16, device=device)
-            # separate step buffers for driving the backward step entry points one by one
+            nt = (f + DGLU_TILE_COLS - 1) // DGLU_TILE_COLS
             self.bstep = dict(dy_pad=torch.empty((P, h), **bf), da=torch.empty((P, f), **bf),
-                              dbm=torch.empty((P, f), **bf), dx_pad=torch.empty((P, h), **bf))
+                              dbm=torch.empty((P, f), **bf), hw=torch.empty((P, f), **bf),
+                              dw_part=torch.empty((P, nt), dtype=torch.float32, device=device),
+                              dx_pad=torch.empty((P, h), **bf))
         else:
             self.ws_fwd = torch.empty(dmoe_workspace_bytes(dims, WS_FORWARD), **u8)
-            bf = dict(dtype=torch.bfloat16, device=device)
             self.step = dict(x_pad=torch.empty((P, h), **bf), h=torch.empty((P, f), **bf),
                              y_pad=torch.empty((P, h), **bf))
 
     def view(self, name: str) -> torch.Tensor:
-        """bf16 [P, cols] view of a saved activation (train=True only)."""
+        """bf16 [P, cols] view of a saved activation (x_pad, a, bm) or, after a training
+        forward, of its workspace (h, y_pad)."""
         if not self.train:
             return self.step[name]
-        off = self.offsets[name]
         cols = self.dims.hidden if name in ("x_pad", "y_pad") else self.dims.ffn
         n = self.P * cols * 2
-        return self.saved[off:off + n].view(torch.bfloat16).view(self.P, cols)
+        if name in self.offsets:
+            off = self.offsets[name]
+            return self.saved[off:off + n].view(torch.bfloat16).view(self.P, cols)
+        # forward workspace layout: H [P,f] | Y_pad [P,h], each start aligned to 256 bytes
+        off = 0 if name == "h" else (self.P * self.dims.ffn * 2 + 255) // 256 * 256
+        return self.ws_fwd[off:off + n].view(torch.bfloat16).view(self.P, cols)

@@ -70,6 +70,7 @@ GemmProblem problem_of(const dmoe_dims *d, const dmoe_map *m) {
   g.k = d->top_k;
   g.bins = m->bins;
   g.indices = m->indices;
+  g.weights = m->weights;
   g.num_blocks = m->num_blocks;
   g.block_expert = m->block_expert;
   g.padded_bins = m->padded_bins;
@@ -77,9 +78,12 @@ GemmProblem problem_of(const dmoe_dims *d, const dmoe_map *m) {
   return g;
 }
 
-// Backward workspace layout: dY_pad [P,h] | dA [P,f] | dBm [P,f] | dX_pad [P,h]
+inline int dglu_tiles(const dmoe_dims *d) { return (d->ffn + kDgluTileCols - 1) / kDgluTileCols; }
+
+// Backward workspace layout: dY_pad [P,h] (reused for dX_pad once the weight gradients have
+// read it) | dA [P,f] | dBm [P,f] | Hw [P,f] | routing-weight partials [P, ceil(f/256)] fp32
 struct BwdLayout {
-  size_t dy, da, db, dx, total;
+  size_t dy, da, db, hw, part, total;
 };
 BwdLayout bwd_layout(const dmoe_dims *d) {
   const size_t P = (size_t)pmax_of(d);
@@ -87,34 +91,35 @@ BwdLayout bwd_layout(const dmoe_dims *d) {
   l.dy = 0;
   l.da = align_up(l.dy + P * d->hidden * 2);
   l.db = align_up(l.da + P * d->ffn * 2);
-  l.dx = align_up(l.db + P * d->ffn * 2);
-  l.total = align_up(l.dx + P * d->hidden * 2);
+  l.hw = align_up(l.db + P * d->ffn * 2);
+  l.part = align_up(l.hw + P * d->ffn * 2);
+  l.total = align_up(l.part + P * dglu_tiles(d) * sizeof(float));
   return l;
 }
 
-// Forward workspace layout (inference): X_pad [P,h] | H [P,f] | Y_pad [P,h]
+// Forward workspace layout: H [P,f] | Y_pad [P,h] | X_pad [P,h].  A training forward keeps
+// X_pad in the saved buffer and uses only the first two (`train` bytes).
 struct FwdLayout {
-  size_t xpad, h, ypad, total;
+  size_t h, ypad, xpad, train, total;
 };
 FwdLayout fwd_layout(const dmoe_dims *d) {
   const size_t P = (size_t)pmax_of(d);
   FwdLayout l;
-  l.xpad = 0;
-  l.h = align_up(l.xpad + P * d->hidden * 2);
+  l.h = 0;
   l.ypad = align_up(l.h + P * d->ffn * 2);
-  l.total = align_up(l.ypad + P * d->hidden * 2);
+  l.xpad = align_up(l.ypad + P * d->hidden * 2);
+  l.train = l.xpad;
+  l.total = align_up(l.xpad + P * d->hidden * 2);
   return l;
 }
 
-// Saved activations: X_pad [P,h] | A [P,f] | Bm [P,f] | H [P,f] | Y_pad [P,h]
-void saved_layout(const dmoe_dims *d, size_t off[5], size_t *total) {
+// Saved activations: X_pad [P,h] | A [P,f] | Bm [P,f]
+void saved_layout(const dmoe_dims *d, size_t off[3], size_t *total) {
   const size_t P = (size_t)pmax_of(d);
   off[0] = 0;
   off[1] = align_up(off[0] + P * d->hidden * 2);
   off[2] = align_up(off[1] + P * d->ffn * 2);
-  off[3] = align_up(off[2] + P * d->ffn * 2);
-  off[4] = align_up(off[3] + P * d->ffn * 2);
-  *total = align_up(off[4] + P * d->hidden * 2);
+  *total = align_up(off[2] + P * d->ffn * 2);
 }
 
 }  // namespace
@@ -133,6 +138,8 @@ size_t dmoe_workspace_bytes(const dmoe_dims *dims, int kind) {
       return align_up(sizeof(int32_t) * map_workspace_ints(dims->T, dims->num_experts));
     case DMOE_WS_FORWARD:
       return fwd_layout(dims).total;
+    case DMOE_WS_FORWARD_TRAIN:
+      return fwd_layout(dims).train;
     case DMOE_WS_BACKWARD:
       return bwd_layout(dims).total;
     default:
@@ -140,12 +147,12 @@ size_t dmoe_workspace_bytes(const dmoe_dims *dims, int kind) {
   }
 }
 
-size_t dmoe_saved_bytes(const dmoe_dims *dims, size_t offsets[5]) {
+size_t dmoe_saved_bytes(const dmoe_dims *dims, size_t offsets[3]) {
   if (check_dims(dims) != DMOE_OK) return 0;
-  size_t off[5], total;
+  size_t off[3], total;
   saved_layout(dims, off, &total);
   if (offsets)
-    for (int i = 0; i < 5; ++i) offsets[i] = off[i];
+    for (int i = 0; i < 3; ++i) offsets[i] = off[i];
   return total;
 }
 
@@ -252,27 +259,22 @@ int dmoe_forward(const dmoe_dims *dims, const void *x, const void *w1, const voi
   if (rc) return rc;
   if ((rc = check_map(map, true))) return rc;
   if (!x || !w1 || !w3 || !w2 || !y) return DMOE_ERR_NULL;
-  uint8_t *xpad, *hbuf, *ypad, *abuf = nullptr, *bbuf = nullptr;
+  if (!ws) return DMOE_ERR_NULL;
+  const FwdLayout l = fwd_layout(dims);
+  if (ws_bytes < (saved ? l.train : l.total)) return DMOE_ERR_WORKSPACE;
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  uint8_t *xpad = w + l.xpad, *hbuf = w + l.h, *ypad = w + l.ypad, *abuf = nullptr,
+          *bbuf = nullptr;
   if (saved) {
-    size_t off[5], total;
+    size_t off[3], total;
     saved_layout(dims, off, &total);
     uint8_t *s = static_cast<uint8_t *>(saved);
     xpad = s + off[0];
     abuf = s + off[1];
     bbuf = s + off[2];
-    hbuf = s + off[3];
-    ypad = s + off[4];
-  } else {
-    if (!ws) return DMOE_ERR_NULL;
-    FwdLayout l = fwd_layout(dims);
-    if (ws_bytes < l.total) return DMOE_ERR_WORKSPACE;
-    uint8_t *w = static_cast<uint8_t *>(ws);
-    xpad = w + l.xpad;
-    hbuf = w + l.h;
-    ypad = w + l.ypad;
   }
   if (!aligned16(x) || !aligned16(w1) || !aligned16(w3) || !aligned16(w2) || !aligned16(y) ||
-      !aligned16(xpad) || !aligned16(map->weights))
+      !aligned16(ws) || !aligned16(xpad) || !aligned16(map->weights))
     return DMOE_ERR_ALIGN;
   // The separate token-major gather (about 80 % of HBM bandwidth) is faster than feeding the
   // GLU GEMM through TMA row gathers, whose instruction rate cannot keep up with the MMAs.
@@ -282,32 +284,33 @@ int dmoe_forward(const dmoe_dims *dims, const void *x, const void *w1, const voi
   return dmoe_padded_scatter(dims, ypad, map, map->weights, y, stream);
 }
 
-int dmoe_bwd_dy_gather(const dmoe_dims *dims, const void *dy, const dmoe_map *map,
-                       const void *y_pad, void *dy_pad, float *dweights, void *stream) {
+int dmoe_bwd_dglu(const dmoe_dims *dims, const void *dy_pad, const void *w2, const void *a_saved,
+                  const void *bm_saved, const dmoe_map *map, void *da, void *dbm, void *hw,
+                  float *dw_part, void *stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_map(map, true))) return rc;
-  if (!dy || !y_pad || !dy_pad || !dweights) return DMOE_ERR_NULL;
-  if (!aligned16(dy) || !aligned16(y_pad) || !aligned16(dy_pad)) return DMOE_ERR_ALIGN;
-  if ((rc = check_device())) return rc;
-  return launch_rc(launch_dy_gather(dims->T, dims->hidden, dims->top_k, dims->num_experts, dy,
-                                    map->dest_row, map->weights, map->tokens_per_expert,
-                                    map->padded_bins, y_pad, dy_pad, dweights,
-                                    static_cast<cudaStream_t>(stream)));
-}
-
-int dmoe_bwd_dglu(const dmoe_dims *dims, const void *dy_pad, const void *w2, const void *a_saved,
-                  const void *bm_saved, const dmoe_map *map, void *da, void *dbm, void *stream) {
-  int rc = check_dims(dims);
-  if (rc) return rc;
-  if ((rc = check_map(map, false))) return rc;
-  if (!dy_pad || !w2 || !a_saved || !bm_saved || !da || !dbm) return DMOE_ERR_NULL;
+  if (!dy_pad || !w2 || !a_saved || !bm_saved || !da || !dbm || !hw || !dw_part)
+    return DMOE_ERR_NULL;
   if (!aligned16(dy_pad) || !aligned16(w2) || !aligned16(a_saved) || !aligned16(bm_saved) ||
-      !aligned16(da) || !aligned16(dbm))
+      !aligned16(da) || !aligned16(dbm) || !aligned16(hw) || !aligned16(dw_part))
     return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
   return launch_rc(launch_dglu_gemm(problem_of(dims, map), dy_pad, w2, a_saved, bm_saved, da, dbm,
-                                    static_cast<cudaStream_t>(stream)));
+                                    hw, dw_part, static_cast<cudaStream_t>(stream)));
+}
+
+int dmoe_bwd_scatter(const dmoe_dims *dims, const void *dx_pad, const float *dw_part,
+                     const dmoe_map *map, void *dx, float *dweights, void *stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if ((rc = check_map(map, false))) return rc;
+  if (!dx_pad || !dw_part || !dx || !dweights) return DMOE_ERR_NULL;
+  if (!aligned16(dx_pad) || !aligned16(dx)) return DMOE_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return launch_rc(launch_bwd_scatter(dims->T, dims->hidden, dims->top_k, dx_pad, map->dest_row,
+                                      dw_part, dglu_tiles(dims), dx, dweights,
+                                      static_cast<cudaStream_t>(stream)));
 }
 
 int dmoe_bwd_dx(const dmoe_dims *dims, const void *da, const void *dbm, const void *w1,
@@ -323,18 +326,18 @@ int dmoe_bwd_dx(const dmoe_dims *dims, const void *da, const void *dbm, const vo
       launch_dx_gemm(problem_of(dims, map), da, dbm, w1, w3, dx_pad, static_cast<cudaStream_t>(stream)));
 }
 
-int dmoe_bwd_wgrad(const dmoe_dims *dims, const void *x_pad, const void *h_saved,
+int dmoe_bwd_wgrad(const dmoe_dims *dims, const void *x_pad, const void *hw,
                    const void *dy_pad, const void *da, const void *dbm, const dmoe_map *map,
                    float *dw1, float *dw3, float *dw2, void *stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_map(map, false))) return rc;
-  if (!x_pad || !h_saved || !dy_pad || !da || !dbm || !dw1 || !dw3 || !dw2) return DMOE_ERR_NULL;
-  if (!aligned16(x_pad) || !aligned16(h_saved) || !aligned16(dy_pad) || !aligned16(da) ||
+  if (!x_pad || !hw || !dy_pad || !da || !dbm || !dw1 || !dw3 || !dw2) return DMOE_ERR_NULL;
+  if (!aligned16(x_pad) || !aligned16(hw) || !aligned16(dy_pad) || !aligned16(da) ||
       !aligned16(dbm) || !aligned16(dw1) || !aligned16(dw3) || !aligned16(dw2))
     return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
-  return launch_rc(launch_wgrad_gemm(problem_of(dims, map), x_pad, h_saved, dy_pad, da, dbm, dw1,
+  return launch_rc(launch_wgrad_gemm(problem_of(dims, map), x_pad, hw, dy_pad, da, dbm, dw1,
                                      dw3, dw2, static_cast<cudaStream_t>(stream)));
 }
 
@@ -350,18 +353,19 @@ int dmoe_backward(const dmoe_dims *dims, const void *dy, const void *w1, const v
   const BwdLayout l = bwd_layout(dims);
   if (ws_bytes < l.total) return DMOE_ERR_WORKSPACE;
   if (!aligned16(saved) || !aligned16(ws) || !aligned16(dx)) return DMOE_ERR_ALIGN;
-  size_t off[5], total;
+  size_t off[3], total;
   saved_layout(dims, off, &total);
   const uint8_t *sv = static_cast<const uint8_t *>(saved);
-  const void *xpad = sv + off[0], *abuf = sv + off[1], *bbuf = sv + off[2], *hbuf = sv + off[3],
-             *ypad = sv + off[4];
+  const void *xpad = sv + off[0], *abuf = sv + off[1], *bbuf = sv + off[2];
   uint8_t *w = static_cast<uint8_t *>(ws);
-  void *dypad = w + l.dy, *da = w + l.da, *db = w + l.db, *dxpad = w + l.dx;
-  if ((rc = dmoe_bwd_dy_gather(dims, dy, map, ypad, dypad, dweights, stream))) return rc;
-  if ((rc = dmoe_bwd_dglu(dims, dypad, w2, abuf, bbuf, map, da, db, stream))) return rc;
-  if ((rc = dmoe_bwd_wgrad(dims, xpad, hbuf, dypad, da, db, map, dw1, dw3, dw2, stream))) return rc;
+  void *dypad = w + l.dy, *da = w + l.da, *db = w + l.db, *hw = w + l.hw;
+  float *part = reinterpret_cast<float *>(w + l.part);
+  void *dxpad = dypad;  // dY_pad is dead once the weight gradients have read it
+  if ((rc = dmoe_padded_gather(dims, dy, map, dypad, stream))) return rc;
+  if ((rc = dmoe_bwd_dglu(dims, dypad, w2, abuf, bbuf, map, da, db, hw, part, stream))) return rc;
+  if ((rc = dmoe_bwd_wgrad(dims, xpad, hw, dypad, da, db, map, dw1, dw3, dw2, stream))) return rc;
   if ((rc = dmoe_bwd_dx(dims, da, db, w1, w3, map, dxpad, stream))) return rc;
-  return dmoe_padded_scatter(dims, dxpad, map, nullptr, dx, stream);
+  return dmoe_bwd_scatter(dims, dxpad, part, map, dx, dweights, stream);
 }
 
 const char *dmoe_error_string(int code) {

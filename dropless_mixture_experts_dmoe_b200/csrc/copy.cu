@@ -85,11 +85,17 @@ __global__ void __launch_bounds__(kCopyThreads) k_gather(int T, int h, int k, in
 
 // y_t = sum_{s<k} w_ts * Y_pad[dest_row[t*k+s]]: fp32, slot order, one fused multiply-add per
 // slot and element, rounded once to bf16.  weights == NULL: w = 1.
+// Backward use (walkthrough section 4.2: the gradient of the gather is this scatter with w = 1,
+// and the routing weight's gradient is <dy_t, Y_ts>): with dweights != NULL the warp that
+// takes a token's first slice also sums the DGLU GEMM's per-column-tile partials of each entry,
+// dweights[t*k+s] = sum_{n<nt} part[dest_row[t*k+s] * nt + n], in column-tile order.
 __global__ void __launch_bounds__(kCopyThreads) k_combine(int T, int h, int k,
                                                           const uint4 *__restrict__ y_pad,
                                                           const int32_t *__restrict__ dest_row,
                                                           const float *__restrict__ weights,
-                                                          uint4 *__restrict__ y) {
+                                                          uint4 *__restrict__ y,
+                                                          const float *__restrict__ part, int nt,
+                                                          float *__restrict__ dweights) {
   const int lane = threadIdx.x & 31;
   const int vpr = h >> 3;
   const int S = (vpr + kSliceVecs - 1) / kSliceVecs;
@@ -102,6 +108,12 @@ __global__ void __launch_bounds__(kCopyThreads) k_combine(int T, int h, int k,
     const int ve = min(vpr, vs + kSliceVecs);
     const int d = (lane < k) ? dest_row[(size_t)t * k + lane] : -1;
     const float wl = (lane < k) ? (weights ? weights[(size_t)t * k + lane] : 1.0f) : 0.0f;
+    if (dweights && vs == 0 && lane < k) {
+      float g = 0.0f;
+      if (d >= 0)
+        for (int n = 0; n < nt; ++n) g += __ldg(part + (size_t)d * nt + n);
+      dweights[(size_t)t * k + lane] = g;  // 0 for an entry dropped from the map
+    }
     for (int v0 = vs; v0 < ve; v0 += 32 * kCombineVPL) {
       float acc[kCombineVPL][8];
 #pragma unroll
@@ -156,84 +168,6 @@ __global__ void __launch_bounds__(kCopyThreads) k_combine(int T, int h, int k,
   }
 }
 
-// Backward of the weighted scatter (walkthrough section 4.2: its gradient is a gather plus the
-// routing-weight gradient).  Warp per token: for each slot s with padded row r,
-//   dY_pad[r] = bf16(w_ts * dy_t)   and   dweights[t*k+s] = <dy_t, Y_pad[r]> (fp32 dot,
-// fixed lane order).  Work items past T zero the padding rows of every expert's last block,
-// like the forward gather, so the weight gradients never see stale rows.
-__global__ void __launch_bounds__(kCopyThreads) k_dy_gather(int T, int h, int k, int E,
-                                                            const uint4 *__restrict__ dy,
-                                                            const int32_t *__restrict__ dest_row,
-                                                            const float *__restrict__ weights,
-                                                            const int32_t *__restrict__ counts,
-                                                            const int32_t *__restrict__ padded_bins,
-                                                            const uint4 *__restrict__ y_pad,
-                                                            uint4 *__restrict__ dy_pad,
-                                                            float *__restrict__ dweights) {
-  const int lane = threadIdx.x & 31;
-  const int vpr = h >> 3;
-  const long long items = (long long)T + (long long)kBlock * E;
-  const long long nw = (long long)gridDim.x * kCopyWarps;
-  for (long long it = (long long)blockIdx.x * kCopyWarps + (threadIdx.x >> 5); it < items;
-       it += nw) {
-    if (it < T) {
-      const int t = (int)it;
-      const int d = (lane < k) ? dest_row[(size_t)t * k + lane] : -1;
-      const float wl = (lane < k) ? weights[(size_t)t * k + lane] : 0.0f;
-      const uint4 *src = dy + (size_t)t * vpr;
-      for (int s = 0; s < k; ++s) {
-        const int r = __shfl_sync(0xFFFFFFFFu, d, s);
-        const float ws = __shfl_sync(0xFFFFFFFFu, wl, s);
-        float dot = 0.0f;
-        if (r >= 0) {
-          const uint4 *yrow = y_pad + (size_t)r * vpr;
-          uint4 *orow = dy_pad + (size_t)r * vpr;
-          for (int v0 = 0; v0 < vpr; v0 += 32 * kGatherVPL) {
-            uint4 g[kGatherVPL], yv[kGatherVPL];
-#pragma unroll
-            for (int u = 0; u < kGatherVPL; ++u) {
-              const int v = v0 + u * 32 + lane;
-              if (v < vpr) {
-                g[u] = __ldg(src + v);
-                yv[u] = ld_nc_v4(yrow + v);
-              }
-            }
-#pragma unroll
-            for (int u = 0; u < kGatherVPL; ++u) {
-              const int v = v0 + u * 32 + lane;
-              if (v < vpr) {
-                const uint32_t *gq = reinterpret_cast<const uint32_t *>(&g[u]);
-                const uint32_t *yq = reinterpret_cast<const uint32_t *>(&yv[u]);
-                uint32_t o[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  const float g0 = bf16_lo(gq[q]), g1 = bf16_hi(gq[q]);
-                  dot = fmaf(g0, bf16_lo(yq[q]), dot);
-                  dot = fmaf(g1, bf16_hi(yq[q]), dot);
-                  o[q] = pack_bf16x2(ws * g0, ws * g1);
-                }
-                orow[v] = make_uint4(o[0], o[1], o[2], o[3]);
-              }
-            }
-          }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xFFFFFFFFu, dot, off);
-        if (lane == 0) dweights[(size_t)t * k + s] = dot;
-      }
-    } else {
-      const long long q = it - T;
-      const int e = (int)(q / kBlock), r = (int)(q % kBlock);
-      const int row = ((e > 0) ? padded_bins[e - 1] : 0) + counts[e] + r;
-      if (row < padded_bins[e]) {
-        uint4 *dst = dy_pad + (size_t)row * vpr;
-        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-        for (int v = lane; v < vpr; v += 32) dst[v] = z;
-      }
-    }
-  }
-}
-
 static int copy_grid(long long items) {
   const long long per_cta = kCopyWarps;
   long long want = (items + per_cta - 1) / per_cta;
@@ -257,23 +191,17 @@ cudaError_t launch_gather(int T, int h, int k, int E, const void *x, const int32
 cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const int32_t *dest_row,
                            const float *weights, void *y, cudaStream_t st) {
   k_combine<<<copy_grid((long long)T * slices(h)), kCopyThreads, 0, st>>>(
-      T, h, k, static_cast<const uint4 *>(y_pad),
-                                                   dest_row, weights, static_cast<uint4 *>(y));
+      T, h, k, static_cast<const uint4 *>(y_pad), dest_row, weights, static_cast<uint4 *>(y),
+      nullptr, 0, nullptr);
   return cudaGetLastError();
 }
 
-}  // namespace dmoe
-
-namespace dmoe {
-
-cudaError_t launch_dy_gather(int T, int h, int k, int E, const void *dy, const int32_t *dest_row,
-                             const float *weights, const int32_t *counts,
-                             const int32_t *padded_bins, const void *y_pad, void *dy_pad,
-                             float *dweights, cudaStream_t st) {
-  const long long items = (long long)T + (long long)kBlock * E;
-  k_dy_gather<<<copy_grid(items), kCopyThreads, 0, st>>>(
-      T, h, k, E, static_cast<const uint4 *>(dy), dest_row, weights, counts, padded_bins,
-      static_cast<const uint4 *>(y_pad), static_cast<uint4 *>(dy_pad), dweights);
+cudaError_t launch_bwd_scatter(int T, int h, int k, const void *dx_pad, const int32_t *dest_row,
+                               const float *part, int nt, void *dx, float *dweights,
+                               cudaStream_t st) {
+  k_combine<<<copy_grid((long long)T * slices(h)), kCopyThreads, 0, st>>>(
+      T, h, k, static_cast<const uint4 *>(dx_pad), dest_row, nullptr, static_cast<uint4 *>(dx),
+      part, nt, dweights);
   return cudaGetLastError();
 }
 

@@ -40,11 +40,15 @@
 //         more than the TMA unit issues in one stage's MMA time: about 3x slower than
 //         gather kernel + GLU on B200, so it is not the default path.
 //   DOWN  A = H (K)          B = W2_e (K)                 out Y_pad
-//   DGLU  A = dY_pad (K)     B = W2_e^T (MN)              dH; epilogue recomputes the
-//         activation from the saved A, Bm: dA = dH*Bm*s*(1+A(1-s)), dBm = dH*A*s, s = sigmoid(A)
+//   DGLU  A = dY_pad (K)     B = W2_e^T (MN)              G = dy W2_e (dY_pad holds the
+//         token rows of dy, unweighted); the epilogue recomputes the activation from the saved
+//         A, Bm (s = sigmoid(A), h = A*s*Bm) and, with w the routing weight of the row, writes
+//         dA = w*G*Bm*s*(1+A(1-s)), dBm = w*G*A*s, Hw = w*h (the dW2 operand) and the partial
+//         routing-weight gradient sum_cols G*h of the row over the tile's columns
 //   DX    A = dA then dBm (K), B = W1_e then W3_e (MN), one accumulator over both K passes
-//   WGRAD dW1_e = dA^T X_pad, dW3_e = dBm^T X_pad, dW2_e = dY^T H over the expert's padded
-//         rows (both operands MN-major); fp32 outputs; experts without rows get exact zeros.
+//   WGRAD dW1_e = dA^T X_pad, dW3_e = dBm^T X_pad, dW2_e = dY_pad^T Hw over the expert's
+//         padded rows (both operands MN-major); fp32 outputs; experts without rows get exact
+//         zeros.
 //
 // Every mbarrier wait is bounded; on expiry the kernel sets DMOE_STATUS_TIMEOUT, raises an
 // abort flag for the other roles of its CTA, drains what it issued and returns.
@@ -116,6 +120,8 @@ struct GemmParams {
   int inject;    // test-only: pair leaders withhold their first stage (waits then expire)
   long long wait_cycles;  // budget of every bounded wait of this launch
   const __nv_bfloat16 *in0, *in1;  // DGLU: saved A, Bm
+  const float *weights;            // DGLU: routing weight of each flattened entry
+  float *part;                     // DGLU: [P_max, n_tiles] partial routing-weight gradients
   int32_t *status;
 };
 
@@ -200,6 +206,15 @@ __device__ __forceinline__ void gather_rows(const GemmParams &p, const Tile &tl,
   }
 }
 
+// DGLU: routing weight of padded row `row` of expert e (0 for a padding row).
+__device__ __forceinline__ float row_weight(const GemmParams &p, int e, int row) {
+  const int pstart = (e > 0) ? p.padded_bins[e - 1] : 0;
+  const int bstart = (e > 0) ? p.bins[e - 1] : 0;
+  const int local = row - pstart;
+  return (local < p.bins[e] - bstart) ? __ldg(p.weights + __ldg(p.indices + bstart + local))
+                                      : 0.0f;
+}
+
 template <int MODE>
 __device__ __forceinline__ void load_stage(const GemmParams &p, const Tile &tl, int kb,
                                            uint32_t rank, uint8_t *sa, uint8_t *sb,
@@ -279,9 +294,28 @@ __device__ __forceinline__ void pack_bf16_row(const uint32_t (&lo)[32], const ui
 
 // Epilogue of one tile for the warp owning TMEM sub-partition `sub` (rows sub*32 .. +31 of
 // this CTA's 128 rows); tb = TMEM address of the warp's lanes at accumulator column 0.
+// Work of a tile's epilogue that does not depend on the accumulator, done before waiting for
+// it: DGLU looks up the routing weight of this thread's row (a chain of dependent loads) and
+// starts pulling the row's saved A and Bm columns of the tile into L2.
+template <int MODE>
+__device__ __forceinline__ float epilogue_prologue(const GemmParams &p, const Tile &tl, int sub,
+                                                   int lane) {
+  if (MODE != MODE_DGLU || tl.dummy) return 0.0f;
+  const int grow = tl.row0 + sub * 32 + lane;
+  const int n0 = tl.n * BN;
+  const int ncols = min(BN, p.f - n0);
+  const __nv_bfloat16 *ra = p.in0 + (size_t)grow * p.f + n0;
+  const __nv_bfloat16 *rb = p.in1 + (size_t)grow * p.f + n0;
+  for (int c = 0; c < ncols; c += 64) {  // one 128-byte line per 64 columns
+    prefetch_l2(ra + c);
+    prefetch_l2(rb + c);
+  }
+  return row_weight(p, tl.e, grow);
+}
+
 template <int MODE, int EPI>
 __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &tl, uint32_t tb,
-                                              int sub, int half, int lane,
+                                              int sub, int half, int lane, float wr,
                                               Stager<Cfg<MODE, EPI>::out_bufs> &st) {
   const int y0 = tl.row0 + sub * 32;  // first row of this warp's boxes
   constexpr int kw = BN / Cfg<MODE, EPI>::col_split;  // accumulator columns per warp (non-GLU)
@@ -330,18 +364,19 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
       tmem_ld_wait();
     }
   } else if (MODE == MODE_DGLU) {
-    const int n0 = tl.n * BN + half * kw;
-    tb += (uint32_t)(half * kw);
-    const size_t grow = (size_t)y0 + lane;
+    static_assert(MODE != MODE_DGLU || EPI == 4, "one warp per row holds a row's partial sum");
+    const int n0 = tl.n * BN;
+    const int grow = y0 + lane;  // this thread's padded row; wr = its routing weight
+    float dot = 0.0f;  // sum over this tile's columns of G * h, in column order
 #pragma unroll 1
     for (int c = 0; c < kw; c += 64) {
       if (n0 + c >= p.f) break;
-      uint32_t v0[32], v1[32], wa[32], wb[32];
+      uint32_t v0[32], v1[32], wa[32], wb[32], wh[32];
       uint4 qa[8], qb[8];
       tmem_ld32(tb + c, v0);
       tmem_ld32(tb + c + 32, v1);
-      const uint4 *sa = reinterpret_cast<const uint4 *>(p.in0 + grow * p.f + n0 + c);
-      const uint4 *sb = reinterpret_cast<const uint4 *>(p.in1 + grow * p.f + n0 + c);
+      const uint4 *sa = reinterpret_cast<const uint4 *>(p.in0 + (size_t)grow * p.f + n0 + c);
+      const uint4 *sb = reinterpret_cast<const uint4 *>(p.in1 + (size_t)grow * p.f + n0 + c);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         qa[i] = __ldg(sa + i);
@@ -352,17 +387,24 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
       for (int i = 0; i < 32; ++i) {  // bf16 pairs 2i, 2i+1 of this 64-column chunk
         const uint32_t aw = reinterpret_cast<const uint32_t *>(qa)[i];
         const uint32_t bw = reinterpret_cast<const uint32_t *>(qb)[i];
-        const float dh0 = __uint_as_float(i < 16 ? v0[2 * i] : v1[2 * i - 32]);
-        const float dh1 = __uint_as_float(i < 16 ? v0[2 * i + 1] : v1[2 * i - 31]);
+        const float g0 = __uint_as_float(i < 16 ? v0[2 * i] : v1[2 * i - 32]);
+        const float g1 = __uint_as_float(i < 16 ? v0[2 * i + 1] : v1[2 * i - 31]);
         const float a0 = bf16_lo(aw), a1 = bf16_hi(aw), b0 = bf16_lo(bw), b1 = bf16_hi(bw);
         const float s0 = sigmoid_f(a0), s1 = sigmoid_f(a1);
+        const float h0 = a0 * s0 * b0, h1 = a1 * s1 * b1;
+        dot = fmaf(g0, h0, dot);
+        dot = fmaf(g1, h1, dot);
+        const float dh0 = wr * g0, dh1 = wr * g1;
         wa[i] = pack_bf16x2(dh0 * b0 * s0 * (1.0f + a0 * (1.0f - s0)),
                             dh1 * b1 * s1 * (1.0f + a1 * (1.0f - s1)));
         wb[i] = pack_bf16x2(dh0 * a0 * s0, dh1 * a1 * s1);
+        wh[i] = pack_bf16x2(wr * h0, wr * h1);
       }
       st.emit(&p.tmo[0], wa, n0 + c, y0);
       st.emit(&p.tmo[1], wb, n0 + c, y0);
+      st.emit(&p.tmo[2], wh, n0 + c, y0);
     }
+    p.part[(size_t)grow * p.n_tiles + tl.n] = dot;
   } else {  // MODE_WGRAD: fp32 results, boxes of 32 columns
     const int rows = (tl.which == 2) ? p.h : p.f;
     const int cols = (tl.which == 2) ? p.f : p.h;
@@ -583,13 +625,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
     for (int t = cluster; t < total; t += nclusters) {
       const Tile tl = decode<MODE>(p, t, ustart, rank);
       if (tl.kit == 0) {  // no accumulator involved
-        if (!tl.dummy) epilogue_tile<MODE, EPI>(p, tl, 0u, sub, half, lane, st);
+        if (!tl.dummy) epilogue_tile<MODE, EPI>(p, tl, 0u, sub, half, lane, 0.0f, st);
         continue;
       }
+      const float wr = epilogue_prologue<MODE>(p, tl, sub, lane);
       if (!mbar_wait(&tfull[acc], acc_phase, p.status, abort_flag, p.wait_cycles)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * ACC_COLS);
-      if (!tl.dummy) epilogue_tile<MODE, EPI>(p, tl, tb, sub, half, lane, st);
+      if (!tl.dummy) epilogue_tile<MODE, EPI>(p, tl, tb, sub, half, lane, wr, st);
       tc_fence_before();
       mbar_arrive_cluster(leader_tempty0 + (uint32_t)(acc * sizeof(uint64_t)));
       acc ^= 1;
@@ -783,13 +826,16 @@ cudaError_t launch_down_gemm(const GemmProblem &g, const void *h_in, const void 
 
 cudaError_t launch_dglu_gemm(const GemmProblem &g, const void *dy_pad, const void *w2,
                              const void *a_in, const void *b_in, void *da_out, void *db_out,
-                             cudaStream_t st) {
+                             void *hw_out, float *part, cudaStream_t st) {
   GemmParams p = base_params(g);
   const uint64_t P = (uint64_t)g.nblk_cap * BM;
   if (!make_tmap(&p.tm[0], dy_pad, P, g.h, BM) ||
       !make_tmap(&p.tm[1], w2, (uint64_t)g.E * g.h, g.f, 64) ||
-      !make_tmap(&p.tmo[0], da_out, P, g.f, 32) || !make_tmap(&p.tmo[1], db_out, P, g.f, 32))
+      !make_tmap(&p.tmo[0], da_out, P, g.f, 32) || !make_tmap(&p.tmo[1], db_out, P, g.f, 32) ||
+      !make_tmap(&p.tmo[2], hw_out, P, g.f, 32))
     return cudaErrorInvalidValue;
+  p.weights = g.weights;
+  p.part = part;
   p.tm[2] = p.tm[3] = p.tm[4] = p.tm[0];
   p.n_tiles = (g.f + BN - 1) / BN;
   p.k_iters = g.h / BK;

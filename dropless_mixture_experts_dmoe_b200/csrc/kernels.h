@@ -39,12 +39,11 @@ cudaError_t launch_gather(int T, int h, int k, int E, const void *x, const int32
 cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const int32_t *dest_row,
                            const float *weights, void *y, cudaStream_t st);
 
-// dY gather for the backward: dY_pad[dest_row[t*k+s]] = bf16(w_ts * dy_t), padding rows zero,
-// and the routing-weight gradient dweights[t*k+s] = <dy_t, Y_pad[dest_row[t*k+s]]>.
-cudaError_t launch_dy_gather(int T, int h, int k, int E, const void *dy, const int32_t *dest_row,
-                             const float *weights, const int32_t *counts,
-                             const int32_t *padded_bins, const void *y_pad, void *dy_pad,
-                             float *dweights, cudaStream_t st);
+// Backward scatter: dx_t = sum_s dX_pad[dest_row[t*k+s]] and, from the DGLU GEMM's partial
+// sums part [P_max, nt], dweights[t*k+s] = sum_n part[dest_row[t*k+s]][n].
+cudaError_t launch_bwd_scatter(int T, int h, int k, const void *dx_pad, const int32_t *dest_row,
+                               const float *part, int nt, void *dx, float *dweights,
+                               cudaStream_t st);
 
 // Shape and map pointers shared by the grouped GEMM launchers.
 struct GemmProblem {
@@ -55,6 +54,7 @@ struct GemmProblem {
   const int32_t *padded_bins;
   const int32_t *bins;
   const int32_t *indices;
+  const float *weights;
   int32_t *status;
 };
 
@@ -68,9 +68,11 @@ cudaError_t launch_glu_gather_gemm(const GemmProblem &g, const void *x, const vo
 cudaError_t launch_down_gemm(const GemmProblem &g, const void *h_in, const void *w2, void *y_pad,
                              cudaStream_t st);
 // ... and the backward: dH with the fused dGLU epilogue, dX, and the weight gradients.
+// DGLU column tile width (part has ceil(f / kDgluTileCols) columns).
+constexpr int kDgluTileCols = 256;
 cudaError_t launch_dglu_gemm(const GemmProblem &g, const void *dy_pad, const void *w2,
                              const void *a_in, const void *b_in, void *da_out, void *db_out,
-                             cudaStream_t st);
+                             void *hw_out, float *part, cudaStream_t st);
 cudaError_t launch_dx_gemm(const GemmProblem &g, const void *da, const void *db, const void *w1,
                            const void *w3, void *dx_pad, cudaStream_t st);
 cudaError_t launch_wgrad_gemm(const GemmProblem &g, const void *x_pad, const void *h_in,

@@ -15,7 +15,9 @@
  *   5. padded_scatter: y_t = sum_s w_ts * Y_pad[dest_row[t*k+s]] (section 4.2);
  *   6. backward: gather and scatter swap roles, plus the routing-weight gradient
  *      (section 4.2); the activation is recomputed from the saved pre-activations
- *      (section 4.4).
+ *      (section 4.4).  Only X_pad, A and Bm are kept for it: the routing-weight gradient
+ *      <dy_t, Y_ts> is formed as <dy_t W2_e, H_ts> inside the dH GEMM, so neither H nor
+ *      Y_pad has to outlive the forward (the activation-memory saving of SonicMoE, abstract).
  *
  * Conventions (all entry points)
  *   - The caller owns and allocates ALL device memory, including workspaces; the library
@@ -120,8 +122,13 @@ typedef struct {
 
 /* Workspace kinds for dmoe_workspace_bytes. */
 #define DMOE_WS_MAP 0      /* dmoe_sparse_map */
-#define DMOE_WS_FORWARD 1  /* dmoe_forward with saved == NULL (inference) */
-#define DMOE_WS_BACKWARD 2 /* dmoe_backward */
+#define DMOE_WS_FORWARD 1        /* dmoe_forward with saved == NULL (inference) */
+#define DMOE_WS_BACKWARD 2       /* dmoe_backward */
+#define DMOE_WS_FORWARD_TRAIN 3  /* dmoe_forward with saved != NULL (training) */
+
+/* Column tile of the dH GEMM: the routing-weight partial sums of dmoe_bwd_dglu have
+ * ceil(ffn / DMOE_DGLU_TILE_COLS) columns. */
+#define DMOE_DGLU_TILE_COLS 256
 
 /* Static bound on the padded row count: floor((T*k + 127*E)/128)*128.  Every padded
  * buffer is sized from it, so no call needs the data-dependent size on the host (the
@@ -134,9 +141,10 @@ DMOE_API size_t dmoe_workspace_bytes(const dmoe_dims *dims, int kind);
 
 /* Bytes of the activations dmoe_forward saves for dmoe_backward, and their byte offsets
  * inside that buffer: offsets[0] X_pad [P_max,h], [1] A = X_pad W1^T [P_max,f],
- * [2] Bm = X_pad W3^T [P_max,f], [3] H = silu(A)*Bm [P_max,f], [4] Y_pad [P_max,h], all bf16.
- * offsets may be NULL.  Returns 0 for invalid dims. */
-DMOE_API size_t dmoe_saved_bytes(const dmoe_dims *dims, size_t offsets[5]);
+ * [2] Bm = X_pad W3^T [P_max,f], all bf16 (H and Y_pad are not kept: the backward recomputes
+ * the activation from A and Bm and never needs Y_pad).  offsets may be NULL.  Returns 0 for
+ * invalid dims. */
+DMOE_API size_t dmoe_saved_bytes(const dmoe_dims *dims, size_t offsets[3]);
 
 /* Routing + sparse map (walkthrough section 4.1; the Fast-LLM get_sparse_map step).
  *   logits: [T, E] bf16 device pointer, or NULL to take map->top_experts as given (then
@@ -154,8 +162,10 @@ DMOE_API int dmoe_sparse_map(const dmoe_dims *dims, const void *logits, const dm
  *   x [T,h], w1 [E,f,h], w3 [E,f,h], w2 [E,h,f]: bf16 inputs.  map: from dmoe_sparse_map.
  *   y [T,h] bf16 output.
  *   saved: NULL for inference, else a buffer of dmoe_saved_bytes(dims) bytes that receives
- *          X_pad, A, Bm, H, Y_pad for dmoe_backward (then ws may be NULL / 0 bytes).
- *   ws: dmoe_workspace_bytes(dims, DMOE_WS_FORWARD) bytes when saved == NULL.
+ *          X_pad, A, Bm for dmoe_backward.
+ *   ws: dmoe_workspace_bytes(dims, DMOE_WS_FORWARD) bytes when saved == NULL, else
+ *       dmoe_workspace_bytes(dims, DMOE_WS_FORWARD_TRAIN) bytes (H and Y_pad, dead after the
+ *       call returns on the stream).
  * Runs padded_gather, the GLU GEMM, the down GEMM and the weighted padded_scatter. */
 DMOE_API int dmoe_forward(const dmoe_dims *dims, const void *x, const void *w1, const void *w3,
                  const void *w2, const dmoe_map *map, void *y, void *saved, void *ws,
@@ -168,8 +178,11 @@ DMOE_API int dmoe_forward(const dmoe_dims *dims, const void *x, const void *w1, 
  *   dmoe_forward(saved != NULL).
  *   Outputs: dx [T,h] bf16; dw1, dw3 [E,f,h] fp32; dw2 [E,h,f] fp32 (the weight gradients
  *   of a mixed-precision step are kept in fp32; experts that receive no token get exact
- *   zeros); dweights [T,k] fp32 = <dy_t, Y_ts>.
- *   ws: dmoe_workspace_bytes(dims, DMOE_WS_BACKWARD) bytes. */
+ *   zeros); dweights [T,k] fp32 = <dy_t, Y_ts>, where Y_ts = H_ts W2_e^T is the expert's
+ *   unweighted output row, computed as <dy_t W2_e, H_ts>.  All results are deterministic.
+ *   ws: dmoe_workspace_bytes(dims, DMOE_WS_BACKWARD) bytes.
+ *   Runs dmoe_padded_gather(dy), dmoe_bwd_dglu, dmoe_bwd_wgrad, dmoe_bwd_dx and
+ *   dmoe_bwd_scatter in that order. */
 DMOE_API int dmoe_backward(const dmoe_dims *dims, const void *dy, const void *w1, const void *w3,
                   const void *w2, const dmoe_map *map, const void *saved, void *dx, float *dw1,
                   float *dw3, float *dw2, float *dweights, void *ws, size_t ws_bytes,
@@ -237,25 +250,24 @@ DMOE_API int dmoe_expert_down(const dmoe_dims *dims, const void *h_in, const voi
 DMOE_API int dmoe_padded_scatter(const dmoe_dims *dims, const void *y_pad, const dmoe_map *map,
                         const float *weights, void *y, void *stream);
 
-/* ---- Backward step entry points (each one kernel); dmoe_backward runs dy_gather, dglu,
- * wgrad, dx and dmoe_padded_scatter(weights = NULL) in that order. ---- */
+/* ---- Backward step entry points (each one kernel).  dmoe_backward is: dy_pad =
+ * dmoe_padded_gather(dy) (the gradient of the weighted scatter is a gather, walkthrough
+ * section 4.2; the weight is applied inside the dH GEMM), then dglu, wgrad, dx, scatter. ---- */
 
-/* Gradient of the weighted padded_scatter (walkthrough section 4.2: a padded_gather of dy
- * plus the routing-weight gradient of _padded_copy_wgrad):
- *   dy_pad[dest_row[t*k+s]] = bf16(w_ts * dy_t); padding rows of every expert's last block = 0;
- *   dweights[t*k+s] = <dy_t, Y_pad[dest_row[t*k+s]]> (fp32; 0 for dropped entries).
- * dy [T,h], y_pad [P_max,h] (forward output rows) -> dy_pad [P_max,h] bf16, dweights [T,k] fp32. */
-DMOE_API int dmoe_bwd_dy_gather(const dmoe_dims *dims, const void *dy, const dmoe_map *map,
-                                const void *y_pad, void *dy_pad, float *dweights, void *stream);
-
-/* dH GEMM with the gated-SiLU gradient fused into its epilogue (walkthrough section 4.4:
- * the activation is recomputed from the saved pre-activations instead of being stored):
- *   dH = dY_pad[b] W2_e (fp32), s = sigmoid(A), dA = bf16(dH * Bm * s * (1 + A (1 - s))),
- *   dBm = bf16(dH * A * s), for every row block b < num_blocks of expert e.
- * a_saved, bm_saved: bf16 A, Bm of dmoe_forward; all [P_max,f] except dy_pad [P_max,h]. */
+/* dH GEMM with the gated-SiLU gradient and the routing-weight gradient fused into its
+ * epilogue (walkthrough section 4.4: the activation is recomputed from the saved
+ * pre-activations instead of being stored; section 4.2: the routing-weight gradient).
+ * For every row block b < num_blocks of expert e, with G = dY_pad[b] W2_e (fp32; dY_pad holds
+ * the unweighted rows of dy), s = sigmoid(A), h = A*s*Bm and w the routing weight of the row
+ * (0 for a padding row):
+ *   da = bf16(w*G*Bm*s*(1 + A(1-s))),  dbm = bf16(w*G*A*s),  hw = bf16(w*h)   [P_max,f];
+ *   dw_part[r * nt + n] = sum over the columns c of tile n of G[r,c]*h[r,c]   (fp32,
+ *     nt = ceil(f / DMOE_DGLU_TILE_COLS) column tiles of 256; since G h^T = dy (H W2_e^T)^T,
+ *     the tiles of a row sum to the routing-weight gradient <dy_t, Y_ts>).
+ * map->weights is read.  a_saved, bm_saved: bf16 A, Bm of dmoe_forward; dy_pad [P_max,h]. */
 DMOE_API int dmoe_bwd_dglu(const dmoe_dims *dims, const void *dy_pad, const void *w2,
                            const void *a_saved, const void *bm_saved, const dmoe_map *map,
-                           void *da, void *dbm, void *stream);
+                           void *da, void *dbm, void *hw, float *dw_part, void *stream);
 
 /* dX GEMM: dX_pad[b] = bf16(dA[b] W1_e + dBm[b] W3_e), one fp32 accumulator over both K
  * passes.  da, dbm [P_max,f] -> dx_pad [P_max,h]. */
@@ -266,12 +278,21 @@ DMOE_API int dmoe_bwd_dx(const dmoe_dims *dims, const void *da, const void *dbm,
  * (padding rows are zero, so they add nothing; the walkthrough's stk path needs a transposed
  * topology for this, section 4.3; here each output tile walks its expert's rows directly):
  *   dW1_e = sum_r dA_r^T X_pad_r,  dW3_e = sum_r dBm_r^T X_pad_r  ([f,h] each),
- *   dW2_e = sum_r dY_pad_r^T H_r  ([h,f]); fp32 accumulation and fp32 output (dw1, dw3,
- * dw2 are float*), no split-K, so the result is deterministic; experts without rows get
- * exact zeros. */
-DMOE_API int dmoe_bwd_wgrad(const dmoe_dims *dims, const void *x_pad, const void *h_saved,
+ *   dW2_e = sum_r dY_pad_r^T Hw_r  ([h,f]; dY_pad unweighted, Hw = w*H from dmoe_bwd_dglu);
+ * fp32 accumulation and fp32 output (dw1, dw3, dw2 are float*), no split-K, so the result is
+ * deterministic; experts without rows get exact zeros. */
+DMOE_API int dmoe_bwd_wgrad(const dmoe_dims *dims, const void *x_pad, const void *hw,
                             const void *dy_pad, const void *da, const void *dbm,
                             const dmoe_map *map, float *dw1, float *dw3, float *dw2, void *stream);
+
+/* Scatter-sum of the backward plus the routing-weight gradient (walkthrough section 4.2: the
+ * gradient of padded_gather is padded_scatter with w = 1):
+ *   dx_t = bf16(sum_s dX_pad[dest_row[t*k+s]])  (fp32 sum in slot order),
+ *   dweights[t*k+s] = sum_{n < nt} dw_part[dest_row[t*k+s] * nt + n]  (fp32, tile order; 0 for
+ *   an entry dropped from the map).
+ * dx_pad [P_max,h] bf16, dw_part from dmoe_bwd_dglu -> dx [T,h] bf16, dweights [T,k] fp32. */
+DMOE_API int dmoe_bwd_scatter(const dmoe_dims *dims, const void *dx_pad, const float *dw_part,
+                              const dmoe_map *map, void *dx, float *dweights, void *stream);
 
 /* ---- Diagnostics. ---- */
 DMOE_API const char *dmoe_error_string(int code);

@@ -41,9 +41,17 @@ def test_sizes():
     assert P == ((4096 * 2 + 127 * 8) // 128) * 128
     assert B.dmoe_workspace_bytes(d, B.WS_MAP) >= 4 * 64 * 8
     assert B.dmoe_workspace_bytes(d, B.WS_FORWARD) >= P * (2 * 4096 + 14336) * 2
+    # a training forward keeps X_pad in the saved buffer: its workspace holds H and Y_pad only
+    assert P * (4096 + 14336) * 2 <= B.dmoe_workspace_bytes(d, B.WS_FORWARD_TRAIN) < \
+        B.dmoe_workspace_bytes(d, B.WS_FORWARD)
+    # backward: dY_pad (reused for dX_pad), dA, dBm, Hw and the routing-weight partials
+    assert B.dmoe_workspace_bytes(d, B.WS_BACKWARD) >= P * (4096 + 3 * 14336) * 2 + P * 56 * 4
     total, offs = B.dmoe_saved_bytes(d)
+    assert len(offs) == 3  # X_pad, A, Bm: neither H nor Y_pad outlives the forward
     assert offs == sorted(offs) and offs[0] == 0 and all(o % 256 == 0 for o in offs)
-    assert total >= offs[4] + P * 4096 * 2
+    assert offs[1] >= P * 4096 * 2 and offs[2] >= offs[1] + P * 14336 * 2
+    assert total >= offs[2] + P * 14336 * 2
+    assert B.dmoe_workspace_bytes(d, 4) == 0  # unknown workspace kind
 
 
 @pytest.mark.parametrize("dims,code", [

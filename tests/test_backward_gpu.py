@@ -1,6 +1,6 @@
-"""Backward parity (dY gather + routing-weight gradient, dH with the fused dGLU epilogue,
-dX, scatter-sum, weight gradients) against the oracle, and each backward GEMM against
-float64 PyTorch on the same bf16 operands."""
+"""Backward parity (dY gather, dH with the fused dGLU and routing-weight epilogue, dX,
+scatter-sum with the routing-weight reduction, weight gradients) against the oracle, and
+each backward step against float64 PyTorch on the same bf16 operands."""
 import numpy as np
 import pytest
 import torch
@@ -42,50 +42,88 @@ def test_backward_full_parity_small(w):
 
 
 @pytest.mark.parametrize("w", SMALL[1:4], ids=lambda w: w.describe())
-def test_backward_gemms_against_float64(w):
-    """Every backward GEMM mode on its own bf16 inputs (MN-major operands included)."""
+def test_backward_steps_against_float64(w):
+    """Every backward step on its own bf16 inputs (MN-major operands included): the dy
+    gather, the dH GEMM with its fused dGLU / weighted-H / routing-weight-partial epilogue,
+    dX, the weight gradients, and the scatter-sum with the routing-weight reduction."""
     inp = make_inputs(w, with_dy=True)
     dims = dims_of(w)
     bufs, dev, y, g = gpu_backward(dims, inp)
     st = bufs.bstep
-    B.dmoe_bwd_dy_gather(dims, dev["dy"], bufs.map, bufs.view("y_pad"), st["dy_pad"],
-                         torch.empty((w.T, w.top_k), dtype=torch.float32, device="cuda"))
+    T, k, h, f = w.T, w.top_k, w.hidden, w.ffn
+    dx = torch.empty((T, h), dtype=torch.bfloat16, device="cuda")
+    dwt = torch.full((T, k), float("nan"), dtype=torch.float32, device="cuda")
+    dw = {n: torch.empty_like(g[n]) for n in ("dw1", "dw3", "dw2")}
+    B.dmoe_padded_gather(dims, dev["dy"], bufs.map, st["dy_pad"])
     B.dmoe_bwd_dglu(dims, st["dy_pad"], dev["w2"], bufs.view("a"), bufs.view("bm"), bufs.map,
-                    st["da"], st["dbm"])
+                    st["da"], st["dbm"], st["hw"], st["dw_part"])
+    B.dmoe_bwd_wgrad(dims, bufs.view("x_pad"), st["hw"], st["dy_pad"], st["da"], st["dbm"],
+                     bufs.map, dw["dw1"], dw["dw3"], dw["dw2"])
     B.dmoe_bwd_dx(dims, st["da"], st["dbm"], dev["w1"], dev["w3"], bufs.map, st["dx_pad"])
+    B.dmoe_bwd_scatter(dims, st["dx_pad"], st["dw_part"], bufs.map, dx, dwt)
     torch.cuda.synchronize()
     nb = int(bufs.map.num_blocks.item())
     P = nb * 128
     be = bufs.map.block_expert.cpu().numpy()
     D = lambda t: t[:P].double().cpu()
-    dy_pad, da, dbm, dx_pad = D(st["dy_pad"]), D(st["da"]), D(st["dbm"]), D(st["dx_pad"])
-    A, Bm, H, Xp = D(bufs.view("a")), D(bufs.view("bm")), D(bufs.view("h")), D(bufs.view("x_pad"))
+    dy_pad, da, dbm, hw, dx_pad = (D(st[n]) for n in ("dy_pad", "da", "dbm", "hw", "dx_pad"))
+    part = st["dw_part"][:P].cpu()
+    A, Bm, Xp = D(bufs.view("a")), D(bufs.view("bm")), D(bufs.view("x_pad"))
     W1, W3, W2 = inp["w1"].double(), inp["w3"].double(), inp["w2"].double()
-    # dY_pad rows hold w * dy of their token (bf16), padding rows are zero
+    # dY_pad rows are the token rows of dy, unchanged; padding rows are zero
     dest = bufs.map.dest_row.cpu().numpy()
-    wts = bufs.map.weights.cpu().double()
-    ref_dy = torch.zeros(P, w.hidden, dtype=torch.float64)
-    tok = torch.arange(w.T * w.top_k) // w.top_k
-    ref_dy[dest] = (wts.reshape(-1, 1) * inp["dy"].double()[tok]).to(torch.bfloat16).double()
+    wts = bufs.map.weights.cpu().double().reshape(-1)
+    tok = torch.arange(T * k) // k
+    ref_dy = torch.zeros(P, h, dtype=torch.float64)
+    ref_dy[dest] = inp["dy"].double()[tok]
     assert torch.equal(dy_pad, ref_dy)
+    wrow = torch.zeros(P, dtype=torch.float64)  # routing weight of each padded row
+    wrow[dest] = wts
+    nt = (f + 255) // 256
     for b in range(nb):
         e = int(be[b])
         rows = slice(b * 128, (b + 1) * 128)
-        dh = dy_pad[rows] @ W2[e]
-        s = torch.sigmoid(A[rows])
-        da_ref = dh * Bm[rows] * s * (1 + A[rows] * (1 - s))
-        db_ref = dh * A[rows] * s
+        G = dy_pad[rows] @ W2[e]
+        a, bm, wr = A[rows], Bm[rows], wrow[rows].unsqueeze(1)
+        s = torch.sigmoid(a)
+        hv = a * s * bm
+        da_ref = wr * G * bm * s * (1 + a * (1 - s))
+        db_ref = wr * G * a * s
         assert torch.allclose(da[rows], da_ref, rtol=2e-2, atol=2e-3), ("dA", b)
         assert torch.allclose(dbm[rows], db_ref, rtol=2e-2, atol=2e-3), ("dBm", b)
+        assert torch.allclose(hw[rows], wr * hv, rtol=2e-2, atol=2e-4), ("Hw", b)
+        gh = G * hv
+        for n in range(nt):  # per-tile partial <G, h>, bounded by the sum of |terms|
+            cols = slice(n * 256, min(f, (n + 1) * 256))
+            ref_p = gh[:, cols].sum(1)
+            bound = 2e-3 * gh[:, cols].abs().sum(1) + 1e-6
+            assert ((part[rows, n].double() - ref_p).abs() <= bound).all(), ("part", b, n)
         dx_ref = da[rows] @ W1[e] + dbm[rows] @ W3[e]
         assert torch.allclose(dx_pad[rows], dx_ref, rtol=2e-2, atol=2e-3), ("dX", b)
+    # scatter-sum: fp32 in slot order, then bf16 (bit-exact); dweights: fp32 in tile order
+    acc = torch.zeros(T, h, dtype=torch.float32)
+    dxp32 = st["dx_pad"].float().cpu()
+    d2 = torch.from_numpy(dest.reshape(T, k)).long()
+    for s_ in range(k):
+        acc = acc + dxp32[d2[:, s_]]
+    assert torch.equal(dx.cpu().view(torch.int16), acc.to(torch.bfloat16).view(torch.int16))
+    ref_w = torch.zeros(T * k, dtype=torch.float32)
+    part_all = st["dw_part"].cpu()
+    for n in range(nt):
+        ref_w = ref_w + part_all[torch.from_numpy(dest).long(), n]
+    assert torch.equal(dwt.cpu().reshape(-1).view(torch.int32), ref_w.view(torch.int32))
+    # the step sequence is dmoe_backward: same bits
+    for n in ("dw1", "dw3", "dw2"):
+        assert torch.equal(dw[n].view(torch.int32), g[n].view(torch.int32)), n
+    assert torch.equal(dx.view(torch.int16), g["dx"].view(torch.int16))
+    assert torch.equal(dwt.view(torch.int32), g["dw"].view(torch.int32))
     pb = bufs.map.padded_bins.cpu().numpy()
     for e in range(w.E):
         r0 = 0 if e == 0 else int(pb[e - 1])
         r1 = int(pb[e])
         dw1 = da[r0:r1].T @ Xp[r0:r1]
         dw3 = dbm[r0:r1].T @ Xp[r0:r1]
-        dw2 = dy_pad[r0:r1].T @ H[r0:r1]
+        dw2 = dy_pad[r0:r1].T @ hw[r0:r1]
         for got, ref, n in ((g["dw1"][e], dw1, "dW1"), (g["dw3"][e], dw3, "dW3"), (g["dw2"][e], dw2, "dW2")):
             got = got.double().cpu()
             assert torch.allclose(got, ref, rtol=1e-4, atol=1e-5 * (ref.abs().max().item() + 1e-30)), (n, e)
