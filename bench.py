@@ -42,7 +42,8 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", type=int, default=2)
     p.add_argument("--shape", default="",
-                   help="T,hidden,ffn,E,top_k[,bwd]: a custom workload (forward, or fwd+bwd)")
+                   help="T,hidden,ffn,E,top_k[,bwd][,zipf]: a custom workload (forward, or "
+                        "fwd+bwd; zipf adds the skewed workload's logit bias)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample", type=int, default=0, help="tokens in the oracle sample")
     return p.parse_args()
@@ -510,7 +511,8 @@ def main():
 
         parts = args.shape.split(",")
         T, h, f, E, k = (int(v) for v in parts[:5])
-        w = custom(T, h, f, E, k, number=100, name="custom", backward="bwd" in parts[5:])
+        w = custom(T, h, f, E, k, number=100, name="custom", backward="bwd" in parts[5:],
+                   zipf_bias="zipf" in parts[5:])
     if args.impl == "reference":
         run_reference(args, w)
     else:

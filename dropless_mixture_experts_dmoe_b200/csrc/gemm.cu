@@ -100,8 +100,11 @@ struct Cfg {
   static constexpr int stages = 5;
   static constexpr int out_bufs = (EPI == 8) ? 1 : 2;
   static constexpr int out_bytes = epi_warps * out_bufs * BOX_BYTES;
+  // WGRAD: one zeroed result box, the source of the zero tiles' stores
+  static constexpr int zero_bytes = (MODE == MODE_WGRAD) ? BOX_BYTES : 0;
   static constexpr size_t smem = 1024 /*align*/ + (size_t)stages * STAGE_BYTES + out_bytes +
-                                 256 /*barriers*/ + sizeof(int) * (DMOE_MAX_EXPERTS + 1);
+                                 zero_bytes + 256 /*barriers*/ +
+                                 sizeof(int) * (DMOE_MAX_EXPERTS + 1);
 };
 
 struct GemmParams {
@@ -414,20 +417,15 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
     if (ncols <= 0) return;
     tb += (uint32_t)(half * kw);
     uint32_t v[32], w[32];
-    if (tl.kit > 0) {
-      tmem_ld32(tb, v);
-      tmem_ld_wait();
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = 0u;  // expert without rows: exact zeros
-    }
+    tmem_ld32(tb, v);
+    tmem_ld_wait();
 #pragma unroll 1
     for (int c = 0; c < ncols; c += 32) {
 #pragma unroll
       for (int i = 0; i < 32; ++i) w[i] = v[i];
-      if (tl.kit > 0 && c + 32 < ncols) tmem_ld32(tb + c + 32, v);  // overlaps the store
+      if (c + 32 < ncols) tmem_ld32(tb + c + 32, v);  // overlaps the store
       st.emit(&p.tmo[tl.which], w, n0 + c, yw);
-      if (tl.kit > 0) tmem_ld_wait();
+      tmem_ld_wait();
     }
   }
 }
@@ -444,7 +442,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
   const uint32_t base_u32 = smem_u32(smem_raw);
   uint8_t *tiles = smem_raw + ((1024u - (base_u32 & 1023u)) & 1023u);
   uint8_t *outbuf = tiles + STAGES * STAGE_BYTES;  // 1024-aligned
-  uint64_t *bars = reinterpret_cast<uint64_t *>(outbuf + C::out_bytes);
+  uint8_t *zbuf = outbuf + C::out_bytes;           // 1024-aligned (WGRAD only)
+  uint64_t *bars = reinterpret_cast<uint64_t *>(zbuf + C::zero_bytes);
   uint64_t *full = bars;                       // [STAGES] leader: both halves landed
   uint64_t *empty = bars + STAGES;             // [STAGES] MMAs done reading the stage
   uint64_t *tfull = bars + 2 * STAGES;         // [2] accumulator ready
@@ -452,7 +451,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
   uint64_t *drain = bars + 2 * STAGES + 4;     // leader: all MMAs finished
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  int *ustart = reinterpret_cast<int *>(outbuf + C::out_bytes + 256);  // [E + 1]
+  int *ustart = reinterpret_cast<int *>(zbuf + C::zero_bytes + 256);  // [E + 1]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -497,6 +496,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
       if (lane == 0) ustart[0] = 0;
     }
   }
+  if (MODE == MODE_WGRAD) {  // zero box for the stores of experts without rows
+    for (int i = threadIdx.x; i < C::zero_bytes / 16; i += C::threads)
+      st_shared_v4(smem_u32(zbuf) + (uint32_t)(i * 16), 0u, 0u, 0u, 0u);
+    fence_async_smem();
+  }
   if (warp == 1) tmem_alloc_pair(tmem_slot, TMEM_COLS);
   tc_fence_before();
   __syncthreads();
@@ -524,6 +528,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
     int rows[4] = {0, 0, 0, 0};
     for (int t = cluster; t < total; t += nclusters) {
       const Tile tl = decode<MODE>(p, t, ustart, rank);
+      if (MODE == MODE_WGRAD && tl.kit == 0) continue;  // zero tile: see the peer's warp 1
       if (MODE == MODE_GLU_GATHER) gather_rows(p, tl, lane, rows);
       bool ok = true;
       for (int kb = 0; kb < tl.kit; ++kb) {
@@ -612,6 +617,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
     }
     tc_commit_pair(drain);
     mbar_wait_plain(drain, 0, p.wait_cycles);
+  } else if (MODE == MODE_WGRAD && warp == 1 && lane == 0 && !leader) {
+    // ---------------- zero tiles (peer CTA; its warp 1 has no MMA to issue) ----------------
+    // Experts without rows have zero weight gradients.  Both halves of such a pair tile are
+    // stored here from the zero box, as a background stream of TMA stores that overlaps the
+    // other tiles' MMAs and never touches the accumulator hand-off.
+    for (int t = cluster; t < total; t += nclusters) {
+#pragma unroll 1
+      for (uint32_t half = 0; half < 2; ++half) {
+        const Tile tl = decode<MODE>(p, t, ustart, half);
+        if (tl.kit != 0 || tl.dummy) break;
+        const int rows_ = (tl.which == 2) ? p.h : p.f;
+        const int cols = (tl.which == 2) ? p.f : p.h;
+        const int y = tl.e * rows_ + tl.m * BM;
+        const int n0 = tl.n * BN;
+        const int ncols = min(BN, cols - n0);
+        for (int r = 0; r < BM; r += 32)
+          for (int c = 0; c < ncols; c += 32)
+            tma_store_2d_u32(&p.tmo[tl.which], smem_u32(zbuf), n0 + c, y + r);
+        bulk_commit();
+        bulk_wait_read<8>();  // bounded number of groups in flight
+      }
+    }
+    bulk_wait_all();  // every zero store has completed before the CTA exits
   } else if (warp >= 2) {
     // ---------------- epilogue (both CTAs) ----------------
     const int sub = warp & 3;           // TMEM sub-partition this warp may read
@@ -624,10 +652,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
     uint32_t acc_phase = 0;
     for (int t = cluster; t < total; t += nclusters) {
       const Tile tl = decode<MODE>(p, t, ustart, rank);
-      if (tl.kit == 0) {  // no accumulator involved
-        if (!tl.dummy) epilogue_tile<MODE, EPI>(p, tl, 0u, sub, half, lane, 0.0f, st);
-        continue;
-      }
+      if (tl.kit == 0) continue;  // WGRAD zero tile: stored by the producer warp
       const float wr = epilogue_prologue<MODE>(p, tl, sub, lane);
       if (!mbar_wait(&tfull[acc], acc_phase, p.status, abort_flag, p.wait_cycles)) break;
       tc_fence_after();
