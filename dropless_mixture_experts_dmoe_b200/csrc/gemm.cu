@@ -432,6 +432,15 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
 
 // ---- the kernel -------------------------------------------------------------------------------
 
+// The r-th tile of a cluster in the persistent loop.  Round r covers tiles [r*n, r*n + n); the
+// clusters take them in increasing order on even rounds and in decreasing order on odd ones
+// (a snake), which evens out the per-cluster sums when tile costs fall along the list (the
+// weight-gradient tiles of large experts first, then ever smaller ones).  Every role of both
+// CTAs uses the same sequence.
+__device__ __forceinline__ int snake_tile(int r, int cluster, int nclusters) {
+  return r * nclusters + ((r & 1) ? nclusters - 1 - cluster : cluster);
+}
+
 template <int MODE, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::threads, 1)
     k_grouped_gemm(const __grid_constant__ GemmParams p) {
@@ -526,7 +535,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
     uint32_t phase = 0;
     long long issued = 0;
     int rows[4] = {0, 0, 0, 0};
-    for (int t = cluster; t < total; t += nclusters) {
+    for (int r = 0, t = snake_tile(0, cluster, nclusters); t < total;
+         t = snake_tile(++r, cluster, nclusters)) {
       const Tile tl = decode<MODE>(p, t, ustart, rank);
       if (MODE == MODE_WGRAD && tl.kit == 0) continue;  // zero tile: see the peer's warp 1
       if (MODE == MODE_GLU_GATHER) gather_rows(p, tl, lane, rows);
@@ -579,7 +589,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
     uint32_t phase = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = cluster; t < total; t += nclusters) {
+    for (int r = 0, t = snake_tile(0, cluster, nclusters); t < total;
+         t = snake_tile(++r, cluster, nclusters)) {
       const Tile tl = decode<MODE>(p, t, ustart, rank);
       if (tl.kit == 0) continue;  // weight gradient of an expert without rows: no MMA
       if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.status, abort_flag, p.wait_cycles)) break;
@@ -622,7 +633,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
     // Experts without rows have zero weight gradients.  Both halves of such a pair tile are
     // stored here from the zero box, as a background stream of TMA stores that overlaps the
     // other tiles' MMAs and never touches the accumulator hand-off.
-    for (int t = cluster; t < total; t += nclusters) {
+    for (int r = 0, t = snake_tile(0, cluster, nclusters); t < total;
+         t = snake_tile(++r, cluster, nclusters)) {
 #pragma unroll 1
       for (uint32_t half = 0; half < 2; ++half) {
         const Tile tl = decode<MODE>(p, t, ustart, half);
@@ -650,7 +662,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
     st.lane = lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = cluster; t < total; t += nclusters) {
+    for (int r = 0, t = snake_tile(0, cluster, nclusters); t < total;
+         t = snake_tile(++r, cluster, nclusters)) {
       const Tile tl = decode<MODE>(p, t, ustart, rank);
       if (tl.kit == 0) continue;  // WGRAD zero tile: stored by the producer warp
       const float wr = epilogue_prologue<MODE>(p, tl, sub, lane);
