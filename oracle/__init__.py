@@ -19,6 +19,10 @@ cites the passage of the pages it follows, in the C source:
 * ``backward``, ``backward_tokens``, ``wgrad_elements`` -- chain rule per (token, slot);
                          role swap and routing-weight gradient of walkthrough §4.2, activation
                          recompute of §4.4.
+* ``router_logits``, ``router_backward`` -- the linear router whose output is the issue's
+                         ``(scores, top_experts)`` (walkthrough §4.5 ``router(x)``), and the
+                         chain rule through the softmax routing weights into the logits, the
+                         router input and the router weight.
 
 Pins (tests/test_oracle_pins.py) tie every routine to something other than itself: brute
 force, closed forms, library special cases, the walkthrough's block diagram (§3), invariants
@@ -63,8 +67,11 @@ def _load():
         lib.oracle_backward.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P, P]
         lib.oracle_backward_tokens.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, P, I]
         lib.oracle_wgrad_elements.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, I]
+        lib.oracle_router_logits.argtypes = [I, I, I, P, P, I, P, P, I]
+        lib.oracle_router_backward.argtypes = [I, I, I, I, P, P, P, P, P, P, I, P, P, I, P, P, I]
         for fn in (lib.oracle_route, lib.oracle_sparse_map, lib.oracle_forward, lib.oracle_backward,
-                   lib.oracle_backward_tokens, lib.oracle_wgrad_elements, lib.oracle_max_threads):
+                   lib.oracle_backward_tokens, lib.oracle_wgrad_elements, lib.oracle_max_threads,
+                   lib.oracle_router_logits, lib.oracle_router_backward):
             fn.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -200,3 +207,50 @@ def wgrad_elements(x, dy, W1, W3, W2, top_experts, weights, queries, threads=1):
     if rc != 0:
         raise RuntimeError(f"oracle_wgrad_elements failed ({rc})")
     return out
+
+
+def router_logits(x, Wr, tokens=None, threads=1):
+    """logits [n,E] float64 = x[tokens] Wr^T (all tokens when ``tokens`` is None)."""
+    x, Wr = _f32(x), _f32(Wr)
+    T, h = x.shape
+    E = Wr.shape[0]
+    toks = None if tokens is None else _i32(tokens)
+    n = T if toks is None else toks.shape[0]
+    out = np.empty((n, E), np.float64)
+    rc = _load().oracle_router_logits(T, h, E, _p(x), _p(Wr), n,
+                                      None if toks is None else _p(toks), _p(out), int(threads))
+    if rc != 0:
+        raise ValueError(f"oracle_router_logits failed ({rc})")
+    return out
+
+
+def router_backward(x, Wr, logits, top_experts, dweights, tokens=None, elems=None,
+                    want_dx=True, want_dwr=True, threads=1):
+    """Gradient through the routing weights.  Returns dict dlogits [T,E], dx_r ([n,h] for
+    ``tokens`` or [T,h]) and dWr ([len(elems)] for ``elems`` = [(e, c), ...] or [E,h]),
+    all float64."""
+    x, Wr, lg = _f32(x), _f32(Wr), _f32(logits)
+    top, dw = _i32(top_experts), _f64(dweights)
+    T, h = x.shape
+    E = Wr.shape[0]
+    k = top.shape[1]
+    dl = np.empty((T, E), np.float64)
+    toks = None if tokens is None else _i32(tokens)
+    n_tok = T if toks is None else toks.shape[0]
+    dx = np.empty((n_tok, h), np.float64) if want_dx else None
+    el = None if elems is None else _i32(np.asarray(elems).reshape(-1, 2))
+    n_el = E * h if el is None else el.shape[0]
+    dwr = np.empty(n_el, np.float64) if want_dwr else None
+    rc = _load().oracle_router_backward(
+        T, h, E, k, _p(x), _p(Wr), _p(lg), _p(top), _p(dw), _p(dl), n_tok,
+        None if toks is None else _p(toks), None if dx is None else _p(dx),
+        n_el, None if el is None else _p(el), None if dwr is None else _p(dwr), int(threads))
+    if rc != 0:
+        raise ValueError(f"oracle_router_backward failed ({rc})")
+    out = dict(dlogits=dl)
+    if dx is not None:
+        out["dx_r"] = dx
+    if dwr is not None:
+        out["dWr"] = dwr if el is not None else dwr.reshape(E, h)
+    return out
+

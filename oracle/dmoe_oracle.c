@@ -99,6 +99,7 @@ int oracle_route(int T, int E, int k, const float *logits, int32_t *top, double 
 int oracle_sparse_map(int T, int E, int k, const int32_t *top, int32_t *counts, int32_t *bins,
                       int32_t *padded_bins, int32_t *indices, int32_t *bin_ids, int32_t *dest_row,
                       int32_t *block_expert, int nblk_cap, int32_t *num_blocks) {
+  if (T < 0 || E < 1 || k < 1) return -1;
   const long N = (long)T * k;
   for (long j = 0; j < N; ++j)
     if (top[j] < 0 || top[j] >= E) return -3;
@@ -392,6 +393,108 @@ int oracle_wgrad_elements(int T, int h, int f, int E, int k, const float *x, con
     }
     out[n] = acc;
   }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Router GEMM and the gradient through the routing weights.                             */
+/* ------------------------------------------------------------------------------------ */
+
+/* Router scores: the "router(x)" step of the walkthrough's schematic forward (section 4.5)
+ * whose output the issue's error log shows as (scores, top_experts).  The pages fix only that
+ * output; the plainest reading is a linear router without bias:
+ *   logits[t][e] = sum_i x[t][i] * Wr[e][i],   Wr [E, h] in the (out, in) layout.
+ * tokens: n token ids, or NULL for all T tokens (then n = T).  out: [n, E] double. */
+int oracle_router_logits(int T, int h, int E, const float *x, const float *Wr, int n,
+                         const int32_t *tokens, double *out, int threads) {
+  if (T < 0 || h < 1 || E < 1 || n < 0) return -1;
+  if (!tokens && n != T) return -1;
+#ifdef _OPENMP
+  if (threads > 0) omp_set_num_threads(threads);
+#pragma omp parallel for schedule(dynamic, 4) if (threads > 1)
+#endif
+  for (int q = 0; q < n; ++q) {
+    const int t = tokens ? tokens[q] : q;
+    const float *xt = x + (size_t)t * h;
+    for (int e = 0; e < E; ++e) {
+      const float *we = Wr + (size_t)e * h;
+      double acc = 0.0;
+      for (int i = 0; i < h; ++i) acc += (double)xt[i] * (double)we[i];
+      out[(size_t)q * E + e] = acc;
+    }
+  }
+  (void)threads;
+  return 0;
+}
+
+/* Gradient through the routing weights of oracle_route (softmax over all E logits read at the
+ * k chosen experts, no renormalisation); the choice of experts is piecewise constant, so it
+ * carries no gradient.  With p_t = softmax(logits_t) and j_s = top[t][s]:
+ *   w_ts = p_t[j_s],   d w_ts / d l_ti = p_t[j_s] * ([i == j_s] - p_t[i]),
+ *   dlogits[t][i] = sum_s dw[t][s] * d w_ts / d l_ti                       (chain rule),
+ * and, through logits = x Wr^T,
+ *   dx_r[t][c] = sum_e dlogits[t][e] * Wr[e][c],   dWr[e][c] = sum_t dlogits[t][e] * x[t][c].
+ * logits [T, E] are the routed scores (fp32 widened from bf16), dw [T, k] double.
+ * dlogits: [T, E] double out (always computed).
+ * dx_r: [n_tok, h] for tokens (NULL = all T, n_tok = T); skipped when dx_r is NULL.
+ * dWr: one value per (e, c) pair of `elems` ([n_el, 2] int32), or the full [E, h] when elems
+ *      is NULL; skipped when dWr is NULL. */
+int oracle_router_backward(int T, int h, int E, int k, const float *x, const float *Wr,
+                           const float *logits, const int32_t *top, const double *dw,
+                           double *dlogits, int n_tok, const int32_t *tokens, double *dx_r,
+                           int n_el, const int32_t *elems, double *dWr, int threads) {
+  if (T < 0 || h < 1 || E < 1 || k < 1 || k > E) return -1;
+  if (!tokens && dx_r && n_tok != T) return -1;
+  double *prob = (double *)malloc(sizeof(double) * (size_t)E);
+  if (!prob) return -2;
+  for (int t = 0; t < T; ++t) {
+    const float *l = logits + (size_t)t * E;
+    double m = -INFINITY;
+    for (int e = 0; e < E; ++e)
+      if ((double)l[e] > m) m = (double)l[e];
+    double z = 0.0;
+    for (int e = 0; e < E; ++e) z += exp((double)l[e] - m);
+    for (int e = 0; e < E; ++e) prob[e] = exp((double)l[e] - m) / z;
+    for (int i = 0; i < E; ++i) {
+      double g = 0.0;
+      for (int s = 0; s < k; ++s) {
+        const int j = top[(size_t)t * k + s];
+        if (j < 0 || j >= E) continue;
+        g += dw[(size_t)t * k + s] * prob[j] * ((i == j ? 1.0 : 0.0) - prob[i]);
+      }
+      dlogits[(size_t)t * E + i] = g;
+    }
+  }
+  free(prob);
+  if (dx_r) {
+#ifdef _OPENMP
+    if (threads > 0) omp_set_num_threads(threads);
+#pragma omp parallel for schedule(dynamic, 4) if (threads > 1)
+#endif
+    for (int q = 0; q < n_tok; ++q) {
+      const int t = tokens ? tokens[q] : q;
+      for (int c = 0; c < h; ++c) {
+        double acc = 0.0;
+        for (int e = 0; e < E; ++e) acc += dlogits[(size_t)t * E + e] * (double)Wr[(size_t)e * h + c];
+        dx_r[(size_t)q * h + c] = acc;
+      }
+    }
+  }
+  if (dWr) {
+    const int n = elems ? n_el : E * h;
+#ifdef _OPENMP
+    if (threads > 0) omp_set_num_threads(threads);
+#pragma omp parallel for schedule(dynamic, 16) if (threads > 1)
+#endif
+    for (int q = 0; q < n; ++q) {
+      const int e = elems ? elems[2 * q] : q / h;
+      const int c = elems ? elems[2 * q + 1] : q % h;
+      double acc = 0.0;
+      for (int t = 0; t < T; ++t) acc += dlogits[(size_t)t * E + e] * (double)x[(size_t)t * h + c];
+      dWr[q] = acc;
+    }
+  }
+  (void)threads;
   return 0;
 }
 

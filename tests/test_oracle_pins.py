@@ -12,6 +12,11 @@ Forward  -- closed form with permutation/selection weights (catches transposed o
 Backward -- central finite differences of the oracle's own forward (in double) for x, W1,
             W3, W2 and the routing weights; dw = <dy, y_ts>; linearity in dy; the sampled
             routines against the full backward.
+Router   -- logits: one-hot tokens read a column of the router weight (closed form), numpy's
+            float64 matmul (library); gradient through the routing weights: central finite
+            differences of sum dw * softmax(x Wr^T)[picks] in the logits, x and Wr; torch
+            float64 autograd of the same composition; shift invariance (each token's logit
+            gradient sums to zero); k = E with equal dw gives zero; sampled = full.
 """
 import itertools
 import json
@@ -362,3 +367,100 @@ def test_backward_sampled_routines_match_full(oracle_mod):
     full = {1: g["dW1"], 3: g["dW3"], 2: g["dW2"]}
     ref = np.array([full[a][b, c, d] for a, b, c, d in q])
     np.testing.assert_allclose(vals, ref, rtol=1e-11, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------------------
+# router GEMM and the gradient through the routing weights
+# ----------------------------------------------------------------------------------------
+
+def _router_loss(lg64, top, dw):
+    """sum_t sum_s dw_ts * softmax(l_t)[top_ts], in float64 (picks held fixed)."""
+    z = lg64 - lg64.max(1, keepdims=True)
+    p = np.exp(z)
+    p /= p.sum(1, keepdims=True)
+    return float((dw * np.take_along_axis(p, top.astype(np.int64), 1)).sum())
+
+
+def test_router_logits_closed_form_and_library_matmul(oracle_mod):
+    rng = np.random.default_rng(61)
+    T, h, E = 7, 48, 5
+    Wr = rng.standard_normal((E, h)).astype(np.float32)
+    x = np.zeros((T, h), np.float32)
+    cols = rng.integers(0, h, T)
+    x[np.arange(T), cols] = 1.0
+    lg = oracle_mod.router_logits(x, Wr)
+    assert (lg == Wr[:, cols].T.astype(np.float64)).all()  # a one-hot token reads a column
+    x = rng.standard_normal((T, h)).astype(np.float32)
+    lg = oracle_mod.router_logits(x, Wr)
+    np.testing.assert_allclose(lg, x.astype(np.float64) @ Wr.astype(np.float64).T,
+                               rtol=1e-13, atol=1e-12)
+    assert (oracle_mod.router_logits(x, Wr, tokens=np.array([6, 0, 3])) == lg[[6, 0, 3]]).all()
+
+
+def _router_case(oracle_mod, seed, T=6, h=32, E=7, k=3):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((T, h)).astype(np.float32)
+    Wr = (0.3 * rng.standard_normal((E, h))).astype(np.float32)
+    lg = (x.astype(np.float64) @ Wr.astype(np.float64).T).astype(np.float32)
+    top, _ = oracle_mod.route(lg, k)
+    dw = rng.standard_normal((T, k))
+    return x, Wr, lg, top, dw
+
+
+def test_router_backward_finite_differences(oracle_mod):
+    x, Wr, lg, top, dw = _router_case(oracle_mod, 67)
+    g = oracle_mod.router_backward(x, Wr, lg, top, dw)
+    T, E = lg.shape
+    l64 = lg.astype(np.float64)
+    eps = 1e-6
+    for t in range(T):  # every logit: the picks stay fixed under a perturbation this small
+        for i in range(E):
+            lp, lm = l64.copy(), l64.copy()
+            lp[t, i] += eps
+            lm[t, i] -= eps
+            fd = (_router_loss(lp, top, dw) - _router_loss(lm, top, dw)) / (2 * eps)
+            assert abs(fd - g["dlogits"][t, i]) <= 1e-8 + 1e-6 * abs(fd), (t, i)
+    # through logits = x Wr^T: perturb x and Wr (the oracle's dlogits is taken at the
+    # fp32-rounded logits, hence the looser relative bound)
+    rng = np.random.default_rng(71)
+    x64, W64 = x.astype(np.float64), Wr.astype(np.float64)
+    for _ in range(12):
+        t, c = int(rng.integers(T)), int(rng.integers(x.shape[1]))
+        xp, xm = x64.copy(), x64.copy()
+        xp[t, c] += eps
+        xm[t, c] -= eps
+        fd = (_router_loss(xp @ W64.T, top, dw) - _router_loss(xm @ W64.T, top, dw)) / (2 * eps)
+        assert abs(fd - g["dx_r"][t, c]) <= 1e-7 + 1e-5 * abs(fd), ("x", t, c)
+        e = int(rng.integers(E))
+        wp, wm = W64.copy(), W64.copy()
+        wp[e, c] += eps
+        wm[e, c] -= eps
+        fd = (_router_loss(x64 @ wp.T, top, dw) - _router_loss(x64 @ wm.T, top, dw)) / (2 * eps)
+        assert abs(fd - g["dWr"][e, c]) <= 1e-7 + 1e-5 * abs(fd), ("Wr", e, c)
+
+
+def test_router_backward_autograd_and_invariants(oracle_mod):
+    x, Wr, lg, top, dw = _router_case(oracle_mod, 73, T=9, h=40, E=8, k=4)
+    g = oracle_mod.router_backward(x, Wr, lg, top, dw)
+    l = torch.tensor(lg, dtype=torch.float64, requires_grad=True)
+    p = torch.softmax(l, dim=1)
+    (torch.tensor(dw) * p.gather(1, torch.from_numpy(top).long())).sum().backward()
+    np.testing.assert_allclose(g["dlogits"], l.grad.numpy(), rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(g["dx_r"], l.grad.numpy() @ Wr.astype(np.float64), rtol=1e-12,
+                               atol=1e-14)
+    np.testing.assert_allclose(g["dWr"], l.grad.numpy().T @ x.astype(np.float64), rtol=1e-12,
+                               atol=1e-14)
+    # softmax is shift-invariant: each token's logit gradient sums to zero
+    assert np.abs(g["dlogits"].sum(1)).max() <= 1e-14
+    # all experts picked with the same dw: the weights sum to 1, so no gradient reaches the logits
+    T, E = lg.shape
+    topE, _ = oracle_mod.route(lg, E)
+    z = oracle_mod.router_backward(x, Wr, lg, topE, np.full((T, E), 0.7))
+    assert np.abs(z["dlogits"]).max() <= 1e-15
+    # sampled routines equal the full ones
+    toks = np.array([8, 2, 5])
+    el = np.array([[0, 3], [7, 39], [4, 0]])
+    s = oracle_mod.router_backward(x, Wr, lg, top, dw, tokens=toks, elems=el)
+    assert (s["dx_r"] == g["dx_r"][toks]).all()
+    assert (s["dWr"] == g["dWr"][el[:, 0], el[:, 1]]).all()
+
