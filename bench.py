@@ -44,6 +44,9 @@ def parse():
     p.add_argument("--shape", default="",
                    help="T,hidden,ffn,E,top_k[,bwd][,zipf]: a custom workload (forward, or "
                         "fwd+bwd; zipf adds the skewed workload's logit bias)")
+    p.add_argument("--router", action="store_true",
+                   help="compute the logits with the linear router (x W_r^T) inside the step and, "
+                        "for fwd+bwd workloads, run the router backward after the layer's")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample", type=int, default=0, help="tokens in the oracle sample")
     return p.parse_args()
@@ -137,29 +140,37 @@ class ClockSampler:
 # reference arm / CPU baseline: the oracle on the host cores
 # ------------------------------------------------------------------------------------------------
 
-def oracle_sample_run(w, inp32, n_tok, threads):
-    """One bounded sample of the workload through the oracle: routing + map over all tokens,
-    forward of the first n_tok tokens.  Returns (seconds, tokens)."""
+def oracle_sample_run(w, inp32, n_tok, threads, router=False):
+    """One bounded sample of the workload through the oracle: (the router's logits and)
+    routing + map over all tokens, forward (and backward) of the first n_tok tokens.
+    Returns (seconds, tokens)."""
     import numpy as np
 
     import oracle
 
     t0 = time.perf_counter()
-    top, wts = oracle.route(inp32["logits"], w.top_k)
+    logits = inp32["logits"]
+    if router:
+        logits = oracle.router_logits(inp32["x"], inp32["w_router"], threads=threads)
+        logits = logits.astype(np.float32)
+    top, wts = oracle.route(logits, w.top_k)
     oracle.sparse_map(top, w.E)
     toks = np.arange(n_tok, dtype=np.int32)
     oracle.forward(inp32["x"], inp32["w1"], inp32["w3"], inp32["w2"], top, wts, tokens=toks,
                    threads=threads)
     if w.backward:  # the sample's own backward: dx, dw and its weight-gradient contributions
-        oracle.backward(inp32["x"][:n_tok], inp32["dy"][:n_tok], inp32["w1"], inp32["w3"],
-                        inp32["w2"], top[:n_tok], wts[:n_tok])
+        g = oracle.backward(inp32["x"][:n_tok], inp32["dy"][:n_tok], inp32["w1"], inp32["w3"],
+                            inp32["w2"], top[:n_tok], wts[:n_tok])
+        if router:
+            oracle.router_backward(inp32["x"][:n_tok], inp32["w_router"], logits[:n_tok],
+                                   top[:n_tok], g["dw"], threads=threads)
     return time.perf_counter() - t0, n_tok
 
 
-def oracle_inputs32(w):
+def oracle_inputs32(w, router=False):
     from dropless_mixture_experts_dmoe_b200.workloads import make_inputs
 
-    inp = make_inputs(w)
+    inp = make_inputs(w, with_router=router)
     return {k: v.float().numpy() for k, v in inp.items()}
 
 
@@ -181,13 +192,13 @@ def run_reference(args, w):
         return
     oracle.build()
     threads = oracle.max_threads()
-    inp32 = oracle_inputs32(w)
+    inp32 = oracle_inputs32(w, router=args.router)
     # calibrate on a 4-token sample, then size each step so the K steps take about a minute
-    dt4, _ = oracle_sample_run(w, inp32, 4, threads)
+    dt4, _ = oracle_sample_run(w, inp32, 4, threads, router=args.router)
     n_tok = int(max(1, min(w.T, 60.0 / max(args.steps, 1) / (dt4 / 4))))
     times = []
     for _ in range(args.steps):
-        dt, _ = oracle_sample_run(w, inp32, n_tok, threads)
+        dt, _ = oracle_sample_run(w, inp32, n_tok, threads, router=args.router)
         times.append(dt)
     total = sum(times)
     value = n_tok * args.steps / total
@@ -198,7 +209,8 @@ def run_reference(args, w):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{w.name} {w.describe()}", "T": w.T, "hidden": w.hidden,
+        "config": {"workload": f"{w.name} {w.describe()}" + (" +router" if args.router else ""),
+                   "T": w.T, "hidden": w.hidden,
                    "ffn": w.ffn, "num_experts": w.E, "top_k": w.top_k},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
@@ -236,8 +248,11 @@ def run_ours(args, w):
 
     dims = B.make_dims(w.T, w.hidden, w.ffn, w.E, w.top_k)
     train = w.backward
-    inp = make_inputs(w, with_dy=train)
+    router = bool(args.router)
+    inp = make_inputs(w, with_dy=train, with_router=router)
     dev = {k: v.cuda() for k, v in inp.items()}
+    if router:  # the step computes its own logits
+        dev["logits"] = torch.empty((w.T, w.E), dtype=torch.bfloat16, device="cuda")
     bufs = B.Buffers(dims, train=train)
     y = torch.empty((w.T, w.hidden), dtype=torch.bfloat16, device="cuda")
     st = torch.cuda.current_stream()
@@ -255,6 +270,11 @@ def run_ours(args, w):
     names = ["map", "gather", "glu_gemm", "down_gemm", "scatter"]
     if train:
         names += ["dy_gather", "dglu_gemm", "wgrad_gemm", "dx_gemm", "dx_scatter"]
+    if router:
+        names = ["router_gemm"] + names + (["router_bwd"] if train else [])
+        dwr = torch.empty((w.E, w.hidden), dtype=torch.float32, device="cuda")
+        ws_router = torch.empty(B.dmoe_workspace_bytes(dims, B.WS_ROUTER_BACKWARD),
+                                dtype=torch.uint8, device="cuda")
     n_ev = len(names) + 1
 
     def step(ev=None):
@@ -263,6 +283,10 @@ def run_ours(args, w):
                 ev[i].record(st)
         i = 0
         mark(i)
+        if router:
+            B.dmoe_router_forward(dims, dev["x"], dev["w_router"], dev["logits"], bufs.map.status, st)
+            i += 1
+            mark(i)
         B.dmoe_sparse_map(dims, dev["logits"], bufs.map, bufs.ws_map, st)
         i += 1
         mark(i)
@@ -292,6 +316,10 @@ def run_ours(args, w):
             mark(i + 4)
             B.dmoe_bwd_scatter(dims, bs["dy_pad"], bs["dw_part"], bufs.map, grads["dx"], grads["dw"], st)
             mark(i + 5)
+            if router:  # dlogits, dx += dlogits W_r, dW_r (4 kernels)
+                B.dmoe_router_backward(dims, dev["x"], dev["w_router"], dev["logits"], bufs.map,
+                                       grads["dw"], grads["dx"], dwr, ws_router, st)
+                mark(i + 6)
 
     for _ in range(args.warmup):
         step()
@@ -337,7 +365,7 @@ def run_ours(args, w):
     nbuf = 2
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     x_h = [inp["x"].pin_memory() for _ in range(nbuf)]
-    lg_h = [inp["logits"].pin_memory() for _ in range(nbuf)]
+    lg_h = [inp["logits"].pin_memory() for _ in range(nbuf)] if not router else []
     y_h = [torch.empty((w.T, w.hidden), dtype=torch.bfloat16).pin_memory() for _ in range(nbuf)]
     x_d = [torch.empty_like(dev["x"]) for _ in range(nbuf)]
     lg_d = [torch.empty_like(dev["logits"]) for _ in range(nbuf)]
@@ -358,13 +386,16 @@ def run_ours(args, w):
             if used[j]:
                 s_in.wait_event(ev_comp[j])  # the compute that read this buffer is done
             x_d[j].copy_(x_h[j], non_blocking=True)
-            lg_d[j].copy_(lg_h[j], non_blocking=True)
+            if not router:
+                lg_d[j].copy_(lg_h[j], non_blocking=True)
             if train:
                 dy_d[j].copy_(dy_h[j], non_blocking=True)
             ev_in[j].record(s_in)
         st.wait_event(ev_in[j])
         if used[j]:
             st.wait_event(ev_out[j])  # the results of this buffer have been copied out
+        if router:
+            B.dmoe_router_forward(dims, x_d[j], dev["w_router"], lg_d[j], bufs.map.status, st)
         B.dmoe_sparse_map(dims, lg_d[j], bufs.map, bufs.ws_map, st)
         if train:
             B.dmoe_forward(dims, x_d[j], dev["w1"], dev["w3"], dev["w2"], bufs.map, y_d[j], bufs.saved,
@@ -372,6 +403,9 @@ def run_ours(args, w):
             B.dmoe_backward(dims, dy_d[j], dev["w1"], dev["w3"], dev["w2"], bufs.map, bufs.saved,
                             dx_d[j], grads["dw1"], grads["dw3"], grads["dw2"], grads["dw"],
                             bufs.ws_bwd, st)
+            if router:
+                B.dmoe_router_backward(dims, x_d[j], dev["w_router"], lg_d[j], bufs.map,
+                                       grads["dw"], dx_d[j], dwr, ws_router, st)
         else:
             B.dmoe_forward(dims, x_d[j], dev["w1"], dev["w3"], dev["w2"], bufs.map, y_d[j], None,
                            bufs.ws_fwd, st)
@@ -401,7 +435,8 @@ def run_ours(args, w):
     if world > 1:
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
     e2e_value = world * w.T * args.steps / (float(te.item()) / 1e3)
-    h2d = x_h[0].numel() * 2 + lg_h[0].numel() * 2 + (dy_h[0].numel() * 2 if train else 0)
+    h2d = x_h[0].numel() * 2 + (0 if router else lg_h[0].numel() * 2) + \
+        (dy_h[0].numel() * 2 if train else 0)
     d2h = y_h[0].numel() * 2 + (dx_h[0].numel() * 2 if train else 0)
     # the pipelined e2e output is checked against the device-resident one
     torch.cuda.synchronize()
@@ -429,18 +464,32 @@ def run_ours(args, w):
     nhf = N * w.hidden * w.ffn
     flops = dict(glu_gemm=4 * nhf, down_gemm=2 * nhf, dglu_gemm=2 * nhf, dx_gemm=4 * nhf,
                  wgrad_gemm=6 * nhf)
+    the = w.T * w.hidden * w.E
+    router_flops = dict(router_gemm=2 * the, router_bwd=4 * the)
+    if router:
+        useful += 2 * the + (4 * the if train else 0)
     byts = dict(
         map=2 * w.T * w.E + 8 * w.T * w.top_k + 12 * N,
         gather=2 * w.T * w.hidden + 2 * N * w.hidden,
         scatter=2 * N * w.hidden + 8 * N + 4 * N + 2 * w.T * w.hidden,
         dy_gather=2 * w.T * w.hidden + 2 * N * w.hidden,
         dx_scatter=2 * N * w.hidden + 4 * N + 2 * w.T * w.hidden
-        + 4 * N * ((w.ffn + 255) // 256) + 4 * N)
+        + 4 * N * ((w.ffn + 255) // 256) + 4 * N,
+        # router: x and W_r read, logits written; backward: logits, dweights, top read, dlogits
+        # written and read twice, dx read and written, x read, dW_r written
+        router_gemm=2 * w.T * w.hidden + 2 * w.E * w.hidden + 2 * w.T * w.E,
+        router_bwd=2 * w.T * w.E + 8 * w.T * w.top_k + 3 * 2 * w.T * w.E + 4 * w.T * w.hidden
+        + 2 * w.T * w.hidden + 2 * w.E * w.hidden + 4 * w.E * w.hidden)
     km = {n: statistics.mean(v) for n, v in per_kernel.items()}
     kernels = {}
     for n in names:
         ent = {"ms": km[n]}
-        if n in flops:
+        if n in router_flops:  # small E: a thin GEMM, bound by bytes more than by the MMAs
+            ent["TFLOP/s"] = router_flops[n] / km[n] / 1e9
+            ent["frac_bf16"] = ent["TFLOP/s"] / pk["bf16_sus"]
+            ent["GB/s"] = byts[n] / km[n] / 1e6
+            ent["frac_hbm"] = ent["GB/s"] / pk["hbm"]
+        elif n in flops:
             ent["TFLOP/s"] = flops[n] / km[n] / 1e9
             ent["frac_bf16"] = ent["TFLOP/s"] / pk["bf16_sus"]
         else:
@@ -449,7 +498,7 @@ def run_ours(args, w):
         kernels[n] = ent
     dom = max(flops.keys() & set(names), key=lambda n: km[n])
     achieved = flops[dom] / km[dom] / 1e9
-    wl_name = f"{w.name} {w.describe()}"
+    wl_name = f"{w.name} {w.describe()}" + (" +router" if router else "")
     traffic = ncu_traffic(dom, w.name)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -473,7 +522,7 @@ def run_ours(args, w):
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "pipelined": "copies overlap compute (3 streams)",
                 "output_matches_device_run": e2e_matches},
-        "gpu_launches": (len(names) + 2) * args.steps,
+        "gpu_launches": (len(names) + 2 + (3 if router and train else 0)) * args.steps,
         "gpu_launches_note": "kernels of this library in the device-resident timed region",
         "status": status,
     }
@@ -487,10 +536,10 @@ def run_ours(args, w):
             threads = oracle.max_threads()
             inp32 = {k: v.float().numpy() for k, v in inp.items()}
             n_tok = cpu_sample_tokens(w, args.cpu_sample)
-            dt, nt = oracle_sample_run(w, inp32, n_tok, threads)
+            dt, nt = oracle_sample_run(w, inp32, n_tok, threads, router=router)
             line["cpu_baseline"] = {
                 "value": nt / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                "sample": f"routing+map over all {w.T} tokens + forward"
+                "sample": f"{'router logits + ' if router else ''}routing+map over all {w.T} tokens + forward"
                           f"{' and backward' if w.backward else ''} of {nt} tokens "
                           f"({dt:.1f} s, fp64 accumulation, OpenMP over tokens)"}
         except Exception as ex:  # the baseline is reported, never required

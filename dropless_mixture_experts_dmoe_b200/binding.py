@@ -20,7 +20,7 @@ BLOCKING = 128
 MAX_EXPERTS = 1024
 MAX_TOP_K = 32
 
-WS_MAP, WS_FORWARD, WS_BACKWARD, WS_FORWARD_TRAIN = 0, 1, 2, 3
+WS_MAP, WS_FORWARD, WS_BACKWARD, WS_FORWARD_TRAIN, WS_ROUTER_BACKWARD = 0, 1, 2, 3, 4
 DGLU_TILE_COLS = 256
 
 STATUS_NONFINITE_LOGITS = 0x1
@@ -86,11 +86,15 @@ def load():
     lib.dmoe_padded_scatter.argtypes = [D, _P, M, _P, _P, _P]
     lib.dmoe_bwd_dglu.argtypes = [D, _P, _P, _P, _P, M, _P, _P, _P, _P, _P]
     lib.dmoe_bwd_scatter.argtypes = [D, _P, _P, M, _P, _P, _P]
+    lib.dmoe_router_forward.argtypes = [D, _P, _P, _P, _P, _P]
+    lib.dmoe_router_dlogits.argtypes = [D, _P, M, _P, _P, _P]
+    lib.dmoe_router_backward.argtypes = [D, _P, _P, _P, M, _P, _P, _P, _P, _SZ, _P]
     lib.dmoe_bwd_dx.argtypes = [D, _P, _P, _P, _P, M, _P, _P]
     lib.dmoe_bwd_wgrad.argtypes = [D, _P, _P, _P, _P, _P, M, _P, _P, _P, _P]
     for fn in ("dmoe_sparse_map", "dmoe_forward", "dmoe_backward", "dmoe_padded_gather",
                "dmoe_expert_glu", "dmoe_expert_glu_gather", "dmoe_expert_down", "dmoe_padded_scatter",
-               "dmoe_bwd_dglu", "dmoe_bwd_dx", "dmoe_bwd_wgrad", "dmoe_bwd_scatter"):
+               "dmoe_bwd_dglu", "dmoe_bwd_dx", "dmoe_bwd_wgrad", "dmoe_bwd_scatter",
+               "dmoe_router_forward", "dmoe_router_dlogits", "dmoe_router_backward"):
         getattr(lib, fn).restype = _I
     lib.dmoe_error_string.argtypes = [_I]
     lib.dmoe_error_string.restype = ctypes.c_char_p
@@ -275,6 +279,28 @@ def dmoe_bwd_wgrad(dims, x_pad, hw, dy_pad, da, dbm, smap: SparseMap, dw1, dw3, 
     _check(load().dmoe_bwd_wgrad(ctypes.byref(dims), _ptr(x_pad), _ptr(hw), _ptr(dy_pad),
                                  _ptr(da), _ptr(dbm), ctypes.byref(smap.c), _ptr(dw1), _ptr(dw3),
                                  _ptr(dw2), _stream(stream)), "dmoe_bwd_wgrad")
+
+
+def dmoe_router_forward(dims, x, w_router, logits, status, stream=None):
+    """logits [T,E] bf16 = x W_r^T (the linear router; E % 8 == 0)."""
+    _check(load().dmoe_router_forward(ctypes.byref(dims), _ptr(x), _ptr(w_router), _ptr(logits),
+                                      _ptr(status), _stream(stream)), "dmoe_router_forward")
+
+
+def dmoe_router_dlogits(dims, logits, smap: SparseMap, dweights, dlogits, stream=None):
+    _check(load().dmoe_router_dlogits(ctypes.byref(dims), _ptr(logits), ctypes.byref(smap.c),
+                                      _ptr(dweights), _ptr(dlogits), _stream(stream)),
+           "dmoe_router_dlogits")
+
+
+def dmoe_router_backward(dims, x, w_router, logits, smap: SparseMap, dweights, dx, dw_router, ws,
+                         stream=None):
+    """dx += dlogits W_r (in place), dw_router = dlogits^T x (fp32)."""
+    ws_bytes = ws.numel() * ws.element_size()
+    _check(load().dmoe_router_backward(ctypes.byref(dims), _ptr(x), _ptr(w_router), _ptr(logits),
+                                       ctypes.byref(smap.c), _ptr(dweights), _ptr(dx),
+                                       _ptr(dw_router), _ptr(ws), ws_bytes, _stream(stream)),
+           "dmoe_router_backward")
 
 
 def dmoe_sparse_map_noalloc(dims: dmoe_dims, logits, smap: SparseMap, stream=None):

@@ -113,6 +113,27 @@ FwdLayout fwd_layout(const dmoe_dims *d) {
   return l;
 }
 
+// Router backward workspace: dlogits [T,E] bf16 | split-K partials of dW_r
+// [kRouterMaxSplits, round_up(E,128), h] fp32
+struct RouterLayout {
+  size_t dlogits, part, total;
+};
+RouterLayout router_layout(const dmoe_dims *d) {
+  RouterLayout l;
+  const size_t Ep = (size_t)(d->num_experts + DMOE_BLOCKING - 1) / DMOE_BLOCKING * DMOE_BLOCKING;
+  l.dlogits = 0;
+  l.part = align_up(l.dlogits + (size_t)d->T * d->num_experts * 2);
+  l.total = align_up(l.part + (size_t)kRouterMaxSplits * Ep * d->hidden * sizeof(float));
+  return l;
+}
+
+// The router's tensors have E columns; a TMA row must be a multiple of 16 bytes.
+inline int check_router_dims(const dmoe_dims *d) {
+  int rc = check_dims(d);
+  if (rc) return rc;
+  return (d->num_experts % 8 == 0) ? DMOE_OK : DMOE_ERR_SHAPE;
+}
+
 // Saved activations: X_pad [P,h] | A [P,f] | Bm [P,f]
 void saved_layout(const dmoe_dims *d, size_t off[3], size_t *total) {
   const size_t P = (size_t)pmax_of(d);
@@ -140,6 +161,8 @@ size_t dmoe_workspace_bytes(const dmoe_dims *dims, int kind) {
       return fwd_layout(dims).total;
     case DMOE_WS_FORWARD_TRAIN:
       return fwd_layout(dims).train;
+    case DMOE_WS_ROUTER_BACKWARD:
+      return router_layout(dims).total;
     case DMOE_WS_BACKWARD:
       return bwd_layout(dims).total;
     default:
@@ -366,6 +389,58 @@ int dmoe_backward(const dmoe_dims *dims, const void *dy, const void *w1, const v
   if ((rc = dmoe_bwd_wgrad(dims, xpad, hw, dypad, da, db, map, dw1, dw3, dw2, stream))) return rc;
   if ((rc = dmoe_bwd_dx(dims, da, db, w1, w3, map, dxpad, stream))) return rc;
   return dmoe_bwd_scatter(dims, dxpad, part, map, dx, dweights, stream);
+}
+
+int dmoe_router_forward(const dmoe_dims *dims, const void *x, const void *w_router, void *logits,
+                        int32_t *status, void *stream) {
+  int rc = check_router_dims(dims);
+  if (rc) return rc;
+  if (!x || !w_router || !logits || !status) return DMOE_ERR_NULL;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(logits)) return DMOE_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return launch_rc(launch_router_gemm(dims->T, dims->hidden, dims->num_experts, x, w_router,
+                                      logits, status, static_cast<cudaStream_t>(stream)));
+}
+
+int dmoe_router_dlogits(const dmoe_dims *dims, const void *logits, const dmoe_map *map,
+                        const float *dweights, void *dlogits, void *stream) {
+  int rc = check_router_dims(dims);
+  if (rc) return rc;
+  if (!logits || !map || !map->top_experts || !dweights || !dlogits) return DMOE_ERR_NULL;
+  if (!aligned16(logits) || !aligned16(dlogits)) return DMOE_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  return launch_rc(launch_router_dlogits(dims->T, dims->num_experts, dims->top_k,
+                                         static_cast<const uint16_t *>(logits), map->top_experts,
+                                         dweights, static_cast<uint16_t *>(dlogits),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+int dmoe_router_backward(const dmoe_dims *dims, const void *x, const void *w_router,
+                         const void *logits, const dmoe_map *map, const float *dweights,
+                         void *dx, float *dw_router, void *ws, size_t ws_bytes, void *stream) {
+  int rc = check_router_dims(dims);
+  if (rc) return rc;
+  if (!x || !w_router || !logits || !map || !map->top_experts || !map->status || !dweights ||
+      !dx || !dw_router || !ws)
+    return DMOE_ERR_NULL;
+  const RouterLayout l = router_layout(dims);
+  if (ws_bytes < l.total) return DMOE_ERR_WORKSPACE;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(logits) || !aligned16(dx) ||
+      !aligned16(dw_router) || !aligned16(ws))
+    return DMOE_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int T = dims->T, h = dims->hidden, E = dims->num_experts;
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  void *dl = w + l.dlogits;
+  float *part = reinterpret_cast<float *>(w + l.part);
+  if ((rc = dmoe_router_dlogits(dims, logits, map, dweights, dl, stream))) return rc;
+  if ((rc = launch_rc(launch_router_dx_gemm(T, h, E, dl, w_router, dx, map->status, st))))
+    return rc;
+  const int splits = router_wgrad_splits(T, h, E);
+  if ((rc = launch_rc(launch_router_wgrad_gemm(T, h, E, dl, x, part, splits, map->status, st))))
+    return rc;
+  return launch_rc(launch_router_wgrad_reduce(h, E, splits, part, dw_router, st));
 }
 
 const char *dmoe_error_string(int code) {

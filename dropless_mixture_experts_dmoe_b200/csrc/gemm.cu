@@ -49,6 +49,11 @@
 //   WGRAD dW1_e = dA^T X_pad, dW3_e = dBm^T X_pad, dW2_e = dY_pad^T Hw over the expert's
 //         padded rows (both operands MN-major); fp32 outputs; experts without rows get exact
 //         zeros.
+// and the dense GEMMs of the linear router (its output is the (scores, top_experts) pair of
+// the issue's error log; "router(x)" of walkthrough section 4.5), over T unpadded token rows:
+//   ROUTER  A = x (K)        B = W_r (K)                  out logits [T, E]
+//   RDX     A = dlogits (K)  B = W_r (MN)                 dx += dlogits W_r (read-add-store)
+//   RWGRAD  A = dlogits (MN) B = x (MN), K = tokens       fp32 partial dW_r per K split
 //
 // Every mbarrier wait is bounded; on expiry the kernel sets DMOE_STATUS_TIMEOUT, raises an
 // abort flag for the other roles of its CTA, drains what it issued and returns.
@@ -79,11 +84,26 @@ enum GemmMode {
   MODE_DGLU = 2,
   MODE_DX = 3,
   MODE_WGRAD = 4,
-  MODE_GLU_GATHER = 5  // GLU whose A rows are gathered from the token rows of x
+  MODE_GLU_GATHER = 5,  // GLU whose A rows are gathered from the token rows of x
+  MODE_ROUTER = 6,      // router logits
+  MODE_RDX = 7,         // router input gradient, accumulated into dx
+  MODE_RWGRAD = 8       // router weight gradient, split over the token dimension
 };
 
 __host__ __device__ constexpr bool is_glu(int mode) {
   return mode == MODE_GLU || mode == MODE_GLU_GATHER;
+}
+
+// Modes whose tiles are (pair of an expert's row blocks, column tile), enumerated from
+// padded_bins; the others are the weight gradients and the dense router GEMMs.
+__host__ __device__ constexpr bool uses_units(int mode) {
+  return mode == MODE_GLU || mode == MODE_GLU_GATHER || mode == MODE_DOWN ||
+         mode == MODE_DGLU || mode == MODE_DX;
+}
+
+// Dense row modes: tiles are (pair of 128-row blocks of the T token rows, column tile).
+__host__ __device__ constexpr bool is_dense_rows(int mode) {
+  return mode == MODE_ROUTER || mode == MODE_RDX;
 }
 
 // Per-launch configuration.  A 5-stage ring of 32 KB per CTA; 4 epilogue warps (one per TMEM
@@ -92,8 +112,11 @@ __host__ __device__ constexpr bool is_glu(int mode) {
 // short (4 stages per tile) that the epilogue, not the MMA, bounds a tile.
 template <int MODE, int EPI>
 struct Cfg {
-  static constexpr int a_mn = (MODE == MODE_WGRAD) ? 1 : 0;
-  static constexpr int b_mn = (MODE == MODE_DGLU || MODE == MODE_DX || MODE == MODE_WGRAD) ? 1 : 0;
+  static constexpr int a_mn = (MODE == MODE_WGRAD || MODE == MODE_RWGRAD) ? 1 : 0;
+  static constexpr int b_mn = (MODE == MODE_DGLU || MODE == MODE_DX || MODE == MODE_WGRAD ||
+                               MODE == MODE_RDX || MODE == MODE_RWGRAD)
+                                  ? 1
+                                  : 0;
   static constexpr int epi_warps = EPI;
   static constexpr int col_split = epi_warps / 4;  // warps per TMEM sub-partition
   static constexpr int threads = 64 + 32 * epi_warps;
@@ -125,6 +148,9 @@ struct GemmParams {
   const __nv_bfloat16 *in0, *in1;  // DGLU: saved A, Bm
   const float *weights;            // DGLU: routing weight of each flattened entry
   float *part;                     // DGLU: [P_max, n_tiles] partial routing-weight gradients
+  int total;                       // router modes: number of pair tiles
+  int split_k;                     // RWGRAD: 64-wide K steps per split
+  int Ep;                          // RWGRAD: rows of one split's slab (E rounded up to 128)
   int32_t *status;
 };
 
@@ -140,6 +166,29 @@ __device__ __forceinline__ Tile decode(const GemmParams &p, int t, const int *us
   Tile tl;
   tl.which = 0;
   tl.m = 0;
+  if (is_dense_rows(MODE)) {
+    const int u = t / p.n_tiles;
+    tl.n = t - u * p.n_tiles;
+    tl.e = 0;
+    tl.row0 = (2 * u + (int)rank) * BM;
+    tl.dummy = tl.row0 >= p.T;  // past the last token row: loads read zeros, nothing stored
+    tl.kit = p.k_iters;
+    return tl;
+  }
+  if (MODE == MODE_RWGRAD) {  // t -> (K split, pair of 128-row tiles of E, column tile)
+    const int mt = (p.E + BM - 1) / BM, mpairs = (mt + 1) / 2;
+    const int per_split = mpairs * p.n_tiles;
+    const int sp = t / per_split;
+    const int r = t - sp * per_split;
+    const int mp = r / p.n_tiles;
+    tl.n = r - mp * p.n_tiles;
+    tl.m = 2 * mp + (int)rank;
+    tl.dummy = tl.m >= mt;
+    tl.e = sp;
+    tl.row0 = sp * p.split_k * BK;
+    tl.kit = min(p.split_k, p.k_iters - sp * p.split_k);
+    return tl;
+  }
   if (MODE == MODE_WGRAD) {
     const int mt13 = p.f / BM, mt2 = p.h / BM;
     const int mp13 = (mt13 + 1) / 2, mp2 = (mt2 + 1) / 2;
@@ -243,6 +292,22 @@ __device__ __forceinline__ void load_stage(const GemmParams &p, const Tile &tl, 
     for (int c = 0; c < 2; ++c)
       tma_load_2d_pair(sb + c * CHUNK_BYTES, &p.tm[2 + pass], bar,
                        tl.n * BN + (2 * (int)rank + c) * 64, tl.e * p.f + kk * BK);
+  } else if (MODE == MODE_ROUTER) {
+    tma_load_2d_pair(sa, &p.tm[0], bar, kb * BK, tl.row0);
+    tma_load_2d_pair(sb, &p.tm[1], bar, kb * BK, tl.n * BN + (int)rank * (BN / 2));
+  } else if (MODE == MODE_RDX) {
+    tma_load_2d_pair(sa, &p.tm[0], bar, kb * BK, tl.row0);
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+      tma_load_2d_pair(sb + c * CHUNK_BYTES, &p.tm[1], bar, tl.n * BN + (2 * (int)rank + c) * 64,
+                       kb * BK);
+  } else if (MODE == MODE_RWGRAD) {
+    const int y = tl.row0 + kb * BK;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) tma_load_2d_pair(sa + c * CHUNK_BYTES, &p.tm[0], bar, tl.m * BM + c * 64, y);
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+      tma_load_2d_pair(sb + c * CHUNK_BYTES, &p.tm[1], bar, tl.n * BN + (2 * (int)rank + c) * 64, y);
   } else {  // MODE_WGRAD
     const int y = tl.row0 + kb * BK;
     const CUtensorMap *ta = &p.tm[tl.which];               // dA, dBm, dY_pad
@@ -300,9 +365,18 @@ __device__ __forceinline__ void pack_bf16_row(const uint32_t (&lo)[32], const ui
 // Work of a tile's epilogue that does not depend on the accumulator, done before waiting for
 // it: DGLU looks up the routing weight of this thread's row (a chain of dependent loads) and
 // starts pulling the row's saved A and Bm columns of the tile into L2.
-template <int MODE>
+template <int MODE, int EPI>
 __device__ __forceinline__ float epilogue_prologue(const GemmParams &p, const Tile &tl, int sub,
-                                                   int lane) {
+                                                   int half, int lane) {
+  if (MODE == MODE_RDX && !tl.dummy) {  // the dx values this thread will add to
+    constexpr int kw = BN / Cfg<MODE, EPI>::col_split;
+    const int grow = tl.row0 + sub * 32 + lane;
+    const int n0 = tl.n * BN + half * kw;
+    const int ncols = min(kw, p.h - n0);
+    if (grow < p.T)
+      for (int c = 0; c < ncols; c += 64) prefetch_l2(p.in0 + (size_t)grow * p.h + n0 + c);
+    return 0.0f;
+  }
   if (MODE != MODE_DGLU || tl.dummy) return 0.0f;
   const int grow = tl.row0 + sub * 32 + lane;
   const int n0 = tl.n * BN;
@@ -408,6 +482,63 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
       st.emit(&p.tmo[2], wh, n0 + c, y0);
     }
     p.part[(size_t)grow * p.n_tiles + tl.n] = dot;
+  } else if (MODE == MODE_ROUTER) {  // logits [T, E]: bf16 boxes, rows past T not stored
+    if (y0 >= p.T) return;
+    const int n0 = tl.n * BN;
+    const int ncols = min(BN, p.E - n0);
+    uint32_t v0[32], v1[32], w[32];
+#pragma unroll 1
+    for (int c = 0; c < ncols; c += 64) {
+      tmem_ld32(tb + c, v0);
+      tmem_ld32(tb + c + 32, v1);
+      tmem_ld_wait();
+      pack_bf16_row(v0, v1, w);
+      st.emit(&p.tmo[0], w, n0 + c, y0);
+    }
+  } else if (MODE == MODE_RDX) {  // dx [T, h] += accumulator, in fp32, rounded once
+    if (y0 >= p.T) return;
+    const int n0 = tl.n * BN + half * kw;  // this warp's columns
+    const int ncols = min(kw, p.h - n0);   // multiple of 64 (may be <= 0)
+    if (ncols <= 0) return;
+    tb += (uint32_t)(half * kw);
+    const int grow = y0 + lane;
+    const bool live = grow < p.T;
+#pragma unroll 1
+    for (int c = 0; c < ncols; c += 64) {
+      uint32_t v0[32], v1[32], w[32];
+      uint4 q[8];
+      tmem_ld32(tb + c, v0);
+      tmem_ld32(tb + c + 32, v1);
+      const uint4 *src = reinterpret_cast<const uint4 *>(p.in0 + (size_t)grow * p.h + n0 + c);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) q[i] = live ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const uint32_t ow = reinterpret_cast<const uint32_t *>(q)[i];
+        const float a0 = __uint_as_float(i < 16 ? v0[2 * i] : v1[2 * i - 32]);
+        const float a1 = __uint_as_float(i < 16 ? v0[2 * i + 1] : v1[2 * i - 31]);
+        w[i] = pack_bf16x2(bf16_lo(ow) + a0, bf16_hi(ow) + a1);
+      }
+      st.emit(&p.tmo[0], w, n0 + c, y0);
+    }
+  } else if (MODE == MODE_RWGRAD) {  // fp32 partial of split tl.e, slab rows [tl.e * Ep, +Ep)
+    const int r0 = tl.m * BM + sub * 32;
+    if (r0 >= p.E) return;
+    const int yw = tl.e * p.Ep + r0;
+    const int n0 = tl.n * BN;
+    const int ncols = min(BN, p.h - n0);
+    uint32_t v[32], w[32];
+    tmem_ld32(tb, v);
+    tmem_ld_wait();
+#pragma unroll 1
+    for (int c = 0; c < ncols; c += 32) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) w[i] = v[i];
+      if (c + 32 < ncols) tmem_ld32(tb + c + 32, v);
+      st.emit(&p.tmo[0], w, n0 + c, yw);
+      tmem_ld_wait();
+    }
   } else {  // MODE_WGRAD: fp32 results, boxes of 32 columns
     const int rows = (tl.which == 2) ? p.h : p.f;
     const int cols = (tl.which == 2) ? p.f : p.h;
@@ -482,7 +613,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
 #pragma unroll
     for (int i = 0; i < 5; ++i) prefetch_tmap(&p.tm[i]);
   }
-  if (MODE != MODE_WGRAD) {
+  if (uses_units(MODE)) {
     // units (pairs of row blocks) per expert -> exclusive prefix ustart[0..E]
     for (int e = threadIdx.x; e < p.E; e += C::threads) {
       const int blocks = (p.padded_bins[e] - ((e > 0) ? p.padded_bins[e - 1] : 0)) / BM;
@@ -518,7 +649,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
   const uint32_t tmem_base = *tmem_slot;
 
   int total;
-  if (MODE == MODE_WGRAD) {
+  if (!uses_units(MODE) && MODE != MODE_WGRAD) {
+    total = p.total;
+  } else if (MODE == MODE_WGRAD) {
     const int mp13 = (p.f / BM + 1) / 2, mp2 = (p.h / BM + 1) / 2;
     total = p.E * (2 * mp13 * ((p.h + BN - 1) / BN) + mp2 * ((p.f + BN - 1) / BN));
   } else {
@@ -666,7 +799,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
          t = snake_tile(++r, cluster, nclusters)) {
       const Tile tl = decode<MODE>(p, t, ustart, rank);
       if (tl.kit == 0) continue;  // WGRAD zero tile: stored by the producer warp
-      const float wr = epilogue_prologue<MODE>(p, tl, sub, lane);
+      const float wr = epilogue_prologue<MODE, EPI>(p, tl, sub, half, lane);
       if (!mbar_wait(&tfull[acc], acc_phase, p.status, abort_flag, p.wait_cycles)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * ACC_COLS);
@@ -913,6 +1046,82 @@ cudaError_t launch_wgrad_gemm(const GemmProblem &g, const void *x_pad, const voi
   const long long t13 = (long long)((g.f / BM + 1) / 2) * ((g.h + BN - 1) / BN);
   const long long t2 = (long long)((g.h / BM + 1) / 2) * ((g.f + BN - 1) / BN);
   return launch_gemm<MODE_WGRAD, 4>(p, (long long)g.E * (2 * t13 + t2), st);
+}
+
+// ---- the linear router's GEMMs (dense token rows) ----------------------------------------------
+
+static GemmParams dense_params(int T, int h, int E, int32_t *status) {
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.T = T;
+  p.h = h;
+  p.E = E;
+  p.group = 1;
+  p.outs = 1;
+  p.status = status;
+  return p;
+}
+
+static inline int row_units(int T) { return (T + 2 * BM - 1) / (2 * BM); }
+
+cudaError_t launch_router_gemm(int T, int h, int E, const void *x, const void *wr, void *logits,
+                               int32_t *status, cudaStream_t st) {
+  GemmParams p = dense_params(T, h, E, status);
+  if (!make_tmap(&p.tm[0], x, (uint64_t)T, h, BM) || !make_tmap(&p.tm[1], wr, (uint64_t)E, h, BN / 2) ||
+      !make_tmap(&p.tmo[0], logits, (uint64_t)T, E, 32))
+    return cudaErrorInvalidValue;
+  p.tm[2] = p.tm[3] = p.tm[4] = p.tm[0];
+  p.n_tiles = (E + BN - 1) / BN;
+  p.k_iters = h / BK;
+  p.total = row_units(T) * p.n_tiles;
+  return launch_gemm<MODE_ROUTER, 4>(p, p.total, st);
+}
+
+cudaError_t launch_router_dx_gemm(int T, int h, int E, const void *dlogits, const void *wr, void *dx,
+                                  int32_t *status, cudaStream_t st) {
+  GemmParams p = dense_params(T, h, E, status);
+  if (!make_tmap(&p.tm[0], dlogits, (uint64_t)T, E, BM) ||
+      !make_tmap(&p.tm[1], wr, (uint64_t)E, h, 64) || !make_tmap(&p.tmo[0], dx, (uint64_t)T, h, 32))
+    return cudaErrorInvalidValue;
+  p.tm[2] = p.tm[3] = p.tm[4] = p.tm[0];
+  p.in0 = static_cast<const __nv_bfloat16 *>(dx);
+  p.n_tiles = (h + BN - 1) / BN;
+  p.k_iters = (E + BK - 1) / BK;
+  p.total = row_units(T) * p.n_tiles;
+  // K = E is short (a few K steps per tile): the read-add-store epilogue bounds a tile, so it
+  // gets 8 warps (two per TMEM sub-partition, each half of the columns)
+  return launch_gemm<MODE_RDX, 8>(p, p.total, st);
+}
+
+int router_wgrad_splits(int T, int h, int E) {
+  const int mpairs = ((E + BM - 1) / BM + 1) / 2;
+  const int tiles = mpairs * ((h + BN - 1) / BN);
+  const int k_iters = (T + BK - 1) / BK;
+  int s = (device_sm_count() / 2) / tiles;  // at most one tile per SM pair: a single wave
+  s = min(s, kRouterMaxSplits);
+  s = min(s, k_iters);
+  if (s < 1) s = 1;
+  const int per = (k_iters + s - 1) / s;
+  return (k_iters + per - 1) / per;  // no empty split
+}
+
+cudaError_t launch_router_wgrad_gemm(int T, int h, int E, const void *dlogits, const void *x,
+                                     float *partials, int splits, int32_t *status,
+                                     cudaStream_t st) {
+  GemmParams p = dense_params(T, h, E, status);
+  p.Ep = (E + BM - 1) / BM * BM;
+  if (!make_tmap(&p.tm[0], dlogits, (uint64_t)T, E, 64) || !make_tmap(&p.tm[1], x, (uint64_t)T, h, 64) ||
+      !make_tmap(&p.tmo[0], partials, (uint64_t)splits * p.Ep, h, 32, 4))
+    return cudaErrorInvalidValue;
+  p.tm[2] = p.tm[3] = p.tm[4] = p.tm[0];
+  p.n_tiles = (h + BN - 1) / BN;
+  p.k_iters = (T + BK - 1) / BK;
+  p.split_k = (p.k_iters + splits - 1) / splits;
+  if (splits < 1 || splits > kRouterMaxSplits || (splits - 1) * p.split_k >= p.k_iters)
+    return cudaErrorInvalidValue;  // every split must own K steps: its slab is read back
+  const int mpairs = ((E + BM - 1) / BM + 1) / 2;
+  p.total = splits * mpairs * p.n_tiles;
+  return launch_gemm<MODE_RWGRAD, 4>(p, p.total, st);
 }
 
 }  // namespace dmoe

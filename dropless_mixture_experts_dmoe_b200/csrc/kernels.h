@@ -79,6 +79,25 @@ cudaError_t launch_wgrad_gemm(const GemmProblem &g, const void *x_pad, const voi
                               const void *dy_pad, const void *da, const void *db, float *dw1,
                               float *dw3, float *dw2, cudaStream_t st);
 
+// The linear router (dense rows over T tokens; E % 8 == 0):
+//   logits = bf16(x W_r^T);  dx += dlogits W_r;  partial dW_r of each K split (fp32 slabs of
+//   round_up(E, 128) rows), summed by launch_router_wgrad_reduce;  dlogits from the routing
+//   weights' gradient.
+constexpr int kRouterMaxSplits = 16;
+cudaError_t launch_router_gemm(int T, int h, int E, const void *x, const void *wr, void *logits,
+                               int32_t *status, cudaStream_t st);
+cudaError_t launch_router_dx_gemm(int T, int h, int E, const void *dlogits, const void *wr, void *dx,
+                                  int32_t *status, cudaStream_t st);
+int router_wgrad_splits(int T, int h, int E);
+cudaError_t launch_router_wgrad_gemm(int T, int h, int E, const void *dlogits, const void *x,
+                                     float *partials, int splits, int32_t *status,
+                                     cudaStream_t st);
+cudaError_t launch_router_wgrad_reduce(int h, int E, int splits, const float *partials,
+                                       float *dw_router, cudaStream_t st);
+cudaError_t launch_router_dlogits(int T, int E, int k, const uint16_t *logits,
+                                  const int32_t *top, const float *dweights, uint16_t *dlogits,
+                                  cudaStream_t st);
+
 int device_sm_count();
 
 // Test-only: make the next grouped-GEMM launch stall on purpose (see dmoe_debug_inject_stall).

@@ -4,13 +4,16 @@ This module holds only the shapes and the seeded random inputs; it contains none
 layer's arithmetic, so both the CUDA path and the CPU oracle can take their inputs from it.
 
 Recipe: workload seed s = 1000 + workload number; every tensor has its own torch CPU
-generator seeded with 100*s + i (i = 0 x, 1 W1, 2 W3, 3 W2, 4 logits, 5 dy), so any tensor
-can be regenerated alone; each is drawn in fp32 and rounded to bf16 (round-to-nearest-even):
+generator seeded with 100*s + i (i = 0 x, 1 W1, 2 W3, 3 W2, 4 logits, 5 dy, 6 W_r), so any
+tensor can be regenerated alone; each is drawn in fp32 and rounded to bf16
+(round-to-nearest-even):
   x ~ N(0, 1)                         [T, hidden]
   W1, W3 ~ 0.02 * N(0, 1)             [E, ffn, hidden]   (out, in) layout; W1 = gate
   W2 ~ 0.02 * N(0, 1)                 [E, hidden, ffn]
   logits ~ N(0, 1) (+ bias_e)         [T, E]
   dy ~ N(0, 1)                        [T, hidden]        (backward workloads only)
+  W_r ~ N(0, 1) / sqrt(hidden)        [E, hidden]        (router weight, router runs only:
+                                                          x W_r^T then has N(0, 1) logits)
 The skewed workload adds bias_e = -1.5 * ln(e + 1) (Zipf-like skew toward low expert ids) to
 the logits in fp32 before the bf16 rounding.  Std 0.02 matches the issue's
 ``init_method_std: 0.02``.
@@ -71,7 +74,7 @@ def zipf_bias(E: int) -> torch.Tensor:
     return torch.tensor([-1.5 * math.log(e + 1) for e in range(E)], dtype=torch.float32)
 
 
-TENSORS = ("x", "w1", "w3", "w2", "logits", "dy")
+TENSORS = ("x", "w1", "w3", "w2", "logits", "dy", "w_router")
 
 
 def make_tensor(w: Workload, name: str, seed: int | None = None) -> torch.Tensor:
@@ -85,6 +88,7 @@ def make_tensor(w: Workload, name: str, seed: int | None = None) -> torch.Tensor
         "w2": ((w.E, w.hidden, w.ffn), 0.02),
         "logits": ((w.T, w.E), 1.0),
         "dy": ((w.T, w.hidden), 1.0),
+        "w_router": ((w.E, w.hidden), 1.0 / math.sqrt(w.hidden)),
     }[name]
     t = torch.randn(shape, generator=g, dtype=torch.float32)
     if scale != 1.0:
@@ -94,9 +98,13 @@ def make_tensor(w: Workload, name: str, seed: int | None = None) -> torch.Tensor
     return t.to(torch.bfloat16)
 
 
-def make_inputs(w: Workload, seed: int | None = None, with_dy: bool | None = None) -> dict:
-    """CPU bf16 tensors x, w1, w3, w2, logits (and dy) for workload ``w``."""
+def make_inputs(w: Workload, seed: int | None = None, with_dy: bool | None = None,
+                with_router: bool = False) -> dict:
+    """CPU bf16 tensors x, w1, w3, w2, logits (and dy, and the router weight w_router) for
+    workload ``w``."""
     names = list(TENSORS[:5])
     if w.backward if with_dy is None else with_dy:
         names.append("dy")
+    if with_router:
+        names.append("w_router")
     return {n: make_tensor(w, n, seed) for n in names}

@@ -125,6 +125,7 @@ typedef struct {
 #define DMOE_WS_FORWARD 1        /* dmoe_forward with saved == NULL (inference) */
 #define DMOE_WS_BACKWARD 2       /* dmoe_backward */
 #define DMOE_WS_FORWARD_TRAIN 3  /* dmoe_forward with saved != NULL (training) */
+#define DMOE_WS_ROUTER_BACKWARD 4 /* dmoe_router_backward */
 
 /* Column tile of the dH GEMM: the routing-weight partial sums of dmoe_bwd_dglu have
  * ceil(ffn / DMOE_DGLU_TILE_COLS) columns. */
@@ -293,6 +294,41 @@ DMOE_API int dmoe_bwd_wgrad(const dmoe_dims *dims, const void *x_pad, const void
  * dx_pad [P_max,h] bf16, dw_part from dmoe_bwd_dglu -> dx [T,h] bf16, dweights [T,k] fp32. */
 DMOE_API int dmoe_bwd_scatter(const dmoe_dims *dims, const void *dx_pad, const float *dw_part,
                               const dmoe_map *map, void *dx, float *dweights, void *stream);
+
+/* ---- The linear router (the steps on either side of the routing). ----
+ * The pages fix only the router's output, (scores, top_experts) (issue #56 error log;
+ * "router(x)" in the walkthrough's schematic forward, section 4.5).  These calls implement
+ * the plainest reading: a linear router without bias, logits = x W_r^T with W_r [E, h] bf16
+ * in the (out, in) layout, whose bf16 logits feed dmoe_sparse_map.  They require
+ * num_experts % 8 == 0 (DMOE_ERR_SHAPE otherwise: the [T, E] rows must be multiples of 16
+ * bytes). */
+
+/* logits [T, E] = bf16(x W_r^T), fp32 accumulation on the tensor cores.  x [T, h] bf16.
+ * status: the int32 device status word that a bounded wait that gives up marks with
+ * DMOE_STATUS_TIMEOUT (e.g. map->status). */
+DMOE_API int dmoe_router_forward(const dmoe_dims *dims, const void *x, const void *w_router,
+                                 void *logits, int32_t *status, void *stream);
+
+/* Gradient of the routing weights with respect to the logits: with p_t = softmax(logits_t)
+ * over all E (fp32) and j_s = map->top_experts[t][s],
+ *   dlogits[t][i] = sum_s dweights[t][s] * p_t[j_s] * ([i == j_s] - p_t[i])
+ * (the expert choice itself carries no gradient).  logits [T, E] bf16 (the ones routed),
+ * dweights [T, k] fp32 (from dmoe_backward) -> dlogits [T, E] bf16. */
+DMOE_API int dmoe_router_dlogits(const dmoe_dims *dims, const void *logits, const dmoe_map *map,
+                                 const float *dweights, void *dlogits, void *stream);
+
+/* Backward of the router: dlogits as in dmoe_router_dlogits, then
+ *   dx [T, h] bf16 += dlogits W_r    (in place: dx holds the expert path's input gradient from
+ *                                     dmoe_backward; the sum is formed in fp32, rounded once),
+ *   dw_router [E, h] fp32 = dlogits^T x   (overwritten; split over the tokens into fp32
+ *                                     partials that are summed in a fixed order, so the result
+ *                                     is deterministic).
+ * ws: dmoe_workspace_bytes(dims, DMOE_WS_ROUTER_BACKWARD) bytes (dlogits and the partials).
+ * map: from dmoe_sparse_map (top_experts; status receives timeout bits). */
+DMOE_API int dmoe_router_backward(const dmoe_dims *dims, const void *x, const void *w_router,
+                                  const void *logits, const dmoe_map *map, const float *dweights,
+                                  void *dx, float *dw_router, void *ws, size_t ws_bytes,
+                                  void *stream);
 
 /* ---- Diagnostics. ---- */
 DMOE_API const char *dmoe_error_string(int code);

@@ -51,7 +51,7 @@ def test_sizes():
     assert offs == sorted(offs) and offs[0] == 0 and all(o % 256 == 0 for o in offs)
     assert offs[1] >= P * 4096 * 2 and offs[2] >= offs[1] + P * 14336 * 2
     assert total >= offs[2] + P * 14336 * 2
-    assert B.dmoe_workspace_bytes(d, 4) == 0  # unknown workspace kind
+    assert B.dmoe_workspace_bytes(d, 5) == 0  # unknown workspace kind
 
 
 @pytest.mark.parametrize("dims,code", [
@@ -74,6 +74,21 @@ def test_bad_dims_rejected_before_launch(lib, dims, code):
                           0, None)
     assert rc == code
     assert B.error_string(code) != "unknown error"
+
+
+def test_router_needs_E_multiple_of_8(lib):
+    """The router's [T, E] rows must be multiples of 16 bytes: E % 8 != 0 is a shape error,
+    reported before any launch (and before the null-pointer checks)."""
+    m = B.dmoe_map()
+    for E, code in ((12, -2), (8, -1), (1025, -3)):
+        d = B.make_dims(256, 128, 128, E, 2)
+        assert lib.dmoe_router_forward(ctypes.byref(d), None, None, None, None, None) == code
+        assert lib.dmoe_router_dlogits(ctypes.byref(d), None, ctypes.byref(m), None, None, None) == code
+        assert lib.dmoe_router_backward(ctypes.byref(d), None, None, None, ctypes.byref(m), None,
+                                        None, None, None, 0, None) == code
+    d = B.make_dims(4096, 2048, 512, 256, 8)
+    # dlogits [T, E] bf16 plus 16 split slabs of round_up(E, 128) x h fp32 partials
+    assert B.dmoe_workspace_bytes(d, B.WS_ROUTER_BACKWARD) >= 4096 * 256 * 2 + 16 * 256 * 2048 * 4
 
 
 def test_null_and_workspace_checks(lib):
