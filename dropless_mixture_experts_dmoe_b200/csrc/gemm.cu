@@ -106,10 +106,10 @@ __host__ __device__ constexpr bool is_dense_rows(int mode) {
   return mode == MODE_ROUTER || mode == MODE_RDX;
 }
 
-// Per-launch configuration.  A 5-stage ring of 32 KB per CTA; 4 epilogue warps (one per TMEM
-// sub-partition, double-buffered result staging) by default, or 8 (two per sub-partition,
-// each taking half of the tile's columns, one staging buffer each) for GEMMs whose K is so
-// short (4 stages per tile) that the epilogue, not the MMA, bounds a tile.
+// Per-launch configuration.  A 5-stage ring of 32 KB per CTA and 4 epilogue warps (one per
+// TMEM sub-partition) by default, or 8 epilogue warps (two per sub-partition, each taking half
+// of the tile's columns) and a 4-stage ring for GEMMs whose K is so short (a few K steps per
+// tile) that the epilogue, not the MMA, bounds a tile.  Two 4 KB staging buffers per warp.
 template <int MODE, int EPI>
 struct Cfg {
   static constexpr int a_mn = (MODE == MODE_WGRAD || MODE == MODE_RWGRAD) ? 1 : 0;
@@ -120,8 +120,8 @@ struct Cfg {
   static constexpr int epi_warps = EPI;
   static constexpr int col_split = epi_warps / 4;  // warps per TMEM sub-partition
   static constexpr int threads = 64 + 32 * epi_warps;
-  static constexpr int stages = 5;
-  static constexpr int out_bufs = (EPI == 8) ? 1 : 2;
+  static constexpr int stages = (EPI == 8) ? 4 : 5;
+  static constexpr int out_bufs = 2;
   static constexpr int out_bytes = epi_warps * out_bufs * BOX_BYTES;
   // WGRAD: one zeroed result box, the source of the zero tiles' stores
   static constexpr int zero_bytes = (MODE == MODE_WGRAD) ? BOX_BYTES : 0;
@@ -349,6 +349,29 @@ struct Stager {
     }
     cur = (cur + 1) % OUT_BUFS;
   }
+
+  // Batched form: write box i of a batch into buffer i (put), then publish the whole batch
+  // with one proxy fence and one store per box (flush).  reclaim() first waits until the
+  // previous batch's stores have read their buffers.
+  __device__ __forceinline__ void reclaim() {
+    if (lane == 0) bulk_wait_read<0>();
+    __syncwarp();
+  }
+  __device__ __forceinline__ void put(int i, const uint32_t (&w)[32]) {
+    const uint32_t row = bufs + (uint32_t)(i * BOX_BYTES) + (uint32_t)(lane * 128);
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      st_shared_v4(row + (uint32_t)((c ^ (lane & 7)) << 4), w[4 * c], w[4 * c + 1], w[4 * c + 2],
+                   w[4 * c + 3]);
+  }
+  __device__ __forceinline__ void flush(const CUtensorMap *map, int n, int x0, int dx, int y) {
+    fence_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      for (int i = 0; i < n; ++i) tma_store_2d_u32(map, bufs + (uint32_t)(i * BOX_BYTES), x0 + i * dx, y);
+      bulk_commit();
+    }
+  }
 };
 
 __device__ __forceinline__ void pack_bf16_row(const uint32_t (&lo)[32], const uint32_t (&hi)[32],
@@ -427,6 +450,21 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
     if (ncols <= 0) return;
     tb += (uint32_t)(half * kw);
     uint32_t v0[32], v1[32], w[32];
+    if (EPI == 8 && ncols == 2 * 64) {  // both of this warp's boxes staged, one proxy fence
+      uint32_t v2[32], v3[32];
+      tmem_ld32(tb, v0);
+      tmem_ld32(tb + 32, v1);
+      tmem_ld32(tb + 64, v2);
+      tmem_ld32(tb + 96, v3);
+      st.reclaim();
+      tmem_ld_wait();
+      pack_bf16_row(v0, v1, w);
+      st.put(0, w);
+      pack_bf16_row(v2, v3, w);
+      st.put(1, w);
+      st.flush(&p.tmo[0], 2, n0, 64, y0);
+      return;
+    }
     tmem_ld32(tb, v0);
     tmem_ld32(tb + 32, v1);
     tmem_ld_wait();
@@ -587,7 +625,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
   uint64_t *full = bars;                       // [STAGES] leader: both halves landed
   uint64_t *empty = bars + STAGES;             // [STAGES] MMAs done reading the stage
   uint64_t *tfull = bars + 2 * STAGES;         // [2] accumulator ready
-  uint64_t *tempty = bars + 2 * STAGES + 2;    // [2] leader: accumulator drained (256 arrivals)
+  uint64_t *tempty = bars + 2 * STAGES + 2;    // [2] leader: accumulator drained (one arrival
+                                               //     per epilogue warp of both CTAs)
   uint64_t *drain = bars + 2 * STAGES + 4;     // leader: all MMAs finished
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -605,7 +644,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 2 * EPI_THREADS);
+      mbar_init(&tempty[a], 2 * C::epi_warps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -800,12 +839,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
       const Tile tl = decode<MODE>(p, t, ustart, rank);
       if (tl.kit == 0) continue;  // WGRAD zero tile: stored by the producer warp
       const float wr = epilogue_prologue<MODE, EPI>(p, tl, sub, half, lane);
-      if (!mbar_wait(&tfull[acc], acc_phase, p.status, abort_flag, p.wait_cycles)) break;
+      int good = 1;  // lane 0 waits for the accumulator; the warp follows its verdict
+      if (lane == 0) good = mbar_wait(&tfull[acc], acc_phase, p.status, abort_flag, p.wait_cycles) ? 1 : 0;
+      if (!__shfl_sync(0xFFFFFFFFu, good, 0)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * ACC_COLS);
       if (!tl.dummy) epilogue_tile<MODE, EPI>(p, tl, tb, sub, half, lane, wr, st);
+      // every lane's accumulator reads are complete (tcgen05.wait::ld inside the tile), ordered
+      // before the warp barrier by the fence; one arrival per warp releases the accumulator
       tc_fence_before();
-      mbar_arrive_cluster(leader_tempty0 + (uint32_t)(acc * sizeof(uint64_t)));
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_tempty0 + (uint32_t)(acc * sizeof(uint64_t)));
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
