@@ -15,8 +15,6 @@ namespace dmoe {
 constexpr int kCopyThreads = 256;
 constexpr int kCopyWarps = kCopyThreads / 32;
 constexpr int kGatherVPL = 8;   // 16-byte vectors in flight per lane (gather)
-constexpr int kCombineVPL = 2;  // 16-byte vectors per lane per slot (combine)
-constexpr int kCombineSlots = 8;
 
 __device__ __forceinline__ uint4 ld_nc_v4(const uint4 *p) {
   uint4 v;
@@ -89,6 +87,9 @@ __global__ void __launch_bounds__(kCopyThreads) k_gather(int T, int h, int k, in
 // and the routing weight's gradient is <dy_t, Y_ts>): with dweights != NULL the warp that
 // takes a token's first slice also sums the DGLU GEMM's per-column-tile partials of each entry,
 // dweights[t*k+s] = sum_{n<nt} part[dest_row[t*k+s] * nt + n], in column-tile order.
+// VPL 16-byte vectors per lane for each of SLOTS slots are loaded before any is consumed
+// (VPL * SLOTS = 16 loads in flight per lane): few slots (small top_k) take wide row pieces.
+template <int VPL, int SLOTS>
 __global__ void __launch_bounds__(kCopyThreads) k_combine(int T, int h, int k,
                                                           const uint4 *__restrict__ y_pad,
                                                           const int32_t *__restrict__ dest_row,
@@ -114,34 +115,34 @@ __global__ void __launch_bounds__(kCopyThreads) k_combine(int T, int h, int k,
         for (int n = 0; n < nt; ++n) g += __ldg(part + (size_t)d * nt + n);
       dweights[(size_t)t * k + lane] = g;  // 0 for an entry dropped from the map
     }
-    for (int v0 = vs; v0 < ve; v0 += 32 * kCombineVPL) {
-      float acc[kCombineVPL][8];
+    for (int v0 = vs; v0 < ve; v0 += 32 * VPL) {
+      float acc[VPL][8];
 #pragma unroll
-      for (int u = 0; u < kCombineVPL; ++u)
+      for (int u = 0; u < VPL; ++u)
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[u][q] = 0.0f;
-      for (int s0 = 0; s0 < k; s0 += kCombineSlots) {
-        uint4 buf[kCombineSlots][kCombineVPL];
+      for (int s0 = 0; s0 < k; s0 += SLOTS) {
+        uint4 buf[SLOTS][VPL];
 #pragma unroll
-        for (int ss = 0; ss < kCombineSlots; ++ss) {
+        for (int ss = 0; ss < SLOTS; ++ss) {
           const int s = s0 + ss;
           const int r = __shfl_sync(0xFFFFFFFFu, d, s & 31);
           if (s < k && r >= 0) {
 #pragma unroll
-            for (int u = 0; u < kCombineVPL; ++u) {
+            for (int u = 0; u < VPL; ++u) {
               const int v = v0 + u * 32 + lane;
               if (v < ve) buf[ss][u] = ld_nc_v4(y_pad + (size_t)r * vpr + v);
             }
           }
         }
 #pragma unroll
-        for (int ss = 0; ss < kCombineSlots; ++ss) {
+        for (int ss = 0; ss < SLOTS; ++ss) {
           const int s = s0 + ss;
           const int r = __shfl_sync(0xFFFFFFFFu, d, s & 31);
           const float ws = __shfl_sync(0xFFFFFFFFu, wl, s & 31);
           if (s < k && r >= 0) {
 #pragma unroll
-            for (int u = 0; u < kCombineVPL; ++u) {
+            for (int u = 0; u < VPL; ++u) {
               const uint32_t *q = reinterpret_cast<const uint32_t *>(&buf[ss][u]);
 #pragma unroll
               for (int p = 0; p < 4; ++p) {
@@ -153,7 +154,7 @@ __global__ void __launch_bounds__(kCopyThreads) k_combine(int T, int h, int k,
         }
       }
 #pragma unroll
-      for (int u = 0; u < kCombineVPL; ++u) {
+      for (int u = 0; u < VPL; ++u) {
         const int v = v0 + u * 32 + lane;
         if (v < ve) {
           uint4 o;
@@ -188,21 +189,33 @@ cudaError_t launch_gather(int T, int h, int k, int E, const void *x, const int32
   return cudaGetLastError();
 }
 
+static cudaError_t combine(int T, int h, int k, const void *y_pad, const int32_t *dest_row,
+                           const float *weights, void *y, const float *part, int nt,
+                           float *dweights, cudaStream_t st) {
+  const int grid = copy_grid((long long)T * slices(h));
+  const uint4 *src = static_cast<const uint4 *>(y_pad);
+  uint4 *dst = static_cast<uint4 *>(y);
+  if (k <= 2)
+    k_combine<8, 2><<<grid, kCopyThreads, 0, st>>>(T, h, k, src, dest_row, weights, dst, part, nt,
+                                                   dweights);
+  else if (k <= 4)
+    k_combine<4, 4><<<grid, kCopyThreads, 0, st>>>(T, h, k, src, dest_row, weights, dst, part, nt,
+                                                   dweights);
+  else
+    k_combine<2, 8><<<grid, kCopyThreads, 0, st>>>(T, h, k, src, dest_row, weights, dst, part, nt,
+                                                   dweights);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const int32_t *dest_row,
                            const float *weights, void *y, cudaStream_t st) {
-  k_combine<<<copy_grid((long long)T * slices(h)), kCopyThreads, 0, st>>>(
-      T, h, k, static_cast<const uint4 *>(y_pad), dest_row, weights, static_cast<uint4 *>(y),
-      nullptr, 0, nullptr);
-  return cudaGetLastError();
+  return combine(T, h, k, y_pad, dest_row, weights, y, nullptr, 0, nullptr, st);
 }
 
 cudaError_t launch_bwd_scatter(int T, int h, int k, const void *dx_pad, const int32_t *dest_row,
                                const float *part, int nt, void *dx, float *dweights,
                                cudaStream_t st) {
-  k_combine<<<copy_grid((long long)T * slices(h)), kCopyThreads, 0, st>>>(
-      T, h, k, static_cast<const uint4 *>(dx_pad), dest_row, nullptr, static_cast<uint4 *>(dx),
-      part, nt, dweights);
-  return cudaGetLastError();
+  return combine(T, h, k, dx_pad, dest_row, nullptr, dx, part, nt, dweights, st);
 }
 
 }  // namespace dmoe
