@@ -106,10 +106,12 @@ __host__ __device__ constexpr bool is_dense_rows(int mode) {
   return mode == MODE_ROUTER || mode == MODE_RDX;
 }
 
-// Per-launch configuration.  A 5-stage ring of 32 KB per CTA and 4 epilogue warps (one per
-// TMEM sub-partition) by default, or 8 epilogue warps (two per sub-partition, each taking half
-// of the tile's columns) and a 4-stage ring for GEMMs whose K is so short (a few K steps per
-// tile) that the epilogue, not the MMA, bounds a tile.  Two 4 KB staging buffers per warp.
+// Per-launch configuration.  4 epilogue warps (one per TMEM sub-partition) by default, or 8
+// (two per sub-partition, each taking half of the tile's columns) for GEMMs whose K is so short
+// (a few K steps per tile) that the epilogue, not the MMA, bounds a tile.  The ring of 32 KB
+// stages is as deep as shared memory allows next to the result staging: 6 stages with one
+// 4 KB staging buffer per warp for the forward GEMMs (few result boxes per tile; the deeper
+// ring hides more operand latency), else 5 (4 with 8 warps) with two.
 template <int MODE, int EPI>
 struct Cfg {
   static constexpr int a_mn = (MODE == MODE_WGRAD || MODE == MODE_RWGRAD) ? 1 : 0;
@@ -120,8 +122,9 @@ struct Cfg {
   static constexpr int epi_warps = EPI;
   static constexpr int col_split = epi_warps / 4;  // warps per TMEM sub-partition
   static constexpr int threads = 64 + 32 * epi_warps;
-  static constexpr int stages = (EPI == 8) ? 4 : 5;
-  static constexpr int out_bufs = 2;
+  static constexpr int stages =
+      (EPI == 8) ? 4 : ((MODE == MODE_GLU || MODE == MODE_DOWN) ? 6 : 5);
+  static constexpr int out_bufs = (stages == 6) ? 1 : 2;
   static constexpr int out_bytes = epi_warps * out_bufs * BOX_BYTES;
   // WGRAD: one zeroed result box, the source of the zero tiles' stores
   static constexpr int zero_bytes = (MODE == MODE_WGRAD) ? BOX_BYTES : 0;
