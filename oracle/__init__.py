@@ -61,14 +61,14 @@ def _load():
         lib = ctypes.CDLL(_LIB_PATH)
         P = ctypes.c_void_p
         I = ctypes.c_int
-        lib.oracle_route.argtypes = [I, I, I, P, P, P]
+        lib.oracle_route.argtypes = [I, I, I, I, P, P, P]
         lib.oracle_sparse_map.argtypes = [I, I, I, P, P, P, P, P, P, P, P, I, P]
         lib.oracle_forward.argtypes = [I, I, I, I, I, P, P, P, P, P, P, I, P, P, P, I]
         lib.oracle_backward.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P, P]
         lib.oracle_backward_tokens.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, P, I]
         lib.oracle_wgrad_elements.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, I]
         lib.oracle_router_logits.argtypes = [I, I, I, P, P, I, P, P, I]
-        lib.oracle_router_backward.argtypes = [I, I, I, I, P, P, P, P, P, P, I, P, P, I, P, P, I]
+        lib.oracle_router_backward.argtypes = [I, I, I, I, I, P, P, P, P, P, P, I, P, P, I, P, P, I]
         for fn in (lib.oracle_route, lib.oracle_sparse_map, lib.oracle_forward, lib.oracle_backward,
                    lib.oracle_backward_tokens, lib.oracle_wgrad_elements, lib.oracle_max_threads,
                    lib.oracle_router_logits, lib.oracle_router_backward):
@@ -103,13 +103,14 @@ def padded_rows_max(T: int, E: int, k: int) -> int:
     return ((T * k + (BLOCKING - 1) * E) // BLOCKING) * BLOCKING
 
 
-def route(logits, k: int):
-    """logits [T,E] -> (top_experts [T,k] int32, weights [T,k] float64)."""
+def route(logits, k: int, renorm: bool = False):
+    """logits [T,E] -> (top_experts [T,k] int32, weights [T,k] float64); renorm: weights are
+    the softmax over the k chosen logits (they sum to 1)."""
     lg = _f32(logits)
     T, E = lg.shape
     top = np.empty((T, k), np.int32)
     w = np.empty((T, k), np.float64)
-    rc = _load().oracle_route(T, E, k, _p(lg), _p(top), _p(w))
+    rc = _load().oracle_route(T, E, k, int(bool(renorm)), _p(lg), _p(top), _p(w))
     if rc != 0:
         raise ValueError(f"oracle_route failed ({rc})")
     return top, w
@@ -225,7 +226,7 @@ def router_logits(x, Wr, tokens=None, threads=1):
 
 
 def router_backward(x, Wr, logits, top_experts, dweights, tokens=None, elems=None,
-                    want_dx=True, want_dwr=True, threads=1):
+                    want_dx=True, want_dwr=True, threads=1, renorm=False):
     """Gradient through the routing weights.  Returns dict dlogits [T,E], dx_r ([n,h] for
     ``tokens`` or [T,h]) and dWr ([len(elems)] for ``elems`` = [(e, c), ...] or [E,h]),
     all float64."""
@@ -242,7 +243,7 @@ def router_backward(x, Wr, logits, top_experts, dweights, tokens=None, elems=Non
     n_el = E * h if el is None else el.shape[0]
     dwr = np.empty(n_el, np.float64) if want_dwr else None
     rc = _load().oracle_router_backward(
-        T, h, E, k, _p(x), _p(Wr), _p(lg), _p(top), _p(dw), _p(dl), n_tok,
+        T, h, E, k, int(bool(renorm)), _p(x), _p(Wr), _p(lg), _p(top), _p(dw), _p(dl), n_tok,
         None if toks is None else _p(toks), None if dx is None else _p(dx),
         n_el, None if el is None else _p(el), None if dwr is None else _p(dwr), int(threads))
     if rc != 0:

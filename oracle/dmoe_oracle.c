@@ -47,9 +47,12 @@ static int preferred(double a, double b) {
  * For each token: pick k experts by repeatedly taking the preferred remaining logit; slot s
  * holds the s-th pick.  The weight of slot s is the softmax over all E logits read at the
  * chosen expert: w = exp(l_e - m) / sum_j exp(l_j - m), m = max logit.  No renormalisation
- * over the k chosen experts.
+ * over the k chosen experts -- unless renorm != 0, the routing variant in which the weights are
+ * the softmax over the k chosen logits only: w = exp(l_e - m) / sum_{chosen j} exp(l_j - m),
+ * so that they sum to 1.
  * logits: [T, E] (fp32 widened from bf16); top: [T, k] int32 out; w: [T, k] double out. */
-int oracle_route(int T, int E, int k, const float *logits, int32_t *top, double *w) {
+int oracle_route(int T, int E, int k, int renorm, const float *logits, int32_t *top,
+                 double *w) {
   if (T < 0 || E < 1 || k < 1 || k > E) return -1;
   unsigned char *chosen = (unsigned char *)malloc((size_t)E);
   if (!chosen) return -2;
@@ -69,7 +72,10 @@ int oracle_route(int T, int E, int k, const float *logits, int32_t *top, double 
     for (int e = 0; e < E; ++e)
       if (!isnan(l[e]) && (double)l[e] > m) m = l[e];
     double denom = 0.0;
-    for (int e = 0; e < E; ++e) denom += exp((double)l[e] - m);
+    if (renorm)
+      for (int s = 0; s < k; ++s) denom += exp((double)l[top[(size_t)t * k + s]] - m);
+    else
+      for (int e = 0; e < E; ++e) denom += exp((double)l[e] - m);
     for (int s = 0; s < k; ++s) {
       int e = top[(size_t)t * k + s];
       w[(size_t)t * k + s] = exp((double)l[e] - m) / denom;
@@ -427,9 +433,10 @@ int oracle_router_logits(int T, int h, int E, const float *x, const float *Wr, i
   return 0;
 }
 
-/* Gradient through the routing weights of oracle_route (softmax over all E logits read at the
- * k chosen experts, no renormalisation); the choice of experts is piecewise constant, so it
- * carries no gradient.  With p_t = softmax(logits_t) and j_s = top[t][s]:
+/* Gradient through the routing weights of oracle_route; the choice of experts is piecewise
+ * constant, so it carries no gradient.  With j_s = top[t][s] and p_t the softmax of logits_t
+ * over all E experts (renorm == 0), or over the k chosen experts only, zero elsewhere
+ * (renorm != 0):
  *   w_ts = p_t[j_s],   d w_ts / d l_ti = p_t[j_s] * ([i == j_s] - p_t[i]),
  *   dlogits[t][i] = sum_s dw[t][s] * d w_ts / d l_ti                       (chain rule),
  * and, through logits = x Wr^T,
@@ -439,8 +446,9 @@ int oracle_router_logits(int T, int h, int E, const float *x, const float *Wr, i
  * dx_r: [n_tok, h] for tokens (NULL = all T, n_tok = T); skipped when dx_r is NULL.
  * dWr: one value per (e, c) pair of `elems` ([n_el, 2] int32), or the full [E, h] when elems
  *      is NULL; skipped when dWr is NULL. */
-int oracle_router_backward(int T, int h, int E, int k, const float *x, const float *Wr,
-                           const float *logits, const int32_t *top, const double *dw,
+int oracle_router_backward(int T, int h, int E, int k, int renorm, const float *x,
+                           const float *Wr, const float *logits, const int32_t *top,
+                           const double *dw,
                            double *dlogits, int n_tok, const int32_t *tokens, double *dx_r,
                            int n_el, const int32_t *elems, double *dWr, int threads) {
   if (T < 0 || h < 1 || E < 1 || k < 1 || k > E) return -1;
@@ -453,8 +461,14 @@ int oracle_router_backward(int T, int h, int E, int k, const float *x, const flo
     for (int e = 0; e < E; ++e)
       if ((double)l[e] > m) m = (double)l[e];
     double z = 0.0;
-    for (int e = 0; e < E; ++e) z += exp((double)l[e] - m);
-    for (int e = 0; e < E; ++e) prob[e] = exp((double)l[e] - m) / z;
+    for (int e = 0; e < E; ++e) prob[e] = renorm ? 0.0 : exp((double)l[e] - m);
+    if (renorm)
+      for (int s = 0; s < k; ++s) {
+        const int j = top[(size_t)t * k + s];
+        if (j >= 0 && j < E) prob[j] = exp((double)l[j] - m);
+      }
+    for (int e = 0; e < E; ++e) z += prob[e];
+    for (int e = 0; e < E; ++e) prob[e] /= z;
     for (int i = 0; i < E; ++i) {
       double g = 0.0;
       for (int s = 0; s < k; ++s) {

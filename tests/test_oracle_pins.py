@@ -17,6 +17,10 @@ Router   -- logits: one-hot tokens read a column of the router weight (closed fo
             differences of sum dw * softmax(x Wr^T)[picks] in the logits, x and Wr; torch
             float64 autograd of the same composition; shift invariance (each token's logit
             gradient sums to zero); k = E with equal dw gives zero; sampled = full.
+Renormalised routing (variant flag) -- weights sum to 1, their ratios are exp(l_i - l_j),
+            k = 1 gives 1 and k = E gives the plain softmax; torch float64 softmax over the
+            chosen logits; its logit gradient by finite differences and autograd, zero outside
+            the chosen experts.
 """
 import itertools
 import json
@@ -463,4 +467,63 @@ def test_router_backward_autograd_and_invariants(oracle_mod):
     s = oracle_mod.router_backward(x, Wr, lg, top, dw, tokens=toks, elems=el)
     assert (s["dx_r"] == g["dx_r"][toks]).all()
     assert (s["dWr"] == g["dWr"][el[:, 0], el[:, 1]]).all()
+
+
+# ----------------------------------------------------------------------------------------
+# renormalised routing (the weights are the softmax over the k chosen logits)
+# ----------------------------------------------------------------------------------------
+
+def test_route_renorm_closed_forms(oracle_mod):
+    rng = np.random.default_rng(83)
+    T, E = 40, 12
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    for k in (1, 3, E):
+        top, w = oracle_mod.route(lg, k, renorm=True)
+        top0, w0 = oracle_mod.route(lg, k)
+        assert (top == top0).all()  # the choice does not depend on the weights
+        np.testing.assert_allclose(w.sum(1), 1.0, rtol=0, atol=1e-15)
+        sel = np.take_along_axis(lg.astype(np.float64), top.astype(np.int64), 1)
+        np.testing.assert_allclose(w[:, :1] / w, np.exp(sel[:, :1] - sel), rtol=1e-13)
+        if k == 1:
+            assert (w == 1.0).all()
+        if k == E:
+            np.testing.assert_allclose(w, w0, rtol=1e-14, atol=1e-16)
+        ref = torch.softmax(torch.from_numpy(sel), dim=1).numpy()  # library softmax
+        np.testing.assert_allclose(w, ref, rtol=1e-13, atol=1e-16)
+
+
+def test_router_backward_renorm_finite_differences_and_autograd(oracle_mod):
+    rng = np.random.default_rng(89)
+    T, h, E, k = 5, 24, 9, 3
+    x = rng.standard_normal((T, h)).astype(np.float32)
+    Wr = (0.3 * rng.standard_normal((E, h))).astype(np.float32)
+    lg = (x.astype(np.float64) @ Wr.astype(np.float64).T).astype(np.float32)
+    top, _ = oracle_mod.route(lg, k, renorm=True)
+    dw = rng.standard_normal((T, k))
+    g = oracle_mod.router_backward(x, Wr, lg, top, dw, renorm=True)
+
+    def loss(l64):
+        sel = np.take_along_axis(l64, top.astype(np.int64), 1)
+        z = np.exp(sel - sel.max(1, keepdims=True))
+        return float((dw * z / z.sum(1, keepdims=True)).sum())
+
+    l64 = lg.astype(np.float64)
+    eps = 1e-6
+    for t in range(T):
+        for i in range(E):
+            lp, lm = l64.copy(), l64.copy()
+            lp[t, i] += eps
+            lm[t, i] -= eps
+            fd = (loss(lp) - loss(lm)) / (2 * eps)
+            assert abs(fd - g["dlogits"][t, i]) <= 1e-8 + 1e-6 * abs(fd), (t, i)
+    chosen = np.zeros((T, E), bool)
+    np.put_along_axis(chosen, top.astype(np.int64), True, 1)
+    assert (g["dlogits"][~chosen] == 0).all()
+    assert np.abs(g["dlogits"].sum(1)).max() <= 1e-14
+    l = torch.tensor(lg, dtype=torch.float64, requires_grad=True)
+    sel = l.gather(1, torch.from_numpy(top).long())
+    (torch.tensor(dw) * torch.softmax(sel, dim=1)).sum().backward()
+    np.testing.assert_allclose(g["dlogits"], l.grad.numpy(), rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(g["dx_r"], l.grad.numpy() @ Wr.astype(np.float64), rtol=1e-12,
+                               atol=1e-14)
 
