@@ -19,7 +19,7 @@ inline unsigned int *map_ticket(int32_t *tile_hist, int T, int E) {
 }
 
 // Map: routing + per-tile histogram (logits given) or histogram of given top_experts.
-cudaError_t launch_route_hist(const uint16_t *logits, int T, int E, int k, int32_t *top,
+cudaError_t launch_route_hist(const uint16_t *logits, int T, int E, int k, bool renorm, int32_t *top,
                               float *weights, int32_t *tile_hist, int32_t *status,
                               cudaStream_t st);
 // Map: scan over tiles and experts, bins / padded_bins / block table.
@@ -94,7 +94,7 @@ cudaError_t launch_router_wgrad_gemm(int T, int h, int E, const void *dlogits, c
                                      cudaStream_t st);
 cudaError_t launch_router_wgrad_reduce(int h, int E, int splits, const float *partials,
                                        float *dw_router, cudaStream_t st);
-cudaError_t launch_router_dlogits(int T, int E, int k, const uint16_t *logits,
+cudaError_t launch_router_dlogits(int T, int E, int k, bool renorm, const uint16_t *logits,
                                   const int32_t *top, const float *dweights, uint16_t *dlogits,
                                   cudaStream_t st);
 

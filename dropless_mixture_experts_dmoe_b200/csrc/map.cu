@@ -27,7 +27,7 @@ __device__ __forceinline__ bool bf16_nonfinite(uint16_t b) { return (b & 0x7F80u
 // KPL = logits per lane (E <= 32*KPL).
 template <int KPL>
 __global__ void __launch_bounds__(kMapThreads) k_route_hist(const uint16_t *__restrict__ logits,
-                                                            int T, int E, int k,
+                                                            int T, int E, int k, int renorm,
                                                             int32_t *__restrict__ top,
                                                             float *__restrict__ weights,
                                                             int32_t *__restrict__ tile_hist,
@@ -92,18 +92,23 @@ __global__ void __launch_bounds__(kMapThreads) k_route_hist(const uint16_t *__re
         my_key = wb;
       }
     }
-    // softmax over all E logits, max = the first pick.
+    // softmax over all E logits (or, renormalised, over the k picks), max = the first pick.
     const float m = ((top_key >> 16) == 0u) ? __uint_as_float(0x7FC00000u)
                                            : bf16_from_order(top_key >> 16);
+    const float v = (lane < k) ? (((my_key >> 16) == 0u) ? __uint_as_float(0x7FC00000u)
+                                                         : bf16_from_order(my_key >> 16))
+                               : 0.0f;
     float sum = 0.0f;
+    if (renorm) {
+      if (lane < k) sum = expf(v - m);
+    } else {
 #pragma unroll
-    for (int i = 0; i < KPL; ++i)
-      if (lane + 32 * i < E) sum += expf(val[i] - m);
+      for (int i = 0; i < KPL; ++i)
+        if (lane + 32 * i < E) sum += expf(val[i] - m);
+    }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
     if (lane < k) {
-      const float v = ((my_key >> 16) == 0u) ? __uint_as_float(0x7FC00000u)
-                                             : bf16_from_order(my_key >> 16);
       top[(size_t)t * k + lane] = my_e;
       weights[(size_t)t * k + lane] = expf(v - m) / sum;
       atomicAdd(&hist[my_e], 1);
@@ -346,7 +351,7 @@ __global__ void __launch_bounds__(kMapThreads) k_map_scatter(int T, int E, int k
 
 // ---- launchers -------------------------------------------------------------------------------
 
-cudaError_t launch_route_hist(const uint16_t *logits, int T, int E, int k, int32_t *top,
+cudaError_t launch_route_hist(const uint16_t *logits, int T, int E, int k, bool renorm, int32_t *top,
                               float *weights, int32_t *tile_hist, int32_t *status,
                               cudaStream_t st) {
   const int tiles = map_tiles(T);
@@ -357,7 +362,8 @@ cudaError_t launch_route_hist(const uint16_t *logits, int T, int E, int k, int32
     return cudaGetLastError();
   }
 #define DMOE_ROUTE(KPL)                                                                      \
-  k_route_hist<KPL><<<tiles, kMapThreads, smem, st>>>(logits, T, E, k, top, weights, tile_hist, \
+  k_route_hist<KPL><<<tiles, kMapThreads, smem, st>>>(logits, T, E, k, renorm ? 1 : 0, top,    \
+                                                      weights, tile_hist,                      \
                                                       status, done)
   if (E <= 32)
     DMOE_ROUTE(1);

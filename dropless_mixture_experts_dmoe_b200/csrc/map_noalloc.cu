@@ -85,7 +85,8 @@ extern "C" int dmoe_sparse_map_noalloc(const dmoe_dims *dims, const void *logits
   // zeroes the counter after them, so nothing left over from an earlier call is ever read;
   // the status word is cleared here.
   if (cudaMemsetAsync(map->status, 0, sizeof(int32_t), st) != cudaSuccess) return DMOE_ERR_LAUNCH;
-  if ((rc = rc_of(dmoe::launch_route_hist(static_cast<const uint16_t *>(logits), T, E, k,
+  const bool renorm = (dims->route_flags & DMOE_ROUTE_RENORMALIZE) != 0;
+  if ((rc = rc_of(dmoe::launch_route_hist(static_cast<const uint16_t *>(logits), T, E, k, renorm,
                                           map->top_experts, map->weights, scratch, map->status,
                                           st))))
     return rc;

@@ -6,6 +6,8 @@
 // renormalisation.  Its gradient flows back through that softmax:
 //   dlogits[t][i] = sum_s dw_ts * p_t[j_s] * ([i == j_s] - p_t[i]) = p_t[i] * (g_ti - c_t),
 //   g_ti = dw_ts if expert i is the pick of slot s (else 0),  c_t = sum_s dw_ts * p_t[j_s].
+// With the renormalised routing variant p_t is the softmax over the k chosen logits (zero at
+// the other experts), and the same formula applies.
 // The router GEMMs themselves (logits, dx += dlogits W_r, dW_r = dlogits^T x) are modes of the
 // grouped tcgen05 kernel in gemm.cu; dW_r is split over the token dimension there, and the
 // fp32 partials are summed here in split order, so the result is deterministic.
@@ -22,7 +24,7 @@ constexpr int kRouterWarps = kRouterThreads / 32;
 // the next token's row is loaded while the current one is processed.
 template <int GPL>
 __global__ void __launch_bounds__(kRouterThreads)
-    k_router_dlogits(int T, int E, int k, const uint16_t *__restrict__ logits,
+    k_router_dlogits(int T, int E, int k, int renorm, const uint16_t *__restrict__ logits,
                      const int32_t *__restrict__ top, const float *__restrict__ dweights,
                      uint16_t *__restrict__ dlogits) {
   const int lane = threadIdx.x & 31;
@@ -47,6 +49,27 @@ __global__ void __launch_bounds__(kRouterThreads)
       nxt[i] = (tn < T && lane + 32 * i < groups)
                    ? __ldg(reinterpret_cast<const uint4 *>(logits + (size_t)tn * E) + lane + 32 * i)
                    : make_uint4(0u, 0u, 0u, 0u);
+    float g[GPL][8];   // dweights scattered to the chosen experts
+    bool sel[GPL][8];  // chosen experts
+#pragma unroll
+    for (int i = 0; i < GPL; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        g[i][j] = 0.0f;
+        sel[i][j] = false;
+      }
+    for (int s = 0; s < k; ++s) {
+      const int e = __shfl_sync(0xFFFFFFFFu, jl, s);
+      const float d = __shfl_sync(0xFFFFFFFFu, dl, s);
+#pragma unroll
+      for (int i = 0; i < GPL; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const bool hit = (e == 8 * (lane + 32 * i) + j);
+          g[i][j] += hit ? d : 0.0f;
+          sel[i][j] |= hit;
+        }
+    }
     float p[GPL][8];
     float m = -INFINITY;
 #pragma unroll
@@ -67,28 +90,17 @@ __global__ void __launch_bounds__(kRouterThreads)
     for (int i = 0; i < GPL; ++i)
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        p[i][j] = (lane + 32 * i < groups) ? __expf(p[i][j] - m) : 0.0f;
+        const bool in = (lane + 32 * i < groups) && (!renorm || sel[i][j]);
+        p[i][j] = in ? __expf(p[i][j] - m) : 0.0f;
         z += p[i][j];
       }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xFFFFFFFFu, z, off);
     const float rz = 1.0f / z;
-    float g[GPL][8];
 #pragma unroll
     for (int i = 0; i < GPL; ++i)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        p[i][j] *= rz;
-        g[i][j] = 0.0f;
-      }
-    for (int s = 0; s < k; ++s) {  // g = dweights scattered to the picked experts
-      const int e = __shfl_sync(0xFFFFFFFFu, jl, s);
-      const float d = __shfl_sync(0xFFFFFFFFu, dl, s);
-#pragma unroll
-      for (int i = 0; i < GPL; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) g[i][j] += (e == 8 * (lane + 32 * i) + j) ? d : 0.0f;
-    }
+      for (int j = 0; j < 8; ++j) p[i][j] *= rz;
     float c = 0.0f;  // sum_s dw_ts p_t[j_s]
 #pragma unroll
     for (int i = 0; i < GPL; ++i)
@@ -141,12 +153,13 @@ static int grid_for(long long items, long long per_cta) {
   return (int)(g < 1 ? 1 : g);
 }
 
-cudaError_t launch_router_dlogits(int T, int E, int k, const uint16_t *logits,
+cudaError_t launch_router_dlogits(int T, int E, int k, bool renorm, const uint16_t *logits,
                                   const int32_t *top, const float *dweights, uint16_t *dlogits,
                                   cudaStream_t st) {
   const int grid = grid_for(T, kRouterWarps);
 #define DMOE_DLOGITS(GPL) \
-  k_router_dlogits<GPL><<<grid, kRouterThreads, 0, st>>>(T, E, k, logits, top, dweights, dlogits)
+  k_router_dlogits<GPL><<<grid, kRouterThreads, 0, st>>>(T, E, k, renorm ? 1 : 0, logits, top, \
+                                                         dweights, dlogits)
   if (E <= 256)
     DMOE_DLOGITS(1);
   else if (E <= 512)

@@ -83,10 +83,18 @@ extern "C" {
 #define DMOE_STATUS_DUPLICATE_EXPERT 0x4   /* caller-given top_experts repeat within a token */
 #define DMOE_STATUS_TIMEOUT 0x8            /* a bounded in-kernel wait gave up */
 
-/* Problem shape.  T tokens, hidden size h, ffn size f (per expert), E experts, top_k. */
+/* Problem shape.  T tokens, hidden size h, ffn size f (per expert), E experts, top_k, and
+ * the routing variant: route_flags = 0 (the default: weights are the softmax over all E
+ * logits at the chosen experts) or DMOE_ROUTE_RENORMALIZE.  Other bits are rejected. */
 typedef struct {
   int32_t T, hidden, ffn, num_experts, top_k;
+  int32_t route_flags;
 } dmoe_dims;
+
+/* Routing variant: the k weights of a token are the softmax over its k chosen logits only,
+ * so they sum to 1 (the top-k renormalisation some MoE layers use; the pages' default does
+ * not renormalise).  Read by dmoe_sparse_map (weights) and the router backward (dlogits). */
+#define DMOE_ROUTE_RENORMALIZE 0x1
 
 /* The sparse map.  All device pointers, caller-owned; N = T*top_k entries,
  * P_max = dmoe_padded_rows_max(dims).  Meaning (walkthrough sections 4.1-4.3):
@@ -94,7 +102,8 @@ typedef struct {
  *                              logit order, ties to the lower expert index.  Output of
  *                              dmoe_sparse_map when logits are given, else its INPUT.
  *   weights     [T, k] fp32    softmax over all E logits at the chosen expert (no
- *                              renormalisation over the k picks).  Output when logits are
+ *                              renormalisation over the k picks; with DMOE_ROUTE_RENORMALIZE,
+ *                              the softmax over the k chosen logits).  Output when logits are
  *                              given; otherwise caller-provided and only read by forward.
  *   tokens_per_expert [E]      histogram of top_experts
  *   bins [E]                   inclusive cumsum of tokens_per_expert
@@ -310,7 +319,8 @@ DMOE_API int dmoe_router_forward(const dmoe_dims *dims, const void *x, const voi
                                  void *logits, int32_t *status, void *stream);
 
 /* Gradient of the routing weights with respect to the logits: with p_t = softmax(logits_t)
- * over all E (fp32) and j_s = map->top_experts[t][s],
+ * over all E (fp32; with DMOE_ROUTE_RENORMALIZE over the k chosen experts, zero elsewhere)
+ * and j_s = map->top_experts[t][s],
  *   dlogits[t][i] = sum_s dweights[t][s] * p_t[j_s] * ([i == j_s] - p_t[i])
  * (the expert choice itself carries no gradient).  logits [T, E] bf16 (the ones routed),
  * dweights [T, k] fp32 (from dmoe_backward) -> dlogits [T, E] bf16. */

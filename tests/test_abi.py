@@ -76,6 +76,15 @@ def test_bad_dims_rejected_before_launch(lib, dims, code):
     assert B.error_string(code) != "unknown error"
 
 
+def test_unknown_route_flag_rejected(lib):
+    m = B.dmoe_map()
+    d = B.make_dims(256, 128, 128, 8, 2, route_flags=0x2)
+    assert B.dmoe_padded_rows_max(d) == 0
+    assert lib.dmoe_sparse_map(ctypes.byref(d), None, ctypes.byref(m), None, 0, None) == -2
+    d = B.make_dims(256, 128, 128, 8, 2, route_flags=B.ROUTE_RENORMALIZE)
+    assert B.dmoe_padded_rows_max(d) > 0  # the one defined flag is accepted
+
+
 def test_router_needs_E_multiple_of_8(lib):
     """The router's [T, E] rows must be multiples of 16 bytes: E % 8 != 0 is a shape error,
     reported before any launch (and before the null-pointer checks)."""

@@ -66,6 +66,22 @@ def test_map_parity_edge_cases(T, E, k, kind):
     np.testing.assert_allclose(gm["weights"], wts, rtol=WEIGHT_RTOL, atol=0)
 
 
+@pytest.mark.parametrize("T,E,k", [(4096, 64, 8), (1000, 8, 2), (300, 16, 16), (777, 1024, 1),
+                                   (2000, 256, 32)])
+def test_map_renormalised_weights(T, E, k):
+    """Routing variant DMOE_ROUTE_RENORMALIZE: the same choice, weights = softmax over the k
+    chosen logits (summing to 1), against the oracle's renormalised mode."""
+    g = torch.Generator().manual_seed(T + 31 * E + k)
+    logits = torch.randn((T, E), generator=g).to(torch.bfloat16)
+    dims = B.make_dims(T, 128, 128, E, k, route_flags=B.ROUTE_RENORMALIZE)
+    _, gm = gpu_map(dims, logits)
+    top, wts = oracle.route(logits.float().numpy(), k, renorm=True)
+    compare_map(gm, oracle.sparse_map(top, E), top_expected=top)
+    np.testing.assert_allclose(gm["weights"], wts, rtol=WEIGHT_RTOL, atol=0)
+    np.testing.assert_allclose(gm["weights"].sum(1), 1.0, rtol=0, atol=k * 2e-7)
+    assert gm["status"] == 0
+
+
 def test_map_skew_and_empty_experts_given_top():
     """Caller-given top_experts: one expert takes every token, most experts are empty."""
     T, E, k = 5000, 256, 8

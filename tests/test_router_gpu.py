@@ -21,10 +21,10 @@ SMALL = [
 ]
 
 
-def _forward_backward(w):
+def _forward_backward(w, route_flags=0):
     """Router forward, map, expert forward + backward, router backward, all on the GPU."""
     inp = make_inputs(w, with_dy=True, with_router=True)
-    dims = dims_of(w)
+    dims = B.make_dims(w.T, w.hidden, w.ffn, w.E, w.top_k, route_flags=route_flags)
     dev = {k: v.cuda() for k, v in inp.items()}
     bufs = B.Buffers(dims, train=True)
     bf = dict(dtype=torch.bfloat16, device="cuda")
@@ -70,32 +70,37 @@ def test_router_logits_parity(w):
     assert (np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-4 * rms).all()
 
 
+@pytest.mark.parametrize("renorm", [False, True], ids=["softmax", "renormalised"])
 @pytest.mark.parametrize("w", SMALL, ids=lambda w: w.describe())
-def test_router_backward_full_chain_parity(w):
-    """x -> router -> map -> experts -> loss, backward into x, W_r (and the experts)."""
-    inp, dims, dev, bufs, logits, g, dx_experts, dwr, _ = _forward_backward(w)
+def test_router_backward_full_chain_parity(w, renorm):
+    """x -> router -> map -> experts -> loss, backward into x, W_r (and the experts); both
+    routing variants."""
+    flags = B.ROUTE_RENORMALIZE if renorm else 0
+    inp, dims, dev, bufs, logits, g, dx_experts, dwr, _ = _forward_backward(w, flags)
     o = {k: v.float().numpy() for k, v in inp.items()}
     lg = logits.float().cpu().numpy()  # the routed scores (bf16, widened exactly)
-    top, wts = oracle.route(lg, w.top_k)
+    top, wts = oracle.route(lg, w.top_k, renorm=renorm)
     assert (bufs.map.top_experts.cpu().numpy() == top).all()
     ref = oracle.backward(o["x"], o["dy"], o["w1"], o["w3"], o["w2"], top, wts)
     r = oracle.router_backward(o["x"], o["w_router"], lg, top, ref["dw"],
-                               threads=oracle.max_threads())
+                               threads=oracle.max_threads(), renorm=renorm)
     assert_close(to_np(g["dx"]), ref["dx"] + r["dx_r"], f"dx {w.describe()}",
                  max_abs_rms=MAX_ABS_RMS_STRESS)
     assert_close(to_np(dwr), r["dWr"], f"dW_r {w.describe()}", max_abs_rms=MAX_ABS_RMS_STRESS)
 
 
+@pytest.mark.parametrize("renorm", [False, True], ids=["softmax", "renormalised"])
 @pytest.mark.parametrize("w", SMALL[1:3], ids=lambda w: w.describe())
-def test_router_steps_against_oracle_on_gpu_inputs(w):
+def test_router_steps_against_oracle_on_gpu_inputs(w, renorm):
     """Each router backward step on the GPU's own inputs: dlogits from the GPU's dweights, the
     dx increment, and dW_r, each against the oracle given exactly those inputs."""
-    inp, dims, dev, bufs, logits, g, dx_experts, dwr, ws = _forward_backward(w)
+    flags = B.ROUTE_RENORMALIZE if renorm else 0
+    inp, dims, dev, bufs, logits, g, dx_experts, dwr, ws = _forward_backward(w, flags)
     lg = logits.float().cpu().numpy()
     top = bufs.map.top_experts.cpu().numpy()
     dw_gpu = g["dw"].double().cpu().numpy()
     r = oracle.router_backward(inp["x"].float().numpy(), inp["w_router"].float().numpy(), lg, top,
-                               dw_gpu)
+                               dw_gpu, renorm=renorm)
     dl = torch.empty((w.T, w.E), dtype=torch.bfloat16, device="cuda")
     B.dmoe_router_dlogits(dims, logits, bufs.map, g["dw"], dl)
     torch.cuda.synchronize()
