@@ -282,6 +282,17 @@ __device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const CUtensorM
       : "memory");
 }
 
+// 3D variant: coordinates (x, y, z) of a tensor map with three dimensions.
+__device__ __forceinline__ void tma_load_3d_pair(void *smem_dst, const CUtensorMap *map,
+                                                 uint32_t bar_cluster, int32_t x, int32_t y,
+                                                 int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar_cluster)
+      : "memory");
+}
+
 // TMA gather of 4 rows (row indices y0..y3, 64 bf16 columns from x) by either CTA of a pair,
 // completing on the pair leader's mbarrier.  The tensor map's box is one row high; the rows
 // land at 4 consecutive 128-byte smem rows (128-byte swizzle).  Out-of-range rows read zeros.

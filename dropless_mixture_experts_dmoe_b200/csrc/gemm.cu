@@ -282,19 +282,15 @@ __device__ __forceinline__ void load_stage(const GemmParams &p, const Tile &tl, 
     tma_load_2d_pair(sb, &p.tm[1], bar, kb * BK, tl.e * p.h + tl.n * BN + (int)rank * (BN / 2));
   } else if (MODE == MODE_DGLU) {
     tma_load_2d_pair(sa, &p.tm[0], bar, kb * BK, tl.row0);
-#pragma unroll
-    for (int c = 0; c < 2; ++c)
-      tma_load_2d_pair(sb + c * CHUNK_BYTES, &p.tm[1], bar, tl.n * BN + (2 * (int)rank + c) * 64,
-                       tl.e * p.h + kb * BK);
+    // MN-major B: both 64-column chunks of this CTA's half in one box of the chunked map
+    tma_load_3d_pair(sb, &p.tm[1], bar, 0, tl.e * p.h + kb * BK, (tl.n * BN) / 64 + 2 * (int)rank);
   } else if (MODE == MODE_DX) {
     const int kf = p.f / BK;
     const int pass = (kb < kf) ? 0 : 1;
     const int kk = kb - pass * kf;
     tma_load_2d_pair(sa, &p.tm[pass], bar, kk * BK, tl.row0);
-#pragma unroll
-    for (int c = 0; c < 2; ++c)
-      tma_load_2d_pair(sb + c * CHUNK_BYTES, &p.tm[2 + pass], bar,
-                       tl.n * BN + (2 * (int)rank + c) * 64, tl.e * p.f + kk * BK);
+    tma_load_3d_pair(sb, &p.tm[2 + pass], bar, 0, tl.e * p.f + kk * BK,
+                     (tl.n * BN) / 64 + 2 * (int)rank);
   } else if (MODE == MODE_ROUTER) {
     tma_load_2d_pair(sa, &p.tm[0], bar, kb * BK, tl.row0);
     tma_load_2d_pair(sb, &p.tm[1], bar, kb * BK, tl.n * BN + (int)rank * (BN / 2));
@@ -311,15 +307,12 @@ __device__ __forceinline__ void load_stage(const GemmParams &p, const Tile &tl, 
 #pragma unroll
     for (int c = 0; c < 2; ++c)
       tma_load_2d_pair(sb + c * CHUNK_BYTES, &p.tm[1], bar, tl.n * BN + (2 * (int)rank + c) * 64, y);
-  } else {  // MODE_WGRAD
+  } else {  // MODE_WGRAD: both operands MN-major, each one box of two 64-column chunks
     const int y = tl.row0 + kb * BK;
     const CUtensorMap *ta = &p.tm[tl.which];               // dA, dBm, dY_pad
-    const CUtensorMap *tb = &p.tm[tl.which == 2 ? 4 : 3];  // X_pad, X_pad, H
-#pragma unroll
-    for (int c = 0; c < 2; ++c) tma_load_2d_pair(sa + c * CHUNK_BYTES, ta, bar, tl.m * BM + c * 64, y);
-#pragma unroll
-    for (int c = 0; c < 2; ++c)
-      tma_load_2d_pair(sb + c * CHUNK_BYTES, tb, bar, tl.n * BN + (2 * (int)rank + c) * 64, y);
+    const CUtensorMap *tb = &p.tm[tl.which == 2 ? 4 : 3];  // X_pad, X_pad, Hw
+    tma_load_3d_pair(sa, ta, bar, 0, y, (tl.m * BM) / 64);
+    tma_load_3d_pair(sb, tb, bar, 0, y, (tl.n * BN) / 64 + 2 * (int)rank);
   }
 }
 
@@ -906,6 +899,24 @@ static bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t c
   return r == CUDA_SUCCESS;
 }
 
+// MN-major operand [rows, cols] bf16 (cols % 64 == 0) viewed as 3D: dim0 = 64 columns of a
+// chunk (contiguous), dim1 = rows (stride = row pitch), dim2 = 64-column chunks (stride 128 B).
+// A box of {64, box_rows, 2} lands as two consecutive [box_rows x 128 B] swizzled chunks,
+// exactly the layout of two 2D boxes of 64 columns, in one TMA instruction.
+static bool make_tmap_chunked(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols,
+                              uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc || cols % 64 != 0) return false;
+  cuuint64_t dims[3] = {64, rows, cols / 64};
+  cuuint64_t strides[2] = {cols * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int device_sm_count() {
   static int cached = 0;
   if (cached > 0) return cached;
@@ -1048,7 +1059,7 @@ cudaError_t launch_dglu_gemm(const GemmProblem &g, const void *dy_pad, const voi
   GemmParams p = base_params(g);
   const uint64_t P = (uint64_t)g.nblk_cap * BM;
   if (!make_tmap(&p.tm[0], dy_pad, P, g.h, BM) ||
-      !make_tmap(&p.tm[1], w2, (uint64_t)g.E * g.h, g.f, 64) ||
+      !make_tmap_chunked(&p.tm[1], w2, (uint64_t)g.E * g.h, g.f, 64) ||
       !make_tmap(&p.tmo[0], da_out, P, g.f, 32) || !make_tmap(&p.tmo[1], db_out, P, g.f, 32) ||
       !make_tmap(&p.tmo[2], hw_out, P, g.f, 32))
     return cudaErrorInvalidValue;
@@ -1069,7 +1080,8 @@ cudaError_t launch_dx_gemm(const GemmProblem &g, const void *da, const void *db,
   const uint64_t P = (uint64_t)g.nblk_cap * BM;
   const uint64_t EF = (uint64_t)g.E * g.f;
   if (!make_tmap(&p.tm[0], da, P, g.f, BM) || !make_tmap(&p.tm[1], db, P, g.f, BM) ||
-      !make_tmap(&p.tm[2], w1, EF, g.h, 64) || !make_tmap(&p.tm[3], w3, EF, g.h, 64) ||
+      !make_tmap_chunked(&p.tm[2], w1, EF, g.h, 64) ||
+      !make_tmap_chunked(&p.tm[3], w3, EF, g.h, 64) ||
       !make_tmap(&p.tmo[0], dx_pad, P, g.h, 32))
     return cudaErrorInvalidValue;
   p.tm[4] = p.tm[0];
@@ -1085,9 +1097,11 @@ cudaError_t launch_wgrad_gemm(const GemmProblem &g, const void *x_pad, const voi
   GemmParams p = base_params(g);
   const uint64_t P = (uint64_t)g.nblk_cap * BM;
   const uint64_t EF = (uint64_t)g.E * g.f, EH = (uint64_t)g.E * g.h;
-  if (!make_tmap(&p.tm[0], da, P, g.f, 64) || !make_tmap(&p.tm[1], db, P, g.f, 64) ||
-      !make_tmap(&p.tm[2], dy_pad, P, g.h, 64) || !make_tmap(&p.tm[3], x_pad, P, g.h, 64) ||
-      !make_tmap(&p.tm[4], h_in, P, g.f, 64) || !make_tmap(&p.tmo[0], dw1, EF, g.h, 32, 4) ||
+  if (!make_tmap_chunked(&p.tm[0], da, P, g.f, 64) ||
+      !make_tmap_chunked(&p.tm[1], db, P, g.f, 64) ||
+      !make_tmap_chunked(&p.tm[2], dy_pad, P, g.h, 64) ||
+      !make_tmap_chunked(&p.tm[3], x_pad, P, g.h, 64) ||
+      !make_tmap_chunked(&p.tm[4], h_in, P, g.f, 64) || !make_tmap(&p.tmo[0], dw1, EF, g.h, 32, 4) ||
       !make_tmap(&p.tmo[1], dw3, EF, g.h, 32, 4) || !make_tmap(&p.tmo[2], dw2, EH, g.f, 32, 4))
     return cudaErrorInvalidValue;
   const long long t13 = (long long)((g.f / BM + 1) / 2) * ((g.h + BN - 1) / BN);
