@@ -109,9 +109,9 @@ __host__ __device__ constexpr bool is_dense_rows(int mode) {
 // Per-launch configuration.  4 epilogue warps (one per TMEM sub-partition) by default, or 8
 // (two per sub-partition, each taking half of the tile's columns) for GEMMs whose K is so short
 // (a few K steps per tile) that the epilogue, not the MMA, bounds a tile.  The ring of 32 KB
-// stages is as deep as shared memory allows next to the result staging: 6 stages with one
-// 4 KB staging buffer per warp for the forward GEMMs (few result boxes per tile; the deeper
-// ring hides more operand latency), else 5 (4 with 8 warps) with two.
+// stages is as deep as shared memory allows next to the result staging: for the forward GEMMs
+// (few result boxes per tile) 3 stages of two K slabs (64 KB) and one 4 KB staging buffer per
+// warp, else 5 stages of one slab (4 with 8 warps) and two staging buffers.
 template <int MODE, int EPI>
 struct Cfg {
   static constexpr int a_mn = (MODE == MODE_WGRAD || MODE == MODE_RWGRAD) ? 1 : 0;
@@ -122,13 +122,18 @@ struct Cfg {
   static constexpr int epi_warps = EPI;
   static constexpr int col_split = epi_warps / 4;  // warps per TMEM sub-partition
   static constexpr int threads = 64 + 32 * epi_warps;
-  static constexpr int stages =
-      (EPI == 8) ? 4 : ((MODE == MODE_GLU || MODE == MODE_DOWN) ? 6 : 5);
-  static constexpr int out_bufs = (stages == 6) ? 1 : 2;
+  // K slabs (64 deep) per stage: the forward GEMMs with K-major operands load two slabs of
+  // each operand with one 3D box, halving the TMA instructions per byte.
+  static constexpr int kslabs = (EPI == 4 && (MODE == MODE_GLU || MODE == MODE_DOWN)) ? 2 : 1;
+  static constexpr int bk = BK * kslabs;  // K per stage
+  static constexpr int a_bytes = A_BYTES * kslabs;
+  static constexpr int stage_bytes = (A_BYTES + B_BYTES) * kslabs;
+  static constexpr int stages = (kslabs == 2) ? 3 : ((EPI == 8) ? 4 : 5);
+  static constexpr int out_bufs = (kslabs == 2) ? 1 : 2;
   static constexpr int out_bytes = epi_warps * out_bufs * BOX_BYTES;
   // WGRAD: one zeroed result box, the source of the zero tiles' stores
   static constexpr int zero_bytes = (MODE == MODE_WGRAD) ? BOX_BYTES : 0;
-  static constexpr size_t smem = 1024 /*align*/ + (size_t)stages * STAGE_BYTES + out_bytes +
+  static constexpr size_t smem = 1024 /*align*/ + (size_t)stages * stage_bytes + out_bytes +
                                  zero_bytes + 256 /*barriers*/ +
                                  sizeof(int) * (DMOE_MAX_EXPERTS + 1);
 };
@@ -270,13 +275,18 @@ __device__ __forceinline__ float row_weight(const GemmParams &p, int e, int row)
                                       : 0.0f;
 }
 
-template <int MODE>
+// The operand boxes of stage kb (KSLABS slabs of 64 K) of tile tl, this CTA's half of the pair.
+template <int MODE, int KSLABS>
 __device__ __forceinline__ void load_stage(const GemmParams &p, const Tile &tl, int kb,
                                            uint32_t rank, uint8_t *sa, uint8_t *sb,
                                            uint32_t bar) {
-  if (MODE == MODE_GLU) {
-    tma_load_2d_pair(sa, &p.tm[0], bar, kb * BK, tl.row0);
-    tma_load_2d_pair(sb, &p.tm[rank == 0 ? 1 : 2], bar, kb * BK, tl.e * p.f + tl.n * (BN / 2));
+  if (MODE == MODE_GLU) {  // two K slabs per stage: 3D maps {64, rows, K/64}
+    static_assert(MODE != MODE_GLU || KSLABS == 2, "GLU stages hold two K slabs");
+    tma_load_3d_pair(sa, &p.tm[0], bar, 0, tl.row0, 2 * kb);
+    tma_load_3d_pair(sb, &p.tm[rank == 0 ? 1 : 2], bar, 0, tl.e * p.f + tl.n * (BN / 2), 2 * kb);
+  } else if (MODE == MODE_DOWN && KSLABS == 2) {
+    tma_load_3d_pair(sa, &p.tm[0], bar, 0, tl.row0, 2 * kb);
+    tma_load_3d_pair(sb, &p.tm[1], bar, 0, tl.e * p.h + tl.n * BN + (int)rank * (BN / 2), 2 * kb);
   } else if (MODE == MODE_DOWN) {
     tma_load_2d_pair(sa, &p.tm[0], bar, kb * BK, tl.row0);
     tma_load_2d_pair(sb, &p.tm[1], bar, kb * BK, tl.e * p.h + tl.n * BN + (int)rank * (BN / 2));
@@ -615,7 +625,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base_u32 = smem_u32(smem_raw);
   uint8_t *tiles = smem_raw + ((1024u - (base_u32 & 1023u)) & 1023u);
-  uint8_t *outbuf = tiles + STAGES * STAGE_BYTES;  // 1024-aligned
+  uint8_t *outbuf = tiles + STAGES * C::stage_bytes;  // 1024-aligned
   uint8_t *zbuf = outbuf + C::out_bytes;           // 1024-aligned (WGRAD only)
   uint64_t *bars = reinterpret_cast<uint64_t *>(zbuf + C::zero_bytes);
   uint64_t *full = bars;                       // [STAGES] leader: both halves landed
@@ -717,7 +727,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
           ok = false;
           break;
         }
-        uint8_t *sa = tiles + stage * STAGE_BYTES;
+        uint8_t *sa = tiles + stage * C::stage_bytes;
         const uint32_t bar = leader_full0 + (uint32_t)(stage * sizeof(uint64_t));
         if (p.inject && leader && issued == 0 && kb == 0) {
           // test-only stall: this stage is never armed, so the MMA's wait on it expires
@@ -728,15 +738,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
           ++issued;
           continue;
         }
-        if (lane == 0 && leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+        if (lane == 0 && leader) mbar_arrive_expect_tx(&full[stage], 2 * C::stage_bytes);
         if (MODE == MODE_GLU_GATHER) {
           tma_gather4_pair(sa + lane * 4 * 128, &p.tm[3], bar, kb * BK, rows[0], rows[1], rows[2],
                            rows[3]);
           if (lane == 0)
-            tma_load_2d_pair(sa + A_BYTES, &p.tm[rank == 0 ? 1 : 2], bar, kb * BK,
+            tma_load_2d_pair(sa + C::a_bytes, &p.tm[rank == 0 ? 1 : 2], bar, kb * BK,
                              tl.e * p.f + tl.n * (BN / 2));
         } else if (lane == 0) {
-          load_stage<MODE>(p, tl, kb, rank, sa, sa + A_BYTES, bar);
+          load_stage<MODE, C::kslabs>(p, tl, kb, rank, sa, sa + C::a_bytes, bar);
         }
         ++issued;
         if (++stage == STAGES) {
@@ -771,16 +781,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
           break;
         }
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(tiles + stage * STAGE_BYTES);
-        const uint32_t b_addr = a_addr + A_BYTES;
+        const uint32_t a_addr = smem_u32(tiles + stage * C::stage_bytes);
+        const uint32_t b_addr = a_addr + C::a_bytes;
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
+        for (int kk = 0; kk < C::bk / 16; ++kk) {
+          // K-major: slab kk / 4 (one 128 B swizzle row of 64 K per slab), 32 B per 16 K inside
           const uint64_t ad = C::a_mn
                                   ? sdesc_mnmajor_sw128(a_addr + kk * 2048, CHUNK_BYTES)
-                                  : sdesc_kmajor_sw128(a_addr + kk * 32);
+                                  : sdesc_kmajor_sw128(a_addr + (kk >> 2) * A_BYTES + (kk & 3) * 32);
           const uint64_t bd = C::b_mn
                                   ? sdesc_mnmajor_sw128(b_addr + kk * 2048, CHUNK_BYTES)
-                                  : sdesc_kmajor_sw128(b_addr + kk * 32);
+                                  : sdesc_kmajor_sw128(b_addr + (kk >> 2) * B_BYTES + (kk & 3) * 32);
           tc_mma_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
         }
         tc_commit_pair_mc(&empty[stage]);
@@ -999,8 +1010,11 @@ cudaError_t launch_glu_gemm(const GemmProblem &g, const void *x_pad, const void 
   GemmParams p = base_params(g);
   const uint64_t P = (uint64_t)g.nblk_cap * BM;
   const uint64_t EF = (uint64_t)g.E * g.f;
-  if (!make_tmap(&p.tm[0], x_pad, P, g.h, BM) || !make_tmap(&p.tm[1], w1, EF, g.h, BN / 2) ||
-      !make_tmap(&p.tm[2], w3, EF, g.h, BN / 2) || !make_tmap(&p.tmo[0], h_out, P, g.f, 32))
+  // K-major operands viewed as {64, rows, K/64}: one box brings two 64-deep K slabs
+  if (!make_tmap_chunked(&p.tm[0], x_pad, P, g.h, BM) ||
+      !make_tmap_chunked(&p.tm[1], w1, EF, g.h, BN / 2) ||
+      !make_tmap_chunked(&p.tm[2], w3, EF, g.h, BN / 2) ||
+      !make_tmap(&p.tmo[0], h_out, P, g.f, 32))
     return cudaErrorInvalidValue;
   if (a_out && b_out) {
     if (!make_tmap(&p.tmo[1], a_out, P, g.f, 32) || !make_tmap(&p.tmo[2], b_out, P, g.f, 32))
@@ -1009,7 +1023,7 @@ cudaError_t launch_glu_gemm(const GemmProblem &g, const void *x_pad, const void 
   }
   p.tm[3] = p.tm[4] = p.tm[0];
   p.n_tiles = g.f / (BN / 2);
-  p.k_iters = g.h / BK;
+  p.k_iters = g.h / Cfg<MODE_GLU, 4>::bk;
   p.group = raster_units(g.h);
   return launch_gemm<MODE_GLU, 4>(p, max_units(g) * p.n_tiles, st);
 }
@@ -1040,16 +1054,20 @@ cudaError_t launch_down_gemm(const GemmProblem &g, const void *h_in, const void 
                              cudaStream_t st) {
   GemmParams p = base_params(g);
   const uint64_t P = (uint64_t)g.nblk_cap * BM;
-  if (!make_tmap(&p.tm[0], h_in, P, g.f, BM) ||
-      !make_tmap(&p.tm[1], w2, (uint64_t)g.E * g.h, g.f, BN / 2) ||
-      !make_tmap(&p.tmo[0], y_pad, P, g.h, 32))
-    return cudaErrorInvalidValue;
+  const bool short_k = g.f / BK <= 4;  // ffn <= 256: the epilogue bounds a tile (8 warps)
+  const bool ok = short_k ? (make_tmap(&p.tm[0], h_in, P, g.f, BM) &&
+                             make_tmap(&p.tm[1], w2, (uint64_t)g.E * g.h, g.f, BN / 2))
+                          : (make_tmap_chunked(&p.tm[0], h_in, P, g.f, BM) &&
+                             make_tmap_chunked(&p.tm[1], w2, (uint64_t)g.E * g.h, g.f, BN / 2));
+  if (!ok || !make_tmap(&p.tmo[0], y_pad, P, g.h, 32)) return cudaErrorInvalidValue;
   p.tm[2] = p.tm[3] = p.tm[4] = p.tm[0];
   p.n_tiles = (g.h + BN - 1) / BN;
-  p.k_iters = g.f / BK;
   p.group = raster_units(g.f);
-  if (p.k_iters <= 4)  // ffn <= 256: the epilogue bounds a tile; give it 8 warps
+  if (short_k) {
+    p.k_iters = g.f / Cfg<MODE_DOWN, 8>::bk;
     return launch_gemm<MODE_DOWN, 8>(p, max_units(g) * p.n_tiles, st);
+  }
+  p.k_iters = g.f / Cfg<MODE_DOWN, 4>::bk;
   return launch_gemm<MODE_DOWN, 4>(p, max_units(g) * p.n_tiles, st);
 }
 
