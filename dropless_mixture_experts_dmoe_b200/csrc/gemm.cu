@@ -94,6 +94,15 @@ __host__ __device__ constexpr bool is_glu(int mode) {
   return mode == MODE_GLU || mode == MODE_GLU_GATHER;
 }
 
+// 64-deep K slabs per pipeline stage: two (operands as 3D TMA boxes, one instruction per
+// operand and stage, a 3-deep ring of 64 KB stages and one staging buffer per epilogue warp)
+// for the GEMMs with 4 epilogue warps and few result boxes per tile; one for the others.
+// Measured: two slabs speed up GLU, DOWN and DX, and slow DGLU (12 result boxes per tile
+// through one staging buffer) and the weight gradients.
+__host__ __device__ constexpr int mode_kslabs(int mode, int epi) {
+  return (epi == 4 && (mode == MODE_GLU || mode == MODE_DOWN || mode == MODE_DX)) ? 2 : 1;
+}
+
 // Modes whose tiles are (pair of an expert's row blocks, column tile), enumerated from
 // padded_bins; the others are the weight gradients and the dense router GEMMs.
 __host__ __device__ constexpr bool uses_units(int mode) {
@@ -124,7 +133,7 @@ struct Cfg {
   static constexpr int threads = 64 + 32 * epi_warps;
   // K slabs (64 deep) per stage: the forward GEMMs with K-major operands load two slabs of
   // each operand with one 3D box, halving the TMA instructions per byte.
-  static constexpr int kslabs = (EPI == 4 && (MODE == MODE_GLU || MODE == MODE_DOWN)) ? 2 : 1;
+  static constexpr int kslabs = mode_kslabs(MODE, EPI);
   static constexpr int bk = BK * kslabs;  // K per stage
   static constexpr int a_bytes = A_BYTES * kslabs;
   static constexpr int stage_bytes = (A_BYTES + B_BYTES) * kslabs;
@@ -222,7 +231,7 @@ __device__ __forceinline__ Tile decode(const GemmParams &p, int t, const int *us
     tl.dummy = tl.m >= mtiles;  // its A boxes start past the matrix: zeros
     const int start = (tl.e > 0) ? p.padded_bins[tl.e - 1] : 0;
     tl.row0 = start;
-    tl.kit = (p.padded_bins[tl.e] - start) / BK;
+    tl.kit = (p.padded_bins[tl.e] - start) / (BK * mode_kslabs(MODE_WGRAD, 4));
     return tl;
   }
   const int vu = t / p.n_tiles;  // units partition the tile list in order
@@ -294,12 +303,12 @@ __device__ __forceinline__ void load_stage(const GemmParams &p, const Tile &tl, 
     tma_load_2d_pair(sa, &p.tm[0], bar, kb * BK, tl.row0);
     // MN-major B: both 64-column chunks of this CTA's half in one box of the chunked map
     tma_load_3d_pair(sb, &p.tm[1], bar, 0, tl.e * p.h + kb * BK, (tl.n * BN) / 64 + 2 * (int)rank);
-  } else if (MODE == MODE_DX) {
-    const int kf = p.f / BK;
+  } else if (MODE == MODE_DX) {  // two K slabs per stage
+    const int kf = p.f / (2 * BK);
     const int pass = (kb < kf) ? 0 : 1;
     const int kk = kb - pass * kf;
-    tma_load_2d_pair(sa, &p.tm[pass], bar, kk * BK, tl.row0);
-    tma_load_3d_pair(sb, &p.tm[2 + pass], bar, 0, tl.e * p.f + kk * BK,
+    tma_load_3d_pair(sa, &p.tm[pass], bar, 0, tl.row0, 2 * kk);
+    tma_load_3d_pair(sb, &p.tm[2 + pass], bar, 0, tl.e * p.f + kk * 2 * BK,
                      (tl.n * BN) / 64 + 2 * (int)rank);
   } else if (MODE == MODE_ROUTER) {
     tma_load_2d_pair(sa, &p.tm[0], bar, kb * BK, tl.row0);
@@ -787,10 +796,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
         for (int kk = 0; kk < C::bk / 16; ++kk) {
           // K-major: slab kk / 4 (one 128 B swizzle row of 64 K per slab), 32 B per 16 K inside
           const uint64_t ad = C::a_mn
-                                  ? sdesc_mnmajor_sw128(a_addr + kk * 2048, CHUNK_BYTES)
+                                  ? sdesc_mnmajor_sw128(a_addr + kk * 2048, CHUNK_BYTES * C::kslabs)
                                   : sdesc_kmajor_sw128(a_addr + (kk >> 2) * A_BYTES + (kk & 3) * 32);
           const uint64_t bd = C::b_mn
-                                  ? sdesc_mnmajor_sw128(b_addr + kk * 2048, CHUNK_BYTES)
+                                  ? sdesc_mnmajor_sw128(b_addr + kk * 2048, CHUNK_BYTES * C::kslabs)
                                   : sdesc_kmajor_sw128(b_addr + (kk >> 2) * B_BYTES + (kk & 3) * 32);
           tc_mma_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
         }
@@ -1077,7 +1086,7 @@ cudaError_t launch_dglu_gemm(const GemmProblem &g, const void *dy_pad, const voi
   GemmParams p = base_params(g);
   const uint64_t P = (uint64_t)g.nblk_cap * BM;
   if (!make_tmap(&p.tm[0], dy_pad, P, g.h, BM) ||
-      !make_tmap_chunked(&p.tm[1], w2, (uint64_t)g.E * g.h, g.f, 64) ||
+      !make_tmap_chunked(&p.tm[1], w2, (uint64_t)g.E * g.h, g.f, BK) ||
       !make_tmap(&p.tmo[0], da_out, P, g.f, 32) || !make_tmap(&p.tmo[1], db_out, P, g.f, 32) ||
       !make_tmap(&p.tmo[2], hw_out, P, g.f, 32))
     return cudaErrorInvalidValue;
@@ -1085,7 +1094,7 @@ cudaError_t launch_dglu_gemm(const GemmProblem &g, const void *dy_pad, const voi
   p.part = part;
   p.tm[2] = p.tm[3] = p.tm[4] = p.tm[0];
   p.n_tiles = (g.f + BN - 1) / BN;
-  p.k_iters = g.h / BK;
+  p.k_iters = g.h / Cfg<MODE_DGLU, 4>::bk;
   p.group = raster_units(g.h);
   p.in0 = static_cast<const __nv_bfloat16 *>(a_in);
   p.in1 = static_cast<const __nv_bfloat16 *>(b_in);
@@ -1097,14 +1106,15 @@ cudaError_t launch_dx_gemm(const GemmProblem &g, const void *da, const void *db,
   GemmParams p = base_params(g);
   const uint64_t P = (uint64_t)g.nblk_cap * BM;
   const uint64_t EF = (uint64_t)g.E * g.f;
-  if (!make_tmap(&p.tm[0], da, P, g.f, BM) || !make_tmap(&p.tm[1], db, P, g.f, BM) ||
-      !make_tmap_chunked(&p.tm[2], w1, EF, g.h, 64) ||
-      !make_tmap_chunked(&p.tm[3], w3, EF, g.h, 64) ||
+  if (!make_tmap_chunked(&p.tm[0], da, P, g.f, BM) ||
+      !make_tmap_chunked(&p.tm[1], db, P, g.f, BM) ||
+      !make_tmap_chunked(&p.tm[2], w1, EF, g.h, 2 * BK) ||
+      !make_tmap_chunked(&p.tm[3], w3, EF, g.h, 2 * BK) ||
       !make_tmap(&p.tmo[0], dx_pad, P, g.h, 32))
     return cudaErrorInvalidValue;
   p.tm[4] = p.tm[0];
   p.n_tiles = (g.h + BN - 1) / BN;
-  p.k_iters = 2 * (g.f / BK);
+  p.k_iters = 2 * (g.f / Cfg<MODE_DX, 4>::bk);
   p.group = raster_units(2 * g.f);
   return launch_gemm<MODE_DX, 4>(p, max_units(g) * p.n_tiles, st);
 }
@@ -1115,11 +1125,11 @@ cudaError_t launch_wgrad_gemm(const GemmProblem &g, const void *x_pad, const voi
   GemmParams p = base_params(g);
   const uint64_t P = (uint64_t)g.nblk_cap * BM;
   const uint64_t EF = (uint64_t)g.E * g.f, EH = (uint64_t)g.E * g.h;
-  if (!make_tmap_chunked(&p.tm[0], da, P, g.f, 64) ||
-      !make_tmap_chunked(&p.tm[1], db, P, g.f, 64) ||
-      !make_tmap_chunked(&p.tm[2], dy_pad, P, g.h, 64) ||
-      !make_tmap_chunked(&p.tm[3], x_pad, P, g.h, 64) ||
-      !make_tmap_chunked(&p.tm[4], h_in, P, g.f, 64) || !make_tmap(&p.tmo[0], dw1, EF, g.h, 32, 4) ||
+  if (!make_tmap_chunked(&p.tm[0], da, P, g.f, BK) ||
+      !make_tmap_chunked(&p.tm[1], db, P, g.f, BK) ||
+      !make_tmap_chunked(&p.tm[2], dy_pad, P, g.h, BK) ||
+      !make_tmap_chunked(&p.tm[3], x_pad, P, g.h, BK) ||
+      !make_tmap_chunked(&p.tm[4], h_in, P, g.f, BK) || !make_tmap(&p.tmo[0], dw1, EF, g.h, 32, 4) ||
       !make_tmap(&p.tmo[1], dw3, EF, g.h, 32, 4) || !make_tmap(&p.tmo[2], dw2, EH, g.f, 32, 4))
     return cudaErrorInvalidValue;
   const long long t13 = (long long)((g.f / BM + 1) / 2) * ((g.h + BN - 1) / BN);
