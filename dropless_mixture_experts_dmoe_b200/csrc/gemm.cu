@@ -72,7 +72,6 @@ constexpr int BN = 256;  // output columns per tile
 constexpr int BK = 64;   // K per pipeline stage (one 128-byte swizzle row of bf16)
 constexpr int A_BYTES = BM * BK * 2;        // 16 KB: this CTA's 128 rows of A
 constexpr int B_BYTES = (BN / 2) * BK * 2;  // 16 KB: this CTA's half of B
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int CHUNK_BYTES = 64 * BK * 2;    // one 64 x 64 MN-major box: 8 KB
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = 256;
