@@ -184,6 +184,21 @@ def cpu_sample_tokens(w, requested):
     return max(8, min(w.T, int(4e11 / per_tok)))
 
 
+def job_throughput(ms_local: float, world: int, tokens_per_rank: int, steps: int, device: str):
+    """Whole-job figures of a timed region: the slowest rank's time (max over ranks, one
+    all-reduce when world > 1; every rank takes part) and the tokens all ranks processed per
+    second over it.  Returns (ms_max, tokens/s)."""
+    import torch
+
+    t = torch.tensor([float(ms_local)], device=device, dtype=torch.float64)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    return ms_max, world * tokens_per_rank * steps / (ms_max / 1e3)
+
+
 def run_reference(args, w):
     import oracle
 
@@ -350,12 +365,8 @@ def run_ours(args, w):
     ms = start.elapsed_time(stop)
     per_kernel = {n: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)]
                   for j, n in enumerate(names)}
-    t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max, value = job_throughput(ms, world, w.T, args.steps, "cuda")
     ms_per_step = ms_max / args.steps
-    value = world * w.T * args.steps / (ms_max / 1e3)
 
     # ---- e2e through the public API with host buffers ----
     # Every step copies its inputs from pinned host memory and its results back.  Three
@@ -431,10 +442,7 @@ def run_ours(args, w):
     s_out.wait_stream(s_in)
     e1.record(s_out)
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1)], device="cuda", dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = world * w.T * args.steps / (float(te.item()) / 1e3)
+    _, e2e_value = job_throughput(e0.elapsed_time(e1), world, w.T, args.steps, "cuda")
     h2d = x_h[0].numel() * 2 + (0 if router else lg_h[0].numel() * 2) + \
         (dy_h[0].numel() * 2 if train else 0)
     d2h = y_h[0].numel() * 2 + (dx_h[0].numel() * 2 if train else 0)
