@@ -11,20 +11,28 @@
 // section 4.3's transposed topology) are a tile per (expert, pair of output row tiles, column
 // tile) whose K loop walks that expert's padded rows.
 //
-// Kernel structure (clusters of 2 CTAs on an SM pair, 192 threads each, persistent):
+// Kernel structure (clusters of 2 CTAs on an SM pair, 192 or 320 threads each, persistent,
+// tiles taken in snake order: round r of the loop covers tiles [r*n, r*n + n), increasing on
+// even rounds and decreasing on odd ones):
 //   warp 0      TMA producer (both CTAs): this CTA's 128 rows of A and its half (128 rows)
-//               of B per stage, 5-stage ring of 32 KB, 128-byte swizzle; every load completes
-//               on the pair leader's mbarrier (expect-tx of both halves).
+//               of B per stage, 128-byte swizzle; every load completes on the pair leader's
+//               mbarrier (expect-tx of both halves).  GLU, DOWN (ffn > 256) and DX stages hold
+//               two 64-deep K slabs (64 KB, three stages), each operand brought by one box of a
+//               3D view of its tensor; the other modes use 32 KB one-slab stages (five, four
+//               with 8 epilogue warps), MN-major operands again as one 3D box of two 64-column
+//               chunks.
 //   warp 1      allocates 512 TMEM columns in both CTAs; one thread of the leader issues
 //               tcgen05.mma.cta_group::2 (bf16 in, fp32 accumulate), which reads both CTAs'
 //               shared memory and writes each CTA's 128 accumulator rows into its own TMEM,
 //               and tcgen05.commit (multicast to both CTAs) to free stages and hand over
-//               accumulators.
-//   warps 2..   epilogue (both CTAs; 4 warps, or 8 for a DOWN GEMM with ffn <= 256): tcgen05.ld of
-//               the accumulator (each warp its 32-lane TMEM sub-partition and, with 8 warps,
-//               half of the columns), fused element-wise work, results staged in 128-byte-
-//               swizzled shared memory (32 rows x 128 B per box) and written with TMA
-//               bulk-tensor stores, double-buffered per warp.
+//               accumulators.  In the weight-gradient mode the peer CTA's warp 1 stores the zero
+//               tiles of experts without rows.
+//   warps 2..   epilogue (both CTAs; 4 warps, or 8 for a DOWN GEMM with ffn <= 256 and the
+//               router's dx GEMM): tcgen05.ld of the accumulator (each warp its 32-lane TMEM
+//               sub-partition and, with 8 warps, half of the columns), fused element-wise work,
+//               results staged in 128-byte-swizzled shared memory (32 rows x 128 B per box)
+//               and written with TMA bulk-tensor stores; one arrival per warp releases the
+//               accumulator.
 // Two accumulators (2 x 256 columns) let the epilogue of tile i overlap the MMAs of i+1.
 // An expert with an odd number of row blocks ends with a unit whose second CTA reads zero
 // rows (TMA fill past the last padded row) and stores nothing.
