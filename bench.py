@@ -62,10 +62,17 @@ def peaks():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the GEMM kernel's code (comments and whitespace removed, so that an edit of the
+    documentation does not discard counters that still describe the kernel)."""
+    import re
+
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "dropless_mixture_experts_dmoe_b200", "csrc")
     for fn in ("gemm.cu", "common.cuh"):
-        h.update(open(os.path.join(csrc, fn), "rb").read())
+        text = open(os.path.join(csrc, fn), encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 
