@@ -195,19 +195,16 @@ int dmoe_sparse_map(const dmoe_dims *dims, const void *logits, const dmoe_map *m
   const int T = dims->T, E = dims->num_experts, k = dims->top_k;
   const int nblk_cap = (int)(pmax_of(dims) / DMOE_BLOCKING);
   int32_t *tile_hist = static_cast<int32_t *>(ws);
-  if (cudaMemsetAsync(map->status, 0, sizeof(int32_t), st) != cudaSuccess) return DMOE_ERR_LAUNCH;
   const bool renorm = (dims->route_flags & DMOE_ROUTE_RENORMALIZE) != 0;
   if ((rc = launch_rc(launch_route_hist(static_cast<const uint16_t *>(logits), T, E, k, renorm,
-                                        map->top_experts, map->weights, tile_hist, map->status,
-                                        st))))
+                                        map->top_experts, map->weights, tile_hist, st))))
     return rc;
-  if ((rc = launch_rc(launch_map_scan(T, E, nblk_cap, tile_hist, map->tokens_per_expert,
-                                      map->bins, map->padded_bins, map->block_expert,
-                                      map->num_blocks, st))))
+  if ((rc = launch_rc(launch_map_scan(T, E, tile_hist, map->tokens_per_expert, map->bins,
+                                      map->padded_bins, map->num_blocks, map->status, st))))
     return rc;
-  return launch_rc(launch_map_scatter(T, E, k, map->top_experts, tile_hist, map->bins,
+  return launch_rc(launch_map_scatter(T, E, k, nblk_cap, map->top_experts, tile_hist, map->bins,
                                       map->padded_bins, map->indices, map->bin_ids,
-                                      map->dest_row, st));
+                                      map->dest_row, map->block_expert, st));
 }
 
 int dmoe_padded_gather(const dmoe_dims *dims, const void *x, const dmoe_map *map, void *x_pad,

@@ -11,6 +11,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/dmoe.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
@@ -28,6 +30,45 @@ constexpr long long kInjectedWaitCycles = 10000000LL;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---- programmatic dependent launch ---------------------------------------------------------
+//
+// Every kernel of the library is launched with programmatic stream serialisation: the next
+// kernel on the stream may be scheduled before this one has finished, runs only its
+// prologue (shared-memory and barrier setup, tensor-memory allocation), and then blocks in
+// pdl_wait() until every earlier kernel of the stream has completed and its writes are
+// visible.  So each kernel calls pdl_wait() before its first global-memory access (read or
+// write: a later kernel may overwrite what an earlier one still reads), and pdl_trigger()
+// right after it, which lets the next launch proceed once every CTA of this grid is past its
+// wait: at most one kernel waits behind the running one (triggering before the wait let a
+// chain of small kernels sit resident and idle, taking occupancy from the running one).
+// The persistent GEMM does not trigger: its dependents are released as its CTAs exit.
+// Without the launch attribute both are no-ops.
+#ifndef DMOE_PDL
+#define DMOE_PDL 1
+#endif
+
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Launch `kernel` on `st` with the programmatic-serialisation attribute.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = DMOE_PDL;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 __device__ __forceinline__ void set_status(int32_t *status, int bits) {

@@ -36,6 +36,8 @@ __global__ void __launch_bounds__(kCopyThreads) k_gather(int T, int h, int k, in
                                                          const int32_t *__restrict__ counts,
                                                          const int32_t *__restrict__ padded_bins,
                                                          uint4 *__restrict__ x_pad) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int vpr = h >> 3;  // 16-byte vectors per row
   const int S = (vpr + kSliceVecs - 1) / kSliceVecs;
@@ -97,6 +99,8 @@ __global__ void __launch_bounds__(kCopyThreads) k_combine(int T, int h, int k,
                                                           uint4 *__restrict__ y,
                                                           const float *__restrict__ part, int nt,
                                                           float *__restrict__ dweights) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int vpr = h >> 3;
   const int S = (vpr + kSliceVecs - 1) / kSliceVecs;
@@ -183,10 +187,9 @@ cudaError_t launch_gather(int T, int h, int k, int E, const void *x, const int32
                           const int32_t *counts, const int32_t *padded_bins, void *x_pad,
                           cudaStream_t st) {
   const long long items = (long long)T * slices(h) + (long long)kBlock * E;
-  k_gather<<<copy_grid(items), kCopyThreads, 0, st>>>(
-      T, h, k, E, static_cast<const uint4 *>(x), dest_row, counts, padded_bins,
-      static_cast<uint4 *>(x_pad));
-  return cudaGetLastError();
+  return launch_pdl(k_gather, copy_grid(items), kCopyThreads, 0, st, T, h, k, E,
+                    static_cast<const uint4 *>(x), dest_row, counts, padded_bins,
+                    static_cast<uint4 *>(x_pad));
 }
 
 static cudaError_t combine(int T, int h, int k, const void *y_pad, const int32_t *dest_row,
@@ -195,16 +198,9 @@ static cudaError_t combine(int T, int h, int k, const void *y_pad, const int32_t
   const int grid = copy_grid((long long)T * slices(h));
   const uint4 *src = static_cast<const uint4 *>(y_pad);
   uint4 *dst = static_cast<uint4 *>(y);
-  if (k <= 2)
-    k_combine<8, 2><<<grid, kCopyThreads, 0, st>>>(T, h, k, src, dest_row, weights, dst, part, nt,
-                                                   dweights);
-  else if (k <= 4)
-    k_combine<4, 4><<<grid, kCopyThreads, 0, st>>>(T, h, k, src, dest_row, weights, dst, part, nt,
-                                                   dweights);
-  else
-    k_combine<2, 8><<<grid, kCopyThreads, 0, st>>>(T, h, k, src, dest_row, weights, dst, part, nt,
-                                                   dweights);
-  return cudaGetLastError();
+  auto kernel = (k <= 2) ? k_combine<8, 2> : (k <= 4) ? k_combine<4, 4> : k_combine<2, 8>;
+  return launch_pdl(kernel, grid, kCopyThreads, 0, st, T, h, k, src, dest_row, weights, dst, part,
+                    nt, dweights);
 }
 
 cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const int32_t *dest_row,

@@ -12,24 +12,31 @@ constexpr int kMapTokTile = 64;
 
 inline int map_tiles(int T) { return (T + kMapTokTile - 1) / kMapTokTile; }
 
-// Map workspace: per-tile histograms [map_tiles(T), E] int32, then one ticket counter.
-inline size_t map_workspace_ints(int T, int E) { return (size_t)map_tiles(T) * E + 1; }
+// Map workspace: per-tile histograms [map_tiles(T), E] int32, one ticket counter, then one
+// status word per tile.
+inline size_t map_workspace_ints(int T, int E) {
+  return (size_t)map_tiles(T) * E + 1 + (size_t)map_tiles(T);
+}
 inline unsigned int *map_ticket(int32_t *tile_hist, int T, int E) {
   return reinterpret_cast<unsigned int *>(tile_hist + (size_t)map_tiles(T) * E);
+}
+inline int32_t *map_flags(int32_t *tile_hist, int T, int E) {
+  return tile_hist + (size_t)map_tiles(T) * E + 1;
 }
 
 // Map: routing + per-tile histogram (logits given) or histogram of given top_experts.
 cudaError_t launch_route_hist(const uint16_t *logits, int T, int E, int k, bool renorm, int32_t *top,
-                              float *weights, int32_t *tile_hist, int32_t *status,
-                              cudaStream_t st);
-// Map: scan over tiles and experts, bins / padded_bins / block table.
-cudaError_t launch_map_scan(int T, int E, int nblk_cap, int32_t *tile_hist,
-                            int32_t *tokens_per_expert, int32_t *bins, int32_t *padded_bins,
-                            int32_t *block_expert, int32_t *num_blocks, cudaStream_t st);
-// Map: stable scatter of entries to sorted order; indices, bin_ids, dest_row.
-cudaError_t launch_map_scatter(int T, int E, int k, const int32_t *top, const int32_t *tile_off,
-                               const int32_t *bins, const int32_t *padded_bins, int32_t *indices,
-                               int32_t *bin_ids, int32_t *dest_row, cudaStream_t st);
+                              float *weights, int32_t *tile_hist, cudaStream_t st);
+// Map: scan over tiles and experts; bins, padded_bins, num_blocks and the status word.
+cudaError_t launch_map_scan(int T, int E, int32_t *tile_hist, int32_t *tokens_per_expert,
+                            int32_t *bins, int32_t *padded_bins, int32_t *num_blocks,
+                            int32_t *status, cudaStream_t st);
+// Map: stable scatter of entries to sorted order (indices, bin_ids, dest_row) and the
+// block -> expert table.
+cudaError_t launch_map_scatter(int T, int E, int k, int nblk_cap, const int32_t *top,
+                               const int32_t *tile_off, const int32_t *bins,
+                               const int32_t *padded_bins, int32_t *indices, int32_t *bin_ids,
+                               int32_t *dest_row, int32_t *block_expert, cudaStream_t st);
 
 // Token-major padded gather with zero-filled padding rows.
 cudaError_t launch_gather(int T, int h, int k, int E, const void *x, const int32_t *dest_row,

@@ -3,15 +3,17 @@
 //
 // Three kernels, no spin-waits, deterministic results (the only global atomic is the scan's
 // completion ticket):
-//   k_route_hist   one warp per token: top-k by integer max over order-preserving keys
-//                  (ties -> lower expert index), fp32 softmax weights, per-tile histogram in
-//                  shared memory (O(E) bytes, independent of T).
+//   k_route_hist   16 warps per 64-token tile, 4 tokens per warp with all their logits loaded
+//                  at once: top-k by integer max over order-preserving keys (ties -> lower
+//                  expert index), fp32 softmax weights, per-tile histogram in shared memory
+//                  (O(E) bytes, independent of T) and a per-tile status word.
 //   k_map_scan     one CTA per 32 experts: per-expert exclusive offsets of every tile; the
 //                  last CTA to finish (a ticket counter, no waiting) computes bins,
-//                  padded_bins (round_up to 128), num_blocks and the block -> expert table.
+//                  padded_bins (round_up to 128), num_blocks and stores the status word.
 //   k_map_scatter  one CTA per tile: stable rank of every entry inside its expert (warp
 //                  histograms + __match_any_sync ranks in entry order), then indices,
-//                  bin_ids and dest_row from the index math of section 4.2.
+//                  bin_ids and dest_row from the index math of section 4.2; every CTA also
+//                  fills a slice of the block -> expert table.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -20,76 +22,204 @@ namespace dmoe {
 constexpr int kMapThreads = 256;
 constexpr int kMapWarps = kMapThreads / 32;
 
-__device__ __forceinline__ bool bf16_nonfinite(uint16_t b) { return (b & 0x7F80u) == 0x7F80u; }
+
+// 2^x with the hardware approximation (a few ulp; subnormal results kept).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// e^(v - m) for v <= m: the difference of two bf16 values is exact in fp32, so only the
+// scaling by log2(e) and the 2^x approximation round.
+__device__ __forceinline__ float exp_diff(float v, float m) {
+  return ex2_approx(__fmul_rn(__fsub_rn(v, m), 1.4426950408889634f));
+}
+
+// Selection key of a logit given as its fp32 image u (a bf16 value in the high half): the high
+// half is the order-preserving image (negative -> bits inverted, else sign bit set; -0 taken as
+// +0; NaN -> 0, below -inf), the low half is `low` = 0xFFFF - expert, so among equal logits the
+// lower expert has the larger key.
+__device__ __forceinline__ uint32_t route_key(uint32_t u, uint32_t low) {
+  const float f = __fadd_rn(__uint_as_float(u), 0.0f);  // -0 + 0 = +0
+  const uint32_t z = __float_as_uint(f);
+  const uint32_t neg = (uint32_t)((int32_t)z >> 31);
+  const uint32_t key = (z ^ (neg & 0x7FFF0000u)) ^ (0x80000000u | low);
+  return ((z & 0x7FFFFFFFu) > 0x7F800000u) ? low : key;
+}
 
 // ---- routing + histogram ---------------------------------------------------------------------
 
-// KPL = logits per lane (E <= 32*KPL).
-template <int KPL>
-__global__ void __launch_bounds__(kMapThreads) k_route_hist(const uint16_t *__restrict__ logits,
-                                                            int T, int E, int k, int renorm,
-                                                            int32_t *__restrict__ top,
-                                                            float *__restrict__ weights,
-                                                            int32_t *__restrict__ tile_hist,
-                                                            int32_t *status,
-                                                            unsigned int *__restrict__ done) {
-  extern __shared__ int hist[];  // [E]
-  if (blockIdx.x == 0 && threadIdx.x == 0) *done = 0u;  // ticket counter of k_map_scan
-  for (int e = threadIdx.x; e < E; e += kMapThreads) hist[e] = 0;
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t0 = blockIdx.x * kMapTokTile;
-  bool bad = false;
-  // this warp's tokens are t0 + warp, t0 + warp + 8, ...; the next token's logits are loaded
-  // while the current token is ranked
-  uint16_t nxt[KPL];
-  auto load_row = [&](int t) {
+// The routing kernel runs 16 warps per 64-token tile, 4 tokens per warp, so that each warp has
+// all of its tokens' logits in flight at once: ranking a token is a chain of k dependent
+// warp reductions, and with one token loaded ahead the load latency was not hidden.
+constexpr int kRouteThreads = 512;
+constexpr int kRouteWarps = kRouteThreads / 32;
+constexpr int kRouteTPW = kMapTokTile / kRouteWarps;  // tokens per warp
+static_assert(kRouteTPW * kRouteWarps == kMapTokTile, "routing tile");
+
+// One lane's share of a token's logits.  KPL = logits per lane (E <= 32*KPL).  VEC (E a
+// multiple of KPL): lane l owns experts KPL*l .. KPL*l + KPL-1, read as one vector load and
+// kept packed two per word; otherwise lane l owns experts l, l + 32, ..., one per word.
+template <int KPL, bool VEC>
+struct RouteRow {
+  static constexpr int kWords = VEC ? (KPL + 1) / 2 : KPL;
+  uint32_t w[kWords];
+
+  __device__ __forceinline__ static int expert(int lane, int i) {
+    return VEC ? KPL * lane + i : lane + 32 * i;
+  }
+  // fp32 image of logit i (the bf16 bits in the high half)
+  __device__ __forceinline__ uint32_t image(int i) const {
+    if constexpr (VEC) return (i & 1) ? (w[i >> 1] & 0xFFFF0000u) : (w[i >> 1] << 16);
+    return w[i] << 16;
+  }
+  __device__ __forceinline__ void load(const uint16_t *__restrict__ row, int E, int lane) {
+    if constexpr (VEC) {
+      const int e0 = KPL * lane;
+      const bool ok = e0 < E;  // E % KPL == 0: the whole vector is in the row or none of it
+      if constexpr (KPL == 1) {
+        w[0] = ok ? (uint32_t)__ldg(row + e0) : 0u;
+      } else if constexpr (KPL == 2) {
+        w[0] = ok ? __ldg(reinterpret_cast<const unsigned int *>(row + e0)) : 0u;
+      } else if constexpr (KPL == 4) {
+        uint2 q = make_uint2(0u, 0u);
+        if (ok) q = __ldg(reinterpret_cast<const uint2 *>(row + e0));
+        w[0] = q.x;
+        w[1] = q.y;
+      } else {
 #pragma unroll
-    for (int i = 0; i < KPL; ++i) {
-      const int e = lane + 32 * i;
-      nxt[i] = (t < T && e < E) ? __ldg(logits + (size_t)t * E + e) : (uint16_t)0;
-    }
-  };
-  load_row(t0 + warp);
-  for (int tt = warp; tt < kMapTokTile; tt += kMapWarps) {
-    const int t = t0 + tt;
-    if (t >= T) break;
-    uint16_t cur[KPL];
+        for (int c = 0; c < kWords / 4; ++c) {
+          uint4 q = make_uint4(0u, 0u, 0u, 0u);
+          if (ok) q = __ldg(reinterpret_cast<const uint4 *>(row + e0) + c);
+          w[4 * c] = q.x;
+          w[4 * c + 1] = q.y;
+          w[4 * c + 2] = q.z;
+          w[4 * c + 3] = q.w;
+        }
+      }
+    } else {
 #pragma unroll
-    for (int i = 0; i < KPL; ++i) cur[i] = nxt[i];
-    if (tt + kMapWarps < kMapTokTile) load_row(t + kMapWarps);
-    uint32_t key[KPL];
-    float val[KPL];
-#pragma unroll
-    for (int i = 0; i < KPL; ++i) {
-      const int e = lane + 32 * i;
-      key[i] = 0u;
-      val[i] = 0.0f;
-      if (e < E) {
-        const uint16_t b = cur[i];
-        bad |= bf16_nonfinite(b);
-        key[i] = (bf16_order(b) << 16) | (0xFFFFu - (uint32_t)e);
-        val[i] = __uint_as_float((uint32_t)b << 16);
+      for (int i = 0; i < KPL; ++i) {
+        const int e = lane + 32 * i;
+        w[i] = (e < E) ? (uint32_t)__ldg(row + e) : 0u;
       }
     }
-    // k rounds of a warp-wide integer max; the winner's lane clears the key.
+  }
+};
+
+// Descending bitonic sort of N (a power of two) keys held in registers.
+template <int N>
+__device__ __forceinline__ void sort_desc(uint32_t (&a)[N]) {
+#pragma unroll
+  for (int size = 2; size <= N; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const uint32_t hi = max(a[i], a[j]), lo = min(a[i], a[j]);
+          if ((i & size) == 0) {
+            a[i] = hi;
+            a[j] = lo;
+          } else {
+            a[i] = lo;
+            a[j] = hi;
+          }
+        }
+      }
+    }
+  }
+}
+
+// Grid: one CTA per 64-token tile.  Per token: every lane turns its logits into unique integer
+// keys (order-preserving image of the bf16 value in the high half, 0xFFFF - expert in the low
+// half, so the larger key is the larger logit and, on equal logits, the lower expert); k rounds
+// of a warp-wide integer max pick the top-k in rank order.  With KPL <= 8 each lane sorts its
+// keys once and a round only pops the winning lane's head; wider rows clear the winner in
+// place.  Weights: fp32 softmax over all E logits (or, renormalised, over the k picks) with
+// the first pick as the maximum.  The tile's expert histogram is built in shared memory and
+// written to tile_hist; the tile's status bits go to tile_flags (a plain store, so the
+// workspace needs no initialisation).
+template <int KPL, bool VEC>
+__global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__restrict__ logits,
+                                                              int T, int E, int k, int renorm,
+                                                              int32_t *__restrict__ top,
+                                                              float *__restrict__ weights,
+                                                              int32_t *__restrict__ tile_hist,
+                                                              int32_t *__restrict__ tile_flags,
+                                                              unsigned int *__restrict__ done) {
+  using Row = RouteRow<KPL, VEC>;
+  constexpr bool kSorted = KPL <= 8;
+  constexpr int kInFlight = (KPL <= 8) ? kRouteTPW : 1;  // token rows loaded ahead per warp
+  extern __shared__ int hist[];  // [E]
+  __shared__ int s_flags;
+  pdl_wait();
+  pdl_trigger();
+  if (blockIdx.x == 0 && threadIdx.x == 0) *done = 0u;  // ticket counter of k_map_scan
+  if (threadIdx.x == 0) s_flags = 0;
+  for (int e = threadIdx.x; e < E; e += kRouteThreads) hist[e] = 0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * kMapTokTile + warp;
+  Row rows[kInFlight];
+#pragma unroll
+  for (int j = 0; j < kInFlight; ++j) {
+    const int t = t0 + kRouteWarps * j;
+    if (t < T) rows[j].load(logits + (size_t)t * E, E, lane);
+  }
+  __syncthreads();
+  bool bad = false;
+#pragma unroll
+  for (int j = 0; j < kRouteTPW; ++j) {
+    const int t = t0 + kRouteWarps * j;
+    if (t >= T) break;
+    Row cur;
+    if constexpr (kInFlight == kRouteTPW) {
+      cur = rows[j];
+    } else {
+      cur.load(logits + (size_t)t * E, E, lane);
+    }
+    uint32_t key[KPL];
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) {
+      const int e = Row::expert(lane, i);
+      const uint32_t u = cur.image(i);
+      key[i] = 0u;
+      if (e < E) {
+        bad |= (u & 0x7F800000u) == 0x7F800000u;
+        key[i] = route_key(u, 0xFFFFu - (uint32_t)e);
+      }
+    }
+    if constexpr (kSorted) sort_desc<KPL>(key);
+    // k rounds of a warp-wide integer max; keys are unique, so exactly one lane holds the
+    // winner, and a valid key is never 0 (its low half is >= 0xFFFF - 1023).
     int my_e = 0;
     uint32_t my_key = 0, top_key = 0;
     for (int s = 0; s < k; ++s) {
       uint32_t best = 0;
+      if constexpr (kSorted) {
+        best = key[0];
+      } else {
 #pragma unroll
-      for (int i = 0; i < KPL; ++i) best = max(best, key[i]);
+        for (int i = 0; i < KPL; ++i) best = max(best, key[i]);
+      }
       const uint32_t wb = __reduce_max_sync(0xFFFFFFFFu, best);
-      const int e = 0xFFFF - (int)(wb & 0xFFFFu);
       if (s == 0) top_key = wb;
-      if ((e & 31) == lane) {
+      if (lane == s) {
+        my_e = 0xFFFF - (int)(wb & 0xFFFFu);
+        my_key = wb;
+      }
+      if constexpr (kSorted) {
+        if (key[0] == wb) {
+#pragma unroll
+          for (int i = 0; i + 1 < KPL; ++i) key[i] = key[i + 1];
+          key[KPL - 1] = 0u;
+        }
+      } else {
 #pragma unroll
         for (int i = 0; i < KPL; ++i)
-          if (i == (e >> 5)) key[i] = 0u;
-      }
-      if (lane == s) {
-        my_e = e;
-        my_key = wb;
+          if (key[i] == wb) key[i] = 0u;
       }
     }
     // softmax over all E logits (or, renormalised, over the k picks), max = the first pick.
@@ -98,36 +228,43 @@ __global__ void __launch_bounds__(kMapThreads) k_route_hist(const uint16_t *__re
     const float v = (lane < k) ? (((my_key >> 16) == 0u) ? __uint_as_float(0x7FC00000u)
                                                          : bf16_from_order(my_key >> 16))
                                : 0.0f;
+    const float ev = exp_diff(v, m);
     float sum = 0.0f;
     if (renorm) {
-      if (lane < k) sum = expf(v - m);
+      if (lane < k) sum = ev;
     } else {
 #pragma unroll
       for (int i = 0; i < KPL; ++i)
-        if (lane + 32 * i < E) sum += expf(val[i] - m);
+        if (Row::expert(lane, i) < E) sum += exp_diff(__uint_as_float(cur.image(i)), m);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
     if (lane < k) {
       top[(size_t)t * k + lane] = my_e;
-      weights[(size_t)t * k + lane] = expf(v - m) / sum;
+      weights[(size_t)t * k + lane] = __fdividef(ev, sum);  // 1 <= sum <= E
       atomicAdd(&hist[my_e], 1);
     }
   }
-  if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) set_status(status, DMOE_STATUS_NONFINITE_LOGITS);
+  if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) atomicOr(&s_flags, DMOE_STATUS_NONFINITE_LOGITS);
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += kMapThreads)
+  for (int e = threadIdx.x; e < E; e += kRouteThreads)
     tile_hist[(size_t)blockIdx.x * E + e] = hist[e];
+  if (threadIdx.x == 0) tile_flags[blockIdx.x] = s_flags;
 }
 
-// Histogram of caller-given top_experts; invalid ids are reported and left out of the map.
+// Histogram of caller-given top_experts; invalid ids are reported (in tile_flags) and left
+// out of the map.
 __global__ void __launch_bounds__(kMapThreads) k_given_hist(const int32_t *__restrict__ top,
                                                             int T, int E, int k,
                                                             int32_t *__restrict__ tile_hist,
-                                                            int32_t *status,
+                                                            int32_t *__restrict__ tile_flags,
                                                             unsigned int *__restrict__ done) {
   extern __shared__ int hist[];
+  __shared__ int s_flags;
+  pdl_wait();
+  pdl_trigger();
   if (blockIdx.x == 0 && threadIdx.x == 0) *done = 0u;  // ticket counter of k_map_scan
+  if (threadIdx.x == 0) s_flags = 0;
   for (int e = threadIdx.x; e < E; e += kMapThreads) hist[e] = 0;
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -151,15 +288,19 @@ __global__ void __launch_bounds__(kMapThreads) k_given_hist(const int32_t *__res
     }
   }
   flags = __reduce_or_sync(0xFFFFFFFFu, flags);
-  if (flags && lane == 0) set_status(status, flags);
+  if (flags && lane == 0) atomicOr(&s_flags, flags);
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += kMapThreads)
     tile_hist[(size_t)blockIdx.x * E + e] = hist[e];
+  if (threadIdx.x == 0) tile_flags[blockIdx.x] = s_flags;
 }
 
 // ---- scan ------------------------------------------------------------------------------------
 
 constexpr int kScanThreads = 1024;
+// Tile counts a thread keeps in registers between its two passes (enough for 512 tiles, i.e.
+// T <= 32768; longer inputs re-read the rest).
+constexpr int kScanCache = 16;
 
 // Inclusive block-wide scan of one int per thread (1024 threads).
 __device__ __forceinline__ int block_incl_scan(int v, int *warp_tot) {
@@ -187,35 +328,38 @@ __device__ __forceinline__ int block_incl_scan(int v, int *warp_tot) {
 }
 
 // Per-tile exclusive offsets inside each expert, then (in the last CTA to finish) bins,
-// padded_bins, num_blocks and the block -> expert table.  Grid: one CTA per 32 experts; warp c
+// padded_bins, num_blocks and the call's status word.  Grid: one CTA per 32 experts; warp c
 // of a CTA owns tile chunk c (32 chunks), lane l owns expert 32*blockIdx.x + l, so every load
-// of a tile's histogram row is one coalesced 128-byte access.  No CTA waits for another: the
-// CTA that takes the last ticket of `done` (zeroed by the routing kernel) does the final part.
-__global__ void __launch_bounds__(kScanThreads) k_map_scan(int n_tiles, int E, int nblk_cap,
+// of a tile's histogram row is one coalesced access.  No CTA waits for another: the CTA that
+// takes the last ticket of `done` (zeroed by the routing kernel) does the final part.
+__global__ void __launch_bounds__(kScanThreads) k_map_scan(int n_tiles, int E,
                                                            int32_t *__restrict__ tile_hist,
+                                                           const int32_t *__restrict__ tile_flags,
                                                            int32_t *__restrict__ tokens_per_expert,
                                                            int32_t *__restrict__ bins,
                                                            int32_t *__restrict__ padded_bins,
-                                                           int32_t *__restrict__ block_expert,
                                                            int32_t *__restrict__ num_blocks,
+                                                           int32_t *__restrict__ status,
                                                            unsigned int *__restrict__ done) {
   __shared__ int chunk[32][33];
-  __shared__ int s_pb[DMOE_MAX_EXPERTS];
   __shared__ int warp_tot[32];
+  __shared__ int s_flags;
   __shared__ bool is_last;
+  pdl_wait();
+  pdl_trigger();
   const int c = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x * 32 + lane;
   const int tpc = (n_tiles + 31) / 32;
   const int tb = c * tpc, te = min(n_tiles, tb + tpc);
+  int cache[kScanCache];
   int sum = 0;
   if (e < E) {
-    int t = tb;
-    for (; t + 4 <= te; t += 4) {  // independent loads in flight
-      const int v0 = tile_hist[(size_t)t * E + e], v1 = tile_hist[(size_t)(t + 1) * E + e];
-      const int v2 = tile_hist[(size_t)(t + 2) * E + e], v3 = tile_hist[(size_t)(t + 3) * E + e];
-      sum += v0 + v1 + v2 + v3;
+#pragma unroll
+    for (int i = 0; i < kScanCache; ++i) {  // all loads in flight at once
+      cache[i] = (tb + i < te) ? tile_hist[(size_t)(tb + i) * E + e] : 0;
+      sum += cache[i];
     }
-    for (; t < te; ++t) sum += tile_hist[(size_t)t * E + e];
+    for (int t = tb + kScanCache; t < te; ++t) sum += tile_hist[(size_t)t * E + e];
   }
   chunk[c][lane] = sum;
   __syncthreads();
@@ -231,13 +375,18 @@ __global__ void __launch_bounds__(kScanThreads) k_map_scan(int n_tiles, int E, i
   __syncthreads();
   if (e < E) {  // counts -> exclusive offsets inside the expert
     int run = chunk[c][lane];
-    for (int t = tb; t < te; ++t) {
+#pragma unroll
+    for (int i = 0; i < kScanCache; ++i) {
+      if (tb + i < te) tile_hist[(size_t)(tb + i) * E + e] = run;
+      run += cache[i];
+    }
+    for (int t = tb + kScanCache; t < te; ++t) {
       const int v = tile_hist[(size_t)t * E + e];
       tile_hist[(size_t)t * E + e] = run;
       run += v;
     }
   }
-  // ---- last CTA: bins, padded_bins, block table ----
+  // ---- last CTA: bins, padded_bins, num_blocks, status ----
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) is_last = (atomicAdd(done, 1u) == gridDim.x - 1);
@@ -245,24 +394,130 @@ __global__ void __launch_bounds__(kScanThreads) k_map_scan(int n_tiles, int E, i
   if (!is_last) return;
   __threadfence();
   const int tid = threadIdx.x;
+  if (tid == 0) s_flags = 0;
+  int flags = 0;
+  for (int t = tid; t < n_tiles; t += kScanThreads) flags |= tile_flags[t];
   const int cnt = (tid < E) ? *((volatile int32_t *)tokens_per_expert + tid) : 0;
   const int pad = ((cnt + kBlock - 1) / kBlock) * kBlock;
-  const int incl = block_incl_scan(cnt, warp_tot);
+  const int incl = block_incl_scan(cnt, warp_tot);  // (its barriers also order s_flags = 0)
   const int pincl = block_incl_scan(pad, warp_tot);
   if (tid < E) {
     bins[tid] = incl;
     padded_bins[tid] = pincl;
-    s_pb[tid] = pincl;
+  }
+  if (tid == E - 1) *num_blocks = pincl / kBlock;
+  flags = __reduce_or_sync(0xFFFFFFFFu, flags);
+  if (flags && lane == 0) atomicOr(&s_flags, flags);
+  __syncthreads();
+  if (tid == 0) {
+    *status = s_flags;  // the map call's own bits; later calls OR theirs in
+    *done = 0u;         // ready for the next call
+  }
+}
+
+// ---- stable scatter --------------------------------------------------------------------------
+
+// Entries a lane keeps in registers between the scatter's two passes: a tile has at most
+// 64 * DMOE_MAX_TOP_K entries, split over 8 warps in whole 32-entry rounds.
+constexpr int kScatRounds = 8;
+static_assert(kMapTokTile * DMOE_MAX_TOP_K <= kMapWarps * 32 * kScatRounds, "scatter rounds");
+
+// Grid: one CTA per tile.  Stable rank of every entry inside its expert (warp histograms and
+// __match_any_sync ranks in entry order), then indices, bin_ids and dest_row from the index
+// math of section 4.2.  Every CTA also writes a grid-strided slice of the block -> expert table
+// (entry b = the expert whose padded range holds row 128*b, -1 past num_blocks).
+__global__ void __launch_bounds__(kMapThreads) k_map_scatter(int T, int E, int k, int nblk_cap,
+                                                             const int32_t *__restrict__ top,
+                                                             const int32_t *__restrict__ tile_off,
+                                                             const int32_t *__restrict__ bins,
+                                                             const int32_t *__restrict__ padded_bins,
+                                                             int32_t *__restrict__ indices,
+                                                             int32_t *__restrict__ bin_ids,
+                                                             int32_t *__restrict__ dest_row,
+                                                             int32_t *__restrict__ block_expert) {
+  extern __shared__ int sm[];
+  int *wh = sm;                           // [kMapWarps][E] counts, then exclusive offsets
+  int *s_base = wh + kMapWarps * E;       // [E] bins[e-1] + this tile's offset inside e
+  int *s_shift = s_base + E;              // [E] padded_bins[e-1] - bins[e-1]
+  int *s_pb = s_shift + E;                // [E] padded_bins
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long N = (long long)T * k;
+  const long long j0 = (long long)blockIdx.x * kMapTokTile * k;
+  const long long j1 = min(N, j0 + (long long)kMapTokTile * k);
+  const int n = (int)(j1 - j0);
+  const int per_warp = (((n + kMapWarps - 1) / kMapWarps) + 31) & ~31;
+  const long long wb = j0 + (long long)warp * per_warp;
+  const long long we = min(j1, wb + per_warp);
+  // this warp's entries, loaded once (all rounds in flight) and kept for both passes
+  int ev[kScatRounds];
+#pragma unroll
+  for (int r = 0; r < kScatRounds; ++r) {
+    const long long j = wb + 32 * r + lane;
+    int e = -1 - lane;
+    if (j < we) {
+      const int v = top[j];
+      if (v >= 0 && v < E) e = v;
+    }
+    ev[r] = e;
+  }
+  for (int i = threadIdx.x; i < kMapWarps * E; i += kMapThreads) wh[i] = 0;
+  for (int e = threadIdx.x; e < E; e += kMapThreads) {
+    const int bp = (e > 0) ? bins[e - 1] : 0;
+    const int pp = (e > 0) ? padded_bins[e - 1] : 0;
+    s_base[e] = bp + tile_off[(size_t)blockIdx.x * E + e];
+    s_shift[e] = pp - bp;
+    s_pb[e] = padded_bins[e];
   }
   __syncthreads();
-  const int nb = s_pb[E - 1] / kBlock;
-  if (tid == 0) {
-    *num_blocks = nb;
-    *done = 0u;  // ready for the next call
+  int *my = wh + warp * E;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  // pass 1: per-warp histogram of its contiguous entry range
+#pragma unroll
+  for (int r = 0; r < kScatRounds; ++r) {
+    if (wb + 32 * r >= we) break;
+    const int e = ev[r];
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
+    __syncwarp();
   }
-  for (int b = tid; b < nblk_cap; b += kScanThreads) {
+  __syncthreads();
+  // exclusive offsets per (warp, expert): expert start + tile offset + earlier warps
+  for (int e = threadIdx.x; e < E; e += kMapThreads) {
+    int run = s_base[e];
+    for (int w = 0; w < kMapWarps; ++w) {
+      const int v = wh[w * E + e];
+      wh[w * E + e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  // pass 2: sorted position of every entry, in entry order within each expert
+#pragma unroll
+  for (int r = 0; r < kScatRounds; ++r) {
+    if (wb + 32 * r >= we) break;
+    const long long j = wb + 32 * r + lane;
+    const int e = ev[r];
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+    if (e >= 0) {
+      const int i = my[e] + __popc(peers & lt_mask);
+      indices[i] = (int32_t)j;
+      bin_ids[i] = e;
+      dest_row[j] = i + s_shift[e];  // offset_in_bin + padded_bins[e-1]
+    } else if (j < we) {
+      dest_row[j] = -1;
+    }
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
+    __syncwarp();
+  }
+  // block -> expert table slice
+  const int nb = s_pb[E - 1] / kBlock;
+  for (int b = blockIdx.x * kMapThreads + threadIdx.x; b < nblk_cap;
+       b += gridDim.x * kMapThreads) {
     int owner = -1;
-    if (b < nb) {  // smallest e with padded_bins[e] > b*128
+    if (b < nb) {  // smallest e with padded_bins[e] > 128*b
       int lo = 0, hi = E - 1;
       const int row = b * kBlock;
       while (lo < hi) {
@@ -278,93 +533,22 @@ __global__ void __launch_bounds__(kScanThreads) k_map_scan(int n_tiles, int E, i
   }
 }
 
-// ---- stable scatter --------------------------------------------------------------------------
-
-__global__ void __launch_bounds__(kMapThreads) k_map_scatter(int T, int E, int k,
-                                                             const int32_t *__restrict__ top,
-                                                             const int32_t *__restrict__ tile_off,
-                                                             const int32_t *__restrict__ bins,
-                                                             const int32_t *__restrict__ padded_bins,
-                                                             int32_t *__restrict__ indices,
-                                                             int32_t *__restrict__ bin_ids,
-                                                             int32_t *__restrict__ dest_row) {
-  extern __shared__ int wh[];  // [kMapWarps][E]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long N = (long long)T * k;
-  const long long j0 = (long long)blockIdx.x * kMapTokTile * k;
-  const long long j1 = min(N, j0 + (long long)kMapTokTile * k);
-  const int n = (int)(j1 - j0);
-  const int per_warp = (((n + kMapWarps - 1) / kMapWarps) + 31) & ~31;
-  const long long wb = j0 + (long long)warp * per_warp;
-  const long long we = min(j1, wb + per_warp);
-  for (int i = threadIdx.x; i < kMapWarps * E; i += kMapThreads) wh[i] = 0;
-  __syncthreads();
-  int *my = wh + warp * E;
-  const unsigned lt_mask = (1u << lane) - 1u;
-  // pass 1: per-warp histogram of its contiguous entry range
-  for (long long base = wb; base < we; base += 32) {
-    const long long j = base + lane;
-    int e = -1 - lane;
-    if (j < we) {
-      const int v = top[j];
-      if (v >= 0 && v < E) e = v;
-    }
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
-    if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
-    __syncwarp();
-  }
-  __syncthreads();
-  // exclusive offsets per (warp, expert): expert start + tile offset + earlier warps
-  for (int e = threadIdx.x; e < E; e += kMapThreads) {
-    int run = ((e > 0) ? bins[e - 1] : 0) + tile_off[(size_t)blockIdx.x * E + e];
-    for (int w = 0; w < kMapWarps; ++w) {
-      const int v = wh[w * E + e];
-      wh[w * E + e] = run;
-      run += v;
-    }
-  }
-  __syncthreads();
-  // pass 2: sorted position of every entry, in entry order within each expert
-  for (long long base = wb; base < we; base += 32) {
-    const long long j = base + lane;
-    int e = -1 - lane;
-    if (j < we) {
-      const int v = top[j];
-      if (v >= 0 && v < E) e = v;
-    }
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
-    if (e >= 0) {
-      const int i = my[e] + __popc(peers & lt_mask);
-      const int bins_prev = (e > 0) ? bins[e - 1] : 0;
-      const int pbins_prev = (e > 0) ? padded_bins[e - 1] : 0;
-      indices[i] = (int32_t)j;
-      bin_ids[i] = e;
-      dest_row[j] = (i - bins_prev) + pbins_prev;  // offset_in_bin + padded_bins[e-1]
-    } else if (j < we) {
-      dest_row[j] = -1;
-    }
-    __syncwarp();
-    if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
-    __syncwarp();
-  }
-}
-
 // ---- launchers -------------------------------------------------------------------------------
 
 cudaError_t launch_route_hist(const uint16_t *logits, int T, int E, int k, bool renorm, int32_t *top,
-                              float *weights, int32_t *tile_hist, int32_t *status,
-                              cudaStream_t st) {
+                              float *weights, int32_t *tile_hist, cudaStream_t st) {
   const int tiles = map_tiles(T);
   const size_t smem = sizeof(int) * (size_t)E;
   unsigned int *done = map_ticket(tile_hist, T, E);
-  if (!logits) {
-    k_given_hist<<<tiles, kMapThreads, smem, st>>>(top, T, E, k, tile_hist, status, done);
-    return cudaGetLastError();
-  }
-#define DMOE_ROUTE(KPL)                                                                      \
-  k_route_hist<KPL><<<tiles, kMapThreads, smem, st>>>(logits, T, E, k, renorm ? 1 : 0, top,    \
-                                                      weights, tile_hist,                      \
-                                                      status, done)
+  int32_t *flags = map_flags(tile_hist, T, E);
+  if (!logits)
+    return launch_pdl(k_given_hist, tiles, kMapThreads, smem, st, top, T, E, k, tile_hist, flags,
+                      done);
+  // logits per lane: the smallest power of two with E <= 32 * KPL
+  using Kernel = void (*)(const uint16_t *, int, int, int, int, int32_t *, float *, int32_t *,
+                          int32_t *, unsigned int *);
+  Kernel kernel;
+#define DMOE_ROUTE(KPL) kernel = (E % KPL == 0) ? k_route_hist<KPL, true> : k_route_hist<KPL, false>
   if (E <= 32)
     DMOE_ROUTE(1);
   else if (E <= 64)
@@ -378,26 +562,25 @@ cudaError_t launch_route_hist(const uint16_t *logits, int T, int E, int k, bool 
   else
     DMOE_ROUTE(32);
 #undef DMOE_ROUTE
-  return cudaGetLastError();
+  return launch_pdl(kernel, tiles, kRouteThreads, smem, st, logits, T, E, k, renorm ? 1 : 0, top,
+                    weights, tile_hist, flags, done);
 }
 
-cudaError_t launch_map_scan(int T, int E, int nblk_cap, int32_t *tile_hist,
-                            int32_t *tokens_per_expert, int32_t *bins, int32_t *padded_bins,
-                            int32_t *block_expert, int32_t *num_blocks, cudaStream_t st) {
-  k_map_scan<<<(E + 31) / 32, kScanThreads, 0, st>>>(map_tiles(T), E, nblk_cap, tile_hist,
-                                                      tokens_per_expert, bins, padded_bins,
-                                                      block_expert, num_blocks,
-                                                      map_ticket(tile_hist, T, E));
-  return cudaGetLastError();
+cudaError_t launch_map_scan(int T, int E, int32_t *tile_hist, int32_t *tokens_per_expert,
+                            int32_t *bins, int32_t *padded_bins, int32_t *num_blocks,
+                            int32_t *status, cudaStream_t st) {
+  return launch_pdl(k_map_scan, (E + 31) / 32, kScanThreads, 0, st, map_tiles(T), E, tile_hist,
+                    map_flags(tile_hist, T, E), tokens_per_expert, bins, padded_bins, num_blocks,
+                    status, map_ticket(tile_hist, T, E));
 }
 
-cudaError_t launch_map_scatter(int T, int E, int k, const int32_t *top, const int32_t *tile_off,
-                               const int32_t *bins, const int32_t *padded_bins, int32_t *indices,
-                               int32_t *bin_ids, int32_t *dest_row, cudaStream_t st) {
-  const size_t smem = sizeof(int) * (size_t)kMapWarps * E;
-  k_map_scatter<<<map_tiles(T), kMapThreads, smem, st>>>(T, E, k, top, tile_off, bins,
-                                                         padded_bins, indices, bin_ids, dest_row);
-  return cudaGetLastError();
+cudaError_t launch_map_scatter(int T, int E, int k, int nblk_cap, const int32_t *top,
+                               const int32_t *tile_off, const int32_t *bins,
+                               const int32_t *padded_bins, int32_t *indices, int32_t *bin_ids,
+                               int32_t *dest_row, int32_t *block_expert, cudaStream_t st) {
+  const size_t smem = sizeof(int) * (size_t)(kMapWarps + 3) * E;
+  return launch_pdl(k_map_scatter, map_tiles(T), kMapThreads, smem, st, T, E, k, nblk_cap, top,
+                    tile_off, bins, padded_bins, indices, bin_ids, dest_row, block_expert);
 }
 
 }  // namespace dmoe

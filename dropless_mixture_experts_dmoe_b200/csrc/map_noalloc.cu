@@ -20,8 +20,9 @@
 
 namespace {
 
-// Capacity of the static scratch in int32 words: the per-tile histograms (ceil(T/64) * E) plus
-// one counter must fit (1 MiB; e.g. T <= 65472 tokens at E = 256, T <= 16320 at E = 1024).
+// Capacity of the static scratch in int32 words: the per-tile histograms (ceil(T/64) * E), one
+// counter and one status word per tile must fit (1 MiB; e.g. T <= 65280 tokens at E = 256,
+// T <= 16320 at E = 1024).
 constexpr size_t kNoAllocScratchInts = DMOE_NOALLOC_SCRATCH_BYTES / sizeof(int32_t);
 
 static __device__ __align__(256) int32_t g_map_scratch[kNoAllocScratchInts];
@@ -81,20 +82,17 @@ extern "C" int dmoe_sparse_map_noalloc(const dmoe_dims *dims, const void *logits
   const long long n = (long long)T * k;
   const int nblk_cap =
       (int)((n + (long long)(DMOE_BLOCKING - 1) * E) / DMOE_BLOCKING);
-  // The histogram kernel writes every (tile, expert) entry of the scratch it later reads and
-  // zeroes the counter after them, so nothing left over from an earlier call is ever read;
-  // the status word is cleared here.
-  if (cudaMemsetAsync(map->status, 0, sizeof(int32_t), st) != cudaSuccess) return DMOE_ERR_LAUNCH;
+  // The histogram kernel writes every (tile, expert) entry and every tile status word of the
+  // scratch it later reads and zeroes the counter after them, so nothing left over from an
+  // earlier call is ever read; the scan kernel stores the call's status word.
   const bool renorm = (dims->route_flags & DMOE_ROUTE_RENORMALIZE) != 0;
   if ((rc = rc_of(dmoe::launch_route_hist(static_cast<const uint16_t *>(logits), T, E, k, renorm,
-                                          map->top_experts, map->weights, scratch, map->status,
-                                          st))))
+                                          map->top_experts, map->weights, scratch, st))))
     return rc;
-  if ((rc = rc_of(dmoe::launch_map_scan(T, E, nblk_cap, scratch, map->tokens_per_expert, map->bins,
-                                        map->padded_bins, map->block_expert, map->num_blocks,
-                                        st))))
+  if ((rc = rc_of(dmoe::launch_map_scan(T, E, scratch, map->tokens_per_expert, map->bins,
+                                        map->padded_bins, map->num_blocks, map->status, st))))
     return rc;
-  return rc_of(dmoe::launch_map_scatter(T, E, k, map->top_experts, scratch, map->bins,
+  return rc_of(dmoe::launch_map_scatter(T, E, k, nblk_cap, map->top_experts, scratch, map->bins,
                                         map->padded_bins, map->indices, map->bin_ids,
-                                        map->dest_row, st));
+                                        map->dest_row, map->block_expert, st));
 }

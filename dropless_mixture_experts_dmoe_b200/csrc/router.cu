@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(kRouterThreads)
     k_router_dlogits(int T, int E, int k, int renorm, const uint16_t *__restrict__ logits,
                      const int32_t *__restrict__ top, const float *__restrict__ dweights,
                      uint16_t *__restrict__ dlogits) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int groups = E >> 3;
   const long long nw = (long long)gridDim.x * kRouterWarps;
@@ -129,6 +131,8 @@ __global__ void __launch_bounds__(kRouterThreads)
 __global__ void __launch_bounds__(kRouterThreads)
     k_router_wgrad_reduce(int h, int E, int Ep, int splits, const float4 *__restrict__ partials,
                           float4 *__restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   const int hv = h >> 2;
   const long long n = (long long)E * hv;
   const size_t slab = (size_t)Ep * hv;
@@ -157,27 +161,19 @@ cudaError_t launch_router_dlogits(int T, int E, int k, bool renorm, const uint16
                                   const int32_t *top, const float *dweights, uint16_t *dlogits,
                                   cudaStream_t st) {
   const int grid = grid_for(T, kRouterWarps);
-#define DMOE_DLOGITS(GPL) \
-  k_router_dlogits<GPL><<<grid, kRouterThreads, 0, st>>>(T, E, k, renorm ? 1 : 0, logits, top, \
-                                                         dweights, dlogits)
-  if (E <= 256)
-    DMOE_DLOGITS(1);
-  else if (E <= 512)
-    DMOE_DLOGITS(2);
-  else
-    DMOE_DLOGITS(4);
-#undef DMOE_DLOGITS
-  return cudaGetLastError();
+  auto kernel = (E <= 256) ? k_router_dlogits<1> : (E <= 512) ? k_router_dlogits<2>
+                                                              : k_router_dlogits<4>;
+  return launch_pdl(kernel, grid, kRouterThreads, 0, st, T, E, k, renorm ? 1 : 0, logits, top,
+                    dweights, dlogits);
 }
 
 cudaError_t launch_router_wgrad_reduce(int h, int E, int splits, const float *partials,
                                        float *dw_router, cudaStream_t st) {
   const int Ep = (E + kBlock - 1) / kBlock * kBlock;
   const long long n = (long long)E * (h >> 2);
-  k_router_wgrad_reduce<<<grid_for(n, kRouterThreads), kRouterThreads, 0, st>>>(
-      h, E, Ep, splits, reinterpret_cast<const float4 *>(partials),
-      reinterpret_cast<float4 *>(dw_router));
-  return cudaGetLastError();
+  return launch_pdl(k_router_wgrad_reduce, grid_for(n, kRouterThreads), kRouterThreads, 0, st, h,
+                    E, Ep, splits, reinterpret_cast<const float4 *>(partials),
+                    reinterpret_cast<float4 *>(dw_router));
 }
 
 }  // namespace dmoe

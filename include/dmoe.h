@@ -114,7 +114,7 @@ typedef struct {
  *                              i its sorted position, e its expert, bins[-1] = 0
  *   block_expert [P_max/128]   expert owning 128-row block b; -1 for b >= num_blocks
  *   num_blocks [1]             padded_bins[E-1] / 128
- *   status [1]                 device status bits; dmoe_sparse_map clears it first          */
+ *   status [1]                 device status bits; dmoe_sparse_map overwrites it with its own */
 typedef struct {
   int32_t *top_experts;
   float *weights;
@@ -160,11 +160,12 @@ DMOE_API size_t dmoe_saved_bytes(const dmoe_dims *dims, size_t offsets[3]);
  *   logits: [T, E] bf16 device pointer, or NULL to take map->top_experts as given (then
  *           map->weights is not written; out-of-range or duplicate experts set status bits
  *           and such entries are dropped from the map).
- *   map:    caller-owned outputs (see dmoe_map); map->status is cleared, then OR-ed.
+ *   map:    caller-owned outputs (see dmoe_map); map->status is overwritten with the map's
+ *           own bits (later calls OR theirs in).
  *   ws:     workspace of dmoe_workspace_bytes(dims, DMOE_WS_MAP) bytes.
  * Shared memory per CTA is O(E) and independent of T (the issue's kernel needed 262144 B
- * at E = 64, top-8, 2 x 2048 tokens).  Three kernels, no atomics on global memory, no
- * host sync; results are deterministic. */
+ * at E = 64, top-8, 2 x 2048 tokens).  Three kernels, no global atomics but one completion
+ * ticket, no host sync; results are deterministic. */
 DMOE_API int dmoe_sparse_map(const dmoe_dims *dims, const void *logits, const dmoe_map *map, void *ws,
                     size_t ws_bytes, void *stream);
 
@@ -206,8 +207,8 @@ DMOE_API int dmoe_backward(const dmoe_dims *dims, const void *dy, const void *w1
  *   Same arguments, results and status bits as dmoe_sparse_map, without ws / ws_bytes.
  *   Scratch: a static array of DMOE_NOALLOC_SCRATCH_BYTES in device global memory inside
  *     libdmoe.so; every GPU that loads the library holds it until the process exits.  The
- *     call needs (ceil(T/64) * num_experts + 1) * 4 bytes of it and returns
- *     DMOE_ERR_WORKSPACE, before any launch, when that exceeds the limit (e.g. T > 65472 at
+ *     call needs (ceil(T/64) * (num_experts + 1) + 1) * 4 bytes of it and returns
+ *     DMOE_ERR_WORKSPACE, before any launch, when that exceeds the limit (e.g. T > 65280 at
  *     E = 256).
  *   The call performs no allocation (no cudaMalloc, no cudaFree, no allocating library
  *     routine).  Its first call on a device looks up the array's device address with

@@ -48,6 +48,16 @@ def test_map_parity_real_inputs_tiny():
     (4097, 32, 32, "few_values"),  # maximum k
     (1, 8, 2, "continuous"),       # single token
     (8192, 64, 8, "continuous"),   # the issue's failing shape with 4096-long sequences
+    # logits layouts of the routing kernel: vector rows when E is a multiple of the logits per
+    # lane, strided lanes otherwise; sorted per-lane candidates up to 8 per lane
+    (7, 7, 3, "few_values"),        # 1 per lane, a partial tile
+    (1000, 33, 4, "continuous"),    # 2 per lane, strided
+    (1000, 100, 8, "few_values"),   # 4 per lane, vector, ties
+    (1500, 250, 8, "continuous"),   # 8 per lane, strided
+    (300, 256, 32, "few_values"),   # 8 per lane, vector, 32 picks drain whole lanes
+    (600, 384, 8, "few_values"),    # 16 per lane, vector, unsorted rounds
+    (700, 1000, 8, "continuous"),   # 32 per lane, strided
+    (40000, 16, 4, "continuous"),   # 625 tiles: the scan re-reads past its register cache
 ])
 def test_map_parity_edge_cases(T, E, k, kind):
     g = torch.Generator().manual_seed(T * 7 + E)
@@ -112,6 +122,21 @@ def test_map_nonfinite_logits_flagged():
     dims = B.make_dims(64, 128, 128, 8, 2)
     _, g = gpu_map(dims, logits.to(torch.bfloat16))
     assert g["status"] & B.STATUS_NONFINITE_LOGITS
+
+
+def test_map_status_is_the_calls_own():
+    """The map call's status word holds its own bits: a flag left by an earlier call, or
+    garbage put there by the caller, does not survive a clean call."""
+    dims = B.make_dims(64, 128, 128, 8, 2)
+    bad = torch.randn(64, 8)
+    bad[3, 2] = float("nan")
+    bufs, g = gpu_map(dims, bad.to(torch.bfloat16))
+    assert g["status"] == B.STATUS_NONFINITE_LOGITS
+    _, g = gpu_map(dims, torch.randn(64, 8).to(torch.bfloat16), bufs=bufs)
+    assert g["status"] == 0
+    bufs.map.status.fill_(0x1234)
+    _, g = gpu_map(dims, torch.randn(64, 8).to(torch.bfloat16), bufs=bufs)
+    assert g["status"] == 0
 
 
 def test_map_deterministic_repeat():
