@@ -52,7 +52,17 @@ def _forward_backward(w, route_flags=0):
     return inp, dims, dev, bufs, logits, g, dx_experts, dwr, ws
 
 
-@pytest.mark.parametrize("w", SMALL + [custom(4096, 2048, 512, 256, 8)], ids=lambda w: w.describe())
+THIN = [  # thin routers (E <= 32): logits GEMMs whose 256-column tile is mostly padding
+    custom(4096, 4096, 128, 8, 2),    # the Mixtral-shaped router (its ffn plays no part; sampled rows)
+    custom(1000, 128, 128, 16, 4),
+    custom(333, 640, 128, 24, 4),     # 24 of 32 expert slots, a partial last token group
+    custom(77, 8192, 128, 32, 8),     # two column passes per lane
+    custom(3, 384, 128, 8, 2),        # fewer tokens than one group
+]
+
+
+@pytest.mark.parametrize("w", SMALL + THIN + [custom(4096, 2048, 512, 256, 8)],
+                         ids=lambda w: w.describe())
 def test_router_logits_parity(w):
     inp = make_inputs(w, with_router=True)
     dims = dims_of(w)
