@@ -55,9 +55,9 @@ def _forward_backward(w, route_flags=0):
 THIN = [  # thin routers (E <= 32): logits GEMMs whose 256-column tile is mostly padding
     custom(4096, 4096, 128, 8, 2),    # the Mixtral-shaped router (its ffn plays no part; sampled rows)
     custom(1000, 128, 128, 16, 4),
-    custom(333, 640, 128, 24, 4),     # 24 of 32 expert slots, a partial last token group
-    custom(77, 8192, 128, 32, 8),     # two column passes per lane
-    custom(3, 384, 128, 8, 2),        # fewer tokens than one group
+    custom(333, 640, 128, 24, 4),     # E not a power of two, a ragged last row tile
+    custom(77, 8192, 128, 32, 8),     # long K (128 steps of 64), one partial row tile
+    custom(3, 384, 128, 8, 2),        # three tokens: a tile of almost only zero-filled rows
 ]
 
 
