@@ -1,7 +1,8 @@
 """dMoE expert layer for NVIDIA B200 (sm_100a): routing, sparse map, padded gather, grouped
 tcgen05 gated-SiLU expert GEMMs, weighted combine and backward, behind the C ABI of
 ``libdmoe.so`` (include/dmoe.h).  ``binding`` is the thin ctypes layer over it."""
-from . import binding  # noqa: F401
+from . import autograd, binding  # noqa: F401
+from .autograd import DMoEFunction, dmoe  # noqa: F401
 from .binding import (Buffers, DMoEError, SparseMap, dmoe_backward, dmoe_bwd_dglu,  # noqa: F401
                       dmoe_bwd_dx, dmoe_bwd_scatter, dmoe_bwd_wgrad, dmoe_expert_down,
                       dmoe_expert_glu, dmoe_expert_glu_gather, dmoe_forward, dmoe_padded_gather, dmoe_padded_rows_max,
