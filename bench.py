@@ -49,6 +49,9 @@ def parse():
     p.add_argument("--router", action="store_true",
                    help="compute the logits with the linear router (x W_r^T) inside the step and, "
                         "for fwd+bwd workloads, run the router backward after the layer's")
+    p.add_argument("--map-only", action="store_true",
+                   help="time dmoe_sparse_map alone (routing + sparse map) on the workload's "
+                        "logits: a supplementary line, not the layer's")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample", type=int, default=0, help="tokens in the oracle sample")
     return p.parse_args()
@@ -580,6 +583,69 @@ def run_ours(args, w):
         dist.destroy_process_group()
 
 
+def run_map_only(args, w):
+    """Routing + sparse map alone: K timed calls of dmoe_sparse_map on the workload's logits
+    (larger than L2 at the sizes this is meant for), one JSON line on rank 0 (single GPU)."""
+    import torch
+
+    from dropless_mixture_experts_dmoe_b200 import binding as B
+    from dropless_mixture_experts_dmoe_b200 import build as build_mod
+    from dropless_mixture_experts_dmoe_b200.workloads import make_tensor
+
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    if int(os.environ.get("RANK", "0")) == 0:
+        build_mod.build()
+    B.load()
+    dims = B.make_dims(w.T, w.hidden, w.ffn, w.E, w.top_k)
+    logits = make_tensor(w, "logits").cuda()
+    smap = B.SparseMap(dims)
+    ws = torch.empty(max(B.dmoe_workspace_bytes(dims, B.WS_MAP), 16), dtype=torch.uint8,
+                     device="cuda")
+    st = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        B.dmoe_sparse_map(dims, logits, smap, ws, st)
+    torch.cuda.synchronize()
+    if int(smap.status.item()):
+        raise RuntimeError(f"device status: {B.status_string(int(smap.status.item()))}")
+    sampler = ClockSampler(torch.cuda.current_device())
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    wall0 = time.time()
+    e0.record(st)
+    for _ in range(args.steps):
+        B.dmoe_sparse_map(dims, logits, smap, ws, st)
+    e1.record(st)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    clocks = sampler.stop(wall0, wall1)
+    ms = e0.elapsed_time(e1) / args.steps
+    N = w.T * w.top_k
+    nb = int(smap.num_blocks.item())
+    # logits read, top_experts + weights written, indices + bin_ids + dest_row written, the
+    # per-expert arrays and the block table (P_max / 128 entries)
+    byts = 2 * w.T * w.E + 8 * w.T * w.top_k + 12 * N + 16 * w.E + \
+        4 * (B.dmoe_padded_rows_max(dims) // 128)
+    pk = peaks()
+    line = {
+        "metric": "routing + sparse map tokens/s (supplementary; the map alone)",
+        "value": w.T / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"map only: T={w.T} E={w.E} top_k={w.top_k}"
+                               f"{' zipf' if w.zipf_bias else ''}",
+                   "l2": "logits %s L2 (%.0f MB)" % ("larger than" if 2 * w.T * w.E > L2_BYTES
+                                                      else "within", 2 * w.T * w.E / 1e6),
+                   "parallelism": "single GPU"},
+        "map": {"ms": ms, "algorithmic_bytes": byts, "GB/s": byts / ms / 1e6,
+                "frac_hbm": byts / ms / 1e6 / pk["hbm"], "num_blocks": nb},
+        "gpu_launches": 3 * args.steps,
+        "status": int(smap.status.item()),
+    }
+    if clocks:
+        line["clocks"] = clocks
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     from dropless_mixture_experts_dmoe_b200.workloads import WORKLOADS
@@ -592,7 +658,13 @@ def main():
         T, h, f, E, k = (int(v) for v in parts[:5])
         w = custom(T, h, f, E, k, number=100, name="custom", backward="bwd" in parts[5:],
                    zipf_bias="zipf" in parts[5:])
-    if args.impl == "reference":
+    if args.map_only:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "--map-only times the GPU "
+                              "map alone; the reference arm times the whole layer"}))
+        else:
+            run_map_only(args, w)
+    elif args.impl == "reference":
         run_reference(args, w)
     else:
         run_ours(args, w)

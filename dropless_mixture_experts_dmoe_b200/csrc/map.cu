@@ -38,14 +38,16 @@ __device__ __forceinline__ float exp_diff(float v, float m) {
 
 // Selection key of a logit given as its fp32 image u (a bf16 value in the high half): the high
 // half is the order-preserving image (negative -> bits inverted, else sign bit set; -0 taken as
-// +0; NaN -> 0, below -inf), the low half is `low` = 0xFFFF - expert, so among equal logits the
-// lower expert has the larger key.
+// +0), the low half is `low` = 0xFFFF - expert, so among equal logits the lower expert has the
+// larger key.  Exact for every value but NaN; route_key_nan also maps NaN to 0 (below -inf).
 __device__ __forceinline__ uint32_t route_key(uint32_t u, uint32_t low) {
   const float f = __fadd_rn(__uint_as_float(u), 0.0f);  // -0 + 0 = +0
   const uint32_t z = __float_as_uint(f);
   const uint32_t neg = (uint32_t)((int32_t)z >> 31);
-  const uint32_t key = (z ^ (neg & 0x7FFF0000u)) ^ (0x80000000u | low);
-  return ((z & 0x7FFFFFFFu) > 0x7F800000u) ? low : key;
+  return (z ^ (neg & 0x7FFF0000u)) ^ (0x80000000u | low);
+}
+__device__ __forceinline__ uint32_t route_key_nan(uint32_t u, uint32_t low) {
+  return ((u & 0x7FFFFFFFu) > 0x7F800000u) ? low : route_key(u, low);
 }
 
 // ---- routing + histogram ---------------------------------------------------------------------
@@ -162,6 +164,8 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__
   for (int e = threadIdx.x; e < E; e += kRouteThreads) hist[e] = 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * kMapTokTile + warp;
+  // expert KPL*lane + i of the vector layout exists iff the lane's first one does (E % KPL == 0)
+  const bool lane_ok = KPL * lane < E;
   Row rows[kInFlight];
 #pragma unroll
   for (int j = 0; j < kInFlight; ++j) {
@@ -181,21 +185,28 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__
       cur.load(logits + (size_t)t * E, E, lane);
     }
     uint32_t key[KPL];
+    bool nonfinite = false;
 #pragma unroll
     for (int i = 0; i < KPL; ++i) {
       const int e = Row::expert(lane, i);
+      const bool ok = VEC ? lane_ok : (e < E);
       const uint32_t u = cur.image(i);
-      key[i] = 0u;
-      if (e < E) {
-        bad |= (u & 0x7F800000u) == 0x7F800000u;
-        key[i] = route_key(u, 0xFFFFu - (uint32_t)e);
+      nonfinite |= ok && (u & 0x7F800000u) == 0x7F800000u;
+      key[i] = ok ? route_key(u, 0xFFFFu - (uint32_t)e) : 0u;
+    }
+    if (__any_sync(0xFFFFFFFFu, nonfinite)) {  // rare: rebuild with NaN ranked lowest
+      bad = true;
+#pragma unroll
+      for (int i = 0; i < KPL; ++i) {
+        const int e = Row::expert(lane, i);
+        const bool ok = VEC ? lane_ok : (e < E);
+        key[i] = ok ? route_key_nan(cur.image(i), 0xFFFFu - (uint32_t)e) : 0u;
       }
     }
     if constexpr (kSorted) sort_desc<KPL>(key);
     // k rounds of a warp-wide integer max; keys are unique, so exactly one lane holds the
     // winner, and a valid key is never 0 (its low half is >= 0xFFFF - 1023).
-    int my_e = 0;
-    uint32_t my_key = 0, top_key = 0;
+    uint32_t my_key = 0;  // lane s < k: the key of pick s
     for (int s = 0; s < k; ++s) {
       uint32_t best = 0;
       if constexpr (kSorted) {
@@ -205,11 +216,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__
         for (int i = 0; i < KPL; ++i) best = max(best, key[i]);
       }
       const uint32_t wb = __reduce_max_sync(0xFFFFFFFFu, best);
-      if (s == 0) top_key = wb;
-      if (lane == s) {
-        my_e = 0xFFFF - (int)(wb & 0xFFFFu);
-        my_key = wb;
-      }
+      my_key = (lane == s) ? wb : my_key;
       if constexpr (kSorted) {
         if (key[0] == wb) {
 #pragma unroll
@@ -222,6 +229,8 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__
           if (key[i] == wb) key[i] = 0u;
       }
     }
+    const uint32_t top_key = __shfl_sync(0xFFFFFFFFu, my_key, 0);
+    const int my_e = 0xFFFF - (int)(my_key & 0xFFFFu);
     // softmax over all E logits (or, renormalised, over the k picks), max = the first pick.
     const float m = ((top_key >> 16) == 0u) ? __uint_as_float(0x7FC00000u)
                                            : bf16_from_order(top_key >> 16);
@@ -235,7 +244,8 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__
     } else {
 #pragma unroll
       for (int i = 0; i < KPL; ++i)
-        if (Row::expert(lane, i) < E) sum += exp_diff(__uint_as_float(cur.image(i)), m);
+        if (VEC ? lane_ok : (Row::expert(lane, i) < E))
+          sum += exp_diff(__uint_as_float(cur.image(i)), m);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
@@ -245,7 +255,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__
       atomicAdd(&hist[my_e], 1);
     }
   }
-  if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) atomicOr(&s_flags, DMOE_STATUS_NONFINITE_LOGITS);
+  if (bad && lane == 0) atomicOr(&s_flags, DMOE_STATUS_NONFINITE_LOGITS);  // warp-uniform
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += kRouteThreads)
     tile_hist[(size_t)blockIdx.x * E + e] = hist[e];
@@ -301,6 +311,7 @@ constexpr int kScanThreads = 1024;
 // Tile counts a thread keeps in registers between its two passes (enough for 512 tiles, i.e.
 // T <= 32768; longer inputs re-read the rest).
 constexpr int kScanCache = 16;
+constexpr int kScanBatch = 8;  // loads in flight per thread past the cache
 
 // Inclusive block-wide scan of one int per thread (1024 threads).
 __device__ __forceinline__ int block_incl_scan(int v, int *warp_tot) {
@@ -359,7 +370,14 @@ __global__ void __launch_bounds__(kScanThreads) k_map_scan(int n_tiles, int E,
       cache[i] = (tb + i < te) ? tile_hist[(size_t)(tb + i) * E + e] : 0;
       sum += cache[i];
     }
-    for (int t = tb + kScanCache; t < te; ++t) sum += tile_hist[(size_t)t * E + e];
+    for (int t0 = tb + kScanCache; t0 < te; t0 += kScanBatch) {  // longer inputs: in batches
+      int v[kScanBatch];
+#pragma unroll
+      for (int i = 0; i < kScanBatch; ++i)
+        v[i] = (t0 + i < te) ? tile_hist[(size_t)(t0 + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < kScanBatch; ++i) sum += v[i];
+    }
   }
   chunk[c][lane] = sum;
   __syncthreads();
@@ -380,10 +398,16 @@ __global__ void __launch_bounds__(kScanThreads) k_map_scan(int n_tiles, int E,
       if (tb + i < te) tile_hist[(size_t)(tb + i) * E + e] = run;
       run += cache[i];
     }
-    for (int t = tb + kScanCache; t < te; ++t) {
-      const int v = tile_hist[(size_t)t * E + e];
-      tile_hist[(size_t)t * E + e] = run;
-      run += v;
+    for (int t0 = tb + kScanCache; t0 < te; t0 += kScanBatch) {
+      int v[kScanBatch];
+#pragma unroll
+      for (int i = 0; i < kScanBatch; ++i)
+        v[i] = (t0 + i < te) ? tile_hist[(size_t)(t0 + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < kScanBatch; ++i) {
+        if (t0 + i < te) tile_hist[(size_t)(t0 + i) * E + e] = run;
+        run += v[i];
+      }
     }
   }
   // ---- last CTA: bins, padded_bins, num_blocks, status ----
