@@ -77,20 +77,6 @@ __device__ __forceinline__ void set_status(int32_t *status, int bits) {
 
 // ---- bf16 -------------------------------------------------------------------------------
 
-// Order-preserving 16-bit image of a bf16 value, used to select experts with integer max:
-// larger float -> larger image; +0 and -0 map to the same image; NaN maps to 0, below -inf.
-__device__ __forceinline__ uint32_t bf16_order(uint16_t bits) {
-  if (bits == 0x8000u) bits = 0;                 // -0 -> +0
-  if ((bits & 0x7FFFu) > 0x7F80u) return 0u;     // NaN: lowest
-  return (bits & 0x8000u) ? (~bits & 0xFFFFu) : (bits | 0x8000u);
-}
-
-// Inverse of bf16_order for non-NaN images.
-__device__ __forceinline__ float bf16_from_order(uint32_t ord) {
-  uint16_t bits = (ord & 0x8000u) ? (uint16_t)(ord & 0x7FFFu) : (uint16_t)(~ord & 0xFFFFu);
-  return __uint_as_float((uint32_t)bits << 16);
-}
-
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 

@@ -50,6 +50,13 @@ __device__ __forceinline__ uint32_t route_key_nan(uint32_t u, uint32_t low) {
   return ((u & 0x7FFFFFFFu) > 0x7F800000u) ? low : route_key(u, low);
 }
 
+// The bf16 value whose order-preserving image (the high half of a route key) is `ord`, for
+// any image but that of NaN.
+__device__ __forceinline__ float bf16_from_order(uint32_t ord) {
+  const uint32_t bits = (ord & 0x8000u) ? (ord & 0x7FFFu) : (~ord & 0xFFFFu);
+  return __uint_as_float(bits << 16);
+}
+
 // ---- routing + histogram ---------------------------------------------------------------------
 
 // The routing kernel runs 16 warps per 64-token tile, 4 tokens per warp, so that each warp has
