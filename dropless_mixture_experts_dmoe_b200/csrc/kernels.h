@@ -12,16 +12,24 @@ constexpr int kMapTokTile = 64;
 
 inline int map_tiles(int T) { return (T + kMapTokTile - 1) / kMapTokTile; }
 
-// Map workspace: per-tile histograms [map_tiles(T), E] int32, one ticket counter, then one
-// status word per tile.
+// The scan covers the tiles in segments of kScanSeg (32 warps x kScanCache tiles in registers).
+constexpr int kScanCache = 16;
+constexpr int kScanSeg = 32 * kScanCache;
+inline int map_segments(int T) { return (map_tiles(T) + kScanSeg - 1) / kScanSeg; }
+
+// Map workspace: per-tile histograms [map_tiles(T), E] int32, one ticket counter, one status
+// word per tile, then the per-segment expert totals (later prefixes) [map_segments(T), E].
 inline size_t map_workspace_ints(int T, int E) {
-  return (size_t)map_tiles(T) * E + 1 + (size_t)map_tiles(T);
+  return (size_t)map_tiles(T) * E + 1 + (size_t)map_tiles(T) + (size_t)map_segments(T) * E;
 }
 inline unsigned int *map_ticket(int32_t *tile_hist, int T, int E) {
   return reinterpret_cast<unsigned int *>(tile_hist + (size_t)map_tiles(T) * E);
 }
 inline int32_t *map_flags(int32_t *tile_hist, int T, int E) {
   return tile_hist + (size_t)map_tiles(T) * E + 1;
+}
+inline int32_t *map_segs(int32_t *tile_hist, int T, int E) {
+  return tile_hist + (size_t)map_tiles(T) * E + 1 + (size_t)map_tiles(T);
 }
 
 // Map: routing + per-tile histogram (logits given) or histogram of given top_experts.

@@ -315,10 +315,7 @@ __global__ void __launch_bounds__(kMapThreads) k_given_hist(const int32_t *__res
 // ---- scan ------------------------------------------------------------------------------------
 
 constexpr int kScanThreads = 1024;
-// Tile counts a thread keeps in registers between its two passes (enough for 512 tiles, i.e.
-// T <= 32768; longer inputs re-read the rest).
-constexpr int kScanCache = 16;
-constexpr int kScanBatch = 8;  // loads in flight per thread past the cache
+static_assert(kScanSeg == 32 * kScanCache, "a scan CTA holds its segment in registers");
 
 // Inclusive block-wide scan of one int per thread (1024 threads).
 __device__ __forceinline__ int block_incl_scan(int v, int *warp_tot) {
@@ -345,14 +342,19 @@ __device__ __forceinline__ int block_incl_scan(int v, int *warp_tot) {
   return v;
 }
 
-// Per-tile exclusive offsets inside each expert, then (in the last CTA to finish) bins,
-// padded_bins, num_blocks and the call's status word.  Grid: one CTA per 32 experts; warp c
-// of a CTA owns tile chunk c (32 chunks), lane l owns expert 32*blockIdx.x + l, so every load
-// of a tile's histogram row is one coalesced access.  No CTA waits for another: the CTA that
-// takes the last ticket of `done` (zeroed by the routing kernel) does the final part.
-__global__ void __launch_bounds__(kScanThreads) k_map_scan(int n_tiles, int E,
+// Two-level scan of the per-tile histograms.  Grid (ceil(E/32), S): CTA (x, y) covers experts
+// 32x .. 32x+31 over the y-th segment of kScanSeg tiles; warp c of it owns kScanCache
+// consecutive tiles of the segment, lane l owns expert 32x + l, so every load of a tile's
+// histogram row is one coalesced access and all of a thread's loads are in flight at once.
+// It rewrites each count as the tile's exclusive offset inside its expert and segment and
+// writes the segment's total per expert to seg_sum[y][e].  The CTA that takes the last ticket
+// of `done` (zeroed by the routing kernel; no CTA waits for another) turns seg_sum into
+// exclusive prefixes over segments and computes tokens_per_expert, bins, padded_bins,
+// num_blocks and the call's status word.
+__global__ void __launch_bounds__(kScanThreads, 1) k_map_scan(int n_tiles, int E,
                                                            int32_t *__restrict__ tile_hist,
                                                            const int32_t *__restrict__ tile_flags,
+                                                           int32_t *__restrict__ seg_sum,
                                                            int32_t *__restrict__ tokens_per_expert,
                                                            int32_t *__restrict__ bins,
                                                            int32_t *__restrict__ padded_bins,
@@ -367,23 +369,16 @@ __global__ void __launch_bounds__(kScanThreads) k_map_scan(int n_tiles, int E,
   pdl_trigger();
   const int c = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x * 32 + lane;
-  const int tpc = (n_tiles + 31) / 32;
-  const int tb = c * tpc, te = min(n_tiles, tb + tpc);
+  const int seg = blockIdx.y;
+  const int tb = seg * kScanSeg + c * kScanCache;
+  const int te = min(n_tiles, tb + kScanCache);
   int cache[kScanCache];
   int sum = 0;
   if (e < E) {
 #pragma unroll
-    for (int i = 0; i < kScanCache; ++i) {  // all loads in flight at once
+    for (int i = 0; i < kScanCache; ++i) {
       cache[i] = (tb + i < te) ? tile_hist[(size_t)(tb + i) * E + e] : 0;
       sum += cache[i];
-    }
-    for (int t0 = tb + kScanCache; t0 < te; t0 += kScanBatch) {  // longer inputs: in batches
-      int v[kScanBatch];
-#pragma unroll
-      for (int i = 0; i < kScanBatch; ++i)
-        v[i] = (t0 + i < te) ? tile_hist[(size_t)(t0 + i) * E + e] : 0;
-#pragma unroll
-      for (int i = 0; i < kScanBatch; ++i) sum += v[i];
     }
   }
   chunk[c][lane] = sum;
@@ -395,32 +390,21 @@ __global__ void __launch_bounds__(kScanThreads) k_map_scan(int n_tiles, int E,
       chunk[cc][lane] = run;
       run += v;
     }
-    if (e < E) tokens_per_expert[e] = run;
+    if (e < E) seg_sum[(size_t)seg * E + e] = run;
   }
   __syncthreads();
-  if (e < E) {  // counts -> exclusive offsets inside the expert
+  if (e < E) {  // counts -> exclusive offsets inside the expert and segment
     int run = chunk[c][lane];
 #pragma unroll
     for (int i = 0; i < kScanCache; ++i) {
       if (tb + i < te) tile_hist[(size_t)(tb + i) * E + e] = run;
       run += cache[i];
     }
-    for (int t0 = tb + kScanCache; t0 < te; t0 += kScanBatch) {
-      int v[kScanBatch];
-#pragma unroll
-      for (int i = 0; i < kScanBatch; ++i)
-        v[i] = (t0 + i < te) ? tile_hist[(size_t)(t0 + i) * E + e] : 0;
-#pragma unroll
-      for (int i = 0; i < kScanBatch; ++i) {
-        if (t0 + i < te) tile_hist[(size_t)(t0 + i) * E + e] = run;
-        run += v[i];
-      }
-    }
   }
-  // ---- last CTA: bins, padded_bins, num_blocks, status ----
+  // ---- last CTA: segment prefixes, bins, padded_bins, num_blocks, status ----
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) is_last = (atomicAdd(done, 1u) == gridDim.x - 1);
+  if (threadIdx.x == 0) is_last = (atomicAdd(done, 1u) == gridDim.x * gridDim.y - 1);
   __syncthreads();
   if (!is_last) return;
   __threadfence();
@@ -428,7 +412,16 @@ __global__ void __launch_bounds__(kScanThreads) k_map_scan(int n_tiles, int E,
   if (tid == 0) s_flags = 0;
   int flags = 0;
   for (int t = tid; t < n_tiles; t += kScanThreads) flags |= tile_flags[t];
-  const int cnt = (tid < E) ? *((volatile int32_t *)tokens_per_expert + tid) : 0;
+  int cnt = 0;
+  if (tid < E) {
+    volatile int32_t *ss = seg_sum;
+    for (int y = 0; y < (int)gridDim.y; ++y) {
+      const int v = ss[(size_t)y * E + tid];
+      ss[(size_t)y * E + tid] = cnt;
+      cnt += v;
+    }
+    tokens_per_expert[tid] = cnt;
+  }
   const int pad = ((cnt + kBlock - 1) / kBlock) * kBlock;
   const int incl = block_incl_scan(cnt, warp_tot);  // (its barriers also order s_flags = 0)
   const int pincl = block_incl_scan(pad, warp_tot);
@@ -460,6 +453,7 @@ static_assert(kMapTokTile * DMOE_MAX_TOP_K <= kMapWarps * 32 * kScatRounds, "sca
 __global__ void __launch_bounds__(kMapThreads) k_map_scatter(int T, int E, int k, int nblk_cap,
                                                              const int32_t *__restrict__ top,
                                                              const int32_t *__restrict__ tile_off,
+                                                             const int32_t *__restrict__ seg_off,
                                                              const int32_t *__restrict__ bins,
                                                              const int32_t *__restrict__ padded_bins,
                                                              int32_t *__restrict__ indices,
@@ -468,7 +462,7 @@ __global__ void __launch_bounds__(kMapThreads) k_map_scatter(int T, int E, int k
                                                              int32_t *__restrict__ block_expert) {
   extern __shared__ int sm[];
   int *wh = sm;                           // [kMapWarps][E] counts, then exclusive offsets
-  int *s_base = wh + kMapWarps * E;       // [E] bins[e-1] + this tile's offset inside e
+  int *s_base = wh + kMapWarps * E;       // [E] bins[e-1] + offset of this tile inside e
   int *s_shift = s_base + E;              // [E] padded_bins[e-1] - bins[e-1]
   int *s_pb = s_shift + E;                // [E] padded_bins
   pdl_wait();
@@ -497,7 +491,8 @@ __global__ void __launch_bounds__(kMapThreads) k_map_scatter(int T, int E, int k
   for (int e = threadIdx.x; e < E; e += kMapThreads) {
     const int bp = (e > 0) ? bins[e - 1] : 0;
     const int pp = (e > 0) ? padded_bins[e - 1] : 0;
-    s_base[e] = bp + tile_off[(size_t)blockIdx.x * E + e];
+    s_base[e] = bp + seg_off[(size_t)(blockIdx.x / kScanSeg) * E + e] +
+                tile_off[(size_t)blockIdx.x * E + e];
     s_shift[e] = pp - bp;
     s_pb[e] = padded_bins[e];
   }
@@ -600,8 +595,9 @@ cudaError_t launch_route_hist(const uint16_t *logits, int T, int E, int k, bool 
 cudaError_t launch_map_scan(int T, int E, int32_t *tile_hist, int32_t *tokens_per_expert,
                             int32_t *bins, int32_t *padded_bins, int32_t *num_blocks,
                             int32_t *status, cudaStream_t st) {
-  return launch_pdl(k_map_scan, (E + 31) / 32, kScanThreads, 0, st, map_tiles(T), E, tile_hist,
-                    map_flags(tile_hist, T, E), tokens_per_expert, bins, padded_bins, num_blocks,
+  return launch_pdl(k_map_scan, dim3((E + 31) / 32, map_segments(T)), kScanThreads, 0, st,
+                    map_tiles(T), E, tile_hist, map_flags(tile_hist, T, E),
+                    map_segs(tile_hist, T, E), tokens_per_expert, bins, padded_bins, num_blocks,
                     status, map_ticket(tile_hist, T, E));
 }
 
@@ -611,7 +607,8 @@ cudaError_t launch_map_scatter(int T, int E, int k, int nblk_cap, const int32_t 
                                int32_t *dest_row, int32_t *block_expert, cudaStream_t st) {
   const size_t smem = sizeof(int) * (size_t)(kMapWarps + 3) * E;
   return launch_pdl(k_map_scatter, map_tiles(T), kMapThreads, smem, st, T, E, k, nblk_cap, top,
-                    tile_off, bins, padded_bins, indices, bin_ids, dest_row, block_expert);
+                    tile_off, map_segs(const_cast<int32_t *>(tile_off), T, E), bins, padded_bins,
+                    indices, bin_ids, dest_row, block_expert);
 }
 
 }  // namespace dmoe

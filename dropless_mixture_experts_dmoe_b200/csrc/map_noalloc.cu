@@ -21,8 +21,8 @@
 namespace {
 
 // Capacity of the static scratch in int32 words: the per-tile histograms (ceil(T/64) * E), one
-// counter and one status word per tile must fit (1 MiB; e.g. T <= 65280 tokens at E = 256,
-// T <= 16320 at E = 1024).
+// counter, one status word per tile and the scan's per-segment totals (ceil(T/32768) * E)
+// must fit (1 MiB; e.g. T <= 65152 tokens at E = 256, T <= 16256 at E = 1024).
 constexpr size_t kNoAllocScratchInts = DMOE_NOALLOC_SCRATCH_BYTES / sizeof(int32_t);
 
 static __device__ __align__(256) int32_t g_map_scratch[kNoAllocScratchInts];

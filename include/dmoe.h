@@ -207,9 +207,9 @@ DMOE_API int dmoe_backward(const dmoe_dims *dims, const void *dy, const void *w1
  *   Same arguments, results and status bits as dmoe_sparse_map, without ws / ws_bytes.
  *   Scratch: a static array of DMOE_NOALLOC_SCRATCH_BYTES in device global memory inside
  *     libdmoe.so; every GPU that loads the library holds it until the process exits.  The
- *     call needs (ceil(T/64) * (num_experts + 1) + 1) * 4 bytes of it and returns
- *     DMOE_ERR_WORKSPACE, before any launch, when that exceeds the limit (e.g. T > 65280 at
- *     E = 256).
+ *     call needs (ceil(T/64) * (num_experts + 1) + 1 + ceil(T/32768) * num_experts) * 4
+ *     bytes of it and returns DMOE_ERR_WORKSPACE, before any launch, when that exceeds the
+ *     limit (e.g. T > 65152 at E = 256).
  *   The call performs no allocation (no cudaMalloc, no cudaFree, no allocating library
  *     routine).  Its first call on a device looks up the array's device address with
  *     cudaGetSymbolAddress (once per device, with that device current); make that first call
