@@ -96,7 +96,9 @@ def load():
     lib.dmoe_router_backward.argtypes = [D, _P, _P, _P, M, _P, _P, _P, _P, _SZ, _P]
     lib.dmoe_bwd_dx.argtypes = [D, _P, _P, _P, _P, M, _P, _P]
     lib.dmoe_bwd_wgrad.argtypes = [D, _P, _P, _P, _P, _P, M, _P, _P, _P, _P]
-    for fn in ("dmoe_sparse_map", "dmoe_forward", "dmoe_backward", "dmoe_padded_gather",
+    lib.dmoe_sparse_map_noalloc.argtypes = [D, _P, M, _P]
+    for fn in ("dmoe_sparse_map", "dmoe_sparse_map_noalloc", "dmoe_forward", "dmoe_backward",
+               "dmoe_padded_gather",
                "dmoe_expert_glu", "dmoe_expert_glu_gather", "dmoe_expert_down", "dmoe_padded_scatter",
                "dmoe_bwd_dglu", "dmoe_bwd_dx", "dmoe_bwd_wgrad", "dmoe_bwd_scatter",
                "dmoe_router_forward", "dmoe_router_dlogits", "dmoe_router_backward"):
@@ -313,10 +315,8 @@ def dmoe_router_backward(dims, x, w_router, logits, smap: SparseMap, dweights, d
 def dmoe_sparse_map_noalloc(dims: dmoe_dims, logits, smap: SparseMap, stream=None):
     """Allocation-free routing + sparse map (static scratch inside the library; see
     include/dmoe.h).  For callers that cannot allocate a workspace."""
-    fn = load().dmoe_sparse_map_noalloc
-    fn.argtypes = [ctypes.POINTER(dmoe_dims), _P, ctypes.POINTER(dmoe_map), _P]
-    fn.restype = _I
-    _check(fn(ctypes.byref(dims), _ptr(logits), ctypes.byref(smap.c), _stream(stream)),
+    _check(load().dmoe_sparse_map_noalloc(ctypes.byref(dims), _ptr(logits),
+                                          ctypes.byref(smap.c), _stream(stream)),
            "dmoe_sparse_map_noalloc")
 
 
