@@ -127,7 +127,9 @@ __host__ __device__ constexpr bool is_dense_rows(int mode) {
 // (a few K steps per tile) that the epilogue, not the MMA, bounds a tile.  The ring of 32 KB
 // stages is as deep as shared memory allows next to the result staging: for the forward GEMMs
 // (few result boxes per tile) 3 stages of two K slabs (64 KB) and one 4 KB staging buffer per
-// warp, else 5 stages of one slab (4 with 8 warps) and two staging buffers.
+// warp; for the weight gradients, whose operand loads are the bound, 6 stages of one slab and
+// one staging buffer (measured 2-6 % faster than 5 and two); else 5 stages (4 with 8 warps)
+// and two staging buffers.
 template <int MODE, int EPI>
 struct Cfg {
   static constexpr int a_mn = (MODE == MODE_WGRAD || MODE == MODE_RWGRAD) ? 1 : 0;
@@ -144,8 +146,8 @@ struct Cfg {
   static constexpr int bk = BK * kslabs;  // K per stage
   static constexpr int a_bytes = A_BYTES * kslabs;
   static constexpr int stage_bytes = (A_BYTES + B_BYTES) * kslabs;
-  static constexpr int stages = (kslabs == 2) ? 3 : ((EPI == 8) ? 4 : 5);
-  static constexpr int out_bufs = (kslabs == 2) ? 1 : 2;
+  static constexpr int stages = (kslabs == 2) ? 3 : ((EPI == 8) ? 4 : (MODE == MODE_WGRAD ? 6 : 5));
+  static constexpr int out_bufs = (kslabs == 2 || MODE == MODE_WGRAD) ? 1 : 2;
   static constexpr int out_bytes = epi_warps * out_bufs * BOX_BYTES;
   // WGRAD: one zeroed result box, the source of the zero tiles' stores
   static constexpr int zero_bytes = (MODE == MODE_WGRAD) ? BOX_BYTES : 0;
