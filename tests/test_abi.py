@@ -114,3 +114,30 @@ def test_status_strings(lib):
     assert B.status_string(0) == "ok"
     s = B.status_string(B.STATUS_TIMEOUT | B.STATUS_NONFINITE_LOGITS)
     assert "timeout" in s and "nonfinite" in s
+
+
+@pytest.mark.parametrize("T,E", [(1, 1), (4096, 8), (32768, 256), (32769, 256), (262144, 256),
+                                 (65536, 1024)])
+def test_map_workspace_formula(T, E):
+    """The map workspace is what include/dmoe.h states: per-tile histograms ceil(T/64)*E, one
+    ticket counter, one status word per tile and the scan's per-segment totals
+    ceil(T/32768)*E, int32 each (rounded up to the 256-byte alignment)."""
+    d = B.make_dims(T, 128, 128, E, 1)
+    tiles = -(-T // 64)
+    segs = -(-tiles // 512)
+    need = 4 * (tiles * E + 1 + tiles + segs * E)
+    assert need <= B.dmoe_workspace_bytes(d, B.WS_MAP) < need + 256
+
+
+def test_noalloc_capacity_limits(lib):
+    """dmoe_sparse_map_noalloc's static scratch holds exactly the documented sizes: the largest
+    T that fits passes the capacity check (and is then refused for its unaligned logits pointer,
+    still before any device call); 64 more tokens are refused with DMOE_ERR_WORKSPACE."""
+    fake = 1 << 20  # host-side checks only: every case below is refused before a launch
+    m = B.dmoe_map(*([fake] * len(B.MAP_FIELDS)))
+    for E, t_max in ((256, 65152), (1024, 16256)):
+        fits = B.make_dims(t_max, 128, 128, E, 1)
+        over = B.make_dims(t_max + 64, 128, 128, E, 1)
+        assert lib.dmoe_sparse_map_noalloc(ctypes.byref(over), fake, ctypes.byref(m), None) == -4
+        assert lib.dmoe_sparse_map_noalloc(ctypes.byref(fits), fake + 2, ctypes.byref(m),
+                                           None) == -5
