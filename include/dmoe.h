@@ -25,7 +25,11 @@
  *     dmoe_saved_bytes.
  *   - Every launch is asynchronous on `stream` (a cudaStream_t, passed as void*; NULL is
  *     the legacy default stream).  No call reads device memory on the host, so the whole
- *     layer can run without a host synchronisation.
+ *     layer can run without a host synchronisation, and a whole step can be captured in a
+ *     CUDA graph.  Kernels are launched with programmatic dependent launch: a kernel may
+ *     start before the previous kernel on the stream has finished, but it waits for all
+ *     earlier work of the stream before its first access to global memory, so stream
+ *     ordering is exactly as for plain launches, also with the caller's own kernels.
  *   - Every call returns an int: DMOE_OK (0) or a negative DMOE_ERR_* detected on the host
  *     BEFORE any launch (nothing is launched then), or DMOE_ERR_LAUNCH if a launch failed.
  *   - Conditions only the device can see set bits in the caller's int32 status word
