@@ -75,3 +75,34 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
     with contextlib.redirect_stdout(buf):
         bench.run_reference(args, WORKLOADS[1])
     assert buf.getvalue() == ""
+
+
+def test_reference_arm_json_line(monkeypatch):
+    """On rank 0 the reference arm prints one JSON line with the contract's keys: the oracle's
+    tokens/s as value, cpu_baseline describing the run, and an e2e with no transfers."""
+    import json
+
+    bench = _bench()
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--workload", "1",
+                                      "--steps", "2"])
+    args = bench.parse()
+    from dropless_mixture_experts_dmoe_b200.workloads import WORKLOADS
+
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        bench.run_reference(args, WORKLOADS[1])
+    lines = [ln for ln in buf.getvalue().splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["steps"] == 2
+    assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    assert d["config"]["T"] == 256 and d["config"]["num_experts"] == 8
