@@ -141,3 +141,17 @@ def test_noalloc_capacity_limits(lib):
         assert lib.dmoe_sparse_map_noalloc(ctypes.byref(over), fake, ctypes.byref(m), None) == -4
         assert lib.dmoe_sparse_map_noalloc(ctypes.byref(fits), fake + 2, ctypes.byref(m),
                                            None) == -5
+
+
+def test_autograd_wrapper_validates_inputs_on_the_host():
+    """dmoe() rejects non-CUDA, non-bf16 or mis-shaped inputs before calling the library."""
+    import torch
+
+    from dropless_mixture_experts_dmoe_b200 import autograd as A
+
+    x = torch.zeros(4, 128, dtype=torch.bfloat16)  # a CPU tensor
+    w = torch.zeros(2, 128, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        A.dmoe(x, torch.zeros(4, 2, dtype=torch.bfloat16), w, w, w, 1)
+    with pytest.raises(ValueError):
+        A.dmoe(x.float(), x, w, w, w, 1)
