@@ -30,6 +30,8 @@ import os
 import numpy as np
 import pytest
 import torch
+from hypothesis import HealthCheck, given, settings
+from hypothesis import strategies as st
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -527,3 +529,36 @@ def test_router_backward_renorm_finite_differences_and_autograd(oracle_mod):
     np.testing.assert_allclose(g["dx_r"], l.grad.numpy() @ Wr.astype(np.float64), rtol=1e-12,
                                atol=1e-14)
 
+
+
+# ---- property sweeps (hypothesis) ----------------------------------------------------------
+
+
+@settings(max_examples=60, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(T=st.integers(1, 300), E=st.integers(1, 64), data=st.data())
+def test_map_invariants_property(oracle_mod, T, E, data):
+    """Every map invariant on random routings: k distinct experts per token, any T and E."""
+    k = data.draw(st.integers(1, min(E, 8)), label="k")
+    rng = np.random.default_rng(data.draw(st.integers(0, 2 ** 31 - 1), label="seed"))
+    top = np.argsort(rng.random((T, E)), axis=1)[:, :k].astype(np.int32)
+    _check_map_invariants(top, E, oracle_mod.sparse_map(top, E))
+
+
+@settings(max_examples=60, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(E=st.integers(1, 7), data=st.data())
+def test_route_brute_force_property(oracle_mod, E, data):
+    """The chosen k-subset is the unique one that beats every other expert under (value
+    descending, index ascending), on logits drawn from a small set full of ties and signed
+    zeros; slots follow the same order."""
+    k = data.draw(st.integers(1, E), label="k")
+    vals = np.array([-2.0, -0.0, 0.0, 0.5, 0.5, 3.0, -np.inf], dtype=np.float32)
+    rng = np.random.default_rng(data.draw(st.integers(0, 2 ** 31 - 1), label="seed"))
+    logits = rng.choice(vals, size=(16, E)).astype(np.float32)
+    top, _ = oracle_mod.route(logits, k)
+    for t in range(16):
+        l = [float(v) for v in logits[t]]
+        winners = [set(S) for S in itertools.combinations(range(E), k)
+                   if all(_beats(l[a], a, l[b], b) for a in S for b in range(E) if b not in S)]
+        assert len(winners) == 1 and set(top[t].tolist()) == winners[0]
+        for s in range(k - 1):
+            assert _beats(l[top[t, s]], top[t, s], l[top[t, s + 1]], top[t, s + 1])
