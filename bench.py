@@ -1,13 +1,17 @@
 """Benchmark of the dMoE layer on B200: one JSON line on rank 0.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload 2]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload 5]
 
-A step is one pass of the whole hot path over one batch: routing + sparse map (3 kernels),
-padded gather, GLU GEMM, down GEMM and weighted scatter (workloads with a backward add the
-backward).  The default workload is the Mixtral-shaped forward (T=4096, hidden 4096, ffn
-14336, 8 experts, top-2).  ``value`` is layer tokens/s with inputs resident in HBM; ``e2e``
-is the same through dmoe_sparse_map + dmoe_forward with the step's inputs copied from pinned
-host memory and the output copied back inside the timed region.  The timed K steps carry no
+A step is one pass of the whole hot path over one batch: routing + sparse map, padded
+gather, GLU GEMM, down GEMM and weighted scatter, and for the workloads with a backward the
+dY gather, the dH GEMM with its dGLU epilogue, the weight-gradient GEMM, the dX GEMM and the
+scatter-sum.  The default workload is the largest one, the skewed forward + backward
+(T=32768, hidden 2048, ffn 512, 256 experts, top-8, Zipf-skewed logits); ``--workload 2``
+is the Mixtral-shaped forward.  ``value`` is layer tokens/s with inputs resident in HBM;
+``e2e`` is the same through dmoe_sparse_map + dmoe_forward (+ dmoe_backward) with the step's
+inputs copied from pinned host memory and the outputs copied back inside the timed region.
+Fractions of the bf16 tensor peak use the measured burst peak when the timed region is
+shorter than a second and the measured sustained (power-capped) peak otherwise.  The timed K steps carry no
 events between kernels (each kernel's launch overlaps the previous kernel's tail through
 programmatic dependent launch); per-kernel times come from a second pass of K steps with CUDA
 events recorded on the launch stream around every entry point.
@@ -42,7 +46,8 @@ def parse():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    p.add_argument("--workload", type=int, default=2)
+    p.add_argument("--workload", type=int, default=5,
+                   help="1..5 (default 5: the skewed forward+backward workload, the largest)")
     p.add_argument("--shape", default="",
                    help="T,hidden,ffn,E,top_k[,bwd][,zipf]: a custom workload (forward, or "
                         "fwd+bwd; zipf adds the skewed workload's logit bias)")
@@ -97,23 +102,86 @@ def ncu_traffic(kernel: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling; keeps the samples taken inside [t0, t1]."""
+    """SM clock and throttle-reason sampling while a region runs; keeps the samples taken
+    inside [t0, t1] (wall clock).  NVML is polled every 5 ms from a thread (reads only), so
+    even a timed region of a tenth of a second gets a few dozen samples; without NVML the
+    fallback is ``nvidia-smi -lms 100``."""
 
     FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.005
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, pci_bus_id: str | None = None):
         self.proc = None
+        self.thread = None
+        self.samples = []  # (wall time, sm MHz, reasons bit mask)
+        self.max_mhz = None
+        try:
+            import threading
+
+            import pynvml
+
+            pynvml.nvmlInit()
+            h = None
+            if pci_bus_id:
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByPciBusId(pci_bus_id)
+                except Exception:
+                    h = None
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.nvml, self.handle = pynvml, h
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            self.running = True
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            self.source = "nvml, 5 ms"
+            return
+        except Exception:
+            self.thread = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(index), f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.source = "nvidia-smi, 100 ms"
         except Exception:
             self.proc = None
 
+    def _poll(self):
+        nv, h = self.nvml, self.handle
+        while self.running:
+            try:
+                mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                reasons = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                self.samples.append((time.time(), mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(self.PERIOD_S)
+
+    def _summary(self, sm, mx, reasons):
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "samples": 0, "reasons": [],
+                    "source": self.source}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "sm_mhz_min": min(sm), "reasons": sorted(reasons), "source": self.source}
+
     def stop(self, t0: float, t1: float):
+        if self.thread is not None:
+            self.running = False
+            self.thread.join(timeout=2)
+            nv = self.nvml
+            bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+            sm, reasons = [], set()
+            for ts, mhz, r in self.samples:
+                if t0 <= ts <= t1:
+                    sm.append(mhz)
+                    reasons |= {n for n, b in bits.items() if r & b}
+            return self._summary(sm, [self.max_mhz] * len(sm), reasons)
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -142,10 +210,39 @@ class ClockSampler:
             for n, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "samples": 0, "reasons": []}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
-                "reasons": sorted(reasons)}
+        return self._summary(sm, mx, reasons)
+
+
+def sampler_for(device: int):
+    import torch
+
+    bus = None
+    try:
+        p = torch.cuda.get_device_properties(device)
+        bus = "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+    except Exception:
+        bus = None
+    return ClockSampler(device, bus)
+
+
+def tensor_peak(pk: dict, timed_s: float):
+    """The bf16 tensor peak that matches how a kernel was timed: the burst figure for a timed
+    region under one second (the clocks have not yet settled under the power cap), the
+    sustained one for a region of seconds.  Returns (peak TFLOP/s, description)."""
+    if timed_s < 1.0:
+        return pk["bf16"], (f"{pk['source']} burst bf16 (timed region {timed_s:.2f} s < 1 s; "
+                            f"sustained {pk['bf16_sus']})")
+    return pk["bf16_sus"], (f"{pk['source']} sustained bf16 (timed region {timed_s:.2f} s >= 1 s; "
+                            f"burst {pk['bf16']})")
+
+
+def config_of(w, router: bool, world: int) -> dict:
+    """The workload description shared by both arms of the bench."""
+    return {"workload": f"{w.name} {w.describe()}" + (" +router" if router else ""),
+            "T": w.T, "hidden": w.hidden, "ffn": w.ffn, "num_experts": w.E, "top_k": w.top_k,
+            "l2": "inputs larger than L2 (expert weights %.2f GB per step)" %
+                  (3 * w.E * w.hidden * w.ffn * 2 / 1e9),
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
 # ------------------------------------------------------------------------------------------------
@@ -236,9 +333,7 @@ def run_reference(args, w):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{w.name} {w.describe()}" + (" +router" if args.router else ""),
-                   "T": w.T, "hidden": w.hidden,
-                   "ffn": w.ffn, "num_experts": w.E, "top_k": w.top_k},
+        "config": config_of(w, args.router, int(os.environ.get("WORLD_SIZE", "1"))),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -357,7 +452,7 @@ def run_ours(args, w):
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    sampler = sampler_for(torch.cuda.current_device()) if rank == 0 else None
     time.sleep(0.3 if sampler else 0.0)  # let the sampler start before the timed region
     for _ in range(args.warmup):
         step()
@@ -511,41 +606,38 @@ def run_ours(args, w):
         router_bwd=2 * w.T * w.E + 8 * w.T * w.top_k + 3 * 2 * w.T * w.E + 4 * w.T * w.hidden
         + 2 * w.T * w.hidden + 2 * w.E * w.hidden + 4 * w.E * w.hidden)
     km = {n: statistics.mean(v) for n, v in per_kernel.items()}
+    # the tensor peak that matches how the kernels were timed (burst below a second)
+    pk_t, pk_kind = tensor_peak(pk, ms / 1e3)
     kernels = {}
     for n in names:
         ent = {"ms": km[n]}
         if n in router_flops:  # small E: a thin GEMM, bound by bytes more than by the MMAs
             ent["TFLOP/s"] = router_flops[n] / km[n] / 1e9
-            ent["frac_bf16"] = ent["TFLOP/s"] / pk["bf16_sus"]
+            ent["frac_bf16"] = ent["TFLOP/s"] / pk_t
             ent["GB/s"] = byts[n] / km[n] / 1e6
             ent["frac_hbm"] = ent["GB/s"] / pk["hbm"]
         elif n in flops:
             ent["TFLOP/s"] = flops[n] / km[n] / 1e9
-            ent["frac_bf16"] = ent["TFLOP/s"] / pk["bf16_sus"]
+            ent["frac_bf16"] = ent["TFLOP/s"] / pk_t
         else:
             ent["GB/s"] = byts[n] / km[n] / 1e6
             ent["frac_hbm"] = ent["GB/s"] / pk["hbm"]
         kernels[n] = ent
     dom = max(flops.keys() & set(names), key=lambda n: km[n])
     achieved = flops[dom] / km[dom] / 1e9
-    wl_name = f"{w.name} {w.describe()}" + (" +router" if router else "")
     traffic = ncu_traffic(dom, w.name)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": wl_name, "T": w.T, "hidden": w.hidden, "ffn": w.ffn,
-                   "num_experts": w.E, "top_k": w.top_k,
-                   "l2": "inputs larger than L2 (expert weights %.2f GB per step)" %
-                         (3 * w.E * w.hidden * w.ffn * 2 / 1e9),
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "config": config_of(w, router, world),
         "useful_tflops": useful / (ms_per_step / 1e3) / 1e12,
-        "useful_tflops_frac_bf16": useful / (ms_per_step / 1e3) / 1e12 / pk["bf16_sus"],
+        "useful_tflops_frac_bf16": useful / (ms_per_step / 1e3) / 1e12 / pk_t,
         "padded_frac": pad_frac,
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved,
-                     "peak": pk["bf16_sus"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_sus"],
-                     "peak_kind": f"{pk['source']} sustained bf16 (burst {pk['bf16']})",
+                     "peak": pk_t, "unit": "TFLOP/s", "frac": achieved / pk_t,
+                     "peak_kind": pk_kind,
                      "traffic": traffic,
                      "algorithmic_flops_per_launch": flops[dom]},
         "kernels": kernels,
@@ -607,7 +699,7 @@ def run_map_only(args, w):
     torch.cuda.synchronize()
     if int(smap.status.item()):
         raise RuntimeError(f"device status: {B.status_string(int(smap.status.item()))}")
-    sampler = ClockSampler(torch.cuda.current_device())
+    sampler = sampler_for(torch.cuda.current_device())
     time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     wall0 = time.time()

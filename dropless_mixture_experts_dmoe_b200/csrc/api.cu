@@ -4,6 +4,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -38,16 +40,23 @@ long long pmax_of(const dmoe_dims *d) {
   return (n + (long long)(DMOE_BLOCKING - 1) * d->num_experts) / DMOE_BLOCKING * DMOE_BLOCKING;
 }
 
+// The current device must be an sm_100 part.  The answer is cached per device ordinal (a
+// process may see GPUs of several kinds); ordinals past the cache are checked on every call.
+constexpr int kDeviceCache = 64;
+std::atomic<int> g_device_ok[kDeviceCache];  // 0 unknown, 1 sm_100, 2 other
+
 int check_device() {
-  static int cached = -1;
-  if (cached < 0) {
-    int dev = 0, major = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return DMOE_ERR_DEVICE;
+  int known = (dev < kDeviceCache) ? g_device_ok[dev].load(std::memory_order_relaxed) : 0;
+  if (known == 0) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
       return DMOE_ERR_DEVICE;
-    cached = (major == 10) ? 1 : 0;
+    known = (major == 10) ? 1 : 2;
+    if (dev < kDeviceCache) g_device_ok[dev].store(known, std::memory_order_relaxed);
   }
-  return cached == 1 ? DMOE_OK : DMOE_ERR_DEVICE;
+  return known == 1 ? DMOE_OK : DMOE_ERR_DEVICE;
 }
 
 int check_map(const dmoe_map *m, bool need_weights) {

@@ -217,7 +217,10 @@ DMOE_API int dmoe_backward(const dmoe_dims *dims, const void *dy, const void *w1
  *   The call performs no allocation (no cudaMalloc, no cudaFree, no allocating library
  *     routine).  Its first call on a device looks up the array's device address with
  *     cudaGetSymbolAddress (once per device, with that device current); make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address stays cached for the life of the process: after
+ *     cudaDeviceReset (or anything else that destroys and re-creates the device's primary
+ *     context) the array may move, so such a caller must unload and reload libdmoe.so before
+ *     calling this entry point again.
  *   Every call on a device shares the one array and leaves its contents behind; each call
  *     rewrites all of the scratch it reads before reading it, so stale contents never leak
  *     into a result.  Calls whose executions overlap on the GPU (different streams, or
