@@ -16,7 +16,8 @@ cites the passage of the pages it follows, in the C source:
                          math, the block->expert table (walkthrough §2, §4.1-§4.3).
 * ``forward``         -- per-token loop y_t = sum_s w_ts W2_e(silu(W1_e x_t) * W3_e x_t)
                          (walkthrough §4.5 schematic, gated SiLU per the issue's config).
-* ``backward``, ``backward_tokens``, ``wgrad_elements`` -- chain rule per (token, slot);
+* ``backward``, ``backward_tokens``, ``wgrad_elements``, ``wgrad_expert`` -- chain rule per
+                         (token, slot);
                          role swap and routing-weight gradient of walkthrough §4.2, activation
                          recompute of §4.4.
 * ``router_logits``, ``router_backward`` -- the linear router whose output is the issue's
@@ -67,10 +68,12 @@ def _load():
         lib.oracle_backward.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P, P]
         lib.oracle_backward_tokens.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, P, I]
         lib.oracle_wgrad_elements.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, I]
+        lib.oracle_wgrad_expert.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, P, I]
         lib.oracle_router_logits.argtypes = [I, I, I, P, P, I, P, P, I]
         lib.oracle_router_backward.argtypes = [I, I, I, I, I, P, P, P, P, P, P, I, P, P, I, P, P, I]
         for fn in (lib.oracle_route, lib.oracle_sparse_map, lib.oracle_forward, lib.oracle_backward,
-                   lib.oracle_backward_tokens, lib.oracle_wgrad_elements, lib.oracle_max_threads,
+                   lib.oracle_backward_tokens, lib.oracle_wgrad_elements, lib.oracle_wgrad_expert,
+                   lib.oracle_max_threads,
                    lib.oracle_router_logits, lib.oracle_router_backward):
             fn.restype = ctypes.c_int
         _lib = lib
@@ -208,6 +211,22 @@ def wgrad_elements(x, dy, W1, W3, W2, top_experts, weights, queries, threads=1):
     if rc != 0:
         raise RuntimeError(f"oracle_wgrad_elements failed ({rc})")
     return out
+
+
+def wgrad_expert(x, dy, W1, W3, W2, top_experts, weights, e: int, threads=1):
+    """Whole weight-gradient slabs of expert ``e``: (dW1_e [f,h], dW3_e [f,h], dW2_e [h,f]),
+    float64, each element summed over the expert's entries in entry order."""
+    x, dy, W1, W3, W2 = _f32(x), _f32(dy), _f32(W1), _f32(W3), _f32(W2)
+    top, w = _i32(top_experts), _f64(weights)
+    T, h = x.shape
+    E, f, _ = W1.shape
+    k = top.shape[1]
+    d1, d3, d2 = np.empty((f, h)), np.empty((f, h)), np.empty((h, f))
+    rc = _load().oracle_wgrad_expert(T, h, f, E, k, _p(x), _p(dy), _p(W1), _p(W3), _p(W2),
+                                     _p(top), _p(w), int(e), _p(d1), _p(d3), _p(d2), int(threads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_wgrad_expert failed ({rc})")
+    return d1, d3, d2
 
 
 def router_logits(x, Wr, tokens=None, threads=1):

@@ -402,6 +402,92 @@ int oracle_wgrad_elements(int T, int h, int f, int E, int k, const float *x, con
   return 0;
 }
 
+/* The three weight-gradient slabs of one expert e, summed over every entry routed to it
+ * (entries visited in increasing j, the chain rule of entry_backward):
+ *   dW1e[r][c] = sum da_ts[r] x_t[c],  dW3e[r][c] = sum db_ts[r] x_t[c]   ([f, h])
+ *   dW2e[r][c] = sum g_ts[r] hh_ts[c]                                      ([h, f])
+ * The per-entry vectors (da, db, hh, g) of a chunk of entries are formed first (parallel over
+ * the entries), then added to the slabs (parallel over slab rows, entries in order), so every
+ * slab element is the same ordered sum whatever the thread count.  Outputs double,
+ * overwritten. */
+int oracle_wgrad_expert(int T, int h, int f, int E, int k, const float *x, const float *dy,
+                        const float *W1, const float *W3, const float *W2, const int32_t *top,
+                        const double *w, int e, double *dW1e, double *dW3e, double *dW2e,
+                        int nthreads) {
+  if (e < 0 || e >= E) return -1;
+  const long N = (long)T * k;
+  const int CH = 512; /* entries per chunk */
+  const float *W1e = W1 + (size_t)e * f * h, *W3e = W3 + (size_t)e * f * h;
+  const float *W2e = W2 + (size_t)e * h * f;
+  long *ent = (long *)malloc(sizeof(long) * (size_t)(N > 0 ? N : 1));
+  double *da = (double *)malloc(sizeof(double) * (size_t)CH * f);
+  double *db = (double *)malloc(sizeof(double) * (size_t)CH * f);
+  double *hh = (double *)malloc(sizeof(double) * (size_t)CH * f);
+  double *g = (double *)malloc(sizeof(double) * (size_t)CH * h);
+  if (!ent || !da || !db || !hh || !g) {
+    free(ent); free(da); free(db); free(hh); free(g);
+    return -2;
+  }
+  long n = 0;
+  for (long j = 0; j < N; ++j)
+    if (top[j] == e) ent[n++] = j;
+  memset(dW1e, 0, sizeof(double) * (size_t)f * h);
+  memset(dW3e, 0, sizeof(double) * (size_t)f * h);
+  memset(dW2e, 0, sizeof(double) * (size_t)h * f);
+  if (nthreads < 1) nthreads = 1;
+  for (long c0 = 0; c0 < n; c0 += CH) {
+    const int m = (int)((n - c0 < CH) ? n - c0 : CH);
+#ifdef _OPENMP
+#pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1)
+#endif
+    for (int q = 0; q < m; ++q) {
+      const long j = ent[c0 + q];
+      const long t = j / k;
+      const float *xt = x + (size_t)t * h, *dyt = dy + (size_t)t * h;
+      double *gq = g + (size_t)q * h;
+      for (int o = 0; o < h; ++o) gq[o] = w[j] * (double)dyt[o];
+      for (int i = 0; i < f; ++i) {
+        double sa = 0.0, sb = 0.0, d = 0.0;
+        const float *r1 = W1e + (size_t)i * h, *r3 = W3e + (size_t)i * h;
+        for (int jj = 0; jj < h; ++jj) {
+          sa += (double)r1[jj] * (double)xt[jj];
+          sb += (double)r3[jj] * (double)xt[jj];
+        }
+        for (int o = 0; o < h; ++o) d += (double)W2e[(size_t)o * f + i] * gq[o];
+        const double sig = 1.0 / (1.0 + exp(-sa));
+        da[(size_t)q * f + i] = d * sb * sig * (1.0 + sa * (1.0 - sig));
+        db[(size_t)q * f + i] = d * (sa * sig);
+        hh[(size_t)q * f + i] = silu(sa) * sb;
+      }
+    }
+#ifdef _OPENMP
+#pragma omp parallel for num_threads(nthreads) schedule(static)
+#endif
+    for (int r = 0; r < f + h; ++r) {
+      for (int q = 0; q < m; ++q) {
+        const long t = ent[c0 + q] / k;
+        if (r < f) { /* row r of dW1e and dW3e */
+          const float *xt = x + (size_t)t * h;
+          const double a1 = da[(size_t)q * f + r], a3 = db[(size_t)q * f + r];
+          double *o1 = dW1e + (size_t)r * h, *o3 = dW3e + (size_t)r * h;
+          for (int c = 0; c < h; ++c) {
+            o1[c] += a1 * (double)xt[c];
+            o3[c] += a3 * (double)xt[c];
+          }
+        } else { /* row r - f of dW2e */
+          const int o = r - f;
+          const double go = g[(size_t)q * h + o];
+          double *o2 = dW2e + (size_t)o * f;
+          const double *hq = hh + (size_t)q * f;
+          for (int c = 0; c < f; ++c) o2[c] += go * hq[c];
+        }
+      }
+    }
+  }
+  free(ent); free(da); free(db); free(hh); free(g);
+  return 0;
+}
+
 /* ------------------------------------------------------------------------------------ */
 /* Router GEMM and the gradient through the routing weights.                             */
 /* ------------------------------------------------------------------------------------ */

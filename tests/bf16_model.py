@@ -1,0 +1,89 @@
+"""Float64 model of where the CUDA path rounds to bf16, used only to size the max-abs
+tolerance of the stress shapes (shapes outside the five named workloads).
+
+The layer stores its intermediates in bf16 with fp32 accumulation: H = bf16(silu(A) * Bm),
+Y_pad = bf16(H W2^T), y = bf16(sum_s w_s Y_s); in the backward A, Bm are the saved bf16
+values, dA, dBm and Hw = w h are bf16, dX = bf16(dA W1 + dBm W3), dx = bf16(sum_s dX_s), and
+the weight gradients stay fp32.  This module applies exactly those roundings to float64
+arithmetic on the same inputs (no other error source), so its max-abs error against the
+oracle is what an ideal bf16 pipeline of this design reaches on that shape.  With few
+products per output element (few tokens per expert) that error can exceed 5 % of the RMS,
+although every element is computed correctly: the tests then allow 1.5 x the modelled error,
+and keep the 5e-2 bound wherever the model stays within 5e-2 / 1.25.
+
+It shares nothing with the CUDA path and runs on the CPU (torch float64)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from helpers import MAX_ABS_RMS, metrics
+
+
+def _bf(t: torch.Tensor) -> torch.Tensor:
+    return t.to(torch.bfloat16).double()
+
+
+def stress_bound(modelled: float) -> float:
+    """Max-abs / RMS bound for a stress shape whose modelled bf16 error is ``modelled``."""
+    return MAX_ABS_RMS if 1.25 * modelled <= MAX_ABS_RMS else 1.5 * modelled
+
+
+def forward_model(inp: dict, top: np.ndarray, wts: np.ndarray) -> np.ndarray:
+    X = inp["x"].double()
+    W1, W3, W2 = inp["w1"].double(), inp["w3"].double(), inp["w2"].double()
+    E = W1.shape[0]
+    wf = torch.from_numpy(wts.astype(np.float32)).double()
+    y = torch.zeros_like(X)
+    for s in range(top.shape[1]):
+        for e in range(E):
+            ts = np.nonzero(top[:, s] == e)[0]
+            if len(ts) == 0:
+                continue
+            Xe = X[ts]
+            a = (Xe @ W1[e].T).float().double()
+            b = (Xe @ W3[e].T).float().double()
+            Y = _bf(_bf(torch.nn.functional.silu(a) * b) @ W2[e].T)
+            y[ts] += wf[ts, s][:, None] * Y
+    return _bf(y).numpy()
+
+
+def backward_model(inp: dict, top: np.ndarray, wts: np.ndarray) -> dict:
+    X, dy = inp["x"].double(), inp["dy"].double()
+    W1, W3, W2 = inp["w1"].double(), inp["w3"].double(), inp["w2"].double()
+    E, f, h = W1.shape
+    T, k = top.shape
+    dW1 = torch.zeros(E, f, h, dtype=torch.float64)
+    dW3 = torch.zeros_like(dW1)
+    dW2 = torch.zeros(E, h, f, dtype=torch.float64)
+    dxs = torch.zeros(T, k, h, dtype=torch.float64)
+    dw = torch.zeros(T, k, dtype=torch.float64)
+    wf = torch.from_numpy(wts.astype(np.float32)).double()
+    for e in range(E):
+        ts, ss = np.nonzero(top == e)
+        if len(ts) == 0:
+            continue
+        Xe = X[ts]
+        A, Bm = _bf(Xe @ W1[e].T), _bf(Xe @ W3[e].T)
+        s = torch.sigmoid(A)
+        hv = A * s * Bm
+        G = dy[ts] @ W2[e]
+        wr = wf[ts, ss][:, None]
+        dA = _bf(wr * G * Bm * s * (1 + A * (1 - s)))
+        dB = _bf(wr * G * A * s)
+        dw[ts, ss] = (G * hv).sum(1)
+        dxs[ts, ss] = _bf(dA @ W1[e] + dB @ W3[e])
+        dW1[e] = dA.T @ Xe
+        dW3[e] = dB.T @ Xe
+        dW2[e] = dy[ts].T @ _bf(wr * hv)
+    return {"dx": _bf(dxs.sum(1)).numpy(), "dW1": dW1.numpy(), "dW3": dW3.numpy(),
+            "dW2": dW2.numpy(), "dw": dw.numpy()}
+
+
+def bounds(model: dict, ref: dict) -> dict:
+    """Per-output max-abs / RMS bound from the modelled errors against the oracle."""
+    out = {}
+    for n, v in model.items():
+        _, mx, rms = metrics(v, ref[n])
+        out[n] = stress_bound(mx / rms if rms else 0.0)
+    return out

@@ -10,7 +10,7 @@ from dropless_mixture_experts_dmoe_b200 import autograd as A
 from dropless_mixture_experts_dmoe_b200 import binding as B
 from dropless_mixture_experts_dmoe_b200.workloads import custom, make_inputs
 
-from helpers import MAX_ABS_RMS_STRESS, assert_close, to_np
+from helpers import assert_close, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -62,8 +62,10 @@ def test_autograd_matches_direct_calls(w, renorm):
     r = oracle.router_backward(inp["x"].float().numpy(), wr, lg, top,
                                g["dw"].double().cpu().numpy(), want_dx=False, want_dwr=False,
                                renorm=renorm)
-    assert_close(to_np(leaves["logits"].grad), r["dlogits"], "dlogits",
-                 max_abs_rms=MAX_ABS_RMS_STRESS)
+    # dlogits: fp32 arithmetic rounded once to bf16 per element
+    got, ref = to_np(leaves["logits"].grad), r["dlogits"]
+    assert (np.abs(got - ref) <= 2.0 ** -7 * np.abs(ref) + 1e-4 * np.abs(ref).max()).all()
+    assert_close(got, ref, "dlogits")
 
 
 def test_autograd_rejects_bad_inputs():

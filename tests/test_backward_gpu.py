@@ -9,8 +9,9 @@ import oracle
 from dropless_mixture_experts_dmoe_b200 import binding as B
 from dropless_mixture_experts_dmoe_b200.workloads import WORKLOADS, custom, make_inputs
 
-from helpers import (MAX_ABS_RMS, MAX_ABS_RMS_STRESS, assert_close, dims_of, gpu_backward,
-                     oracle_inputs, sample_tokens, to_np)
+import bf16_model
+from helpers import (MAX_ABS_RMS, assert_close, dims_of, gpu_backward, oracle_inputs, to_np,
+                     tokens_covering_blocks)
 
 pytestmark = pytest.mark.gpu
 
@@ -33,9 +34,11 @@ def test_backward_full_parity_small(w):
     o = oracle_inputs(inp)
     top, wts = oracle.route(o["logits"], w.top_k)
     ref = oracle.backward(o["x"], o["dy"], o["w1"], o["w3"], o["w2"], top, wts)
-    tol = MAX_ABS_RMS if w.number else MAX_ABS_RMS_STRESS  # named workload vs stress shape
+    tol = dict.fromkeys(ref, MAX_ABS_RMS)
+    if not w.number:  # stress shape: the modelled bf16 error decides (tests/bf16_model.py)
+        tol = bf16_model.bounds(bf16_model.backward_model(inp, top, wts), ref)
     for gk, rk in (("dx", "dx"), ("dw1", "dW1"), ("dw3", "dW3"), ("dw2", "dW2"), ("dw", "dw")):
-        assert_close(to_np(g[gk]), ref[rk], f"{rk} {w.describe()}", max_abs_rms=tol)
+        assert_close(to_np(g[gk]), ref[rk], f"{rk} {w.describe()}", max_abs_rms=tol[rk])
     counts = np.bincount(top.ravel(), minlength=w.E)
     for e in np.nonzero(counts == 0)[0]:  # experts without tokens: exact zeros
         assert (g["dw1"][e] == 0).all() and (g["dw3"][e] == 0).all() and (g["dw2"][e] == 0).all()
@@ -129,9 +132,12 @@ def test_backward_steps_against_float64(w):
             assert torch.allclose(got, ref, rtol=1e-4, atol=1e-5 * (ref.abs().max().item() + 1e-30)), (n, e)
 
 
-def test_backward_skewed_full_size_sampled():
-    """The skewed fwd+bwd workload at full size: sampled dx / dw tokens and sampled weight-
-    gradient elements (heavy, light and empty experts) against the oracle."""
+def test_backward_skewed_full_size():
+    """The skewed fwd+bwd workload at full size.  dx and dw for the tokens whose entries hold
+    the first real row of every 128-row block (every tile of the dH and dX GEMMs) plus random
+    tokens; whole dW1, dW3, dW2 slabs for the heaviest expert (its K loop runs over hundreds of
+    row blocks), three light experts and an expert with an odd number of row blocks (its last
+    pair has an empty half); exact zeros for the experts without tokens."""
     w = WORKLOADS[5]
     inp = make_inputs(w, with_dy=True)
     dims = dims_of(w)
@@ -142,31 +148,30 @@ def test_backward_skewed_full_size_sampled():
     o = {k: inp[k].float().numpy() for k in ("x", "dy", "w1", "w3", "w2")}
     top, wts = oracle.route(inp["logits"].float().numpy(), w.top_k)
     assert (bufs.map.top_experts.cpu().numpy() == top).all()
-    toks = sample_tokens(top, w.E, 48, seed=5)
+    m = oracle.sparse_map(top, w.E)
+    toks = tokens_covering_blocks(m, w.top_k, w.T, 512, seed=5, last_rows=False)
+    assert len(np.unique(m["dest_row"].reshape(w.T, w.top_k)[toks] // 128)) == m["num_blocks"]
+    nt = oracle.max_threads()
     dx_ref, dw_ref = oracle.backward_tokens(o["x"], o["dy"], o["w1"], o["w3"], o["w2"], top, wts,
-                                            toks, threads=oracle.max_threads())
-    assert_close(to_np(g["dx"])[toks], dx_ref, "dx sampled")
-    assert_close(to_np(g["dw"])[toks], dw_ref, "dw sampled")
+                                            toks, threads=nt)
+    assert_close(to_np(g["dx"])[toks], dx_ref, f"dx ({len(toks)} tokens)")
+    assert_close(to_np(g["dw"])[toks], dw_ref, f"dw ({len(toks)} tokens)")
     counts = np.bincount(top.ravel(), minlength=w.E)
-    empty = np.nonzero(counts == 0)[0]
-    for e in empty:
-        assert (g["dw1"][e] == 0).all() and (g["dw2"][e] == 0).all()
-    rng = np.random.default_rng(55)
+    for e in np.nonzero(counts == 0)[0]:
+        for n in ("dw1", "dw3", "dw2"):
+            assert (g[n][e] == 0).all(), (n, e)
+    blocks = (counts + 127) // 128
     heavy = int(np.argmax(counts))
     light = [int(e) for e in np.nonzero((counts > 0) & (counts < 200))[0][:3]]
-    experts = [heavy] + light + [int(e) for e in rng.choice(np.nonzero(counts > 0)[0], 4)]
-    q = []
-    for e in experts:
-        for _ in range(3):
-            q.append((1, e, rng.integers(w.ffn), rng.integers(w.hidden)))
-            q.append((3, e, rng.integers(w.ffn), rng.integers(w.hidden)))
-            q.append((2, e, rng.integers(w.hidden), rng.integers(w.ffn)))
-    q = np.array(q, np.int32)
-    ref = oracle.wgrad_elements(o["x"], o["dy"], o["w1"], o["w3"], o["w2"], top, wts, q,
-                                threads=oracle.max_threads())
-    gm = {1: g["dw1"], 3: g["dw3"], 2: g["dw2"]}
-    got = np.array([float(gm[a][b, c, d]) for a, b, c, d in q])
-    assert_close(got, ref, "sampled weight-gradient elements")
+    odd = sorted((int(e) for e in np.nonzero((blocks % 2 == 1) & (blocks > 1))[0] if e != heavy),
+                 key=lambda e: blocks[e])[:1]  # the cheapest such expert for the oracle
+    assert len(light) == 3 and len(odd) == 1
+    for e in [heavy] + light + odd:
+        d1, d3, d2 = oracle.wgrad_expert(o["x"], o["dy"], o["w1"], o["w3"], o["w2"], top, wts, e,
+                                         threads=nt)
+        for got, ref, n in ((g["dw1"][e], d1, "dW1"), (g["dw3"][e], d3, "dW3"),
+                            (g["dw2"][e], d2, "dW2")):
+            assert_close(to_np(got), ref, f"{n} expert {e} ({counts[e]} entries)")
 
 
 def test_backward_deterministic():

@@ -11,7 +11,8 @@ Forward  -- closed form with permutation/selection weights (catches transposed o
             (textbook gated MLP); invariance under relabelling experts.
 Backward -- central finite differences of the oracle's own forward (in double) for x, W1,
             W3, W2 and the routing weights; dw = <dy, y_ts>; linearity in dy; the sampled
-            routines against the full backward.
+            routines against the full backward; whole per-expert weight-gradient slabs
+            against torch float64 autograd of the layer's composition.
 Router   -- logits: one-hot tokens read a column of the router weight (closed form), numpy's
             float64 matmul (library); gradient through the routing weights: central finite
             differences of sum dw * softmax(x Wr^T)[picks] in the logits, x and Wr; torch
@@ -373,6 +374,36 @@ def test_backward_sampled_routines_match_full(oracle_mod):
     full = {1: g["dW1"], 3: g["dW3"], 2: g["dW2"]}
     ref = np.array([full[a][b, c, d] for a, b, c, d in q])
     np.testing.assert_allclose(vals, ref, rtol=1e-11, atol=1e-14)
+
+
+def test_wgrad_expert_slabs_against_autograd(oracle_mod):
+    """Whole per-expert weight-gradient slabs against torch float64 autograd of the layer's
+    composition y = sum_s w_ts W2_e(silu(W1_e x_t) * W3_e x_t), loss = <dy, y>; and the
+    same bits as the full backward's slabs (one ordered sum per element)."""
+    rng = np.random.default_rng(37)
+    T, h, f, E, k = 40, 24, 16, 5, 3
+    x, W1, W3, W2, logits = _rand_layer(rng, T, h, f, E, k, scale=0.2)
+    dy = rng.standard_normal((T, h)).astype(np.float32)
+    top, w = oracle_mod.route(logits, k)
+    tw = [torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (W1, W3, W2)]
+    tx, tdy = torch.tensor(x, dtype=torch.float64), torch.tensor(dy, dtype=torch.float64)
+    idx = torch.tensor(top, dtype=torch.long)
+    a = torch.einsum("tkfh,th->tkf", tw[0][idx], tx)
+    b = torch.einsum("tkfh,th->tkf", tw[1][idx], tx)
+    yts = torch.einsum("tkhf,tkf->tkh", tw[2][idx], torch.nn.functional.silu(a) * b)
+    y = (torch.tensor(w) [:, :, None] * yts).sum(1)
+    (y * tdy).sum().backward()
+    full = oracle_mod.backward(x, dy, W1, W3, W2, top, w)
+    counts = np.bincount(top.ravel(), minlength=E)
+    for e in range(E):
+        d1, d3, d2 = oracle_mod.wgrad_expert(x, dy, W1, W3, W2, top, w, e, threads=3)
+        for got, ref, n in ((d1, tw[0].grad[e], "dW1"), (d3, tw[1].grad[e], "dW3"),
+                            (d2, tw[2].grad[e], "dW2")):
+            np.testing.assert_allclose(got, ref.numpy(), rtol=1e-10, atol=1e-12, err_msg=(n, e))
+        assert (d1 == full["dW1"][e]).all() and (d3 == full["dW3"][e]).all()
+        assert (d2 == full["dW2"][e]).all()
+        if counts[e] == 0:
+            assert not d1.any() and not d3.any() and not d2.any()
 
 
 # ----------------------------------------------------------------------------------------

@@ -5,11 +5,25 @@ import numpy as np
 import pytest
 import torch
 
+import bf16_model
 import oracle
 from dropless_mixture_experts_dmoe_b200 import binding as B
 from dropless_mixture_experts_dmoe_b200.workloads import custom, make_inputs
 
-from helpers import MAX_ABS_RMS_STRESS, assert_close, dims_of, sample_tokens, to_np
+from helpers import assert_close, dims_of, sample_tokens, to_np
+
+
+def assert_increment_close(got_total, base, ref_inc, what):
+    """The router adds its dx increment to the experts' dx in fp32 and rounds the total once
+    to bf16, so the increment read back as total - base carries that rounding: up to half a
+    bf16 ulp of the total, which can be far above the increment's own size.  Each element must
+    be within that plus 5e-2 of the increment's RMS, and the relative L2 error within 1e-2."""
+    inc = got_total - base
+    rms = float(np.sqrt(np.mean(ref_inc * ref_inc)))
+    bound = 2.0 ** -8 * np.abs(got_total) + 5e-2 * rms
+    assert (np.abs(inc - ref_inc) <= bound).all(), what
+    rel = float(np.linalg.norm(inc - ref_inc) / np.linalg.norm(ref_inc))
+    assert rel <= 1e-2, f"{what}: relative L2 {rel:.3e}"
 
 pytestmark = pytest.mark.gpu
 
@@ -94,9 +108,10 @@ def test_router_backward_full_chain_parity(w, renorm):
     ref = oracle.backward(o["x"], o["dy"], o["w1"], o["w3"], o["w2"], top, wts)
     r = oracle.router_backward(o["x"], o["w_router"], lg, top, ref["dw"],
                                threads=oracle.max_threads(), renorm=renorm)
+    tol = bf16_model.bounds(bf16_model.backward_model(inp, top, wts), ref)["dx"]
     assert_close(to_np(g["dx"]), ref["dx"] + r["dx_r"], f"dx {w.describe()}",
-                 max_abs_rms=MAX_ABS_RMS_STRESS)
-    assert_close(to_np(dwr), r["dWr"], f"dW_r {w.describe()}", max_abs_rms=MAX_ABS_RMS_STRESS)
+                 max_abs_rms=max(tol, 5e-2))
+    assert_close(to_np(dwr), r["dWr"], f"dW_r {w.describe()}")
 
 
 @pytest.mark.parametrize("renorm", [False, True], ids=["softmax", "renormalised"])
@@ -119,9 +134,8 @@ def test_router_steps_against_oracle_on_gpu_inputs(w, renorm):
     # fp32 softmax, then one bf16 rounding
     assert (np.abs(got - ref) <= 2.0 ** -7 * np.abs(ref) + 1e-4 * np.abs(ref).max()).all()
     # the dx increment: its rounding adds at most one bf16 ulp of the sum
-    inc = to_np(g["dx"]) - to_np(dx_experts)
-    assert_close(inc, r["dx_r"], "dx_r", max_abs_rms=MAX_ABS_RMS_STRESS)
-    assert_close(to_np(dwr), r["dWr"], "dW_r", max_abs_rms=MAX_ABS_RMS_STRESS)
+    assert_increment_close(to_np(g["dx"]), to_np(dx_experts), r["dx_r"], "dx_r")
+    assert_close(to_np(dwr), r["dWr"], "dW_r")
 
 
 def test_router_backward_deterministic_and_full_size_sampled():
@@ -143,6 +157,5 @@ def test_router_backward_deterministic_and_full_size_sampled():
     r = oracle.router_backward(inp["x"].float().numpy(), inp["w_router"].float().numpy(), lg, top,
                                g["dw"].double().cpu().numpy(), tokens=toks, elems=el,
                                threads=oracle.max_threads())
-    inc = (to_np(g["dx"]) - to_np(dx_experts))[toks]
-    assert_close(inc, r["dx_r"], "dx_r sampled", max_abs_rms=MAX_ABS_RMS_STRESS)
+    assert_increment_close(to_np(g["dx"])[toks], to_np(dx_experts)[toks], r["dx_r"], "dx_r sampled")
     assert_close(to_np(dwr)[el[:, 0], el[:, 1]], r["dWr"], "dW_r sampled")
