@@ -354,7 +354,7 @@ class Buffers:
             self.bstep = dict(dy_pad=torch.empty((P, h), **bf), da=torch.empty((P, f), **bf),
                               dbm=torch.empty((P, f), **bf), hw=torch.empty((P, f), **bf),
                               dw_part=torch.empty((P, nt), dtype=torch.float32, device=device),
-                              dx_pad=torch.empty((P, h), **bf))
+                              dx_pad=torch.empty((P, h), dtype=torch.float32, device=device))
         else:
             self.ws_fwd = torch.empty(dmoe_workspace_bytes(dims, WS_FORWARD), **u8)
             self.step = dict(x_pad=torch.empty((P, h), **bf), h=torch.empty((P, f), **bf),

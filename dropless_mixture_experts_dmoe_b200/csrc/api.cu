@@ -90,8 +90,9 @@ GemmProblem problem_of(const dmoe_dims *d, const dmoe_map *m) {
 
 inline int dglu_tiles(const dmoe_dims *d) { return (d->ffn + kDgluTileCols - 1) / kDgluTileCols; }
 
-// Backward workspace layout: dY_pad [P,h] (reused for dX_pad once the weight gradients have
-// read it) | dA [P,f] | dBm [P,f] | Hw [P,f] | routing-weight partials [P, ceil(f/256)] fp32
+// Backward workspace layout: dY_pad [P,h] bf16, whose region is reused for dX_pad [P,h] fp32
+// once the weight gradients have read dY_pad | dA [P,f] | dBm [P,f] | Hw [P,f] | routing-weight
+// partials [P, ceil(f/256)] fp32
 struct BwdLayout {
   size_t dy, da, db, hw, part, total;
 };
@@ -99,7 +100,7 @@ BwdLayout bwd_layout(const dmoe_dims *d) {
   const size_t P = (size_t)pmax_of(d);
   BwdLayout l;
   l.dy = 0;
-  l.da = align_up(l.dy + P * d->hidden * 2);
+  l.da = align_up(l.dy + P * d->hidden * 4);
   l.db = align_up(l.da + P * d->ffn * 2);
   l.hw = align_up(l.db + P * d->ffn * 2);
   l.part = align_up(l.hw + P * d->ffn * 2);
@@ -339,7 +340,8 @@ int dmoe_bwd_scatter(const dmoe_dims *dims, const void *dx_pad, const float *dw_
   if (!dx_pad || !dw_part || !dx || !dweights) return DMOE_ERR_NULL;
   if (!aligned16(dx_pad) || !aligned16(dx)) return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
-  return launch_rc(launch_bwd_scatter(dims->T, dims->hidden, dims->top_k, dx_pad, map->dest_row,
+  return launch_rc(launch_bwd_scatter(dims->T, dims->hidden, dims->top_k,
+                                      static_cast<const float *>(dx_pad), map->dest_row,
                                       dw_part, dglu_tiles(dims), dx, dweights,
                                       static_cast<cudaStream_t>(stream)));
 }
@@ -391,7 +393,8 @@ int dmoe_backward(const dmoe_dims *dims, const void *dy, const void *w1, const v
   uint8_t *w = static_cast<uint8_t *>(ws);
   void *dypad = w + l.dy, *da = w + l.da, *db = w + l.db, *hw = w + l.hw;
   float *part = reinterpret_cast<float *>(w + l.part);
-  void *dxpad = dypad;  // dY_pad is dead once the weight gradients have read it
+  void *dxpad = dypad;  // dY_pad is dead once the weight gradients have read it (dX_pad is
+                        // fp32, twice its size: the region is sized for it)
   if ((rc = dmoe_padded_gather(dims, dy, map, dypad, stream))) return rc;
   if ((rc = dmoe_bwd_dglu(dims, dypad, w2, abuf, bbuf, map, da, db, hw, part, stream))) return rc;
   if ((rc = dmoe_bwd_wgrad(dims, xpad, hw, dypad, da, db, map, dw1, dw3, dw2, stream))) return rc;

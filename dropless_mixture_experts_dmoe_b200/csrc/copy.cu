@@ -85,10 +85,6 @@ __global__ void __launch_bounds__(kCopyThreads) k_gather(int T, int h, int k, in
 
 // y_t = sum_{s<k} w_ts * Y_pad[dest_row[t*k+s]]: fp32, slot order, one fused multiply-add per
 // slot and element, rounded once to bf16.  weights == NULL: w = 1.
-// Backward use (walkthrough section 4.2: the gradient of the gather is this scatter with w = 1,
-// and the routing weight's gradient is <dy_t, Y_ts>): with dweights != NULL the warp that
-// takes a token's first slice also sums the DGLU GEMM's per-column-tile partials of each entry,
-// dweights[t*k+s] = sum_{n<nt} part[dest_row[t*k+s] * nt + n], in column-tile order.
 // VPL 16-byte vectors per lane for each of SLOTS slots are loaded before any is consumed
 // (VPL * SLOTS = 16 loads in flight per lane): few slots (small top_k) take wide row pieces.
 template <int VPL, int SLOTS>
@@ -96,9 +92,7 @@ __global__ void __launch_bounds__(kCopyThreads) k_combine(int T, int h, int k,
                                                           const uint4 *__restrict__ y_pad,
                                                           const int32_t *__restrict__ dest_row,
                                                           const float *__restrict__ weights,
-                                                          uint4 *__restrict__ y,
-                                                          const float *__restrict__ part, int nt,
-                                                          float *__restrict__ dweights) {
+                                                          uint4 *__restrict__ y) {
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
@@ -113,12 +107,6 @@ __global__ void __launch_bounds__(kCopyThreads) k_combine(int T, int h, int k,
     const int ve = min(vpr, vs + kSliceVecs);
     const int d = (lane < k) ? dest_row[(size_t)t * k + lane] : -1;
     const float wl = (lane < k) ? (weights ? weights[(size_t)t * k + lane] : 1.0f) : 0.0f;
-    if (dweights && vs == 0 && lane < k) {
-      float g = 0.0f;
-      if (d >= 0)
-        for (int n = 0; n < nt; ++n) g += __ldg(part + (size_t)d * nt + n);
-      dweights[(size_t)t * k + lane] = g;  // 0 for an entry dropped from the map
-    }
     for (int v0 = vs; v0 < ve; v0 += 32 * VPL) {
       float acc[VPL][8];
 #pragma unroll
@@ -173,6 +161,83 @@ __global__ void __launch_bounds__(kCopyThreads) k_combine(int T, int h, int k,
   }
 }
 
+// Backward scatter-sum over fp32 rows: dx_t = sum_{s<k} dX_pad[dest_row[t*k+s]] in fp32, slot
+// order, rounded once to bf16 (the gradient of the gather, walkthrough section 4.2), and the
+// routing-weight gradient dweights[t*k+s] = sum_{n<nt} part[dest_row[t*k+s] * nt + n] in
+// column-tile order.  A lane covers 4 consecutive columns (one 16-byte fp32 vector per slot);
+// VPL such vectors per lane and SLOTS slots are loaded before any is consumed.
+template <int VPL, int SLOTS>
+__global__ void __launch_bounds__(kCopyThreads) k_scatter_sum32(int T, int h, int k,
+                                                                const float4 *__restrict__ dx_pad,
+                                                                const int32_t *__restrict__ dest_row,
+                                                                uint2 *__restrict__ dx,
+                                                                const float *__restrict__ part,
+                                                                int nt,
+                                                                float *__restrict__ dweights) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int vpr = h >> 2;  // fp32 vectors of 4 per row
+  constexpr int kSlice = 32 * VPL;
+  const int S = (vpr + kSlice - 1) / kSlice;
+  const long long items = (long long)T * S;
+  const long long nw = (long long)gridDim.x * kCopyWarps;
+  for (long long it = (long long)blockIdx.x * kCopyWarps + (threadIdx.x >> 5); it < items;
+       it += nw) {
+    const int t = (int)(it / S);
+    const int v0 = (int)(it - (long long)t * S) * kSlice;
+    const int d = (lane < k) ? dest_row[(size_t)t * k + lane] : -1;
+    if (v0 == 0 && lane < k) {
+      float g = 0.0f;
+      if (d >= 0)
+        for (int n = 0; n < nt; ++n) g += __ldg(part + (size_t)d * nt + n);
+      dweights[(size_t)t * k + lane] = g;  // 0 for an entry dropped from the map
+    }
+    float4 acc[VPL];
+#pragma unroll
+    for (int u = 0; u < VPL; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < k; s0 += SLOTS) {
+      float4 buf[SLOTS][VPL];
+#pragma unroll
+      for (int ss = 0; ss < SLOTS; ++ss) {
+        const int s = s0 + ss;
+        const int r = __shfl_sync(0xFFFFFFFFu, d, s & 31);
+        if (s < k && r >= 0) {
+#pragma unroll
+          for (int u = 0; u < VPL; ++u) {
+            const int v = v0 + u * 32 + lane;
+            if (v < vpr) {
+              const uint4 q = ld_nc_v4(reinterpret_cast<const uint4 *>(dx_pad + (size_t)r * vpr + v));
+              buf[ss][u] = make_float4(__uint_as_float(q.x), __uint_as_float(q.y),
+                                       __uint_as_float(q.z), __uint_as_float(q.w));
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int ss = 0; ss < SLOTS; ++ss) {
+        const int s = s0 + ss;
+        const int r = __shfl_sync(0xFFFFFFFFu, d, s & 31);
+        if (s < k && r >= 0) {
+#pragma unroll
+          for (int u = 0; u < VPL; ++u) {
+            acc[u].x = __fadd_rn(acc[u].x, buf[ss][u].x);
+            acc[u].y = __fadd_rn(acc[u].y, buf[ss][u].y);
+            acc[u].z = __fadd_rn(acc[u].z, buf[ss][u].z);
+            acc[u].w = __fadd_rn(acc[u].w, buf[ss][u].w);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < VPL; ++u) {
+      const int v = v0 + u * 32 + lane;
+      if (v < vpr) dx[(size_t)t * vpr + v] = make_uint2(pack_bf16x2(acc[u].x, acc[u].y),
+                                                        pack_bf16x2(acc[u].z, acc[u].w));
+    }
+  }
+}
+
 static int copy_grid(long long items) {
   const long long per_cta = kCopyWarps;
   long long want = (items + per_cta - 1) / per_cta;
@@ -192,26 +257,25 @@ cudaError_t launch_gather(int T, int h, int k, int E, const void *x, const int32
                     static_cast<uint4 *>(x_pad));
 }
 
-static cudaError_t combine(int T, int h, int k, const void *y_pad, const int32_t *dest_row,
-                           const float *weights, void *y, const float *part, int nt,
-                           float *dweights, cudaStream_t st) {
+cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const int32_t *dest_row,
+                           const float *weights, void *y, cudaStream_t st) {
   const int grid = copy_grid((long long)T * slices(h));
   const uint4 *src = static_cast<const uint4 *>(y_pad);
   uint4 *dst = static_cast<uint4 *>(y);
   auto kernel = (k <= 2) ? k_combine<8, 2> : (k <= 4) ? k_combine<4, 4> : k_combine<2, 8>;
-  return launch_pdl(kernel, grid, kCopyThreads, 0, st, T, h, k, src, dest_row, weights, dst, part,
-                    nt, dweights);
+  return launch_pdl(kernel, grid, kCopyThreads, 0, st, T, h, k, src, dest_row, weights, dst);
 }
 
-cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const int32_t *dest_row,
-                           const float *weights, void *y, cudaStream_t st) {
-  return combine(T, h, k, y_pad, dest_row, weights, y, nullptr, 0, nullptr, st);
-}
-
-cudaError_t launch_bwd_scatter(int T, int h, int k, const void *dx_pad, const int32_t *dest_row,
+cudaError_t launch_bwd_scatter(int T, int h, int k, const float *dx_pad, const int32_t *dest_row,
                                const float *part, int nt, void *dx, float *dweights,
                                cudaStream_t st) {
-  return combine(T, h, k, dx_pad, dest_row, nullptr, dx, part, nt, dweights, st);
+  const int vpl = (k <= 2) ? 8 : (k <= 4) ? 4 : 2;  // 16-byte vectors per lane and slot
+  auto kernel = (k <= 2) ? k_scatter_sum32<8, 2> : (k <= 4) ? k_scatter_sum32<4, 4>
+                                                            : k_scatter_sum32<2, 8>;
+  const long long items = (long long)T * (((h >> 2) + 32 * vpl - 1) / (32 * vpl));
+  return launch_pdl(kernel, copy_grid(items), kCopyThreads, 0, st, T, h, k,
+                    reinterpret_cast<const float4 *>(dx_pad), dest_row, static_cast<uint2 *>(dx),
+                    part, nt, dweights);
 }
 
 }  // namespace dmoe

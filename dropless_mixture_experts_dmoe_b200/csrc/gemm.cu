@@ -53,7 +53,9 @@
 //         A, Bm (s = sigmoid(A), h = A*s*Bm) and, with w the routing weight of the row, writes
 //         dA = w*G*Bm*s*(1+A(1-s)), dBm = w*G*A*s, Hw = w*h (the dW2 operand) and the partial
 //         routing-weight gradient sum_cols G*h of the row over the tile's columns
-//   DX    A = dA then dBm (K), B = W1_e then W3_e (MN), one accumulator over both K passes
+//   DX    A = dA then dBm (K), B = W1_e then W3_e (MN), one accumulator over both K passes;
+//         out dX_pad in fp32 (the k rows of a token are summed afterwards: rounding each of
+//         them to bf16 first would put k roundings into every dx element)
 //   WGRAD dW1_e = dA^T X_pad, dW3_e = dBm^T X_pad, dW2_e = dY_pad^T Hw over the expert's
 //         padded rows (both operands MN-major); fp32 outputs; experts without rows get exact
 //         zeros.
@@ -468,7 +470,23 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
         st.emit(&p.tmo[2], w, n0 + c, y0);
       }
     }
-  } else if (MODE == MODE_DOWN || MODE == MODE_DX) {
+  } else if (MODE == MODE_DX) {  // fp32 dX_pad rows, boxes of 32 columns
+    const int n0 = tl.n * BN + half * kw;
+    const int ncols = min(kw, p.h - n0);  // multiple of 64 (may be <= 0)
+    if (ncols <= 0) return;
+    tb += (uint32_t)(half * kw);
+    uint32_t v[32], w[32];
+    tmem_ld32(tb, v);
+    tmem_ld_wait();
+#pragma unroll 1
+    for (int c = 0; c < ncols; c += 32) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) w[i] = v[i];
+      if (c + 32 < ncols) tmem_ld32(tb + c + 32, v);  // overlaps the store
+      st.emit(&p.tmo[0], w, n0 + c, y0);
+      tmem_ld_wait();
+    }
+  } else if (MODE == MODE_DOWN) {
     const int n0 = tl.n * BN + half * kw;  // this warp's first column
     const int ncols = min(kw, p.h - n0);   // multiple of 64 (may be <= 0)
     if (ncols <= 0) return;
@@ -1123,7 +1141,7 @@ cudaError_t launch_dx_gemm(const GemmProblem &g, const void *da, const void *db,
       !make_tmap_chunked(&p.tm[1], db, P, g.f, BM) ||
       !make_tmap_chunked(&p.tm[2], w1, EF, g.h, 2 * BK) ||
       !make_tmap_chunked(&p.tm[3], w3, EF, g.h, 2 * BK) ||
-      !make_tmap(&p.tmo[0], dx_pad, P, g.h, 32))
+      !make_tmap(&p.tmo[0], dx_pad, P, g.h, 32, 4))
     return cudaErrorInvalidValue;
   p.tm[4] = p.tm[0];
   p.n_tiles = (g.h + BN - 1) / BN;

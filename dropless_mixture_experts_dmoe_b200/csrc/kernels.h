@@ -54,9 +54,9 @@ cudaError_t launch_gather(int T, int h, int k, int E, const void *x, const int32
 cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const int32_t *dest_row,
                            const float *weights, void *y, cudaStream_t st);
 
-// Backward scatter: dx_t = sum_s dX_pad[dest_row[t*k+s]] and, from the DGLU GEMM's partial
-// sums part [P_max, nt], dweights[t*k+s] = sum_n part[dest_row[t*k+s]][n].
-cudaError_t launch_bwd_scatter(int T, int h, int k, const void *dx_pad, const int32_t *dest_row,
+// Backward scatter: dx_t = bf16(sum_s dX_pad[dest_row[t*k+s]]) over fp32 rows and, from the
+// DGLU GEMM's partial sums part [P_max, nt], dweights[t*k+s] = sum_n part[dest_row[t*k+s]][n].
+cudaError_t launch_bwd_scatter(int T, int h, int k, const float *dx_pad, const int32_t *dest_row,
                                const float *part, int nt, void *dx, float *dweights,
                                cudaStream_t st);
 

@@ -287,8 +287,10 @@ DMOE_API int dmoe_bwd_dglu(const dmoe_dims *dims, const void *dy_pad, const void
                            const void *a_saved, const void *bm_saved, const dmoe_map *map,
                            void *da, void *dbm, void *hw, float *dw_part, void *stream);
 
-/* dX GEMM: dX_pad[b] = bf16(dA[b] W1_e + dBm[b] W3_e), one fp32 accumulator over both K
- * passes.  da, dbm [P_max,f] -> dx_pad [P_max,h]. */
+/* dX GEMM: dX_pad[b] = dA[b] W1_e + dBm[b] W3_e, one fp32 accumulator over both K passes,
+ * stored in fp32: the k rows of a token are summed by dmoe_bwd_scatter, and rounding each of
+ * them to bf16 first would put k roundings into every element of dx.
+ * da, dbm [P_max,f] bf16 -> dx_pad [P_max,h] fp32. */
 DMOE_API int dmoe_bwd_dx(const dmoe_dims *dims, const void *da, const void *dbm, const void *w1,
                          const void *w3, const dmoe_map *map, void *dx_pad, void *stream);
 
@@ -308,7 +310,8 @@ DMOE_API int dmoe_bwd_wgrad(const dmoe_dims *dims, const void *x_pad, const void
  *   dx_t = bf16(sum_s dX_pad[dest_row[t*k+s]])  (fp32 sum in slot order),
  *   dweights[t*k+s] = sum_{n < nt} dw_part[dest_row[t*k+s] * nt + n]  (fp32, tile order; 0 for
  *   an entry dropped from the map).
- * dx_pad [P_max,h] bf16, dw_part from dmoe_bwd_dglu -> dx [T,h] bf16, dweights [T,k] fp32. */
+ * dx_pad [P_max,h] fp32 (from dmoe_bwd_dx), dw_part from dmoe_bwd_dglu -> dx [T,h] bf16,
+ * dweights [T,k] fp32. */
 DMOE_API int dmoe_bwd_scatter(const dmoe_dims *dims, const void *dx_pad, const float *dw_part,
                               const dmoe_map *map, void *dx, float *dweights, void *stream);
 
