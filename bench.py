@@ -434,9 +434,11 @@ def run_ours(args, w):
             B.dmoe_bwd_wgrad(dims, xp, bs["hw"], bs["dy_pad"], bs["da"], bs["dbm"], bufs.map,
                              grads["dw1"], grads["dw3"], grads["dw2"], st)
             mark(i + 3)
-            B.dmoe_bwd_dx(dims, bs["da"], bs["dbm"], dev["w1"], dev["w3"], bufs.map, bs["dx_pad"], st)
+            B.dmoe_bwd_dx(dims, bs["da"], bs["dbm"], dev["w1"], dev["w3"], bufs.map, bs["dx_pad"],
+                          bs["dx_scale"], st)
             mark(i + 4)
-            B.dmoe_bwd_scatter(dims, bs["dx_pad"], bs["dw_part"], bufs.map, grads["dx"], grads["dw"], st)
+            B.dmoe_bwd_scatter(dims, bs["dx_pad"], bs["dx_scale"], bs["dw_part"], bufs.map,
+                               grads["dx"], grads["dw"], st)
             mark(i + 5)
             if router:  # dlogits, dx += dlogits W_r, dW_r (4 kernels)
                 B.dmoe_router_backward(dims, dev["x"], dev["w_router"], dev["logits"], bufs.map,
@@ -598,7 +600,7 @@ def run_ours(args, w):
         gather=2 * w.T * w.hidden + 2 * N * w.hidden,
         scatter=2 * N * w.hidden + 8 * N + 4 * N + 2 * w.T * w.hidden,
         dy_gather=2 * w.T * w.hidden + 2 * N * w.hidden,
-        dx_scatter=4 * N * w.hidden + 4 * N + 2 * w.T * w.hidden
+        dx_scatter=2 * N * w.hidden + 4 * N * ((w.hidden + 255) // 256) + 4 * N + 2 * w.T * w.hidden
         + 4 * N * ((w.ffn + 255) // 256) + 4 * N,
         # router: x and W_r read, logits written; backward: logits, dweights, top read, dlogits
         # written and read twice, dx read and written, x read, dW_r written

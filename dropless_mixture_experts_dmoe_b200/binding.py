@@ -22,6 +22,7 @@ MAX_TOP_K = 32
 
 WS_MAP, WS_FORWARD, WS_BACKWARD, WS_FORWARD_TRAIN, WS_ROUTER_BACKWARD = 0, 1, 2, 3, 4
 DGLU_TILE_COLS = 256
+DX_TILE_COLS = 256
 
 STATUS_NONFINITE_LOGITS = 0x1
 STATUS_EXPERT_OUT_OF_RANGE = 0x2
@@ -90,11 +91,11 @@ def load():
     lib.dmoe_expert_down.argtypes = [D, _P, _P, M, _P, _P]
     lib.dmoe_padded_scatter.argtypes = [D, _P, M, _P, _P, _P]
     lib.dmoe_bwd_dglu.argtypes = [D, _P, _P, _P, _P, M, _P, _P, _P, _P, _P]
-    lib.dmoe_bwd_scatter.argtypes = [D, _P, _P, M, _P, _P, _P]
+    lib.dmoe_bwd_scatter.argtypes = [D, _P, _P, _P, M, _P, _P, _P]
     lib.dmoe_router_forward.argtypes = [D, _P, _P, _P, _P, _P]
     lib.dmoe_router_dlogits.argtypes = [D, _P, M, _P, _P, _P]
     lib.dmoe_router_backward.argtypes = [D, _P, _P, _P, M, _P, _P, _P, _P, _SZ, _P]
-    lib.dmoe_bwd_dx.argtypes = [D, _P, _P, _P, _P, M, _P, _P]
+    lib.dmoe_bwd_dx.argtypes = [D, _P, _P, _P, _P, M, _P, _P, _P]
     lib.dmoe_bwd_wgrad.argtypes = [D, _P, _P, _P, _P, _P, M, _P, _P, _P, _P]
     lib.dmoe_sparse_map_noalloc.argtypes = [D, _P, M, _P]
     for fn in ("dmoe_sparse_map", "dmoe_sparse_map_noalloc", "dmoe_forward", "dmoe_backward",
@@ -272,15 +273,18 @@ def dmoe_bwd_dglu(dims, dy_pad, w2, a_saved, bm_saved, smap: SparseMap, da, dbm,
                                 _ptr(hw), _ptr(dw_part), _stream(stream)), "dmoe_bwd_dglu")
 
 
-def dmoe_bwd_scatter(dims, dx_pad, dw_part, smap: SparseMap, dx, dweights, stream=None):
-    _check(load().dmoe_bwd_scatter(ctypes.byref(dims), _ptr(dx_pad), _ptr(dw_part),
-                                   ctypes.byref(smap.c), _ptr(dx), _ptr(dweights),
+def dmoe_bwd_scatter(dims, dx_pad, dx_scale, dw_part, smap: SparseMap, dx, dweights,
+                     stream=None):
+    _check(load().dmoe_bwd_scatter(ctypes.byref(dims), _ptr(dx_pad), _ptr(dx_scale),
+                                   _ptr(dw_part), ctypes.byref(smap.c), _ptr(dx), _ptr(dweights),
                                    _stream(stream)), "dmoe_bwd_scatter")
 
 
-def dmoe_bwd_dx(dims, da, dbm, w1, w3, smap: SparseMap, dx_pad, stream=None):
+def dmoe_bwd_dx(dims, da, dbm, w1, w3, smap: SparseMap, dx_pad, dx_scale, stream=None):
+    """dx_pad [P_max,h] fp16 and dx_scale [P_max, ceil(h/256)] fp32: block floating point."""
     _check(load().dmoe_bwd_dx(ctypes.byref(dims), _ptr(da), _ptr(dbm), _ptr(w1), _ptr(w3),
-                              ctypes.byref(smap.c), _ptr(dx_pad), _stream(stream)), "dmoe_bwd_dx")
+                              ctypes.byref(smap.c), _ptr(dx_pad), _ptr(dx_scale),
+                              _stream(stream)), "dmoe_bwd_dx")
 
 
 def dmoe_bwd_wgrad(dims, x_pad, hw, dy_pad, da, dbm, smap: SparseMap, dw1, dw3, dw2,
@@ -327,7 +331,7 @@ class Buffers:
 
     train=True: ``saved`` (X_pad, A, Bm for the backward), the training forward workspace
     ``ws_fwd`` (H, Y_pad), the backward workspace, and separate step buffers ``bstep``
-    (dy_pad, da, dbm, hw, dw_part, dx_pad) for driving the backward step entry points one by
+    (dy_pad, da, dbm, hw, dw_part, dx_pad, dx_scale) for driving the backward step entry points one by
     one.  train=False: the inference workspace of ``dmoe_forward`` plus separate X_pad / H /
     Y_pad tensors (``step``) for the forward step entry points.  ``view(name)`` gives bf16
     [P_max, cols] views: x_pad, a, bm of the saved buffer, and h, y_pad of the forward
@@ -354,7 +358,9 @@ class Buffers:
             self.bstep = dict(dy_pad=torch.empty((P, h), **bf), da=torch.empty((P, f), **bf),
                               dbm=torch.empty((P, f), **bf), hw=torch.empty((P, f), **bf),
                               dw_part=torch.empty((P, nt), dtype=torch.float32, device=device),
-                              dx_pad=torch.empty((P, h), dtype=torch.float32, device=device))
+                              dx_pad=torch.empty((P, h), dtype=torch.float16, device=device),
+                              dx_scale=torch.empty((P, (h + DX_TILE_COLS - 1) // DX_TILE_COLS),
+                                                   dtype=torch.float32, device=device))
         else:
             self.ws_fwd = torch.empty(dmoe_workspace_bytes(dims, WS_FORWARD), **u8)
             self.step = dict(x_pad=torch.empty((P, h), **bf), h=torch.empty((P, f), **bf),

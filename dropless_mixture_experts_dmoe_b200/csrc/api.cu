@@ -90,21 +90,24 @@ GemmProblem problem_of(const dmoe_dims *d, const dmoe_map *m) {
 
 inline int dglu_tiles(const dmoe_dims *d) { return (d->ffn + kDgluTileCols - 1) / kDgluTileCols; }
 
-// Backward workspace layout: dY_pad [P,h] bf16, whose region is reused for dX_pad [P,h] fp32
+inline int dx_tiles(const dmoe_dims *d) { return (d->hidden + kDxTileCols - 1) / kDxTileCols; }
+
+// Backward workspace layout: dY_pad [P,h] bf16, whose region is reused for dX_pad [P,h] fp16
 // once the weight gradients have read dY_pad | dA [P,f] | dBm [P,f] | Hw [P,f] | routing-weight
-// partials [P, ceil(f/256)] fp32
+// partials [P, ceil(f/256)] fp32 | dX_pad scales [P, ceil(h/256)] fp32
 struct BwdLayout {
-  size_t dy, da, db, hw, part, total;
+  size_t dy, da, db, hw, part, dxs, total;
 };
 BwdLayout bwd_layout(const dmoe_dims *d) {
   const size_t P = (size_t)pmax_of(d);
   BwdLayout l;
   l.dy = 0;
-  l.da = align_up(l.dy + P * d->hidden * 4);
+  l.da = align_up(l.dy + P * d->hidden * 2);
   l.db = align_up(l.da + P * d->ffn * 2);
   l.hw = align_up(l.db + P * d->ffn * 2);
   l.part = align_up(l.hw + P * d->ffn * 2);
-  l.total = align_up(l.part + P * dglu_tiles(d) * sizeof(float));
+  l.dxs = align_up(l.part + P * dglu_tiles(d) * sizeof(float));
+  l.total = align_up(l.dxs + P * dx_tiles(d) * sizeof(float));
   return l;
 }
 
@@ -332,31 +335,34 @@ int dmoe_bwd_dglu(const dmoe_dims *dims, const void *dy_pad, const void *w2, con
                                     hw, dw_part, static_cast<cudaStream_t>(stream)));
 }
 
-int dmoe_bwd_scatter(const dmoe_dims *dims, const void *dx_pad, const float *dw_part,
-                     const dmoe_map *map, void *dx, float *dweights, void *stream) {
+int dmoe_bwd_scatter(const dmoe_dims *dims, const void *dx_pad, const float *dx_scale,
+                     const float *dw_part, const dmoe_map *map, void *dx, float *dweights,
+                     void *stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_map(map, false))) return rc;
-  if (!dx_pad || !dw_part || !dx || !dweights) return DMOE_ERR_NULL;
+  if (!dx_pad || !dx_scale || !dw_part || !dx || !dweights) return DMOE_ERR_NULL;
   if (!aligned16(dx_pad) || !aligned16(dx)) return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
-  return launch_rc(launch_bwd_scatter(dims->T, dims->hidden, dims->top_k,
-                                      static_cast<const float *>(dx_pad), map->dest_row,
+  return launch_rc(launch_bwd_scatter(dims->T, dims->hidden, dims->top_k, dx_pad, dx_scale,
+                                      map->dest_row,
                                       dw_part, dglu_tiles(dims), dx, dweights,
                                       static_cast<cudaStream_t>(stream)));
 }
 
 int dmoe_bwd_dx(const dmoe_dims *dims, const void *da, const void *dbm, const void *w1,
-                const void *w3, const dmoe_map *map, void *dx_pad, void *stream) {
+                const void *w3, const dmoe_map *map, void *dx_pad, float *dx_scale,
+                void *stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_map(map, false))) return rc;
-  if (!da || !dbm || !w1 || !w3 || !dx_pad) return DMOE_ERR_NULL;
+  if (!da || !dbm || !w1 || !w3 || !dx_pad || !dx_scale) return DMOE_ERR_NULL;
   if (!aligned16(da) || !aligned16(dbm) || !aligned16(w1) || !aligned16(w3) || !aligned16(dx_pad))
     return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
   return launch_rc(
-      launch_dx_gemm(problem_of(dims, map), da, dbm, w1, w3, dx_pad, static_cast<cudaStream_t>(stream)));
+      launch_dx_gemm(problem_of(dims, map), da, dbm, w1, w3, dx_pad, dx_scale,
+                     static_cast<cudaStream_t>(stream)));
 }
 
 int dmoe_bwd_wgrad(const dmoe_dims *dims, const void *x_pad, const void *hw,
@@ -393,13 +399,13 @@ int dmoe_backward(const dmoe_dims *dims, const void *dy, const void *w1, const v
   uint8_t *w = static_cast<uint8_t *>(ws);
   void *dypad = w + l.dy, *da = w + l.da, *db = w + l.db, *hw = w + l.hw;
   float *part = reinterpret_cast<float *>(w + l.part);
-  void *dxpad = dypad;  // dY_pad is dead once the weight gradients have read it (dX_pad is
-                        // fp32, twice its size: the region is sized for it)
+  float *dxs = reinterpret_cast<float *>(w + l.dxs);
+  void *dxpad = dypad;  // dY_pad is dead once the weight gradients have read it
   if ((rc = dmoe_padded_gather(dims, dy, map, dypad, stream))) return rc;
   if ((rc = dmoe_bwd_dglu(dims, dypad, w2, abuf, bbuf, map, da, db, hw, part, stream))) return rc;
   if ((rc = dmoe_bwd_wgrad(dims, xpad, hw, dypad, da, db, map, dw1, dw3, dw2, stream))) return rc;
-  if ((rc = dmoe_bwd_dx(dims, da, db, w1, w3, map, dxpad, stream))) return rc;
-  return dmoe_bwd_scatter(dims, dxpad, part, map, dx, dweights, stream);
+  if ((rc = dmoe_bwd_dx(dims, da, db, w1, w3, map, dxpad, dxs, stream))) return rc;
+  return dmoe_bwd_scatter(dims, dxpad, dxs, part, map, dx, dweights, stream);
 }
 
 int dmoe_router_forward(const dmoe_dims *dims, const void *x, const void *w_router, void *logits,

@@ -161,23 +161,28 @@ __global__ void __launch_bounds__(kCopyThreads) k_combine(int T, int h, int k,
   }
 }
 
-// Backward scatter-sum over fp32 rows: dx_t = sum_{s<k} dX_pad[dest_row[t*k+s]] in fp32, slot
-// order, rounded once to bf16 (the gradient of the gather, walkthrough section 4.2), and the
-// routing-weight gradient dweights[t*k+s] = sum_{n<nt} part[dest_row[t*k+s] * nt + n] in
-// column-tile order.  A lane covers 4 consecutive columns (one 16-byte fp32 vector per slot);
-// VPL such vectors per lane and SLOTS slots are loaded before any is consumed.
+// Backward scatter-sum (the gradient of the gather, walkthrough section 4.2): dx_t =
+// bf16(sum_{s<k} dX_pad[dest_row[t*k+s]]) in fp32, slot order, rounded once.  dX_pad rows are
+// block floating point: fp16 values times a power-of-two scale per row and 256-column tile
+// (scale[r * nsc + c / 256]); fp16 * scale is exact in fp32, so each slot adds its value with
+// one fused multiply-add.  With it the routing-weight gradient dweights[t*k+s] =
+// sum_{n<nt} part[dest_row[t*k+s] * nt + n] in column-tile order.  A lane covers 8 consecutive
+// columns (one 16-byte vector) per slot; VPL such vectors per lane and SLOTS slots are loaded
+// before any is consumed.
 template <int VPL, int SLOTS>
-__global__ void __launch_bounds__(kCopyThreads) k_scatter_sum32(int T, int h, int k,
-                                                                const float4 *__restrict__ dx_pad,
-                                                                const int32_t *__restrict__ dest_row,
-                                                                uint2 *__restrict__ dx,
-                                                                const float *__restrict__ part,
-                                                                int nt,
-                                                                float *__restrict__ dweights) {
+__global__ void __launch_bounds__(kCopyThreads) k_scatter_sum(int T, int h, int k,
+                                                              const uint4 *__restrict__ dx_pad,
+                                                              const float *__restrict__ scale,
+                                                              const int32_t *__restrict__ dest_row,
+                                                              uint4 *__restrict__ dx,
+                                                              const float *__restrict__ part,
+                                                              int nt,
+                                                              float *__restrict__ dweights) {
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
-  const int vpr = h >> 2;  // fp32 vectors of 4 per row
+  const int vpr = h >> 3;      // 16-byte vectors (8 columns) per row
+  const int nsc = (h + 255) >> 8;  // scales per row
   constexpr int kSlice = 32 * VPL;
   const int S = (vpr + kSlice - 1) / kSlice;
   const long long items = (long long)T * S;
@@ -193,11 +198,14 @@ __global__ void __launch_bounds__(kCopyThreads) k_scatter_sum32(int T, int h, in
         for (int n = 0; n < nt; ++n) g += __ldg(part + (size_t)d * nt + n);
       dweights[(size_t)t * k + lane] = g;  // 0 for an entry dropped from the map
     }
-    float4 acc[VPL];
+    float acc[VPL][8];
 #pragma unroll
-    for (int u = 0; u < VPL; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < VPL; ++u)
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[u][q] = 0.0f;
     for (int s0 = 0; s0 < k; s0 += SLOTS) {
-      float4 buf[SLOTS][VPL];
+      uint4 buf[SLOTS][VPL];
+      float sc[SLOTS][VPL];
 #pragma unroll
       for (int ss = 0; ss < SLOTS; ++ss) {
         const int s = s0 + ss;
@@ -207,9 +215,8 @@ __global__ void __launch_bounds__(kCopyThreads) k_scatter_sum32(int T, int h, in
           for (int u = 0; u < VPL; ++u) {
             const int v = v0 + u * 32 + lane;
             if (v < vpr) {
-              const uint4 q = ld_nc_v4(reinterpret_cast<const uint4 *>(dx_pad + (size_t)r * vpr + v));
-              buf[ss][u] = make_float4(__uint_as_float(q.x), __uint_as_float(q.y),
-                                       __uint_as_float(q.z), __uint_as_float(q.w));
+              buf[ss][u] = ld_nc_v4(dx_pad + (size_t)r * vpr + v);
+              sc[ss][u] = __ldg(scale + (size_t)r * nsc + (v >> 5));
             }
           }
         }
@@ -221,10 +228,12 @@ __global__ void __launch_bounds__(kCopyThreads) k_scatter_sum32(int T, int h, in
         if (s < k && r >= 0) {
 #pragma unroll
           for (int u = 0; u < VPL; ++u) {
-            acc[u].x = __fadd_rn(acc[u].x, buf[ss][u].x);
-            acc[u].y = __fadd_rn(acc[u].y, buf[ss][u].y);
-            acc[u].z = __fadd_rn(acc[u].z, buf[ss][u].z);
-            acc[u].w = __fadd_rn(acc[u].w, buf[ss][u].w);
+            const uint32_t *q = reinterpret_cast<const uint32_t *>(&buf[ss][u]);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              acc[u][2 * p] = fmaf(f16_lo(q[p]), sc[ss][u], acc[u][2 * p]);
+              acc[u][2 * p + 1] = fmaf(f16_hi(q[p]), sc[ss][u], acc[u][2 * p + 1]);
+            }
           }
         }
       }
@@ -232,8 +241,14 @@ __global__ void __launch_bounds__(kCopyThreads) k_scatter_sum32(int T, int h, in
 #pragma unroll
     for (int u = 0; u < VPL; ++u) {
       const int v = v0 + u * 32 + lane;
-      if (v < vpr) dx[(size_t)t * vpr + v] = make_uint2(pack_bf16x2(acc[u].x, acc[u].y),
-                                                        pack_bf16x2(acc[u].z, acc[u].w));
+      if (v < vpr) {
+        uint4 o;
+        o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+        o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+        o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+        o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+        dx[(size_t)t * vpr + v] = o;
+      }
     }
   }
 }
@@ -266,16 +281,16 @@ cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const int32_t
   return launch_pdl(kernel, grid, kCopyThreads, 0, st, T, h, k, src, dest_row, weights, dst);
 }
 
-cudaError_t launch_bwd_scatter(int T, int h, int k, const float *dx_pad, const int32_t *dest_row,
-                               const float *part, int nt, void *dx, float *dweights,
-                               cudaStream_t st) {
+cudaError_t launch_bwd_scatter(int T, int h, int k, const void *dx_pad, const float *dx_scale,
+                               const int32_t *dest_row, const float *part, int nt, void *dx,
+                               float *dweights, cudaStream_t st) {
   const int vpl = (k <= 2) ? 8 : (k <= 4) ? 4 : 2;  // 16-byte vectors per lane and slot
-  auto kernel = (k <= 2) ? k_scatter_sum32<8, 2> : (k <= 4) ? k_scatter_sum32<4, 4>
-                                                            : k_scatter_sum32<2, 8>;
-  const long long items = (long long)T * (((h >> 2) + 32 * vpl - 1) / (32 * vpl));
+  auto kernel = (k <= 2) ? k_scatter_sum<8, 2> : (k <= 4) ? k_scatter_sum<4, 4>
+                                                          : k_scatter_sum<2, 8>;
+  const long long items = (long long)T * (((h >> 3) + 32 * vpl - 1) / (32 * vpl));
   return launch_pdl(kernel, copy_grid(items), kCopyThreads, 0, st, T, h, k,
-                    reinterpret_cast<const float4 *>(dx_pad), dest_row, static_cast<uint2 *>(dx),
-                    part, nt, dweights);
+                    static_cast<const uint4 *>(dx_pad), dx_scale, dest_row,
+                    static_cast<uint4 *>(dx), part, nt, dweights);
 }
 
 }  // namespace dmoe

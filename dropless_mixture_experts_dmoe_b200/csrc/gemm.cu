@@ -54,8 +54,9 @@
 //         dA = w*G*Bm*s*(1+A(1-s)), dBm = w*G*A*s, Hw = w*h (the dW2 operand) and the partial
 //         routing-weight gradient sum_cols G*h of the row over the tile's columns
 //   DX    A = dA then dBm (K), B = W1_e then W3_e (MN), one accumulator over both K passes;
-//         out dX_pad in fp32 (the k rows of a token are summed afterwards: rounding each of
-//         them to bf16 first would put k roundings into every dx element)
+//         out dX_pad as fp16 with a power-of-two scale per row and 256-column tile (the k
+//         rows of a token are summed afterwards; rounding each of them to bf16 first would put
+//         k bf16 roundings into every dx element)
 //   WGRAD dW1_e = dA^T X_pad, dW3_e = dBm^T X_pad, dW2_e = dY_pad^T Hw over the expert's
 //         padded rows (both operands MN-major); fp32 outputs; experts without rows get exact
 //         zeros.
@@ -175,7 +176,8 @@ struct GemmParams {
   long long wait_cycles;  // budget of every bounded wait of this launch
   const __nv_bfloat16 *in0, *in1;  // DGLU: saved A, Bm
   const float *weights;            // DGLU: routing weight of each flattened entry
-  float *part;                     // DGLU: [P_max, n_tiles] partial routing-weight gradients
+  float *part;                     // DGLU: [P_max, n_tiles] partial routing-weight gradients;
+                                   // DX: [P_max, n_tiles] inverse scales of the dX_pad rows
   int total;                       // router modes: number of pair tiles
   int split_k;                     // RWGRAD: 64-wide K steps per split
   int Ep;                          // RWGRAD: rows of one split's slab (E rounded up to 128)
@@ -470,21 +472,41 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
         st.emit(&p.tmo[2], w, n0 + c, y0);
       }
     }
-  } else if (MODE == MODE_DX) {  // fp32 dX_pad rows, boxes of 32 columns
-    const int n0 = tl.n * BN + half * kw;
-    const int ncols = min(kw, p.h - n0);  // multiple of 64 (may be <= 0)
-    if (ncols <= 0) return;
-    tb += (uint32_t)(half * kw);
-    uint32_t v[32], w[32];
-    tmem_ld32(tb, v);
-    tmem_ld_wait();
+  } else if (MODE == MODE_DX) {
+    // dX_pad in block floating point: fp16 values with one power-of-two scale per row and
+    // 256-column tile, so that the largest value of the tile's row lands in [2^13, 2^14) and
+    // every value keeps fp16's 11 significant bits (bf16 has 8); the scale's inverse goes to
+    // p.part[row * n_tiles + n].  Pass 1 reads the row's accumulator for its largest magnitude,
+    // pass 2 converts and stores 64-column boxes.
+    static_assert(MODE != MODE_DX || EPI == 4, "one warp holds a row's whole tile");
+    const int n0 = tl.n * BN;
+    const int ncols = min(BN, p.h - n0);  // multiple of 64
+    float m = 0.0f;
 #pragma unroll 1
     for (int c = 0; c < ncols; c += 32) {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) w[i] = v[i];
-      if (c + 32 < ncols) tmem_ld32(tb + c + 32, v);  // overlaps the store
-      st.emit(&p.tmo[0], w, n0 + c, y0);
+      uint32_t v[32];
+      tmem_ld32(tb + c, v);
       tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(__uint_as_float(v[i])));
+    }
+    int es = 13 - ((int)((__float_as_uint(m) >> 23) & 0xFFu) - 127);  // m * 2^es < 2^14
+    if (m == 0.0f || !(m <= 3.402823466e38f)) es = 0;  // zero, inf or NaN: unscaled
+    es = min(max(es, -126), 126);
+    const float sc = __uint_as_float((uint32_t)(127 + es) << 23);
+    p.part[(size_t)(y0 + lane) * p.n_tiles + tl.n] = __uint_as_float((uint32_t)(127 - es) << 23);
+#pragma unroll 1
+    for (int c = 0; c < ncols; c += 64) {
+      uint32_t v0[32], v1[32], w[32];
+      tmem_ld32(tb + c, v0);
+      tmem_ld32(tb + c + 32, v1);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        w[i] = pack_f16x2(__uint_as_float(v0[2 * i]) * sc, __uint_as_float(v0[2 * i + 1]) * sc);
+        w[16 + i] = pack_f16x2(__uint_as_float(v1[2 * i]) * sc, __uint_as_float(v1[2 * i + 1]) * sc);
+      }
+      st.emit(&p.tmo[0], w, n0 + c, y0);
     }
   } else if (MODE == MODE_DOWN) {
     const int n0 = tl.n * BN + half * kw;  // this warp's first column
@@ -1133,7 +1155,7 @@ cudaError_t launch_dglu_gemm(const GemmProblem &g, const void *dy_pad, const voi
 }
 
 cudaError_t launch_dx_gemm(const GemmProblem &g, const void *da, const void *db, const void *w1,
-                           const void *w3, void *dx_pad, cudaStream_t st) {
+                           const void *w3, void *dx_pad, float *dx_scale, cudaStream_t st) {
   GemmParams p = base_params(g);
   const uint64_t P = (uint64_t)g.nblk_cap * BM;
   const uint64_t EF = (uint64_t)g.E * g.f;
@@ -1141,9 +1163,10 @@ cudaError_t launch_dx_gemm(const GemmProblem &g, const void *da, const void *db,
       !make_tmap_chunked(&p.tm[1], db, P, g.f, BM) ||
       !make_tmap_chunked(&p.tm[2], w1, EF, g.h, 2 * BK) ||
       !make_tmap_chunked(&p.tm[3], w3, EF, g.h, 2 * BK) ||
-      !make_tmap(&p.tmo[0], dx_pad, P, g.h, 32, 4))
+      !make_tmap(&p.tmo[0], dx_pad, P, g.h, 32))  // fp16 boxes (2-byte copies)
     return cudaErrorInvalidValue;
   p.tm[4] = p.tm[0];
+  p.part = dx_scale;
   p.n_tiles = (g.h + BN - 1) / BN;
   p.k_iters = 2 * (g.f / Cfg<MODE_DX, 4>::bk);
   p.group = raster_units(2 * g.f);

@@ -54,9 +54,11 @@ cudaError_t launch_gather(int T, int h, int k, int E, const void *x, const int32
 cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const int32_t *dest_row,
                            const float *weights, void *y, cudaStream_t st);
 
-// Backward scatter: dx_t = bf16(sum_s dX_pad[dest_row[t*k+s]]) over fp32 rows and, from the
-// DGLU GEMM's partial sums part [P_max, nt], dweights[t*k+s] = sum_n part[dest_row[t*k+s]][n].
-cudaError_t launch_bwd_scatter(int T, int h, int k, const float *dx_pad, const int32_t *dest_row,
+// Backward scatter: dx_t = bf16(sum_s dX_pad[dest_row[t*k+s]]) over the block-floating-point
+// rows of launch_dx_gemm (value = fp16 * scale, summed in fp32) and, from the DGLU GEMM's
+// partial sums part [P_max, nt], dweights[t*k+s] = sum_n part[dest_row[t*k+s]][n].
+cudaError_t launch_bwd_scatter(int T, int h, int k, const void *dx_pad, const float *dx_scale,
+                               const int32_t *dest_row,
                                const float *part, int nt, void *dx, float *dweights,
                                cudaStream_t st);
 
@@ -88,8 +90,11 @@ constexpr int kDgluTileCols = 256;
 cudaError_t launch_dglu_gemm(const GemmProblem &g, const void *dy_pad, const void *w2,
                              const void *a_in, const void *b_in, void *da_out, void *db_out,
                              void *hw_out, float *part, cudaStream_t st);
+// dX_pad [P_max,h] fp16 with dx_scale [P_max, ceil(h/256)] fp32: row r, columns of tile n hold
+// value * 2^-e; dx_scale[r][n] = 2^e (block floating point, 11 significant bits per value).
+constexpr int kDxTileCols = 256;
 cudaError_t launch_dx_gemm(const GemmProblem &g, const void *da, const void *db, const void *w1,
-                           const void *w3, void *dx_pad, cudaStream_t st);
+                           const void *w3, void *dx_pad, float *dx_scale, cudaStream_t st);
 cudaError_t launch_wgrad_gemm(const GemmProblem &g, const void *x_pad, const void *h_in,
                               const void *dy_pad, const void *da, const void *db, float *dw1,
                               float *dw3, float *dw2, cudaStream_t st);

@@ -288,11 +288,17 @@ DMOE_API int dmoe_bwd_dglu(const dmoe_dims *dims, const void *dy_pad, const void
                            void *da, void *dbm, void *hw, float *dw_part, void *stream);
 
 /* dX GEMM: dX_pad[b] = dA[b] W1_e + dBm[b] W3_e, one fp32 accumulator over both K passes,
- * stored in fp32: the k rows of a token are summed by dmoe_bwd_scatter, and rounding each of
- * them to bf16 first would put k roundings into every element of dx.
- * da, dbm [P_max,f] bf16 -> dx_pad [P_max,h] fp32. */
+ * stored in block floating point: dx_pad [P_max,h] holds fp16 values and dx_scale
+ * [P_max, ceil(h / DMOE_DX_TILE_COLS)] fp32 one power-of-two scale per row and 256-column
+ * tile (value = fp16 * scale; the scale puts the row's largest magnitude in the tile into
+ * [2^13, 2^14)).  That keeps 11 significant bits per value at bf16's size: the k rows of a
+ * token are summed by dmoe_bwd_scatter, and rounding each of them to bf16 first would put k
+ * bf16 roundings into every element of dx.
+ * da, dbm [P_max,f] bf16 -> dx_pad [P_max,h] fp16, dx_scale fp32. */
+#define DMOE_DX_TILE_COLS 256
 DMOE_API int dmoe_bwd_dx(const dmoe_dims *dims, const void *da, const void *dbm, const void *w1,
-                         const void *w3, const dmoe_map *map, void *dx_pad, void *stream);
+                         const void *w3, const dmoe_map *map, void *dx_pad, float *dx_scale,
+                         void *stream);
 
 /* Weight gradients, per expert e over its padded rows r in [padded_bins[e-1], padded_bins[e])
  * (padding rows are zero, so they add nothing; the walkthrough's stk path needs a transposed
@@ -310,10 +316,11 @@ DMOE_API int dmoe_bwd_wgrad(const dmoe_dims *dims, const void *x_pad, const void
  *   dx_t = bf16(sum_s dX_pad[dest_row[t*k+s]])  (fp32 sum in slot order),
  *   dweights[t*k+s] = sum_{n < nt} dw_part[dest_row[t*k+s] * nt + n]  (fp32, tile order; 0 for
  *   an entry dropped from the map).
- * dx_pad [P_max,h] fp32 (from dmoe_bwd_dx), dw_part from dmoe_bwd_dglu -> dx [T,h] bf16,
- * dweights [T,k] fp32. */
-DMOE_API int dmoe_bwd_scatter(const dmoe_dims *dims, const void *dx_pad, const float *dw_part,
-                              const dmoe_map *map, void *dx, float *dweights, void *stream);
+ * dx_pad, dx_scale from dmoe_bwd_dx (each row's values are fp16 * scale, exact in fp32),
+ * dw_part from dmoe_bwd_dglu -> dx [T,h] bf16, dweights [T,k] fp32. */
+DMOE_API int dmoe_bwd_scatter(const dmoe_dims *dims, const void *dx_pad, const float *dx_scale,
+                              const float *dw_part, const dmoe_map *map, void *dx,
+                              float *dweights, void *stream);
 
 /* ---- The linear router (the steps on either side of the routing). ----
  * The pages fix only the router's output, (scores, top_experts) (issue #56 error log;

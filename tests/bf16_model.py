@@ -80,6 +80,23 @@ def backward_model(inp: dict, top: np.ndarray, wts: np.ndarray) -> dict:
             "dW2": dW2.numpy(), "dw": dw.numpy()}
 
 
+def expert_wgrad_model(inp: dict, top: np.ndarray, wts: np.ndarray, e: int):
+    """The weight-gradient slabs (dW1_e, dW3_e, dW2_e) of one expert under the same roundings
+    as backward_model."""
+    X, dy = inp["x"].double(), inp["dy"].double()
+    W1, W3, W2 = inp["w1"][e].double(), inp["w3"][e].double(), inp["w2"][e].double()
+    ts, ss = np.nonzero(top == e)
+    wf = torch.from_numpy(wts.astype(np.float32)).double()
+    Xe = X[ts]
+    A, Bm = _bf(Xe @ W1.T), _bf(Xe @ W3.T)
+    s = torch.sigmoid(A)
+    G = dy[ts] @ W2
+    wr = wf[ts, ss][:, None]
+    dA = _bf(wr * G * Bm * s * (1 + A * (1 - s)))
+    dB = _bf(wr * G * A * s)
+    return ((dA.T @ Xe).numpy(), (dB.T @ Xe).numpy(), (dy[ts].T @ _bf(wr * A * s * Bm)).numpy())
+
+
 def bounds(model: dict, ref: dict) -> dict:
     """Per-output max-abs / RMS bound from the modelled errors against the oracle."""
     out = {}
