@@ -39,10 +39,10 @@ def _check_inputs(x, logits, w1, w3, w2):
 
 class DMoEFunction(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, x, logits, w1, w3, w2, top_k: int, route_flags: int = 0):
+    def forward(ctx, x, logits, w1, w3, w2, top_k: int, flags: int = 0):
         global _last_map
         T, h, f, E = _check_inputs(x, logits, w1, w3, w2)
-        dims = B.make_dims(T, h, f, E, top_k, route_flags=route_flags)
+        dims = B.make_dims(T, h, f, E, top_k, flags=flags)
         dev = x.device
         u8 = dict(dtype=torch.uint8, device=dev)
         smap = B.SparseMap(dims, dev)
@@ -81,7 +81,7 @@ class DMoEFunction(torch.autograd.Function):
         return dx, dlogits, dw1, dw3, dw2, None, None
 
 
-def dmoe(x, logits, w1, w3, w2, top_k: int, route_flags: int = 0):
+def dmoe(x, logits, w1, w3, w2, top_k: int, flags: int = 0):
     """y = dMoE(x) with the experts chosen by the top-k of softmax(logits); differentiable in
     x, logits, W1, W3 and W2."""
-    return DMoEFunction.apply(x, logits, w1, w3, w2, top_k, route_flags)
+    return DMoEFunction.apply(x, logits, w1, w3, w2, top_k, flags)

@@ -40,12 +40,12 @@ ROUTE_RENORMALIZE = 0x1
 class dmoe_dims(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("hidden", ctypes.c_int32), ("ffn", ctypes.c_int32),
                 ("num_experts", ctypes.c_int32), ("top_k", ctypes.c_int32),
-                ("route_flags", ctypes.c_int32)]
+                ("flags", ctypes.c_int32)]
 
     def __repr__(self):
         return (f"dmoe_dims(T={self.T}, hidden={self.hidden}, ffn={self.ffn}, "
                 f"num_experts={self.num_experts}, top_k={self.top_k}, "
-                f"route_flags={self.route_flags})")
+                f"flags={self.flags})")
 
 
 MAP_FIELDS = ("top_experts", "weights", "tokens_per_expert", "bins", "padded_bins", "indices",
@@ -135,9 +135,9 @@ def dmoe_debug_inject_stall(enable: bool = True) -> None:
 
 
 def make_dims(T: int, hidden: int, ffn: int, num_experts: int, top_k: int,
-              route_flags: int = 0) -> dmoe_dims:
-    """route_flags: 0, or ROUTE_RENORMALIZE (weights = softmax over the k chosen logits)."""
-    return dmoe_dims(T, hidden, ffn, num_experts, top_k, route_flags)
+              flags: int = 0) -> dmoe_dims:
+    """flags: 0, or ROUTE_RENORMALIZE (weights = softmax over the k chosen logits)."""
+    return dmoe_dims(T, hidden, ffn, num_experts, top_k, flags)
 
 
 def _ptr(t) -> int | None:

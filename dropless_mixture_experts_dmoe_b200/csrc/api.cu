@@ -27,7 +27,7 @@ int check_dims(const dmoe_dims *d) {
     return DMOE_ERR_SHAPE;
   if (d->ffn < DMOE_BLOCKING || d->ffn % DMOE_BLOCKING != 0) return DMOE_ERR_SHAPE;
   if (d->hidden < DMOE_BLOCKING || d->hidden % DMOE_BLOCKING != 0) return DMOE_ERR_SHAPE;
-  if (d->route_flags & ~DMOE_ROUTE_RENORMALIZE) return DMOE_ERR_SHAPE;
+  if (d->flags & ~DMOE_ROUTE_RENORMALIZE) return DMOE_ERR_SHAPE;
   const long long n = (long long)d->T * d->top_k;
   const long long pmax =
       (n + (long long)(DMOE_BLOCKING - 1) * d->num_experts) / DMOE_BLOCKING * DMOE_BLOCKING;
@@ -208,7 +208,7 @@ int dmoe_sparse_map(const dmoe_dims *dims, const void *logits, const dmoe_map *m
   const int T = dims->T, E = dims->num_experts, k = dims->top_k;
   const int nblk_cap = (int)(pmax_of(dims) / DMOE_BLOCKING);
   int32_t *tile_hist = static_cast<int32_t *>(ws);
-  const bool renorm = (dims->route_flags & DMOE_ROUTE_RENORMALIZE) != 0;
+  const bool renorm = (dims->flags & DMOE_ROUTE_RENORMALIZE) != 0;
   if ((rc = launch_rc(launch_route_hist(static_cast<const uint16_t *>(logits), T, E, k, renorm,
                                         map->top_experts, map->weights, tile_hist, st))))
     return rc;
@@ -427,7 +427,7 @@ int dmoe_router_dlogits(const dmoe_dims *dims, const void *logits, const dmoe_ma
   if (!aligned16(logits) || !aligned16(dlogits)) return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
   return launch_rc(launch_router_dlogits(dims->T, dims->num_experts, dims->top_k,
-                                         (dims->route_flags & DMOE_ROUTE_RENORMALIZE) != 0,
+                                         (dims->flags & DMOE_ROUTE_RENORMALIZE) != 0,
                                          static_cast<const uint16_t *>(logits), map->top_experts,
                                          dweights, static_cast<uint16_t *>(dlogits),
                                          static_cast<cudaStream_t>(stream)));

@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(kCopyThreads) k_combine(int T, int h, int k,
 // columns (one 16-byte vector) per slot; VPL such vectors per lane and SLOTS slots are loaded
 // before any is consumed.
 template <int VPL, int SLOTS>
-__global__ void __launch_bounds__(kCopyThreads) k_scatter_sum(int T, int h, int k,
+__global__ void __launch_bounds__(kCopyThreads, 2) k_scatter_sum(int T, int h, int k,
                                                               const uint4 *__restrict__ dx_pad,
                                                               const float *__restrict__ scale,
                                                               const int32_t *__restrict__ dest_row,
@@ -284,8 +284,10 @@ cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const int32_t
 cudaError_t launch_bwd_scatter(int T, int h, int k, const void *dx_pad, const float *dx_scale,
                                const int32_t *dest_row, const float *part, int nt, void *dx,
                                float *dweights, cudaStream_t st) {
-  const int vpl = (k <= 2) ? 8 : (k <= 4) ? 4 : 2;  // 16-byte vectors per lane and slot
-  auto kernel = (k <= 2) ? k_scatter_sum<8, 2> : (k <= 4) ? k_scatter_sum<4, 4>
+  // 16-byte vectors per lane and slot: at most 16 loads in flight per lane within 128
+  // registers (two CTAs per SM)
+  const int vpl = (k <= 2) ? 4 : 2;
+  auto kernel = (k <= 2) ? k_scatter_sum<4, 2> : (k <= 4) ? k_scatter_sum<2, 4>
                                                           : k_scatter_sum<2, 8>;
   const long long items = (long long)T * (((h >> 3) + 32 * vpl - 1) / (32 * vpl));
   return launch_pdl(kernel, copy_grid(items), kCopyThreads, 0, st, T, h, k,

@@ -5,8 +5,9 @@
 // completion ticket):
 //   k_route_hist   16 warps per 64-token tile, 4 tokens per warp with all their logits loaded
 //                  at once: top-k by integer max over order-preserving keys (ties -> lower
-//                  expert index), fp32 softmax weights, per-tile histogram in shared memory
-//                  (O(E) bytes, independent of T) and a per-tile status word.
+//                  expert index; each lane keeps its three best candidates), fp32 softmax
+//                  weights, per-tile histogram in shared memory (O(E) bytes, independent of
+//                  T) and a per-tile status word.
 //   k_map_scan     one CTA per 32 experts: per-expert exclusive offsets of every tile; the
 //                  last CTA to finish (a ticket counter, no waiting) computes bins,
 //                  padded_bins (round_up to 128), num_blocks and stores the status word.
@@ -28,12 +29,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// e^(v - m) for v <= m: the difference of two bf16 values is exact in fp32, so only the
-// scaling by log2(e) and the 2^x approximation round.
-__device__ __forceinline__ float exp_diff(float v, float m) {
-  return ex2_approx(__fmul_rn(__fsub_rn(v, m), 1.4426950408889634f));
 }
 
 // Selection key of a logit given as its fp32 image u (a bf16 value in the high half): the high
@@ -117,40 +112,52 @@ struct RouteRow {
   }
 };
 
-// Descending bitonic sort of N (a power of two) keys held in registers.
-template <int N>
-__device__ __forceinline__ void sort_desc(uint32_t (&a)[N]) {
+// Order-preserving 16-bit images of the two bf16 values packed in w, in the same halves:
+// for non-NaN a, b, a < b iff image(a) < image(b) (negative values have every bit inverted,
+// the others their sign bit set), and -0 is first turned into +0 (-0 + +0 = +0), so that the
+// two zeros tie.  NaN is not ordered here (the caller takes a separate path for it).
+__device__ __forceinline__ uint32_t order2(uint32_t w) {
+  __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(&w);
+  v = __hadd2(v, __nv_bfloat162(__float2bfloat16_rn(0.0f), __float2bfloat16_rn(0.0f)));
+  const uint32_t z = *reinterpret_cast<const uint32_t *>(&v);
+  const uint32_t neg = (z >> 15) & 0x00010001u;  // sign bit of each half, at bit 0 / bit 16
+  return z ^ ((neg * 0x7FFFu) | 0x80008000u);
+}
+
+// The C largest keys seen so far, largest first (0 = empty slot): one insertion costs C
+// max/min pairs, with no branches.
+template <int C>
+struct TopC {
+  uint32_t c[C];
+  __device__ __forceinline__ void clear() {
 #pragma unroll
-  for (int size = 2; size <= N; size <<= 1) {
+    for (int i = 0; i < C; ++i) c[i] = 0u;
+  }
+  __device__ __forceinline__ void insert(uint32_t x) {
 #pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-#pragma unroll
-      for (int i = 0; i < N; ++i) {
-        const int j = i ^ stride;
-        if (j > i) {
-          const uint32_t hi = max(a[i], a[j]), lo = min(a[i], a[j]);
-          if ((i & size) == 0) {
-            a[i] = hi;
-            a[j] = lo;
-          } else {
-            a[i] = lo;
-            a[j] = hi;
-          }
-        }
-      }
+    for (int i = 0; i < C; ++i) {
+      const uint32_t hi = max(c[i], x);
+      x = min(c[i], x);
+      c[i] = hi;
     }
   }
-}
+  __device__ __forceinline__ void pop() {
+#pragma unroll
+    for (int i = 0; i + 1 < C; ++i) c[i] = c[i + 1];
+    c[C - 1] = 0u;
+  }
+};
 
 // Grid: one CTA per 64-token tile.  Per token: every lane turns its logits into unique integer
 // keys (order-preserving image of the bf16 value in the high half, 0xFFFF - expert in the low
-// half, so the larger key is the larger logit and, on equal logits, the lower expert); k rounds
-// of a warp-wide integer max pick the top-k in rank order.  With KPL <= 8 each lane sorts its
-// keys once and a round only pops the winning lane's head; wider rows clear the winner in
-// place.  Weights: fp32 softmax over all E logits (or, renormalised, over the k picks) with
-// the first pick as the maximum.  The tile's expert histogram is built in shared memory and
-// written to tile_hist; the tile's status bits go to tile_flags (a plain store, so the
-// workspace needs no initialisation).
+// half, so the larger key is the larger logit and, on equal logits, the lower expert) and
+// keeps its three largest; k rounds of a warp-wide integer max then pick the top-k in rank
+// order, the winning lane dropping its head.  A lane that gives up all three of its
+// candidates while rounds remain (it holds more than three of the top-k) refills them from
+// its keys below the last pick.  Weights: fp32 softmax over all E logits (or, renormalised,
+// over the k picks) with the first pick as the maximum.  The tile's expert histogram is built
+// in shared memory and written to tile_hist; the tile's status bits go to tile_flags (a plain
+// store, so the workspace needs no initialisation).
 template <int KPL, bool VEC>
 __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__restrict__ logits,
                                                               int T, int E, int k, int renorm,
@@ -160,8 +167,10 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__
                                                               int32_t *__restrict__ tile_flags,
                                                               unsigned int *__restrict__ done) {
   using Row = RouteRow<KPL, VEC>;
-  constexpr bool kSorted = KPL <= 8;
+  constexpr int C = (KPL < 3) ? KPL : 3;                  // candidates kept per lane
   constexpr int kInFlight = (KPL <= 8) ? kRouteTPW : 1;  // token rows loaded ahead per warp
+  constexpr bool kPacked = VEC && KPL >= 2;              // two logits per word
+  constexpr float kLog2e = 1.4426950408889634f;
   extern __shared__ int hist[];  // [E]
   __shared__ int s_flags;
   pdl_wait();
@@ -173,6 +182,12 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__
   const int t0 = blockIdx.x * kMapTokTile + warp;
   // expert KPL*lane + i of the vector layout exists iff the lane's first one does (E % KPL == 0)
   const bool lane_ok = KPL * lane < E;
+  uint32_t low[KPL];  // low halves of this lane's keys; 0 marks a slot past the last expert
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    const int e = Row::expert(lane, i);
+    low[i] = (VEC ? lane_ok : (e < E)) ? 0xFFFFu - (uint32_t)e : 0u;
+  }
   Row rows[kInFlight];
 #pragma unroll
   for (int j = 0; j < kInFlight; ++j) {
@@ -191,68 +206,66 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__
     } else {
       cur.load(logits + (size_t)t * E, E, lane);
     }
+    // keys, and a test for Inf / NaN: a half whose exponent bits are all ones carries into
+    // its bit 15 when 0x0080 is added to its exponent field (slots past E hold 0: no carry)
     uint32_t key[KPL];
-    bool nonfinite = false;
+    uint32_t nf = 0u;
 #pragma unroll
-    for (int i = 0; i < KPL; ++i) {
-      const int e = Row::expert(lane, i);
-      const bool ok = VEC ? lane_ok : (e < E);
-      const uint32_t u = cur.image(i);
-      nonfinite |= ok && (u & 0x7F800000u) == 0x7F800000u;
-      key[i] = ok ? route_key(u, 0xFFFFu - (uint32_t)e) : 0u;
-    }
-    if (__any_sync(0xFFFFFFFFu, nonfinite)) {  // rare: rebuild with NaN ranked lowest
-      bad = true;
-#pragma unroll
-      for (int i = 0; i < KPL; ++i) {
-        const int e = Row::expert(lane, i);
-        const bool ok = VEC ? lane_ok : (e < E);
-        key[i] = ok ? route_key_nan(cur.image(i), 0xFFFFu - (uint32_t)e) : 0u;
+    for (int i = 0; i < Row::kWords; ++i) {
+      const uint32_t wv = cur.w[i];
+      nf |= (wv & 0x7F807F80u) + 0x00800080u;
+      const uint32_t o = order2(wv);
+      if constexpr (kPacked) {
+        key[2 * i] = __byte_perm(o, low[2 * i], 0x1054);        // (image lo << 16) | low
+        key[2 * i + 1] = __byte_perm(o, low[2 * i + 1], 0x3254);  // (image hi << 16) | low
+      } else {
+        key[i] = __byte_perm(o, low[i], 0x1054);
       }
     }
-    if constexpr (kSorted) sort_desc<KPL>(key);
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) key[i] = low[i] ? key[i] : 0u;
+    if (__any_sync(0xFFFFFFFFu, (nf & 0x80008000u) != 0u)) {  // rare: NaN ranked lowest
+      bad = true;
+#pragma unroll
+      for (int i = 0; i < KPL; ++i) key[i] = low[i] ? route_key_nan(cur.image(i), low[i]) : 0u;
+    }
+    TopC<C> cand;
+    cand.clear();
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) cand.insert(key[i]);
     // k rounds of a warp-wide integer max; keys are unique, so exactly one lane holds the
     // winner, and a valid key is never 0 (its low half is >= 0xFFFF - 1023).
     uint32_t my_key = 0;  // lane s < k: the key of pick s
     for (int s = 0; s < k; ++s) {
-      uint32_t best = 0;
-      if constexpr (kSorted) {
-        best = key[0];
-      } else {
-#pragma unroll
-        for (int i = 0; i < KPL; ++i) best = max(best, key[i]);
-      }
-      const uint32_t wb = __reduce_max_sync(0xFFFFFFFFu, best);
+      const uint32_t wb = __reduce_max_sync(0xFFFFFFFFu, cand.c[0]);
       my_key = (lane == s) ? wb : my_key;
-      if constexpr (kSorted) {
-        if (key[0] == wb) {
+      if (cand.c[0] == wb) {
+        cand.pop();
+        if (KPL > C && cand.c[0] == 0u && s + 1 < k) {
 #pragma unroll
-          for (int i = 0; i + 1 < KPL; ++i) key[i] = key[i + 1];
-          key[KPL - 1] = 0u;
+          for (int i = 0; i < KPL; ++i)
+            if (key[i] < wb) cand.insert(key[i]);
         }
-      } else {
-#pragma unroll
-        for (int i = 0; i < KPL; ++i)
-          if (key[i] == wb) key[i] = 0u;
       }
     }
     const uint32_t top_key = __shfl_sync(0xFFFFFFFFu, my_key, 0);
     const int my_e = 0xFFFF - (int)(my_key & 0xFFFFu);
-    // softmax over all E logits (or, renormalised, over the k picks), max = the first pick.
+    // softmax over all E logits (or, renormalised, over the k picks), max = the first pick;
+    // e^(x - m) = 2^(x log2(e) - m log2(e)) with one fused multiply-add per logit
     const float m = ((top_key >> 16) == 0u) ? __uint_as_float(0x7FC00000u)
                                            : bf16_from_order(top_key >> 16);
     const float v = (lane < k) ? (((my_key >> 16) == 0u) ? __uint_as_float(0x7FC00000u)
                                                          : bf16_from_order(my_key >> 16))
                                : 0.0f;
-    const float ev = exp_diff(v, m);
+    const float ml = m * kLog2e;
+    const float ev = ex2_approx(fmaf(v, kLog2e, -ml));
     float sum = 0.0f;
     if (renorm) {
       if (lane < k) sum = ev;
     } else {
 #pragma unroll
       for (int i = 0; i < KPL; ++i)
-        if (VEC ? lane_ok : (Row::expert(lane, i) < E))
-          sum += exp_diff(__uint_as_float(cur.image(i)), m);
+        if (low[i]) sum += ex2_approx(fmaf(__uint_as_float(cur.image(i)), kLog2e, -ml));
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
@@ -499,12 +512,17 @@ __global__ void __launch_bounds__(kMapThreads) k_map_scatter(int T, int E, int k
   __syncthreads();
   int *my = wh + warp * E;
   const unsigned lt_mask = (1u << lane) - 1u;
-  // pass 1: per-warp histogram of its contiguous entry range
+  // pass 1: per-warp histogram of its contiguous entry range; the lanes sharing each lane's
+  // expert in a round are kept for pass 2
+  unsigned peers_of[kScatRounds];
+#pragma unroll
+  for (int r = 0; r < kScatRounds; ++r) peers_of[r] = 0u;
 #pragma unroll
   for (int r = 0; r < kScatRounds; ++r) {
     if (wb + 32 * r >= we) break;
     const int e = ev[r];
     const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+    peers_of[r] = peers;
     if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
     __syncwarp();
   }
@@ -525,7 +543,7 @@ __global__ void __launch_bounds__(kMapThreads) k_map_scatter(int T, int E, int k
     if (wb + 32 * r >= we) break;
     const long long j = wb + 32 * r + lane;
     const int e = ev[r];
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+    const unsigned peers = peers_of[r];
     if (e >= 0) {
       const int i = my[e] + __popc(peers & lt_mask);
       indices[i] = (int32_t)j;

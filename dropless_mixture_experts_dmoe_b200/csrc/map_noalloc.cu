@@ -85,7 +85,7 @@ extern "C" int dmoe_sparse_map_noalloc(const dmoe_dims *dims, const void *logits
   // The histogram kernel writes every (tile, expert) entry and every tile status word of the
   // scratch it later reads and zeroes the counter after them, so nothing left over from an
   // earlier call is ever read; the scan kernel stores the call's status word.
-  const bool renorm = (dims->route_flags & DMOE_ROUTE_RENORMALIZE) != 0;
+  const bool renorm = (dims->flags & DMOE_ROUTE_RENORMALIZE) != 0;
   if ((rc = rc_of(dmoe::launch_route_hist(static_cast<const uint16_t *>(logits), T, E, k, renorm,
                                           map->top_experts, map->weights, scratch, st))))
     return rc;

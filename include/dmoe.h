@@ -88,11 +88,11 @@ extern "C" {
 #define DMOE_STATUS_TIMEOUT 0x8            /* a bounded in-kernel wait gave up */
 
 /* Problem shape.  T tokens, hidden size h, ffn size f (per expert), E experts, top_k, and
- * the routing variant: route_flags = 0 (the default: weights are the softmax over all E
+ * the routing variant: flags = 0 (the default: weights are the softmax over all E
  * logits at the chosen experts) or DMOE_ROUTE_RENORMALIZE.  Other bits are rejected. */
 typedef struct {
   int32_t T, hidden, ffn, num_experts, top_k;
-  int32_t route_flags;
+  int32_t flags;
 } dmoe_dims;
 
 /* Routing variant: the k weights of a token are the softmax over its k chosen logits only,

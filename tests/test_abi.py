@@ -78,10 +78,10 @@ def test_bad_dims_rejected_before_launch(lib, dims, code):
 
 def test_unknown_route_flag_rejected(lib):
     m = B.dmoe_map()
-    d = B.make_dims(256, 128, 128, 8, 2, route_flags=0x2)
+    d = B.make_dims(256, 128, 128, 8, 2, flags=0x2)
     assert B.dmoe_padded_rows_max(d) == 0
     assert lib.dmoe_sparse_map(ctypes.byref(d), None, ctypes.byref(m), None, 0, None) == -2
-    d = B.make_dims(256, 128, 128, 8, 2, route_flags=B.ROUTE_RENORMALIZE)
+    d = B.make_dims(256, 128, 128, 8, 2, flags=B.ROUTE_RENORMALIZE)
     assert B.dmoe_padded_rows_max(d) > 0  # the one defined flag is accepted
 
 

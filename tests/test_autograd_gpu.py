@@ -30,7 +30,7 @@ def test_autograd_matches_direct_calls(w, renorm):
     assert A.last_status() == 0
 
     # the same steps through the C ABI
-    dims = B.make_dims(w.T, w.hidden, w.ffn, w.E, w.top_k, route_flags=flags)
+    dims = B.make_dims(w.T, w.hidden, w.ffn, w.E, w.top_k, flags=flags)
     bufs = B.Buffers(dims, train=True)
     bf, f32 = dict(dtype=torch.bfloat16, device="cuda"), dict(dtype=torch.float32, device="cuda")
     y_ref = torch.empty((w.T, w.hidden), **bf)

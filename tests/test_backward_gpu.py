@@ -79,10 +79,10 @@ def test_backward_steps_against_float64(w):
     scl = st["dx_scale"][:P].cpu()
     assert (scl > 0).all() and (torch.frexp(scl)[0] == 0.5).all()  # powers of two
     f16 = st["dx_pad"][:P].float().cpu().abs()
-    for n in range(nsc):  # each row's largest stored magnitude of a tile is in [2^13, 2^14)
-        mx = f16[:, n * 256:(n + 1) * 256].amax(1)
+    for n in range(nsc):  # each row's largest stored magnitude of a tile is in [2^13, 2^14]
+        mx = f16[:, n * 256:(n + 1) * 256].amax(1)  # (2^14 when fp16 rounding carries up)
         nz = mx > 0
-        assert ((mx[nz] >= 2.0 ** 13) & (mx[nz] < 2.0 ** 14)).all(), n
+        assert ((mx[nz] >= 2.0 ** 13) & (mx[nz] <= 2.0 ** 14)).all(), n
         assert (scl[~nz, n] == 1).all(), n  # all-zero rows (padding) are stored unscaled
     part = st["dw_part"][:P].cpu()
     A, Bm, Xp = D(bufs.view("a")), D(bufs.view("bm")), D(bufs.view("x_pad"))

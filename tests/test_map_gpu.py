@@ -58,6 +58,8 @@ def test_map_parity_real_inputs_tiny():
     (600, 384, 8, "few_values"),    # 16 per lane, vector, unsorted rounds
     (700, 1000, 8, "continuous"),   # 32 per lane, strided
     (40000, 16, 4, "continuous"),   # 625 tiles: the scan re-reads past its register cache
+    (500, 64, 8, "tiny_values"),    # bf16 subnormals of both signs next to +0 / -0
+    (2048, 256, 8, "skewed"),       # the skewed workload's bias: one lane holds most picks
 ])
 def test_map_parity_edge_cases(T, E, k, kind):
     g = torch.Generator().manual_seed(T * 7 + E)
@@ -66,6 +68,11 @@ def test_map_parity_edge_cases(T, E, k, kind):
     elif kind == "few_values":
         vals = torch.tensor([-1.0, -0.0, 0.0, 0.5, 0.5, 2.0])
         logits = vals[torch.randint(0, len(vals), (T, E), generator=g)]
+    elif kind == "tiny_values":
+        vals = torch.tensor([-2e-39, -1e-39, -0.0, 0.0, 1e-39, 2e-39, 3e-39, 1e-38])
+        logits = vals[torch.randint(0, len(vals), (T, E), generator=g)]
+    elif kind == "skewed":
+        logits = torch.randn((T, E), generator=g) - 1.5 * torch.log(torch.arange(E) + 1.0)
     else:
         logits = torch.randn((T, E), generator=g)
     logits = logits.to(torch.bfloat16)
@@ -83,7 +90,7 @@ def test_map_renormalised_weights(T, E, k):
     chosen logits (summing to 1), against the oracle's renormalised mode."""
     g = torch.Generator().manual_seed(T + 31 * E + k)
     logits = torch.randn((T, E), generator=g).to(torch.bfloat16)
-    dims = B.make_dims(T, 128, 128, E, k, route_flags=B.ROUTE_RENORMALIZE)
+    dims = B.make_dims(T, 128, 128, E, k, flags=B.ROUTE_RENORMALIZE)
     _, gm = gpu_map(dims, logits)
     top, wts = oracle.route(logits.float().numpy(), k, renorm=True)
     compare_map(gm, oracle.sparse_map(top, E), top_expected=top)

@@ -35,10 +35,10 @@ SMALL = [
 ]
 
 
-def _forward_backward(w, route_flags=0):
+def _forward_backward(w, flags=0):
     """Router forward, map, expert forward + backward, router backward, all on the GPU."""
     inp = make_inputs(w, with_dy=True, with_router=True)
-    dims = B.make_dims(w.T, w.hidden, w.ffn, w.E, w.top_k, route_flags=route_flags)
+    dims = B.make_dims(w.T, w.hidden, w.ffn, w.E, w.top_k, flags=flags)
     dev = {k: v.cuda() for k, v in inp.items()}
     bufs = B.Buffers(dims, train=True)
     bf = dict(dtype=torch.bfloat16, device="cuda")
