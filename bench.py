@@ -54,6 +54,9 @@ def parse():
     p.add_argument("--router", action="store_true",
                    help="compute the logits with the linear router (x W_r^T) inside the step and, "
                         "for fwd+bwd workloads, run the router backward after the layer's")
+    p.add_argument("--save-x-only", action="store_true",
+                   help="the memory variant: the forward saves X_pad only and the backward "
+                        "recomputes A and Bm with one more GLU GEMM")
     p.add_argument("--map-only", action="store_true",
                    help="time dmoe_sparse_map alone (routing + sparse map) on the workload's "
                         "logits: a supplementary line, not the layer's")
@@ -236,9 +239,10 @@ def tensor_peak(pk: dict, timed_s: float):
                             f"burst {pk['bf16']})")
 
 
-def config_of(w, router: bool, world: int) -> dict:
+def config_of(w, router: bool, world: int, save_x_only: bool = False) -> dict:
     """The workload description shared by both arms of the bench."""
-    return {"workload": f"{w.name} {w.describe()}" + (" +router" if router else ""),
+    return {"workload": f"{w.name} {w.describe()}" + (" +router" if router else "") +
+                        (" save_x_only" if save_x_only and w.backward else ""),
             "T": w.T, "hidden": w.hidden, "ffn": w.ffn, "num_experts": w.E, "top_k": w.top_k,
             "l2": "inputs larger than L2 (expert weights %.2f GB per step)" %
                   (3 * w.E * w.hidden * w.ffn * 2 / 1e9),
@@ -333,7 +337,8 @@ def run_reference(args, w):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(w, args.router, int(os.environ.get("WORLD_SIZE", "1"))),
+        "config": config_of(w, args.router, int(os.environ.get("WORLD_SIZE", "1")),
+                            args.save_x_only),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -368,7 +373,9 @@ def run_ours(args, w):
         dist.barrier()
     B.load()
 
-    dims = B.make_dims(w.T, w.hidden, w.ffn, w.E, w.top_k)
+    recompute = bool(args.save_x_only) and w.backward
+    dims = B.make_dims(w.T, w.hidden, w.ffn, w.E, w.top_k,
+                       flags=B.SAVE_X_ONLY if recompute else 0)
     train = w.backward
     router = bool(args.router)
     inp = make_inputs(w, with_dy=train, with_router=router)
@@ -380,7 +387,14 @@ def run_ours(args, w):
     st = torch.cuda.current_stream()
     if train:
         xp, hb, yp = bufs.view("x_pad"), bufs.view("h"), bufs.view("y_pad")
-        ab, bb = bufs.view("a"), bufs.view("bm")
+        if recompute:  # A and Bm live in backward scratch, recomputed there
+            P_ = B.dmoe_padded_rows_max(dims)
+            ab_bwd = torch.empty((P_, w.ffn), dtype=torch.bfloat16, device="cuda")
+            bb_bwd = torch.empty_like(ab_bwd)
+            ab = bb = None
+        else:
+            ab, bb = bufs.view("a"), bufs.view("bm")
+            ab_bwd, bb_bwd = ab, bb
         bs = bufs.bstep
         f32 = dict(dtype=torch.float32, device="cuda")
         grads = dict(dx=torch.empty_like(y), dw1=torch.empty((w.E, w.ffn, w.hidden), **f32),
@@ -391,7 +405,8 @@ def run_ours(args, w):
         ab = bb = None
     names = ["map", "gather", "glu_gemm", "down_gemm", "scatter"]
     if train:
-        names += ["dy_gather", "dglu_gemm", "wgrad_gemm", "dx_gemm", "dx_scatter"]
+        names += (["glu_recompute"] if recompute else []) + \
+            ["dy_gather", "dglu_gemm", "wgrad_gemm", "dx_gemm", "dx_scatter"]
     if router:
         names = ["router_gemm"] + names + (["router_bwd"] if train else [])
         dwr = torch.empty((w.E, w.hidden), dtype=torch.float32, device="cuda")
@@ -425,11 +440,15 @@ def run_ours(args, w):
         i += 1
         mark(i)
         if train:
-            # the sequence of dmoe_backward (which reuses dY_pad's region for the fp32 dX_pad)
+            # the sequence of dmoe_backward (which reuses dY_pad's region for dX_pad)
+            if recompute:
+                B.dmoe_expert_glu(dims, xp, dev["w1"], dev["w3"], bufs.map, None, ab_bwd, bb_bwd, st)
+                i += 1
+                mark(i)
             B.dmoe_padded_gather(dims, dev["dy"], bufs.map, bs["dy_pad"], st)
             mark(i + 1)
-            B.dmoe_bwd_dglu(dims, bs["dy_pad"], dev["w2"], ab, bb, bufs.map, bs["da"], bs["dbm"],
-                            bs["hw"], bs["dw_part"], st)
+            B.dmoe_bwd_dglu(dims, bs["dy_pad"], dev["w2"], ab_bwd, bb_bwd, bufs.map, bs["da"],
+                            bs["dbm"], bs["hw"], bs["dw_part"], st)
             mark(i + 2)
             B.dmoe_bwd_wgrad(dims, xp, bs["hw"], bs["dy_pad"], bs["da"], bs["dbm"], bufs.map,
                              grads["dw1"], grads["dw3"], grads["dw2"], st)
@@ -590,7 +609,7 @@ def run_ours(args, w):
     useful = w.useful_flops()
     nhf = N * w.hidden * w.ffn
     flops = dict(glu_gemm=4 * nhf, down_gemm=2 * nhf, dglu_gemm=2 * nhf, dx_gemm=4 * nhf,
-                 wgrad_gemm=6 * nhf)
+                 wgrad_gemm=6 * nhf, glu_recompute=4 * nhf)
     the = w.T * w.hidden * w.E
     router_flops = dict(router_gemm=2 * the, router_bwd=4 * the)
     if router:
@@ -633,7 +652,7 @@ def run_ours(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": config_of(w, router, world),
+        "config": config_of(w, router, world, recompute),
         "useful_tflops": useful / (ms_per_step / 1e3) / 1e12,
         "useful_tflops_frac_bf16": useful / (ms_per_step / 1e3) / 1e12 / pk_t,
         "padded_frac": pad_frac,

@@ -35,6 +35,7 @@ _I = ctypes.c_int
 
 
 ROUTE_RENORMALIZE = 0x1
+SAVE_X_ONLY = 0x4
 
 
 class dmoe_dims(ctypes.Structure):
@@ -136,7 +137,8 @@ def dmoe_debug_inject_stall(enable: bool = True) -> None:
 
 def make_dims(T: int, hidden: int, ffn: int, num_experts: int, top_k: int,
               flags: int = 0) -> dmoe_dims:
-    """flags: 0, or ROUTE_RENORMALIZE (weights = softmax over the k chosen logits)."""
+    """flags: an OR of ROUTE_RENORMALIZE (weights = softmax over the k chosen logits) and
+    SAVE_X_ONLY (the forward saves X_pad only; the backward recomputes A and Bm)."""
     return dmoe_dims(T, hidden, ffn, num_experts, top_k, flags)
 
 
@@ -352,6 +354,8 @@ class Buffers:
             total, offs = dmoe_saved_bytes(dims)
             self.saved = torch.empty(total, **u8)
             self.offsets = dict(x_pad=offs[0], a=offs[1], bm=offs[2])
+            if dims.flags & SAVE_X_ONLY:  # A and Bm are not saved
+                del self.offsets["a"], self.offsets["bm"]
             self.ws_fwd = torch.empty(dmoe_workspace_bytes(dims, WS_FORWARD_TRAIN), **u8)
             self.ws_bwd = torch.empty(max(dmoe_workspace_bytes(dims, WS_BACKWARD), 16), **u8)
             nt = (f + DGLU_TILE_COLS - 1) // DGLU_TILE_COLS
@@ -376,6 +380,8 @@ class Buffers:
         if name in self.offsets:
             off = self.offsets[name]
             return self.saved[off:off + n].view(torch.bfloat16).view(self.P, cols)
+        if name not in ("h", "y_pad"):
+            raise KeyError(f"{name} is not saved with these flags")
         # forward workspace layout: H [P,f] | Y_pad [P,h], each start aligned to 256 bytes
         off = 0 if name == "h" else (self.P * self.dims.ffn * 2 + 255) // 256 * 256
         return self.ws_fwd[off:off + n].view(torch.bfloat16).view(self.P, cols)

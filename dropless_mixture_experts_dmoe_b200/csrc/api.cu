@@ -27,7 +27,7 @@ int check_dims(const dmoe_dims *d) {
     return DMOE_ERR_SHAPE;
   if (d->ffn < DMOE_BLOCKING || d->ffn % DMOE_BLOCKING != 0) return DMOE_ERR_SHAPE;
   if (d->hidden < DMOE_BLOCKING || d->hidden % DMOE_BLOCKING != 0) return DMOE_ERR_SHAPE;
-  if (d->flags & ~DMOE_ROUTE_RENORMALIZE) return DMOE_ERR_SHAPE;
+  if (d->flags & ~(DMOE_ROUTE_RENORMALIZE | DMOE_SAVE_X_ONLY)) return DMOE_ERR_SHAPE;
   const long long n = (long long)d->T * d->top_k;
   const long long pmax =
       (n + (long long)(DMOE_BLOCKING - 1) * d->num_experts) / DMOE_BLOCKING * DMOE_BLOCKING;
@@ -92,11 +92,14 @@ inline int dglu_tiles(const dmoe_dims *d) { return (d->ffn + kDgluTileCols - 1) 
 
 inline int dx_tiles(const dmoe_dims *d) { return (d->hidden + kDxTileCols - 1) / kDxTileCols; }
 
+inline bool save_x_only(const dmoe_dims *d) { return (d->flags & DMOE_SAVE_X_ONLY) != 0; }
+
 // Backward workspace layout: dY_pad [P,h] bf16, whose region is reused for dX_pad [P,h] fp16
 // once the weight gradients have read dY_pad | dA [P,f] | dBm [P,f] | Hw [P,f] | routing-weight
-// partials [P, ceil(f/256)] fp32 | dX_pad scales [P, ceil(h/256)] fp32
+// partials [P, ceil(f/256)] fp32 | dX_pad scales [P, ceil(h/256)] fp32 | with DMOE_SAVE_X_ONLY
+// the recomputed A [P,f] and Bm [P,f]
 struct BwdLayout {
-  size_t dy, da, db, hw, part, dxs, total;
+  size_t dy, da, db, hw, part, dxs, a, bm, total;
 };
 BwdLayout bwd_layout(const dmoe_dims *d) {
   const size_t P = (size_t)pmax_of(d);
@@ -107,7 +110,11 @@ BwdLayout bwd_layout(const dmoe_dims *d) {
   l.hw = align_up(l.db + P * d->ffn * 2);
   l.part = align_up(l.hw + P * d->ffn * 2);
   l.dxs = align_up(l.part + P * dglu_tiles(d) * sizeof(float));
-  l.total = align_up(l.dxs + P * dx_tiles(d) * sizeof(float));
+  l.a = l.bm = l.total = align_up(l.dxs + P * dx_tiles(d) * sizeof(float));
+  if (save_x_only(d)) {
+    l.bm = align_up(l.a + P * d->ffn * 2);
+    l.total = align_up(l.bm + P * d->ffn * 2);
+  }
   return l;
 }
 
@@ -148,10 +155,16 @@ inline int check_router_dims(const dmoe_dims *d) {
   return (d->num_experts % 8 == 0) ? DMOE_OK : DMOE_ERR_SHAPE;
 }
 
-// Saved activations: X_pad [P,h] | A [P,f] | Bm [P,f]
+// Saved activations: X_pad [P,h] | A [P,f] | Bm [P,f]; X_pad only with DMOE_SAVE_X_ONLY
+// (offsets of A and Bm reported as 0)
 void saved_layout(const dmoe_dims *d, size_t off[3], size_t *total) {
   const size_t P = (size_t)pmax_of(d);
   off[0] = 0;
+  if (save_x_only(d)) {
+    off[1] = off[2] = 0;
+    *total = align_up(P * d->hidden * 2);
+    return;
+  }
   off[1] = align_up(off[0] + P * d->hidden * 2);
   off[2] = align_up(off[1] + P * d->ffn * 2);
   *total = align_up(off[2] + P * d->ffn * 2);
@@ -238,8 +251,9 @@ int dmoe_expert_glu(const dmoe_dims *dims, const void *x_pad, const void *w1, co
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_map(map, false))) return rc;
-  if (!x_pad || !w1 || !w3 || !h_out) return DMOE_ERR_NULL;
-  if (!aligned16(x_pad) || !aligned16(w1) || !aligned16(w3) || !aligned16(h_out) ||
+  if (!x_pad || !w1 || !w3 || (a_out == nullptr) != (b_out == nullptr) || (!h_out && !a_out))
+    return DMOE_ERR_NULL;
+  if (!aligned16(x_pad) || !aligned16(w1) || !aligned16(w3) || (h_out && !aligned16(h_out)) ||
       (a_out && !aligned16(a_out)) || (b_out && !aligned16(b_out)))
     return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
@@ -305,8 +319,10 @@ int dmoe_forward(const dmoe_dims *dims, const void *x, const void *w1, const voi
     saved_layout(dims, off, &total);
     uint8_t *s = static_cast<uint8_t *>(saved);
     xpad = s + off[0];
-    abuf = s + off[1];
-    bbuf = s + off[2];
+    if (!save_x_only(dims)) {  // else the backward recomputes A and Bm from X_pad
+      abuf = s + off[1];
+      bbuf = s + off[2];
+    }
   }
   if (!aligned16(x) || !aligned16(w1) || !aligned16(w3) || !aligned16(w2) || !aligned16(y) ||
       !aligned16(ws) || !aligned16(xpad) || !aligned16(map->weights))
@@ -398,6 +414,12 @@ int dmoe_backward(const dmoe_dims *dims, const void *dy, const void *w1, const v
   const void *xpad = sv + off[0], *abuf = sv + off[1], *bbuf = sv + off[2];
   uint8_t *w = static_cast<uint8_t *>(ws);
   void *dypad = w + l.dy, *da = w + l.da, *db = w + l.db, *hw = w + l.hw;
+  if (save_x_only(dims)) {  // A and Bm again, from the saved X_pad: the forward's exact bits
+    abuf = w + l.a;
+    bbuf = w + l.bm;
+    if ((rc = dmoe_expert_glu(dims, xpad, w1, w3, map, nullptr, w + l.a, w + l.bm, stream)))
+      return rc;
+  }
   float *part = reinterpret_cast<float *>(w + l.part);
   float *dxs = reinterpret_cast<float *>(w + l.dxs);
   void *dxpad = dypad;  // dY_pad is dead once the weight gradients have read it

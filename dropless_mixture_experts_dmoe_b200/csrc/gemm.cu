@@ -171,7 +171,7 @@ struct GemmParams {
   int k_iters;   // row-block modes: 64-wide K steps per tile
   int nblk_cap;  // P_max / 128: rows at or past nblk_cap * 128 read as zeros
   int group;     // row-block modes: units per raster chunk
-  int outs;      // GLU: 1 (H) or 3 (H, A, Bm)
+  int outs;      // GLU: bit 0 H, bit 1 A and Bm
   int inject;    // test-only: pair leaders withhold their first stage (waits then expire)
   long long wait_cycles;  // budget of every bounded wait of this launch
   const __nv_bfloat16 *in0, *in1;  // DGLU: saved A, Bm
@@ -457,15 +457,17 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
       tmem_ld32(tb + BN / 2 + c, u0);
       tmem_ld32(tb + BN / 2 + c + 32, u1);
       tmem_ld_wait();
+      if (p.outs & 1) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        w[i] = pack_bf16x2(silu_f(__uint_as_float(g0[2 * i])) * __uint_as_float(u0[2 * i]),
-                           silu_f(__uint_as_float(g0[2 * i + 1])) * __uint_as_float(u0[2 * i + 1]));
-        w[16 + i] = pack_bf16x2(silu_f(__uint_as_float(g1[2 * i])) * __uint_as_float(u1[2 * i]),
-                                silu_f(__uint_as_float(g1[2 * i + 1])) * __uint_as_float(u1[2 * i + 1]));
+        for (int i = 0; i < 16; ++i) {
+          w[i] = pack_bf16x2(silu_f(__uint_as_float(g0[2 * i])) * __uint_as_float(u0[2 * i]),
+                             silu_f(__uint_as_float(g0[2 * i + 1])) * __uint_as_float(u0[2 * i + 1]));
+          w[16 + i] = pack_bf16x2(silu_f(__uint_as_float(g1[2 * i])) * __uint_as_float(u1[2 * i]),
+                                  silu_f(__uint_as_float(g1[2 * i + 1])) * __uint_as_float(u1[2 * i + 1]));
+        }
+        st.emit(&p.tmo[0], w, n0 + c, y0);
       }
-      st.emit(&p.tmo[0], w, n0 + c, y0);
-      if (p.outs > 1) {
+      if (p.outs & 2) {
         pack_bf16_row(g0, g1, w);
         st.emit(&p.tmo[1], w, n0 + c, y0);
         pack_bf16_row(u0, u1, w);
@@ -1075,14 +1077,19 @@ cudaError_t launch_glu_gemm(const GemmProblem &g, const void *x_pad, const void 
   // K-major operands viewed as {64, rows, K/64}: one box brings two 64-deep K slabs
   if (!make_tmap_chunked(&p.tm[0], x_pad, P, g.h, BM) ||
       !make_tmap_chunked(&p.tm[1], w1, EF, g.h, BN / 2) ||
-      !make_tmap_chunked(&p.tm[2], w3, EF, g.h, BN / 2) ||
-      !make_tmap(&p.tmo[0], h_out, P, g.f, 32))
+      !make_tmap_chunked(&p.tm[2], w3, EF, g.h, BN / 2))
     return cudaErrorInvalidValue;
+  p.outs = 0;
+  if (h_out) {
+    if (!make_tmap(&p.tmo[0], h_out, P, g.f, 32)) return cudaErrorInvalidValue;
+    p.outs |= 1;
+  }
   if (a_out && b_out) {
     if (!make_tmap(&p.tmo[1], a_out, P, g.f, 32) || !make_tmap(&p.tmo[2], b_out, P, g.f, 32))
       return cudaErrorInvalidValue;
-    p.outs = 3;
+    p.outs |= 2;
   }
+  if (p.outs == 0) return cudaErrorInvalidValue;
   p.tm[3] = p.tm[4] = p.tm[0];
   p.n_tiles = g.f / (BN / 2);
   p.k_iters = g.h / Cfg<MODE_GLU, 4>::bk;

@@ -88,8 +88,10 @@ extern "C" {
 #define DMOE_STATUS_TIMEOUT 0x8            /* a bounded in-kernel wait gave up */
 
 /* Problem shape.  T tokens, hidden size h, ffn size f (per expert), E experts, top_k, and
- * the routing variant: flags = 0 (the default: weights are the softmax over all E
- * logits at the chosen experts) or DMOE_ROUTE_RENORMALIZE.  Other bits are rejected. */
+ * the variant flags: 0 (the default: weights are the softmax over all E logits at the chosen
+ * experts, and the forward saves X_pad, A and Bm for the backward) or an OR of
+ * DMOE_ROUTE_RENORMALIZE and DMOE_SAVE_X_ONLY.  Other bits are rejected.  Every call of one
+ * layer instance must see the same flags. */
 typedef struct {
   int32_t T, hidden, ffn, num_experts, top_k;
   int32_t flags;
@@ -99,6 +101,13 @@ typedef struct {
  * so they sum to 1 (the top-k renormalisation some MoE layers use; the pages' default does
  * not renormalise).  Read by dmoe_sparse_map (weights) and the router backward (dlogits). */
 #define DMOE_ROUTE_RENORMALIZE 0x1
+
+/* Memory variant (walkthrough section 4.4's MemoryOptimizedMLP; the SonicMoE abstract's
+ * activation-memory saving): the training forward saves only X_pad (dmoe_saved_bytes shrinks
+ * from (2h + 4f) to 2h bytes per padded row) and dmoe_backward recomputes A and Bm with one
+ * more GLU GEMM (4*N*h*f FLOP) into its workspace (DMOE_WS_BACKWARD grows by 4f bytes per
+ * padded row).  Every result is bit-identical to the default variant's. */
+#define DMOE_SAVE_X_ONLY 0x4
 
 /* The sparse map.  All device pointers, caller-owned; N = T*top_k entries,
  * P_max = dmoe_padded_rows_max(dims).  Meaning (walkthrough sections 4.1-4.3):
@@ -156,8 +165,8 @@ DMOE_API size_t dmoe_workspace_bytes(const dmoe_dims *dims, int kind);
 /* Bytes of the activations dmoe_forward saves for dmoe_backward, and their byte offsets
  * inside that buffer: offsets[0] X_pad [P_max,h], [1] A = X_pad W1^T [P_max,f],
  * [2] Bm = X_pad W3^T [P_max,f], all bf16 (H and Y_pad are not kept: the backward recomputes
- * the activation from A and Bm and never needs Y_pad).  offsets may be NULL.  Returns 0 for
- * invalid dims. */
+ * the activation from A and Bm and never needs Y_pad).  With DMOE_SAVE_X_ONLY only X_pad is
+ * kept (offsets[1] = offsets[2] = 0).  offsets may be NULL.  Returns 0 for invalid dims. */
 DMOE_API size_t dmoe_saved_bytes(const dmoe_dims *dims, size_t offsets[3]);
 
 /* Routing + sparse map (walkthrough section 4.1; the Fast-LLM get_sparse_map step).
@@ -240,8 +249,9 @@ DMOE_API int dmoe_padded_gather(const dmoe_dims *dims, const void *x, const dmoe
 
 /* GLU GEMM over the non-empty row blocks: for every block b < num_blocks with expert
  * e = block_expert[b], A = X_pad[b] W1_e^T, Bm = X_pad[b] W3_e^T (fp32 accumulation in
- * tensor memory) and H[b] = bf16(silu(A) * Bm).  a_out / b_out (may be NULL) receive
- * bf16(A), bf16(Bm).  x_pad [P_max,h] -> h_out, a_out, b_out [P_max,f], all bf16. */
+ * tensor memory) and H[b] = bf16(silu(A) * Bm).  a_out / b_out (both or neither) receive
+ * bf16(A), bf16(Bm); h_out may be NULL when they are given (the recompute of
+ * DMOE_SAVE_X_ONLY).  x_pad [P_max,h] -> h_out, a_out, b_out [P_max,f], all bf16. */
 DMOE_API int dmoe_expert_glu(const dmoe_dims *dims, const void *x_pad, const void *w1, const void *w3,
                     const dmoe_map *map, void *h_out, void *a_out, void *b_out, void *stream);
 

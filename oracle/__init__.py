@@ -14,6 +14,7 @@ cites the passage of the pages it follows, in the C source:
                          与 block-sparse 重构" §4.5 ``router(x)``).
 * ``sparse_map``      -- histogram, cumsum, round_up to 128, stable sort, the padded-row index
                          math, the block->expert table (walkthrough §2, §4.1-§4.3).
+* ``round_tokens``    -- tile-aware token rounding of a routing (SonicMoE abstract).
 * ``forward``         -- per-token loop y_t = sum_s w_ts W2_e(silu(W1_e x_t) * W3_e x_t)
                          (walkthrough §4.5 schematic, gated SiLU per the issue's config).
 * ``backward``, ``backward_tokens``, ``wgrad_elements``, ``wgrad_expert`` -- chain rule per
@@ -69,10 +70,12 @@ def _load():
         lib.oracle_backward_tokens.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, P, I]
         lib.oracle_wgrad_elements.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, I]
         lib.oracle_wgrad_expert.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, P, I]
+        lib.oracle_round_tokens.argtypes = [I, I, I, I, P, P, I, P, P]
         lib.oracle_router_logits.argtypes = [I, I, I, P, P, I, P, P, I]
         lib.oracle_router_backward.argtypes = [I, I, I, I, I, P, P, P, P, P, P, I, P, P, I, P, P, I]
         for fn in (lib.oracle_route, lib.oracle_sparse_map, lib.oracle_forward, lib.oracle_backward,
                    lib.oracle_backward_tokens, lib.oracle_wgrad_elements, lib.oracle_wgrad_expert,
+                   lib.oracle_round_tokens,
                    lib.oracle_max_threads,
                    lib.oracle_router_logits, lib.oracle_router_backward):
             fn.restype = ctypes.c_int
@@ -117,6 +120,31 @@ def route(logits, k: int, renorm: bool = False):
     if rc != 0:
         raise ValueError(f"oracle_route failed ({rc})")
     return top, w
+
+
+def round_tokens(logits, top_experts, block: int = BLOCKING, kmax: int | None = None):
+    """Tile-aware token rounding of a top-k routing (dmoe_oracle.c, oracle_round_tokens).
+    Returns (top [T, kmax] int32 with -1 in unused positions, weights [T, kmax] float64)."""
+    lg, top = _f32(logits), _i32(top_experts)
+    T, E = lg.shape
+    k = top.shape[1]
+    kmax = E if kmax is None else kmax
+    out_top = np.empty((T, kmax), np.int32)
+    out_w = np.empty((T, kmax), np.float64)
+    rc = _load().oracle_round_tokens(T, E, k, int(block), _p(lg), _p(top), kmax, _p(out_top),
+                                     _p(out_w))
+    if rc < 0:
+        raise ValueError(f"oracle_round_tokens failed ({rc})")
+    return out_top[:, :max(rc, 1)].copy(), out_w[:, :max(rc, 1)].copy()
+
+
+def compact_entries(top, weights):
+    """Token-major entry list of a routing with absent (-1) positions: (offsets [T+1],
+    experts [N'], weights [N']), each token's entries in position order."""
+    top = np.asarray(top)
+    keep = top >= 0
+    offsets = np.concatenate([[0], np.cumsum(keep.sum(1))]).astype(np.int32)
+    return offsets, top[keep].astype(np.int32), np.asarray(weights)[keep]
 
 
 def sparse_map(top_experts, E: int, nblk_cap: int | None = None) -> dict:

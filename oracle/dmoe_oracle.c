@@ -11,7 +11,8 @@
  *     double precision; all floating outputs are double.
  *   - Entries are flattened j = t*k + s (token t, slot s).  This is the flattening that the
  *     gather rule "source row = index_a // TOP_K" implies (MegaBlocks walkthrough,
- *     "dropless MoE and block-sparse", section 4.2).
+ *     "dropless MoE and block-sparse", section 4.2).  In the forward and backward, an entry
+ *     whose expert is -1 is absent (the rounded routing's unused positions).
  *   - Weights use the (out, in) layout: W1, W3 are [E, f, h]; W2 is [E, h, f].
  *   - Gated SiLU: W1 is the gate projection (passed through silu), W3 the up projection.
  *     silu(z) = z / (1 + exp(-z)).
@@ -83,6 +84,131 @@ int oracle_route(int T, int E, int k, int renorm, const float *logits, int32_t *
   }
   free(chosen);
   return 0;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Tile-aware token rounding (SonicMoE abstract: the routing is rounded so that each       */
+/* expert's token count is a multiple of the GEMM tile, removing the padding the grouped   */
+/* GEMM would otherwise compute; reported 1.16x kernel time).                              */
+/* ------------------------------------------------------------------------------------ */
+
+/* One (token, logit) candidate of an expert. */
+typedef struct {
+  float v;
+  int32_t t;
+} rank_item;
+
+/* Rank order of the rounding: the larger logit first; equal logits (+0 and -0 included)
+ * -> the lower token index first; NaN last.  qsort comparator: negative when a ranks first. */
+static int rank_cmp(const void *pa, const void *pb) {
+  const rank_item *a = (const rank_item *)pa, *b = (const rank_item *)pb;
+  if (preferred(a->v, b->v)) return -1;
+  if (preferred(b->v, a->v)) return 1;
+  return (a->t < b->t) ? -1 : (a->t > b->t);
+}
+
+/* The abstract gives the method in one sentence; the reading taken here:
+ *   - start from the top-k routing `top` [T, k] and its counts c_e;
+ *   - for every expert with r = c_e mod B != 0: round up -- add the B - r best-ranked tokens
+ *     not routed to e -- when r >= B/2 and at least B - r such tokens exist; otherwise round
+ *     down -- drop e's r worst-ranked entries.  So each count becomes the multiple of B
+ *     nearest to it (ties upward), or the one below when too few tokens are left to add;
+ *   - rank of a token for expert e: its logit l[t][e] (rank_cmp), the quantity both the
+ *     softmax weight and the top-k choice are monotone in for a token;
+ *   - a token keeps its surviving slots in slot order, then its added experts in increasing
+ *     expert index; every entry's weight is the softmax over all E logits at its expert
+ *     (as for a routed entry, no renormalisation).
+ * out_top / out_w: [T, kmax] entries per token; unused positions hold expert -1, weight 0.
+ * Returns the largest number of entries of a token (<= kmax), -4 if kmax is too small. */
+int oracle_round_tokens(int T, int E, int k, int B, const float *logits, const int32_t *top,
+                        int kmax, int32_t *out_top, double *out_w) {
+  if (T < 0 || E < 1 || k < 1 || k > E || B < 1 || kmax < 1) return -1;
+  const long N = (long)T * k;
+  long *count = (long *)calloc((size_t)E, sizeof(long));
+  unsigned char *drop = (unsigned char *)calloc((size_t)(N > 0 ? N : 1), 1);
+  unsigned char *add = (unsigned char *)calloc((size_t)T * E > 0 ? (size_t)T * E : 1, 1);
+  unsigned char *routed = (unsigned char *)calloc((size_t)T * E > 0 ? (size_t)T * E : 1, 1);
+  rank_item *items = (rank_item *)malloc(sizeof(rank_item) * (size_t)(T > 0 ? T : 1));
+  long *where = (long *)malloc(sizeof(long) * (size_t)(T > 0 ? T : 1));
+  if (!count || !drop || !add || !routed || !items || !where) {
+    free(count); free(drop); free(add); free(routed); free(items); free(where);
+    return -2;
+  }
+  for (long j = 0; j < N; ++j) {
+    count[top[j]] += 1;
+    routed[(size_t)(j / k) * E + top[j]] = 1;
+  }
+  for (int e = 0; e < E; ++e) {
+    const long r = count[e] % B;
+    if (r == 0) continue;
+    const long need = B - r;
+    if (2 * r >= B && (long)T - count[e] >= need) {  /* round up */
+      int n = 0;
+      for (int t = 0; t < T; ++t)
+        if (!routed[(size_t)t * E + e]) {
+          items[n].v = logits[(size_t)t * E + e];
+          items[n].t = t;
+          ++n;
+        }
+      qsort(items, (size_t)n, sizeof(rank_item), rank_cmp);
+      for (long q = 0; q < need; ++q) add[(size_t)items[q].t * E + e] = 1;
+    } else {  /* round down: the r worst-ranked entries of e */
+      int n = 0;
+      for (long j = 0; j < N; ++j)
+        if (top[j] == e) {
+          items[n].v = logits[(size_t)(j / k) * E + e];
+          items[n].t = (int32_t)(j / k);
+          where[n] = j;
+          ++n;
+        }
+      /* sort the positions along with the items: order indices by rank */
+      for (int a = 1; a < n; ++a) { /* insertion sort keeps it plain; n is one expert's count */
+        rank_item it = items[a];
+        long wj = where[a];
+        int b = a - 1;
+        while (b >= 0 && rank_cmp(&items[b], &it) > 0) {
+          items[b + 1] = items[b];
+          where[b + 1] = where[b];
+          --b;
+        }
+        items[b + 1] = it;
+        where[b + 1] = wj;
+      }
+      for (long q = n - r; q < n; ++q) drop[where[q]] = 1;
+    }
+  }
+  int most = 0, err = 0;
+  for (int t = 0; t < T && !err; ++t) {
+    const float *l = logits + (size_t)t * E;
+    double m = -INFINITY;
+    for (int e = 0; e < E; ++e)
+      if (!isnan(l[e]) && (double)l[e] > m) m = l[e];
+    double denom = 0.0;
+    for (int e = 0; e < E; ++e) denom += exp((double)l[e] - m);
+    int n = 0;
+    for (int s = 0; s < k; ++s) {
+      const long j = (long)t * k + s;
+      if (drop[j]) continue;
+      if (n >= kmax) { err = 1; break; }
+      out_top[(size_t)t * kmax + n] = top[j];
+      out_w[(size_t)t * kmax + n] = exp((double)l[top[j]] - m) / denom;
+      ++n;
+    }
+    for (int e = 0; e < E && !err; ++e) {
+      if (!add[(size_t)t * E + e]) continue;
+      if (n >= kmax) { err = 1; break; }
+      out_top[(size_t)t * kmax + n] = e;
+      out_w[(size_t)t * kmax + n] = exp((double)l[e] - m) / denom;
+      ++n;
+    }
+    for (int q = n; q < kmax; ++q) {
+      out_top[(size_t)t * kmax + q] = -1;
+      out_w[(size_t)t * kmax + q] = 0.0;
+    }
+    if (n > most) most = n;
+  }
+  free(count); free(drop); free(add); free(routed); free(items); free(where);
+  return err ? -4 : most;
 }
 
 /* ------------------------------------------------------------------------------------ */
@@ -219,6 +345,11 @@ int oracle_forward(int T, int h, int f, int E, int k, const float *x, const floa
         for (int o = 0; o < h; ++o) yt[o] = 0.0;
         for (int s = 0; s < k; ++s) {
           int e = top[(size_t)t * k + s];
+          if (e < 0) { /* no entry in this position (rounded routing) */
+            if (yts)
+              for (int o = 0; o < h; ++o) yts[((size_t)n * k + s) * h + o] = 0.0;
+            continue;
+          }
           expert_ffn(h, f, xt, W1 + (size_t)e * f * h, W3 + (size_t)e * f * h,
                      W2 + (size_t)e * h * f, a, b, hh, yo);
           double wts = w[(size_t)t * k + s];
@@ -299,6 +430,10 @@ int oracle_backward(int T, int h, int f, int E, int k, const float *x, const flo
   for (int t = 0; t < T; ++t) {
     for (int s = 0; s < k; ++s) {
       int e = top[(size_t)t * k + s];
+      if (e < 0) { /* no entry in this position (rounded routing) */
+        dw[(size_t)t * k + s] = 0.0;
+        continue;
+      }
       dw[(size_t)t * k + s] = entry_backward(
           h, f, x + (size_t)t * h, dy + (size_t)t * h, w[(size_t)t * k + s],
           W1 + (size_t)e * f * h, W3 + (size_t)e * f * h, W2 + (size_t)e * h * f, a, b, hh, yo,
@@ -338,6 +473,10 @@ int oracle_backward_tokens(int T, int h, int f, int E, int k, const float *x, co
         for (int j = 0; j < h; ++j) dxt[j] = 0.0;
         for (int s = 0; s < k; ++s) {
           int e = top[(size_t)t * k + s];
+          if (e < 0) { /* no entry in this position (rounded routing) */
+            dw[(size_t)n * k + s] = 0.0;
+            continue;
+          }
           dw[(size_t)n * k + s] = entry_backward(
               h, f, x + (size_t)t * h, dy + (size_t)t * h, w[(size_t)t * k + s],
               W1 + (size_t)e * f * h, W3 + (size_t)e * f * h, W2 + (size_t)e * h * f, a, b,

@@ -76,13 +76,32 @@ def test_bad_dims_rejected_before_launch(lib, dims, code):
     assert B.error_string(code) != "unknown error"
 
 
-def test_unknown_route_flag_rejected(lib):
+def test_unknown_flag_rejected(lib):
     m = B.dmoe_map()
-    d = B.make_dims(256, 128, 128, 8, 2, flags=0x2)
+    d = B.make_dims(256, 128, 128, 8, 2, flags=0x8)
     assert B.dmoe_padded_rows_max(d) == 0
     assert lib.dmoe_sparse_map(ctypes.byref(d), None, ctypes.byref(m), None, 0, None) == -2
-    d = B.make_dims(256, 128, 128, 8, 2, flags=B.ROUTE_RENORMALIZE)
-    assert B.dmoe_padded_rows_max(d) > 0  # the one defined flag is accepted
+    for fl in (B.ROUTE_RENORMALIZE, B.SAVE_X_ONLY, B.ROUTE_RENORMALIZE | B.SAVE_X_ONLY):
+        d = B.make_dims(256, 128, 128, 8, 2, flags=fl)
+        assert B.dmoe_padded_rows_max(d) > 0  # the defined flags are accepted
+
+
+def test_save_x_only_sizes(lib):
+    """DMOE_SAVE_X_ONLY: the saved activations shrink to X_pad (2h bytes per padded row, from
+    2h + 4f) and the backward workspace grows by the recomputed A and Bm (4f per row)."""
+    T, h, f, E, k = 32768, 2048, 512, 256, 8
+    d0 = B.make_dims(T, h, f, E, k)
+    d1 = B.make_dims(T, h, f, E, k, flags=B.SAVE_X_ONLY)
+    P = B.dmoe_padded_rows_max(d0)
+    s0, off0 = B.dmoe_saved_bytes(d0)
+    s1, off1 = B.dmoe_saved_bytes(d1)
+    assert s0 >= P * (2 * h + 4 * f) and s1 == P * 2 * h and off1 == [0, 0, 0]
+    assert off0[1] >= P * 2 * h and off0[2] >= off0[1] + P * 2 * f
+    assert abs((1 - s1 / s0) - 4 * f / (2 * h + 4 * f)) < 1e-3  # a third at this shape
+    w0 = B.dmoe_workspace_bytes(d0, B.WS_BACKWARD)
+    w1 = B.dmoe_workspace_bytes(d1, B.WS_BACKWARD)
+    assert P * 4 * f <= w1 - w0 <= P * 4 * f + 512
+    assert B.dmoe_workspace_bytes(d1, B.WS_FORWARD_TRAIN) == B.dmoe_workspace_bytes(d0, B.WS_FORWARD_TRAIN)
 
 
 def test_router_needs_E_multiple_of_8(lib):

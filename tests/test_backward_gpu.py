@@ -212,3 +212,24 @@ def test_backward_deterministic():
         else:
             a, b = a.view(torch.int32), b.view(torch.int32)
         assert torch.equal(a, b), k
+
+
+@pytest.mark.parametrize("w", [SMALL[1], SMALL[4], WORKLOADS[5]], ids=lambda w: w.describe())
+def test_save_x_only_is_bit_identical(w):
+    """DMOE_SAVE_X_ONLY (the forward saves X_pad only; the backward recomputes A and Bm with
+    one more GLU GEMM, walkthrough section 4.4): every output equals the default variant's
+    bit for bit, and the saved buffer holds X_pad only."""
+    inp = make_inputs(w, with_dy=True)
+    d0 = dims_of(w)
+    d1 = B.make_dims(w.T, w.hidden, w.ffn, w.E, w.top_k, flags=B.SAVE_X_ONLY)
+    b0, _, y0, g0 = gpu_backward(d0, inp)
+    b1, _, y1, g1 = gpu_backward(d1, inp)
+    assert int(b1.map.status.item()) == 0
+    assert b1.saved.numel() == B.dmoe_padded_rows_max(d1) * w.hidden * 2
+    assert b1.saved.numel() < b0.saved.numel()
+    assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
+    for k in g0:
+        a, b = g0[k], g1[k]
+        a, b = (a.view(torch.int16), b.view(torch.int16)) if a.dtype == torch.bfloat16 else \
+            (a.view(torch.int32), b.view(torch.int32))
+        assert torch.equal(a, b), k

@@ -18,6 +18,10 @@ Router   -- logits: one-hot tokens read a column of the router weight (closed fo
             differences of sum dw * softmax(x Wr^T)[picks] in the logits, x and Wr; torch
             float64 autograd of the same composition; shift invariance (each token's logit
             gradient sums to zero); k = E with equal dw gives zero; sampled = full.
+Token rounding (variant flag) -- every count a multiple of the tile and the nearest one (ties
+            up), the dropped / added entries against sorted() of the rank key, slot order kept,
+            weights against torch's float64 softmax, block 1 = identity; absent positions (-1)
+            contribute nothing in the forward and backward.
 Renormalised routing (variant flag) -- weights sum to 1, their ratios are exp(l_i - l_j),
             k = 1 gives 1 and k = E gives the plain softmax; torch float64 softmax over the
             chosen logits; its logit gradient by finite differences and autograd, zero outside
@@ -404,6 +408,104 @@ def test_wgrad_expert_slabs_against_autograd(oracle_mod):
         assert (d2 == full["dW2"][e]).all()
         if counts[e] == 0:
             assert not d1.any() and not d3.any() and not d2.any()
+
+
+# ----------------------------------------------------------------------------------------
+# tile-aware token rounding
+# ----------------------------------------------------------------------------------------
+
+def _rank_key(lg, t, e):
+    """Rank of token t for expert e, larger first: (logit, -token)."""
+    return (float(lg[t, e]), -int(t))
+
+
+def _check_rounding(oracle_mod, lg, k, B):
+    T, E = lg.shape
+    top, w = oracle_mod.route(lg, k)
+    tr, wr = oracle_mod.round_tokens(lg, top, block=B)
+    c = np.bincount(top.ravel(), minlength=E)
+    c2 = np.bincount(tr[tr >= 0], minlength=E)
+    for e in range(E):
+        r = c[e] % B
+        routed = set(np.nonzero((top == e).any(1))[0].tolist())
+        now = set(np.nonzero((tr == e).any(1))[0].tolist())
+        if r == 0:
+            assert now == routed, e
+            continue
+        up = 2 * r >= B and T - c[e] >= B - r
+        if up:  # the B - r best-ranked tokens not routed to e are added, nothing dropped
+            assert c2[e] == c[e] + (B - r) and routed <= now
+            cand = sorted(set(range(T)) - routed, key=lambda t: _rank_key(lg, t, e), reverse=True)
+            assert now - routed == set(cand[:B - r]), e
+        else:  # e's r worst-ranked entries are dropped, nothing added
+            assert c2[e] == c[e] - r and now <= routed
+            ranked = sorted(routed, key=lambda t: _rank_key(lg, t, e))
+            assert routed - now == set(ranked[:r]), e
+        assert c2[e] % B == 0
+        assert abs(int(c2[e]) - int(c[e])) <= B // 2
+    # each token: its surviving slots in slot order, then added experts in increasing order
+    p = torch.softmax(torch.tensor(lg, dtype=torch.float64), dim=1).numpy()
+    for t in range(T):
+        row = [e for e in tr[t] if e >= 0]
+        kept = [e for e in top[t] if e in row]
+        assert row[:len(kept)] == kept
+        assert row[len(kept):] == sorted(set(row) - set(top[t].tolist()))
+        assert len(set(row)) == len(row)
+        np.testing.assert_allclose(wr[t, :len(row)], p[t, row], rtol=1e-12)
+        assert (tr[t, len(row):] == -1).all() and (wr[t, len(row):] == 0).all()
+    return top, tr, wr
+
+
+@pytest.mark.parametrize("T,E,k,B,seed", [(3000, 16, 2, 128, 0), (700, 8, 3, 128, 1),
+                                          (40, 5, 2, 4, 2), (9, 3, 1, 2, 3), (500, 64, 8, 16, 4),
+                                          (200, 4, 2, 128, 5)])
+def test_token_rounding_definition(oracle_mod, T, E, k, B, seed):
+    """Every count becomes the nearest multiple of the tile (ties upward; downward when too
+    few tokens are left to add), the dropped entries are the worst-ranked ones and the added
+    tokens the best-ranked unrouted ones (checked against sorted() of the rank key), the
+    slot order is kept, and every weight is the float64 softmax at its expert."""
+    rng = np.random.default_rng(seed)
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    if seed == 2:  # ties: few distinct values, +0 and -0 among them
+        lg = np.array([-1.0, -0.0, 0.0, 0.5, 2.0], np.float32)[rng.integers(0, 5, (T, E))]
+    _check_rounding(oracle_mod, lg, k, B)
+
+
+def test_token_rounding_identity_and_skew(oracle_mod):
+    """Block 1 leaves the routing unchanged; a skewed routing (the skewed workload's bias)
+    rounds every expert, including ones with fewer than 64 entries, which drop to zero."""
+    rng = np.random.default_rng(7)
+    lg = rng.standard_normal((300, 8)).astype(np.float32)
+    top, w = oracle_mod.route(lg, 2)
+    tr, wr = oracle_mod.round_tokens(lg, top, block=1)
+    assert (tr == top).all() and np.allclose(wr, w, rtol=1e-15)
+    lg = (rng.standard_normal((2000, 32)) - 1.5 * np.log(np.arange(32) + 1.0)).astype(np.float32)
+    top, tr, wr = _check_rounding(oracle_mod, lg, 4, 128)
+    c2 = np.bincount(tr[tr >= 0], minlength=32)
+    assert (c2 % 128 == 0).all() and (c2 == 0).any()
+
+
+def test_absent_entries_contribute_nothing(oracle_mod):
+    """Forward and backward skip positions whose expert is -1 (the rounded routing's unused
+    positions): the same as a valid expert with weight 0 in the forward and in dx, with the
+    position's own routing-weight gradient 0."""
+    rng = np.random.default_rng(41)
+    T, h, f, E, k = 6, 128, 128, 4, 3
+    x, W1, W3, W2, logits = _rand_layer(rng, T, h, f, E, k)
+    top, w = oracle_mod.route(logits, k)
+    dy = rng.standard_normal((T, h)).astype(np.float32)
+    top_a, w_a = top.copy(), w.copy()
+    top_a[[1, 4], [2, 0]] = -1
+    w_z = w.copy()
+    w_z[[1, 4], [2, 0]] = 0.0
+    ya = oracle_mod.forward(x, W1, W3, W2, top_a, w_a)
+    yz = oracle_mod.forward(x, W1, W3, W2, top, w_z)
+    np.testing.assert_array_equal(ya, yz)
+    ga = oracle_mod.backward(x, dy, W1, W3, W2, top_a, w_a)
+    gz = oracle_mod.backward(x, dy, W1, W3, W2, top, w_z)
+    np.testing.assert_allclose(ga["dx"], gz["dx"], rtol=1e-13, atol=1e-15)
+    assert ga["dw"][1, 2] == 0 and ga["dw"][4, 0] == 0
+    assert ga["dw"][0, 0] == gz["dw"][0, 0]
 
 
 # ----------------------------------------------------------------------------------------
