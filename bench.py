@@ -54,6 +54,9 @@ def parse():
     p.add_argument("--router", action="store_true",
                    help="compute the logits with the linear router (x W_r^T) inside the step and, "
                         "for fwd+bwd workloads, run the router backward after the layer's")
+    p.add_argument("--token-rounding", action="store_true",
+                   help="the routing variant that rounds every expert's token count to a "
+                        "multiple of 128 (no padding rows)")
     p.add_argument("--save-x-only", action="store_true",
                    help="the memory variant: the forward saves X_pad only and the backward "
                         "recomputes A and Bm with one more GLU GEMM")
@@ -239,10 +242,12 @@ def tensor_peak(pk: dict, timed_s: float):
                             f"burst {pk['bf16']})")
 
 
-def config_of(w, router: bool, world: int, save_x_only: bool = False) -> dict:
+def config_of(w, router: bool, world: int, save_x_only: bool = False,
+              token_rounding: bool = False) -> dict:
     """The workload description shared by both arms of the bench."""
     return {"workload": f"{w.name} {w.describe()}" + (" +router" if router else "") +
-                        (" save_x_only" if save_x_only and w.backward else ""),
+                        (" save_x_only" if save_x_only and w.backward else "") +
+                        (" token_rounding" if token_rounding else ""),
             "T": w.T, "hidden": w.hidden, "ffn": w.ffn, "num_experts": w.E, "top_k": w.top_k,
             "l2": "inputs larger than L2 (expert weights %.2f GB per step)" %
                   (3 * w.E * w.hidden * w.ffn * 2 / 1e9),
@@ -338,7 +343,7 @@ def run_reference(args, w):
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(w, args.router, int(os.environ.get("WORLD_SIZE", "1")),
-                            args.save_x_only),
+                            args.save_x_only, args.token_rounding),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -374,8 +379,10 @@ def run_ours(args, w):
     B.load()
 
     recompute = bool(args.save_x_only) and w.backward
+    rounded = bool(args.token_rounding)
     dims = B.make_dims(w.T, w.hidden, w.ffn, w.E, w.top_k,
-                       flags=B.SAVE_X_ONLY if recompute else 0)
+                       flags=(B.SAVE_X_ONLY if recompute else 0) |
+                       (B.ROUTE_TOKEN_ROUNDING if rounded else 0))
     train = w.backward
     router = bool(args.router)
     inp = make_inputs(w, with_dy=train, with_router=router)
@@ -387,6 +394,7 @@ def run_ours(args, w):
     st = torch.cuda.current_stream()
     if train:
         xp, hb, yp = bufs.view("x_pad"), bufs.view("h"), bufs.view("y_pad")
+        ys = bufs.view("y_scale")
         if recompute:  # A and Bm live in backward scratch, recomputed there
             P_ = B.dmoe_padded_rows_max(dims)
             ab_bwd = torch.empty((P_, w.ffn), dtype=torch.bfloat16, device="cuda")
@@ -399,9 +407,11 @@ def run_ours(args, w):
         f32 = dict(dtype=torch.float32, device="cuda")
         grads = dict(dx=torch.empty_like(y), dw1=torch.empty((w.E, w.ffn, w.hidden), **f32),
                      dw3=torch.empty((w.E, w.ffn, w.hidden), **f32),
-                     dw2=torch.empty((w.E, w.hidden, w.ffn), **f32), dw=torch.empty((w.T, w.top_k), **f32))
+                     dw2=torch.empty((w.E, w.hidden, w.ffn), **f32),
+                     dw=torch.empty(B.dmoe_entries_max(dims) if rounded else (w.T, w.top_k), **f32))
     else:
         xp, hb, yp = bufs.step["x_pad"], bufs.step["h"], bufs.step["y_pad"]
+        ys = bufs.step["y_scale"]
         ab = bb = None
     names = ["map", "gather", "glu_gemm", "down_gemm", "scatter"]
     if train:
@@ -433,10 +443,10 @@ def run_ours(args, w):
         B.dmoe_expert_glu(dims, xp, dev["w1"], dev["w3"], bufs.map, hb, ab, bb, st)
         i += 1
         mark(i)
-        B.dmoe_expert_down(dims, hb, dev["w2"], bufs.map, yp, st)
+        B.dmoe_expert_down(dims, hb, dev["w2"], bufs.map, yp, ys, st)
         i += 1
         mark(i)
-        B.dmoe_padded_scatter(dims, yp, bufs.map, bufs.map.weights, y, st)
+        B.dmoe_padded_scatter(dims, yp, ys, bufs.map, bufs.map.weights, y, st)
         i += 1
         mark(i)
         if train:
@@ -604,9 +614,10 @@ def run_ours(args, w):
     pk = peaks()
     nb = int(bufs.map.num_blocks.item())
     P = nb * 128
-    N = w.entries
+    # entries the layer computes: T*k, or the rounded routing's list (no padding rows)
+    N = int(bufs.map.bins[-1].item()) if rounded else w.entries
     pad_frac = (P - N) / P
-    useful = w.useful_flops()
+    useful = w.useful_flops() * N // w.entries
     nhf = N * w.hidden * w.ffn
     flops = dict(glu_gemm=4 * nhf, down_gemm=2 * nhf, dglu_gemm=2 * nhf, dx_gemm=4 * nhf,
                  wgrad_gemm=6 * nhf, glu_recompute=4 * nhf)
@@ -652,7 +663,7 @@ def run_ours(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": config_of(w, router, world, recompute),
+        "config": config_of(w, router, world, recompute, rounded),
         "useful_tflops": useful / (ms_per_step / 1e3) / 1e12,
         "useful_tflops_frac_bf16": useful / (ms_per_step / 1e3) / 1e12 / pk_t,
         "padded_frac": pad_frac,

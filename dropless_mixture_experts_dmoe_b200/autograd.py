@@ -69,13 +69,17 @@ class DMoEFunction(torch.autograd.Function):
         dw1 = torch.empty(w1.shape, **f32)
         dw3 = torch.empty(w3.shape, **f32)
         dw2 = torch.empty(w2.shape, **f32)
-        dweights = torch.empty((dims.T, dims.top_k), **f32)
+        rounded = bool(dims.flags & B.ROUTE_TOKEN_ROUNDING)  # one weight per listed entry
+        dweights = torch.empty(B.dmoe_entries_max(dims) if rounded else (dims.T, dims.top_k), **f32)
         ws_bwd = torch.empty(max(B.dmoe_workspace_bytes(dims, B.WS_BACKWARD), 16),
                              dtype=torch.uint8, device=dev)
         B.dmoe_backward(dims, dy, w1, w3, w2, smap, ctx.saved_act, dx, dw1, dw3, dw2, dweights,
                         ws_bwd)
         dlogits = None
         if ctx.needs_input_grad[1]:
+            if rounded:
+                raise NotImplementedError("the logit gradient of the token-rounded routing is "
+                                          "not provided")
             dlogits = torch.empty_like(logits)
             B.dmoe_router_dlogits(dims, logits, smap, dweights, dlogits)
         return dx, dlogits, dw1, dw3, dw2, None, None

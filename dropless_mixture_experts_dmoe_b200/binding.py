@@ -22,7 +22,6 @@ MAX_TOP_K = 32
 
 WS_MAP, WS_FORWARD, WS_BACKWARD, WS_FORWARD_TRAIN, WS_ROUTER_BACKWARD = 0, 1, 2, 3, 4
 DGLU_TILE_COLS = 256
-DX_TILE_COLS = 256
 
 STATUS_NONFINITE_LOGITS = 0x1
 STATUS_EXPERT_OUT_OF_RANGE = 0x2
@@ -35,7 +34,9 @@ _I = ctypes.c_int
 
 
 ROUTE_RENORMALIZE = 0x1
+ROUTE_TOKEN_ROUNDING = 0x2
 SAVE_X_ONLY = 0x4
+SCALE_COLS = 128  # block floating point of Y_pad / dX_pad: one scale per row and 128 columns
 
 
 class dmoe_dims(ctypes.Structure):
@@ -50,7 +51,7 @@ class dmoe_dims(ctypes.Structure):
 
 
 MAP_FIELDS = ("top_experts", "weights", "tokens_per_expert", "bins", "padded_bins", "indices",
-              "bin_ids", "dest_row", "block_expert", "num_blocks", "status")
+              "bin_ids", "dest_row", "block_expert", "num_blocks", "status", "entry_offsets")
 
 
 class dmoe_map(ctypes.Structure):
@@ -79,6 +80,8 @@ def load():
     M = ctypes.POINTER(dmoe_map)
     lib.dmoe_padded_rows_max.argtypes = [D]
     lib.dmoe_padded_rows_max.restype = _SZ
+    lib.dmoe_entries_max.argtypes = [D]
+    lib.dmoe_entries_max.restype = _SZ
     lib.dmoe_workspace_bytes.argtypes = [D, _I]
     lib.dmoe_workspace_bytes.restype = _SZ
     lib.dmoe_saved_bytes.argtypes = [D, ctypes.POINTER(_SZ)]
@@ -89,8 +92,8 @@ def load():
     lib.dmoe_padded_gather.argtypes = [D, _P, M, _P, _P]
     lib.dmoe_expert_glu.argtypes = [D, _P, _P, _P, M, _P, _P, _P, _P]
     lib.dmoe_expert_glu_gather.argtypes = [D, _P, _P, _P, M, _P, _P, _P, _P]
-    lib.dmoe_expert_down.argtypes = [D, _P, _P, M, _P, _P]
-    lib.dmoe_padded_scatter.argtypes = [D, _P, M, _P, _P, _P]
+    lib.dmoe_expert_down.argtypes = [D, _P, _P, M, _P, _P, _P]
+    lib.dmoe_padded_scatter.argtypes = [D, _P, _P, M, _P, _P, _P]
     lib.dmoe_bwd_dglu.argtypes = [D, _P, _P, _P, _P, M, _P, _P, _P, _P, _P]
     lib.dmoe_bwd_scatter.argtypes = [D, _P, _P, _P, M, _P, _P, _P]
     lib.dmoe_router_forward.argtypes = [D, _P, _P, _P, _P, _P]
@@ -169,6 +172,10 @@ def dmoe_padded_rows_max(dims: dmoe_dims) -> int:
     return int(load().dmoe_padded_rows_max(ctypes.byref(dims)))
 
 
+def dmoe_entries_max(dims: dmoe_dims) -> int:
+    return int(load().dmoe_entries_max(ctypes.byref(dims)))
+
+
 def dmoe_workspace_bytes(dims: dmoe_dims, kind: int) -> int:
     return int(load().dmoe_workspace_bytes(ctypes.byref(dims), kind))
 
@@ -191,25 +198,34 @@ class SparseMap:
             raise DMoEError(-2, "SparseMap")
         i32 = dict(dtype=torch.int32, device=device)
         self.dims = dims
-        self.top_experts = torch.empty((T, k), **i32)
-        self.weights = torch.empty((T, k), dtype=torch.float32, device=device)
+        rounding = bool(dims.flags & ROUTE_TOKEN_ROUNDING)
+        N = dmoe_entries_max(dims)
+        if rounding:  # experts and weights of the token-major entry list
+            self.top_experts = torch.empty(N, **i32)
+            self.weights = torch.empty(N, dtype=torch.float32, device=device)
+        else:
+            self.top_experts = torch.empty((T, k), **i32)
+            self.weights = torch.empty((T, k), dtype=torch.float32, device=device)
         self.tokens_per_expert = torch.empty(E, **i32)
         self.bins = torch.empty(E, **i32)
         self.padded_bins = torch.empty(E, **i32)
-        self.indices = torch.empty(T * k, **i32)
-        self.bin_ids = torch.empty(T * k, **i32)
-        self.dest_row = torch.empty(T * k, **i32)
+        self.indices = torch.empty(N, **i32)
+        self.bin_ids = torch.empty(N, **i32)
+        self.dest_row = torch.empty(N, **i32)
         self.block_expert = torch.empty(max(P // BLOCKING, 1), **i32)
         self.num_blocks = torch.empty(1, **i32)
         self.status = torch.zeros(1, **i32)
-        self._c = dmoe_map(*[getattr(self, n).data_ptr() for n in MAP_FIELDS])
+        # token rounding: a token-major entry list (see include/dmoe.h)
+        self.entry_offsets = torch.empty(T + 1, **i32) if rounding else None
+        self._c = dmoe_map(*[0 if getattr(self, n) is None else getattr(self, n).data_ptr()
+                             for n in MAP_FIELDS])
 
     @property
     def c(self) -> dmoe_map:
         return self._c
 
     def as_dict(self) -> dict:
-        return {n: getattr(self, n) for n in MAP_FIELDS}
+        return {n: getattr(self, n) for n in MAP_FIELDS if getattr(self, n) is not None}
 
 
 def dmoe_sparse_map(dims: dmoe_dims, logits, smap: SparseMap, ws, stream=None):
@@ -257,15 +273,17 @@ def dmoe_expert_glu_gather(dims, x, w1, w3, smap: SparseMap, h_out, a_out=None, 
                                          _ptr(b_out), _stream(stream)), "dmoe_expert_glu_gather")
 
 
-def dmoe_expert_down(dims, h_in, w2, smap: SparseMap, y_pad, stream=None):
+def dmoe_expert_down(dims, h_in, w2, smap: SparseMap, y_pad, y_scale, stream=None):
+    """y_pad [P_max,h] fp16 and y_scale [P_max, ceil(h/128)] fp32: block floating point."""
     _check(load().dmoe_expert_down(ctypes.byref(dims), _ptr(h_in), _ptr(w2), ctypes.byref(smap.c),
-                                   _ptr(y_pad), _stream(stream)), "dmoe_expert_down")
+                                   _ptr(y_pad), _ptr(y_scale), _stream(stream)), "dmoe_expert_down")
 
 
-def dmoe_padded_scatter(dims, y_pad, smap: SparseMap, weights, y, stream=None):
-    _check(load().dmoe_padded_scatter(ctypes.byref(dims), _ptr(y_pad), ctypes.byref(smap.c),
-                                      _ptr(weights), _ptr(y), _stream(stream)),
-           "dmoe_padded_scatter")
+def dmoe_padded_scatter(dims, y_pad, y_scale, smap: SparseMap, weights, y, stream=None):
+    """y_scale None: y_pad is bf16; else block floating point (fp16 y_pad and its scales)."""
+    _check(load().dmoe_padded_scatter(ctypes.byref(dims), _ptr(y_pad), _ptr(y_scale),
+                                      ctypes.byref(smap.c), _ptr(weights), _ptr(y),
+                                      _stream(stream)), "dmoe_padded_scatter")
 
 
 def dmoe_bwd_dglu(dims, dy_pad, w2, a_saved, bm_saved, smap: SparseMap, da, dbm, hw, dw_part,
@@ -332,12 +350,13 @@ class Buffers:
     """Caller-side device allocations for one layer shape: map, workspaces, saved activations.
 
     train=True: ``saved`` (X_pad, A, Bm for the backward), the training forward workspace
-    ``ws_fwd`` (H, Y_pad), the backward workspace, and separate step buffers ``bstep``
-    (dy_pad, da, dbm, hw, dw_part, dx_pad, dx_scale) for driving the backward step entry points one by
-    one.  train=False: the inference workspace of ``dmoe_forward`` plus separate X_pad / H /
-    Y_pad tensors (``step``) for the forward step entry points.  ``view(name)`` gives bf16
-    [P_max, cols] views: x_pad, a, bm of the saved buffer, and h, y_pad of the forward
-    workspace (valid until the workspace is reused)."""
+    ``ws_fwd`` (H, Y_pad and its scales), the backward workspace, and separate step buffers
+    ``bstep`` (dy_pad, da, dbm, hw, dw_part, dx_pad, dx_scale) for driving the backward step
+    entry points one by one.  train=False: the inference workspace of ``dmoe_forward`` plus
+    separate X_pad / H / Y_pad / Y_pad-scale tensors (``step``) for the forward step entry
+    points.  ``view(name)`` gives [P_max, cols] views: x_pad, a, bm (bf16) of the saved buffer,
+    and h (bf16), y_pad (fp16) and y_scale (fp32) of the forward workspace (valid until the
+    workspace is reused)."""
 
     def __init__(self, dims: dmoe_dims, train: bool = False, device="cuda"):
         self.dims = dims
@@ -347,7 +366,9 @@ class Buffers:
         self.ws_map = torch.empty(max(dmoe_workspace_bytes(dims, WS_MAP), 16), **u8)
         self.train = train
         P, h, f = self.P, dims.hidden, dims.ffn
+        nsc = (h + SCALE_COLS - 1) // SCALE_COLS
         bf = dict(dtype=torch.bfloat16, device=device)
+        f32 = dict(dtype=torch.float32, device=device)
         self.saved = self.ws_bwd = None
         self.step = {}
         if train:
@@ -361,27 +382,35 @@ class Buffers:
             nt = (f + DGLU_TILE_COLS - 1) // DGLU_TILE_COLS
             self.bstep = dict(dy_pad=torch.empty((P, h), **bf), da=torch.empty((P, f), **bf),
                               dbm=torch.empty((P, f), **bf), hw=torch.empty((P, f), **bf),
-                              dw_part=torch.empty((P, nt), dtype=torch.float32, device=device),
+                              dw_part=torch.empty((P, nt), **f32),
                               dx_pad=torch.empty((P, h), dtype=torch.float16, device=device),
-                              dx_scale=torch.empty((P, (h + DX_TILE_COLS - 1) // DX_TILE_COLS),
-                                                   dtype=torch.float32, device=device))
+                              dx_scale=torch.empty((P, nsc), **f32))
         else:
             self.ws_fwd = torch.empty(dmoe_workspace_bytes(dims, WS_FORWARD), **u8)
             self.step = dict(x_pad=torch.empty((P, h), **bf), h=torch.empty((P, f), **bf),
-                             y_pad=torch.empty((P, h), **bf))
+                             y_pad=torch.empty((P, h), dtype=torch.float16, device=device),
+                             y_scale=torch.empty((P, nsc), **f32))
 
     def view(self, name: str) -> torch.Tensor:
-        """bf16 [P, cols] view of a saved activation (x_pad, a, bm) or, after a training
-        forward, of its workspace (h, y_pad)."""
+        """[P, cols] view of a saved activation (x_pad, a, bm) or, after a training forward,
+        of its workspace (h, y_pad, y_scale)."""
         if not self.train:
             return self.step[name]
-        cols = self.dims.hidden if name in ("x_pad", "y_pad") else self.dims.ffn
-        n = self.P * cols * 2
+        P, h, f = self.P, self.dims.hidden, self.dims.ffn
         if name in self.offsets:
+            cols = h if name == "x_pad" else f
             off = self.offsets[name]
-            return self.saved[off:off + n].view(torch.bfloat16).view(self.P, cols)
-        if name not in ("h", "y_pad"):
-            raise KeyError(f"{name} is not saved with these flags")
-        # forward workspace layout: H [P,f] | Y_pad [P,h], each start aligned to 256 bytes
-        off = 0 if name == "h" else (self.P * self.dims.ffn * 2 + 255) // 256 * 256
-        return self.ws_fwd[off:off + n].view(torch.bfloat16).view(self.P, cols)
+            return self.saved[off:off + P * cols * 2].view(torch.bfloat16).view(P, cols)
+        # forward workspace layout: H [P,f] bf16 | Y_pad [P,h] fp16 | scales [P, ceil(h/128)]
+        # fp32, each start aligned to 256 bytes
+        up = lambda v: (v + 255) // 256 * 256
+        nsc = (h + SCALE_COLS - 1) // SCALE_COLS
+        o_y = up(P * f * 2)
+        o_s = up(o_y + P * h * 2)
+        if name == "h":
+            return self.ws_fwd[:P * f * 2].view(torch.bfloat16).view(P, f)
+        if name == "y_pad":
+            return self.ws_fwd[o_y:o_y + P * h * 2].view(torch.float16).view(P, h)
+        if name == "y_scale":
+            return self.ws_fwd[o_s:o_s + P * nsc * 4].view(torch.float32).view(P, nsc)
+        raise KeyError(f"{name} is not saved with these flags")

@@ -19,6 +19,15 @@ inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+inline bool rounding(const dmoe_dims *d) { return (d->flags & DMOE_ROUTE_TOKEN_ROUNDING) != 0; }
+
+// Entries of the map: T*k, plus up to 64 added per expert with token rounding (an expert
+// rounds up only from a remainder of at least 64, adding at most 64).
+long long entries_of(const dmoe_dims *d) {
+  return (long long)d->T * d->top_k +
+         (rounding(d) ? (long long)(DMOE_BLOCKING / 2) * d->num_experts : 0);
+}
+
 // Shape validation shared by all entry points.
 int check_dims(const dmoe_dims *d) {
   if (!d) return DMOE_ERR_NULL;
@@ -27,8 +36,11 @@ int check_dims(const dmoe_dims *d) {
     return DMOE_ERR_SHAPE;
   if (d->ffn < DMOE_BLOCKING || d->ffn % DMOE_BLOCKING != 0) return DMOE_ERR_SHAPE;
   if (d->hidden < DMOE_BLOCKING || d->hidden % DMOE_BLOCKING != 0) return DMOE_ERR_SHAPE;
-  if (d->flags & ~(DMOE_ROUTE_RENORMALIZE | DMOE_SAVE_X_ONLY)) return DMOE_ERR_SHAPE;
-  const long long n = (long long)d->T * d->top_k;
+  if (d->flags & ~(DMOE_ROUTE_RENORMALIZE | DMOE_ROUTE_TOKEN_ROUNDING | DMOE_SAVE_X_ONLY))
+    return DMOE_ERR_SHAPE;
+  if (rounding(d) && ((d->flags & DMOE_ROUTE_RENORMALIZE) || d->T > kRoundMaxT))
+    return DMOE_ERR_SHAPE;
+  const long long n = entries_of(d);
   const long long pmax =
       (n + (long long)(DMOE_BLOCKING - 1) * d->num_experts) / DMOE_BLOCKING * DMOE_BLOCKING;
   if (n > 0x7FFFFFFFLL || pmax > 0x7FFFFFFFLL) return DMOE_ERR_TOO_LARGE;
@@ -36,7 +48,7 @@ int check_dims(const dmoe_dims *d) {
 }
 
 long long pmax_of(const dmoe_dims *d) {
-  const long long n = (long long)d->T * d->top_k;
+  const long long n = entries_of(d);
   return (n + (long long)(DMOE_BLOCKING - 1) * d->num_experts) / DMOE_BLOCKING * DMOE_BLOCKING;
 }
 
@@ -59,13 +71,49 @@ int check_device() {
   return known == 1 ? DMOE_OK : DMOE_ERR_DEVICE;
 }
 
-int check_map(const dmoe_map *m, bool need_weights) {
+int check_map(const dmoe_map *m, bool need_weights, const dmoe_dims *d = nullptr) {
   if (!m || !m->top_experts || !m->tokens_per_expert || !m->bins || !m->padded_bins ||
       !m->indices || !m->bin_ids || !m->dest_row || !m->block_expert || !m->num_blocks ||
       !m->status)
     return DMOE_ERR_NULL;
   if (need_weights && !m->weights) return DMOE_ERR_NULL;
+  if (d && rounding(d) && !m->entry_offsets) return DMOE_ERR_NULL;
   return DMOE_OK;
+}
+
+// The token-major entry list's row offsets (token rounding), else NULL (t*k + s).
+inline const int32_t *entry_offsets_of(const dmoe_dims *d, const dmoe_map *m) {
+  return rounding(d) ? m->entry_offsets : nullptr;
+}
+
+// Map workspace.  Plain routing: the map kernels' scratch for (T, E).  Token rounding: that
+// scratch sized for the larger of the two maps it builds (T tokens x k, then the entry list
+// as entries_of(d) single entries) | the top-k routing top [T,k] int32, weights [T,k] fp32 |
+// rank images [E][T] u16 | per-expert thresholds [3E] | per-token counts [T] | tile totals
+// [tiles] | tile offsets [tiles + 1].
+struct MapLayout {
+  size_t top, w, img, param, tokc, tsum, toff, total;
+};
+MapLayout map_layout(const dmoe_dims *d) {
+  MapLayout l = {};
+  size_t hist = sizeof(int32_t) * map_workspace_ints(d->T, d->num_experts);
+  if (!rounding(d)) {
+    l.total = align_up(hist);
+    return l;
+  }
+  const size_t hist2 = sizeof(int32_t) * map_workspace_ints((int)entries_of(d), d->num_experts);
+  if (hist2 > hist) hist = hist2;
+  const size_t T = (size_t)d->T, Tk = T * d->top_k, E = (size_t)d->num_experts;
+  const size_t tiles = (size_t)map_tiles(d->T);
+  l.top = align_up(hist);
+  l.w = align_up(l.top + Tk * 4);
+  l.img = align_up(l.w + Tk * 4);
+  l.param = align_up(l.img + E * T * 2);
+  l.tokc = align_up(l.param + 3 * E * 4);
+  l.tsum = align_up(l.tokc + T * 4);
+  l.toff = align_up(l.tsum + tiles * 4);
+  l.total = align_up(l.toff + (tiles + 1) * 4);
+  return l;
 }
 
 inline int launch_rc(cudaError_t e) { return e == cudaSuccess ? DMOE_OK : DMOE_ERR_LAUNCH; }
@@ -90,13 +138,16 @@ GemmProblem problem_of(const dmoe_dims *d, const dmoe_map *m) {
 
 inline int dglu_tiles(const dmoe_dims *d) { return (d->ffn + kDgluTileCols - 1) / kDgluTileCols; }
 
-inline int dx_tiles(const dmoe_dims *d) { return (d->hidden + kDxTileCols - 1) / kDxTileCols; }
+
+inline int scale_cols(const dmoe_dims *d) {
+  return (d->hidden + DMOE_SCALE_COLS - 1) / DMOE_SCALE_COLS;
+}
 
 inline bool save_x_only(const dmoe_dims *d) { return (d->flags & DMOE_SAVE_X_ONLY) != 0; }
 
 // Backward workspace layout: dY_pad [P,h] bf16, whose region is reused for dX_pad [P,h] fp16
 // once the weight gradients have read dY_pad | dA [P,f] | dBm [P,f] | Hw [P,f] | routing-weight
-// partials [P, ceil(f/256)] fp32 | dX_pad scales [P, ceil(h/256)] fp32 | with DMOE_SAVE_X_ONLY
+// partials [P, ceil(f/256)] fp32 | dX_pad scales [P, ceil(h/128)] fp32 | with DMOE_SAVE_X_ONLY
 // the recomputed A [P,f] and Bm [P,f]
 struct BwdLayout {
   size_t dy, da, db, hw, part, dxs, a, bm, total;
@@ -110,7 +161,7 @@ BwdLayout bwd_layout(const dmoe_dims *d) {
   l.hw = align_up(l.db + P * d->ffn * 2);
   l.part = align_up(l.hw + P * d->ffn * 2);
   l.dxs = align_up(l.part + P * dglu_tiles(d) * sizeof(float));
-  l.a = l.bm = l.total = align_up(l.dxs + P * dx_tiles(d) * sizeof(float));
+  l.a = l.bm = l.total = align_up(l.dxs + P * scale_cols(d) * sizeof(float));
   if (save_x_only(d)) {
     l.bm = align_up(l.a + P * d->ffn * 2);
     l.total = align_up(l.bm + P * d->ffn * 2);
@@ -118,17 +169,19 @@ BwdLayout bwd_layout(const dmoe_dims *d) {
   return l;
 }
 
-// Forward workspace layout: H [P,f] | Y_pad [P,h] | X_pad [P,h].  A training forward keeps
-// X_pad in the saved buffer and uses only the first two (`train` bytes).
+// Forward workspace layout: H [P,f] | Y_pad [P,h] fp16 | Y_pad scales [P, ceil(h/128)] fp32 |
+// X_pad [P,h].  A training forward keeps X_pad in the saved buffer and uses only the first
+// three (`train` bytes).
 struct FwdLayout {
-  size_t h, ypad, xpad, train, total;
+  size_t h, ypad, yscale, xpad, train, total;
 };
 FwdLayout fwd_layout(const dmoe_dims *d) {
   const size_t P = (size_t)pmax_of(d);
   FwdLayout l;
   l.h = 0;
   l.ypad = align_up(l.h + P * d->ffn * 2);
-  l.xpad = align_up(l.ypad + P * d->hidden * 2);
+  l.yscale = align_up(l.ypad + P * d->hidden * 2);
+  l.xpad = align_up(l.yscale + P * scale_cols(d) * sizeof(float));
   l.train = l.xpad;
   l.total = align_up(l.xpad + P * d->hidden * 2);
   return l;
@@ -148,11 +201,12 @@ RouterLayout router_layout(const dmoe_dims *d) {
   return l;
 }
 
-// The router's tensors have E columns; a TMA row must be a multiple of 16 bytes.
+// The router's tensors have E columns; a TMA row must be a multiple of 16 bytes.  Its
+// gradient is defined for the top-k routing only (not for the rounded one).
 inline int check_router_dims(const dmoe_dims *d) {
   int rc = check_dims(d);
   if (rc) return rc;
-  return (d->num_experts % 8 == 0) ? DMOE_OK : DMOE_ERR_SHAPE;
+  return (d->num_experts % 8 == 0 && !rounding(d)) ? DMOE_OK : DMOE_ERR_SHAPE;
 }
 
 // Saved activations: X_pad [P,h] | A [P,f] | Bm [P,f]; X_pad only with DMOE_SAVE_X_ONLY
@@ -174,6 +228,11 @@ void saved_layout(const dmoe_dims *d, size_t off[3], size_t *total) {
 
 extern "C" {
 
+size_t dmoe_entries_max(const dmoe_dims *dims) {
+  if (check_dims(dims) != DMOE_OK) return 0;
+  return (size_t)entries_of(dims);
+}
+
 size_t dmoe_padded_rows_max(const dmoe_dims *dims) {
   if (check_dims(dims) != DMOE_OK) return 0;
   return (size_t)pmax_of(dims);
@@ -183,7 +242,7 @@ size_t dmoe_workspace_bytes(const dmoe_dims *dims, int kind) {
   if (check_dims(dims) != DMOE_OK) return 0;
   switch (kind) {
     case DMOE_WS_MAP:
-      return align_up(sizeof(int32_t) * map_workspace_ints(dims->T, dims->num_experts));
+      return map_layout(dims).total;
     case DMOE_WS_FORWARD:
       return fwd_layout(dims).total;
     case DMOE_WS_FORWARD_TRAIN:
@@ -210,8 +269,8 @@ int dmoe_sparse_map(const dmoe_dims *dims, const void *logits, const dmoe_map *m
                     size_t ws_bytes, void *stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
-  if ((rc = check_map(map, logits != nullptr))) return rc;
-  if (!ws) return DMOE_ERR_NULL;
+  if ((rc = check_map(map, logits != nullptr || rounding(dims), dims))) return rc;
+  if (!ws || (rounding(dims) && !logits)) return DMOE_ERR_NULL;  // rounding ranks by logit
   if (ws_bytes < dmoe_workspace_bytes(dims, DMOE_WS_MAP)) return DMOE_ERR_WORKSPACE;
   if ((logits && !aligned16(logits)) || !aligned16(ws) || !aligned16(map->top_experts) ||
       (logits && !aligned16(map->weights)))
@@ -222,6 +281,40 @@ int dmoe_sparse_map(const dmoe_dims *dims, const void *logits, const dmoe_map *m
   const int nblk_cap = (int)(pmax_of(dims) / DMOE_BLOCKING);
   int32_t *tile_hist = static_cast<int32_t *>(ws);
   const bool renorm = (dims->flags & DMOE_ROUTE_RENORMALIZE) != 0;
+  if (rounding(dims)) {
+    // top-k routing and its counts, the rounding into the token-major entry list, then the
+    // map of that list (one entry per "token"; absent entries past its end are left out)
+    const MapLayout l = map_layout(dims);
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    int32_t *top = reinterpret_cast<int32_t *>(w + l.top);
+    float *wts = reinterpret_cast<float *>(w + l.w);
+    RoundScratch s;
+    s.img = reinterpret_cast<uint16_t *>(w + l.img);
+    s.param = reinterpret_cast<int32_t *>(w + l.param);
+    s.tok_count = reinterpret_cast<int32_t *>(w + l.tokc);
+    s.tile_sum = reinterpret_cast<int32_t *>(w + l.tsum);
+    s.tile_off = reinterpret_cast<int32_t *>(w + l.toff);
+    const int N = (int)entries_of(dims);
+    const uint16_t *lg = static_cast<const uint16_t *>(logits);
+    if ((rc = launch_rc(launch_route_hist(lg, T, E, k, false, top, wts, tile_hist, st)))) return rc;
+    if ((rc = launch_rc(launch_map_scan(T, E, tile_hist, map->tokens_per_expert, map->bins,
+                                        map->padded_bins, map->num_blocks, map->status, st))))
+      return rc;
+    if ((rc = launch_rc(launch_round_tokens(lg, top, wts, map->tokens_per_expert, T, E, k, s,
+                                            map->entry_offsets, map->top_experts, map->weights,
+                                            N, st))))
+      return rc;
+    if ((rc = launch_rc(launch_route_hist(nullptr, N, E, 1, false, map->top_experts, nullptr,
+                                          tile_hist, st, /*absent_ok=*/true))))
+      return rc;
+    if ((rc = launch_rc(launch_map_scan(N, E, tile_hist, map->tokens_per_expert, map->bins,
+                                        map->padded_bins, map->num_blocks, map->status, st,
+                                        /*or_status=*/true))))
+      return rc;
+    return launch_rc(launch_map_scatter(N, E, 1, nblk_cap, map->top_experts, tile_hist, map->bins,
+                                        map->padded_bins, map->indices, map->bin_ids,
+                                        map->dest_row, map->block_expert, st));
+  }
   if ((rc = launch_rc(launch_route_hist(static_cast<const uint16_t *>(logits), T, E, k, renorm,
                                         map->top_experts, map->weights, tile_hist, st))))
     return rc;
@@ -237,13 +330,13 @@ int dmoe_padded_gather(const dmoe_dims *dims, const void *x, const dmoe_map *map
                        void *stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
-  if ((rc = check_map(map, false))) return rc;
+  if ((rc = check_map(map, false, dims))) return rc;
   if (!x || !x_pad) return DMOE_ERR_NULL;
   if (!aligned16(x) || !aligned16(x_pad)) return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
   return launch_rc(launch_gather(dims->T, dims->hidden, dims->top_k, dims->num_experts, x,
                                  map->dest_row, map->tokens_per_expert, map->padded_bins, x_pad,
-                                 static_cast<cudaStream_t>(stream)));
+                                 static_cast<cudaStream_t>(stream), entry_offsets_of(dims, map)));
 }
 
 int dmoe_expert_glu(const dmoe_dims *dims, const void *x_pad, const void *w1, const void *w3,
@@ -266,6 +359,7 @@ int dmoe_expert_glu_gather(const dmoe_dims *dims, const void *x, const void *w1,
                            void *stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
+  if (rounding(dims)) return DMOE_ERR_SHAPE;  // its row gathers assume t*k + s entries
   if ((rc = check_map(map, false))) return rc;
   if (!x || !w1 || !w3 || !h_out) return DMOE_ERR_NULL;
   if ((a_out == nullptr) != (b_out == nullptr)) return DMOE_ERR_NULL;
@@ -278,27 +372,28 @@ int dmoe_expert_glu_gather(const dmoe_dims *dims, const void *x, const void *w1,
 }
 
 int dmoe_expert_down(const dmoe_dims *dims, const void *h_in, const void *w2,
-                     const dmoe_map *map, void *y_pad, void *stream) {
+                     const dmoe_map *map, void *y_pad, float *y_scale, void *stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if ((rc = check_map(map, false))) return rc;
-  if (!h_in || !w2 || !y_pad) return DMOE_ERR_NULL;
+  if (!h_in || !w2 || !y_pad || !y_scale) return DMOE_ERR_NULL;
   if (!aligned16(h_in) || !aligned16(w2) || !aligned16(y_pad)) return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
-  return launch_rc(
-      launch_down_gemm(problem_of(dims, map), h_in, w2, y_pad, static_cast<cudaStream_t>(stream)));
+  return launch_rc(launch_down_gemm(problem_of(dims, map), h_in, w2, y_pad, y_scale,
+                                    static_cast<cudaStream_t>(stream)));
 }
 
-int dmoe_padded_scatter(const dmoe_dims *dims, const void *y_pad, const dmoe_map *map,
-                        const float *weights, void *y, void *stream) {
+int dmoe_padded_scatter(const dmoe_dims *dims, const void *y_pad, const float *y_scale,
+                        const dmoe_map *map, const float *weights, void *y, void *stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
-  if ((rc = check_map(map, false))) return rc;
+  if ((rc = check_map(map, false, dims))) return rc;
   if (!y_pad || !y) return DMOE_ERR_NULL;
   if (!aligned16(y_pad) || !aligned16(y)) return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
-  return launch_rc(launch_combine(dims->T, dims->hidden, dims->top_k, y_pad, map->dest_row,
-                                  weights, y, static_cast<cudaStream_t>(stream)));
+  return launch_rc(launch_combine(dims->T, dims->hidden, dims->top_k, y_pad, y_scale,
+                                  map->dest_row, weights, y, static_cast<cudaStream_t>(stream),
+                                  entry_offsets_of(dims, map)));
 }
 
 int dmoe_forward(const dmoe_dims *dims, const void *x, const void *w1, const void *w3,
@@ -312,6 +407,7 @@ int dmoe_forward(const dmoe_dims *dims, const void *x, const void *w1, const voi
   const FwdLayout l = fwd_layout(dims);
   if (ws_bytes < (saved ? l.train : l.total)) return DMOE_ERR_WORKSPACE;
   uint8_t *w = static_cast<uint8_t *>(ws);
+  float *yscale = reinterpret_cast<float *>(w + l.yscale);
   uint8_t *xpad = w + l.xpad, *hbuf = w + l.h, *ypad = w + l.ypad, *abuf = nullptr,
           *bbuf = nullptr;
   if (saved) {
@@ -331,8 +427,8 @@ int dmoe_forward(const dmoe_dims *dims, const void *x, const void *w1, const voi
   // GLU GEMM through TMA row gathers, whose instruction rate cannot keep up with the MMAs.
   if ((rc = dmoe_padded_gather(dims, x, map, xpad, stream))) return rc;
   if ((rc = dmoe_expert_glu(dims, xpad, w1, w3, map, hbuf, abuf, bbuf, stream))) return rc;
-  if ((rc = dmoe_expert_down(dims, hbuf, w2, map, ypad, stream))) return rc;
-  return dmoe_padded_scatter(dims, ypad, map, map->weights, y, stream);
+  if ((rc = dmoe_expert_down(dims, hbuf, w2, map, ypad, yscale, stream))) return rc;
+  return dmoe_padded_scatter(dims, ypad, yscale, map, map->weights, y, stream);
 }
 
 int dmoe_bwd_dglu(const dmoe_dims *dims, const void *dy_pad, const void *w2, const void *a_saved,
@@ -356,14 +452,14 @@ int dmoe_bwd_scatter(const dmoe_dims *dims, const void *dx_pad, const float *dx_
                      void *stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
-  if ((rc = check_map(map, false))) return rc;
+  if ((rc = check_map(map, false, dims))) return rc;
   if (!dx_pad || !dx_scale || !dw_part || !dx || !dweights) return DMOE_ERR_NULL;
   if (!aligned16(dx_pad) || !aligned16(dx)) return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
   return launch_rc(launch_bwd_scatter(dims->T, dims->hidden, dims->top_k, dx_pad, dx_scale,
-                                      map->dest_row,
-                                      dw_part, dglu_tiles(dims), dx, dweights,
-                                      static_cast<cudaStream_t>(stream)));
+                                      map->dest_row, dw_part, dglu_tiles(dims), dx, dweights,
+                                      static_cast<cudaStream_t>(stream),
+                                      entry_offsets_of(dims, map)));
 }
 
 int dmoe_bwd_dx(const dmoe_dims *dims, const void *da, const void *dbm, const void *w1,

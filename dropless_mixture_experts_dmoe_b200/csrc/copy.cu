@@ -24,6 +24,19 @@ __device__ __forceinline__ uint4 ld_nc_v4(const uint4 *p) {
   return v;
 }
 
+// The entries of token t: [t*k, t*k + k), or [offsets[t], offsets[t+1]) for a token-major
+// entry list (the rounded routing, where tokens have different entry counts).
+__device__ __forceinline__ void token_entries(const int32_t *__restrict__ offsets, int t, int k,
+                                              long long &base, int &cnt) {
+  if (offsets) {
+    base = offsets[t];
+    cnt = offsets[t + 1] - (int)base;
+  } else {
+    base = (long long)t * k;
+    cnt = k;
+  }
+}
+
 // A row slice is 32 * kGatherVPL 16-byte vectors (4 KB); a token's row is split into
 // ceil(vpr / slice) slices so that short-T workloads still keep many warps busy.
 constexpr int kSliceVecs = 32 * kGatherVPL;
@@ -35,7 +48,8 @@ __global__ void __launch_bounds__(kCopyThreads) k_gather(int T, int h, int k, in
                                                          const int32_t *__restrict__ dest_row,
                                                          const int32_t *__restrict__ counts,
                                                          const int32_t *__restrict__ padded_bins,
-                                                         uint4 *__restrict__ x_pad) {
+                                                         uint4 *__restrict__ x_pad,
+                                                         const int32_t *__restrict__ offsets) {
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
@@ -49,7 +63,9 @@ __global__ void __launch_bounds__(kCopyThreads) k_gather(int T, int h, int k, in
     if (it < ntok) {
       const int t = (int)(it / S);
       const int v0 = (int)(it - (long long)t * S) * kSliceVecs;
-      const int d = (lane < k) ? dest_row[(size_t)t * k + lane] : -1;
+      long long base;
+      int cnt;
+      token_entries(offsets, t, k, base, cnt);
       const uint4 *src = x + (size_t)t * vpr;
       uint4 buf[kGatherVPL];
 #pragma unroll
@@ -57,14 +73,18 @@ __global__ void __launch_bounds__(kCopyThreads) k_gather(int T, int h, int k, in
         const int v = v0 + u * 32 + lane;
         if (v < vpr) buf[u] = ld_nc_v4(src + v);
       }
-      for (int s = 0; s < k; ++s) {
-        const int r = __shfl_sync(0xFFFFFFFFu, d, s);
-        if (r < 0) continue;
-        uint4 *dst = x_pad + (size_t)r * vpr;
+      for (int c0 = 0; c0 < cnt; c0 += 32) {  // one pass of up to 32 entries (k <= 32)
+        const int nc = min(32, cnt - c0);
+        const int d = (lane < nc) ? dest_row[base + c0 + lane] : -1;
+        for (int s = 0; s < nc; ++s) {
+          const int r = __shfl_sync(0xFFFFFFFFu, d, s);
+          if (r < 0) continue;
+          uint4 *dst = x_pad + (size_t)r * vpr;
 #pragma unroll
-        for (int u = 0; u < kGatherVPL; ++u) {
-          const int v = v0 + u * 32 + lane;
-          if (v < vpr) dst[v] = buf[u];
+          for (int u = 0; u < kGatherVPL; ++u) {
+            const int v = v0 + u * 32 + lane;
+            if (v < vpr) dst[v] = buf[u];
+          }
         }
       }
     } else {
@@ -83,106 +103,32 @@ __global__ void __launch_bounds__(kCopyThreads) k_gather(int T, int h, int k, in
   }
 }
 
-// y_t = sum_{s<k} w_ts * Y_pad[dest_row[t*k+s]]: fp32, slot order, one fused multiply-add per
-// slot and element, rounded once to bf16.  weights == NULL: w = 1.
-// VPL 16-byte vectors per lane for each of SLOTS slots are loaded before any is consumed
-// (VPL * SLOTS = 16 loads in flight per lane): few slots (small top_k) take wide row pieces.
+// Token-major sum of each token's padded rows, the padded_scatter of walkthrough section 4.2:
+//   out_t = bf16(sum_s c_s * rows[dest_row[e_s]])   over the token's entries e_s in order,
+// fp32 accumulation rounded once, no atomics.  Forward combine: c_s = w_s, the routing weight
+// (weights != NULL).  Backward (the gradient of the gather, section 4.2): c_s = 1 and, with
+// dweights != NULL, the routing-weight gradient dweights[e] = sum_{n<nt} part[dest_row[e]*nt + n]
+// in column-tile order.  Row format: bf16 (scale == NULL) or block floating point, fp16 values
+// times a power-of-two scale per row and DMOE_SCALE_COLS columns (scale[r * nsc + c / 128]),
+// which is exact in fp32, so each entry adds c_s * scale * value with one rounding.
+// A lane covers 8 consecutive columns (one 16-byte vector) per entry; VPL vectors per lane
+// and SLOTS entries are loaded before any is consumed.
 template <int VPL, int SLOTS>
-__global__ void __launch_bounds__(kCopyThreads) k_combine(int T, int h, int k,
-                                                          const uint4 *__restrict__ y_pad,
+__global__ void __launch_bounds__(kCopyThreads, 2) k_combine(int T, int h, int k,
+                                                          const uint4 *__restrict__ rows,
+                                                          const float *__restrict__ scale,
                                                           const int32_t *__restrict__ dest_row,
                                                           const float *__restrict__ weights,
-                                                          uint4 *__restrict__ y) {
+                                                          uint4 *__restrict__ out,
+                                                          const float *__restrict__ part, int nt,
+                                                          float *__restrict__ dweights,
+                                                          const int32_t *__restrict__ offsets) {
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
-  const int vpr = h >> 3;
-  const int S = (vpr + kSliceVecs - 1) / kSliceVecs;
-  const long long items = (long long)T * S;
-  const long long nw = (long long)gridDim.x * kCopyWarps;
-  for (long long it = (long long)blockIdx.x * kCopyWarps + (threadIdx.x >> 5); it < items;
-       it += nw) {
-    const int t = (int)(it / S);
-    const int vs = (int)(it - (long long)t * S) * kSliceVecs;
-    const int ve = min(vpr, vs + kSliceVecs);
-    const int d = (lane < k) ? dest_row[(size_t)t * k + lane] : -1;
-    const float wl = (lane < k) ? (weights ? weights[(size_t)t * k + lane] : 1.0f) : 0.0f;
-    for (int v0 = vs; v0 < ve; v0 += 32 * VPL) {
-      float acc[VPL][8];
-#pragma unroll
-      for (int u = 0; u < VPL; ++u)
-#pragma unroll
-        for (int q = 0; q < 8; ++q) acc[u][q] = 0.0f;
-      for (int s0 = 0; s0 < k; s0 += SLOTS) {
-        uint4 buf[SLOTS][VPL];
-#pragma unroll
-        for (int ss = 0; ss < SLOTS; ++ss) {
-          const int s = s0 + ss;
-          const int r = __shfl_sync(0xFFFFFFFFu, d, s & 31);
-          if (s < k && r >= 0) {
-#pragma unroll
-            for (int u = 0; u < VPL; ++u) {
-              const int v = v0 + u * 32 + lane;
-              if (v < ve) buf[ss][u] = ld_nc_v4(y_pad + (size_t)r * vpr + v);
-            }
-          }
-        }
-#pragma unroll
-        for (int ss = 0; ss < SLOTS; ++ss) {
-          const int s = s0 + ss;
-          const int r = __shfl_sync(0xFFFFFFFFu, d, s & 31);
-          const float ws = __shfl_sync(0xFFFFFFFFu, wl, s & 31);
-          if (s < k && r >= 0) {
-#pragma unroll
-            for (int u = 0; u < VPL; ++u) {
-              const uint32_t *q = reinterpret_cast<const uint32_t *>(&buf[ss][u]);
-#pragma unroll
-              for (int p = 0; p < 4; ++p) {
-                acc[u][2 * p] = fmaf(ws, bf16_lo(q[p]), acc[u][2 * p]);
-                acc[u][2 * p + 1] = fmaf(ws, bf16_hi(q[p]), acc[u][2 * p + 1]);
-              }
-            }
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < VPL; ++u) {
-        const int v = v0 + u * 32 + lane;
-        if (v < ve) {
-          uint4 o;
-          o.x = pack_bf16x2(acc[u][0], acc[u][1]);
-          o.y = pack_bf16x2(acc[u][2], acc[u][3]);
-          o.z = pack_bf16x2(acc[u][4], acc[u][5]);
-          o.w = pack_bf16x2(acc[u][6], acc[u][7]);
-          y[(size_t)t * vpr + v] = o;
-        }
-      }
-    }
-  }
-}
-
-// Backward scatter-sum (the gradient of the gather, walkthrough section 4.2): dx_t =
-// bf16(sum_{s<k} dX_pad[dest_row[t*k+s]]) in fp32, slot order, rounded once.  dX_pad rows are
-// block floating point: fp16 values times a power-of-two scale per row and 256-column tile
-// (scale[r * nsc + c / 256]); fp16 * scale is exact in fp32, so each slot adds its value with
-// one fused multiply-add.  With it the routing-weight gradient dweights[t*k+s] =
-// sum_{n<nt} part[dest_row[t*k+s] * nt + n] in column-tile order.  A lane covers 8 consecutive
-// columns (one 16-byte vector) per slot; VPL such vectors per lane and SLOTS slots are loaded
-// before any is consumed.
-template <int VPL, int SLOTS>
-__global__ void __launch_bounds__(kCopyThreads, 2) k_scatter_sum(int T, int h, int k,
-                                                              const uint4 *__restrict__ dx_pad,
-                                                              const float *__restrict__ scale,
-                                                              const int32_t *__restrict__ dest_row,
-                                                              uint4 *__restrict__ dx,
-                                                              const float *__restrict__ part,
-                                                              int nt,
-                                                              float *__restrict__ dweights) {
-  pdl_wait();
-  pdl_trigger();
-  const int lane = threadIdx.x & 31;
-  const int vpr = h >> 3;      // 16-byte vectors (8 columns) per row
-  const int nsc = (h + 255) >> 8;  // scales per row
+  const int vpr = h >> 3;                                      // 16-byte vectors per row
+  const int nsc = (h + DMOE_SCALE_COLS - 1) / DMOE_SCALE_COLS;  // scales per row
+  constexpr int kVecPerScale = DMOE_SCALE_COLS / 8;
   constexpr int kSlice = 32 * VPL;
   const int S = (vpr + kSlice - 1) / kSlice;
   const long long items = (long long)T * S;
@@ -191,48 +137,59 @@ __global__ void __launch_bounds__(kCopyThreads, 2) k_scatter_sum(int T, int h, i
        it += nw) {
     const int t = (int)(it / S);
     const int v0 = (int)(it - (long long)t * S) * kSlice;
-    const int d = (lane < k) ? dest_row[(size_t)t * k + lane] : -1;
-    if (v0 == 0 && lane < k) {
-      float g = 0.0f;
-      if (d >= 0)
-        for (int n = 0; n < nt; ++n) g += __ldg(part + (size_t)d * nt + n);
-      dweights[(size_t)t * k + lane] = g;  // 0 for an entry dropped from the map
-    }
+    long long base;
+    int cnt;
+    token_entries(offsets, t, k, base, cnt);
     float acc[VPL][8];
 #pragma unroll
     for (int u = 0; u < VPL; ++u)
 #pragma unroll
       for (int q = 0; q < 8; ++q) acc[u][q] = 0.0f;
-    for (int s0 = 0; s0 < k; s0 += SLOTS) {
-      uint4 buf[SLOTS][VPL];
-      float sc[SLOTS][VPL];
+    for (int c0 = 0; c0 < cnt; c0 += 32) {  // one pass of up to 32 entries (k <= 32)
+      const int kk = min(32, cnt - c0);
+      const int d = (lane < kk) ? dest_row[base + c0 + lane] : -1;
+      const float wl = (lane < kk && weights) ? weights[base + c0 + lane] : 1.0f;
+      if (dweights && v0 == 0 && lane < kk) {
+        float g = 0.0f;
+        if (d >= 0)
+          for (int n = 0; n < nt; ++n) g += __ldg(part + (size_t)d * nt + n);
+        dweights[base + c0 + lane] = g;  // 0 for an entry dropped from the map
+      }
+      for (int s0 = 0; s0 < kk; s0 += SLOTS) {
+        uint4 buf[SLOTS][VPL];
+        float cf[SLOTS][VPL];
 #pragma unroll
-      for (int ss = 0; ss < SLOTS; ++ss) {
-        const int s = s0 + ss;
-        const int r = __shfl_sync(0xFFFFFFFFu, d, s & 31);
-        if (s < k && r >= 0) {
+        for (int ss = 0; ss < SLOTS; ++ss) {
+          const int s = s0 + ss;
+          const int r = __shfl_sync(0xFFFFFFFFu, d, s & 31);
+          const float ws = __shfl_sync(0xFFFFFFFFu, wl, s & 31);
+          if (s < kk && r >= 0) {
 #pragma unroll
-          for (int u = 0; u < VPL; ++u) {
-            const int v = v0 + u * 32 + lane;
-            if (v < vpr) {
-              buf[ss][u] = ld_nc_v4(dx_pad + (size_t)r * vpr + v);
-              sc[ss][u] = __ldg(scale + (size_t)r * nsc + (v >> 5));
+            for (int u = 0; u < VPL; ++u) {
+              const int v = v0 + u * 32 + lane;
+              if (v < vpr) {
+                buf[ss][u] = ld_nc_v4(rows + (size_t)r * vpr + v);
+                cf[ss][u] = scale ? ws * __ldg(scale + (size_t)r * nsc + v / kVecPerScale) : ws;
+              }
             }
           }
         }
-      }
 #pragma unroll
-      for (int ss = 0; ss < SLOTS; ++ss) {
-        const int s = s0 + ss;
-        const int r = __shfl_sync(0xFFFFFFFFu, d, s & 31);
-        if (s < k && r >= 0) {
+        for (int ss = 0; ss < SLOTS; ++ss) {
+          const int s = s0 + ss;
+          const int r = __shfl_sync(0xFFFFFFFFu, d, s & 31);
+          if (s < kk && r >= 0) {
 #pragma unroll
-          for (int u = 0; u < VPL; ++u) {
-            const uint32_t *q = reinterpret_cast<const uint32_t *>(&buf[ss][u]);
+            for (int u = 0; u < VPL; ++u) {
+              const uint32_t *q = reinterpret_cast<const uint32_t *>(&buf[ss][u]);
+              const float c = cf[ss][u];
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
-              acc[u][2 * p] = fmaf(f16_lo(q[p]), sc[ss][u], acc[u][2 * p]);
-              acc[u][2 * p + 1] = fmaf(f16_hi(q[p]), sc[ss][u], acc[u][2 * p + 1]);
+              for (int p = 0; p < 4; ++p) {
+                const float lo = scale ? f16_lo(q[p]) : bf16_lo(q[p]);
+                const float hi = scale ? f16_hi(q[p]) : bf16_hi(q[p]);
+                acc[u][2 * p] = fmaf(c, lo, acc[u][2 * p]);
+                acc[u][2 * p + 1] = fmaf(c, hi, acc[u][2 * p + 1]);
+              }
             }
           }
         }
@@ -247,7 +204,7 @@ __global__ void __launch_bounds__(kCopyThreads, 2) k_scatter_sum(int T, int h, i
         o.y = pack_bf16x2(acc[u][2], acc[u][3]);
         o.z = pack_bf16x2(acc[u][4], acc[u][5]);
         o.w = pack_bf16x2(acc[u][6], acc[u][7]);
-        dx[(size_t)t * vpr + v] = o;
+        out[(size_t)t * vpr + v] = o;
       }
     }
   }
@@ -265,34 +222,38 @@ static long long slices(int h) { return ((h >> 3) + kSliceVecs - 1) / kSliceVecs
 
 cudaError_t launch_gather(int T, int h, int k, int E, const void *x, const int32_t *dest_row,
                           const int32_t *counts, const int32_t *padded_bins, void *x_pad,
-                          cudaStream_t st) {
+                          cudaStream_t st, const int32_t *offsets) {
   const long long items = (long long)T * slices(h) + (long long)kBlock * E;
   return launch_pdl(k_gather, copy_grid(items), kCopyThreads, 0, st, T, h, k, E,
                     static_cast<const uint4 *>(x), dest_row, counts, padded_bins,
-                    static_cast<uint4 *>(x_pad));
+                    static_cast<uint4 *>(x_pad), offsets);
 }
 
-cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const int32_t *dest_row,
-                           const float *weights, void *y, cudaStream_t st) {
-  const int grid = copy_grid((long long)T * slices(h));
-  const uint4 *src = static_cast<const uint4 *>(y_pad);
-  uint4 *dst = static_cast<uint4 *>(y);
-  auto kernel = (k <= 2) ? k_combine<8, 2> : (k <= 4) ? k_combine<4, 4> : k_combine<2, 8>;
-  return launch_pdl(kernel, grid, kCopyThreads, 0, st, T, h, k, src, dest_row, weights, dst);
+// Shape of the combine: at most 16 row loads in flight per lane within 128 registers (two
+// CTAs per SM); few entries per token take wide row pieces.
+static cudaError_t combine(int T, int h, int k, const void *rows, const float *scale,
+                           const int32_t *dest_row, const float *weights, void *out,
+                           const float *part, int nt, float *dweights, const int32_t *offsets,
+                           cudaStream_t st) {
+  const int vpl = (k <= 2) ? 4 : 2;
+  auto kernel = (k <= 2) ? k_combine<4, 2> : (k <= 4) ? k_combine<2, 4> : k_combine<2, 8>;
+  const long long items = (long long)T * (((h >> 3) + 32 * vpl - 1) / (32 * vpl));
+  return launch_pdl(kernel, copy_grid(items), kCopyThreads, 0, st, T, h, k,
+                    static_cast<const uint4 *>(rows), scale, dest_row, weights,
+                    static_cast<uint4 *>(out), part, nt, dweights, offsets);
+}
+
+cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const float *y_scale,
+                           const int32_t *dest_row, const float *weights, void *y,
+                           cudaStream_t st, const int32_t *offsets) {
+  return combine(T, h, k, y_pad, y_scale, dest_row, weights, y, nullptr, 0, nullptr, offsets, st);
 }
 
 cudaError_t launch_bwd_scatter(int T, int h, int k, const void *dx_pad, const float *dx_scale,
                                const int32_t *dest_row, const float *part, int nt, void *dx,
-                               float *dweights, cudaStream_t st) {
-  // 16-byte vectors per lane and slot: at most 16 loads in flight per lane within 128
-  // registers (two CTAs per SM)
-  const int vpl = (k <= 2) ? 4 : 2;
-  auto kernel = (k <= 2) ? k_scatter_sum<4, 2> : (k <= 4) ? k_scatter_sum<2, 4>
-                                                          : k_scatter_sum<2, 8>;
-  const long long items = (long long)T * (((h >> 3) + 32 * vpl - 1) / (32 * vpl));
-  return launch_pdl(kernel, copy_grid(items), kCopyThreads, 0, st, T, h, k,
-                    static_cast<const uint4 *>(dx_pad), dx_scale, dest_row,
-                    static_cast<uint4 *>(dx), part, nt, dweights);
+                               float *dweights, cudaStream_t st, const int32_t *offsets) {
+  return combine(T, h, k, dx_pad, dx_scale, dest_row, nullptr, dx, part, nt, dweights, offsets,
+                 st);
 }
 
 }  // namespace dmoe

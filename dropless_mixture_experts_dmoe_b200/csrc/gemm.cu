@@ -47,16 +47,17 @@
 //         fused into the GEMM's operand load).  32 gather instructions per 16 KB stage are
 //         more than the TMA unit issues in one stage's MMA time: about 3x slower than
 //         gather kernel + GLU on B200, so it is not the default path.
-//   DOWN  A = H (K)          B = W2_e (K)                 out Y_pad
+//   DOWN  A = H (K)          B = W2_e (K)                 out Y_pad (block floating point:
+//         fp16 values and a power-of-two scale per row and 128 columns)
 //   DGLU  A = dY_pad (K)     B = W2_e^T (MN)              G = dy W2_e (dY_pad holds the
 //         token rows of dy, unweighted); the epilogue recomputes the activation from the saved
 //         A, Bm (s = sigmoid(A), h = A*s*Bm) and, with w the routing weight of the row, writes
 //         dA = w*G*Bm*s*(1+A(1-s)), dBm = w*G*A*s, Hw = w*h (the dW2 operand) and the partial
 //         routing-weight gradient sum_cols G*h of the row over the tile's columns
 //   DX    A = dA then dBm (K), B = W1_e then W3_e (MN), one accumulator over both K passes;
-//         out dX_pad as fp16 with a power-of-two scale per row and 256-column tile (the k
-//         rows of a token are summed afterwards; rounding each of them to bf16 first would put
-//         k bf16 roundings into every dx element)
+//         out dX_pad, block floating point as Y_pad (the k rows of a token are summed
+//         afterwards; rounding each of them to bf16 first would put k bf16 roundings into every
+//         output element)
 //   WGRAD dW1_e = dA^T X_pad, dW3_e = dBm^T X_pad, dW2_e = dY_pad^T Hw over the expert's
 //         padded rows (both operands MN-major); fp32 outputs; experts without rows get exact
 //         zeros.
@@ -177,7 +178,7 @@ struct GemmParams {
   const __nv_bfloat16 *in0, *in1;  // DGLU: saved A, Bm
   const float *weights;            // DGLU: routing weight of each flattened entry
   float *part;                     // DGLU: [P_max, n_tiles] partial routing-weight gradients;
-                                   // DX: [P_max, n_tiles] inverse scales of the dX_pad rows
+                                   // DOWN, DX: [P_max, ceil(h/128)] scales of the output rows
   int total;                       // router modes: number of pair tiles
   int split_k;                     // RWGRAD: 64-wide K steps per split
   int Ep;                          // RWGRAD: rows of one split's slab (E rounded up to 128)
@@ -474,75 +475,46 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
         st.emit(&p.tmo[2], w, n0 + c, y0);
       }
     }
-  } else if (MODE == MODE_DX) {
-    // dX_pad in block floating point: fp16 values with one power-of-two scale per row and
-    // 256-column tile, so that the largest value of the tile's row lands in [2^13, 2^14) and
-    // every value keeps fp16's 11 significant bits (bf16 has 8); the scale's inverse goes to
-    // p.part[row * n_tiles + n].  Pass 1 reads the row's accumulator for its largest magnitude,
-    // pass 2 converts and stores 64-column boxes.
-    static_assert(MODE != MODE_DX || EPI == 4, "one warp holds a row's whole tile");
-    const int n0 = tl.n * BN;
-    const int ncols = min(BN, p.h - n0);  // multiple of 64
-    float m = 0.0f;
-#pragma unroll 1
-    for (int c = 0; c < ncols; c += 32) {
-      uint32_t v[32];
-      tmem_ld32(tb + c, v);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(__uint_as_float(v[i])));
-    }
-    int es = 13 - ((int)((__float_as_uint(m) >> 23) & 0xFFu) - 127);  // m * 2^es < 2^14
-    if (m == 0.0f || !(m <= 3.402823466e38f)) es = 0;  // zero, inf or NaN: unscaled
-    es = min(max(es, -126), 126);
-    const float sc = __uint_as_float((uint32_t)(127 + es) << 23);
-    p.part[(size_t)(y0 + lane) * p.n_tiles + tl.n] = __uint_as_float((uint32_t)(127 - es) << 23);
-#pragma unroll 1
-    for (int c = 0; c < ncols; c += 64) {
-      uint32_t v0[32], v1[32], w[32];
-      tmem_ld32(tb + c, v0);
-      tmem_ld32(tb + c + 32, v1);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        w[i] = pack_f16x2(__uint_as_float(v0[2 * i]) * sc, __uint_as_float(v0[2 * i + 1]) * sc);
-        w[16 + i] = pack_f16x2(__uint_as_float(v1[2 * i]) * sc, __uint_as_float(v1[2 * i + 1]) * sc);
-      }
-      st.emit(&p.tmo[0], w, n0 + c, y0);
-    }
-  } else if (MODE == MODE_DOWN) {
+  } else if (MODE == MODE_DOWN || MODE == MODE_DX) {
+    // Y_pad / dX_pad in block floating point: per DMOE_SCALE_COLS columns of this thread's row,
+    // the largest magnitude picks a power-of-two scale that puts it into [2^13, 2^14); the
+    // values go out as fp16 (11 significant bits) and 1/scale to p.part[row * nsc + chunk].
     const int n0 = tl.n * BN + half * kw;  // this warp's first column
     const int ncols = min(kw, p.h - n0);   // multiple of 64 (may be <= 0)
     if (ncols <= 0) return;
     tb += (uint32_t)(half * kw);
-    uint32_t v0[32], v1[32], w[32];
-    if (EPI == 8 && ncols == 2 * 64) {  // both of this warp's boxes staged, one proxy fence
-      uint32_t v2[32], v3[32];
-      tmem_ld32(tb, v0);
-      tmem_ld32(tb + 32, v1);
-      tmem_ld32(tb + 64, v2);
-      tmem_ld32(tb + 96, v3);
-      st.reclaim();
-      tmem_ld_wait();
-      pack_bf16_row(v0, v1, w);
-      st.put(0, w);
-      pack_bf16_row(v2, v3, w);
-      st.put(1, w);
-      st.flush(&p.tmo[0], 2, n0, 64, y0);
-      return;
-    }
-    tmem_ld32(tb, v0);
-    tmem_ld32(tb + 32, v1);
-    tmem_ld_wait();
+    const int nsc = (p.h + DMOE_SCALE_COLS - 1) / DMOE_SCALE_COLS;
+    float *srow = p.part + (size_t)(y0 + lane) * nsc;
 #pragma unroll 1
-    for (int c = 0; c < ncols; c += 64) {
-      pack_bf16_row(v0, v1, w);
-      if (c + 64 < ncols) {  // the next box's accumulator loads overlap this box's store
-        tmem_ld32(tb + c + 64, v0);
-        tmem_ld32(tb + c + 96, v1);
+    for (int c0 = 0; c0 < ncols; c0 += DMOE_SCALE_COLS) {
+      const int cn = min(DMOE_SCALE_COLS, ncols - c0);
+      float m = 0.0f;
+#pragma unroll 1
+      for (int c = 0; c < cn; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tb + c0 + c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(__uint_as_float(v[i])));
       }
-      st.emit(&p.tmo[0], w, n0 + c, y0);
-      tmem_ld_wait();
+      int es = 13 - ((int)((__float_as_uint(m) >> 23) & 0xFFu) - 127);  // m * 2^es < 2^14
+      if (m == 0.0f || !(m <= 3.402823466e38f)) es = 0;  // zero, inf or NaN: unscaled
+      es = min(max(es, -126), 126);
+      const float sc = __uint_as_float((uint32_t)(127 + es) << 23);
+      srow[(n0 + c0) / DMOE_SCALE_COLS] = __uint_as_float((uint32_t)(127 - es) << 23);
+#pragma unroll 1
+      for (int c = 0; c < cn; c += 64) {
+        uint32_t v0[32], v1[32], w[32];
+        tmem_ld32(tb + c0 + c, v0);
+        tmem_ld32(tb + c0 + c + 32, v1);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          w[i] = pack_f16x2(__uint_as_float(v0[2 * i]) * sc, __uint_as_float(v0[2 * i + 1]) * sc);
+          w[16 + i] = pack_f16x2(__uint_as_float(v1[2 * i]) * sc, __uint_as_float(v1[2 * i + 1]) * sc);
+        }
+        st.emit(&p.tmo[0], w, n0 + c0 + c, y0);
+      }
     }
   } else if (MODE == MODE_DGLU) {
     static_assert(MODE != MODE_DGLU || EPI == 4, "one warp per row holds a row's partial sum");
@@ -1120,7 +1092,7 @@ cudaError_t launch_glu_gather_gemm(const GemmProblem &g, const void *x, const vo
 }
 
 cudaError_t launch_down_gemm(const GemmProblem &g, const void *h_in, const void *w2, void *y_pad,
-                             cudaStream_t st) {
+                             float *y_scale, cudaStream_t st) {
   GemmParams p = base_params(g);
   const uint64_t P = (uint64_t)g.nblk_cap * BM;
   const bool short_k = g.f / BK <= 4;  // ffn <= 256: the epilogue bounds a tile (8 warps)
@@ -1128,8 +1100,9 @@ cudaError_t launch_down_gemm(const GemmProblem &g, const void *h_in, const void 
                              make_tmap(&p.tm[1], w2, (uint64_t)g.E * g.h, g.f, BN / 2))
                           : (make_tmap_chunked(&p.tm[0], h_in, P, g.f, BM) &&
                              make_tmap_chunked(&p.tm[1], w2, (uint64_t)g.E * g.h, g.f, BN / 2));
-  if (!ok || !make_tmap(&p.tmo[0], y_pad, P, g.h, 32)) return cudaErrorInvalidValue;
+  if (!ok || !make_tmap(&p.tmo[0], y_pad, P, g.h, 32)) return cudaErrorInvalidValue;  // fp16
   p.tm[2] = p.tm[3] = p.tm[4] = p.tm[0];
+  p.part = y_scale;
   p.n_tiles = (g.h + BN - 1) / BN;
   p.group = raster_units(g.f);
   if (short_k) {

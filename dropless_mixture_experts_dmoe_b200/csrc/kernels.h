@@ -32,13 +32,16 @@ inline int32_t *map_segs(int32_t *tile_hist, int T, int E) {
   return tile_hist + (size_t)map_tiles(T) * E + 1 + (size_t)map_tiles(T);
 }
 
-// Map: routing + per-tile histogram (logits given) or histogram of given top_experts.
+// Map: routing + per-tile histogram (logits given) or histogram of given top_experts
+// (absent_ok: an expert id of -1 marks an absent entry, left out without a status bit).
 cudaError_t launch_route_hist(const uint16_t *logits, int T, int E, int k, bool renorm, int32_t *top,
-                              float *weights, int32_t *tile_hist, cudaStream_t st);
-// Map: scan over tiles and experts; bins, padded_bins, num_blocks and the status word.
+                              float *weights, int32_t *tile_hist, cudaStream_t st,
+                              bool absent_ok = false);
+// Map: scan over tiles and experts; bins, padded_bins, num_blocks and the status word
+// (overwritten with the call's bits, or OR-ed into with or_status).
 cudaError_t launch_map_scan(int T, int E, int32_t *tile_hist, int32_t *tokens_per_expert,
                             int32_t *bins, int32_t *padded_bins, int32_t *num_blocks,
-                            int32_t *status, cudaStream_t st);
+                            int32_t *status, cudaStream_t st, bool or_status = false);
 // Map: stable scatter of entries to sorted order (indices, bin_ids, dest_row) and the
 // block -> expert table.
 cudaError_t launch_map_scatter(int T, int E, int k, int nblk_cap, const int32_t *top,
@@ -46,13 +49,35 @@ cudaError_t launch_map_scatter(int T, int E, int k, int nblk_cap, const int32_t 
                                const int32_t *padded_bins, int32_t *indices, int32_t *bin_ids,
                                int32_t *dest_row, int32_t *block_expert, cudaStream_t st);
 
+// Tile-aware token rounding (round.cu): scratch of the rounding kernels and the launcher.
+// The routing's top [T,k] / weights [T,k] and the counts of the top-k routing go in; the
+// rounded routing comes out as a token-major entry list: entry_offsets [T+1], experts and
+// weights [cap] (entries past the list's end: expert -1, weight 0).
+constexpr int kRoundMaxT = 1 << 20;  // the selection keeps a bitmap of T bits per CTA
+constexpr size_t kRoundMaxSelectSmem = kRoundMaxT / 8;
+struct RoundScratch {
+  uint16_t *img;       // [E][T] rank images of the logits, one column per expert
+  int32_t *param;      // [3E] per expert: mode, threshold image, threshold token
+  int32_t *tok_count;  // [T]
+  int32_t *tile_sum;   // [map_tiles(T)]
+  int32_t *tile_off;   // [map_tiles(T) + 1]
+};
+cudaError_t launch_round_tokens(const uint16_t *logits, const int32_t *top, const float *weights,
+                                const int32_t *counts, int T, int E, int k, const RoundScratch &s,
+                                int32_t *entry_offsets, int32_t *out_expert, float *out_weight,
+                                long long cap, cudaStream_t st);
+
+// Entries of token t: [t*k, t*k + k), or with a token-major entry list (offsets != NULL, the
+// rounded routing) [offsets[t], offsets[t+1]).
 // Token-major padded gather with zero-filled padding rows.
 cudaError_t launch_gather(int T, int h, int k, int E, const void *x, const int32_t *dest_row,
                           const int32_t *counts, const int32_t *padded_bins, void *x_pad,
-                          cudaStream_t st);
-// Token-major weighted combine (weights may be NULL: w = 1).
-cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const int32_t *dest_row,
-                           const float *weights, void *y, cudaStream_t st);
+                          cudaStream_t st, const int32_t *offsets = nullptr);
+// Token-major weighted combine (weights may be NULL: w = 1) of bf16 rows (y_scale NULL) or of
+// block-floating-point rows (fp16 values, y_scale [P_max, ceil(h/DMOE_SCALE_COLS)]).
+cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const float *y_scale,
+                           const int32_t *dest_row, const float *weights, void *y,
+                           cudaStream_t st, const int32_t *offsets = nullptr);
 
 // Backward scatter: dx_t = bf16(sum_s dX_pad[dest_row[t*k+s]]) over the block-floating-point
 // rows of launch_dx_gemm (value = fp16 * scale, summed in fp32) and, from the DGLU GEMM's
@@ -60,7 +85,7 @@ cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const int32_t
 cudaError_t launch_bwd_scatter(int T, int h, int k, const void *dx_pad, const float *dx_scale,
                                const int32_t *dest_row,
                                const float *part, int nt, void *dx, float *dweights,
-                               cudaStream_t st);
+                               cudaStream_t st, const int32_t *offsets = nullptr);
 
 // Shape and map pointers shared by the grouped GEMM launchers.
 struct GemmProblem {
@@ -82,17 +107,20 @@ cudaError_t launch_glu_gemm(const GemmProblem &g, const void *x_pad, const void 
 cudaError_t launch_glu_gather_gemm(const GemmProblem &g, const void *x, const void *w1,
                                    const void *w3, void *h_out, void *a_out, void *b_out,
                                    cudaStream_t st);
+// Y_pad [P_max,h] in block floating point: fp16 values, y_scale [P_max, ceil(h/128)] fp32 one
+// power-of-two scale per row and DMOE_SCALE_COLS columns (value = fp16 * scale), 11 significant
+// bits per value at bf16's size (the k rows of a token are summed by the combine; a bf16
+// rounding of each would put k roundings into every output element).
 cudaError_t launch_down_gemm(const GemmProblem &g, const void *h_in, const void *w2, void *y_pad,
-                             cudaStream_t st);
+                             float *y_scale, cudaStream_t st);
 // ... and the backward: dH with the fused dGLU epilogue, dX, and the weight gradients.
 // DGLU column tile width (part has ceil(f / kDgluTileCols) columns).
 constexpr int kDgluTileCols = 256;
 cudaError_t launch_dglu_gemm(const GemmProblem &g, const void *dy_pad, const void *w2,
                              const void *a_in, const void *b_in, void *da_out, void *db_out,
                              void *hw_out, float *part, cudaStream_t st);
-// dX_pad [P_max,h] fp16 with dx_scale [P_max, ceil(h/256)] fp32: row r, columns of tile n hold
-// value * 2^-e; dx_scale[r][n] = 2^e (block floating point, 11 significant bits per value).
-constexpr int kDxTileCols = 256;
+// dX_pad [P_max,h] fp16 with dx_scale [P_max, ceil(h/DMOE_SCALE_COLS)] fp32 (block floating
+// point, as Y_pad of the down GEMM).
 cudaError_t launch_dx_gemm(const GemmProblem &g, const void *da, const void *db, const void *w1,
                            const void *w3, void *dx_pad, float *dx_scale, cudaStream_t st);
 cudaError_t launch_wgrad_gemm(const GemmProblem &g, const void *x_pad, const void *h_in,

@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__
 // Histogram of caller-given top_experts; invalid ids are reported (in tile_flags) and left
 // out of the map.
 __global__ void __launch_bounds__(kMapThreads) k_given_hist(const int32_t *__restrict__ top,
-                                                            int T, int E, int k,
+                                                            int T, int E, int k, int absent_ok,
                                                             int32_t *__restrict__ tile_hist,
                                                             int32_t *__restrict__ tile_flags,
                                                             unsigned int *__restrict__ done) {
@@ -307,7 +307,7 @@ __global__ void __launch_bounds__(kMapThreads) k_given_hist(const int32_t *__res
     if (lane < k) {
       e = top[(size_t)t * k + lane];
       if (e < 0 || e >= E) {
-        flags |= DMOE_STATUS_EXPERT_OUT_OF_RANGE;
+        if (!(absent_ok && e == -1)) flags |= DMOE_STATUS_EXPERT_OUT_OF_RANGE;
         e = -1 - lane;
       }
     }
@@ -373,7 +373,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_map_scan(int n_tiles, int E
                                                            int32_t *__restrict__ padded_bins,
                                                            int32_t *__restrict__ num_blocks,
                                                            int32_t *__restrict__ status,
-                                                           unsigned int *__restrict__ done) {
+                                                           unsigned int *__restrict__ done,
+                                                           int or_status) {
   __shared__ int chunk[32][33];
   __shared__ int warp_tot[32];
   __shared__ int s_flags;
@@ -447,8 +448,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_map_scan(int n_tiles, int E
   if (flags && lane == 0) atomicOr(&s_flags, flags);
   __syncthreads();
   if (tid == 0) {
-    *status = s_flags;  // the map call's own bits; later calls OR theirs in
-    *done = 0u;         // ready for the next call
+    // the map call's own bits (later calls OR theirs in); a second map of the same call ORs
+    if (or_status) {
+      if (s_flags) atomicOr(status, s_flags);
+    } else {
+      *status = s_flags;
+    }
+    *done = 0u;  // ready for the next call
   }
 }
 
@@ -580,14 +586,15 @@ __global__ void __launch_bounds__(kMapThreads) k_map_scatter(int T, int E, int k
 // ---- launchers -------------------------------------------------------------------------------
 
 cudaError_t launch_route_hist(const uint16_t *logits, int T, int E, int k, bool renorm, int32_t *top,
-                              float *weights, int32_t *tile_hist, cudaStream_t st) {
+                              float *weights, int32_t *tile_hist, cudaStream_t st,
+                              bool absent_ok) {
   const int tiles = map_tiles(T);
   const size_t smem = sizeof(int) * (size_t)E;
   unsigned int *done = map_ticket(tile_hist, T, E);
   int32_t *flags = map_flags(tile_hist, T, E);
   if (!logits)
-    return launch_pdl(k_given_hist, tiles, kMapThreads, smem, st, top, T, E, k, tile_hist, flags,
-                      done);
+    return launch_pdl(k_given_hist, tiles, kMapThreads, smem, st, top, T, E, k,
+                      absent_ok ? 1 : 0, tile_hist, flags, done);
   // logits per lane: the smallest power of two with E <= 32 * KPL
   using Kernel = void (*)(const uint16_t *, int, int, int, int, int32_t *, float *, int32_t *,
                           int32_t *, unsigned int *);
@@ -612,11 +619,11 @@ cudaError_t launch_route_hist(const uint16_t *logits, int T, int E, int k, bool 
 
 cudaError_t launch_map_scan(int T, int E, int32_t *tile_hist, int32_t *tokens_per_expert,
                             int32_t *bins, int32_t *padded_bins, int32_t *num_blocks,
-                            int32_t *status, cudaStream_t st) {
+                            int32_t *status, cudaStream_t st, bool or_status) {
   return launch_pdl(k_map_scan, dim3((E + 31) / 32, map_segments(T)), kScanThreads, 0, st,
                     map_tiles(T), E, tile_hist, map_flags(tile_hist, T, E),
                     map_segs(tile_hist, T, E), tokens_per_expert, bins, padded_bins, num_blocks,
-                    status, map_ticket(tile_hist, T, E));
+                    status, map_ticket(tile_hist, T, E), or_status ? 1 : 0);
 }
 
 cudaError_t launch_map_scatter(int T, int E, int k, int nblk_cap, const int32_t *top,

@@ -59,6 +59,7 @@ extern "C" int dmoe_sparse_map_noalloc(const dmoe_dims *dims, const void *logits
     dmoe_map empty = {};
     return dmoe_sparse_map(dims, logits, map ? map : &empty, nullptr, 0, stream);
   }
+  if (dims->flags & DMOE_ROUTE_TOKEN_ROUNDING) return DMOE_ERR_SHAPE;  // needs its own scratch
   if (!map || !map->top_experts || !map->tokens_per_expert || !map->bins || !map->padded_bins ||
       !map->indices || !map->bin_ids || !map->dest_row || !map->block_expert ||
       !map->num_blocks || !map->status || (logits && !map->weights))

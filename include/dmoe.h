@@ -90,8 +90,8 @@ extern "C" {
 /* Problem shape.  T tokens, hidden size h, ffn size f (per expert), E experts, top_k, and
  * the variant flags: 0 (the default: weights are the softmax over all E logits at the chosen
  * experts, and the forward saves X_pad, A and Bm for the backward) or an OR of
- * DMOE_ROUTE_RENORMALIZE and DMOE_SAVE_X_ONLY.  Other bits are rejected.  Every call of one
- * layer instance must see the same flags. */
+ * DMOE_ROUTE_RENORMALIZE or DMOE_ROUTE_TOKEN_ROUNDING (not both) and DMOE_SAVE_X_ONLY.  Other
+ * bits are rejected.  Every call of one layer instance must see the same flags. */
 typedef struct {
   int32_t T, hidden, ffn, num_experts, top_k;
   int32_t flags;
@@ -102,6 +102,35 @@ typedef struct {
  * not renormalise).  Read by dmoe_sparse_map (weights) and the router backward (dlogits). */
 #define DMOE_ROUTE_RENORMALIZE 0x1
 
+/* Block floating point of the padded expert outputs (Y_pad of dmoe_expert_down, dX_pad of
+ * dmoe_bwd_dx): fp16 values [P_max, h] and fp32 scales [P_max, ceil(h / DMOE_SCALE_COLS)]; the
+ * value of row r, column c is fp16[r][c] * scale[r][c / DMOE_SCALE_COLS].  Each scale is a
+ * power of two that puts the largest magnitude of its 128 columns into [2^13, 2^14] (1 for an
+ * all-zero or non-finite group), so every value keeps fp16's 11 significant bits at bf16's
+ * size.  The k rows of a token are summed afterwards in fp32; rounding each to bf16 first (8
+ * bits) would put k roundings into every output element (measured at full size: 5.2-5.4 % of
+ * the output's RMS at the largest element, against 3.1-3.3 % this way). */
+#define DMOE_SCALE_COLS 128
+
+/* Routing variant: tile-aware token rounding (SonicMoE abstract: the routing is rounded so that
+ * every expert's token count is a multiple of the GEMM tile, and the grouped GEMMs compute no
+ * padding rows).  The abstract gives the method in one sentence; this library's reading: for
+ * every expert e whose top-k count c_e has r = c_e mod 128 != 0, when r >= 64 and at least
+ * 128 - r tokens are not routed to e, the 128 - r best-ranked such tokens are added to e
+ * (round up); otherwise e's r worst-ranked entries are dropped (round down).  A token ranks
+ * for expert e by its logit l[t][e], larger first, equal logits by the lower token index.  A
+ * token keeps its surviving slots in slot order, then its added experts in increasing expert
+ * order; every entry's weight is the softmax over all E logits at its expert.
+ *   The map then holds a token-major entry list of N' <= dmoe_entries_max(dims) = T*k + 64*E
+ *   entries: map->entry_offsets [T+1] (token t owns entries [offsets[t], offsets[t+1])),
+ *   top_experts / weights [entries_max] (expert and weight of each entry; past N': -1 and 0),
+ *   indices / bin_ids / dest_row [entries_max] over those entries (dest_row -1 past N'), and
+ *   tokens_per_expert / bins / padded_bins of the rounded counts (padded_bins == bins).
+ *   Forward, backward and the step calls follow the list (dweights per entry).  The router
+ *   calls, dmoe_expert_glu_gather and dmoe_sparse_map_noalloc reject the flag
+ *   (DMOE_ERR_SHAPE), as does T > 2^20; dmoe_sparse_map needs the logits. */
+#define DMOE_ROUTE_TOKEN_ROUNDING 0x2
+
 /* Memory variant (walkthrough section 4.4's MemoryOptimizedMLP; the SonicMoE abstract's
  * activation-memory saving): the training forward saves only X_pad (dmoe_saved_bytes shrinks
  * from (2h + 4f) to 2h bytes per padded row) and dmoe_backward recomputes A and Bm with one
@@ -109,8 +138,9 @@ typedef struct {
  * padded row).  Every result is bit-identical to the default variant's. */
 #define DMOE_SAVE_X_ONLY 0x4
 
-/* The sparse map.  All device pointers, caller-owned; N = T*top_k entries,
- * P_max = dmoe_padded_rows_max(dims).  Meaning (walkthrough sections 4.1-4.3):
+/* The sparse map.  All device pointers, caller-owned; N = T*top_k entries (with
+ * DMOE_ROUTE_TOKEN_ROUNDING: dmoe_entries_max(dims) and the token-major layout described
+ * there), P_max = dmoe_padded_rows_max(dims).  Meaning (walkthrough sections 4.1-4.3):
  *   top_experts [T, k] int32   expert of entry t*k+s, slot s = s-th pick in descending
  *                              logit order, ties to the lower expert index.  Output of
  *                              dmoe_sparse_map when logits are given, else its INPUT.
@@ -140,6 +170,7 @@ typedef struct {
   int32_t *block_expert;
   int32_t *num_blocks;
   int32_t *status;
+  int32_t *entry_offsets; /* [T+1], DMOE_ROUTE_TOKEN_ROUNDING only (may be NULL otherwise) */
 } dmoe_map;
 
 /* Workspace kinds for dmoe_workspace_bytes. */
@@ -158,6 +189,10 @@ typedef struct {
  * walkthrough's padded_gather reads padded_bins[-1] on the host, section 4.2; this library
  * does not). Returns 0 for invalid dims. */
 DMOE_API size_t dmoe_padded_rows_max(const dmoe_dims *dims);
+
+/* Entries of the map: T*top_k, or with DMOE_ROUTE_TOKEN_ROUNDING the bound T*top_k + 64*E on
+ * the rounded entry list (0 for invalid dims).  P_max is computed from it. */
+DMOE_API size_t dmoe_entries_max(const dmoe_dims *dims);
 
 /* Bytes of workspace the call `kind` needs (0 for invalid dims). */
 DMOE_API size_t dmoe_workspace_bytes(const dmoe_dims *dims, int kind);
@@ -266,17 +301,21 @@ DMOE_API int dmoe_expert_glu_gather(const dmoe_dims *dims, const void *x, const 
                                     const void *w3, const dmoe_map *map, void *h_out, void *a_out,
                                     void *b_out, void *stream);
 
-/* Down GEMM: Y_pad[b] = bf16(H[b] W2_e^T) for every block b < num_blocks.
- * h_in [P_max,f] -> y_pad [P_max,h], bf16. */
+/* Down GEMM: Y_pad[b] = H[b] W2_e^T for every block b < num_blocks, fp32 accumulation,
+ * stored in block floating point (see DMOE_SCALE_COLS).
+ * h_in [P_max,f] bf16 -> y_pad [P_max,h] fp16, y_scale [P_max, ceil(h/128)] fp32. */
 DMOE_API int dmoe_expert_down(const dmoe_dims *dims, const void *h_in, const void *w2,
-                     const dmoe_map *map, void *y_pad, void *stream);
+                              const dmoe_map *map, void *y_pad, float *y_scale, void *stream);
 
 /* Weighted padded_scatter (walkthrough section 4.2, B_TO_A direction, times the routing
  * weight): y_t = bf16(sum_{s=0..k-1} w_ts * Y_pad[dest_row[t*k+s]]), summed in fp32 in
- * slot order, no atomics.  weights == NULL means w = 1 (the backward's gather gradient,
- * dx_t = sum_s dX_pad[dest_row[t*k+s]]).  y_pad [P_max,h] -> y [T,h], bf16. */
-DMOE_API int dmoe_padded_scatter(const dmoe_dims *dims, const void *y_pad, const dmoe_map *map,
-                        const float *weights, void *y, void *stream);
+ * slot order (each entry one fused multiply-add), no atomics.  weights == NULL means w = 1
+ * (the backward's gather gradient, dx_t = sum_s dX_pad[dest_row[t*k+s]]).  Row format:
+ * y_scale == NULL: y_pad [P_max,h] bf16; otherwise block floating point as written by
+ * dmoe_expert_down (y_pad fp16, y_scale [P_max, ceil(h/128)]).  -> y [T,h] bf16. */
+DMOE_API int dmoe_padded_scatter(const dmoe_dims *dims, const void *y_pad, const float *y_scale,
+                                 const dmoe_map *map, const float *weights, void *y,
+                                 void *stream);
 
 /* ---- Backward step entry points (each one kernel).  dmoe_backward is: dy_pad =
  * dmoe_padded_gather(dy) (the gradient of the weighted scatter is a gather, walkthrough
@@ -298,14 +337,10 @@ DMOE_API int dmoe_bwd_dglu(const dmoe_dims *dims, const void *dy_pad, const void
                            void *da, void *dbm, void *hw, float *dw_part, void *stream);
 
 /* dX GEMM: dX_pad[b] = dA[b] W1_e + dBm[b] W3_e, one fp32 accumulator over both K passes,
- * stored in block floating point: dx_pad [P_max,h] holds fp16 values and dx_scale
- * [P_max, ceil(h / DMOE_DX_TILE_COLS)] fp32 one power-of-two scale per row and 256-column
- * tile (value = fp16 * scale; the scale puts the row's largest magnitude in the tile into
- * [2^13, 2^14)).  That keeps 11 significant bits per value at bf16's size: the k rows of a
- * token are summed by dmoe_bwd_scatter, and rounding each of them to bf16 first would put k
- * bf16 roundings into every element of dx.
- * da, dbm [P_max,f] bf16 -> dx_pad [P_max,h] fp16, dx_scale fp32. */
-#define DMOE_DX_TILE_COLS 256
+ * stored in block floating point (see DMOE_SCALE_COLS): the k rows of a token are summed by
+ * dmoe_bwd_scatter, and rounding each of them to bf16 first would put k bf16 roundings into
+ * every element of dx.
+ * da, dbm [P_max,f] bf16 -> dx_pad [P_max,h] fp16, dx_scale [P_max, ceil(h/128)] fp32. */
 DMOE_API int dmoe_bwd_dx(const dmoe_dims *dims, const void *da, const void *dbm, const void *w1,
                          const void *w3, const dmoe_map *map, void *dx_pad, float *dx_scale,
                          void *stream);

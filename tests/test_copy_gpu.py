@@ -54,7 +54,7 @@ def test_scatter_of_gather_is_k_times_x(w):
     xp = bufs.view("x_pad")
     B.dmoe_padded_gather(dims, x, bufs.map, xp)
     y = torch.empty_like(x)
-    B.dmoe_padded_scatter(dims, xp, bufs.map, None, y)  # w = 1: the gather's gradient
+    B.dmoe_padded_scatter(dims, xp, None, bufs.map, None, y)  # w = 1, bf16 rows
     torch.cuda.synchronize()
     ref = (x.float() * w.top_k).to(torch.bfloat16)  # k*x is exact in fp32
     assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
@@ -63,10 +63,9 @@ def test_scatter_of_gather_is_k_times_x(w):
 @pytest.mark.parametrize("w", SHAPES[:3], ids=lambda w: w.describe())
 def test_weighted_scatter(w):
     dims, bufs, g, x = _setup(w)
-    yp = bufs.view("y_pad")
-    yp.copy_(torch.randn(yp.shape, device="cuda").to(torch.bfloat16))
+    yp = torch.randn((bufs.P, w.hidden), device="cuda").to(torch.bfloat16)
     y = torch.empty_like(x)
-    B.dmoe_padded_scatter(dims, yp, bufs.map, bufs.map.weights, y)
+    B.dmoe_padded_scatter(dims, yp, None, bufs.map, bufs.map.weights, y)
     torch.cuda.synchronize()
     ypn = to_np(yp).astype(np.float64)
     wts = g["weights"].astype(np.float64)
@@ -75,3 +74,27 @@ def test_weighted_scatter(w):
     got = to_np(y).astype(np.float64)
     # one bf16 rounding of an fp32 sum: within 2^-8 relative, plus fp32 summation slack
     assert (np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5).all()
+
+
+@pytest.mark.parametrize("w", SHAPES[:3], ids=lambda w: w.describe())
+def test_weighted_scatter_block_floating_point(w):
+    """Rows in block floating point (fp16 values, one power-of-two scale per row and 128
+    columns, the format of the down GEMM's output): y_t = bf16(sum_s fma(w_s * scale, value)),
+    bit for bit against the same fp32 sum in slot order."""
+    dims, bufs, g, x = _setup(w)
+    P, h = bufs.P, w.hidden
+    nsc = (h + 127) // 128
+    gen = torch.Generator(device="cpu").manual_seed(5)
+    vals = (torch.randn((P, h), generator=gen) * 4096).to(torch.float16)
+    expo = torch.randint(-20, 5, (P, nsc), generator=gen).float()
+    scale = torch.pow(2.0, expo)
+    y = torch.empty_like(x)
+    B.dmoe_padded_scatter(dims, vals.cuda(), scale.cuda(), bufs.map, bufs.map.weights, y)
+    torch.cuda.synchronize()
+    full = vals.float() * scale.repeat_interleave(128, dim=1)[:, :h]  # exact in fp32
+    wts = torch.from_numpy(g["weights"]).float()
+    rows = torch.from_numpy(g["dest_row"].reshape(w.T, w.top_k)).long()
+    acc = torch.zeros((w.T, h), dtype=torch.float32)
+    for s in range(w.top_k):  # w * (value * scale) is one rounding, as the kernel's fma
+        acc = (acc.double() + wts[:, s:s + 1].double() * full[rows[:, s]].double()).float()
+    assert torch.equal(y.cpu().view(torch.int16), acc.to(torch.bfloat16).view(torch.int16))

@@ -55,7 +55,9 @@ def test_gemm_intermediates(w):
     A = bufs.view("a")[: nb * 128].double().cpu()
     Bm = bufs.view("bm")[: nb * 128].double().cpu()
     H = bufs.view("h")[: nb * 128].double().cpu()
-    Yp = bufs.view("y_pad")[: nb * 128].double().cpu()
+    # Y_pad is block floating point: fp16 values times one power-of-two scale per 128 columns
+    ys = bufs.view("y_scale")[: nb * 128].double().cpu().repeat_interleave(128, dim=1)
+    Yp = bufs.view("y_pad")[: nb * 128].double().cpu() * ys[:, : w.hidden]
     W1 = inp["w1"].double()
     W3 = inp["w3"].double()
     W2 = inp["w2"].double()
