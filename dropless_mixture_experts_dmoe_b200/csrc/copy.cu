@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(kCopyThreads) k_gather(int T, int h, int k, in
 // which is exact in fp32, so each entry adds c_s * scale * value with one rounding.
 // A lane covers 8 consecutive columns (one 16-byte vector) per entry; VPL vectors per lane
 // and SLOTS entries are loaded before any is consumed.
-template <int VPL, int SLOTS>
+template <int VPL, int SLOTS, bool F16S>
 __global__ void __launch_bounds__(kCopyThreads, 2) k_combine(int T, int h, int k,
                                                           const uint4 *__restrict__ rows,
                                                           const float *__restrict__ scale,
@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(kCopyThreads, 2) k_combine(int T, int h, int k
               const int v = v0 + u * 32 + lane;
               if (v < vpr) {
                 buf[ss][u] = ld_nc_v4(rows + (size_t)r * vpr + v);
-                cf[ss][u] = scale ? ws * __ldg(scale + (size_t)r * nsc + v / kVecPerScale) : ws;
+                cf[ss][u] = F16S ? ws * __ldg(scale + (size_t)r * nsc + v / kVecPerScale) : ws;
               }
             }
           }
@@ -185,8 +185,8 @@ __global__ void __launch_bounds__(kCopyThreads, 2) k_combine(int T, int h, int k
               const float c = cf[ss][u];
 #pragma unroll
               for (int p = 0; p < 4; ++p) {
-                const float lo = scale ? f16_lo(q[p]) : bf16_lo(q[p]);
-                const float hi = scale ? f16_hi(q[p]) : bf16_hi(q[p]);
+                const float lo = F16S ? f16_lo(q[p]) : bf16_lo(q[p]);
+                const float hi = F16S ? f16_hi(q[p]) : bf16_hi(q[p]);
                 acc[u][2 * p] = fmaf(c, lo, acc[u][2 * p]);
                 acc[u][2 * p + 1] = fmaf(c, hi, acc[u][2 * p + 1]);
               }
@@ -236,7 +236,10 @@ static cudaError_t combine(int T, int h, int k, const void *rows, const float *s
                            const float *part, int nt, float *dweights, const int32_t *offsets,
                            cudaStream_t st) {
   const int vpl = (k <= 2) ? 4 : 2;
-  auto kernel = (k <= 2) ? k_combine<4, 2> : (k <= 4) ? k_combine<2, 4> : k_combine<2, 8>;
+  auto kernel = scale ? ((k <= 2) ? k_combine<4, 2, true> : (k <= 4) ? k_combine<2, 4, true>
+                                                                    : k_combine<2, 8, true>)
+                      : ((k <= 2) ? k_combine<4, 2, false> : (k <= 4) ? k_combine<2, 4, false>
+                                                                      : k_combine<2, 8, false>);
   const long long items = (long long)T * (((h >> 3) + 32 * vpl - 1) / (32 * vpl));
   return launch_pdl(kernel, copy_grid(items), kCopyThreads, 0, st, T, h, k,
                     static_cast<const uint4 *>(rows), scale, dest_row, weights,

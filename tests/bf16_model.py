@@ -97,6 +97,13 @@ def expert_wgrad_model(inp: dict, top: np.ndarray, wts: np.ndarray, e: int):
     return ((dA.T @ Xe).numpy(), (dB.T @ Xe).numpy(), (dy[ts].T @ _bf(wr * A * s * Bm)).numpy())
 
 
+def router_wgrad_model(dlogits: np.ndarray, x) -> np.ndarray:
+    """dW_r = dlogits^T x with the logit gradient rounded to bf16 (the router backward's
+    rounding point), float64 otherwise."""
+    dl = _bf(torch.from_numpy(np.asarray(dlogits, np.float64)).float())
+    return (dl.T @ x.double()).numpy()
+
+
 def bounds(model: dict, ref: dict) -> dict:
     """Per-output max-abs / RMS bound from the modelled errors against the oracle."""
     out = {}

@@ -71,16 +71,16 @@ def test_backward_steps_against_float64(w):
     be = bufs.map.block_expert.cpu().numpy()
     D = lambda t: t[:P].double().cpu()
     dy_pad, da, dbm, hw = (D(st[n]) for n in ("dy_pad", "da", "dbm", "hw"))
-    # dX_pad rows are block floating point: fp16 * a power-of-two scale per 256 columns
-    sc32 = st["dx_scale"].cpu().repeat_interleave(256, dim=1)[:, :h]
+    # dX_pad rows are block floating point: fp16 * a power-of-two scale per 128 columns
+    sc32 = st["dx_scale"].cpu().repeat_interleave(B.SCALE_COLS, dim=1)[:, :h]
     dxp32 = st["dx_pad"].float().cpu() * sc32
     dx_pad = dxp32[:P].double()
-    nsc = (h + 255) // 256
+    nsc = (h + B.SCALE_COLS - 1) // B.SCALE_COLS
     scl = st["dx_scale"][:P].cpu()
     assert (scl > 0).all() and (torch.frexp(scl)[0] == 0.5).all()  # powers of two
     f16 = st["dx_pad"][:P].float().cpu().abs()
-    for n in range(nsc):  # each row's largest stored magnitude of a tile is in [2^13, 2^14]
-        mx = f16[:, n * 256:(n + 1) * 256].amax(1)  # (2^14 when fp16 rounding carries up)
+    for n in range(nsc):  # each row's largest stored magnitude of a group is in [2^13, 2^14]
+        mx = f16[:, n * B.SCALE_COLS:(n + 1) * B.SCALE_COLS].amax(1)  # (2^14: rounding carry)
         nz = mx > 0
         assert ((mx[nz] >= 2.0 ** 13) & (mx[nz] <= 2.0 ** 14)).all(), n
         assert (scl[~nz, n] == 1).all(), n  # all-zero rows (padding) are stored unscaled

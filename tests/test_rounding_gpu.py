@@ -10,6 +10,7 @@ import oracle
 from dropless_mixture_experts_dmoe_b200 import binding as B
 from dropless_mixture_experts_dmoe_b200.workloads import WORKLOADS, custom, make_inputs
 
+import bf16_model
 from helpers import MAX_ABS_RMS, WEIGHT_RTOL, assert_close, to_np
 
 pytestmark = pytest.mark.gpu
@@ -118,13 +119,17 @@ def test_rounded_layer_forward_backward(w):
     torch.cuda.synchronize()
     o = {k: v.float().numpy() for k, v in inp.items()}
     tr, wr, offsets = _check_map(bufs, o["logits"], w)
+    # stress shapes (few rows per expert): the bf16 rounding model of the pipeline sizes the
+    # max-abs bound where it exceeds 5e-2 / 1.25 (tests/bf16_model.py)
     yref = oracle.forward(o["x"], o["w1"], o["w3"], o["w2"], tr, wr, threads=8)
-    assert_close(to_np(y), yref, f"y {w.describe()}", max_abs_rms=MAX_ABS_RMS)
+    ytol = bf16_model.bounds({"y": bf16_model.forward_model(inp, tr, wr)}, {"y": yref})["y"]
+    assert_close(to_np(y), yref, f"y {w.describe()}", max_abs_rms=ytol)
     g = oracle.backward(o["x"], o["dy"], o["w1"], o["w3"], o["w2"], tr, wr)
+    tol = bf16_model.bounds(bf16_model.backward_model(inp, tr, wr), g)
     for got, name in ((dx, "dx"), (dw1, "dW1"), (dw3, "dW3"), (dw2, "dW2")):
-        assert_close(to_np(got), g[name], f"{name} {w.describe()}", max_abs_rms=MAX_ABS_RMS)
+        assert_close(to_np(got), g[name], f"{name} {w.describe()}", max_abs_rms=tol[name])
     n = int(offsets[-1])
-    assert_close(to_np(dwt)[:n], g["dw"][tr >= 0], f"dw {w.describe()}")
+    assert_close(to_np(dwt)[:n], g["dw"][tr >= 0], f"dw {w.describe()}", max_abs_rms=tol["dw"])
 
 
 def test_rounded_forward_high_granularity():
