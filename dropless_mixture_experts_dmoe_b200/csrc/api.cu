@@ -282,8 +282,9 @@ int dmoe_sparse_map(const dmoe_dims *dims, const void *logits, const dmoe_map *m
   int32_t *tile_hist = static_cast<int32_t *>(ws);
   const bool renorm = (dims->flags & DMOE_ROUTE_RENORMALIZE) != 0;
   if (rounding(dims)) {
-    // top-k routing and its counts, the rounding into the token-major entry list, then the
-    // map of that list (one entry per "token"; absent entries past its end are left out)
+    // top-k routing and its map (in the map's arrays, rebuilt below), the rounding into the
+    // token-major entry list, then the map of that list (one entry per "token"; absent
+    // entries past its end are left out)
     const MapLayout l = map_layout(dims);
     uint8_t *w = static_cast<uint8_t *>(ws);
     int32_t *top = reinterpret_cast<int32_t *>(w + l.top);
@@ -300,9 +301,13 @@ int dmoe_sparse_map(const dmoe_dims *dims, const void *logits, const dmoe_map *m
     if ((rc = launch_rc(launch_map_scan(T, E, tile_hist, map->tokens_per_expert, map->bins,
                                         map->padded_bins, map->num_blocks, map->status, st))))
       return rc;
-    if ((rc = launch_rc(launch_round_tokens(lg, top, wts, map->tokens_per_expert, T, E, k, s,
-                                            map->entry_offsets, map->top_experts, map->weights,
-                                            N, st))))
+    if ((rc = launch_rc(launch_map_scatter(T, E, k, nblk_cap, top, tile_hist, map->bins,
+                                           map->padded_bins, map->indices, map->bin_ids,
+                                           map->dest_row, map->block_expert, st))))
+      return rc;
+    if ((rc = launch_rc(launch_round_tokens(lg, top, wts, map->tokens_per_expert, map->bins,
+                                            map->indices, T, E, k, s, map->entry_offsets,
+                                            map->top_experts, map->weights, N, st))))
       return rc;
     if ((rc = launch_rc(launch_route_hist(nullptr, N, E, 1, false, map->top_experts, nullptr,
                                           tile_hist, st, /*absent_ok=*/true))))

@@ -129,82 +129,100 @@ __global__ void __launch_bounds__(kCopyThreads, 2) k_combine(int T, int h, int k
   const int vpr = h >> 3;                                      // 16-byte vectors per row
   const int nsc = (h + DMOE_SCALE_COLS - 1) / DMOE_SCALE_COLS;  // scales per row
   constexpr int kVecPerScale = DMOE_SCALE_COLS / 8;
-  constexpr int kSlice = 32 * VPL;
-  const int S = (vpr + kSlice - 1) / kSlice;
+  const int S = (vpr + kSliceVecs - 1) / kSliceVecs;  // 4 KB row slices per token
   const long long items = (long long)T * S;
   const long long nw = (long long)gridDim.x * kCopyWarps;
   for (long long it = (long long)blockIdx.x * kCopyWarps + (threadIdx.x >> 5); it < items;
        it += nw) {
     const int t = (int)(it / S);
-    const int v0 = (int)(it - (long long)t * S) * kSlice;
+    const int vs = (int)(it - (long long)t * S) * kSliceVecs;
+    const int ve = min(vpr, vs + kSliceVecs);
     long long base;
     int cnt;
     token_entries(offsets, t, k, base, cnt);
-    float acc[VPL][8];
-#pragma unroll
-    for (int u = 0; u < VPL; ++u)
-#pragma unroll
-      for (int q = 0; q < 8; ++q) acc[u][q] = 0.0f;
-    for (int c0 = 0; c0 < cnt; c0 += 32) {  // one pass of up to 32 entries (k <= 32)
-      const int kk = min(32, cnt - c0);
+    // the token's entries (up to 32 per pass; more only with the rounded routing), loaded
+    // once per slice and reused by its row pieces
+    for (int c0 = 0; c0 == 0 || c0 < cnt; c0 += 32) {
+      const int kk = max(0, min(32, cnt - c0));
       const int d = (lane < kk) ? dest_row[base + c0 + lane] : -1;
       const float wl = (lane < kk && weights) ? weights[base + c0 + lane] : 1.0f;
-      if (dweights && v0 == 0 && lane < kk) {
+      if (dweights && vs == 0 && lane < kk) {
         float g = 0.0f;
         if (d >= 0)
           for (int n = 0; n < nt; ++n) g += __ldg(part + (size_t)d * nt + n);
         dweights[base + c0 + lane] = g;  // 0 for an entry dropped from the map
       }
-      for (int s0 = 0; s0 < kk; s0 += SLOTS) {
-        uint4 buf[SLOTS][VPL];
-        float cf[SLOTS][VPL];
+      for (int v0 = vs; v0 < ve; v0 += 32 * VPL) {
+        float acc[VPL][8];
+        if (c0 == 0) {
 #pragma unroll
-        for (int ss = 0; ss < SLOTS; ++ss) {
-          const int s = s0 + ss;
-          const int r = __shfl_sync(0xFFFFFFFFu, d, s & 31);
-          const float ws = __shfl_sync(0xFFFFFFFFu, wl, s & 31);
-          if (s < kk && r >= 0) {
+          for (int u = 0; u < VPL; ++u)
 #pragma unroll
-            for (int u = 0; u < VPL; ++u) {
-              const int v = v0 + u * 32 + lane;
-              if (v < vpr) {
-                buf[ss][u] = ld_nc_v4(rows + (size_t)r * vpr + v);
-                cf[ss][u] = F16S ? ws * __ldg(scale + (size_t)r * nsc + v / kVecPerScale) : ws;
+            for (int q = 0; q < 8; ++q) acc[u][q] = 0.0f;
+        } else {  // a later pass of a token with more than 32 entries: continue the sum
+#pragma unroll
+          for (int u = 0; u < VPL; ++u) {
+            const int v = v0 + u * 32 + lane;
+            const uint4 o = (v < ve) ? out[(size_t)t * vpr + v] : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t *q = reinterpret_cast<const uint32_t *>(&o);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              acc[u][2 * p] = bf16_lo(q[p]);
+              acc[u][2 * p + 1] = bf16_hi(q[p]);
+            }
+          }
+        }
+        for (int s0 = 0; s0 < kk; s0 += SLOTS) {
+          uint4 buf[SLOTS][VPL];
+          float cf[SLOTS][VPL];
+#pragma unroll
+          for (int ss = 0; ss < SLOTS; ++ss) {
+            const int s = s0 + ss;
+            const int r = __shfl_sync(0xFFFFFFFFu, d, s & 31);
+            const float ws = __shfl_sync(0xFFFFFFFFu, wl, s & 31);
+            if (s < kk && r >= 0) {
+#pragma unroll
+              for (int u = 0; u < VPL; ++u) {
+                const int v = v0 + u * 32 + lane;
+                if (v < ve) {
+                  buf[ss][u] = ld_nc_v4(rows + (size_t)r * vpr + v);
+                  cf[ss][u] = F16S ? ws * __ldg(scale + (size_t)r * nsc + v / kVecPerScale) : ws;
+                }
+              }
+            }
+          }
+#pragma unroll
+          for (int ss = 0; ss < SLOTS; ++ss) {
+            const int s = s0 + ss;
+            const int r = __shfl_sync(0xFFFFFFFFu, d, s & 31);
+            if (s < kk && r >= 0) {
+#pragma unroll
+              for (int u = 0; u < VPL; ++u) {
+                const uint32_t *q = reinterpret_cast<const uint32_t *>(&buf[ss][u]);
+                const float c = cf[ss][u];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                  const float lo = F16S ? f16_lo(q[p]) : bf16_lo(q[p]);
+                  const float hi = F16S ? f16_hi(q[p]) : bf16_hi(q[p]);
+                  acc[u][2 * p] = fmaf(c, lo, acc[u][2 * p]);
+                  acc[u][2 * p + 1] = fmaf(c, hi, acc[u][2 * p + 1]);
+                }
               }
             }
           }
         }
 #pragma unroll
-        for (int ss = 0; ss < SLOTS; ++ss) {
-          const int s = s0 + ss;
-          const int r = __shfl_sync(0xFFFFFFFFu, d, s & 31);
-          if (s < kk && r >= 0) {
-#pragma unroll
-            for (int u = 0; u < VPL; ++u) {
-              const uint32_t *q = reinterpret_cast<const uint32_t *>(&buf[ss][u]);
-              const float c = cf[ss][u];
-#pragma unroll
-              for (int p = 0; p < 4; ++p) {
-                const float lo = F16S ? f16_lo(q[p]) : bf16_lo(q[p]);
-                const float hi = F16S ? f16_hi(q[p]) : bf16_hi(q[p]);
-                acc[u][2 * p] = fmaf(c, lo, acc[u][2 * p]);
-                acc[u][2 * p + 1] = fmaf(c, hi, acc[u][2 * p + 1]);
-              }
-            }
+        for (int u = 0; u < VPL; ++u) {
+          const int v = v0 + u * 32 + lane;
+          if (v < ve) {
+            uint4 o;
+            o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+            o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+            o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+            o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+            out[(size_t)t * vpr + v] = o;
           }
         }
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < VPL; ++u) {
-      const int v = v0 + u * 32 + lane;
-      if (v < vpr) {
-        uint4 o;
-        o.x = pack_bf16x2(acc[u][0], acc[u][1]);
-        o.y = pack_bf16x2(acc[u][2], acc[u][3]);
-        o.z = pack_bf16x2(acc[u][4], acc[u][5]);
-        o.w = pack_bf16x2(acc[u][6], acc[u][7]);
-        out[(size_t)t * vpr + v] = o;
       }
     }
   }
@@ -229,18 +247,15 @@ cudaError_t launch_gather(int T, int h, int k, int E, const void *x, const int32
                     static_cast<uint4 *>(x_pad), offsets);
 }
 
-// Shape of the combine: at most 16 row loads in flight per lane within 128 registers (two
-// CTAs per SM); few entries per token take wide row pieces.
+// Shape of the combine: work items of one token's 4 KB row slice; 8 row loads in flight per
+// lane within 128 registers (two CTAs per SM); few entries take wide row pieces.
 static cudaError_t combine(int T, int h, int k, const void *rows, const float *scale,
                            const int32_t *dest_row, const float *weights, void *out,
                            const float *part, int nt, float *dweights, const int32_t *offsets,
                            cudaStream_t st) {
-  const int vpl = (k <= 2) ? 4 : 2;
-  auto kernel = scale ? ((k <= 2) ? k_combine<4, 2, true> : (k <= 4) ? k_combine<2, 4, true>
-                                                                    : k_combine<2, 8, true>)
-                      : ((k <= 2) ? k_combine<4, 2, false> : (k <= 4) ? k_combine<2, 4, false>
-                                                                      : k_combine<2, 8, false>);
-  const long long items = (long long)T * (((h >> 3) + 32 * vpl - 1) / (32 * vpl));
+  auto kernel = scale ? ((k <= 2) ? k_combine<4, 2, true> : k_combine<2, 4, true>)
+                      : ((k <= 2) ? k_combine<4, 2, false> : k_combine<2, 4, false>);
+  const long long items = (long long)T * slices(h);
   return launch_pdl(kernel, copy_grid(items), kCopyThreads, 0, st, T, h, k,
                     static_cast<const uint4 *>(rows), scale, dest_row, weights,
                     static_cast<uint4 *>(out), part, nt, dweights, offsets);

@@ -86,7 +86,6 @@ constexpr int A_BYTES = BM * BK * 2;        // 16 KB: this CTA's 128 rows of A
 constexpr int B_BYTES = (BN / 2) * BK * 2;  // 16 KB: this CTA's half of B
 constexpr int CHUNK_BYTES = 64 * BK * 2;    // one 64 x 64 MN-major box: 8 KB
 constexpr int TMEM_COLS = 512;
-constexpr int ACC_COLS = 256;
 constexpr int BOX_BYTES = 32 * 128;  // one result box: 32 rows x 128 B
 
 enum GemmMode {
@@ -149,8 +148,13 @@ struct Cfg {
   static constexpr int kslabs = mode_kslabs(MODE, EPI);
   static constexpr int bk = BK * kslabs;  // K per stage
   static constexpr int a_bytes = A_BYTES * kslabs;
-  static constexpr int stage_bytes = (A_BYTES + B_BYTES) * kslabs;
-  static constexpr int stages = (kslabs == 2) ? 3 : ((EPI == 8) ? 4 : (MODE == MODE_WGRAD ? 6 : 5));
+  // WGRAD stages hold three operand slabs: two products per K step share the third
+  static constexpr int stage_bytes = (MODE == MODE_WGRAD) ? 3 * A_BYTES : (A_BYTES + B_BYTES) * kslabs;
+  static constexpr int stages = (kslabs == 2) ? 3 : ((EPI == 8) ? 4 : (MODE == MODE_WGRAD ? 4 : 5));
+  // accumulator buffers in tensor memory: two of 256 columns (tile i's epilogue overlaps tile
+  // i+1's MMAs), or for WGRAD one of 512 columns holding its two products
+  static constexpr int nacc = (MODE == MODE_WGRAD) ? 1 : 2;
+  static constexpr int acc_stride = TMEM_COLS / nacc;
   static constexpr int out_bufs = (kslabs == 2 || MODE == MODE_WGRAD) ? 1 : 2;
   static constexpr int out_bytes = epi_warps * out_bufs * BOX_BYTES;
   // WGRAD: one zeroed result box, the source of the zero tiles' stores
@@ -221,21 +225,22 @@ __device__ __forceinline__ Tile decode(const GemmParams &p, int t, const int *us
     return tl;
   }
   if (MODE == MODE_WGRAD) {
+    // which 0: the (dW1, dW3) blocks of one (m, n) tile, sharing the X_pad operand;
+    // which 2: two 256-column halves of one dW2 row-tile pair, sharing the dY_pad operand
     const int mt13 = p.f / BM, mt2 = p.h / BM;
     const int mp13 = (mt13 + 1) / 2, mp2 = (mt2 + 1) / 2;
-    const int nt13 = (p.h + BN - 1) / BN, nt2 = (p.f + BN - 1) / BN;
-    const int tpe = 2 * mp13 * nt13 + mp2 * nt2;
+    const int nt13 = (p.h + BN - 1) / BN, nt2 = (p.f + 2 * BN - 1) / (2 * BN);
+    const int tpe = mp13 * nt13 + mp2 * nt2;
     tl.e = t / tpe;
     int r = t - tl.e * tpe;
     int ncols, mtiles;
-    if (r < 2 * mp13 * nt13) {
-      tl.which = r / (mp13 * nt13);
-      r -= tl.which * mp13 * nt13;
+    if (r < mp13 * nt13) {
+      tl.which = 0;
       ncols = nt13;
       mtiles = mt13;
     } else {
       tl.which = 2;
-      r -= 2 * mp13 * nt13;
+      r -= mp13 * nt13;
       ncols = nt2;
       mtiles = mt2;
     }
@@ -340,12 +345,18 @@ __device__ __forceinline__ void load_stage(const GemmParams &p, const Tile &tl, 
 #pragma unroll
     for (int c = 0; c < 2; ++c)
       tma_load_2d_pair(sb + c * CHUNK_BYTES, &p.tm[1], bar, tl.n * BN + (2 * (int)rank + c) * 64, y);
-  } else {  // MODE_WGRAD: both operands MN-major, each one box of two 64-column chunks
+  } else {  // MODE_WGRAD: three MN-major slabs, each one box of two 64-column chunks
     const int y = tl.row0 + kb * BK;
-    const CUtensorMap *ta = &p.tm[tl.which];               // dA, dBm, dY_pad
-    const CUtensorMap *tb = &p.tm[tl.which == 2 ? 4 : 3];  // X_pad, X_pad, Hw
-    tma_load_3d_pair(sa, ta, bar, 0, y, (tl.m * BM) / 64);
-    tma_load_3d_pair(sb, tb, bar, 0, y, (tl.n * BN) / 64 + 2 * (int)rank);
+    if (tl.which == 0) {  // dA, dBm (128 f-rows each), X_pad (this CTA's 128 h-columns)
+      tma_load_3d_pair(sa, &p.tm[0], bar, 0, y, (tl.m * BM) / 64);
+      tma_load_3d_pair(sa + A_BYTES, &p.tm[1], bar, 0, y, (tl.m * BM) / 64);
+      tma_load_3d_pair(sa + 2 * A_BYTES, &p.tm[3], bar, 0, y, (tl.n * BN) / 64 + 2 * (int)rank);
+    } else {  // dY_pad (128 h-rows), Hw of the two 256-column halves (this CTA's 128 of each)
+      const int c0 = (tl.n * 2 * BN) / 64 + 2 * (int)rank;
+      tma_load_3d_pair(sa, &p.tm[2], bar, 0, y, (tl.m * BM) / 64);
+      tma_load_3d_pair(sa + A_BYTES, &p.tm[4], bar, 0, y, c0);
+      tma_load_3d_pair(sa + 2 * A_BYTES, &p.tm[4], bar, 0, y, c0 + BN / 64);
+    }
   }
 }
 
@@ -615,24 +626,28 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
       st.emit(&p.tmo[0], w, n0 + c, yw);
       tmem_ld_wait();
     }
-  } else {  // MODE_WGRAD: fp32 results, boxes of 32 columns
+  } else {  // MODE_WGRAD: two products, fp32 results, boxes of 32 columns
     const int rows = (tl.which == 2) ? p.h : p.f;
     const int cols = (tl.which == 2) ? p.f : p.h;
     const int yw = tl.e * rows + tl.m * BM + sub * 32;
-    const int n0 = tl.n * BN + half * kw;
-    const int ncols = min(kw, cols - n0);  // multiple of 32 (may be <= 0)
-    if (ncols <= 0) return;
-    tb += (uint32_t)(half * kw);
-    uint32_t v[32], w[32];
-    tmem_ld32(tb, v);
-    tmem_ld_wait();
 #pragma unroll 1
-    for (int c = 0; c < ncols; c += 32) {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) w[i] = v[i];
-      if (c + 32 < ncols) tmem_ld32(tb + c + 32, v);  // overlaps the store
-      st.emit(&p.tmo[tl.which], w, n0 + c, yw);
+    for (int q = 0; q < 2; ++q) {  // product q: dW1 / dW3 (which 0), or dW2's half q
+      const CUtensorMap *map = &p.tmo[tl.which == 0 ? q : 2];
+      const int n0 = (tl.which == 0 ? tl.n * BN : tl.n * 2 * BN + q * BN) + half * kw;
+      const int ncols = min(kw, cols - n0);  // multiple of 32 (may be <= 0)
+      if (ncols <= 0) continue;
+      const uint32_t tq = tb + (uint32_t)(q * BN + half * kw);
+      uint32_t v[32], w[32];
+      tmem_ld32(tq, v);
       tmem_ld_wait();
+#pragma unroll 1
+      for (int c = 0; c < ncols; c += 32) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) w[i] = v[i];
+        if (c + 32 < ncols) tmem_ld32(tq + c + 32, v);  // overlaps the store
+        st.emit(map, w, n0 + c, yw);
+        tmem_ld_wait();
+      }
     }
   }
 }
@@ -735,7 +750,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
     total = p.total;
   } else if (MODE == MODE_WGRAD) {
     const int mp13 = (p.f / BM + 1) / 2, mp2 = (p.h / BM + 1) / 2;
-    total = p.E * (2 * mp13 * ((p.h + BN - 1) / BN) + mp2 * ((p.f + BN - 1) / BN));
+    total = p.E * (mp13 * ((p.h + BN - 1) / BN) + mp2 * ((p.f + 2 * BN - 1) / (2 * BN)));
   } else {
     total = ustart[p.E] * p.n_tiles;
   }
@@ -810,7 +825,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
       if (tl.kit == 0) continue;  // weight gradient of an expert without rows: no MMA
       if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.status, abort_flag, p.wait_cycles)) break;
       tc_fence_after();
-      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
+      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * C::acc_stride);
       bool ok = true;
       for (int kb = 0; kb < tl.kit; ++kb) {
         if (!mbar_wait(&full[stage], phase, p.status, abort_flag, p.wait_cycles)) {
@@ -820,6 +835,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
         tc_fence_after();
         const uint32_t a_addr = smem_u32(tiles + stage * C::stage_bytes);
         const uint32_t b_addr = a_addr + C::a_bytes;
+        if (MODE == MODE_WGRAD) {  // two products per K step; slabs s0, s1, s2 of the stage
+          const bool shared_b = tl.which == 0;  // (dA, dBm) x X_pad, else dY_pad x (Hw, Hw')
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t s0 = sdesc_mnmajor_sw128(a_addr + kk * 2048, CHUNK_BYTES);
+            const uint64_t s1 = sdesc_mnmajor_sw128(a_addr + A_BYTES + kk * 2048, CHUNK_BYTES);
+            const uint64_t s2 = sdesc_mnmajor_sw128(a_addr + 2 * A_BYTES + kk * 2048, CHUNK_BYTES);
+            const uint32_t acc_flag = (kb | kk) != 0 ? 1u : 0u;
+            tc_mma_pair(d_tmem, s0, shared_b ? s2 : s1, idesc, acc_flag);
+            tc_mma_pair(d_tmem + BN, shared_b ? s1 : s0, s2, idesc, acc_flag);
+          }
+        } else {
 #pragma unroll
         for (int kk = 0; kk < C::bk / 16; ++kk) {
           // K-major: slab kk / 4 (one 128 B swizzle row of 64 K per slab), 32 B per 16 K inside
@@ -831,6 +858,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
                                   : sdesc_kmajor_sw128(b_addr + (kk >> 2) * B_BYTES + (kk & 3) * 32);
           tc_mma_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
         }
+        }
         tc_commit_pair_mc(&empty[stage]);
         if (++stage == STAGES) {
           stage = 0;
@@ -839,8 +867,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
       }
       if (!ok) break;
       tc_commit_pair_mc(&tfull[acc]);
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (++acc == C::nacc) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
     tc_commit_pair(drain);
     mbar_wait_plain(drain, 0, p.wait_cycles);
@@ -858,13 +888,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
         const int rows_ = (tl.which == 2) ? p.h : p.f;
         const int cols = (tl.which == 2) ? p.f : p.h;
         const int y = tl.e * rows_ + tl.m * BM;
-        const int n0 = tl.n * BN;
-        const int ncols = min(BN, cols - n0);
-        for (int r = 0; r < BM; r += 32)
-          for (int c = 0; c < ncols; c += 32)
-            tma_store_2d_u32(&p.tmo[tl.which], smem_u32(zbuf), n0 + c, y + r);
-        bulk_commit();
-        bulk_wait_read<8>();  // bounded number of groups in flight
+        for (int q = 0; q < 2; ++q) {  // both products of the tile
+          const CUtensorMap *map = &p.tmo[tl.which == 0 ? q : 2];
+          const int n0 = (tl.which == 0) ? tl.n * BN : tl.n * 2 * BN + q * BN;
+          const int ncols = min(BN, cols - n0);
+          for (int r = 0; r < BM; r += 32)
+            for (int c = 0; c < ncols; c += 32) tma_store_2d_u32(map, smem_u32(zbuf), n0 + c, y + r);
+          bulk_commit();
+          bulk_wait_read<8>();  // bounded number of groups in flight
+        }
       }
     }
     bulk_wait_all();  // every zero store has completed before the CTA exits
@@ -887,15 +919,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
       if (lane == 0) good = mbar_wait(&tfull[acc], acc_phase, p.status, abort_flag, p.wait_cycles) ? 1 : 0;
       if (!__shfl_sync(0xFFFFFFFFu, good, 0)) break;
       tc_fence_after();
-      const uint32_t tb = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+      const uint32_t tb = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * C::acc_stride);
       if (!tl.dummy) epilogue_tile<MODE, EPI>(p, tl, tb, sub, half, lane, wr, st);
       // every lane's accumulator reads are complete (tcgen05.wait::ld inside the tile), ordered
       // before the warp barrier by the fence; one arrival per warp releases the accumulator
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_tempty0 + (uint32_t)(acc * sizeof(uint64_t)));
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (++acc == C::nacc) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
     if (lane == 0) bulk_wait_all();  // results written before the CTA exits
     __syncwarp();
@@ -1167,8 +1201,8 @@ cudaError_t launch_wgrad_gemm(const GemmProblem &g, const void *x_pad, const voi
       !make_tmap(&p.tmo[1], dw3, EF, g.h, 32, 4) || !make_tmap(&p.tmo[2], dw2, EH, g.f, 32, 4))
     return cudaErrorInvalidValue;
   const long long t13 = (long long)((g.f / BM + 1) / 2) * ((g.h + BN - 1) / BN);
-  const long long t2 = (long long)((g.h / BM + 1) / 2) * ((g.f + BN - 1) / BN);
-  return launch_gemm<MODE_WGRAD, 4>(p, (long long)g.E * (2 * t13 + t2), st);
+  const long long t2 = (long long)((g.h / BM + 1) / 2) * ((g.f + 2 * BN - 1) / (2 * BN));
+  return launch_gemm<MODE_WGRAD, 4>(p, (long long)g.E * (t13 + t2), st);
 }
 
 // ---- the linear router's GEMMs (dense token rows) ----------------------------------------------

@@ -62,8 +62,10 @@ struct RoundScratch {
   int32_t *tile_sum;   // [map_tiles(T)]
   int32_t *tile_off;   // [map_tiles(T) + 1]
 };
+// counts, bins, indices: the top-k routing's map (its sorted entries find each expert's tokens).
 cudaError_t launch_round_tokens(const uint16_t *logits, const int32_t *top, const float *weights,
-                                const int32_t *counts, int T, int E, int k, const RoundScratch &s,
+                                const int32_t *counts, const int32_t *bins,
+                                const int32_t *indices, int T, int E, int k, const RoundScratch &s,
                                 int32_t *entry_offsets, int32_t *out_expert, float *out_weight,
                                 long long cap, cudaStream_t st);
 

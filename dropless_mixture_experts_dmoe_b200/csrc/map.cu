@@ -182,6 +182,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__
   const int t0 = blockIdx.x * kMapTokTile + warp;
   // expert KPL*lane + i of the vector layout exists iff the lane's first one does (E % KPL == 0)
   const bool lane_ok = KPL * lane < E;
+  const bool full_rows = (E == 32 * KPL);  // every slot of every lane holds an expert
   uint32_t low[KPL];  // low halves of this lane's keys; 0 marks a slot past the last expert
 #pragma unroll
   for (int i = 0; i < KPL; ++i) {
@@ -222,8 +223,10 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__
         key[i] = __byte_perm(o, low[i], 0x1054);
       }
     }
+    if (!full_rows) {  // warp-uniform: slots past the last expert hold no candidate
 #pragma unroll
-    for (int i = 0; i < KPL; ++i) key[i] = low[i] ? key[i] : 0u;
+      for (int i = 0; i < KPL; ++i) key[i] = low[i] ? key[i] : 0u;
+    }
     if (__any_sync(0xFFFFFFFFu, (nf & 0x80008000u) != 0u)) {  // rare: NaN ranked lowest
       bad = true;
 #pragma unroll
@@ -239,12 +242,20 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__
     for (int s = 0; s < k; ++s) {
       const uint32_t wb = __reduce_max_sync(0xFFFFFFFFu, cand.c[0]);
       my_key = (lane == s) ? wb : my_key;
-      if (cand.c[0] == wb) {
-        cand.pop();
-        if (KPL > C && cand.c[0] == 0u && s + 1 < k) {
+      const bool win = cand.c[0] == wb;
 #pragma unroll
-          for (int i = 0; i < KPL; ++i)
-            if (key[i] < wb) cand.insert(key[i]);
+      for (int i = 0; i + 1 < C; ++i) cand.c[i] = win ? cand.c[i + 1] : cand.c[i];
+      cand.c[C - 1] = win ? 0u : cand.c[C - 1];
+      if constexpr (KPL > C) {
+        // a lane that has given up all its candidates refills them from its keys below the
+        // last pick (it holds more than C of the top-k); warp-uniform test, rarely true
+        const bool dry = win && cand.c[0] == 0u && s + 1 < k;
+        if (__any_sync(0xFFFFFFFFu, dry)) {
+          if (dry) {
+#pragma unroll
+            for (int i = 0; i < KPL; ++i)
+              if (key[i] < wb) cand.insert(key[i]);
+          }
         }
       }
     }
@@ -262,6 +273,10 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__
     float sum = 0.0f;
     if (renorm) {
       if (lane < k) sum = ev;
+    } else if (full_rows) {
+#pragma unroll
+      for (int i = 0; i < KPL; ++i)
+        sum += ex2_approx(fmaf(__uint_as_float(cur.image(i)), kLog2e, -ml));
     } else {
 #pragma unroll
       for (int i = 0; i < KPL; ++i)

@@ -15,6 +15,8 @@
 // no padding rows.
 //
 // Kernels, all without inter-CTA waiting:
+//   k_round_images   the logits' rank images transposed to one contiguous column per expert
+//                    (64 x 64 tiles through shared memory, coalesced on both sides).
 //   k_round_select   one CTA per expert: decides round up / down and finds the rank threshold
 //                    (logit image v*, token t*) with two 8-bit histogram passes over the
 //                    candidates' logit images and one ordered pass over the tied tokens.
@@ -40,12 +42,6 @@ __device__ __forceinline__ uint32_t rank_image(uint16_t b) {
   return (b & 0x8000u) ? (uint32_t)(~b & 0xFFFFu) : (uint32_t)(b | 0x8000u);
 }
 
-// Whether token t is routed to expert e by the top-k routing (its row of top holds e).
-__device__ __forceinline__ bool is_routed(const int32_t *__restrict__ top, int k, int t, int e) {
-  bool r = false;
-  for (int s = 0; s < k; ++s) r |= (__ldg(top + (size_t)t * k + s) == e);
-  return r;
-}
 
 // Block-wide sum of one int per thread (kSelThreads threads).
 __device__ __forceinline__ int block_sum(int v, int *red) {
@@ -61,19 +57,40 @@ __device__ __forceinline__ int block_sum(int v, int *red) {
 
 }  // namespace
 
+// img[e][t] = rank_image(logits[t][e]): 64 tokens x 64 experts per CTA through shared memory.
+__global__ void __launch_bounds__(256) k_round_images(const uint16_t *__restrict__ logits, int T,
+                                                      int E, uint16_t *__restrict__ img) {
+  __shared__ uint16_t tile[64][66];
+  pdl_wait();
+  pdl_trigger();
+  const int e0 = blockIdx.x * 64, t0 = blockIdx.y * 64;
+  for (int i = threadIdx.x; i < 64 * 64; i += 256) {
+    const int tt = i / 64, ee = i % 64;  // read along a token's row
+    const int t = t0 + tt, e = e0 + ee;
+    tile[tt][ee] = (t < T && e < E) ? (uint16_t)rank_image(logits[(size_t)t * E + e]) : 0;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < 64 * 64; i += 256) {
+    const int ee = i / 64, tt = i % 64;  // write along an expert's column
+    const int t = t0 + tt, e = e0 + ee;
+    if (t < T && e < E) img[(size_t)e * T + t] = tile[tt][ee];
+  }
+}
+
 // One CTA per expert e.  Candidates: for round down, the tokens routed to e (drop the r worst
 // ranked); for round up, the tokens not routed to e (add the 128 - r best ranked).  Finds the
 // rank threshold so that exactly m = r (down) or 128 - r (up) candidates are on the chosen side:
 //   up:    t added   iff image > v*, or image == v* and t <= t*
 //   down:  t dropped iff image < v*, or image == v* and t >= t*
-// param[3e..3e+2] = {mode (0 none, 1 down, 2 up), v*, t*}.  img [E][T] receives the logit
-// images of column e (coalesced reuse by the later passes).  routed_bits: this CTA's bitmap
-// of routed tokens (dynamic shared memory, T bits).
-__global__ void __launch_bounds__(kSelThreads) k_round_select(const uint16_t *__restrict__ logits,
-                                                              const int32_t *__restrict__ top,
+// param[3e..3e+2] = {mode (0 none, 1 down, 2 up), v*, t*}.  img [E][T]: the rank images, one
+// column per expert.  The tokens routed to e are its entries of the top-k routing's sorted
+// order (indices[bins[e-1] .. bins[e]), entry j of token j / k); routed_bits: this CTA's
+// bitmap of them (dynamic shared memory, T bits).
+__global__ void __launch_bounds__(kSelThreads) k_round_select(const int32_t *__restrict__ indices,
+                                                              const int32_t *__restrict__ bins,
                                                               const int32_t *__restrict__ counts,
                                                               int T, int E, int k,
-                                                              uint16_t *__restrict__ img,
+                                                              const uint16_t *__restrict__ img,
                                                               int32_t *__restrict__ param) {
   extern __shared__ uint32_t routed_bits[];  // [ceil(T/32)]
   __shared__ int hist[256];
@@ -94,17 +111,21 @@ __global__ void __launch_bounds__(kSelThreads) k_round_select(const uint16_t *__
     return;
   }
   const int m = up ? kBlock - r : r;  // candidates to take
-  uint16_t *col = img + (size_t)e * T;
+  const uint16_t *col = img + (size_t)e * T;
   const int words = (T + 31) / 32;
   for (int i = threadIdx.x; i < words; i += kSelThreads) routed_bits[i] = 0u;
   for (int i = threadIdx.x; i < 256; i += kSelThreads) hist[i] = 0;
   __syncthreads();
-  // pass A: routed bitmap, logit images, histogram of the candidates' high bytes
+  const int b0 = (e > 0) ? bins[e - 1] : 0;
+  for (int i = b0 + threadIdx.x; i < b0 + c; i += kSelThreads) {
+    const int t = indices[i] / k;
+    atomicOr(&routed_bits[t >> 5], 1u << (t & 31));
+  }
+  __syncthreads();
+  // pass A: histogram of the candidates' high bytes
   for (int t = threadIdx.x; t < T; t += kSelThreads) {
-    const bool rt = is_routed(top, k, t, e);
-    if (rt) atomicOr(&routed_bits[t >> 5], 1u << (t & 31));
-    const uint32_t v = rank_image(__ldg(logits + (size_t)t * E + e));
-    col[t] = (uint16_t)v;
+    const bool rt = (routed_bits[t >> 5] >> (t & 31)) & 1u;
+    const uint32_t v = col[t];
     if (rt != up) atomicAdd(&hist[v >> 8], 1);
   }
   __syncthreads();
@@ -361,7 +382,8 @@ __global__ void __launch_bounds__(1024) k_round_offsets(const int32_t *__restric
 }
 
 cudaError_t launch_round_tokens(const uint16_t *logits, const int32_t *top, const float *weights,
-                                const int32_t *counts, int T, int E, int k, const RoundScratch &s,
+                                const int32_t *counts, const int32_t *bins,
+                                const int32_t *indices, int T, int E, int k, const RoundScratch &s,
                                 int32_t *entry_offsets, int32_t *out_expert, float *out_weight,
                                 long long cap, cudaStream_t st) {
   const size_t sel_smem = sizeof(uint32_t) * (size_t)((T + 31) / 32);
@@ -369,8 +391,11 @@ cudaError_t launch_round_tokens(const uint16_t *logits, const int32_t *top, cons
   static cudaError_t attr = cudaFuncSetAttribute(
       k_round_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRoundMaxSelectSmem);
   if (attr != cudaSuccess) return attr;
-  if ((err = launch_pdl(k_round_select, E, kSelThreads, sel_smem, st, logits, top, counts, T, E, k,
-                        s.img, s.param)) != cudaSuccess)
+  if ((err = launch_pdl(k_round_images, dim3((E + 63) / 64, (T + 63) / 64), 256, 0, st, logits, T,
+                        E, s.img)) != cudaSuccess)
+    return err;
+  if ((err = launch_pdl(k_round_select, E, kSelThreads, sel_smem, st, indices, bins, counts, T, E,
+                        k, (const uint16_t *)s.img, s.param)) != cudaSuccess)
     return err;
   const int tiles = map_tiles(T);
   const size_t ap_smem = sizeof(uint32_t) * (size_t)kApplyWarps * ((E + 31) / 32);
