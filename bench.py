@@ -57,6 +57,9 @@ def parse():
     p.add_argument("--token-rounding", action="store_true",
                    help="the routing variant that rounds every expert's token count to a "
                         "multiple of 128 (no padding rows)")
+    p.add_argument("--fused-combine", action="store_true",
+                   help="the forward variant whose down GEMM adds the weighted rows into an "
+                        "fp32 token accumulator (no Y_pad)")
     p.add_argument("--save-x-only", action="store_true",
                    help="the memory variant: the forward saves X_pad only and the backward "
                         "recomputes A and Bm with one more GLU GEMM")
@@ -243,11 +246,12 @@ def tensor_peak(pk: dict, timed_s: float):
 
 
 def config_of(w, router: bool, world: int, save_x_only: bool = False,
-              token_rounding: bool = False) -> dict:
+              token_rounding: bool = False, fused_combine: bool = False) -> dict:
     """The workload description shared by both arms of the bench."""
     return {"workload": f"{w.name} {w.describe()}" + (" +router" if router else "") +
                         (" save_x_only" if save_x_only and w.backward else "") +
-                        (" token_rounding" if token_rounding else ""),
+                        (" token_rounding" if token_rounding else "") +
+                        (" fused_combine" if fused_combine else ""),
             "T": w.T, "hidden": w.hidden, "ffn": w.ffn, "num_experts": w.E, "top_k": w.top_k,
             "l2": "inputs larger than L2 (expert weights %.2f GB per step)" %
                   (3 * w.E * w.hidden * w.ffn * 2 / 1e9),
@@ -343,7 +347,7 @@ def run_reference(args, w):
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(w, args.router, int(os.environ.get("WORLD_SIZE", "1")),
-                            args.save_x_only, args.token_rounding),
+                            args.save_x_only, args.token_rounding, args.fused_combine),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -380,9 +384,11 @@ def run_ours(args, w):
 
     recompute = bool(args.save_x_only) and w.backward
     rounded = bool(args.token_rounding)
+    fused = bool(args.fused_combine)
     dims = B.make_dims(w.T, w.hidden, w.ffn, w.E, w.top_k,
                        flags=(B.SAVE_X_ONLY if recompute else 0) |
-                       (B.ROUTE_TOKEN_ROUNDING if rounded else 0))
+                       (B.ROUTE_TOKEN_ROUNDING if rounded else 0) |
+                       (B.FUSED_COMBINE if fused else 0))
     train = w.backward
     router = bool(args.router)
     inp = make_inputs(w, with_dy=train, with_router=router)
@@ -393,8 +399,11 @@ def run_ours(args, w):
     y = torch.empty((w.T, w.hidden), dtype=torch.bfloat16, device="cuda")
     st = torch.cuda.current_stream()
     if train:
-        xp, hb, yp = bufs.view("x_pad"), bufs.view("h"), bufs.view("y_pad")
-        ys = bufs.view("y_scale")
+        xp, hb = bufs.view("x_pad"), bufs.view("h")
+        if fused:
+            ya = bufs.view("y_acc")
+        else:
+            yp, ys = bufs.view("y_pad"), bufs.view("y_scale")
         if recompute:  # A and Bm live in backward scratch, recomputed there
             P_ = B.dmoe_padded_rows_max(dims)
             ab_bwd = torch.empty((P_, w.ffn), dtype=torch.bfloat16, device="cuda")
@@ -411,9 +420,9 @@ def run_ours(args, w):
                      dw=torch.empty(B.dmoe_entries_max(dims) if rounded else (w.T, w.top_k), **f32))
     else:
         xp, hb, yp = bufs.step["x_pad"], bufs.step["h"], bufs.step["y_pad"]
-        ys = bufs.step["y_scale"]
+        ys, ya = bufs.step["y_scale"], bufs.step["y_acc"]
         ab = bb = None
-    names = ["map", "gather", "glu_gemm", "down_gemm", "scatter"]
+    names = ["map", "gather", "glu_gemm"] + (["down_combine"] if fused else ["down_gemm", "scatter"])
     if train:
         names += (["glu_recompute"] if recompute else []) + \
             ["dy_gather", "dglu_gemm", "wgrad_gemm", "dx_gemm", "dx_scatter"]
@@ -443,12 +452,17 @@ def run_ours(args, w):
         B.dmoe_expert_glu(dims, xp, dev["w1"], dev["w3"], bufs.map, hb, ab, bb, st)
         i += 1
         mark(i)
-        B.dmoe_expert_down(dims, hb, dev["w2"], bufs.map, yp, ys, st)
-        i += 1
-        mark(i)
-        B.dmoe_padded_scatter(dims, yp, ys, bufs.map, bufs.map.weights, y, st)
-        i += 1
-        mark(i)
+        if fused:  # down GEMM with the weighted combine in its epilogue (3 launches)
+            B.dmoe_expert_down_combine(dims, hb, dev["w2"], bufs.map, y, ya, st)
+            i += 1
+            mark(i)
+        else:
+            B.dmoe_expert_down(dims, hb, dev["w2"], bufs.map, yp, ys, st)
+            i += 1
+            mark(i)
+            B.dmoe_padded_scatter(dims, yp, ys, bufs.map, bufs.map.weights, y, st)
+            i += 1
+            mark(i)
         if train:
             # the sequence of dmoe_backward (which reuses dY_pad's region for dX_pad)
             if recompute:
@@ -620,7 +634,7 @@ def run_ours(args, w):
     useful = w.useful_flops() * N // w.entries
     nhf = N * w.hidden * w.ffn
     flops = dict(glu_gemm=4 * nhf, down_gemm=2 * nhf, dglu_gemm=2 * nhf, dx_gemm=4 * nhf,
-                 wgrad_gemm=6 * nhf, glu_recompute=4 * nhf)
+                 wgrad_gemm=6 * nhf, glu_recompute=4 * nhf, down_combine=2 * nhf)
     the = w.T * w.hidden * w.E
     router_flops = dict(router_gemm=2 * the, router_bwd=4 * the)
     if router:
@@ -663,7 +677,7 @@ def run_ours(args, w):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": config_of(w, router, world, recompute, rounded),
+        "config": config_of(w, router, world, recompute, rounded, fused),
         "useful_tflops": useful / (ms_per_step / 1e3) / 1e12,
         "useful_tflops_frac_bf16": useful / (ms_per_step / 1e3) / 1e12 / pk_t,
         "padded_frac": pad_frac,
@@ -679,7 +693,10 @@ def run_ours(args, w):
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "pipelined": "copies overlap compute (3 streams)",
                 "output_matches_device_run": e2e_matches},
-        "gpu_launches": (len(names) + 2 + (3 if router and train else 0)) * args.steps,
+        # the map is 3 kernels (11 with token rounding), the fused down + combine 3, the
+        # router backward 4; every other name is one kernel
+        "gpu_launches": (len(names) + (10 if rounded else 2) + (2 if fused else 0) +
+                         (3 if router and train else 0)) * args.steps,
         "gpu_launches_note": "kernels of this library in the device-resident timed region",
         "status": status,
     }

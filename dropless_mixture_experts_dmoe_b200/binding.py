@@ -36,7 +36,13 @@ _I = ctypes.c_int
 ROUTE_RENORMALIZE = 0x1
 ROUTE_TOKEN_ROUNDING = 0x2
 SAVE_X_ONLY = 0x4
+FUSED_COMBINE = 0x8
 SCALE_COLS = 128  # block floating point of Y_pad / dX_pad: one scale per row and 128 columns
+
+
+def scale_stride(h: int) -> int:
+    """Row stride of the scale arrays: ceil(h/128) scales padded to a multiple of 4."""
+    return (h + 511) // 512 * 4
 
 
 class dmoe_dims(ctypes.Structure):
@@ -94,6 +100,7 @@ def load():
     lib.dmoe_expert_glu_gather.argtypes = [D, _P, _P, _P, M, _P, _P, _P, _P]
     lib.dmoe_expert_down.argtypes = [D, _P, _P, M, _P, _P, _P]
     lib.dmoe_padded_scatter.argtypes = [D, _P, _P, M, _P, _P, _P]
+    lib.dmoe_expert_down_combine.argtypes = [D, _P, _P, M, _P, _P, _P]
     lib.dmoe_bwd_dglu.argtypes = [D, _P, _P, _P, _P, M, _P, _P, _P, _P, _P]
     lib.dmoe_bwd_scatter.argtypes = [D, _P, _P, _P, M, _P, _P, _P]
     lib.dmoe_router_forward.argtypes = [D, _P, _P, _P, _P, _P]
@@ -105,6 +112,7 @@ def load():
     for fn in ("dmoe_sparse_map", "dmoe_sparse_map_noalloc", "dmoe_forward", "dmoe_backward",
                "dmoe_padded_gather",
                "dmoe_expert_glu", "dmoe_expert_glu_gather", "dmoe_expert_down", "dmoe_padded_scatter",
+               "dmoe_expert_down_combine",
                "dmoe_bwd_dglu", "dmoe_bwd_dx", "dmoe_bwd_wgrad", "dmoe_bwd_scatter",
                "dmoe_router_forward", "dmoe_router_dlogits", "dmoe_router_backward"):
         getattr(lib, fn).restype = _I
@@ -279,6 +287,13 @@ def dmoe_expert_down(dims, h_in, w2, smap: SparseMap, y_pad, y_scale, stream=Non
                                    _ptr(y_pad), _ptr(y_scale), _stream(stream)), "dmoe_expert_down")
 
 
+def dmoe_expert_down_combine(dims, h_in, w2, smap: SparseMap, y, y_acc, stream=None):
+    """y = the weighted combine of the down GEMM, fused (y_acc: T*h fp32 workspace)."""
+    _check(load().dmoe_expert_down_combine(ctypes.byref(dims), _ptr(h_in), _ptr(w2),
+                                           ctypes.byref(smap.c), _ptr(y), _ptr(y_acc),
+                                           _stream(stream)), "dmoe_expert_down_combine")
+
+
 def dmoe_padded_scatter(dims, y_pad, y_scale, smap: SparseMap, weights, y, stream=None):
     """y_scale None: y_pad is bf16; else block floating point (fp16 y_pad and its scales)."""
     _check(load().dmoe_padded_scatter(ctypes.byref(dims), _ptr(y_pad), _ptr(y_scale),
@@ -366,7 +381,7 @@ class Buffers:
         self.ws_map = torch.empty(max(dmoe_workspace_bytes(dims, WS_MAP), 16), **u8)
         self.train = train
         P, h, f = self.P, dims.hidden, dims.ffn
-        nsc = (h + SCALE_COLS - 1) // SCALE_COLS
+        nsc = scale_stride(h)
         bf = dict(dtype=torch.bfloat16, device=device)
         f32 = dict(dtype=torch.float32, device=device)
         self.saved = self.ws_bwd = None
@@ -389,7 +404,8 @@ class Buffers:
             self.ws_fwd = torch.empty(dmoe_workspace_bytes(dims, WS_FORWARD), **u8)
             self.step = dict(x_pad=torch.empty((P, h), **bf), h=torch.empty((P, f), **bf),
                              y_pad=torch.empty((P, h), dtype=torch.float16, device=device),
-                             y_scale=torch.empty((P, nsc), **f32))
+                             y_scale=torch.empty((P, nsc), **f32),
+                             y_acc=torch.empty((dims.T, h), **f32))
 
     def view(self, name: str) -> torch.Tensor:
         """[P, cols] view of a saved activation (x_pad, a, bm) or, after a training forward,
@@ -404,11 +420,14 @@ class Buffers:
         # forward workspace layout: H [P,f] bf16 | Y_pad [P,h] fp16 | scales [P, ceil(h/128)]
         # fp32, each start aligned to 256 bytes
         up = lambda v: (v + 255) // 256 * 256
-        nsc = (h + SCALE_COLS - 1) // SCALE_COLS
+        nsc = scale_stride(h)
         o_y = up(P * f * 2)
         o_s = up(o_y + P * h * 2)
         if name == "h":
             return self.ws_fwd[:P * f * 2].view(torch.bfloat16).view(P, f)
+        if name == "y_acc" and self.dims.flags & FUSED_COMBINE:  # [T,h] fp32 after H
+            T = self.dims.T
+            return self.ws_fwd[o_y:o_y + T * h * 4].view(torch.float32).view(T, h)
         if name == "y_pad":
             return self.ws_fwd[o_y:o_y + P * h * 2].view(torch.float16).view(P, h)
         if name == "y_scale":

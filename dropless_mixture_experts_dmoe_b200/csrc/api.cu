@@ -36,9 +36,11 @@ int check_dims(const dmoe_dims *d) {
     return DMOE_ERR_SHAPE;
   if (d->ffn < DMOE_BLOCKING || d->ffn % DMOE_BLOCKING != 0) return DMOE_ERR_SHAPE;
   if (d->hidden < DMOE_BLOCKING || d->hidden % DMOE_BLOCKING != 0) return DMOE_ERR_SHAPE;
-  if (d->flags & ~(DMOE_ROUTE_RENORMALIZE | DMOE_ROUTE_TOKEN_ROUNDING | DMOE_SAVE_X_ONLY))
+  if (d->flags & ~(DMOE_ROUTE_RENORMALIZE | DMOE_ROUTE_TOKEN_ROUNDING | DMOE_SAVE_X_ONLY |
+                   DMOE_FUSED_COMBINE))
     return DMOE_ERR_SHAPE;
-  if (rounding(d) && ((d->flags & DMOE_ROUTE_RENORMALIZE) || d->T > kRoundMaxT))
+  if (rounding(d) && ((d->flags & (DMOE_ROUTE_RENORMALIZE | DMOE_FUSED_COMBINE)) ||
+                      d->T > kRoundMaxT))
     return DMOE_ERR_SHAPE;
   const long long n = entries_of(d);
   const long long pmax =
@@ -139,9 +141,7 @@ GemmProblem problem_of(const dmoe_dims *d, const dmoe_map *m) {
 inline int dglu_tiles(const dmoe_dims *d) { return (d->ffn + kDgluTileCols - 1) / kDgluTileCols; }
 
 
-inline int scale_cols(const dmoe_dims *d) {
-  return (d->hidden + DMOE_SCALE_COLS - 1) / DMOE_SCALE_COLS;
-}
+inline int scale_cols(const dmoe_dims *d) { return dmoe_scale_stride(d->hidden); }
 
 inline bool save_x_only(const dmoe_dims *d) { return (d->flags & DMOE_SAVE_X_ONLY) != 0; }
 
@@ -169,19 +169,25 @@ BwdLayout bwd_layout(const dmoe_dims *d) {
   return l;
 }
 
-// Forward workspace layout: H [P,f] | Y_pad [P,h] fp16 | Y_pad scales [P, ceil(h/128)] fp32 |
-// X_pad [P,h].  A training forward keeps X_pad in the saved buffer and uses only the first
-// three (`train` bytes).
+inline bool fused_combine(const dmoe_dims *d) { return (d->flags & DMOE_FUSED_COMBINE) != 0; }
+
+// Forward workspace layout: H [P,f] | Y_pad [P,h] fp16 | Y_pad scales [P, ceil(h/128)] fp32
+// (with DMOE_FUSED_COMBINE instead the token accumulator y_acc [T,h] fp32) | X_pad [P,h].  A
+// training forward keeps X_pad in the saved buffer and uses only the first part (`train`).
 struct FwdLayout {
-  size_t h, ypad, yscale, xpad, train, total;
+  size_t h, ypad, yscale, yacc, xpad, train, total;
 };
 FwdLayout fwd_layout(const dmoe_dims *d) {
   const size_t P = (size_t)pmax_of(d);
   FwdLayout l;
   l.h = 0;
-  l.ypad = align_up(l.h + P * d->ffn * 2);
-  l.yscale = align_up(l.ypad + P * d->hidden * 2);
-  l.xpad = align_up(l.yscale + P * scale_cols(d) * sizeof(float));
+  l.ypad = l.yscale = l.yacc = align_up(l.h + P * d->ffn * 2);
+  if (fused_combine(d)) {
+    l.xpad = align_up(l.yacc + (size_t)d->T * d->hidden * sizeof(float));
+  } else {
+    l.yscale = align_up(l.ypad + P * d->hidden * 2);
+    l.xpad = align_up(l.yscale + P * scale_cols(d) * sizeof(float));
+  }
   l.train = l.xpad;
   l.total = align_up(l.xpad + P * d->hidden * 2);
   return l;
@@ -388,6 +394,24 @@ int dmoe_expert_down(const dmoe_dims *dims, const void *h_in, const void *w2,
                                     static_cast<cudaStream_t>(stream)));
 }
 
+int dmoe_expert_down_combine(const dmoe_dims *dims, const void *h_in, const void *w2,
+                             const dmoe_map *map, void *y, float *y_acc, void *stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (rounding(dims)) return DMOE_ERR_SHAPE;  // the epilogue finds a row's token as j / k
+  if ((rc = check_map(map, true))) return rc;
+  if (!h_in || !w2 || !y || !y_acc) return DMOE_ERR_NULL;
+  if (!aligned16(h_in) || !aligned16(w2) || !aligned16(y) || !aligned16(y_acc) ||
+      !aligned16(map->weights))
+    return DMOE_ERR_ALIGN;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long n = (long long)dims->T * dims->hidden;
+  if ((rc = launch_rc(launch_acc_zero(n, y_acc, st)))) return rc;
+  if ((rc = launch_rc(launch_down_red_gemm(problem_of(dims, map), h_in, w2, y_acc, st)))) return rc;
+  return launch_rc(launch_acc_round(n, y_acc, y, st));
+}
+
 int dmoe_padded_scatter(const dmoe_dims *dims, const void *y_pad, const float *y_scale,
                         const dmoe_map *map, const float *weights, void *y, void *stream) {
   int rc = check_dims(dims);
@@ -397,8 +421,8 @@ int dmoe_padded_scatter(const dmoe_dims *dims, const void *y_pad, const float *y
   if (!aligned16(y_pad) || !aligned16(y)) return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
   return launch_rc(launch_combine(dims->T, dims->hidden, dims->top_k, y_pad, y_scale,
-                                  map->dest_row, weights, y, static_cast<cudaStream_t>(stream),
-                                  entry_offsets_of(dims, map)));
+                                  map->dest_row, weights, y, map->status,
+                                  static_cast<cudaStream_t>(stream), entry_offsets_of(dims, map)));
 }
 
 int dmoe_forward(const dmoe_dims *dims, const void *x, const void *w1, const void *w3,
@@ -413,6 +437,7 @@ int dmoe_forward(const dmoe_dims *dims, const void *x, const void *w1, const voi
   if (ws_bytes < (saved ? l.train : l.total)) return DMOE_ERR_WORKSPACE;
   uint8_t *w = static_cast<uint8_t *>(ws);
   float *yscale = reinterpret_cast<float *>(w + l.yscale);
+  float *yacc = reinterpret_cast<float *>(w + l.yacc);
   uint8_t *xpad = w + l.xpad, *hbuf = w + l.h, *ypad = w + l.ypad, *abuf = nullptr,
           *bbuf = nullptr;
   if (saved) {
@@ -432,6 +457,7 @@ int dmoe_forward(const dmoe_dims *dims, const void *x, const void *w1, const voi
   // GLU GEMM through TMA row gathers, whose instruction rate cannot keep up with the MMAs.
   if ((rc = dmoe_padded_gather(dims, x, map, xpad, stream))) return rc;
   if ((rc = dmoe_expert_glu(dims, xpad, w1, w3, map, hbuf, abuf, bbuf, stream))) return rc;
+  if (fused_combine(dims)) return dmoe_expert_down_combine(dims, hbuf, w2, map, y, yacc, stream);
   if ((rc = dmoe_expert_down(dims, hbuf, w2, map, ypad, yscale, stream))) return rc;
   return dmoe_padded_scatter(dims, ypad, yscale, map, map->weights, y, stream);
 }
@@ -463,7 +489,7 @@ int dmoe_bwd_scatter(const dmoe_dims *dims, const void *dx_pad, const float *dx_
   if ((rc = check_device())) return rc;
   return launch_rc(launch_bwd_scatter(dims->T, dims->hidden, dims->top_k, dx_pad, dx_scale,
                                       map->dest_row, dw_part, dglu_tiles(dims), dx, dweights,
-                                      static_cast<cudaStream_t>(stream),
+                                      map->status, static_cast<cudaStream_t>(stream),
                                       entry_offsets_of(dims, map)));
 }
 

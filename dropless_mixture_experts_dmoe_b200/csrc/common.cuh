@@ -24,6 +24,10 @@ namespace dmoe {
 
 constexpr int kBlock = DMOE_BLOCKING;  // rows per padded block
 
+// Row stride of the block-floating-point scale arrays: ceil(h / 128) scales padded to a
+// multiple of 4 (16 bytes, so that the row slices can be bulk-copied).
+__host__ __device__ constexpr int dmoe_scale_stride(int h) { return ((h + 511) / 512) * 4; }
+
 // Cycle budget of one bounded wait (about a second at B200 clocks).
 constexpr long long kWaitCycles = 2000000000LL;
 // Budget used by a launch with a stall injected on purpose (a few milliseconds).
@@ -97,6 +101,13 @@ __device__ __forceinline__ float f16_lo(uint32_t v) {
 }
 __device__ __forceinline__ float f16_hi(uint32_t v) {
   return __half2float(__ushort_as_half((unsigned short)(v >> 16)));
+}
+
+// Vector reduction into global fp32 memory: [p .. p+3] += {a, b, c, d} (16-byte aligned).
+__device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
 }
 
 // ---- mbarrier -----------------------------------------------------------------------------
@@ -340,6 +351,17 @@ __device__ __forceinline__ void tma_store_2d_u32(const CUtensorMap *map, uint32_
       "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
           reinterpret_cast<uint64_t>(map)),
       "r"(smem_src), "r"(x), "r"(y)
+      : "memory");
+}
+
+// Untiled bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from global
+// to this CTA's shared memory, completing on the mbarrier at shared address `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t smem_dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_dst),
+      "l"(src), "r"(bytes), "r"(bar)
       : "memory");
 }
 

@@ -97,7 +97,8 @@ enum GemmMode {
   MODE_GLU_GATHER = 5,  // GLU whose A rows are gathered from the token rows of x
   MODE_ROUTER = 6,      // router logits
   MODE_RDX = 7,         // router input gradient, accumulated into dx
-  MODE_RWGRAD = 8       // router weight gradient, split over the token dimension
+  MODE_RWGRAD = 8,      // router weight gradient, split over the token dimension
+  MODE_DOWN_RED = 9     // down GEMM with the weighted combine in its epilogue
 };
 
 __host__ __device__ constexpr bool is_glu(int mode) {
@@ -110,14 +111,17 @@ __host__ __device__ constexpr bool is_glu(int mode) {
 // Measured: two slabs speed up GLU, DOWN and DX, and slow DGLU (12 result boxes per tile
 // through one staging buffer) and the weight gradients.
 __host__ __device__ constexpr int mode_kslabs(int mode, int epi) {
-  return (epi == 4 && (mode == MODE_GLU || mode == MODE_DOWN || mode == MODE_DX)) ? 2 : 1;
+  return (epi == 4 && (mode == MODE_GLU || mode == MODE_DOWN || mode == MODE_DOWN_RED ||
+                       mode == MODE_DX))
+             ? 2
+             : 1;
 }
 
 // Modes whose tiles are (pair of an expert's row blocks, column tile), enumerated from
 // padded_bins; the others are the weight gradients and the dense router GEMMs.
 __host__ __device__ constexpr bool uses_units(int mode) {
   return mode == MODE_GLU || mode == MODE_GLU_GATHER || mode == MODE_DOWN ||
-         mode == MODE_DGLU || mode == MODE_DX;
+         mode == MODE_DOWN_RED || mode == MODE_DGLU || mode == MODE_DX;
 }
 
 // Dense row modes: tiles are (pair of 128-row blocks of the T token rows, column tile).
@@ -312,10 +316,10 @@ __device__ __forceinline__ void load_stage(const GemmParams &p, const Tile &tl, 
     static_assert(MODE != MODE_GLU || KSLABS == 2, "GLU stages hold two K slabs");
     tma_load_3d_pair(sa, &p.tm[0], bar, 0, tl.row0, 2 * kb);
     tma_load_3d_pair(sb, &p.tm[rank == 0 ? 1 : 2], bar, 0, tl.e * p.f + tl.n * (BN / 2), 2 * kb);
-  } else if (MODE == MODE_DOWN && KSLABS == 2) {
+  } else if ((MODE == MODE_DOWN || MODE == MODE_DOWN_RED) && KSLABS == 2) {
     tma_load_3d_pair(sa, &p.tm[0], bar, 0, tl.row0, 2 * kb);
     tma_load_3d_pair(sb, &p.tm[1], bar, 0, tl.e * p.h + tl.n * BN + (int)rank * (BN / 2), 2 * kb);
-  } else if (MODE == MODE_DOWN) {
+  } else if (MODE == MODE_DOWN || MODE == MODE_DOWN_RED) {
     tma_load_2d_pair(sa, &p.tm[0], bar, kb * BK, tl.row0);
     tma_load_2d_pair(sb, &p.tm[1], bar, kb * BK, tl.e * p.h + tl.n * BN + (int)rank * (BN / 2));
   } else if (MODE == MODE_DGLU) {
@@ -494,7 +498,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
     const int ncols = min(kw, p.h - n0);   // multiple of 64 (may be <= 0)
     if (ncols <= 0) return;
     tb += (uint32_t)(half * kw);
-    const int nsc = (p.h + DMOE_SCALE_COLS - 1) / DMOE_SCALE_COLS;
+    const int nsc = dmoe_scale_stride(p.h);
     float *srow = p.part + (size_t)(y0 + lane) * nsc;
 #pragma unroll 1
     for (int c0 = 0; c0 < ncols; c0 += DMOE_SCALE_COLS) {
@@ -525,6 +529,38 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
           w[16 + i] = pack_f16x2(__uint_as_float(v1[2 * i]) * sc, __uint_as_float(v1[2 * i + 1]) * sc);
         }
         st.emit(&p.tmo[0], w, n0 + c0 + c, y0);
+      }
+    }
+  } else if (MODE == MODE_DOWN_RED) {
+    // the weighted combine fused in: the row's routing weight times its fp32 accumulator row,
+    // added into y_acc [T, h] fp32 at the row's token with vector reductions (no Y_pad)
+    const int n0 = tl.n * BN + half * kw;
+    const int ncols = min(kw, p.h - n0);  // multiple of 64 (may be <= 0)
+    if (ncols <= 0) return;
+    const int grow = y0 + lane;
+    const int pstart = (tl.e > 0) ? p.padded_bins[tl.e - 1] : 0;
+    const int bstart = (tl.e > 0) ? p.bins[tl.e - 1] : 0;
+    const int local = grow - pstart;
+    int tok = -1;
+    float wr = 0.0f;
+    if (local < p.bins[tl.e] - bstart) {  // a real row, not padding
+      const int j = __ldg(p.indices + bstart + local);
+      tok = j / p.k;
+      wr = __ldg(p.weights + j);
+    }
+    tb += (uint32_t)(half * kw);
+    float *dst = p.part + (size_t)(tok < 0 ? 0 : tok) * p.h + n0;
+#pragma unroll 1
+    for (int c = 0; c < ncols; c += 32) {
+      uint32_t v[32];
+      tmem_ld32(tb + c, v);
+      tmem_ld_wait();
+      if (tok >= 0) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          red_add_v4(dst + c + 4 * q, wr * __uint_as_float(v[4 * q]),
+                     wr * __uint_as_float(v[4 * q + 1]), wr * __uint_as_float(v[4 * q + 2]),
+                     wr * __uint_as_float(v[4 * q + 3]));
       }
     }
   } else if (MODE == MODE_DGLU) {
@@ -1145,6 +1181,30 @@ cudaError_t launch_down_gemm(const GemmProblem &g, const void *h_in, const void 
   }
   p.k_iters = g.f / Cfg<MODE_DOWN, 4>::bk;
   return launch_gemm<MODE_DOWN, 4>(p, max_units(g) * p.n_tiles, st);
+}
+
+cudaError_t launch_down_red_gemm(const GemmProblem &g, const void *h_in, const void *w2,
+                                 float *y_acc, cudaStream_t st) {
+  GemmParams p = base_params(g);
+  const uint64_t P = (uint64_t)g.nblk_cap * BM;
+  const bool short_k = g.f / BK <= 4;  // ffn <= 256: the epilogue bounds a tile (8 warps)
+  const bool ok = short_k ? (make_tmap(&p.tm[0], h_in, P, g.f, BM) &&
+                             make_tmap(&p.tm[1], w2, (uint64_t)g.E * g.h, g.f, BN / 2))
+                          : (make_tmap_chunked(&p.tm[0], h_in, P, g.f, BM) &&
+                             make_tmap_chunked(&p.tm[1], w2, (uint64_t)g.E * g.h, g.f, BN / 2));
+  if (!ok) return cudaErrorInvalidValue;
+  p.tm[2] = p.tm[3] = p.tm[4] = p.tm[0];
+  p.tmo[0] = p.tm[0];  // no result stores: the epilogue reduces into y_acc
+  p.weights = g.weights;
+  p.part = y_acc;
+  p.n_tiles = (g.h + BN - 1) / BN;
+  p.group = raster_units(g.f);
+  if (short_k) {
+    p.k_iters = g.f / Cfg<MODE_DOWN_RED, 8>::bk;
+    return launch_gemm<MODE_DOWN_RED, 8>(p, max_units(g) * p.n_tiles, st);
+  }
+  p.k_iters = g.f / Cfg<MODE_DOWN_RED, 4>::bk;
+  return launch_gemm<MODE_DOWN_RED, 4>(p, max_units(g) * p.n_tiles, st);
 }
 
 cudaError_t launch_dglu_gemm(const GemmProblem &g, const void *dy_pad, const void *w2,

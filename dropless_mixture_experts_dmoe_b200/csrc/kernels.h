@@ -79,7 +79,7 @@ cudaError_t launch_gather(int T, int h, int k, int E, const void *x, const int32
 // block-floating-point rows (fp16 values, y_scale [P_max, ceil(h/DMOE_SCALE_COLS)]).
 cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const float *y_scale,
                            const int32_t *dest_row, const float *weights, void *y,
-                           cudaStream_t st, const int32_t *offsets = nullptr);
+                           int32_t *status, cudaStream_t st, const int32_t *offsets = nullptr);
 
 // Backward scatter: dx_t = bf16(sum_s dX_pad[dest_row[t*k+s]]) over the block-floating-point
 // rows of launch_dx_gemm (value = fp16 * scale, summed in fp32) and, from the DGLU GEMM's
@@ -87,7 +87,8 @@ cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const float *
 cudaError_t launch_bwd_scatter(int T, int h, int k, const void *dx_pad, const float *dx_scale,
                                const int32_t *dest_row,
                                const float *part, int nt, void *dx, float *dweights,
-                               cudaStream_t st, const int32_t *offsets = nullptr);
+                               int32_t *status, cudaStream_t st,
+                               const int32_t *offsets = nullptr);
 
 // Shape and map pointers shared by the grouped GEMM launchers.
 struct GemmProblem {
@@ -118,6 +119,13 @@ cudaError_t launch_down_gemm(const GemmProblem &g, const void *h_in, const void 
 // ... and the backward: dH with the fused dGLU epilogue, dX, and the weight gradients.
 // DGLU column tile width (part has ceil(f / kDgluTileCols) columns).
 constexpr int kDgluTileCols = 256;
+// Down GEMM with the weighted combine fused into its epilogue: y_acc[t] += w_ts * (H W2_e^T)
+// row of each real padded row (fp32 vector reductions into y_acc [T, h]; no Y_pad).
+cudaError_t launch_down_red_gemm(const GemmProblem &g, const void *h_in, const void *w2,
+                                 float *y_acc, cudaStream_t st);
+// n (a multiple of 8) fp32 accumulator values: zeroed / rounded to bf16.
+cudaError_t launch_acc_zero(long long n, float *acc, cudaStream_t st);
+cudaError_t launch_acc_round(long long n, const float *acc, void *y, cudaStream_t st);
 cudaError_t launch_dglu_gemm(const GemmProblem &g, const void *dy_pad, const void *w2,
                              const void *a_in, const void *b_in, void *da_out, void *db_out,
                              void *hw_out, float *part, cudaStream_t st);

@@ -90,8 +90,9 @@ extern "C" {
 /* Problem shape.  T tokens, hidden size h, ffn size f (per expert), E experts, top_k, and
  * the variant flags: 0 (the default: weights are the softmax over all E logits at the chosen
  * experts, and the forward saves X_pad, A and Bm for the backward) or an OR of
- * DMOE_ROUTE_RENORMALIZE or DMOE_ROUTE_TOKEN_ROUNDING (not both) and DMOE_SAVE_X_ONLY.  Other
- * bits are rejected.  Every call of one layer instance must see the same flags. */
+ * DMOE_ROUTE_RENORMALIZE or DMOE_ROUTE_TOKEN_ROUNDING (not both), DMOE_FUSED_COMBINE and
+ * DMOE_SAVE_X_ONLY.  Other bits are rejected.  Every call of one layer instance must see the
+ * same flags. */
 typedef struct {
   int32_t T, hidden, ffn, num_experts, top_k;
   int32_t flags;
@@ -103,8 +104,9 @@ typedef struct {
 #define DMOE_ROUTE_RENORMALIZE 0x1
 
 /* Block floating point of the padded expert outputs (Y_pad of dmoe_expert_down, dX_pad of
- * dmoe_bwd_dx): fp16 values [P_max, h] and fp32 scales [P_max, ceil(h / DMOE_SCALE_COLS)]; the
- * value of row r, column c is fp16[r][c] * scale[r][c / DMOE_SCALE_COLS].  Each scale is a
+ * dmoe_bwd_dx): fp16 values [P_max, h] and fp32 scales [P_max, 4 * ceil(h / 512)] (ceil(h/128)
+ * scales per row, the row padded to a multiple of 4); the value of row r, column c is
+ * fp16[r][c] * scale[r][c / DMOE_SCALE_COLS].  Each scale is a
  * power of two that puts the largest magnitude of its 128 columns into [2^13, 2^14] (1 for an
  * all-zero or non-finite group), so every value keeps fp16's 11 significant bits at bf16's
  * size.  The k rows of a token are summed afterwards in fp32; rounding each to bf16 first (8
@@ -130,6 +132,16 @@ typedef struct {
  *   calls, dmoe_expert_glu_gather and dmoe_sparse_map_noalloc reject the flag
  *   (DMOE_ERR_SHAPE), as does T > 2^20; dmoe_sparse_map needs the logits. */
 #define DMOE_ROUTE_TOKEN_ROUNDING 0x2
+
+/* Forward variant: the weighted combine fused into the down GEMM (the walkthrough's padded
+ * scatter, section 4.2, done by the GEMM's epilogue; the SonicMoE abstract's IO overlap).  The
+ * epilogue multiplies each real padded row's fp32 result by its routing weight and adds it,
+ * with vector reductions, into an fp32 token-major accumulator; a last pass rounds it to
+ * bf16.  Y_pad is never written or read.  The additions of a token's k rows happen in any
+ * order: bit-for-bit reproducible for top_k <= 2 (a + b = b + a from zero), reproducible to
+ * fp32 rounding otherwise.  dmoe_forward then runs dmoe_padded_gather, dmoe_expert_glu and
+ * dmoe_expert_down_combine.  Not combined with DMOE_ROUTE_TOKEN_ROUNDING (DMOE_ERR_SHAPE). */
+#define DMOE_FUSED_COMBINE 0x8
 
 /* Memory variant (walkthrough section 4.4's MemoryOptimizedMLP; the SonicMoE abstract's
  * activation-memory saving): the training forward saves only X_pad (dmoe_saved_bytes shrinks
@@ -303,16 +315,23 @@ DMOE_API int dmoe_expert_glu_gather(const dmoe_dims *dims, const void *x, const 
 
 /* Down GEMM: Y_pad[b] = H[b] W2_e^T for every block b < num_blocks, fp32 accumulation,
  * stored in block floating point (see DMOE_SCALE_COLS).
- * h_in [P_max,f] bf16 -> y_pad [P_max,h] fp16, y_scale [P_max, ceil(h/128)] fp32. */
+ * h_in [P_max,f] bf16 -> y_pad [P_max,h] fp16, y_scale [P_max, 4*ceil(h/512)] fp32. */
 DMOE_API int dmoe_expert_down(const dmoe_dims *dims, const void *h_in, const void *w2,
                               const dmoe_map *map, void *y_pad, float *y_scale, void *stream);
+
+/* Down GEMM and weighted combine in one (DMOE_FUSED_COMBINE): y_t = bf16(sum over the
+ * token's entries of w_ts * (H W2_e^T) row), the sum in fp32 in y_acc by vector reductions
+ * from the GEMM's epilogue.  h_in [P_max,f] bf16, map->weights -> y [T,h] bf16; y_acc: T*h
+ * fp32 of caller workspace (zeroed by the call).  Three launches: zero, GEMM, rounding. */
+DMOE_API int dmoe_expert_down_combine(const dmoe_dims *dims, const void *h_in, const void *w2,
+                                      const dmoe_map *map, void *y, float *y_acc, void *stream);
 
 /* Weighted padded_scatter (walkthrough section 4.2, B_TO_A direction, times the routing
  * weight): y_t = bf16(sum_{s=0..k-1} w_ts * Y_pad[dest_row[t*k+s]]), summed in fp32 in
  * slot order (each entry one fused multiply-add), no atomics.  weights == NULL means w = 1
  * (the backward's gather gradient, dx_t = sum_s dX_pad[dest_row[t*k+s]]).  Row format:
  * y_scale == NULL: y_pad [P_max,h] bf16; otherwise block floating point as written by
- * dmoe_expert_down (y_pad fp16, y_scale [P_max, ceil(h/128)]).  -> y [T,h] bf16. */
+ * dmoe_expert_down (y_pad fp16, y_scale [P_max, 4*ceil(h/512)]).  -> y [T,h] bf16. */
 DMOE_API int dmoe_padded_scatter(const dmoe_dims *dims, const void *y_pad, const float *y_scale,
                                  const dmoe_map *map, const float *weights, void *y,
                                  void *stream);
@@ -340,7 +359,7 @@ DMOE_API int dmoe_bwd_dglu(const dmoe_dims *dims, const void *dy_pad, const void
  * stored in block floating point (see DMOE_SCALE_COLS): the k rows of a token are summed by
  * dmoe_bwd_scatter, and rounding each of them to bf16 first would put k bf16 roundings into
  * every element of dx.
- * da, dbm [P_max,f] bf16 -> dx_pad [P_max,h] fp16, dx_scale [P_max, ceil(h/128)] fp32. */
+ * da, dbm [P_max,f] bf16 -> dx_pad [P_max,h] fp16, dx_scale [P_max, 4*ceil(h/512)] fp32. */
 DMOE_API int dmoe_bwd_dx(const dmoe_dims *dims, const void *da, const void *dbm, const void *w1,
                          const void *w3, const dmoe_map *map, void *dx_pad, float *dx_scale,
                          void *stream);

@@ -78,12 +78,29 @@ def test_bad_dims_rejected_before_launch(lib, dims, code):
 
 def test_unknown_flag_rejected(lib):
     m = B.dmoe_map()
-    d = B.make_dims(256, 128, 128, 8, 2, flags=0x8)
-    assert B.dmoe_padded_rows_max(d) == 0
-    assert lib.dmoe_sparse_map(ctypes.byref(d), None, ctypes.byref(m), None, 0, None) == -2
-    for fl in (B.ROUTE_RENORMALIZE, B.SAVE_X_ONLY, B.ROUTE_RENORMALIZE | B.SAVE_X_ONLY):
+    for bad in (0x10, 0x40, B.ROUTE_TOKEN_ROUNDING | B.ROUTE_RENORMALIZE,
+                B.ROUTE_TOKEN_ROUNDING | B.FUSED_COMBINE):
+        d = B.make_dims(256, 128, 128, 8, 2, flags=bad)
+        assert B.dmoe_padded_rows_max(d) == 0
+        assert lib.dmoe_sparse_map(ctypes.byref(d), None, ctypes.byref(m), None, 0, None) == -2
+    for fl in (B.ROUTE_RENORMALIZE, B.SAVE_X_ONLY, B.ROUTE_RENORMALIZE | B.SAVE_X_ONLY,
+               B.ROUTE_TOKEN_ROUNDING, B.ROUTE_TOKEN_ROUNDING | B.SAVE_X_ONLY, B.FUSED_COMBINE,
+               B.FUSED_COMBINE | B.ROUTE_RENORMALIZE | B.SAVE_X_ONLY):
         d = B.make_dims(256, 128, 128, 8, 2, flags=fl)
         assert B.dmoe_padded_rows_max(d) > 0  # the defined flags are accepted
+
+
+def test_token_rounding_sizes(lib):
+    """DMOE_ROUTE_TOKEN_ROUNDING: up to 64 added entries per expert (T*k + 64E), the padded
+    bound from that, and T above 2^20 rejected; the router calls reject the flag."""
+    d = B.make_dims(4096, 128, 128, 64, 8, flags=B.ROUTE_TOKEN_ROUNDING)
+    assert B.dmoe_entries_max(d) == 4096 * 8 + 64 * 64
+    assert B.dmoe_padded_rows_max(d) == (4096 * 8 + 64 * 64 + 127 * 64) // 128 * 128
+    assert B.dmoe_entries_max(B.make_dims(4096, 128, 128, 64, 8)) == 4096 * 8
+    assert B.dmoe_entries_max(B.make_dims((1 << 20) + 1, 128, 128, 8, 1,
+                                          flags=B.ROUTE_TOKEN_ROUNDING)) == 0
+    m = B.dmoe_map()
+    assert lib.dmoe_router_dlogits(ctypes.byref(d), None, ctypes.byref(m), None, None, None) == -2
 
 
 def test_save_x_only_sizes(lib):

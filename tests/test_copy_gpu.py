@@ -83,7 +83,7 @@ def test_weighted_scatter_block_floating_point(w):
     bit for bit against the same fp32 sum in slot order."""
     dims, bufs, g, x = _setup(w)
     P, h = bufs.P, w.hidden
-    nsc = (h + 127) // 128
+    nsc = B.scale_stride(h)  # ceil(h/128) scales per row, padded to a multiple of 4
     gen = torch.Generator(device="cpu").manual_seed(5)
     vals = (torch.randn((P, h), generator=gen) * 4096).to(torch.float16)
     expo = torch.randint(-20, 5, (P, nsc), generator=gen).float()
