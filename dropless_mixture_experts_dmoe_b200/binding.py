@@ -282,7 +282,7 @@ def dmoe_expert_glu_gather(dims, x, w1, w3, smap: SparseMap, h_out, a_out=None, 
 
 
 def dmoe_expert_down(dims, h_in, w2, smap: SparseMap, y_pad, y_scale, stream=None):
-    """y_pad [P_max,h] fp16 and y_scale [P_max, ceil(h/128)] fp32: block floating point."""
+    """y_pad [P_max,h] fp16 and y_scale [P_max, scale_stride(h)] fp32: block floating point."""
     _check(load().dmoe_expert_down(ctypes.byref(dims), _ptr(h_in), _ptr(w2), ctypes.byref(smap.c),
                                    _ptr(y_pad), _ptr(y_scale), _stream(stream)), "dmoe_expert_down")
 
@@ -316,7 +316,7 @@ def dmoe_bwd_scatter(dims, dx_pad, dx_scale, dw_part, smap: SparseMap, dx, dweig
 
 
 def dmoe_bwd_dx(dims, da, dbm, w1, w3, smap: SparseMap, dx_pad, dx_scale, stream=None):
-    """dx_pad [P_max,h] fp16 and dx_scale [P_max, ceil(h/256)] fp32: block floating point."""
+    """dx_pad [P_max,h] fp16 and dx_scale [P_max, scale_stride(h)] fp32: block floating point."""
     _check(load().dmoe_bwd_dx(ctypes.byref(dims), _ptr(da), _ptr(dbm), _ptr(w1), _ptr(w3),
                               ctypes.byref(smap.c), _ptr(dx_pad), _ptr(dx_scale),
                               _stream(stream)), "dmoe_bwd_dx")
@@ -417,7 +417,7 @@ class Buffers:
             cols = h if name == "x_pad" else f
             off = self.offsets[name]
             return self.saved[off:off + P * cols * 2].view(torch.bfloat16).view(P, cols)
-        # forward workspace layout: H [P,f] bf16 | Y_pad [P,h] fp16 | scales [P, ceil(h/128)]
+        # forward workspace layout: H [P,f] bf16 | Y_pad [P,h] fp16 | scales [P, scale_stride(h)]
         # fp32, each start aligned to 256 bytes
         up = lambda v: (v + 255) // 256 * 256
         nsc = scale_stride(h)

@@ -147,8 +147,8 @@ inline bool save_x_only(const dmoe_dims *d) { return (d->flags & DMOE_SAVE_X_ONL
 
 // Backward workspace layout: dY_pad [P,h] bf16, whose region is reused for dX_pad [P,h] fp16
 // once the weight gradients have read dY_pad | dA [P,f] | dBm [P,f] | Hw [P,f] | routing-weight
-// partials [P, ceil(f/256)] fp32 | dX_pad scales [P, ceil(h/128)] fp32 | with DMOE_SAVE_X_ONLY
-// the recomputed A [P,f] and Bm [P,f]
+// partials [P, ceil(f/256)] fp32 | dX_pad scales [P, dmoe_scale_stride(h)] fp32 | with
+// DMOE_SAVE_X_ONLY the recomputed A [P,f] and Bm [P,f]
 struct BwdLayout {
   size_t dy, da, db, hw, part, dxs, a, bm, total;
 };
@@ -171,9 +171,9 @@ BwdLayout bwd_layout(const dmoe_dims *d) {
 
 inline bool fused_combine(const dmoe_dims *d) { return (d->flags & DMOE_FUSED_COMBINE) != 0; }
 
-// Forward workspace layout: H [P,f] | Y_pad [P,h] fp16 | Y_pad scales [P, ceil(h/128)] fp32
-// (with DMOE_FUSED_COMBINE instead the token accumulator y_acc [T,h] fp32) | X_pad [P,h].  A
-// training forward keeps X_pad in the saved buffer and uses only the first part (`train`).
+// Forward workspace layout: H [P,f] | Y_pad [P,h] fp16 | Y_pad scales [P, dmoe_scale_stride(h)]
+// fp32 (with DMOE_FUSED_COMBINE instead the token accumulator y_acc [T,h] fp32) | X_pad [P,h].
+// A training forward keeps X_pad in the saved buffer and uses only the first part (`train`).
 struct FwdLayout {
   size_t h, ypad, yscale, yacc, xpad, train, total;
 };
@@ -421,8 +421,8 @@ int dmoe_padded_scatter(const dmoe_dims *dims, const void *y_pad, const float *y
   if (!aligned16(y_pad) || !aligned16(y)) return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
   return launch_rc(launch_combine(dims->T, dims->hidden, dims->top_k, y_pad, y_scale,
-                                  map->dest_row, weights, y, map->status,
-                                  static_cast<cudaStream_t>(stream), entry_offsets_of(dims, map)));
+                                  map->dest_row, weights, y, static_cast<cudaStream_t>(stream),
+                                  entry_offsets_of(dims, map)));
 }
 
 int dmoe_forward(const dmoe_dims *dims, const void *x, const void *w1, const void *w3,
@@ -489,7 +489,7 @@ int dmoe_bwd_scatter(const dmoe_dims *dims, const void *dx_pad, const float *dx_
   if ((rc = check_device())) return rc;
   return launch_rc(launch_bwd_scatter(dims->T, dims->hidden, dims->top_k, dx_pad, dx_scale,
                                       map->dest_row, dw_part, dglu_tiles(dims), dx, dweights,
-                                      map->status, static_cast<cudaStream_t>(stream),
+                                      static_cast<cudaStream_t>(stream),
                                       entry_offsets_of(dims, map)));
 }
 

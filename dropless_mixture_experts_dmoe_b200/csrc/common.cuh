@@ -354,17 +354,6 @@ __device__ __forceinline__ void tma_store_2d_u32(const CUtensorMap *map, uint32_
       : "memory");
 }
 
-// Untiled bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from global
-// to this CTA's shared memory, completing on the mbarrier at shared address `bar`.
-__device__ __forceinline__ void bulk_load(uint32_t smem_dst, const void *src, uint32_t bytes,
-                                          uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
-}
-
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

@@ -186,7 +186,7 @@ struct GemmParams {
   const __nv_bfloat16 *in0, *in1;  // DGLU: saved A, Bm
   const float *weights;            // DGLU: routing weight of each flattened entry
   float *part;                     // DGLU: [P_max, n_tiles] partial routing-weight gradients;
-                                   // DOWN, DX: [P_max, ceil(h/128)] scales of the output rows
+                                   // DOWN, DX: [P_max, dmoe_scale_stride(h)] scales of the rows
   int total;                       // router modes: number of pair tiles
   int split_k;                     // RWGRAD: 64-wide K steps per split
   int Ep;                          // RWGRAD: rows of one split's slab (E rounded up to 128)

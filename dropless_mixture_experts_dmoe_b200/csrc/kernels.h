@@ -76,10 +76,10 @@ cudaError_t launch_gather(int T, int h, int k, int E, const void *x, const int32
                           const int32_t *counts, const int32_t *padded_bins, void *x_pad,
                           cudaStream_t st, const int32_t *offsets = nullptr);
 // Token-major weighted combine (weights may be NULL: w = 1) of bf16 rows (y_scale NULL) or of
-// block-floating-point rows (fp16 values, y_scale [P_max, ceil(h/DMOE_SCALE_COLS)]).
+// block-floating-point rows (fp16 values, y_scale [P_max, dmoe_scale_stride(h)]).
 cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const float *y_scale,
                            const int32_t *dest_row, const float *weights, void *y,
-                           int32_t *status, cudaStream_t st, const int32_t *offsets = nullptr);
+                           cudaStream_t st, const int32_t *offsets = nullptr);
 
 // Backward scatter: dx_t = bf16(sum_s dX_pad[dest_row[t*k+s]]) over the block-floating-point
 // rows of launch_dx_gemm (value = fp16 * scale, summed in fp32) and, from the DGLU GEMM's
@@ -87,8 +87,7 @@ cudaError_t launch_combine(int T, int h, int k, const void *y_pad, const float *
 cudaError_t launch_bwd_scatter(int T, int h, int k, const void *dx_pad, const float *dx_scale,
                                const int32_t *dest_row,
                                const float *part, int nt, void *dx, float *dweights,
-                               int32_t *status, cudaStream_t st,
-                               const int32_t *offsets = nullptr);
+                               cudaStream_t st, const int32_t *offsets = nullptr);
 
 // Shape and map pointers shared by the grouped GEMM launchers.
 struct GemmProblem {
@@ -110,9 +109,9 @@ cudaError_t launch_glu_gemm(const GemmProblem &g, const void *x_pad, const void 
 cudaError_t launch_glu_gather_gemm(const GemmProblem &g, const void *x, const void *w1,
                                    const void *w3, void *h_out, void *a_out, void *b_out,
                                    cudaStream_t st);
-// Y_pad [P_max,h] in block floating point: fp16 values, y_scale [P_max, ceil(h/128)] fp32 one
-// power-of-two scale per row and DMOE_SCALE_COLS columns (value = fp16 * scale), 11 significant
-// bits per value at bf16's size (the k rows of a token are summed by the combine; a bf16
+// Y_pad [P_max,h] in block floating point: fp16 values, y_scale [P_max, dmoe_scale_stride(h)]
+// fp32, one power-of-two scale per row and DMOE_SCALE_COLS columns (value = fp16 * scale), 11
+// significant bits per value at bf16's size (the k rows of a token are summed by the combine; a bf16
 // rounding of each would put k roundings into every output element).
 cudaError_t launch_down_gemm(const GemmProblem &g, const void *h_in, const void *w2, void *y_pad,
                              float *y_scale, cudaStream_t st);

@@ -2,9 +2,12 @@
 tolerance of the stress shapes (shapes outside the five named workloads).
 
 The layer stores its intermediates in bf16 with fp32 accumulation: H = bf16(silu(A) * Bm),
-Y_pad = bf16(H W2^T), y = bf16(sum_s w_s Y_s); in the backward A, Bm are the saved bf16
-values, dA, dBm and Hw = w h are bf16, dX = bf16(dA W1 + dBm W3), dx = bf16(sum_s dX_s), and
-the weight gradients stay fp32.  This module applies exactly those roundings to float64
+Y_pad = bfp(H W2^T), y = bf16(sum_s w_s Y_s); in the backward A, Bm are the saved bf16
+values, dA, dBm and Hw = w h are bf16, dX = bfp(dA W1 + dBm W3), dx = bf16(sum_s dX_s), and
+the weight gradients stay fp32.  bfp is the block floating point of Y_pad and dX_pad: per row
+and 128 columns, a power of two that puts the group's largest magnitude into [2^13, 2^14),
+then fp16 (round to nearest even).  With the fused combine Y is not stored at all: y =
+bf16(sum_s w_s (H W2^T)_s) with fp32 sums.  This module applies exactly those roundings to float64
 arithmetic on the same inputs (no other error source), so its max-abs error against the
 oracle is what an ideal bf16 pipeline of this design reaches on that shape.  With few
 products per output element (few tokens per expert) that error can exceed 5 % of the RMS,
@@ -24,12 +27,27 @@ def _bf(t: torch.Tensor) -> torch.Tensor:
     return t.to(torch.bfloat16).double()
 
 
+def _bfp(t: torch.Tensor, cols: int = 128) -> torch.Tensor:
+    """Round rows of ``t`` [rows, n] (n a multiple of 64) to the block floating point format."""
+    rows, n = t.shape
+    out = torch.empty_like(t)
+    for c0 in range(0, n, cols):
+        g = t[:, c0:c0 + cols].float().double()  # the kernel scales its fp32 accumulator
+        m = g.abs().amax(dim=1, keepdim=True)
+        _, ex = torch.frexp(m)                   # m = mant * 2^ex, mant in [0.5, 1)
+        es = torch.where(m > 0, 14 - ex, torch.zeros_like(ex)).clamp(-126, 126).double()
+        sc = torch.pow(2.0, es)
+        out[:, c0:c0 + cols] = (g * sc).half().double() / sc
+    return out
+
+
 def stress_bound(modelled: float) -> float:
     """Max-abs / RMS bound for a stress shape whose modelled bf16 error is ``modelled``."""
     return MAX_ABS_RMS if 1.25 * modelled <= MAX_ABS_RMS else 1.5 * modelled
 
 
-def forward_model(inp: dict, top: np.ndarray, wts: np.ndarray) -> np.ndarray:
+def forward_model(inp: dict, top: np.ndarray, wts: np.ndarray, fused: bool = False) -> np.ndarray:
+    """y under the roundings above; ``fused`` models the fused combine (no Y_pad)."""
     X = inp["x"].double()
     W1, W3, W2 = inp["w1"].double(), inp["w3"].double(), inp["w2"].double()
     E = W1.shape[0]
@@ -43,7 +61,8 @@ def forward_model(inp: dict, top: np.ndarray, wts: np.ndarray) -> np.ndarray:
             Xe = X[ts]
             a = (Xe @ W1[e].T).float().double()
             b = (Xe @ W3[e].T).float().double()
-            Y = _bf(_bf(torch.nn.functional.silu(a) * b) @ W2[e].T)
+            Y = _bf(torch.nn.functional.silu(a) * b) @ W2[e].T
+            Y = Y.float().double() if fused else _bfp(Y)
             y[ts] += wf[ts, s][:, None] * Y
     return _bf(y).numpy()
 
@@ -72,7 +91,7 @@ def backward_model(inp: dict, top: np.ndarray, wts: np.ndarray) -> dict:
         dA = _bf(wr * G * Bm * s * (1 + A * (1 - s)))
         dB = _bf(wr * G * A * s)
         dw[ts, ss] = (G * hv).sum(1)
-        dxs[ts, ss] = _bf(dA @ W1[e] + dB @ W3[e])
+        dxs[ts, ss] = _bfp(dA @ W1[e] + dB @ W3[e])
         dW1[e] = dA.T @ Xe
         dW3[e] = dB.T @ Xe
         dW2[e] = dy[ts].T @ _bf(wr * hv)
