@@ -388,7 +388,8 @@ int dmoe_expert_down(const dmoe_dims *dims, const void *h_in, const void *w2,
   if (rc) return rc;
   if ((rc = check_map(map, false))) return rc;
   if (!h_in || !w2 || !y_pad || !y_scale) return DMOE_ERR_NULL;
-  if (!aligned16(h_in) || !aligned16(w2) || !aligned16(y_pad)) return DMOE_ERR_ALIGN;
+  if (!aligned16(h_in) || !aligned16(w2) || !aligned16(y_pad) || !aligned16(y_scale))
+    return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
   return launch_rc(launch_down_gemm(problem_of(dims, map), h_in, w2, y_pad, y_scale,
                                     static_cast<cudaStream_t>(stream)));
@@ -418,7 +419,7 @@ int dmoe_padded_scatter(const dmoe_dims *dims, const void *y_pad, const float *y
   if (rc) return rc;
   if ((rc = check_map(map, false, dims))) return rc;
   if (!y_pad || !y) return DMOE_ERR_NULL;
-  if (!aligned16(y_pad) || !aligned16(y)) return DMOE_ERR_ALIGN;
+  if (!aligned16(y_pad) || !aligned16(y) || !aligned16(y_scale)) return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
   return launch_rc(launch_combine(dims->T, dims->hidden, dims->top_k, y_pad, y_scale,
                                   map->dest_row, weights, y, static_cast<cudaStream_t>(stream),
@@ -485,7 +486,7 @@ int dmoe_bwd_scatter(const dmoe_dims *dims, const void *dx_pad, const float *dx_
   if (rc) return rc;
   if ((rc = check_map(map, false, dims))) return rc;
   if (!dx_pad || !dx_scale || !dw_part || !dx || !dweights) return DMOE_ERR_NULL;
-  if (!aligned16(dx_pad) || !aligned16(dx)) return DMOE_ERR_ALIGN;
+  if (!aligned16(dx_pad) || !aligned16(dx) || !aligned16(dx_scale)) return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
   return launch_rc(launch_bwd_scatter(dims->T, dims->hidden, dims->top_k, dx_pad, dx_scale,
                                       map->dest_row, dw_part, dglu_tiles(dims), dx, dweights,
@@ -500,7 +501,8 @@ int dmoe_bwd_dx(const dmoe_dims *dims, const void *da, const void *dbm, const vo
   if (rc) return rc;
   if ((rc = check_map(map, false))) return rc;
   if (!da || !dbm || !w1 || !w3 || !dx_pad || !dx_scale) return DMOE_ERR_NULL;
-  if (!aligned16(da) || !aligned16(dbm) || !aligned16(w1) || !aligned16(w3) || !aligned16(dx_pad))
+  if (!aligned16(da) || !aligned16(dbm) || !aligned16(w1) || !aligned16(w3) ||
+      !aligned16(dx_pad) || !aligned16(dx_scale))
     return DMOE_ERR_ALIGN;
   if ((rc = check_device())) return rc;
   return launch_rc(

@@ -103,6 +103,19 @@ __device__ __forceinline__ float f16_hi(uint32_t v) {
   return __half2float(__ushort_as_half((unsigned short)(v >> 16)));
 }
 
+// fp16 -> fp32 scaled by 2^-112, exactly, for every finite fp16 value (zero and subnormals
+// included): the fp16 sign goes to bit 31 and its exponent and mantissa bits are placed under
+// the fp32 exponent field unchanged, so an exponent field e reads as 2^(e-127) instead of
+// 2^(e-15).  Two integer operations instead of a conversion; a caller multiplies its
+// coefficient by 2^112 (exact while it stays finite) to get the value back.  Not for
+// infinities and NaNs (exponent field 31), which read as finite numbers.
+__device__ __forceinline__ float f16_lo_rebiased(uint32_t v) {
+  return __uint_as_float(((v & 0x7FFFu) << 13) | ((v & 0x8000u) << 16));
+}
+__device__ __forceinline__ float f16_hi_rebiased(uint32_t v) {
+  return __uint_as_float(((v >> 3) & 0x0FFFE000u) | (v & 0x80000000u));
+}
+
 // Vector reduction into global fp32 memory: [p .. p+3] += {a, b, c, d} (16-byte aligned).
 __device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),

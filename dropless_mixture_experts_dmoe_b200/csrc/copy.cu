@@ -131,6 +131,8 @@ __global__ void __launch_bounds__(kCopyThreads, 2) k_combine(int T, int h, int k
   const int vpr = h >> 3;                                      // 16-byte vectors per row
   const int nsc = dmoe_scale_stride(h);  // scales per row (padded to a multiple of 4)
   constexpr int kVecPerScale = DMOE_SCALE_COLS / 8;
+  static_assert(VPL % 2 == 0, "scales are loaded for pairs of vectors");
+  constexpr float kRebias = 5.192296858534828e33f;  // 2^112, see f16_lo_rebiased
   const int S = (vpr + kSliceVecs - 1) / kSliceVecs;  // 4 KB row slices per token
   const long long items = (long long)T * S;
   const long long nw = (long long)gridDim.x * kCopyWarps;
@@ -191,6 +193,7 @@ __global__ void __launch_bounds__(kCopyThreads, 2) k_combine(int T, int h, int k
         for (int s0 = 0; s0 < kk; s0 += SLOTS) {
           uint4 buf[SLOTS][VPL];
           float cf[SLOTS][VPL];
+          uint32_t slow = 0;  // F16S: (slot, vector) pairs that take the converting path
 #pragma unroll
           for (int ss = 0; ss < SLOTS; ++ss) {
             const int s = s0 + ss;
@@ -200,9 +203,30 @@ __global__ void __launch_bounds__(kCopyThreads, 2) k_combine(int T, int h, int k
 #pragma unroll
               for (int u = 0; u < VPL; ++u) {
                 const int v = v0 + u * 32 + lane;
-                if (v < ve) {
-                  buf[ss][u] = ld_nc_v4(rows + (size_t)r * vpr + v);
-                  cf[ss][u] = F16S ? ws * __ldg(scale + (size_t)r * nsc + v / kVecPerScale) : ws;
+                if (v < ve) buf[ss][u] = ld_nc_v4(rows + (size_t)r * vpr + v);
+                cf[ss][u] = ws;
+              }
+              if (F16S) {
+                // The scales of this lane's vectors: vector v lies in group v / 16, and v0 is a
+                // multiple of 64 vectors (4 groups), so one 16-byte load serves two vectors
+                // (lanes 0-15 take groups 0 and 2 of it, lanes 16-31 groups 1 and 3).  Scale
+                // rows are padded to a multiple of 4 groups, so the load stays in the row.
+#pragma unroll
+                for (int u2 = 0; u2 < VPL / 2; ++u2) {
+                  if (v0 + u2 * 64 < ve) {
+                    const float4 s4 = __ldg(reinterpret_cast<const float4 *>(
+                        scale + (size_t)r * nsc + v0 / kVecPerScale + 4 * u2));
+                    const float sa = (lane < 16) ? s4.x : s4.y, sb = (lane < 16) ? s4.z : s4.w;
+                    const float ca = ws * fabsf(sa), cb = ws * fabsf(sb);
+                    // exact rebias unless the coefficient overflows or the group is marked
+                    // non-finite (negative scale): those take the converting path
+                    const bool pa = sa > 0.0f && fabsf(ca * kRebias) <= 3.402823466e38f;
+                    const bool pb = sb > 0.0f && fabsf(cb * kRebias) <= 3.402823466e38f;
+                    cf[ss][2 * u2] = pa ? ca * kRebias : ca;
+                    cf[ss][2 * u2 + 1] = pb ? cb * kRebias : cb;
+                    slow |= (pa ? 0u : 1u) << (ss * VPL + 2 * u2);
+                    slow |= (pb ? 0u : 1u) << (ss * VPL + 2 * u2 + 1);
+                  }
                 }
               }
             }
@@ -216,12 +240,20 @@ __global__ void __launch_bounds__(kCopyThreads, 2) k_combine(int T, int h, int k
               for (int u = 0; u < VPL; ++u) {
                 const uint32_t *q = reinterpret_cast<const uint32_t *>(&buf[ss][u]);
                 const float c = cf[ss][u];
+                if (F16S && !((slow >> (ss * VPL + u)) & 1u)) {
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                  const float lo = F16S ? f16_lo(q[p]) : bf16_lo(q[p]);
-                  const float hi = F16S ? f16_hi(q[p]) : bf16_hi(q[p]);
-                  acc[u][2 * p] = fmaf(c, lo, acc[u][2 * p]);
-                  acc[u][2 * p + 1] = fmaf(c, hi, acc[u][2 * p + 1]);
+                  for (int p = 0; p < 4; ++p) {
+                    acc[u][2 * p] = fmaf(c, f16_lo_rebiased(q[p]), acc[u][2 * p]);
+                    acc[u][2 * p + 1] = fmaf(c, f16_hi_rebiased(q[p]), acc[u][2 * p + 1]);
+                  }
+                } else {
+#pragma unroll
+                  for (int p = 0; p < 4; ++p) {
+                    const float lo = F16S ? f16_lo(q[p]) : bf16_lo(q[p]);
+                    const float hi = F16S ? f16_hi(q[p]) : bf16_hi(q[p]);
+                    acc[u][2 * p] = fmaf(c, lo, acc[u][2 * p]);
+                    acc[u][2 * p + 1] = fmaf(c, hi, acc[u][2 * p + 1]);
+                  }
                 }
               }
             }

@@ -493,7 +493,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
   } else if (MODE == MODE_DOWN || MODE == MODE_DX) {
     // Y_pad / dX_pad in block floating point: per DMOE_SCALE_COLS columns of this thread's row,
     // the largest magnitude picks a power-of-two scale that puts it into [2^13, 2^14); the
-    // values go out as fp16 (11 significant bits) and 1/scale to p.part[row * nsc + chunk].
+    // values go out as fp16 (11 significant bits) and 1/scale to p.part[row * nsc + chunk]
+    // (-1 for a group holding an inf or NaN, whose values go out unscaled).
     const int n0 = tl.n * BN + half * kw;  // this warp's first column
     const int ncols = min(kw, p.h - n0);   // multiple of 64 (may be <= 0)
     if (ncols <= 0) return;
@@ -513,10 +514,13 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
         for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(__uint_as_float(v[i])));
       }
       int es = 13 - ((int)((__float_as_uint(m) >> 23) & 0xFFu) - 127);  // m * 2^es < 2^14
-      if (m == 0.0f || !(m <= 3.402823466e38f)) es = 0;  // zero, inf or NaN: unscaled
+      const bool finite = m <= 3.402823466e38f;
+      if (m == 0.0f || !finite) es = 0;  // zero, inf or NaN: unscaled
       es = min(max(es, -126), 126);
       const float sc = __uint_as_float((uint32_t)(127 + es) << 23);
-      srow[(n0 + c0) / DMOE_SCALE_COLS] = __uint_as_float((uint32_t)(127 - es) << 23);
+      // a group holding an inf or NaN is marked by the sign of its scale (magnitude 1)
+      srow[(n0 + c0) / DMOE_SCALE_COLS] =
+          __uint_as_float(((uint32_t)(127 - es) << 23) | (finite ? 0u : 0x80000000u));
 #pragma unroll 1
       for (int c = 0; c < cn; c += 64) {
         uint32_t v0[32], v1[32], w[32];

@@ -106,10 +106,11 @@ typedef struct {
 /* Block floating point of the padded expert outputs (Y_pad of dmoe_expert_down, dX_pad of
  * dmoe_bwd_dx): fp16 values [P_max, h] and fp32 scales [P_max, 4 * ceil(h / 512)] (ceil(h/128)
  * scales per row, the row padded to a multiple of 4); the value of row r, column c is
- * fp16[r][c] * scale[r][c / DMOE_SCALE_COLS].  Each scale is a
+ * fp16[r][c] * |scale[r][c / DMOE_SCALE_COLS]|.  Each scale is a
  * power of two that puts the largest magnitude of its 128 columns into [2^13, 2^14] (1 for an
- * all-zero or non-finite group), so every value keeps fp16's 11 significant bits at bf16's
- * size.  The k rows of a token are summed afterwards in fp32; rounding each to bf16 first (8
+ * all-zero group; -1, i.e. magnitude 1 with the sign bit set, for a group holding an inf or a
+ * NaN), so every value keeps fp16's 11 significant bits at bf16's size.  Scale pointers are
+ * 16-byte aligned like every other pointer.  The k rows of a token are summed afterwards in fp32; rounding each to bf16 first (8
  * bits) would put k roundings into every output element (measured at full size: 5.2-5.4 % of
  * the output's RMS at the largest element, against 3.1-3.3 % this way). */
 #define DMOE_SCALE_COLS 128

@@ -76,25 +76,67 @@ def test_weighted_scatter(w):
     assert (np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-5).all()
 
 
+def _add_round_f32(a: torch.Tensor, p: torch.Tensor) -> torch.Tensor:
+    """fp32 a + p rounded once to fp32 (round to nearest even), p a float64 tensor holding an
+    exact product: the double sum plus its exact remainder (two-sum), then a correction where
+    the double sum sits exactly halfway between two floats."""
+    a = a.double()
+    s = a + p
+    bb = s - a
+    err = (a - (s - bb)) + (p - bb)  # s + err == a + p exactly (finite values)
+    r = s.float()
+    inf = torch.tensor(float("inf"))
+    lo = torch.where(r.double() <= s, r, torch.nextafter(r, -inf))
+    hi = torch.nextafter(lo, inf)
+    fix = (s == (lo.double() + hi.double()) / 2) & torch.isfinite(err) & (err != 0)
+    return torch.where(fix & (err > 0), hi, torch.where(fix & (err < 0), lo, r))
+
+
+@pytest.mark.parametrize("kind", ["normal", "wide", "nonfinite"])
 @pytest.mark.parametrize("w", SHAPES[:3], ids=lambda w: w.describe())
-def test_weighted_scatter_block_floating_point(w):
+def test_weighted_scatter_block_floating_point(w, kind):
     """Rows in block floating point (fp16 values, one power-of-two scale per row and 128
     columns, the format of the down GEMM's output): y_t = bf16(sum_s fma(w_s * scale, value)),
-    bit for bit against the same fp32 sum in slot order."""
+    bit for bit against the same fp32 sum in slot order.  "wide" adds zeros, fp16 subnormals
+    and scales up to 2^24 (coefficients past 2^16 take the kernel's converting path);
+    "nonfinite" marks some groups with scale -1 and puts an inf or a NaN in them."""
     dims, bufs, g, x = _setup(w)
     P, h = bufs.P, w.hidden
     nsc = B.scale_stride(h)  # ceil(h/128) scales per row, padded to a multiple of 4
     gen = torch.Generator(device="cpu").manual_seed(5)
     vals = (torch.randn((P, h), generator=gen) * 4096).to(torch.float16)
     expo = torch.randint(-20, 5, (P, nsc), generator=gen).float()
+    if kind == "wide":
+        tiny = (torch.randn((P, h), generator=gen) * 2.0 ** -18).to(torch.float16)  # subnormal
+        pick = torch.randint(0, 4, (P, h), generator=gen)
+        vals = torch.where(pick == 0, tiny, vals)
+        vals = torch.where(pick == 1, torch.zeros_like(vals), vals)
+        expo = torch.randint(-30, 25, (P, nsc), generator=gen).float()
     scale = torch.pow(2.0, expo)
+    if kind == "nonfinite":
+        grp = torch.rand((P, nsc), generator=gen) < 0.05
+        grp[:, (h + 127) // 128:] = False
+        scale = torch.where(grp, torch.full_like(scale, -1.0), scale)
+        cols = grp.repeat_interleave(128, dim=1)[:, :h]
+        hit = cols & (torch.rand((P, h), generator=gen) < 0.02)
+        special = torch.where(torch.rand((P, h), generator=gen) < 0.5,
+                              torch.full_like(vals, float("inf")),
+                              torch.full_like(vals, float("nan")))
+        vals = torch.where(hit, special, vals)
     y = torch.empty_like(x)
     B.dmoe_padded_scatter(dims, vals.cuda(), scale.cuda(), bufs.map, bufs.map.weights, y)
     torch.cuda.synchronize()
-    full = vals.float() * scale.repeat_interleave(128, dim=1)[:, :h]  # exact in fp32
+    full = vals.double() * scale.abs().double().repeat_interleave(128, dim=1)[:, :h]  # exact
     wts = torch.from_numpy(g["weights"]).float()
     rows = torch.from_numpy(g["dest_row"].reshape(w.T, w.top_k)).long()
     acc = torch.zeros((w.T, h), dtype=torch.float32)
-    for s in range(w.top_k):  # w * (value * scale) is one rounding, as the kernel's fma
-        acc = (acc.double() + wts[:, s:s + 1].double() * full[rows[:, s]].double()).float()
-    assert torch.equal(y.cpu().view(torch.int16), acc.to(torch.bfloat16).view(torch.int16))
+    for s in range(w.top_k):  # w * |scale| * value (exact in double), one rounding: an fma
+        acc = _add_round_f32(acc, wts[:, s:s + 1].double() * full[rows[:, s]])
+    ref = acc.to(torch.bfloat16)
+    got = y.cpu()
+    nan_ref, nan_got = torch.isnan(ref), torch.isnan(got)
+    assert torch.equal(nan_ref, nan_got)
+    if kind == "nonfinite":
+        assert nan_ref.any() and torch.isinf(ref).any()
+    assert torch.equal(torch.where(nan_got, 0, got.view(torch.int16)),
+                       torch.where(nan_ref, 0, ref.view(torch.int16)))
