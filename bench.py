@@ -460,7 +460,7 @@ def run_ours(args, w):
             B.dmoe_expert_down(dims, hb, dev["w2"], bufs.map, yp, ys, st)
             i += 1
             mark(i)
-            B.dmoe_padded_scatter(dims, yp, ys, bufs.map, bufs.map.weights, y, st)
+            B.dmoe_padded_scatter(dims, yp, ys, bufs.map, None, y, st)  # rows weighted
             i += 1
             mark(i)
         if train:

@@ -386,7 +386,7 @@ int dmoe_expert_down(const dmoe_dims *dims, const void *h_in, const void *w2,
                      const dmoe_map *map, void *y_pad, float *y_scale, void *stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
-  if ((rc = check_map(map, false))) return rc;
+  if ((rc = check_map(map, true))) return rc;  // the rows go out weighted
   if (!h_in || !w2 || !y_pad || !y_scale) return DMOE_ERR_NULL;
   if (!aligned16(h_in) || !aligned16(w2) || !aligned16(y_pad) || !aligned16(y_scale))
     return DMOE_ERR_ALIGN;
@@ -460,7 +460,7 @@ int dmoe_forward(const dmoe_dims *dims, const void *x, const void *w1, const voi
   if ((rc = dmoe_expert_glu(dims, xpad, w1, w3, map, hbuf, abuf, bbuf, stream))) return rc;
   if (fused_combine(dims)) return dmoe_expert_down_combine(dims, hbuf, w2, map, y, yacc, stream);
   if ((rc = dmoe_expert_down(dims, hbuf, w2, map, ypad, yscale, stream))) return rc;
-  return dmoe_padded_scatter(dims, ypad, yscale, map, map->weights, y, stream);
+  return dmoe_padded_scatter(dims, ypad, yscale, map, nullptr, y, stream);  // rows weighted
 }
 
 int dmoe_bwd_dglu(const dmoe_dims *dims, const void *dy_pad, const void *w2, const void *a_saved,

@@ -103,17 +103,21 @@ __device__ __forceinline__ float f16_hi(uint32_t v) {
   return __half2float(__ushort_as_half((unsigned short)(v >> 16)));
 }
 
-// fp16 -> fp32 scaled by 2^-112, exactly, for every finite fp16 value (zero and subnormals
-// included): the fp16 sign goes to bit 31 and its exponent and mantissa bits are placed under
-// the fp32 exponent field unchanged, so an exponent field e reads as 2^(e-127) instead of
-// 2^(e-15).  Two integer operations instead of a conversion; a caller multiplies its
-// coefficient by 2^112 (exact while it stays finite) to get the value back.  Not for
-// infinities and NaNs (exponent field 31), which read as finite numbers.
-__device__ __forceinline__ float f16_lo_rebiased(uint32_t v) {
-  return __uint_as_float(((v & 0x7FFFu) << 13) | ((v & 0x8000u) << 16));
+// acc0 += lo(v) * s, acc1 += hi(v) * s for the two fp16 values packed in v and an fp16
+// coefficient s, with fp32 accumulation: the mixed-precision fma (f16 x f16 + f32 -> f32, the
+// product exact, one rounding), no separate conversion.
+__device__ __forceinline__ void fma2_f16_f32(float &acc0, float &acc1, uint32_t v, uint16_t s) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "fma.rn.f32.f16 %0, l, %3, %0;\n\tfma.rn.f32.f16 %1, h, %3, %1;\n\t}"
+      : "+f"(acc0), "+f"(acc1)
+      : "r"(v), "h"(s));
 }
-__device__ __forceinline__ float f16_hi_rebiased(uint32_t v) {
-  return __uint_as_float(((v >> 3) & 0x0FFFE000u) | (v & 0x80000000u));
+
+// Whether a block-floating-point scale takes the fp16 path: a positive power of two that fp16
+// represents exactly, 2^-24 ... 2^15 (fp32 exponent field 103 ... 142, zero mantissa).
+__device__ __forceinline__ bool scale_fits_f16(float s) {
+  const uint32_t b = __float_as_uint(s);
+  return (b & 0x807FFFFFu) == 0u && (b >> 23) - 103u <= 39u;
 }
 
 // Vector reduction into global fp32 memory: [p .. p+3] += {a, b, c, d} (16-byte aligned).

@@ -132,7 +132,6 @@ __global__ void __launch_bounds__(kCopyThreads, 2) k_combine(int T, int h, int k
   const int nsc = dmoe_scale_stride(h);  // scales per row (padded to a multiple of 4)
   constexpr int kVecPerScale = DMOE_SCALE_COLS / 8;
   static_assert(VPL % 2 == 0, "scales are loaded for pairs of vectors");
-  constexpr float kRebias = 5.192296858534828e33f;  // 2^112, see f16_lo_rebiased
   const int S = (vpr + kSliceVecs - 1) / kSliceVecs;  // 4 KB row slices per token
   const long long items = (long long)T * S;
   const long long nw = (long long)gridDim.x * kCopyWarps;
@@ -211,19 +210,21 @@ __global__ void __launch_bounds__(kCopyThreads, 2) k_combine(int T, int h, int k
                 // multiple of 64 vectors (4 groups), so one 16-byte load serves two vectors
                 // (lanes 0-15 take groups 0 and 2 of it, lanes 16-31 groups 1 and 3).  Scale
                 // rows are padded to a multiple of 4 groups, so the load stays in the row.
+                // Unweighted rows whose scale fp16 holds exactly take the fp16 path (the
+                // coefficient kept as fp16 bits); the others are converted (coefficient
+                // w * |scale| in fp32).
 #pragma unroll
                 for (int u2 = 0; u2 < VPL / 2; ++u2) {
                   if (v0 + u2 * 64 < ve) {
                     const float4 s4 = __ldg(reinterpret_cast<const float4 *>(
                         scale + (size_t)r * nsc + v0 / kVecPerScale + 4 * u2));
                     const float sa = (lane < 16) ? s4.x : s4.y, sb = (lane < 16) ? s4.z : s4.w;
-                    const float ca = ws * fabsf(sa), cb = ws * fabsf(sb);
-                    // exact rebias unless the coefficient overflows or the group is marked
-                    // non-finite (negative scale): those take the converting path
-                    const bool pa = sa > 0.0f && fabsf(ca * kRebias) <= 3.402823466e38f;
-                    const bool pb = sb > 0.0f && fabsf(cb * kRebias) <= 3.402823466e38f;
-                    cf[ss][2 * u2] = pa ? ca * kRebias : ca;
-                    cf[ss][2 * u2 + 1] = pb ? cb * kRebias : cb;
+                    const bool pa = !weights && scale_fits_f16(sa);
+                    const bool pb = !weights && scale_fits_f16(sb);
+                    cf[ss][2 * u2] = pa ? __uint_as_float(__half_as_ushort(__float2half_rn(sa)))
+                                        : ws * fabsf(sa);
+                    cf[ss][2 * u2 + 1] =
+                        pb ? __uint_as_float(__half_as_ushort(__float2half_rn(sb))) : ws * fabsf(sb);
                     slow |= (pa ? 0u : 1u) << (ss * VPL + 2 * u2);
                     slow |= (pb ? 0u : 1u) << (ss * VPL + 2 * u2 + 1);
                   }
@@ -241,11 +242,10 @@ __global__ void __launch_bounds__(kCopyThreads, 2) k_combine(int T, int h, int k
                 const uint32_t *q = reinterpret_cast<const uint32_t *>(&buf[ss][u]);
                 const float c = cf[ss][u];
                 if (F16S && !((slow >> (ss * VPL + u)) & 1u)) {
+                  const uint16_t c16 = (uint16_t)__float_as_uint(c);
 #pragma unroll
-                  for (int p = 0; p < 4; ++p) {
-                    acc[u][2 * p] = fmaf(c, f16_lo_rebiased(q[p]), acc[u][2 * p]);
-                    acc[u][2 * p + 1] = fmaf(c, f16_hi_rebiased(q[p]), acc[u][2 * p + 1]);
-                  }
+                  for (int p = 0; p < 4; ++p)
+                    fma2_f16_f32(acc[u][2 * p], acc[u][2 * p + 1], q[p], c16);
                 } else {
 #pragma unroll
                   for (int p = 0; p < 4; ++p) {

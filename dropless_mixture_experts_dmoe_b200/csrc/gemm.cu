@@ -298,7 +298,7 @@ __device__ __forceinline__ void gather_rows(const GemmParams &p, const Tile &tl,
   }
 }
 
-// DGLU: routing weight of padded row `row` of expert e (0 for a padding row).
+// DOWN, DGLU: routing weight of padded row `row` of expert e (0 for a padding row).
 __device__ __forceinline__ float row_weight(const GemmParams &p, int e, int row) {
   const int pstart = (e > 0) ? p.padded_bins[e - 1] : 0;
   const int bstart = (e > 0) ? p.bins[e - 1] : 0;
@@ -491,16 +491,22 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
       }
     }
   } else if (MODE == MODE_DOWN || MODE == MODE_DX) {
-    // Y_pad / dX_pad in block floating point: per DMOE_SCALE_COLS columns of this thread's row,
-    // the largest magnitude picks a power-of-two scale that puts it into [2^13, 2^14); the
-    // values go out as fp16 (11 significant bits) and 1/scale to p.part[row * nsc + chunk]
-    // (-1 for a group holding an inf or NaN, whose values go out unscaled).
+    // Y_pad / dX_pad in block floating point.  DOWN first weights the row by its routing
+    // weight (0 for a padding row), so the combine sums unweighted rows.  Per DMOE_SCALE_COLS
+    // columns of this thread's row, the largest magnitude m picks a power-of-two scale that
+    // puts it into [2^13, 2^14) -- for m < 2^-11 the scale stops at 2^24 (fp16's range of
+    // powers of two), which still leaves the group's largest value a normal fp16 down to
+    // m = 2^-38.  The values go out as fp16 (11 significant bits) and 1/scale to
+    // p.part[row * nsc + chunk], its sign set when fp16 cannot hold 1/scale (m < 2^-38 or
+    // m >= 2^29) or when the group holds an inf or NaN (values unscaled, 1/scale = -1).
     const int n0 = tl.n * BN + half * kw;  // this warp's first column
     const int ncols = min(kw, p.h - n0);   // multiple of 64 (may be <= 0)
     if (ncols <= 0) return;
     tb += (uint32_t)(half * kw);
     const int nsc = dmoe_scale_stride(p.h);
-    float *srow = p.part + (size_t)(y0 + lane) * nsc;
+    const int grow = y0 + lane;
+    const float wr = (MODE == MODE_DOWN) ? row_weight(p, tl.e, grow) : 1.0f;
+    float *srow = p.part + (size_t)grow * nsc;
 #pragma unroll 1
     for (int c0 = 0; c0 < ncols; c0 += DMOE_SCALE_COLS) {
       const int cn = min(DMOE_SCALE_COLS, ncols - c0);
@@ -513,14 +519,17 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
 #pragma unroll
         for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(__uint_as_float(v[i])));
       }
+      m *= fabsf(wr);  // the largest weighted magnitude (rounding is monotone)
       int es = 13 - ((int)((__float_as_uint(m) >> 23) & 0xFFu) - 127);  // m * 2^es < 2^14
       const bool finite = m <= 3.402823466e38f;
       if (m == 0.0f || !finite) es = 0;  // zero, inf or NaN: unscaled
+      if (es > 24 && es <= 51) es = 24;  // see above
       es = min(max(es, -126), 126);
+      const bool fits = finite && es >= -15 && es <= 24;
       const float sc = __uint_as_float((uint32_t)(127 + es) << 23);
-      // a group holding an inf or NaN is marked by the sign of its scale (magnitude 1)
+      const float k = wr * sc;  // weight and scale in one exact product
       srow[(n0 + c0) / DMOE_SCALE_COLS] =
-          __uint_as_float(((uint32_t)(127 - es) << 23) | (finite ? 0u : 0x80000000u));
+          __uint_as_float(((uint32_t)(127 - es) << 23) | (fits ? 0u : 0x80000000u));
 #pragma unroll 1
       for (int c = 0; c < cn; c += 64) {
         uint32_t v0[32], v1[32], w[32];
@@ -529,8 +538,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
         tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          w[i] = pack_f16x2(__uint_as_float(v0[2 * i]) * sc, __uint_as_float(v0[2 * i + 1]) * sc);
-          w[16 + i] = pack_f16x2(__uint_as_float(v1[2 * i]) * sc, __uint_as_float(v1[2 * i + 1]) * sc);
+          w[i] = pack_f16x2(__uint_as_float(v0[2 * i]) * k, __uint_as_float(v0[2 * i + 1]) * k);
+          w[16 + i] = pack_f16x2(__uint_as_float(v1[2 * i]) * k, __uint_as_float(v1[2 * i + 1]) * k);
         }
         st.emit(&p.tmo[0], w, n0 + c0 + c, y0);
       }
@@ -1176,6 +1185,7 @@ cudaError_t launch_down_gemm(const GemmProblem &g, const void *h_in, const void 
                              make_tmap_chunked(&p.tm[1], w2, (uint64_t)g.E * g.h, g.f, BN / 2));
   if (!ok || !make_tmap(&p.tmo[0], y_pad, P, g.h, 32)) return cudaErrorInvalidValue;  // fp16
   p.tm[2] = p.tm[3] = p.tm[4] = p.tm[0];
+  p.weights = g.weights;  // the rows go out weighted
   p.part = y_scale;
   p.n_tiles = (g.h + BN - 1) / BN;
   p.group = raster_units(g.f);

@@ -315,7 +315,22 @@ __global__ void __launch_bounds__(kMapThreads) k_given_hist(const int32_t *__res
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * kMapTokTile;
   int flags = 0;
-  for (int tt = warp; tt < kMapTokTile; tt += kMapWarps) {
+  if (k == 1) {  // one entry per token (the rounded routing's entry list): 32 tokens a warp
+    for (int tt = warp * 32; tt < kMapTokTile; tt += kMapWarps * 32) {
+      const int t = t0 + tt + lane;
+      int e = -1;
+      if (t < T) {
+        e = top[t];
+        if (e < -1 || e >= E || (e == -1 && !absent_ok)) {
+          flags |= DMOE_STATUS_EXPERT_OUT_OF_RANGE;
+          e = -1;
+        }
+      }
+      const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+      if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[e], __popc(peers));
+    }
+  }
+  for (int tt = warp; k > 1 && tt < kMapTokTile; tt += kMapWarps) {
     const int t = t0 + tt;
     if (t >= T) break;
     int e = -1 - lane;  // distinct sentinels for lanes >= k

@@ -32,7 +32,7 @@ namespace dmoe {
 namespace {
 
 constexpr int kSelThreads = 512;
-constexpr int kApplyThreads = 256;
+constexpr int kApplyThreads = 512;
 constexpr int kApplyWarps = kApplyThreads / 32;
 
 // Rank image of a bf16 logit: order-preserving 16-bit value (-0 taken as +0), NaN lowest (0).
@@ -42,6 +42,13 @@ __device__ __forceinline__ uint32_t rank_image(uint16_t b) {
   return (b & 0x8000u) ? (uint32_t)(~b & 0xFFFFu) : (uint32_t)(b | 0x8000u);
 }
 
+
+// hist[key] += 1 for every lane with `on` (all 32 lanes call it): one shared-memory atomic per
+// distinct key in the warp.
+__device__ __forceinline__ void warp_hist_add(int *hist, bool on, uint32_t key, int lane) {
+  const unsigned peers = __match_any_sync(0xFFFFFFFFu, on ? key : 0x100u + (uint32_t)lane);
+  if (on && lane == __ffs(peers) - 1) atomicAdd(&hist[key], __popc(peers));
+}
 
 // Block-wide sum of one int per thread (kSelThreads threads).
 __device__ __forceinline__ int block_sum(int v, int *red) {
@@ -122,11 +129,18 @@ __global__ void __launch_bounds__(kSelThreads) k_round_select(const int32_t *__r
     atomicOr(&routed_bits[t >> 5], 1u << (t & 31));
   }
   __syncthreads();
-  // pass A: histogram of the candidates' high bytes
-  for (int t = threadIdx.x; t < T; t += kSelThreads) {
-    const bool rt = (routed_bits[t >> 5] >> (t & 31)) & 1u;
-    const uint32_t v = col[t];
-    if (rt != up) atomicAdd(&hist[v >> 8], 1);
+  const int lane = threadIdx.x & 31;
+  // pass A: histogram of the candidates' high bytes (few distinct values: one atomic per
+  // distinct value and warp)
+  for (int tb = threadIdx.x - lane; tb < T; tb += kSelThreads) {
+    const int t = tb + lane;
+    bool cand = false;
+    uint32_t v = 0;
+    if (t < T) {
+      cand = (((routed_bits[t >> 5] >> (t & 31)) & 1u) != 0) != up;
+      v = col[t];
+    }
+    warp_hist_add(hist, cand, v >> 8, lane);
   }
   __syncthreads();
   // the high byte H holding the m-th candidate on the chosen side (from the top for round
@@ -150,10 +164,15 @@ __global__ void __launch_bounds__(kSelThreads) k_round_select(const int32_t *__r
   for (int i = threadIdx.x; i < 256; i += kSelThreads) hist[i] = 0;
   __syncthreads();
   // pass B: low bytes of the candidates whose high byte is H
-  for (int t = threadIdx.x; t < T; t += kSelThreads) {
-    const bool rt = (routed_bits[t >> 5] >> (t & 31)) & 1u;
-    const uint32_t v = col[t];
-    if (rt != up && (v >> 8) == H) atomicAdd(&hist[v & 0xFFu], 1);
+  for (int tb = threadIdx.x - lane; tb < T; tb += kSelThreads) {
+    const int t = tb + lane;
+    bool cand = false;
+    uint32_t v = 0;
+    if (t < T) {
+      v = col[t];
+      cand = ((((routed_bits[t >> 5] >> (t & 31)) & 1u) != 0) != up) && (v >> 8) == H;
+    }
+    warp_hist_add(hist, cand, v & 0xFFu, lane);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -195,7 +214,7 @@ __global__ void __launch_bounds__(kSelThreads) k_round_select(const int32_t *__r
     }
     // inclusive prefix count of ties over the block, in token order
     const unsigned bal = __ballot_sync(0xFFFFFFFFu, tie);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int warp = threadIdx.x >> 5;
     if (lane == 0) red[warp] = __popc(bal);
     __syncthreads();
     int before = seen;
@@ -227,13 +246,18 @@ __global__ void __launch_bounds__(kApplyThreads) k_round_apply(
     int32_t *__restrict__ tok_count, int32_t *__restrict__ tile_sum,
     const int32_t *__restrict__ tile_off, int32_t *__restrict__ entry_offsets,
     int32_t *__restrict__ out_expert, float *__restrict__ out_weight, long long cap) {
-  extern __shared__ uint32_t sm_bits[];  // [kApplyWarps][ceil(E/32)] routed-expert bitmaps
+  // dynamic shared memory: the thresholds param[3E], then [kApplyWarps][ceil(E/32)]
+  // routed-expert bitmaps
+  extern __shared__ int32_t sm_apply[];
   __shared__ int s_cnt[kMapTokTile];
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ew = (E + 31) / 32;
-  uint32_t *bits = sm_bits + warp * ew;
+  int32_t *sp = sm_apply;
+  uint32_t *bits = reinterpret_cast<uint32_t *>(sm_apply + 3 * E) + warp * ew;
+  for (int i = threadIdx.x; i < 3 * E; i += kApplyThreads) sp[i] = param[i];
+  __syncthreads();
   const int t_first = blockIdx.x * kMapTokTile;
   if (WRITE) {  // offsets of this tile's tokens: an exclusive scan of their counts
     if (threadIdx.x < kMapTokTile) {
@@ -273,10 +297,10 @@ __global__ void __launch_bounds__(kApplyThreads) k_round_apply(
       w_s = weights[(size_t)t * k + lane];
       atomicOr(&bits[e_s >> 5], 1u << (e_s & 31));
       keep = true;
-      if (param[3 * e_s] == 1) {  // round down: dropped below the threshold
+      if (sp[3 * e_s] == 1) {  // round down: dropped below the threshold
         const uint32_t v = rank_image(row[e_s]);
-        const uint32_t vs = (uint32_t)param[3 * e_s + 1];
-        keep = !(v < vs || (v == vs && t >= param[3 * e_s + 2]));
+        const uint32_t vs = (uint32_t)sp[3 * e_s + 1];
+        keep = !(v < vs || (v == vs && t >= sp[3 * e_s + 2]));
       }
     }
     __syncwarp();
@@ -296,10 +320,10 @@ __global__ void __launch_bounds__(kApplyThreads) k_round_apply(
     for (int e0b = 0; e0b < E; e0b += 32) {
       const int e = e0b + lane;
       bool add = false;
-      if (e < E && param[3 * e] == 2 && !((bits[e >> 5] >> (e & 31)) & 1u)) {
+      if (e < E && sp[3 * e] == 2 && !((bits[e >> 5] >> (e & 31)) & 1u)) {
         const uint32_t v = rank_image(row[e]);
-        const uint32_t vs = (uint32_t)param[3 * e + 1];
-        add = v > vs || (v == vs && t <= param[3 * e + 2]);
+        const uint32_t vs = (uint32_t)sp[3 * e + 1];
+        add = v > vs || (v == vs && t <= sp[3 * e + 2]);
       }
       const unsigned am = __ballot_sync(0xFFFFFFFFu, add);
       if (WRITE && add) {
@@ -398,7 +422,7 @@ cudaError_t launch_round_tokens(const uint16_t *logits, const int32_t *top, cons
                         k, (const uint16_t *)s.img, s.param)) != cudaSuccess)
     return err;
   const int tiles = map_tiles(T);
-  const size_t ap_smem = sizeof(uint32_t) * (size_t)kApplyWarps * ((E + 31) / 32);
+  const size_t ap_smem = sizeof(int32_t) * (3 * (size_t)E + (size_t)kApplyWarps * ((E + 31) / 32));
   if ((err = launch_pdl(k_round_apply<false>, tiles, kApplyThreads, ap_smem, st, logits, top,
                         weights, s.param, T, E, k, s.tok_count, s.tile_sum, s.tile_off,
                         entry_offsets, out_expert, out_weight, cap)) != cudaSuccess)

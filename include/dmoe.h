@@ -106,13 +106,17 @@ typedef struct {
 /* Block floating point of the padded expert outputs (Y_pad of dmoe_expert_down, dX_pad of
  * dmoe_bwd_dx): fp16 values [P_max, h] and fp32 scales [P_max, 4 * ceil(h / 512)] (ceil(h/128)
  * scales per row, the row padded to a multiple of 4); the value of row r, column c is
- * fp16[r][c] * |scale[r][c / DMOE_SCALE_COLS]|.  Each scale is a
- * power of two that puts the largest magnitude of its 128 columns into [2^13, 2^14] (1 for an
- * all-zero group; -1, i.e. magnitude 1 with the sign bit set, for a group holding an inf or a
- * NaN), so every value keeps fp16's 11 significant bits at bf16's size.  Scale pointers are
- * 16-byte aligned like every other pointer.  The k rows of a token are summed afterwards in fp32; rounding each to bf16 first (8
- * bits) would put k roundings into every output element (measured at full size: 5.2-5.4 % of
- * the output's RMS at the largest element, against 3.1-3.3 % this way). */
+ * fp16[r][c] * |scale[r][c / DMOE_SCALE_COLS]|.  Each scale is a power of two chosen from the
+ * largest magnitude m of its 128 columns: the one that puts m into [2^13, 2^14), except that
+ * for m < 2^-11 it stops at 2^24 (the largest power of two fp16 holds; m then still lands on a
+ * normal fp16 down to m = 2^-38), and 1 for an all-zero group.  The sign bit of a scale is set
+ * when fp16 cannot hold the scale itself (m < 2^-38 or m >= 2^29) and for a group holding an
+ * inf or NaN (magnitude 1, values unscaled); the combine sums the other groups with the
+ * mixed-precision fma (fp16 value times fp16 scale into fp32) and converts these.  Every value
+ * keeps fp16's 11 significant bits at bf16's size.  Scale pointers are 16-byte aligned like
+ * every other pointer.  The k rows of a token are summed afterwards in fp32; rounding each to
+ * bf16 first (8 bits) would put k roundings into every output element (measured at full
+ * size: 5.2-5.4 % of the output's RMS at the largest element, against 3.1-3.3 % this way). */
 #define DMOE_SCALE_COLS 128
 
 /* Routing variant: tile-aware token rounding (SonicMoE abstract: the routing is rounded so that
@@ -314,8 +318,10 @@ DMOE_API int dmoe_expert_glu_gather(const dmoe_dims *dims, const void *x, const 
                                     const void *w3, const dmoe_map *map, void *h_out, void *a_out,
                                     void *b_out, void *stream);
 
-/* Down GEMM: Y_pad[b] = H[b] W2_e^T for every block b < num_blocks, fp32 accumulation,
- * stored in block floating point (see DMOE_SCALE_COLS).
+/* Down GEMM: Y_pad[b] = w * (H[b] W2_e^T) for every block b < num_blocks, fp32
+ * accumulation, each row times the routing weight w of its entry (map->weights; 0 for a
+ * padding row: the walkthrough's section 4.2 scatter weight, applied here so that the combine
+ * sums unweighted rows), stored in block floating point (see DMOE_SCALE_COLS).
  * h_in [P_max,f] bf16 -> y_pad [P_max,h] fp16, y_scale [P_max, 4*ceil(h/512)] fp32. */
 DMOE_API int dmoe_expert_down(const dmoe_dims *dims, const void *h_in, const void *w2,
                               const dmoe_map *map, void *y_pad, float *y_scale, void *stream);
@@ -329,10 +335,11 @@ DMOE_API int dmoe_expert_down_combine(const dmoe_dims *dims, const void *h_in, c
 
 /* Weighted padded_scatter (walkthrough section 4.2, B_TO_A direction, times the routing
  * weight): y_t = bf16(sum_{s=0..k-1} w_ts * Y_pad[dest_row[t*k+s]]), summed in fp32 in
- * slot order (each entry one fused multiply-add), no atomics.  weights == NULL means w = 1
- * (the backward's gather gradient, dx_t = sum_s dX_pad[dest_row[t*k+s]]).  Row format:
- * y_scale == NULL: y_pad [P_max,h] bf16; otherwise block floating point as written by
- * dmoe_expert_down (y_pad fp16, y_scale [P_max, 4*ceil(h/512)]).  -> y [T,h] bf16. */
+ * slot order (each entry one fused multiply-add), no atomics.  weights == NULL means w = 1:
+ * the rows of dmoe_expert_down, which already carry their routing weight, and the backward's
+ * gather gradient, dx_t = sum_s dX_pad[dest_row[t*k+s]].  Row format: y_scale == NULL:
+ * y_pad [P_max,h] bf16; otherwise block floating point (see DMOE_SCALE_COLS: y_pad fp16,
+ * y_scale [P_max, 4*ceil(h/512)]).  -> y [T,h] bf16. */
 DMOE_API int dmoe_padded_scatter(const dmoe_dims *dims, const void *y_pad, const float *y_scale,
                                  const dmoe_map *map, const float *weights, void *y,
                                  void *stream);

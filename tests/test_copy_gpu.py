@@ -92,14 +92,16 @@ def _add_round_f32(a: torch.Tensor, p: torch.Tensor) -> torch.Tensor:
     return torch.where(fix & (err > 0), hi, torch.where(fix & (err < 0), lo, r))
 
 
+@pytest.mark.parametrize("weighted", [False, True], ids=["unweighted", "weighted"])
 @pytest.mark.parametrize("kind", ["normal", "wide", "nonfinite"])
 @pytest.mark.parametrize("w", SHAPES[:3], ids=lambda w: w.describe())
-def test_weighted_scatter_block_floating_point(w, kind):
+def test_weighted_scatter_block_floating_point(w, kind, weighted):
     """Rows in block floating point (fp16 values, one power-of-two scale per row and 128
-    columns, the format of the down GEMM's output): y_t = bf16(sum_s fma(w_s * scale, value)),
-    bit for bit against the same fp32 sum in slot order.  "wide" adds zeros, fp16 subnormals
-    and scales up to 2^24 (coefficients past 2^16 take the kernel's converting path);
-    "nonfinite" marks some groups with scale -1 and puts an inf or a NaN in them."""
+    columns, the format of the down and dX GEMMs' output): y_t = bf16(sum_s fma(w_s * |scale|,
+    value)), bit for bit against the same fp32 sum in slot order.  Unweighted rows with a scale
+    that fp16 holds take the kernel's mixed-precision path, the others its converting path.
+    "wide" adds zeros, fp16 subnormals and scales from 2^-30 to 2^24 (both paths); "nonfinite"
+    marks some groups with scale -1 and puts an inf or a NaN in them."""
     dims, bufs, g, x = _setup(w)
     P, h = bufs.P, w.hidden
     nsc = B.scale_stride(h)  # ceil(h/128) scales per row, padded to a multiple of 4
@@ -124,10 +126,11 @@ def test_weighted_scatter_block_floating_point(w, kind):
                               torch.full_like(vals, float("nan")))
         vals = torch.where(hit, special, vals)
     y = torch.empty_like(x)
-    B.dmoe_padded_scatter(dims, vals.cuda(), scale.cuda(), bufs.map, bufs.map.weights, y)
+    B.dmoe_padded_scatter(dims, vals.cuda(), scale.cuda(), bufs.map,
+                          bufs.map.weights if weighted else None, y)
     torch.cuda.synchronize()
     full = vals.double() * scale.abs().double().repeat_interleave(128, dim=1)[:, :h]  # exact
-    wts = torch.from_numpy(g["weights"]).float()
+    wts = torch.from_numpy(g["weights"]).float() if weighted else torch.ones(w.T, w.top_k)
     rows = torch.from_numpy(g["dest_row"].reshape(w.T, w.top_k)).long()
     acc = torch.zeros((w.T, h), dtype=torch.float32)
     for s in range(w.top_k):  # w * |scale| * value (exact in double), one rounding: an fma

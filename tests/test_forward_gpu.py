@@ -55,9 +55,12 @@ def test_gemm_intermediates(w):
     A = bufs.view("a")[: nb * 128].double().cpu()
     Bm = bufs.view("bm")[: nb * 128].double().cpu()
     H = bufs.view("h")[: nb * 128].double().cpu()
-    # Y_pad is block floating point: fp16 values times one power-of-two scale per 128 columns
-    ys = bufs.view("y_scale")[: nb * 128].double().cpu().repeat_interleave(128, dim=1)
+    # Y_pad is block floating point: fp16 values times one power-of-two scale per 128 columns,
+    # each row weighted by its routing weight (0 for a padding row)
+    ys = bufs.view("y_scale")[: nb * 128].double().cpu().abs().repeat_interleave(128, dim=1)
     Yp = bufs.view("y_pad")[: nb * 128].double().cpu() * ys[:, : w.hidden]
+    wrow = torch.zeros(nb * 128, dtype=torch.float64)
+    wrow[bufs.map.dest_row.cpu().long()] = bufs.map.weights.cpu().double().reshape(-1)
     W1 = inp["w1"].double()
     W3 = inp["w3"].double()
     W2 = inp["w2"].double()
@@ -70,8 +73,8 @@ def test_gemm_intermediates(w):
         assert torch.allclose(A[rows], a_ref, rtol=1e-2, atol=1e-2), b
         assert torch.allclose(Bm[rows], b_ref, rtol=1e-2, atol=1e-2), b
         assert torch.allclose(H[rows], h_ref, rtol=2e-2, atol=2e-3), b
-        y_ref = H[rows] @ W2[e].T
-        assert torch.allclose(Yp[rows], y_ref, rtol=1e-2, atol=1e-3), b
+        y_ref = wrow[rows, None] * (H[rows] @ W2[e].T)
+        assert torch.allclose(Yp[rows], y_ref, rtol=1e-2, atol=1e-4), b
 
 
 @pytest.mark.parametrize("num", [2, 3, 4, 5])
