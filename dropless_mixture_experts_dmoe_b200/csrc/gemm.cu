@@ -430,8 +430,8 @@ __device__ __forceinline__ void pack_bf16_row(const uint32_t (&lo)[32], const ui
 // Epilogue of one tile for the warp owning TMEM sub-partition `sub` (rows sub*32 .. +31 of
 // this CTA's 128 rows); tb = TMEM address of the warp's lanes at accumulator column 0.
 // Work of a tile's epilogue that does not depend on the accumulator, done before waiting for
-// it: DGLU looks up the routing weight of this thread's row (a chain of dependent loads) and
-// starts pulling the row's saved A and Bm columns of the tile into L2.
+// it: DOWN and DGLU look up the routing weight of this thread's row (a chain of dependent
+// loads), and DGLU starts pulling the row's saved A and Bm columns of the tile into L2.
 template <int MODE, int EPI>
 __device__ __forceinline__ float epilogue_prologue(const GemmParams &p, const Tile &tl, int sub,
                                                    int half, int lane) {
@@ -444,6 +444,8 @@ __device__ __forceinline__ float epilogue_prologue(const GemmParams &p, const Ti
       for (int c = 0; c < ncols; c += 64) prefetch_l2(p.in0 + (size_t)grow * p.h + n0 + c);
     return 0.0f;
   }
+  if (MODE == MODE_DOWN && !tl.dummy)  // the row's routing weight, ahead of the accumulator
+    return row_weight(p, tl.e, tl.row0 + sub * 32 + lane);
   if (MODE != MODE_DGLU || tl.dummy) return 0.0f;
   const int grow = tl.row0 + sub * 32 + lane;
   const int n0 = tl.n * BN;
@@ -505,21 +507,26 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
     tb += (uint32_t)(half * kw);
     const int nsc = dmoe_scale_stride(p.h);
     const int grow = y0 + lane;
-    const float wr = (MODE == MODE_DOWN) ? row_weight(p, tl.e, grow) : 1.0f;
+    const float wrow = (MODE == MODE_DOWN) ? wr : 1.0f;  // DOWN: from epilogue_prologue
     float *srow = p.part + (size_t)grow * nsc;
+    // one pass per group: its 128 accumulator columns in registers (the last group of a
+    // 64-column remainder reads 64 columns past it, inside this CTA's TMEM allocation, and
+    // leaves them out), one wait, then the maximum, the scale and the conversion
+    static_assert(DMOE_SCALE_COLS == 128, "four 32-column loads per group");
 #pragma unroll 1
     for (int c0 = 0; c0 < ncols; c0 += DMOE_SCALE_COLS) {
-      const int cn = min(DMOE_SCALE_COLS, ncols - c0);
-      float m = 0.0f;
-#pragma unroll 1
-      for (int c = 0; c < cn; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(tb + c0 + c, v);
-        tmem_ld_wait();
+      const bool full = ncols - c0 >= DMOE_SCALE_COLS;
+      uint32_t v[4][32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(__uint_as_float(v[i])));
-      }
-      m *= fabsf(wr);  // the largest weighted magnitude (rounding is monotone)
+      for (int j = 0; j < 4; ++j) tmem_ld32(tb + c0 + 32 * j, v[j]);
+      tmem_ld_wait();
+      float m = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (j < 2 || full) m = fmaxf(m, fabsf(__uint_as_float(v[j][i])));
+      m *= fabsf(wrow);  // the largest weighted magnitude (rounding is monotone)
       int es = 13 - ((int)((__float_as_uint(m) >> 23) & 0xFFu) - 127);  // m * 2^es < 2^14
       const bool finite = m <= 3.402823466e38f;
       if (m == 0.0f || !finite) es = 0;  // zero, inf or NaN: unscaled
@@ -527,21 +534,21 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
       es = min(max(es, -126), 126);
       const bool fits = finite && es >= -15 && es <= 24;
       const float sc = __uint_as_float((uint32_t)(127 + es) << 23);
-      const float k = wr * sc;  // weight and scale in one exact product
+      const float k = wrow * sc;  // weight and scale in one exact product
       srow[(n0 + c0) / DMOE_SCALE_COLS] =
           __uint_as_float(((uint32_t)(127 - es) << 23) | (fits ? 0u : 0x80000000u));
-#pragma unroll 1
-      for (int c = 0; c < cn; c += 64) {
-        uint32_t v0[32], v1[32], w[32];
-        tmem_ld32(tb + c0 + c, v0);
-        tmem_ld32(tb + c0 + c + 32, v1);
-        tmem_ld_wait();
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        if (h2 == 1 && !full) break;
+        uint32_t w[32];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          w[i] = pack_f16x2(__uint_as_float(v0[2 * i]) * k, __uint_as_float(v0[2 * i + 1]) * k);
-          w[16 + i] = pack_f16x2(__uint_as_float(v1[2 * i]) * k, __uint_as_float(v1[2 * i + 1]) * k);
+          w[i] = pack_f16x2(__uint_as_float(v[2 * h2][2 * i]) * k,
+                            __uint_as_float(v[2 * h2][2 * i + 1]) * k);
+          w[16 + i] = pack_f16x2(__uint_as_float(v[2 * h2 + 1][2 * i]) * k,
+                                 __uint_as_float(v[2 * h2 + 1][2 * i + 1]) * k);
         }
-        st.emit(&p.tmo[0], w, n0 + c0 + c, y0);
+        st.emit(&p.tmo[0], w, n0 + c0 + 64 * h2, y0);
       }
     }
   } else if (MODE == MODE_DOWN_RED) {
