@@ -642,10 +642,13 @@ def run_ours(args, w):
     byts = dict(
         map=2 * w.T * w.E + 8 * w.T * w.top_k + 12 * N,
         gather=2 * w.T * w.hidden + 2 * N * w.hidden,
-        scatter=2 * N * w.hidden + 8 * N + 4 * N + 2 * w.T * w.hidden,
+        # combine: the fp16 rows and their scales, dest_row, y written (the rows carry their
+        # routing weight); scatter-sum: the same plus the routing-weight partials and dweights
+        scatter=2 * N * w.hidden + 4 * N * B.scale_stride(w.hidden) + 4 * N + 2 * w.T * w.hidden,
         dy_gather=2 * w.T * w.hidden + 2 * N * w.hidden,
-        dx_scatter=2 * N * w.hidden + 4 * N * ((w.hidden + 255) // 256) + 4 * N + 2 * w.T * w.hidden
-        + 4 * N * ((w.ffn + 255) // 256) + 4 * N,
+        dx_scatter=2 * N * w.hidden + 4 * N * B.scale_stride(w.hidden) + 4 * N
+        + 2 * w.T * w.hidden + 4 * N * ((w.ffn + B.DGLU_TILE_COLS - 1) // B.DGLU_TILE_COLS)
+        + 4 * N,
         # router: x and W_r read, logits written; backward: logits, dweights, top read, dlogits
         # written and read twice, dx read and written, x read, dW_r written
         router_gemm=2 * w.T * w.hidden + 2 * w.E * w.hidden + 2 * w.T * w.E,

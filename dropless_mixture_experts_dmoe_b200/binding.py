@@ -21,7 +21,7 @@ MAX_EXPERTS = 1024
 MAX_TOP_K = 32
 
 WS_MAP, WS_FORWARD, WS_BACKWARD, WS_FORWARD_TRAIN, WS_ROUTER_BACKWARD = 0, 1, 2, 3, 4
-DGLU_TILE_COLS = 256
+DGLU_TILE_COLS = 128
 
 STATUS_NONFINITE_LOGITS = 0x1
 STATUS_EXPERT_OUT_OF_RANGE = 0x2

@@ -124,6 +124,12 @@ __host__ __device__ constexpr bool uses_units(int mode) {
          mode == MODE_DOWN_RED || mode == MODE_DGLU || mode == MODE_DX;
 }
 
+// Unit modes whose last unit of an expert with an odd block count runs as one block on the
+// pair (M = 128 paired MMA, 64 rows from each CTA) instead of a block and an empty half.
+__host__ __device__ constexpr bool half_units(int mode) {
+  return mode == MODE_GLU || mode == MODE_DOWN || mode == MODE_DX || mode == MODE_DGLU;
+}
+
 // Dense row modes: tiles are (pair of 128-row blocks of the T token rows, column tile).
 __host__ __device__ constexpr bool is_dense_rows(int mode) {
   return mode == MODE_ROUTER || mode == MODE_RDX;
@@ -185,9 +191,10 @@ struct GemmParams {
   long long wait_cycles;  // budget of every bounded wait of this launch
   const __nv_bfloat16 *in0, *in1;  // DGLU: saved A, Bm
   const float *weights;            // DGLU: routing weight of each flattened entry
-  float *part;                     // DGLU: [P_max, n_tiles] partial routing-weight gradients;
+  float *part;                     // DGLU: [P_max, ceil(f/128)] partial routing-weight gradients;
                                    // DOWN, DX: [P_max, dmoe_scale_stride(h)] scales of the rows
   int total;                       // router modes: number of pair tiles
+  int half_ok;                     // half_units modes: run single-block units with M = 128
   int split_k;                     // RWGRAD: 64-wide K steps per split
   int Ep;                          // RWGRAD: rows of one split's slab (E rounded up to 128)
   int32_t *status;
@@ -196,6 +203,7 @@ struct GemmParams {
 struct Tile {
   int e, n, m, which, row0, kit;
   bool dummy;  // this CTA's half of the unit has no rows: load zeros, store nothing
+  bool half;   // a unit of one block (half_units modes): M = 128, this CTA's 64 rows at row0
 };
 
 // Pair tile t -> expert, column tile, this CTA's rows.
@@ -205,6 +213,7 @@ __device__ __forceinline__ Tile decode(const GemmParams &p, int t, const int *us
   Tile tl;
   tl.which = 0;
   tl.m = 0;
+  tl.half = false;
   if (is_dense_rows(MODE)) {
     const int u = t / p.n_tiles;
     tl.n = t - u * p.n_tiles;
@@ -275,11 +284,18 @@ __device__ __forceinline__ Tile decode(const GemmParams &p, int t, const int *us
   const int unit = c0 + (lt - tl.n * cs);
   const int first = ((e > 0) ? p.padded_bins[e - 1] : 0) / BM;
   const int end = p.padded_bins[e] / BM;
-  const int b = first + 2 * unit + (int)rank;
+  const int b0 = first + 2 * unit;  // the unit's first block
   tl.e = e;
+  tl.kit = p.k_iters;
+  if (half_units(MODE) && p.half_ok && b0 + 1 >= end) {  // one block: 64 rows from each CTA
+    tl.half = true;
+    tl.dummy = false;
+    tl.row0 = b0 * BM + (int)rank * (BM / 2);
+    return tl;
+  }
+  const int b = b0 + (int)rank;
   tl.dummy = b >= end;
   tl.row0 = tl.dummy ? p.nblk_cap * BM : b * BM;  // a dummy half reads rows past P_max: zeros
-  tl.kit = p.k_iters;
   return tl;
 }
 
@@ -315,7 +331,21 @@ __device__ __forceinline__ void load_stage(const GemmParams &p, const Tile &tl, 
   if (MODE == MODE_GLU) {  // two K slabs per stage: 3D maps {64, rows, K/64}
     static_assert(MODE != MODE_GLU || KSLABS == 2, "GLU stages hold two K slabs");
     tma_load_3d_pair(sa, &p.tm[0], bar, 0, tl.row0, 2 * kb);
-    tma_load_3d_pair(sb, &p.tm[rank == 0 ? 1 : 2], bar, 0, tl.e * p.f + tl.n * (BN / 2), 2 * kb);
+    if (tl.half) {
+      // a single-block unit (M = 128): this CTA's B half holds 64 f-rows of W1 then the same
+      // 64 of W3 in each K slab, so a thread's accumulator row has gate and up side by side;
+      // maps 3 and 4 have 64-row boxes of one slab
+      const int fr = tl.e * p.f + tl.n * (BN / 2) + (int)rank * (BN / 4);
+#pragma unroll
+      for (int s2 = 0; s2 < 2; ++s2) {
+        uint8_t *d = sb + s2 * (BN / 2) * 128;
+        tma_load_3d_pair(d, &p.tm[3], bar, 0, fr, 2 * kb + s2);
+        tma_load_3d_pair(d + (BN / 4) * 128, &p.tm[4], bar, 0, fr, 2 * kb + s2);
+      }
+    } else {
+      tma_load_3d_pair(sb, &p.tm[rank == 0 ? 1 : 2], bar, 0, tl.e * p.f + tl.n * (BN / 2),
+                       2 * kb);
+    }
   } else if ((MODE == MODE_DOWN || MODE == MODE_DOWN_RED) && KSLABS == 2) {
     tma_load_3d_pair(sa, &p.tm[0], bar, 0, tl.row0, 2 * kb);
     tma_load_3d_pair(sb, &p.tm[1], bar, 0, tl.e * p.h + tl.n * BN + (int)rank * (BN / 2), 2 * kb);
@@ -427,6 +457,36 @@ __device__ __forceinline__ void pack_bf16_row(const uint32_t (&lo)[32], const ui
   }
 }
 
+// This warp's share of a tile of DOWN, DX or DGLU: output rows y0 .. y0+31 (one per lane),
+// columns n0 .. n0+kw-1, at TMEM column tcol of the accumulator.  A unit of one block
+// (M = 128 paired MMA) holds each CTA's 64 rows in lanes 0-63 for columns 0-127 and again in
+// lanes 64-127 for columns 128-255, all at TMEM columns 0-127: the warp of sub-partition sub
+// owns rows (sub & 1) * 32 and columns (sub >> 1) * 128; with 8 epilogue warps the second
+// column half of warps (half = 1) has nothing to do.
+struct Share {
+  int y0, n0, kw, tcol;
+  bool on;
+};
+template <int MODE, int EPI>
+__device__ __forceinline__ Share share_of(const Tile &tl, int sub, int half) {
+  constexpr int kw = BN / Cfg<MODE, EPI>::col_split;
+  Share s;
+  if (half_units(MODE) && tl.half) {
+    s.y0 = tl.row0 + (sub & 1) * 32;
+    s.n0 = tl.n * BN + (sub >> 1) * (BN / 2);
+    s.kw = BN / 2;
+    s.tcol = 0;
+    s.on = half == 0;
+  } else {
+    s.y0 = tl.row0 + sub * 32;
+    s.n0 = tl.n * BN + half * kw;
+    s.kw = kw;
+    s.tcol = half * kw;
+    s.on = true;
+  }
+  return s;
+}
+
 // Epilogue of one tile for the warp owning TMEM sub-partition `sub` (rows sub*32 .. +31 of
 // this CTA's 128 rows); tb = TMEM address of the warp's lanes at accumulator column 0.
 // Work of a tile's epilogue that does not depend on the accumulator, done before waiting for
@@ -445,11 +505,12 @@ __device__ __forceinline__ float epilogue_prologue(const GemmParams &p, const Ti
     return 0.0f;
   }
   if (MODE == MODE_DOWN && !tl.dummy)  // the row's routing weight, ahead of the accumulator
-    return row_weight(p, tl.e, tl.row0 + sub * 32 + lane);
+    return row_weight(p, tl.e, share_of<MODE, EPI>(tl, sub, half).y0 + lane);
   if (MODE != MODE_DGLU || tl.dummy) return 0.0f;
-  const int grow = tl.row0 + sub * 32 + lane;
-  const int n0 = tl.n * BN;
-  const int ncols = min(BN, p.f - n0);
+  const Share sh = share_of<MODE, EPI>(tl, sub, half);
+  const int grow = sh.y0 + lane;
+  const int n0 = sh.n0;
+  const int ncols = min(sh.kw, p.f - n0);
   const __nv_bfloat16 *ra = p.in0 + (size_t)grow * p.f + n0;
   const __nv_bfloat16 *rb = p.in1 + (size_t)grow * p.f + n0;
   for (int c = 0; c < ncols; c += 64) {  // one 128-byte line per 64 columns
@@ -466,14 +527,19 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
   const int y0 = tl.row0 + sub * 32;  // first row of this warp's boxes
   constexpr int kw = BN / Cfg<MODE, EPI>::col_split;  // accumulator columns per warp (non-GLU)
   if (is_glu(MODE)) {
-    const int n0 = tl.n * (BN / 2);
+    // gate columns at TMEM 0 .. gw-1, up at gw .. 2gw-1.  A single-block unit (M = 128) holds
+    // 64 f-columns per warp: rows (sub & 1) * 32 of this CTA's 64, f-columns (sub >> 1) * 64
+    const bool hu = half_units(MODE) && tl.half;
+    const int gw = hu ? BN / 4 : BN / 2;
+    const int n0 = tl.n * (BN / 2) + (hu ? (sub >> 1) * (BN / 4) : 0);
+    const int yg = hu ? tl.row0 + (sub & 1) * 32 : y0;
 #pragma unroll 1
-    for (int c = 0; c < BN / 2; c += 64) {  // one 64-column box of H (and of A, Bm)
+    for (int c = 0; c < gw; c += 64) {  // one 64-column box of H (and of A, Bm)
       uint32_t g0[32], g1[32], u0[32], u1[32], w[32];
       tmem_ld32(tb + c, g0);
       tmem_ld32(tb + c + 32, g1);
-      tmem_ld32(tb + BN / 2 + c, u0);
-      tmem_ld32(tb + BN / 2 + c + 32, u1);
+      tmem_ld32(tb + gw + c, u0);
+      tmem_ld32(tb + gw + c + 32, u1);
       tmem_ld_wait();
       if (p.outs & 1) {
 #pragma unroll
@@ -483,13 +549,13 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
           w[16 + i] = pack_bf16x2(silu_f(__uint_as_float(g1[2 * i])) * __uint_as_float(u1[2 * i]),
                                   silu_f(__uint_as_float(g1[2 * i + 1])) * __uint_as_float(u1[2 * i + 1]));
         }
-        st.emit(&p.tmo[0], w, n0 + c, y0);
+        st.emit(&p.tmo[0], w, n0 + c, yg);
       }
       if (p.outs & 2) {
         pack_bf16_row(g0, g1, w);
-        st.emit(&p.tmo[1], w, n0 + c, y0);
+        st.emit(&p.tmo[1], w, n0 + c, yg);
         pack_bf16_row(u0, u1, w);
-        st.emit(&p.tmo[2], w, n0 + c, y0);
+        st.emit(&p.tmo[2], w, n0 + c, yg);
       }
     }
   } else if (MODE == MODE_DOWN || MODE == MODE_DX) {
@@ -501,11 +567,14 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
     // m = 2^-38.  The values go out as fp16 (11 significant bits) and 1/scale to
     // p.part[row * nsc + chunk], its sign set when fp16 cannot hold 1/scale (m < 2^-38 or
     // m >= 2^29) or when the group holds an inf or NaN (values unscaled, 1/scale = -1).
-    const int n0 = tl.n * BN + half * kw;  // this warp's first column
-    const int ncols = min(kw, p.h - n0);   // multiple of 64 (may be <= 0)
+    const Share sh = share_of<MODE, EPI>(tl, sub, half);
+    if (!sh.on) return;
+    const int n0 = sh.n0;                     // this warp's first column
+    const int ncols = min(sh.kw, p.h - n0);   // multiple of 64 (may be <= 0)
     if (ncols <= 0) return;
-    tb += (uint32_t)(half * kw);
+    tb += (uint32_t)sh.tcol;
     const int nsc = dmoe_scale_stride(p.h);
+    const int y0 = sh.y0;
     const int grow = y0 + lane;
     const float wrow = (MODE == MODE_DOWN) ? wr : 1.0f;  // DOWN: from epilogue_prologue
     float *srow = p.part + (size_t)grow * nsc;
@@ -585,12 +654,16 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
     }
   } else if (MODE == MODE_DGLU) {
     static_assert(MODE != MODE_DGLU || EPI == 4, "one warp per row holds a row's partial sum");
-    const int n0 = tl.n * BN;
-    const int grow = y0 + lane;  // this thread's padded row; wr = its routing weight
-    float dot = 0.0f;  // sum over this tile's columns of G * h, in column order
+    const Share sh = share_of<MODE, EPI>(tl, sub, half);
+    const int n0 = sh.n0;
+    const int yw = sh.y0;         // first row of this warp's boxes
+    const int grow = yw + lane;   // this thread's padded row; wr = its routing weight
+    tb += (uint32_t)sh.tcol;
+    float dot0 = 0.0f, dot1 = 0.0f;  // per 128 columns: the sum of G * h, in column order
 #pragma unroll 1
-    for (int c = 0; c < kw; c += 64) {
+    for (int c = 0; c < sh.kw; c += 64) {
       if (n0 + c >= p.f) break;
+      float dot = (c < DMOE_DGLU_TILE_COLS) ? dot0 : dot1;
       uint32_t v0[32], v1[32], wa[32], wb[32], wh[32];
       uint4 qa[8], qb[8];
       tmem_ld32(tb + c, v0);
@@ -620,11 +693,18 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams &p, const Tile &t
         wb[i] = pack_bf16x2(dh0 * a0 * s0, dh1 * a1 * s1);
         wh[i] = pack_bf16x2(wr * h0, wr * h1);
       }
-      st.emit(&p.tmo[0], wa, n0 + c, y0);
-      st.emit(&p.tmo[1], wb, n0 + c, y0);
-      st.emit(&p.tmo[2], wh, n0 + c, y0);
+      if (c < DMOE_DGLU_TILE_COLS)
+        dot0 = dot;
+      else
+        dot1 = dot;
+      st.emit(&p.tmo[0], wa, n0 + c, yw);
+      st.emit(&p.tmo[1], wb, n0 + c, yw);
+      st.emit(&p.tmo[2], wh, n0 + c, yw);
     }
-    p.part[(size_t)grow * p.n_tiles + tl.n] = dot;
+    const int pt = (p.f + DMOE_DGLU_TILE_COLS - 1) / DMOE_DGLU_TILE_COLS;  // partials per row
+    float *prow = p.part + (size_t)grow * pt + n0 / DMOE_DGLU_TILE_COLS;
+    prow[0] = dot0;
+    if (DMOE_DGLU_TILE_COLS < sh.kw && n0 + DMOE_DGLU_TILE_COLS < p.f) prow[1] = dot1;
   } else if (MODE == MODE_ROUTER) {  // logits [T, E]: bf16 boxes, rows past T not stored
     if (y0 >= p.T) return;
     const int n0 = tl.n * BN;
@@ -871,6 +951,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
     // ---------------- MMA issuer (leader only) ----------------
     constexpr uint32_t idesc =
         idesc_bf16_f32(2 * BM, BN, C::a_mn, C::b_mn);
+    constexpr uint32_t idesc_half = idesc_bf16_f32(BM, BN, C::a_mn, C::b_mn);  // M = 128
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
@@ -912,7 +993,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg<MODE, EPI>::thre
           const uint64_t bd = C::b_mn
                                   ? sdesc_mnmajor_sw128(b_addr + kk * 2048, CHUNK_BYTES * C::kslabs)
                                   : sdesc_kmajor_sw128(b_addr + (kk >> 2) * B_BYTES + (kk & 3) * 32);
-          tc_mma_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          tc_mma_pair(d_tmem, ad, bd, (half_units(MODE) && tl.half) ? idesc_half : idesc,
+                      (kb | kk) != 0 ? 1u : 0u);
         }
         }
         tc_commit_pair_mc(&empty[stage]);
@@ -1042,12 +1124,12 @@ static bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t c
 // A box of {64, box_rows, 2} lands as two consecutive [box_rows x 128 B] swizzled chunks,
 // exactly the layout of two 2D boxes of 64 columns, in one TMA instruction.
 static bool make_tmap_chunked(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols,
-                              uint32_t box_rows) {
+                              uint32_t box_rows, uint32_t box_chunks = 2) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc || cols % 64 != 0) return false;
   cuuint64_t dims[3] = {64, rows, cols / 64};
   cuuint64_t strides[2] = {cols * 2, 128};
-  cuuint32_t box[3] = {64, box_rows, 2};
+  cuuint32_t box[3] = {64, box_rows, box_chunks};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1152,7 +1234,11 @@ cudaError_t launch_glu_gemm(const GemmProblem &g, const void *x_pad, const void 
     p.outs |= 2;
   }
   if (p.outs == 0) return cudaErrorInvalidValue;
-  p.tm[3] = p.tm[4] = p.tm[0];
+  // single-block units: 64-row, one-slab boxes of W1 and W3 (see load_stage)
+  if (!make_tmap_chunked(&p.tm[3], w1, EF, g.h, BN / 4, 1) ||
+      !make_tmap_chunked(&p.tm[4], w3, EF, g.h, BN / 4, 1))
+    return cudaErrorInvalidValue;
+  p.half_ok = 1;
   p.n_tiles = g.f / (BN / 2);
   p.k_iters = g.h / Cfg<MODE_GLU, 4>::bk;
   p.group = raster_units(g.h);
@@ -1201,6 +1287,9 @@ cudaError_t launch_down_gemm(const GemmProblem &g, const void *h_in, const void 
     p.k_iters = g.f / Cfg<MODE_DOWN, 8>::bk;
     return launch_gemm<MODE_DOWN, 8>(p, max_units(g) * p.n_tiles, st);
   }
+  // single-block units as M = 128 MMAs only with 4 epilogue warps: with 8 the epilogue bounds
+  // the tile and half of its warps would idle (measured slower)
+  p.half_ok = 1;
   p.k_iters = g.f / Cfg<MODE_DOWN, 4>::bk;
   return launch_gemm<MODE_DOWN, 4>(p, max_units(g) * p.n_tiles, st);
 }
@@ -1247,6 +1336,7 @@ cudaError_t launch_dglu_gemm(const GemmProblem &g, const void *dy_pad, const voi
   p.group = raster_units(g.h);
   p.in0 = static_cast<const __nv_bfloat16 *>(a_in);
   p.in1 = static_cast<const __nv_bfloat16 *>(b_in);
+  p.half_ok = 1;
   return launch_gemm<MODE_DGLU, 4>(p, max_units(g) * p.n_tiles, st);
 }
 
@@ -1266,6 +1356,7 @@ cudaError_t launch_dx_gemm(const GemmProblem &g, const void *da, const void *db,
   p.n_tiles = (g.h + BN - 1) / BN;
   p.k_iters = 2 * (g.f / Cfg<MODE_DX, 4>::bk);
   p.group = raster_units(2 * g.f);
+  p.half_ok = 1;
   return launch_gemm<MODE_DX, 4>(p, max_units(g) * p.n_tiles, st);
 }
 

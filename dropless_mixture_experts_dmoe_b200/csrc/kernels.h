@@ -116,8 +116,9 @@ cudaError_t launch_glu_gather_gemm(const GemmProblem &g, const void *x, const vo
 cudaError_t launch_down_gemm(const GemmProblem &g, const void *h_in, const void *w2, void *y_pad,
                              float *y_scale, cudaStream_t st);
 // ... and the backward: dH with the fused dGLU epilogue, dX, and the weight gradients.
-// DGLU column tile width (part has ceil(f / kDgluTileCols) columns).
-constexpr int kDgluTileCols = 256;
+// Columns per routing-weight partial of the DGLU epilogue (part has ceil(f / kDgluTileCols)
+// columns).
+constexpr int kDgluTileCols = DMOE_DGLU_TILE_COLS;
 // Down GEMM with the weighted combine fused into its epilogue: y_acc[t] += w_ts * (H W2_e^T)
 // row of each real padded row (fp32 vector reductions into y_acc [T, h]; no Y_pad).
 cudaError_t launch_down_red_gemm(const GemmProblem &g, const void *h_in, const void *w2,

@@ -197,9 +197,9 @@ typedef struct {
 #define DMOE_WS_FORWARD_TRAIN 3  /* dmoe_forward with saved != NULL (training) */
 #define DMOE_WS_ROUTER_BACKWARD 4 /* dmoe_router_backward */
 
-/* Column tile of the dH GEMM: the routing-weight partial sums of dmoe_bwd_dglu have
- * ceil(ffn / DMOE_DGLU_TILE_COLS) columns. */
-#define DMOE_DGLU_TILE_COLS 256
+/* Columns per routing-weight partial sum of the dH GEMM: dmoe_bwd_dglu's partials have
+ * ceil(ffn / DMOE_DGLU_TILE_COLS) columns per row. */
+#define DMOE_DGLU_TILE_COLS 128
 
 /* Static bound on the padded row count: floor((T*k + 127*E)/128)*128.  Every padded
  * buffer is sized from it, so no call needs the data-dependent size on the host (the
@@ -355,9 +355,9 @@ DMOE_API int dmoe_padded_scatter(const dmoe_dims *dims, const void *y_pad, const
  * the unweighted rows of dy), s = sigmoid(A), h = A*s*Bm and w the routing weight of the row
  * (0 for a padding row):
  *   da = bf16(w*G*Bm*s*(1 + A(1-s))),  dbm = bf16(w*G*A*s),  hw = bf16(w*h)   [P_max,f];
- *   dw_part[r * nt + n] = sum over the columns c of tile n of G[r,c]*h[r,c]   (fp32,
- *     nt = ceil(f / DMOE_DGLU_TILE_COLS) column tiles of 256; since G h^T = dy (H W2_e^T)^T,
- *     the tiles of a row sum to the routing-weight gradient <dy_t, Y_ts>).
+ *   dw_part[r * nt + n] = sum over the columns c of group n of G[r,c]*h[r,c]   (fp32,
+ *     nt = ceil(f / DMOE_DGLU_TILE_COLS) groups of 128 columns; since G h^T = dy (H W2_e^T)^T,
+ *     the groups of a row sum to the routing-weight gradient <dy_t, Y_ts>).
  * map->weights is read.  a_saved, bm_saved: bf16 A, Bm of dmoe_forward; dy_pad [P_max,h]. */
 DMOE_API int dmoe_bwd_dglu(const dmoe_dims *dims, const void *dy_pad, const void *w2,
                            const void *a_saved, const void *bm_saved, const dmoe_map *map,

@@ -72,7 +72,7 @@ def test_backward_steps_against_float64(w):
     D = lambda t: t[:P].double().cpu()
     dy_pad, da, dbm, hw = (D(st[n]) for n in ("dy_pad", "da", "dbm", "hw"))
     # dX_pad rows are block floating point: fp16 * a power-of-two scale per 128 columns
-    sc32 = st["dx_scale"].cpu().repeat_interleave(B.SCALE_COLS, dim=1)[:, :h]
+    sc32 = st["dx_scale"].cpu().abs().repeat_interleave(B.SCALE_COLS, dim=1)[:, :h]
     dxp32 = st["dx_pad"].float().cpu() * sc32
     dx_pad = dxp32[:P].double()
     nsc = (h + B.SCALE_COLS - 1) // B.SCALE_COLS
@@ -99,7 +99,7 @@ def test_backward_steps_against_float64(w):
     assert torch.equal(dy_pad, ref_dy)
     wrow = torch.zeros(P, dtype=torch.float64)  # routing weight of each padded row
     wrow[dest] = wts
-    nt = (f + 255) // 256
+    nt = (f + B.DGLU_TILE_COLS - 1) // B.DGLU_TILE_COLS  # routing-weight partials per row
     for b in range(nb):
         e = int(be[b])
         rows = slice(b * 128, (b + 1) * 128)
@@ -113,8 +113,8 @@ def test_backward_steps_against_float64(w):
         assert torch.allclose(dbm[rows], db_ref, rtol=2e-2, atol=2e-3), ("dBm", b)
         assert torch.allclose(hw[rows], wr * hv, rtol=2e-2, atol=2e-4), ("Hw", b)
         gh = G * hv
-        for n in range(nt):  # per-tile partial <G, h>, bounded by the sum of |terms|
-            cols = slice(n * 256, min(f, (n + 1) * 256))
+        for n in range(nt):  # per-group partial <G, h>, bounded by the sum of |terms|
+            cols = slice(n * B.DGLU_TILE_COLS, min(f, (n + 1) * B.DGLU_TILE_COLS))
             ref_p = gh[:, cols].sum(1)
             bound = 2e-3 * gh[:, cols].abs().sum(1) + 1e-6
             assert ((part[rows, n].double() - ref_p).abs() <= bound).all(), ("part", b, n)
