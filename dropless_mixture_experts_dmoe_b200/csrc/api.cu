@@ -91,8 +91,8 @@ inline const int32_t *entry_offsets_of(const dmoe_dims *d, const dmoe_map *m) {
 // Map workspace.  Plain routing: the map kernels' scratch for (T, E).  Token rounding: that
 // scratch sized for the larger of the two maps it builds (T tokens x k, then the entry list
 // as entries_of(d) single entries) | the top-k routing top [T,k] int32, weights [T,k] fp32 |
-// rank images [E][T] u16 | per-expert thresholds [3E] | per-token counts [T] | tile totals
-// [tiles] | tile offsets [tiles + 1].
+// rank images [E][T rounded up to 32] u16 | per-expert thresholds [3E] | per-token counts
+// [T] | tile totals [tiles] | tile offsets [tiles + 1].
 struct MapLayout {
   size_t top, w, img, param, tokc, tsum, toff, total;
 };
@@ -110,7 +110,7 @@ MapLayout map_layout(const dmoe_dims *d) {
   l.top = align_up(hist);
   l.w = align_up(l.top + Tk * 4);
   l.img = align_up(l.w + Tk * 4);
-  l.param = align_up(l.img + E * T * 2);
+  l.param = align_up(l.img + E * (size_t)round_img_stride((int)T) * 2);
   l.tokc = align_up(l.param + 3 * E * 4);
   l.tsum = align_up(l.tokc + T * 4);
   l.toff = align_up(l.tsum + tiles * 4);

@@ -55,8 +55,10 @@ cudaError_t launch_map_scatter(int T, int E, int k, int nblk_cap, const int32_t 
 // weights [cap] (entries past the list's end: expert -1, weight 0).
 constexpr int kRoundMaxT = 1 << 20;  // the selection keeps a bitmap of T bits per CTA
 constexpr size_t kRoundMaxSelectSmem = kRoundMaxT / 8;
+// Row stride of the rank images: T rounded up to whole 32-token groups.
+inline int round_img_stride(int T) { return (T + 31) / 32 * 32; }
 struct RoundScratch {
-  uint16_t *img;       // [E][T] rank images of the logits, one column per expert
+  uint16_t *img;       // [E][round_img_stride(T)] rank images of the logits, a row per expert
   int32_t *param;      // [3E] per expert: mode, threshold image, threshold token
   int32_t *tok_count;  // [T]
   int32_t *tile_sum;   // [map_tiles(T)]

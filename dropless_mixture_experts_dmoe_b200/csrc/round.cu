@@ -15,11 +15,12 @@
 // no padding rows.
 //
 // Kernels, all without inter-CTA waiting:
-//   k_round_images   the logits' rank images transposed to one contiguous column per expert
+//   k_round_images   the logits' rank images transposed to one contiguous row per expert
 //                    (64 x 64 tiles through shared memory, coalesced on both sides).
 //   k_round_select   one CTA per expert: decides round up / down and finds the rank threshold
 //                    (logit image v*, token t*) with two 8-bit histogram passes over the
-//                    candidates' logit images and one ordered pass over the tied tokens.
+//                    candidates' logit images and one ordered pass over the tied tokens, each
+//                    thread taking groups of 32 consecutive tokens.
 //   k_round_apply    one CTA per 64-token tile, warp per token: applies the thresholds; the
 //                    count pass writes per-token counts and tile totals, the write pass the
 //                    token's entries at its row offset.
@@ -43,13 +44,6 @@ __device__ __forceinline__ uint32_t rank_image(uint16_t b) {
 }
 
 
-// hist[key] += 1 for every lane with `on` (all 32 lanes call it): one shared-memory atomic per
-// distinct key in the warp.
-__device__ __forceinline__ void warp_hist_add(int *hist, bool on, uint32_t key, int lane) {
-  const unsigned peers = __match_any_sync(0xFFFFFFFFu, on ? key : 0x100u + (uint32_t)lane);
-  if (on && lane == __ffs(peers) - 1) atomicAdd(&hist[key], __popc(peers));
-}
-
 // Block-wide sum of one int per thread (kSelThreads threads).
 __device__ __forceinline__ int block_sum(int v, int *red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -64,9 +58,10 @@ __device__ __forceinline__ int block_sum(int v, int *red) {
 
 }  // namespace
 
-// img[e][t] = rank_image(logits[t][e]): 64 tokens x 64 experts per CTA through shared memory.
+// img[e][t] = rank_image(logits[t][e]) (row stride Tp): 64 tokens x 64 experts per CTA
+// through shared memory.
 __global__ void __launch_bounds__(256) k_round_images(const uint16_t *__restrict__ logits, int T,
-                                                      int E, uint16_t *__restrict__ img) {
+                                                      int Tp, int E, uint16_t *__restrict__ img) {
   __shared__ uint16_t tile[64][66];
   pdl_wait();
   pdl_trigger();
@@ -80,7 +75,7 @@ __global__ void __launch_bounds__(256) k_round_images(const uint16_t *__restrict
   for (int i = threadIdx.x; i < 64 * 64; i += 256) {
     const int ee = i / 64, tt = i % 64;  // write along an expert's column
     const int t = t0 + tt, e = e0 + ee;
-    if (t < T && e < E) img[(size_t)e * T + t] = tile[tt][ee];
+    if (t < T && e < E) img[(size_t)e * Tp + t] = tile[tt][ee];
   }
 }
 
@@ -89,14 +84,64 @@ __global__ void __launch_bounds__(256) k_round_images(const uint16_t *__restrict
 // rank threshold so that exactly m = r (down) or 128 - r (up) candidates are on the chosen side:
 //   up:    t added   iff image > v*, or image == v* and t <= t*
 //   down:  t dropped iff image < v*, or image == v* and t >= t*
-// param[3e..3e+2] = {mode (0 none, 1 down, 2 up), v*, t*}.  img [E][T]: the rank images, one
-// column per expert.  The tokens routed to e are its entries of the top-k routing's sorted
-// order (indices[bins[e-1] .. bins[e]), entry j of token j / k); routed_bits: this CTA's
-// bitmap of them (dynamic shared memory, T bits).
+// param[3e..3e+2] = {mode (0 none, 1 down, 2 up), v*, t*}.  img [E][Tp]: the rank images, one
+// row per expert, Tp = T rounded up to 32.  The tokens routed to e are its entries of the
+// top-k routing's sorted order (indices[bins[e-1] .. bins[e]), entry j of token j / k);
+// routed_bits: this CTA's bitmap of them (dynamic shared memory, T bits).  A thread takes
+// groups of 32 consecutive tokens (one bitmap word, four 16-byte loads of images), so every
+// pass is one load round followed by shared-memory work.
+struct SelGroup {
+  uint32_t cand;    // bit j: token 32g + j is a candidate
+  uint16_t v[32];   // the tokens' rank images
+};
+
+__device__ __forceinline__ SelGroup sel_group(const uint32_t *routed_bits,
+                                              const uint16_t *col, int g, int T, bool up) {
+  SelGroup q;
+  const int t0 = g * 32;
+  const uint32_t routed = routed_bits[g];
+  const uint32_t valid = (T - t0 >= 32) ? 0xFFFFFFFFu : ((1u << (T - t0)) - 1u);
+  q.cand = (up ? ~routed : routed) & valid;
+  const uint4 *src = reinterpret_cast<const uint4 *>(col + t0);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 w = __ldg(src + i);
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      q.v[8 * i + 2 * j] = (uint16_t)(ww[j] & 0xFFFFu);
+      q.v[8 * i + 2 * j + 1] = (uint16_t)(ww[j] >> 16);
+    }
+  }
+  return q;
+}
+
+// Exclusive prefix over the block (kSelThreads threads) of one int per thread; *total gets
+// the block's sum.
+__device__ __forceinline__ int block_excl_scan(int v, int *red, int *total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int n = __shfl_up_sync(0xFFFFFFFFu, x, off);
+    if (lane >= off) x += n;
+  }
+  __syncthreads();
+  if (lane == 31) red[warp] = x;
+  __syncthreads();
+  int before = 0, all = 0;
+  for (int w = 0; w < kSelThreads / 32; ++w) {
+    if (w < warp) before += red[w];
+    all += red[w];
+  }
+  *total = all;
+  return before + x - v;
+}
+
 __global__ void __launch_bounds__(kSelThreads) k_round_select(const int32_t *__restrict__ indices,
                                                               const int32_t *__restrict__ bins,
                                                               const int32_t *__restrict__ counts,
-                                                              int T, int E, int k,
+                                                              int T, int Tp, int E, int k,
                                                               const uint16_t *__restrict__ img,
                                                               int32_t *__restrict__ param) {
   extern __shared__ uint32_t routed_bits[];  // [ceil(T/32)]
@@ -118,7 +163,7 @@ __global__ void __launch_bounds__(kSelThreads) k_round_select(const int32_t *__r
     return;
   }
   const int m = up ? kBlock - r : r;  // candidates to take
-  const uint16_t *col = img + (size_t)e * T;
+  const uint16_t *col = img + (size_t)e * Tp;
   const int words = (T + 31) / 32;
   for (int i = threadIdx.x; i < words; i += kSelThreads) routed_bits[i] = 0u;
   for (int i = threadIdx.x; i < 256; i += kSelThreads) hist[i] = 0;
@@ -129,18 +174,12 @@ __global__ void __launch_bounds__(kSelThreads) k_round_select(const int32_t *__r
     atomicOr(&routed_bits[t >> 5], 1u << (t & 31));
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31;
-  // pass A: histogram of the candidates' high bytes (few distinct values: one atomic per
-  // distinct value and warp)
-  for (int tb = threadIdx.x - lane; tb < T; tb += kSelThreads) {
-    const int t = tb + lane;
-    bool cand = false;
-    uint32_t v = 0;
-    if (t < T) {
-      cand = (((routed_bits[t >> 5] >> (t & 31)) & 1u) != 0) != up;
-      v = col[t];
-    }
-    warp_hist_add(hist, cand, v >> 8, lane);
+  // pass A: histogram of the candidates' high bytes
+  for (int g = threadIdx.x; g < words; g += kSelThreads) {
+    const SelGroup q = sel_group(routed_bits, col, g, T, up);
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if ((q.cand >> j) & 1u) atomicAdd(&hist[q.v[j] >> 8], 1);
   }
   __syncthreads();
   // the high byte H holding the m-th candidate on the chosen side (from the top for round
@@ -164,15 +203,11 @@ __global__ void __launch_bounds__(kSelThreads) k_round_select(const int32_t *__r
   for (int i = threadIdx.x; i < 256; i += kSelThreads) hist[i] = 0;
   __syncthreads();
   // pass B: low bytes of the candidates whose high byte is H
-  for (int tb = threadIdx.x - lane; tb < T; tb += kSelThreads) {
-    const int t = tb + lane;
-    bool cand = false;
-    uint32_t v = 0;
-    if (t < T) {
-      v = col[t];
-      cand = ((((routed_bits[t >> 5] >> (t & 31)) & 1u) != 0) != up) && (v >> 8) == H;
-    }
-    warp_hist_add(hist, cand, v & 0xFFu, lane);
+  for (int g = threadIdx.x; g < words; g += kSelThreads) {
+    const SelGroup q = sel_group(routed_bits, col, g, T, up);
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (((q.cand >> j) & 1u) && (uint32_t)(q.v[j] >> 8) == H) atomicAdd(&hist[q.v[j] & 0xFFu], 1);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -191,42 +226,42 @@ __global__ void __launch_bounds__(kSelThreads) k_round_select(const int32_t *__r
   __syncthreads();
   const uint32_t vstar = (H << 8) | (uint32_t)s_sel[0];
   const int beyond = s_sel[1];  // candidates strictly better (up) / worse (down) than v*
-  int ties = 0;                 // candidates with image v*
-  for (int t = threadIdx.x; t < T; t += kSelThreads) {
-    const bool rt = (routed_bits[t >> 5] >> (t & 31)) & 1u;
-    ties += (rt != up && col[t] == vstar) ? 1 : 0;
+  // the tied candidates (image v*), group by group in token order: round up takes the ties
+  // with the lowest token indices (the q-th lowest tied token, q = m - beyond); round down
+  // drops those with the highest (the (ties - q + 1)-th lowest)
+  int ties = 0;
+  for (int g = threadIdx.x; g < words; g += kSelThreads) {
+    const SelGroup q = sel_group(routed_bits, col, g, T, up);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) ties += (((q.cand >> j) & 1u) && q.v[j] == vstar) ? 1 : 0;
   }
   ties = block_sum(ties, red);
-  // pass C: the tied candidate taken last.  Round up takes the ties with the lowest token
-  // indices (the q-th lowest tied token, q = m - beyond); round down drops those with the
-  // highest (the (ties - q + 1)-th lowest).  Walk the tokens in order, 512 at a time.
-  const int q = m - beyond;
-  const int want = up ? q : ties - q + 1;  // 1-based rank among the tied tokens, in t order
-  int seen = 0;
+  const int qn = m - beyond;
+  const int want = up ? qn : ties - qn + 1;  // 1-based rank among the tied tokens, in t order
   if (threadIdx.x == 0) s_sel[0] = -1;
   __syncthreads();
-  for (int t0 = 0; t0 < T; t0 += kSelThreads) {
-    const int t = t0 + threadIdx.x;
-    bool tie = false;
-    if (t < T) {
-      const bool rt = (routed_bits[t >> 5] >> (t & 31)) & 1u;
-      tie = (rt != up && col[t] == vstar);
+  int seen = 0;
+  for (int g0 = 0; g0 < words; g0 += kSelThreads) {  // rounds of kSelThreads groups
+    const int g = g0 + threadIdx.x;
+    uint32_t tiebits = 0u;
+    if (g < words) {
+      const SelGroup q = sel_group(routed_bits, col, g, T, up);
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        tiebits |= (((q.cand >> j) & 1u) && q.v[j] == vstar) ? (1u << j) : 0u;
     }
-    // inclusive prefix count of ties over the block, in token order
-    const unsigned bal = __ballot_sync(0xFFFFFFFFu, tie);
-    const int warp = threadIdx.x >> 5;
-    if (lane == 0) red[warp] = __popc(bal);
-    __syncthreads();
-    int before = seen;
-    for (int w = 0; w < warp; ++w) before += red[w];
-    const int rank = before + __popc(bal & ((2u << lane) - 1u));
-    if (tie && rank == want) s_sel[0] = t;
-    int chunk = 0;
-    for (int w = 0; w < kSelThreads / 32; ++w) chunk += red[w];
-    __syncthreads();
-    seen += chunk;
+    int total;
+    const int before = seen + block_excl_scan(__popc(tiebits), red, &total);
+    const int need = want - before;  // this thread's group holds it when 1 <= need <= popc
+    if (need >= 1 && need <= __popc(tiebits)) {
+      uint32_t b = tiebits;
+      for (int i = 1; i < need; ++i) b &= b - 1u;  // drop the lower ties
+      s_sel[0] = g * 32 + (__ffs(b) - 1);
+    }
+    seen += total;
     if (seen >= want) break;  // uniform: every thread has the same `seen`
   }
+  __syncthreads();
   if (threadIdx.x == 0) {
     param[3 * e] = up ? 2 : 1;
     param[3 * e + 1] = (int32_t)vstar;
@@ -415,11 +450,12 @@ cudaError_t launch_round_tokens(const uint16_t *logits, const int32_t *top, cons
   static cudaError_t attr = cudaFuncSetAttribute(
       k_round_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRoundMaxSelectSmem);
   if (attr != cudaSuccess) return attr;
+  const int Tp = round_img_stride(T);
   if ((err = launch_pdl(k_round_images, dim3((E + 63) / 64, (T + 63) / 64), 256, 0, st, logits, T,
-                        E, s.img)) != cudaSuccess)
+                        Tp, E, s.img)) != cudaSuccess)
     return err;
-  if ((err = launch_pdl(k_round_select, E, kSelThreads, sel_smem, st, indices, bins, counts, T, E,
-                        k, (const uint16_t *)s.img, s.param)) != cudaSuccess)
+  if ((err = launch_pdl(k_round_select, E, kSelThreads, sel_smem, st, indices, bins, counts, T, Tp,
+                        E, k, (const uint16_t *)s.img, s.param)) != cudaSuccess)
     return err;
   const int tiles = map_tiles(T);
   const size_t ap_smem = sizeof(int32_t) * (3 * (size_t)E + (size_t)kApplyWarps * ((E + 31) / 32));
