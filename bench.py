@@ -339,8 +339,8 @@ def run_reference(args, w):
         times.append(dt)
     total = sum(times)
     value = n_tok * args.steps / total
-    sample = (f"routing+map over all {w.T} tokens, forward of the first {n_tok} tokens per step "
-              f"(oracle, fp64 accumulation)")
+    sample = (f"routing+map over all {w.T} tokens, forward{' and backward' if w.backward else ''} "
+              f"of the first {n_tok} tokens per step (oracle, fp64 accumulation)")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
