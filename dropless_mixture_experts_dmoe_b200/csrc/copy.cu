@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(kCopyThreads) k_gather(int T, int h, int k, in
 // A lane covers 8 consecutive columns (one 16-byte vector) per entry; VPL vectors per lane
 // and SLOTS entries are loaded before any is consumed.
 template <int VPL, int SLOTS, bool F16S>
-__global__ void __launch_bounds__(kCopyThreads, (VPL * SLOTS <= 4) ? 4 : 2)
+__global__ void __launch_bounds__(kCopyThreads, 4)
     k_combine(int T, int h, int k, const uint4 *__restrict__ rows,
               const float *__restrict__ scale, const int32_t *__restrict__ dest_row,
               const float *__restrict__ weights, uint4 *__restrict__ out,
@@ -318,15 +318,14 @@ cudaError_t launch_gather(int T, int h, int k, int E, const void *x, const int32
                     static_cast<uint4 *>(x_pad), offsets);
 }
 
-// Shape of the combine: work items of one token's 4 KB row slice.  k > 2: 4 row loads in
-// flight per lane within 64 registers and four CTAs (32 warps) per SM (measured 13 % faster at
-// top-8 than 8 loads at two CTAs per SM); k <= 2: 8 wide row loads per lane, two CTAs per SM.
+// Shape of the combine: work items of one token's 4 KB row slice, 4 row loads in flight per
+// lane within 64 registers and four CTAs (32 warps) per SM (measured 13 % faster at top-8 and
+// 17 % at top-2 than 8 loads per lane at two CTAs per SM).
 static cudaError_t combine(int T, int h, int k, const void *rows, const float *scale,
                            const int32_t *dest_row, const float *weights, void *out,
                            const float *part, int nt, float *dweights, const int32_t *offsets,
                            cudaStream_t st) {
-  auto kernel = scale ? ((k <= 2) ? k_combine<4, 2, true> : k_combine<2, 2, true>)
-                      : ((k <= 2) ? k_combine<4, 2, false> : k_combine<2, 2, false>);
+  auto kernel = scale ? k_combine<2, 2, true> : k_combine<2, 2, false>;
   const long long items = (long long)T * slices(h);
   return launch_pdl(kernel, copy_grid(items), kCopyThreads, 0, st, T, h, k,
                     static_cast<const uint4 *>(rows), scale, dest_row, weights,
