@@ -5,16 +5,17 @@
 // completion ticket):
 //   k_route_hist   16 warps per 64-token tile, 4 tokens per warp with all their logits loaded
 //                  at once: top-k by integer max over order-preserving keys (ties -> lower
-//                  expert index; each lane keeps its three best candidates), fp32 softmax
-//                  weights, per-tile histogram in shared memory (O(E) bytes, independent of
-//                  T) and a per-tile status word.
+//                  expert index; each lane keeps its three best candidates, the picks checked
+//                  afterwards), fp32 softmax weights, per-tile histogram in shared memory
+//                  (O(E) bytes, independent of T) and a per-tile status word.
 //   k_map_scan     one CTA per 32 experts: per-expert exclusive offsets of every tile; the
 //                  last CTA to finish (a ticket counter, no waiting) computes bins,
 //                  padded_bins (round_up to 128), num_blocks and stores the status word.
-//   k_map_scatter  one CTA per tile: stable rank of every entry inside its expert (warp
-//                  histograms + __match_any_sync ranks in entry order), then indices,
-//                  bin_ids and dest_row from the index math of section 4.2; every CTA also
-//                  fills a slice of the block -> expert table.
+//   k_map_scatter  one CTA per up to 2048 entries (up to 4 tiles at top-8): stable rank of
+//                  every entry inside its expert (warp histograms + __match_any_sync ranks in
+//                  entry order), then indices, bin_ids (staged per expert in shared memory)
+//                  and dest_row from the index math of section 4.2; every CTA also fills a
+//                  slice of the block -> expert table.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -62,66 +63,89 @@ constexpr int kRouteWarps = kRouteThreads / 32;
 constexpr int kRouteTPW = kMapTokTile / kRouteWarps;  // tokens per warp
 static_assert(kRouteTPW * kRouteWarps == kMapTokTile, "routing tile");
 
-// One lane's share of a token's logits.  KPL = logits per lane (E <= 32*KPL).  VEC (E a
-// multiple of KPL): lane l owns experts KPL*l .. KPL*l + KPL-1, read as one vector load and
-// kept packed two per word; otherwise lane l owns experts l, l + 32, ..., one per word.
-template <int KPL, bool VEC>
+// One lane's share of a token's logits.  KPL = logits per lane (E <= 32*KPL).  PACKED (E even,
+// KPL >= 2): word c of lane l holds experts 64c + 2l and 64c + 2l + 1, two per word, so that
+// each word is one coalesced 128-byte load across the warp and a run of strong experts (the
+// low indices of a Zipf-skewed router) spreads over many lanes; otherwise lane l owns experts
+// l, l + 32, ..., one per word.
+template <int KPL, bool PACKED>
 struct RouteRow {
-  static constexpr int kWords = VEC ? (KPL + 1) / 2 : KPL;
+  static_assert(!PACKED || KPL >= 2, "two logits per word");
+  static constexpr int kWords = PACKED ? KPL / 2 : KPL;
   uint32_t w[kWords];
 
   __device__ __forceinline__ static int expert(int lane, int i) {
-    return VEC ? KPL * lane + i : lane + 32 * i;
+    return PACKED ? 64 * (i >> 1) + 2 * lane + (i & 1) : lane + 32 * i;
   }
   // fp32 image of logit i (the bf16 bits in the high half)
   __device__ __forceinline__ uint32_t image(int i) const {
-    if constexpr (VEC) return (i & 1) ? (w[i >> 1] & 0xFFFF0000u) : (w[i >> 1] << 16);
+    if constexpr (PACKED) return (i & 1) ? (w[i >> 1] & 0xFFFF0000u) : (w[i >> 1] << 16);
     return w[i] << 16;
   }
   __device__ __forceinline__ void load(const uint16_t *__restrict__ row, int E, int lane) {
-    if constexpr (VEC) {
-      const int e0 = KPL * lane;
-      const bool ok = e0 < E;  // E % KPL == 0: the whole vector is in the row or none of it
-      if constexpr (KPL == 1) {
-        w[0] = ok ? (uint32_t)__ldg(row + e0) : 0u;
-      } else if constexpr (KPL == 2) {
-        w[0] = ok ? __ldg(reinterpret_cast<const unsigned int *>(row + e0)) : 0u;
-      } else if constexpr (KPL == 4) {
-        uint2 q = make_uint2(0u, 0u);
-        if (ok) q = __ldg(reinterpret_cast<const uint2 *>(row + e0));
-        w[0] = q.x;
-        w[1] = q.y;
+#pragma unroll
+    for (int c = 0; c < kWords; ++c) {
+      if constexpr (PACKED) {
+        const int e = 64 * c + 2 * lane;  // E even: both experts of the pair exist or neither
+        w[c] = (e < E) ? __ldg(reinterpret_cast<const unsigned int *>(row + e)) : 0u;
       } else {
-#pragma unroll
-        for (int c = 0; c < kWords / 4; ++c) {
-          uint4 q = make_uint4(0u, 0u, 0u, 0u);
-          if (ok) q = __ldg(reinterpret_cast<const uint4 *>(row + e0) + c);
-          w[4 * c] = q.x;
-          w[4 * c + 1] = q.y;
-          w[4 * c + 2] = q.z;
-          w[4 * c + 3] = q.w;
-        }
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < KPL; ++i) {
-        const int e = lane + 32 * i;
-        w[i] = (e < E) ? (uint32_t)__ldg(row + e) : 0u;
+        const int e = lane + 32 * c;
+        w[c] = (e < E) ? (uint32_t)__ldg(row + e) : 0u;
       }
     }
   }
 };
 
 // Order-preserving 16-bit images of the two bf16 values packed in w, in the same halves:
-// for non-NaN a, b, a < b iff image(a) < image(b) (negative values have every bit inverted,
-// the others their sign bit set), and -0 is first turned into +0 (-0 + +0 = +0), so that the
-// two zeros tie.  NaN is not ordered here (the caller takes a separate path for it).
+// -0 is first turned into +0 (-0 + +0 = +0) so that the two zeros tie; then a negative half
+// has every bit inverted and any other half its sign bit set.  For non-NaN a, b: a < b iff
+// image(a) < image(b).  NaN is not ordered here (the caller takes a separate path for it).
 __device__ __forceinline__ uint32_t order2(uint32_t w) {
-  __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(&w);
-  v = __hadd2(v, __nv_bfloat162(__float2bfloat16_rn(0.0f), __float2bfloat16_rn(0.0f)));
-  const uint32_t z = *reinterpret_cast<const uint32_t *>(&v);
-  const uint32_t neg = (z >> 15) & 0x00010001u;  // sign bit of each half, at bit 0 / bit 16
-  return z ^ ((neg * 0x7FFFu) | 0x80008000u);
+  uint32_t z, sgn, o;
+  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(z) : "r"(w), "r"(0u));
+  // per half: its sign bit replicated (prmt with the selector's sign-extension bit set, which
+  // __byte_perm does not pass on)
+  asm("prmt.b32 %0, %1, %2, 0xBB99;" : "=r"(sgn) : "r"(z), "r"(0u));
+  // per half: bits 0-14 z ^ sgn, bit 15 ~z  (lookup table of c ? a ^ b : ~a)
+  asm("lop3.b32 %0, %1, %2, %3, 0x2D;" : "=r"(o) : "r"(z), "r"(sgn), "r"(0x7FFF7FFFu));
+  return o;
+}
+
+// Non-finite detector over packed bf16 pairs: acc = w * 0 + acc stays +0 in both halves while
+// every value seen is finite (x * 0 = +-0 and +0 + -0 = +0) and is NaN from the first Inf or
+// NaN on.
+__device__ __forceinline__ uint32_t nonfinite_acc(uint32_t acc, uint32_t w) {
+  uint32_t r;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(w), "r"(0u), "r"(acc));
+  return r;
+}
+
+// 2^x without subnormal results (flushed to +0): the terms of a softmax sum, which is >= 1.
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// (a, b) * s + (t, t) on the paired fp32 pipe, and the sum of two pairs.
+__device__ __forceinline__ void fma_f32x2(float &a, float &b, float s, float t) {
+  asm("{.reg .b64 x, y, m, c;\n\t"
+      "mov.b64 x, {%0, %1};\n\t"
+      "mov.b64 m, {%2, %2};\n\t"
+      "mov.b64 c, {%3, %3};\n\t"
+      "fma.rn.f32x2 y, x, m, c;\n\t"
+      "mov.b64 {%0, %1}, y;}"
+      : "+f"(a), "+f"(b)
+      : "f"(s), "f"(t));
+}
+__device__ __forceinline__ void add_f32x2(float &a, float &b, float c, float d) {
+  asm("{.reg .b64 x, y, z;\n\t"
+      "mov.b64 x, {%0, %1};\n\t"
+      "mov.b64 y, {%2, %3};\n\t"
+      "add.rn.f32x2 z, x, y;\n\t"
+      "mov.b64 {%0, %1}, z;}"
+      : "+f"(a), "+f"(b)
+      : "f"(c), "f"(d));
 }
 
 // The C largest keys seen so far, largest first (0 = empty slot): one insertion costs C
@@ -141,35 +165,83 @@ struct TopC {
       c[i] = hi;
     }
   }
-  __device__ __forceinline__ void pop() {
-#pragma unroll
-    for (int i = 0; i + 1 < C; ++i) c[i] = c[i + 1];
-    c[C - 1] = 0u;
-  }
 };
+
+struct Picks {
+  uint32_t mine;   // lane s < k: the key of pick s
+  uint32_t first;  // every lane: pick 0 (the largest key)
+  uint32_t last;   // every lane: pick k - 1
+  bool dry;        // this lane has no candidate left
+};
+
+// The k rounds of a warp-wide integer max over the lanes' best candidates: keys are unique,
+// so exactly one lane holds each winner and drops it.  KC > 0 fixes k at compile time.  Every
+// lane keeps its C largest keys; with REFILL, a lane that has given up all C while rounds
+// remain refills them from its keys below the last pick (warp-uniform test).  Without it the
+// picks are the top-k of the candidates, and the caller checks that they are the top-k of all.
+template <int C, int KPL, int KC, bool REFILL>
+__device__ __forceinline__ Picks select_rounds(const uint32_t (&key)[KPL], int k, int lane) {
+  TopC<C> cand;
+  cand.clear();
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) cand.insert(key[i]);
+  Picks r;
+  r.mine = 0u;
+  r.first = 0u;
+  uint32_t wb = 0u;
+  auto round = [&](int s) {
+    wb = __reduce_max_sync(0xFFFFFFFFu, cand.c[0]);
+    if (s == 0) r.first = wb;
+    r.mine = (lane == s) ? wb : r.mine;
+    const bool win = cand.c[0] == wb;
+#pragma unroll
+    for (int i = 0; i + 1 < C; ++i) cand.c[i] = win ? cand.c[i + 1] : cand.c[i];
+    cand.c[C - 1] = win ? 0u : cand.c[C - 1];
+    if constexpr (REFILL && KPL > C) {
+      const bool dry = win && cand.c[0] == 0u && s + 1 < k;
+      if (__any_sync(0xFFFFFFFFu, dry)) {
+        if (dry) {
+#pragma unroll
+          for (int i = 0; i < KPL; ++i)
+            if (key[i] < wb) cand.insert(key[i]);
+        }
+      }
+    }
+  };
+  if constexpr (KC > 0) {
+#pragma unroll
+    for (int s = 0; s < KC; ++s) round(s);
+  } else {
+#pragma unroll 1
+    for (int s = 0; s < k; ++s) round(s);
+  }
+  r.last = wb;
+  r.dry = cand.c[0] == 0u;
+  return r;
+}
 
 // Grid: one CTA per 64-token tile.  Per token: every lane turns its logits into unique integer
 // keys (order-preserving image of the bf16 value in the high half, 0xFFFF - expert in the low
 // half, so the larger key is the larger logit and, on equal logits, the lower expert) and
 // keeps its three largest; k rounds of a warp-wide integer max then pick the top-k in rank
-// order, the winning lane dropping its head.  A lane that gives up all three of its
-// candidates while rounds remain (it holds more than three of the top-k) refills them from
-// its keys below the last pick.  Weights: fp32 softmax over all E logits (or, renormalised,
-// over the k picks) with the first pick as the maximum.  The tile's expert histogram is built
-// in shared memory and written to tile_hist; the tile's status bits go to tile_flags (a plain
-// store, so the workspace needs no initialisation).
-template <int KPL, bool VEC>
-__global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__restrict__ logits,
+// order.  Those are the top-k of all keys unless some lane holds more than three keys at or
+// above the last pick (if a key of the true top-k were missing from the candidates, its lane
+// would hold three larger ones and it, all above the last pick): then, rarely, the rounds run
+// again with refills.  Weights: fp32 softmax over all E logits (or, renormalised, over the k
+// picks) with the first pick as the maximum.  The tile's expert histogram is built in shared
+// memory and written to tile_hist; the tile's status bits go to tile_flags (a plain store, so
+// the workspace needs no initialisation).
+template <int KPL, bool PACKED, int KC>
+__global__ void __launch_bounds__(kRouteThreads, KPL <= 8 ? 2 : 1) k_route_hist(const uint16_t *__restrict__ logits,
                                                               int T, int E, int k, int renorm,
                                                               int32_t *__restrict__ top,
                                                               float *__restrict__ weights,
                                                               int32_t *__restrict__ tile_hist,
                                                               int32_t *__restrict__ tile_flags,
                                                               unsigned int *__restrict__ done) {
-  using Row = RouteRow<KPL, VEC>;
+  using Row = RouteRow<KPL, PACKED>;
   constexpr int C = (KPL < 3) ? KPL : 3;                  // candidates kept per lane
   constexpr int kInFlight = (KPL <= 8) ? kRouteTPW : 1;  // token rows loaded ahead per warp
-  constexpr bool kPacked = VEC && KPL >= 2;              // two logits per word
   constexpr float kLog2e = 1.4426950408889634f;
   extern __shared__ int hist[];  // [E]
   __shared__ int s_flags;
@@ -180,15 +252,21 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__
   for (int e = threadIdx.x; e < E; e += kRouteThreads) hist[e] = 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * kMapTokTile + warp;
-  // expert KPL*lane + i of the vector layout exists iff the lane's first one does (E % KPL == 0)
-  const bool lane_ok = KPL * lane < E;
   const bool full_rows = (E == 32 * KPL);  // every slot of every lane holds an expert
-  uint32_t low[KPL];  // low halves of this lane's keys; 0 marks a slot past the last expert
+  // low halves of this lane's keys, per word (PACKED: key 2c in bits 0-15, key 2c + 1 in bits
+  // 16-31); 0 marks a word past the last expert
+  uint32_t lowp[Row::kWords];
 #pragma unroll
-  for (int i = 0; i < KPL; ++i) {
-    const int e = Row::expert(lane, i);
-    low[i] = (VEC ? lane_ok : (e < E)) ? 0xFFFFu - (uint32_t)e : 0u;
+  for (int c = 0; c < Row::kWords; ++c) {
+    const int e = Row::expert(lane, PACKED ? 2 * c : c);
+    lowp[c] = (e >= E) ? 0u
+              : PACKED ? (((0xFFFEu - (uint32_t)e) << 16) | (0xFFFFu - (uint32_t)e))
+                       : 0xFFFFu - (uint32_t)e;
   }
+  auto low_of = [&](int i) -> uint32_t {
+    if constexpr (PACKED) return (i & 1) ? (lowp[i >> 1] >> 16) : (lowp[i >> 1] & 0xFFFFu);
+    return lowp[i];
+  };
   Row rows[kInFlight];
 #pragma unroll
   for (int j = 0; j < kInFlight; ++j) {
@@ -207,59 +285,43 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__
     } else {
       cur.load(logits + (size_t)t * E, E, lane);
     }
-    // keys, and a test for Inf / NaN: a half whose exponent bits are all ones carries into
-    // its bit 15 when 0x0080 is added to its exponent field (slots past E hold 0: no carry)
     uint32_t key[KPL];
-    uint32_t nf = 0u;
+    uint32_t nfa = 0u;  // slots past E hold +0: finite
 #pragma unroll
     for (int i = 0; i < Row::kWords; ++i) {
       const uint32_t wv = cur.w[i];
-      nf |= (wv & 0x7F807F80u) + 0x00800080u;
+      nfa = nonfinite_acc(nfa, wv);
       const uint32_t o = order2(wv);
-      if constexpr (kPacked) {
-        key[2 * i] = __byte_perm(o, low[2 * i], 0x1054);        // (image lo << 16) | low
-        key[2 * i + 1] = __byte_perm(o, low[2 * i + 1], 0x3254);  // (image hi << 16) | low
+      if constexpr (PACKED) {
+        key[2 * i] = __byte_perm(o, lowp[i], 0x1054);      // (image lo << 16) | low lo
+        key[2 * i + 1] = __byte_perm(o, lowp[i], 0x3276);  // (image hi << 16) | low hi
       } else {
-        key[i] = __byte_perm(o, low[i], 0x1054);
+        key[i] = __byte_perm(o, lowp[i], 0x1054);
       }
     }
     if (!full_rows) {  // warp-uniform: slots past the last expert hold no candidate
 #pragma unroll
-      for (int i = 0; i < KPL; ++i) key[i] = low[i] ? key[i] : 0u;
+      for (int i = 0; i < KPL; ++i) key[i] = low_of(i) ? key[i] : 0u;
     }
-    if (__any_sync(0xFFFFFFFFu, (nf & 0x80008000u) != 0u)) {  // rare: NaN ranked lowest
+    if (__any_sync(0xFFFFFFFFu, nfa != 0u)) {  // rare: NaN ranked lowest
       bad = true;
 #pragma unroll
-      for (int i = 0; i < KPL; ++i) key[i] = low[i] ? route_key_nan(cur.image(i), low[i]) : 0u;
-    }
-    TopC<C> cand;
-    cand.clear();
-#pragma unroll
-    for (int i = 0; i < KPL; ++i) cand.insert(key[i]);
-    // k rounds of a warp-wide integer max; keys are unique, so exactly one lane holds the
-    // winner, and a valid key is never 0 (its low half is >= 0xFFFF - 1023).
-    uint32_t my_key = 0;  // lane s < k: the key of pick s
-    for (int s = 0; s < k; ++s) {
-      const uint32_t wb = __reduce_max_sync(0xFFFFFFFFu, cand.c[0]);
-      my_key = (lane == s) ? wb : my_key;
-      const bool win = cand.c[0] == wb;
-#pragma unroll
-      for (int i = 0; i + 1 < C; ++i) cand.c[i] = win ? cand.c[i + 1] : cand.c[i];
-      cand.c[C - 1] = win ? 0u : cand.c[C - 1];
-      if constexpr (KPL > C) {
-        // a lane that has given up all its candidates refills them from its keys below the
-        // last pick (it holds more than C of the top-k); warp-uniform test, rarely true
-        const bool dry = win && cand.c[0] == 0u && s + 1 < k;
-        if (__any_sync(0xFFFFFFFFu, dry)) {
-          if (dry) {
-#pragma unroll
-            for (int i = 0; i < KPL; ++i)
-              if (key[i] < wb) cand.insert(key[i]);
-          }
-        }
+      for (int i = 0; i < KPL; ++i) {
+        const uint32_t lo = low_of(i);
+        key[i] = lo ? route_key_nan(cur.image(i), lo) : 0u;
       }
     }
-    const uint32_t top_key = __shfl_sync(0xFFFFFFFFu, my_key, 0);
+    // a valid key is never 0 (its low half is >= 0xFFFF - 1023)
+    Picks pk = select_rounds<C, KPL, KC, false>(key, k, lane);
+    if constexpr (KPL > C) {
+      if (__any_sync(0xFFFFFFFFu, pk.dry)) {
+        int cnt = 0;
+#pragma unroll
+        for (int i = 0; i < KPL; ++i) cnt += (key[i] >= pk.last) ? 1 : 0;
+        if (__any_sync(0xFFFFFFFFu, cnt > C)) pk = select_rounds<C, KPL, KC, true>(key, k, lane);
+      }
+    }
+    const uint32_t my_key = pk.mine, top_key = pk.first;
     const int my_e = 0xFFFF - (int)(my_key & 0xFFFFu);
     // softmax over all E logits (or, renormalised, over the k picks), max = the first pick;
     // e^(x - m) = 2^(x log2(e) - m log2(e)) with one fused multiply-add per logit
@@ -273,14 +335,23 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const uint16_t *__
     float sum = 0.0f;
     if (renorm) {
       if (lane < k) sum = ev;
+    } else if (PACKED && full_rows) {  // two logits per word on the paired fp32 pipe
+      float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+      for (int i = 0; i < Row::kWords; ++i) {
+        float a = __uint_as_float(cur.w[i] << 16), b = __uint_as_float(cur.w[i] & 0xFFFF0000u);
+        fma_f32x2(a, b, kLog2e, -ml);
+        add_f32x2(s0, s1, ex2_ftz(a), ex2_ftz(b));
+      }
+      sum = s0 + s1;
     } else if (full_rows) {
 #pragma unroll
       for (int i = 0; i < KPL; ++i)
-        sum += ex2_approx(fmaf(__uint_as_float(cur.image(i)), kLog2e, -ml));
+        sum += ex2_ftz(fmaf(__uint_as_float(cur.image(i)), kLog2e, -ml));
     } else {
 #pragma unroll
       for (int i = 0; i < KPL; ++i)
-        if (low[i]) sum += ex2_approx(fmaf(__uint_as_float(cur.image(i)), kLog2e, -ml));
+        if (low_of(i)) sum += ex2_ftz(fmaf(__uint_as_float(cur.image(i)), kLog2e, -ml));
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
@@ -360,9 +431,11 @@ __global__ void __launch_bounds__(kMapThreads) k_given_hist(const int32_t *__res
 constexpr int kScanThreads = 1024;
 static_assert(kScanSeg == 32 * kScanCache, "a scan CTA holds its segment in registers");
 
-// Inclusive block-wide scan of one int per thread (1024 threads).
+// Inclusive block-wide scan of one int per thread (whole warps, at most 1024 threads);
+// warp_tot holds 32 ints of shared memory.
 __device__ __forceinline__ int block_incl_scan(int v, int *warp_tot) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = (int)(blockDim.x >> 5);
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const int n = __shfl_up_sync(0xFFFFFFFFu, v, off);
@@ -371,7 +444,7 @@ __device__ __forceinline__ int block_incl_scan(int v, int *warp_tot) {
   if (lane == 31) warp_tot[warp] = v;
   __syncthreads();
   if (warp == 0) {
-    int w = warp_tot[lane];
+    int w = (lane < nwarps) ? warp_tot[lane] : 0;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const int n = __shfl_up_sync(0xFFFFFFFFu, w, off);
@@ -495,11 +568,21 @@ __global__ void __launch_bounds__(kScanThreads, 1) k_map_scan(int n_tiles, int E
 constexpr int kScatRounds = 8;
 static_assert(kMapTokTile * DMOE_MAX_TOP_K <= kMapWarps * 32 * kScatRounds, "scatter rounds");
 
-// Grid: one CTA per tile.  Stable rank of every entry inside its expert (warp histograms and
-// __match_any_sync ranks in entry order), then indices, bin_ids and dest_row from the index
-// math of section 4.2.  Every CTA also writes a grid-strided slice of the block -> expert table
-// (entry b = the expert whose padded range holds row 128*b, -1 past num_blocks).
-__global__ void __launch_bounds__(kMapThreads) k_map_scatter(int T, int E, int k, int nblk_cap,
+// Entries of one scatter CTA: its staging buffers in shared memory hold that many.
+constexpr int kScatEntries = kMapWarps * 32 * kScatRounds;
+
+// Grid: one CTA per S consecutive tiles (S a power of two dividing kScanSeg, at most
+// kScatEntries entries: up to 4 for top-8, fewer where the grid would drop below two CTAs per
+// SM), so that the per-expert work of a CTA (offsets, warp histograms) is shared by S tiles.  The rank r of an entry inside its expert among the CTA's
+// entries (warp histograms and __match_any_sync ranks, in entry order) gives its sorted
+// position s_base[e] + r by the index math of section 4.2: dest_row is stored from there in
+// entry order, while indices and bin_ids are first staged in shared memory, expert by
+// expert, and then stored by consecutive threads, so that each expert's run of the CTA (one
+// contiguous range of both arrays) takes a few wide stores instead of one per entry.  Every
+// CTA also writes a grid-strided slice of the block -> expert table (entry b = the expert
+// whose padded range holds row 128*b, -1 past num_blocks).
+__global__ void __launch_bounds__(kMapThreads) k_map_scatter(int T, int E, int k, int S,
+                                                             int nblk_cap,
                                                              const int32_t *__restrict__ top,
                                                              const int32_t *__restrict__ tile_off,
                                                              const int32_t *__restrict__ seg_off,
@@ -510,16 +593,22 @@ __global__ void __launch_bounds__(kMapThreads) k_map_scatter(int T, int E, int k
                                                              int32_t *__restrict__ dest_row,
                                                              int32_t *__restrict__ block_expert) {
   extern __shared__ int sm[];
-  int *wh = sm;                           // [kMapWarps][E] counts, then exclusive offsets
-  int *s_base = wh + kMapWarps * E;       // [E] bins[e-1] + offset of this tile inside e
-  int *s_shift = s_base + E;              // [E] padded_bins[e-1] - bins[e-1]
-  int *s_pb = s_shift + E;                // [E] padded_bins
+  int *wh = sm;                      // [kMapWarps][E] counts, then offsets inside (CTA, expert)
+  int *s_base = wh + kMapWarps * E;  // [E] bins[e-1] + offset of this CTA's tiles inside e
+  int *s_shift = s_base + E;         // [E] padded_bins[e-1] - bins[e-1]
+  int *s_pb = s_shift + E;           // [E] padded_bins
+  int *s_loff = s_pb + E;            // [E] staging slot of the CTA's first entry of e
+  int *st_j = s_loff + E;            // [kScatEntries] staged entry index, by slot
+  int *st_e = st_j + kScatEntries;   // [kScatEntries] staged expert, by slot
+  __shared__ int warp_tot[32];
+  __shared__ int s_nv;
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long N = (long long)T * k;
-  const long long j0 = (long long)blockIdx.x * kMapTokTile * k;
-  const long long j1 = min(N, j0 + (long long)kMapTokTile * k);
+  const int tile0 = blockIdx.x * S;  // the CTA's first tile
+  const long long j0 = (long long)tile0 * kMapTokTile * k;
+  const long long j1 = min(N, j0 + (long long)S * kMapTokTile * k);
   const int n = (int)(j1 - j0);
   const int per_warp = (((n + kMapWarps - 1) / kMapWarps) + 31) & ~31;
   const long long wb = j0 + (long long)warp * per_warp;
@@ -540,8 +629,8 @@ __global__ void __launch_bounds__(kMapThreads) k_map_scatter(int T, int E, int k
   for (int e = threadIdx.x; e < E; e += kMapThreads) {
     const int bp = (e > 0) ? bins[e - 1] : 0;
     const int pp = (e > 0) ? padded_bins[e - 1] : 0;
-    s_base[e] = bp + seg_off[(size_t)(blockIdx.x / kScanSeg) * E + e] +
-                tile_off[(size_t)blockIdx.x * E + e];
+    s_base[e] = bp + seg_off[(size_t)(tile0 / kScanSeg) * E + e] +
+                tile_off[(size_t)tile0 * E + e];
     s_shift[e] = pp - bp;
     s_pb[e] = padded_bins[e];
   }
@@ -563,17 +652,35 @@ __global__ void __launch_bounds__(kMapThreads) k_map_scatter(int T, int E, int k
     __syncwarp();
   }
   __syncthreads();
-  // exclusive offsets per (warp, expert): expert start + tile offset + earlier warps
-  for (int e = threadIdx.x; e < E; e += kMapThreads) {
-    int run = s_base[e];
+  // per expert: warp counts -> offsets inside (CTA, expert); the CTA's count of each expert,
+  // scanned over the experts in order, gives its staging slots (a thread takes a run of up
+  // to ceil(E / kMapThreads) consecutive experts)
+  const int ept = (E + kMapThreads - 1) / kMapThreads;
+  const int e_lo = min(E, threadIdx.x * ept), e_hi = min(E, e_lo + ept);
+  int tsum = 0;
+  for (int e = e_lo; e < e_hi; ++e) {
+    int run = 0;
     for (int w = 0; w < kMapWarps; ++w) {
       const int v = wh[w * E + e];
       wh[w * E + e] = run;
       run += v;
     }
+    s_loff[e] = run;  // the count, for now
+    tsum += run;
+  }
+  const int incl = block_incl_scan(tsum, warp_tot);
+  if (threadIdx.x == kMapThreads - 1) s_nv = incl;
+  {
+    int pre = incl - tsum;
+    for (int e = e_lo; e < e_hi; ++e) {
+      const int c = s_loff[e];
+      s_loff[e] = pre;
+      pre += c;
+    }
   }
   __syncthreads();
-  // pass 2: sorted position of every entry, in entry order within each expert
+  // pass 2: rank of every entry inside (CTA, expert), in entry order: dest_row, and the
+  // entry's staging slot
 #pragma unroll
   for (int r = 0; r < kScatRounds; ++r) {
     if (wb + 32 * r >= we) break;
@@ -581,16 +688,25 @@ __global__ void __launch_bounds__(kMapThreads) k_map_scatter(int T, int E, int k
     const int e = ev[r];
     const unsigned peers = peers_of[r];
     if (e >= 0) {
-      const int i = my[e] + __popc(peers & lt_mask);
-      indices[i] = (int32_t)j;
-      bin_ids[i] = e;
-      dest_row[j] = i + s_shift[e];  // offset_in_bin + padded_bins[e-1]
+      const int rr = my[e] + __popc(peers & lt_mask);
+      dest_row[j] = s_base[e] + rr + s_shift[e];  // offset_in_bin + padded_bins[e-1]
+      const int slot = s_loff[e] + rr;
+      st_j[slot] = (int)j;  // T * k <= 2^25
+      st_e[slot] = e;
     } else if (j < we) {
       dest_row[j] = -1;
     }
     __syncwarp();
     if (e >= 0 && lane == __ffs(peers) - 1) my[e] += __popc(peers);
     __syncwarp();
+  }
+  __syncthreads();
+  // pass 3: indices and bin_ids, slot by slot (slot - s_loff[e] = the rank inside the expert)
+  for (int t = threadIdx.x; t < s_nv; t += kMapThreads) {
+    const int e = st_e[t];
+    const int i = s_base[e] + (t - s_loff[e]);
+    indices[i] = st_j[t];
+    bin_ids[i] = e;
   }
   // block -> expert table slice
   const int nb = s_pb[E - 1] / kBlock;
@@ -625,13 +741,20 @@ cudaError_t launch_route_hist(const uint16_t *logits, int T, int E, int k, bool 
   if (!logits)
     return launch_pdl(k_given_hist, tiles, kMapThreads, smem, st, top, T, E, k,
                       absent_ok ? 1 : 0, tile_hist, flags, done);
-  // logits per lane: the smallest power of two with E <= 32 * KPL
+  // logits per lane: the smallest power of two with E <= 32 * KPL; two per word when E is
+  // even; the round count fixed at compile time for top-2 and top-8 on those layouts
   using Kernel = void (*)(const uint16_t *, int, int, int, int, int32_t *, float *, int32_t *,
                           int32_t *, unsigned int *);
   Kernel kernel;
-#define DMOE_ROUTE(KPL) kernel = (E % KPL == 0) ? k_route_hist<KPL, true> : k_route_hist<KPL, false>
+#define DMOE_ROUTE_K(KPL, PK) \
+  kernel = (k == 8) ? k_route_hist<KPL, PK, 8> : (k == 2) ? k_route_hist<KPL, PK, 2> : k_route_hist<KPL, PK, 0>
+#define DMOE_ROUTE(KPL)           \
+  if (E % 2 == 0)                 \
+    DMOE_ROUTE_K(KPL, true);      \
+  else                            \
+    kernel = k_route_hist<KPL, false, 0>
   if (E <= 32)
-    DMOE_ROUTE(1);
+    kernel = (k == 2) ? k_route_hist<1, false, 2> : k_route_hist<1, false, 0>;
   else if (E <= 64)
     DMOE_ROUTE(2);
   else if (E <= 128)
@@ -643,6 +766,7 @@ cudaError_t launch_route_hist(const uint16_t *logits, int T, int E, int k, bool 
   else
     DMOE_ROUTE(32);
 #undef DMOE_ROUTE
+#undef DMOE_ROUTE_K
   return launch_pdl(kernel, tiles, kRouteThreads, smem, st, logits, T, E, k, renorm ? 1 : 0, top,
                     weights, tile_hist, flags, done);
 }
@@ -660,8 +784,21 @@ cudaError_t launch_map_scatter(int T, int E, int k, int nblk_cap, const int32_t 
                                const int32_t *tile_off, const int32_t *bins,
                                const int32_t *padded_bins, int32_t *indices, int32_t *bin_ids,
                                int32_t *dest_row, int32_t *block_expert, cudaStream_t st) {
-  const size_t smem = sizeof(int) * (size_t)(kMapWarps + 3) * E;
-  return launch_pdl(k_map_scatter, map_tiles(T), kMapThreads, smem, st, T, E, k, nblk_cap, top,
+  const size_t smem = sizeof(int) * ((size_t)(kMapWarps + 4) * E + 2 * kScatEntries);
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        k_map_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  // tiles per CTA: as many as the staging buffers hold while the grid keeps at least two
+  // CTAs per SM (a small map keeps one tile per CTA)
+  const int tiles = map_tiles(T), min_ctas = 2 * device_sm_count();
+  int S = 1;
+  while (2 * S * kMapTokTile * k <= kScatEntries && 2 * S <= kScanSeg &&
+         tiles / (2 * S) >= min_ctas)
+    S *= 2;
+  return launch_pdl(k_map_scatter, (map_tiles(T) + S - 1) / S, kMapThreads, smem, st, T, E, k, S,
+                    nblk_cap, top,
                     tile_off, map_segs(const_cast<int32_t *>(tile_off), T, E), bins, padded_bins,
                     indices, bin_ids, dest_row, block_expert);
 }

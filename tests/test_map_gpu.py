@@ -59,7 +59,12 @@ def test_map_parity_real_inputs_tiny():
     (700, 1000, 8, "continuous"),   # 32 per lane, strided
     (40000, 16, 4, "continuous"),   # 625 tiles: the scan re-reads past its register cache
     (500, 64, 8, "tiny_values"),    # bf16 subnormals of both signs next to +0 / -0
-    (2048, 256, 8, "skewed"),       # the skewed workload's bias: one lane holds most picks
+    (2048, 256, 8, "skewed"),       # the skewed workload's bias on the low expert indices
+    # two logits per word, word c of lane l = experts 64c + 2l, 64c + 2l + 1
+    (2048, 256, 8, "lane_heavy"),   # lane 0's experts win: the rounds run again with refills
+    (1000, 200, 8, "continuous"),   # a partial last word group (lanes 0-3 of the fourth)
+    (1000, 66, 4, "few_values"),    # one lane of the second group, ties
+    (777, 512, 2, "lane_heavy"),    # 16 per lane, top-2
 ])
 def test_map_parity_edge_cases(T, E, k, kind):
     g = torch.Generator().manual_seed(T * 7 + E)
@@ -73,6 +78,9 @@ def test_map_parity_edge_cases(T, E, k, kind):
         logits = vals[torch.randint(0, len(vals), (T, E), generator=g)]
     elif kind == "skewed":
         logits = torch.randn((T, E), generator=g) - 1.5 * torch.log(torch.arange(E) + 1.0)
+    elif kind == "lane_heavy":  # experts 64c, 64c + 1 (the first lane's) far above the rest
+        logits = torch.randn((T, E), generator=g) - 8.0
+        logits[:, (torch.arange(E) % 64) < 2] += 16.0
     else:
         logits = torch.randn((T, E), generator=g)
     logits = logits.to(torch.bfloat16)
@@ -129,6 +137,27 @@ def test_map_nonfinite_logits_flagged():
     dims = B.make_dims(64, 128, 128, 8, 2)
     _, g = gpu_map(dims, logits.to(torch.bfloat16))
     assert g["status"] & B.STATUS_NONFINITE_LOGITS
+
+
+@pytest.mark.parametrize("E,k", [(256, 8), (64, 4), (250, 8)])
+def test_map_nonfinite_logits_ranked(E, k):
+    """NaN ranks below every value (-inf included), +-inf at its place; the choice and the map
+    stay bit-exact and the call is flagged."""
+    T = 700
+    g = torch.Generator().manual_seed(E + k)
+    logits = torch.randn((T, E), generator=g)
+    r = torch.rand((T, E), generator=g)
+    logits[r < 0.01] = float("nan")
+    logits[(r >= 0.01) & (r < 0.015)] = float("inf")
+    logits[(r >= 0.015) & (r < 0.02)] = float("-inf")
+    logits[5, :] = float("nan")             # a row of NaN only
+    logits[6, : E // 2] = float("-inf")     # half of a row at -inf
+    logits = logits.to(torch.bfloat16)
+    dims = B.make_dims(T, 128, 128, E, k)
+    _, gm = gpu_map(dims, logits)
+    top, _ = oracle.route(logits.float().numpy(), k)
+    compare_map(gm, oracle.sparse_map(top, E), top_expected=top)
+    assert gm["status"] & B.STATUS_NONFINITE_LOGITS
 
 
 def test_map_status_is_the_calls_own():
