@@ -127,16 +127,27 @@ __device__ __forceinline__ float ex2_ftz(float x) {
   return y;
 }
 
-// (a, b) * s + (t, t) on the paired fp32 pipe, and the sum of two pairs.
-__device__ __forceinline__ void fma_f32x2(float &a, float &b, float s, float t) {
-  asm("{.reg .b64 x, y, m, c;\n\t"
+// The two bf16 values packed in w minus m, in fp32 (one rounding each: x * 1 + (-m) on the
+// mixed-precision fused multiply-add, with no unpacking of the pair).
+__device__ __forceinline__ void sub_bf16x2_f32(uint32_t w, float m, float &d0, float &d1) {
+  asm("{.reg .b16 lo, hi, one;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "mov.b16 one, 0x3F80;\n\t"
+      "fma.rn.f32.bf16 %0, lo, one, %3;\n\t"
+      "fma.rn.f32.bf16 %1, hi, one, %3;}"
+      : "=f"(d0), "=f"(d1)
+      : "r"(w), "f"(-m));
+}
+
+// (a, b) * s on the paired fp32 pipe, and the sum of two pairs.
+__device__ __forceinline__ void mul_f32x2(float &a, float &b, float s) {
+  asm("{.reg .b64 x, y, m;\n\t"
       "mov.b64 x, {%0, %1};\n\t"
       "mov.b64 m, {%2, %2};\n\t"
-      "mov.b64 c, {%3, %3};\n\t"
-      "fma.rn.f32x2 y, x, m, c;\n\t"
+      "mul.rn.f32x2 y, x, m;\n\t"
       "mov.b64 {%0, %1}, y;}"
       : "+f"(a), "+f"(b)
-      : "f"(s), "f"(t));
+      : "f"(s));
 }
 __device__ __forceinline__ void add_f32x2(float &a, float &b, float c, float d) {
   asm("{.reg .b64 x, y, z;\n\t"
@@ -321,37 +332,36 @@ __global__ void __launch_bounds__(kRouteThreads, KPL <= 8 ? 2 : 1) k_route_hist(
         if (__any_sync(0xFFFFFFFFu, cnt > C)) pk = select_rounds<C, KPL, KC, true>(key, k, lane);
       }
     }
-    const uint32_t my_key = pk.mine, top_key = pk.first;
+    const uint32_t my_key = pk.mine;
     const int my_e = 0xFFFF - (int)(my_key & 0xFFFFu);
-    // softmax over all E logits (or, renormalised, over the k picks), max = the first pick;
-    // e^(x - m) = 2^(x log2(e) - m log2(e)) with one fused multiply-add per logit
-    const float m = ((top_key >> 16) == 0u) ? __uint_as_float(0x7FC00000u)
-                                           : bf16_from_order(top_key >> 16);
+    // softmax over all E logits (or, renormalised, over the k picks), max m = the first pick
+    // (lane 0's); e^(x - m) = 2^((x - m) log2(e)), x - m rounded once
     const float v = (lane < k) ? (((my_key >> 16) == 0u) ? __uint_as_float(0x7FC00000u)
                                                          : bf16_from_order(my_key >> 16))
                                : 0.0f;
-    const float ml = m * kLog2e;
-    const float ev = ex2_approx(fmaf(v, kLog2e, -ml));
+    const float m = __shfl_sync(0xFFFFFFFFu, v, 0);
+    const float ev = ex2_approx((v - m) * kLog2e);
     float sum = 0.0f;
     if (renorm) {
       if (lane < k) sum = ev;
-    } else if (PACKED && full_rows) {  // two logits per word on the paired fp32 pipe
+    } else if (PACKED && full_rows) {  // two logits per word, on the paired fp32 pipe
       float s0 = 0.0f, s1 = 0.0f;
 #pragma unroll
       for (int i = 0; i < Row::kWords; ++i) {
-        float a = __uint_as_float(cur.w[i] << 16), b = __uint_as_float(cur.w[i] & 0xFFFF0000u);
-        fma_f32x2(a, b, kLog2e, -ml);
+        float a, b;
+        sub_bf16x2_f32(cur.w[i], m, a, b);
+        mul_f32x2(a, b, kLog2e);
         add_f32x2(s0, s1, ex2_ftz(a), ex2_ftz(b));
       }
       sum = s0 + s1;
     } else if (full_rows) {
 #pragma unroll
       for (int i = 0; i < KPL; ++i)
-        sum += ex2_ftz(fmaf(__uint_as_float(cur.image(i)), kLog2e, -ml));
+        sum += ex2_ftz((__uint_as_float(cur.image(i)) - m) * kLog2e);
     } else {
 #pragma unroll
       for (int i = 0; i < KPL; ++i)
-        if (low_of(i)) sum += ex2_ftz(fmaf(__uint_as_float(cur.image(i)), kLog2e, -ml));
+        if (low_of(i)) sum += ex2_ftz((__uint_as_float(cur.image(i)) - m) * kLog2e);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
