@@ -44,11 +44,12 @@ def test_backward_full_parity_small(w):
         assert (g["dw1"][e] == 0).all() and (g["dw3"][e] == 0).all() and (g["dw2"][e] == 0).all()
 
 
-@pytest.mark.parametrize("w", SMALL[1:4], ids=lambda w: w.describe())
+@pytest.mark.parametrize("w", SMALL[1:4] + SMALL[5:], ids=lambda w: w.describe())
 def test_backward_steps_against_float64(w):
     """Every backward step on its own bf16 inputs (MN-major operands included): the dy
     gather, the dH GEMM with its fused dGLU / weighted-H / routing-weight-partial epilogue,
-    dX, the weight gradients, and the scatter-sum with the routing-weight reduction."""
+    dX, the weight gradients (every element written: the buffers start as NaN), and the
+    scatter-sum with the routing-weight reduction."""
     inp = make_inputs(w, with_dy=True)
     dims = dims_of(w)
     bufs, dev, y, g = gpu_backward(dims, inp)
@@ -56,7 +57,7 @@ def test_backward_steps_against_float64(w):
     T, k, h, f = w.T, w.top_k, w.hidden, w.ffn
     dx = torch.empty((T, h), dtype=torch.bfloat16, device="cuda")
     dwt = torch.full((T, k), float("nan"), dtype=torch.float32, device="cuda")
-    dw = {n: torch.empty_like(g[n]) for n in ("dw1", "dw3", "dw2")}
+    dw = {n: torch.full_like(g[n], float("nan")) for n in ("dw1", "dw3", "dw2")}
     B.dmoe_padded_gather(dims, dev["dy"], bufs.map, st["dy_pad"])
     B.dmoe_bwd_dglu(dims, st["dy_pad"], dev["w2"], bufs.view("a"), bufs.view("bm"), bufs.map,
                     st["da"], st["dbm"], st["hw"], st["dw_part"])
