@@ -241,15 +241,14 @@ __device__ __forceinline__ Picks select_rounds(const uint32_t (&key)[KPL], int k
 // again with refills.  Weights: fp32 softmax over all E logits (or, renormalised, over the k
 // picks) with the first pick as the maximum.  The tile's expert histogram is built in shared
 // memory and written to tile_hist; the tile's status bits go to tile_flags (a plain store, so
-// the workspace needs no initialisation).
+// the workspace needs no initialisation).  Up to 8 logits per lane two CTAs share an SM
+// (at most 64 registers a thread).
 template <int KPL, bool PACKED, int KC>
-__global__ void __launch_bounds__(kRouteThreads, KPL <= 8 ? 2 : 1) k_route_hist(const uint16_t *__restrict__ logits,
-                                                              int T, int E, int k, int renorm,
-                                                              int32_t *__restrict__ top,
-                                                              float *__restrict__ weights,
-                                                              int32_t *__restrict__ tile_hist,
-                                                              int32_t *__restrict__ tile_flags,
-                                                              unsigned int *__restrict__ done) {
+__global__ void __launch_bounds__(kRouteThreads, KPL <= 8 ? 2 : 1)
+    k_route_hist(const uint16_t *__restrict__ logits, int T, int E, int k, int renorm,
+                 int32_t *__restrict__ top, float *__restrict__ weights,
+                 int32_t *__restrict__ tile_hist, int32_t *__restrict__ tile_flags,
+                 unsigned int *__restrict__ done) {
   using Row = RouteRow<KPL, PACKED>;
   constexpr int C = (KPL < 3) ? KPL : 3;                  // candidates kept per lane
   constexpr int kInFlight = (KPL <= 8) ? kRouteTPW : 1;  // token rows loaded ahead per warp
