@@ -48,15 +48,18 @@ def test_map_parity_real_inputs_tiny():
     (4097, 32, 32, "few_values"),  # maximum k
     (1, 8, 2, "continuous"),       # single token
     (8192, 64, 8, "continuous"),   # the issue's failing shape with 4096-long sequences
-    # logits layouts of the routing kernel: vector rows when E is a multiple of the logits per
-    # lane, strided lanes otherwise; sorted per-lane candidates up to 8 per lane
+    # logits layouts of the routing kernel: two experts per word for even E (word c of lane l
+    # = experts 64c + 2l, 64c + 2l + 1), lane l = experts l, l + 32, ... for odd E; rounds
+    # unrolled for top-2 and top-8
     (7, 7, 3, "few_values"),        # 1 per lane, a partial tile
-    (1000, 33, 4, "continuous"),    # 2 per lane, strided
-    (1000, 100, 8, "few_values"),   # 4 per lane, vector, ties
-    (1500, 250, 8, "continuous"),   # 8 per lane, strided
-    (300, 256, 32, "few_values"),   # 8 per lane, vector, 32 picks drain whole lanes
-    (600, 384, 8, "few_values"),    # 16 per lane, vector, unsorted rounds
-    (700, 1000, 8, "continuous"),   # 32 per lane, strided
+    (1000, 33, 4, "continuous"),    # 2 per lane, odd E
+    (1000, 100, 8, "few_values"),   # 4 per lane, paired, ties
+    (1500, 250, 8, "continuous"),   # 8 per lane, paired, a partial last word group
+    (1500, 251, 8, "continuous"),   # 8 per lane, odd E
+    (300, 256, 32, "few_values"),   # 8 per lane, 32 picks drain whole lanes (refilled rounds)
+    (600, 384, 8, "few_values"),    # 16 per lane, paired
+    (700, 1000, 8, "continuous"),   # 32 per lane, paired
+    (700, 999, 8, "continuous"),    # 32 per lane, odd E
     (40000, 16, 4, "continuous"),   # 625 tiles: the scan re-reads past its register cache
     (500, 64, 8, "tiny_values"),    # bf16 subnormals of both signs next to +0 / -0
     (2048, 256, 8, "skewed"),       # the skewed workload's bias on the low expert indices
@@ -139,7 +142,7 @@ def test_map_nonfinite_logits_flagged():
     assert g["status"] & B.STATUS_NONFINITE_LOGITS
 
 
-@pytest.mark.parametrize("E,k", [(256, 8), (64, 4), (250, 8)])
+@pytest.mark.parametrize("E,k", [(256, 8), (64, 4), (250, 8), (255, 8), (33, 2)])
 def test_map_nonfinite_logits_ranked(E, k):
     """NaN ranks below every value (-inf included), +-inf at its place; the choice and the map
     stay bit-exact and the call is flagged."""
